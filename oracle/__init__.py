@@ -1,0 +1,50 @@
+"""Plain fp64 CPU oracle for the ELSAA attention operator.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import, call or
+execute anything in this package: only ``tests/``, ``__graft_entry__.smoke()``
+and the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it.
+It shares no code with the CUDA path (no kernels, headers, helpers or
+constants): it receives the same seeded inputs and nothing else.
+
+Every function here is written from the ELSAA pages
+("ELSAA: Efficient Low-Rank and Sparse Attention Approximation for Training
+Transformers" and "Two Efficient Attentions, One Denominator Problem") in the
+order the method takes its steps, with library primitives (matmul, stable
+argsort, bincount, index_add, logsumexp) as the only building blocks.
+
+Parity status of each function (what pins it, see ``tests/test_oracle.py``):
+  simhash_codes        pinned: brute-force sign loop, scale/negation invariants,
+                       angular collision statistics
+  stable_sort_perm     pinned: pure-Python sort by (code, index), permutation
+                       and ordering properties
+  sparse_branch        pinned: one chunk == dense softmax attention, masked dense
+                       softmax over the rank mask, one-hot value support test,
+                       closed form for Q = 0
+  race_build / race_query
+                       pinned: per-table sums, K_r = 0 closed form, collision
+                       count matrix brute force
+  gates / fuse         pinned: lambda = 0 ablation (m == 1), single-branch gate
+                       settings, Z_race = 0, closed form for Q = 0
+  forward_head         pinned through the pieces above and the Q = 0 closed form
+  grads_head           pinned: finite differences (gradcheck) of forward_head,
+                       RACE branch carries no dq/dk
+  interaction_count    parity unpinned (the pages lost the complexity formula;
+                       only its 32K example survives)
+"""
+
+from .elsaa_oracle import (  # noqa: F401
+    simhash_projections,
+    simhash_codes,
+    stable_sort_perm,
+    chunk_window,
+    sparse_branch,
+    race_build,
+    race_query,
+    gates,
+    fuse,
+    forward_head,
+    grads_head,
+    forward_batch,
+    interaction_count,
+    NEAR_ZERO,
+)

@@ -1,0 +1,292 @@
+"""fp64 reference for the ELSAA attention operator (test infrastructure only).
+
+ELSAA ("ELSAA: Efficient Low-Rank and Sparse Attention Approximation for
+Training Transformers", overview) is the attention that follows the dense
+Q/K/V projections.  It adds an exact sparse branch and a low-rank RACE branch,
+rescales the sparse branch by its attention mass relative to the RACE mass and
+mixes both through independent token-wise gates.
+
+The pages lost their display formulas ("Two Efficient Attentions, One
+Denominator Problem", section "Two efficient branches can still be
+mis-scaled": the multiplier and the gated sum are missing).  The readings this
+oracle takes where the text is silent are stated next to each step and, in
+full, in the repository's design notes:
+
+  * hashing is SimHash (sign of a projection on a random hyperplane), bit j of
+    a code has weight 2**j, a projection of exactly 0 gives bit 0;
+  * one shared set of hyperplanes for Q and K and for every (batch, head);
+  * Sort-LSH orders Q and K separately by code, ties by token index; sorted
+    query chunk j attends sorted key chunks j-1 and j (chunk 0: only its own),
+    no wrap-around;
+  * RACE: L tables of 2**K_r buckets, T[l][b] = sum of values, C[l][b] = count;
+    O_race = sum_l T[l][h_l(q)] / sum_l C[l][h_l(q)] (0 when the count is 0),
+    Z_race = sum_l C[l][h_l(q)] / L, each collision weighing exp(0) = 1;
+  * m = Z_sp / (Z_sp + lambda * Z_race) with Z_sp = sum of exp(score) over the
+    sparse window (unshifted), and y = g_s * m * O_sp + g_r * O_race;
+  * gates g = sigmoid(w . q_i + b) per branch, or fixed constants;
+  * score scale 1/sqrt(d) unless given.
+
+All arithmetic is fp64 on the CPU.  Inputs are the exact values the device
+sees (bf16 or fp32), upcast.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Dict, Optional
+
+import numpy as np
+import torch
+
+F64 = torch.float64
+
+# Projections with |x . r| below this are reported separately: their sign can
+# legitimately differ between an fp64 dot product and an fp32-accumulated one.
+NEAR_ZERO = 1e-5
+
+
+# ---------------------------------------------------------------------------
+# Step 1: SimHash codes
+# ---------------------------------------------------------------------------
+
+def simhash_projections(x: torch.Tensor, planes: torch.Tensor) -> torch.Tensor:
+    """Projections x . r_j of every row of ``x`` [n, d] on every hyperplane
+    ``planes`` [m, d], in fp64.  ELSAA overview: the sparse branch is selected
+    by LSH; SimHash is the angular LSH whose edge model the page "Two
+    Efficient Attentions, One Denominator Problem" (section "Full rank explains
+    structural complementarity") relies on."""
+    return x.to(F64) @ planes.to(F64).T
+
+
+def simhash_codes(proj: torch.Tensor) -> torch.Tensor:
+    """Integer codes from projections [n, m]: bit j = (proj[:, j] > 0), code =
+    sum_j bit_j * 2**j.  A projection of exactly zero gives bit 0."""
+    m = proj.shape[-1]
+    bits = (proj > 0).to(torch.int64)
+    weights = torch.tensor([1 << j for j in range(m)], dtype=torch.int64)
+    return (bits * weights).sum(dim=-1)
+
+
+# ---------------------------------------------------------------------------
+# Step 2: Sort-LSH ordering
+# ---------------------------------------------------------------------------
+
+def stable_sort_perm(code: torch.Tensor) -> torch.Tensor:
+    """perm[r] = token index at sorted rank r; stable (equal codes keep token
+    order).  "The ablation isolates the actual contribution" names the
+    Sort-LSH + RACE hybrid; sorting by hash code is what makes consecutive
+    chunks hold similar tokens."""
+    return torch.from_numpy(np.argsort(code.numpy(), kind="stable").astype(np.int64))
+
+
+def chunk_window(rank: int, chunk: int) -> tuple:
+    """Sorted key ranks [lo, hi) seen by the query at sorted rank ``rank``:
+    its own chunk and the previous one (chunk 0 only itself), no wrap-around."""
+    j = rank // chunk
+    return max(0, (j - 1) * chunk), (j + 1) * chunk
+
+
+# ---------------------------------------------------------------------------
+# Step 3: exact sparse branch
+# ---------------------------------------------------------------------------
+
+def sparse_branch(q, k, v, perm_q, perm_k, chunk: int, scale: float):
+    """Exact softmax attention restricted to the Sort-LSH window ("Two
+    Efficient Attentions, One Denominator Problem", section "Two efficient
+    branches can still be mis-scaled": the sparse branch computes only the
+    selected interactions, exactly).  Returns (O_sp [N, d], lse [N]) in token
+    order; Z_sp = exp(lse) is the unshifted attention mass of the window."""
+    n = q.shape[0]
+    qs, ks, vs = q[perm_q], k[perm_k], v[perm_k]
+    outs, lses = [], []
+    for j in range(n // chunk):
+        lo, hi = chunk_window(j * chunk, chunk)
+        s = scale * (qs[j * chunk:(j + 1) * chunk] @ ks[lo:hi].T)
+        lses.append(torch.logsumexp(s, dim=1))
+        outs.append(torch.softmax(s, dim=1) @ vs[lo:hi])
+    o_sorted = torch.cat(outs, 0)
+    lse_sorted = torch.cat(lses, 0)
+    inv = torch.empty_like(perm_q)
+    inv[perm_q] = torch.arange(n, dtype=perm_q.dtype)
+    return o_sorted[inv], lse_sorted[inv]
+
+
+# ---------------------------------------------------------------------------
+# Step 4: low-rank RACE branch
+# ---------------------------------------------------------------------------
+
+def race_build(rcode_k: torch.Tensor, v: torch.Tensor, nbuckets: int):
+    """RACE tables from key codes [N, L] and values [N, d]: C[l][b] = number
+    of keys with h_l(k) = b, T[l][b] = sum of their values ("Two Efficient
+    Attentions, One Denominator Problem": the RACE branch compresses the
+    interaction structure into hash-bucket summaries)."""
+    L = rcode_k.shape[1]
+    d = v.shape[1]
+    counts = torch.stack([torch.bincount(rcode_k[:, l], minlength=nbuckets) for l in range(L)])
+    sums = torch.stack([
+        torch.zeros(nbuckets, d, dtype=F64).index_add(0, rcode_k[:, l], v) for l in range(L)
+    ])
+    return counts, sums
+
+
+def race_query(rcode_q: torch.Tensor, counts: torch.Tensor, sums: torch.Tensor):
+    """Each query reads its bucket in every table: Ctot = sum_l C[l][h_l(q)],
+    O_race = sum_l T[l][h_l(q)] / Ctot (0 when Ctot = 0), Z_race = Ctot / L
+    (the RACE estimate of the collision-kernel mass, each colliding key
+    weighing exp(0) = 1).  Returns (Ctot [N] int64, O_race [N, d], Z_race [N])."""
+    L = rcode_q.shape[1]
+    ctot = sum(counts[l][rcode_q[:, l]] for l in range(L))
+    num = sum(sums[l][rcode_q[:, l]] for l in range(L))
+    safe = torch.where(ctot > 0, ctot, torch.ones_like(ctot)).to(F64)
+    o_race = torch.where((ctot > 0)[:, None], num / safe[:, None], torch.zeros_like(num))
+    z_race = ctot.to(F64) / L
+    return ctot, o_race, z_race
+
+
+# ---------------------------------------------------------------------------
+# Steps 5-6: denominator-aware fusion and token-wise gates
+# ---------------------------------------------------------------------------
+
+def gates(q, gate_w, gate_b, fixed: Optional[tuple] = None):
+    """Independent token-wise gates, learned or fixed (ELSAA overview):
+    g_s = sigmoid(w_s . q_i + b_s), g_r = sigmoid(w_r . q_i + b_r)."""
+    n = q.shape[0]
+    if fixed is not None:
+        return (torch.full((n,), float(fixed[0]), dtype=F64),
+                torch.full((n,), float(fixed[1]), dtype=F64))
+    a_s = q @ gate_w[0] + gate_b[0]
+    a_r = q @ gate_w[1] + gate_b[1]
+    return torch.sigmoid(a_s), torch.sigmoid(a_r)
+
+
+def fuse(o_sp, lse, o_race, z_race, g_s, g_r, lam):
+    """Denominator-aware fusion ("Two Efficient Attentions, One Denominator
+    Problem", section "Two efficient branches can still be mis-scaled"): the
+    sparse output is scaled by its mass relative to the RACE mass,
+    m = Z_sp / (Z_sp + lambda * Z_race), then both branches are gated
+    independently: y = g_s * m * O_sp + g_r * O_race.  With lambda = 0 the
+    multiplier is one (the Sort_Lsh_RACE ablation)."""
+    z_sp = torch.exp(lse)
+    m = z_sp / (z_sp + lam * z_race)
+    y = g_s[:, None] * m[:, None] * o_sp + g_r[:, None] * o_race
+    return y, m
+
+
+# ---------------------------------------------------------------------------
+# One (batch, head) unit, forward and gradients
+# ---------------------------------------------------------------------------
+
+def _hash_all(q64, k64, r_sort, r_race):
+    L, kr, d = r_race.shape
+    pq_s = simhash_projections(q64, r_sort)
+    pk_s = simhash_projections(k64, r_sort)
+    planes = r_race.reshape(L * kr, d)
+    pq_r = simhash_projections(q64, planes).reshape(-1, L, kr)
+    pk_r = simhash_projections(k64, planes).reshape(-1, L, kr)
+    return pq_s, pk_s, pq_r, pk_r
+
+
+def forward_head(q, k, v, r_sort, r_race, chunk: int, scale: Optional[float] = None,
+                 gate_w=None, gate_b=None, lam=1.0, fixed_gates: Optional[tuple] = None,
+                 codes: Optional[Dict[str, torch.Tensor]] = None) -> Dict[str, torch.Tensor]:
+    """The whole operator on one (batch, head) unit.
+
+    q, k, v: [N, d] (any float dtype; upcast to fp64).  r_sort: [b_s, d];
+    r_race: [L, K_r, d].  ``codes`` may carry precomputed code_q / code_k /
+    rcode_q / rcode_k (used to re-run the float steps with another side's
+    codes where a projection sits within NEAR_ZERO of zero, and to freeze the
+    hash in gradient checks).  Returns every intermediate in token order."""
+    q64, k64, v64 = q.to(F64), k.to(F64), v.to(F64)
+    n, d = q64.shape
+    L, kr, _ = r_race.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out: Dict[str, torch.Tensor] = {}
+    if codes is None:
+        with torch.no_grad():
+            pq_s, pk_s, pq_r, pk_r = _hash_all(q64.detach(), k64.detach(), r_sort, r_race)
+        code_q, code_k = simhash_codes(pq_s), simhash_codes(pk_s)
+        rcode_q, rcode_k = simhash_codes(pq_r), simhash_codes(pk_r)
+        near = [p.abs() < NEAR_ZERO for p in (pq_s, pk_s, pq_r, pk_r)]
+        out["near_code_q"] = near[0].any(dim=-1)
+        out["near_code_k"] = near[1].any(dim=-1)
+        out["near_rcode_q"] = near[2].any(dim=-1)
+        out["near_rcode_k"] = near[3].any(dim=-1)
+    else:
+        code_q, code_k = codes["code_q"].to(torch.int64), codes["code_k"].to(torch.int64)
+        rcode_q, rcode_k = codes["rcode_q"].to(torch.int64), codes["rcode_k"].to(torch.int64)
+    perm_q, perm_k = stable_sort_perm(code_q), stable_sort_perm(code_k)
+    o_sp, lse = sparse_branch(q64, k64, v64, perm_q, perm_k, chunk, scale)
+    counts, sums = race_build(rcode_k, v64, 1 << kr)
+    ctot, o_race, z_race = race_query(rcode_q, counts, sums)
+    if fixed_gates is None:
+        g_s, g_r = gates(q64, gate_w.to(F64), gate_b.to(F64))
+    else:
+        g_s, g_r = gates(q64, None, None, fixed=fixed_gates)
+    y, m = fuse(o_sp, lse, o_race, z_race, g_s, g_r, lam)
+    out.update(code_q=code_q, code_k=code_k, rcode_q=rcode_q, rcode_k=rcode_k,
+               perm_q=perm_q, perm_k=perm_k, o_sp=o_sp, lse=lse, race_count=counts,
+               race_sum=sums, ctot=ctot, o_race=o_race, z_race=z_race, g_s=g_s, g_r=g_r,
+               m=m, y=y)
+    return out
+
+
+def grads_head(q, k, v, r_sort, r_race, chunk: int, dy, scale: Optional[float] = None,
+               gate_w=None, gate_b=None, lam=1.0, fixed_gates: Optional[tuple] = None,
+               codes: Optional[Dict[str, torch.Tensor]] = None) -> Dict[str, torch.Tensor]:
+    """Gradients of sum(y * dy) with the hash codes held constant (codes are
+    piecewise constant in q and k), by fp64 autograd through forward_head.
+    The pages state that ELSAA is used in training ("ELSAA combines sparsity
+    and low-rank methods...": the approximation acts at run time during
+    training).  Returns dq, dk, dv [N, d], dgate_w [2, d], dgate_b [2],
+    dlambda (scalar); gate grads are zero for fixed gates."""
+    q64 = q.to(F64).detach().requires_grad_(True)
+    k64 = k.to(F64).detach().requires_grad_(True)
+    v64 = v.to(F64).detach().requires_grad_(True)
+    lam64 = torch.tensor(float(lam), dtype=F64, requires_grad=True)
+    leaves = [q64, k64, v64, lam64]
+    gw = gb = None
+    if fixed_gates is None:
+        gw = gate_w.to(F64).detach().requires_grad_(True)
+        gb = gate_b.to(F64).detach().requires_grad_(True)
+        leaves += [gw, gb]
+    if codes is None:
+        first = forward_head(q, k, v, r_sort, r_race, chunk, scale, gate_w, gate_b, lam,
+                             fixed_gates)
+        codes = {name: first[name] for name in ("code_q", "code_k", "rcode_q", "rcode_k")}
+    out = forward_head(q64, k64, v64, r_sort, r_race, chunk, scale, gw, gb, lam64,
+                       fixed_gates, codes=codes)
+    loss = (out["y"] * dy.to(F64)).sum()
+    g = torch.autograd.grad(loss, leaves, allow_unused=True)
+    res = {"dq": g[0], "dk": g[1], "dv": g[2], "dlambda": g[3]}
+    d = q.shape[1]
+    if fixed_gates is None:
+        res["dgate_w"], res["dgate_b"] = g[4], g[5]
+    else:
+        res["dgate_w"] = torch.zeros(2, d, dtype=F64)
+        res["dgate_b"] = torch.zeros(2, dtype=F64)
+    res["y"] = out["y"].detach()
+    return res
+
+
+def forward_batch(q, k, v, r_sort, r_race, chunk: int, scale=None, gate_w=None,
+                  gate_b=None, lam=1.0, fixed_gates=None, units=None):
+    """forward_head over (batch, head) units of [B, H, N, d] tensors; ``units``
+    selects a subset of (b, h) pairs (default all).  Returns {(b, h): dict}."""
+    B, H = q.shape[0], q.shape[1]
+    if units is None:
+        units = [(b, h) for b in range(B) for h in range(H)]
+    return {(b, h): forward_head(q[b, h], k[b, h], v[b, h], r_sort, r_race, chunk, scale,
+                                 gate_w, gate_b, lam, fixed_gates)
+            for (b, h) in units}
+
+
+def interaction_count(n: int, chunk: int, race_tables: int) -> Dict[str, int]:
+    """Attention-or-bucket interactions of one unit: every query scores the
+    keys of its window and reads one bucket per RACE table.  "Linear
+    interactions are not yet production economics" states the count is
+    linear in N and gives a 32K example; its formula is lost (parity
+    unpinned), so this is the count the algorithm above performs."""
+    window = sum(min((j + 1) * chunk, n) - max(0, (j - 1) * chunk) for j in range(n // chunk))
+    return {"sparse": window * chunk, "race": n * race_tables,
+            "total": window * chunk + n * race_tables, "dense": n * n}
