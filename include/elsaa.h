@@ -1,0 +1,158 @@
+/*
+ * libelsaa: the ELSAA attention operator (forward and backward) on NVIDIA B200.
+ *
+ * ELSAA ("ELSAA: Efficient Low-Rank and Sparse Attention Approximation for
+ * Training Transformers", overview) is the non-causal attention applied after
+ * the dense Q/K/V projections.  Per (batch, head) unit, with Q, K, V in
+ * R^{N x d}:
+ *
+ *   1. SimHash codes: bit j of a row x is [x . r_j > 0].  A sort code of
+ *      sort_bits bits from r_sort, and one code of race_bits bits per RACE
+ *      table l from r_race[l] (bit j has weight 2^j).
+ *   2. Sort-LSH: Q and K are each ordered by their sort code, ties by token
+ *      index (stable).  Sorted query chunk j (chunk rows) attends sorted key
+ *      chunks j-1 and j (chunk 0 only its own), no wrap-around.
+ *   3. Exact sparse branch: O_sp = softmax(scale * q k^T) V over that window
+ *      and its unshifted mass Z_sp = exp(lse_sp) ("Two Efficient Attentions,
+ *      One Denominator Problem", section "Two efficient branches can still be
+ *      mis-scaled": the sparse branch evaluates only the selected
+ *      interactions, exactly).
+ *   4. Low-rank RACE branch: L tables of 2^race_bits buckets; C[l][b] counts
+ *      the keys with h_l(k) = b and T[l][b] sums their values.  A query reads
+ *      its bucket in every table: Ctot = sum_l C[l][h_l(q)],
+ *      O_race = sum_l T[l][h_l(q)] / Ctot (0 if Ctot = 0), Z_race = Ctot / L.
+ *   5. Denominator-aware fusion (same page and section; the formula itself is
+ *      lost from the text, this library takes the mass ratio)
+ *      m = Z_sp / (Z_sp + lambda * Z_race), m = 1 when lambda * Z_race = 0.
+ *   6. Independent token-wise gates (ELSAA overview: "learned or fixed
+ *      gates"): g_s = sigmoid(w_s . q_i + b_s), g_r = sigmoid(w_r . q_i + b_r)
+ *      or fixed constants, and y = g_s * m * O_sp + g_r * O_race.
+ *
+ * Conventions for every entry point:
+ *   - Every pointer named "device" is CUDA device memory owned by the caller.
+ *     The library never allocates or frees device or pinned memory and keeps
+ *     no mutable global state; calls on different streams with different
+ *     workspaces may run concurrently.
+ *   - All work is enqueued on `stream` (a cudaStream_t passed as void*; NULL
+ *     is the legacy default stream).  Calls return without synchronising;
+ *     device-side failures (a bounded wait that ran out) are recorded in the
+ *     workspace's error word and read back by elsaa_check().
+ *   - Layouts are dense and row-major: q, k, v, y, dy, dq, dk, dv are
+ *     [B, H, N, d] with d contiguous, in params->dtype.
+ *   - On an error status the contents of every output are undefined.  Host
+ *     validation errors are returned before anything is enqueued.
+ */
+#ifndef ELSAA_H
+#define ELSAA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ELSAA_OK = 0,
+  ELSAA_ERR_INVALID_ARG = 1,     /* a null pointer, a bad size or misaligned buffer */
+  ELSAA_ERR_UNSUPPORTED = 2,     /* a valid request this build does not implement */
+  ELSAA_ERR_WORKSPACE = 3,       /* ws_bytes smaller than elsaa_workspace_bytes() */
+  ELSAA_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed */
+  ELSAA_ERR_DEVICE_TIMEOUT = 5,  /* a kernel's bounded wait ran out (elsaa_check) */
+  ELSAA_ERR_DEVICE_CHECK = 6     /* a kernel's own index check failed (elsaa_check) */
+} elsaa_status;
+
+typedef enum { ELSAA_BF16 = 0, ELSAA_F32 = 1 } elsaa_dtype;
+
+typedef struct {
+  int32_t B, H, N, d;     /* batch, heads, tokens per unit, head dim d in {32, 64, 128} */
+  int32_t dtype;          /* elsaa_dtype of q, k, v, r_sort, r_race, y, dy, dq, dk, dv */
+  int32_t sort_bits;      /* Sort-LSH code bits, 0..16 */
+  int32_t chunk;          /* Sort-LSH chunk length; N % chunk == 0 */
+  int32_t race_tables;    /* L >= 1 */
+  int32_t race_bits;      /* bits per RACE code, 0..16 (2^race_bits buckets per table) */
+  float scale;            /* score scale; <= 0 selects 1/sqrt(d) */
+  int32_t gate_fixed;     /* nonzero: gates are the constants gate_s, gate_r */
+  float gate_s, gate_r;
+} elsaa_params;
+
+/* Device views into a forward's saved state (see elsaa_saved_views). */
+typedef struct {
+  uint16_t* code_q;       /* [B,H,N] sort codes of the queries */
+  uint16_t* code_k;       /* [B,H,N] sort codes of the keys */
+  int32_t* perm_q;        /* [B,H,N] token index at each sorted rank */
+  int32_t* perm_k;        /* [B,H,N] */
+  void* rcode_q;          /* [B,H,N,L] RACE codes, uint8 if race_bits <= 8 else uint16 */
+  void* rcode_k;          /* [B,H,N,L] */
+  int32_t rcode_bytes;    /* 1 or 2 */
+  int32_t* race_count;    /* [B,H,L,2^race_bits] C */
+  float* race_sum;        /* [B,H,L,2^race_bits,d] T */
+  float* lse_sp;          /* [B,H,N] natural-log mass of the sparse window, token order */
+  void* o_sp;             /* [B,H,N,d] sparse-branch output (dtype), token order */
+  void* o_race;           /* [B,H,N,d] RACE-branch output (dtype), token order */
+  int32_t* ctot;          /* [B,H,N] Ctot */
+} elsaa_views;
+
+/* Returns ELSAA_OK if `p` describes a supported problem, else the reason. */
+elsaa_status elsaa_validate(const elsaa_params* p);
+
+/* Bytes of device workspace one forward or backward needs (the same figure
+ * serves both); 0 if `p` is invalid.  Workspace contents need not be
+ * initialised and are not preserved between calls except its error word. */
+size_t elsaa_workspace_bytes(const elsaa_params* p);
+
+/* Bytes of the saved state a training forward writes and the matching
+ * backward reads; 0 if `p` is invalid. */
+size_t elsaa_saved_bytes(const elsaa_params* p);
+
+/* Forward.  q, k, v: device [B,H,N,d]; r_sort: device [sort_bits, d] (may
+ * be NULL when sort_bits = 0); r_race: device [L, race_bits, d] (may be NULL
+ * when race_bits = 0); hyperplanes are shared by Q and K and by every unit
+ * and have the data dtype.  gate_w: device fp32 [2,d] (row 0 sparse, row 1 RACE),
+ * gate_b: device fp32 [2]; both ignored (may be NULL) if gate_fixed.
+ * lambda: device fp32 scalar.  y: device [B,H,N,d] output.  saved: device
+ * buffer of elsaa_saved_bytes() or NULL for inference.  ws: device buffer of
+ * at least elsaa_workspace_bytes(), 256-byte aligned; its first 4 bytes are
+ * the error word elsaa_check() reads.  All device pointers
+ * must be 16-byte aligned. */
+elsaa_status elsaa_forward(const elsaa_params* p, const void* q, const void* k, const void* v,
+                           const void* r_sort, const void* r_race, const float* gate_w,
+                           const float* gate_b, const float* lambda, void* y, void* saved,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* Backward of sum(y * dy) with the hash codes held constant (they are
+ * piecewise constant).  Inputs as for elsaa_forward plus `saved` written by
+ * a forward with the same inputs and dy: device [B,H,N,d].  Outputs (all
+ * overwritten, never accumulated): dq, dk, dv device [B,H,N,d] (dtype);
+ * dgate_w device fp32 [2,d] and dgate_b device fp32 [2] (written as zeros
+ * when gate_fixed; may be NULL then); dlambda device fp32 scalar.  The gate
+ * weights and lambda are shared by every unit, so their gradients are sums
+ * over B, H and N. */
+elsaa_status elsaa_backward(const elsaa_params* p, const void* q, const void* k, const void* v,
+                            const void* r_sort, const void* r_race, const float* gate_w,
+                            const float* gate_b, const float* lambda, const void* saved,
+                            const void* dy, void* dq, void* dk, void* dv, float* dgate_w,
+                            float* dgate_b, float* dlambda, void* ws, size_t ws_bytes,
+                            void* stream);
+
+/* Fills `out` with device pointers into `saved` (no device access). */
+elsaa_status elsaa_saved_views(const elsaa_params* p, const void* saved, elsaa_views* out);
+
+/* Synchronises `stream`, reads and clears the workspace error word (which
+ * every forward and backward clears when it starts), and
+ * returns ELSAA_OK, ELSAA_ERR_DEVICE_TIMEOUT or ELSAA_ERR_DEVICE_CHECK. */
+elsaa_status elsaa_check(void* ws, void* stream);
+
+/* Static text for a status code. */
+const char* elsaa_status_str(elsaa_status s);
+
+/* Which kernel family the sparse branch and the hash take for `p`:
+ * 1 = tcgen05 tensor-core kernels, 0 = CUDA-core kernels (fp32 data, head
+ * dims other than 64/128, or chunk shapes the tensor kernels do not tile). */
+int32_t elsaa_uses_tensor_cores(const elsaa_params* p);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ELSAA_H */

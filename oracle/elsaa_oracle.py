@@ -181,8 +181,8 @@ def _hash_all(q64, k64, r_sort, r_race):
     pq_s = simhash_projections(q64, r_sort)
     pk_s = simhash_projections(k64, r_sort)
     planes = r_race.reshape(L * kr, d)
-    pq_r = simhash_projections(q64, planes).reshape(-1, L, kr)
-    pk_r = simhash_projections(k64, planes).reshape(-1, L, kr)
+    pq_r = simhash_projections(q64, planes).reshape(q64.shape[0], L, kr)
+    pk_r = simhash_projections(k64, planes).reshape(k64.shape[0], L, kr)
     return pq_s, pk_s, pq_r, pk_r
 
 

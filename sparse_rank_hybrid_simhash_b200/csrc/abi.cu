@@ -1,0 +1,304 @@
+// The C ABI of libelsaa: validation, saved-state and workspace layout, and the
+// launch sequences of the forward and backward (see include/elsaa.h).
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace elsaa {
+
+bool make_geometry(const elsaa_params* p, Geometry* g, elsaa_status* why) {
+  *why = ELSAA_ERR_INVALID_ARG;
+  if (!p) return false;
+  if (p->B <= 0 || p->H <= 0 || p->N <= 0 || p->d <= 0) return false;
+  if (p->dtype != ELSAA_BF16 && p->dtype != ELSAA_F32) return false;
+  if (p->chunk <= 0 || p->N % p->chunk != 0) return false;
+  if (p->sort_bits < 0 || p->sort_bits > 16) return false;
+  if (p->race_tables < 1 || p->race_tables > 4096) return false;
+  if (p->race_bits < 0 || p->race_bits > 16) return false;
+  if ((int64_t)p->B * p->H * p->N * (p->d > p->race_tables ? p->d : p->race_tables) >
+      ((int64_t)1 << 40))
+    return false;
+  *why = ELSAA_ERR_UNSUPPORTED;
+  if (p->d != 32 && p->d != 64 && p->d != 128) return false;
+  g->B = p->B;
+  g->H = p->H;
+  g->N = p->N;
+  g->d = p->d;
+  g->BH = p->B * p->H;
+  g->bf16 = p->dtype == ELSAA_BF16;
+  g->esz = g->bf16 ? 2 : 4;
+  g->sort_bits = p->sort_bits;
+  g->chunk = p->chunk;
+  g->L = p->race_tables;
+  g->kr = p->race_bits;
+  g->NB = 1 << p->race_bits;
+  g->rcode_bytes = p->race_bits <= 8 ? 1 : 2;
+  g->scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
+  g->gate_fixed = p->gate_fixed ? 1 : 0;
+  g->gate_s = p->gate_s;
+  g->gate_r = p->gate_r;
+  g->sort_passes = p->sort_bits <= 8 ? 1 : 2;
+  g->sort_digit_bits = (p->sort_bits + g->sort_passes - 1) / g->sort_passes;
+  g->sort_bins = 1 << g->sort_digit_bits;
+  g->sort_tiles = (p->N + kSortTile - 1) / kSortTile;
+  g->tc_hash = hash_tc_supported(*g);
+  g->tc_attn = attn_tc_supported(*g);
+  *why = ELSAA_OK;
+  return true;
+}
+
+SavedLayout saved_layout(const Geometry& g) {
+  SavedLayout s;
+  const size_t bhn = (size_t)g.BH * g.N;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t o = off; off = align_up(off + bytes); return o; };
+  s.code = take(2 * bhn * 2);
+  s.perm = take(2 * bhn * 4);
+  s.rcode = take(2 * bhn * g.L * g.rcode_bytes);
+  s.race_count = take((size_t)g.BH * g.L * g.NB * 4);
+  s.race_sum = take((size_t)g.BH * g.L * g.NB * g.d * 4);
+  s.lse = take(bhn * 4);
+  s.o_sp = take(bhn * g.d * g.esz);
+  s.o_race = take(bhn * g.d * g.esz);
+  s.ctot = take(bhn * 4);
+  s.total = off;
+  return s;
+}
+
+WorkLayout work_layout(const Geometry& g) {
+  WorkLayout w;
+  const size_t bhn = (size_t)g.BH * g.N;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t o = off; off = align_up(off + bytes); return o; };
+  w.err = take(256);
+  w.sort_hist = take((size_t)2 * g.BH * g.sort_bins * g.sort_tiles * 4);
+  w.sort_tmp = take(2 * bhn * 4);
+  const size_t shared_base = off;
+  // forward without a saved buffer: the saved layout lives here
+  w.saved = take(saved_layout(g).total);
+  const size_t fwd_end = off;
+  // backward temporaries reuse the same bytes (a backward always has a saved buffer)
+  off = shared_base;
+  w.d_o = take(bhn * g.d * g.esz);
+  w.dprime = take(bhn * 4);
+  w.dq_acc = take(bhn * g.d * 4);
+  w.dk_acc = take(bhn * g.d * 4);
+  w.dv_acc = take(bhn * g.d * 4);
+  w.dor = take(bhn * g.d * 4);
+  w.d_t = take((size_t)g.BH * g.L * g.NB * g.d * 4);
+  w.partials = take((size_t)kParamBlocks * (2 * g.d + 3) * 4);
+  w.total = off > fwd_end ? off : fwd_end;
+  return w;
+}
+
+}  // namespace elsaa
+
+using namespace elsaa;
+
+namespace {
+
+inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+#define ELSAA_TRY(expr)                               \
+  do {                                                \
+    if ((expr) != cudaSuccess) return ELSAA_ERR_CUDA; \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+elsaa_status elsaa_validate(const elsaa_params* p) {
+  Geometry g;
+  elsaa_status why;
+  make_geometry(p, &g, &why);
+  return why;
+}
+
+size_t elsaa_workspace_bytes(const elsaa_params* p) {
+  Geometry g;
+  elsaa_status why;
+  if (!make_geometry(p, &g, &why)) return 0;
+  return work_layout(g).total;
+}
+
+size_t elsaa_saved_bytes(const elsaa_params* p) {
+  Geometry g;
+  elsaa_status why;
+  if (!make_geometry(p, &g, &why)) return 0;
+  return saved_layout(g).total;
+}
+
+int32_t elsaa_uses_tensor_cores(const elsaa_params* p) {
+  Geometry g;
+  elsaa_status why;
+  if (!make_geometry(p, &g, &why)) return 0;
+  return (g.tc_hash && g.tc_attn) ? 1 : 0;
+}
+
+elsaa_status elsaa_saved_views(const elsaa_params* p, const void* saved, elsaa_views* out) {
+  Geometry g;
+  elsaa_status why;
+  if (!make_geometry(p, &g, &why)) return why;
+  if (!saved || !out) return ELSAA_ERR_INVALID_ARG;
+  const SavedLayout s = saved_layout(g);
+  char* b = (char*)saved;
+  const size_t bhn = (size_t)g.BH * g.N;
+  out->code_q = (uint16_t*)(b + s.code);
+  out->code_k = out->code_q + bhn;
+  out->perm_q = (int32_t*)(b + s.perm);
+  out->perm_k = out->perm_q + bhn;
+  out->rcode_q = b + s.rcode;
+  out->rcode_k = b + s.rcode + bhn * g.L * g.rcode_bytes;
+  out->rcode_bytes = g.rcode_bytes;
+  out->race_count = (int32_t*)(b + s.race_count);
+  out->race_sum = (float*)(b + s.race_sum);
+  out->lse_sp = (float*)(b + s.lse);
+  out->o_sp = b + s.o_sp;
+  out->o_race = b + s.o_race;
+  out->ctot = (int32_t*)(b + s.ctot);
+  return ELSAA_OK;
+}
+
+elsaa_status elsaa_forward(const elsaa_params* p, const void* q, const void* k, const void* v,
+                           const void* r_sort, const void* r_race, const float* gate_w,
+                           const float* gate_b, const float* lambda, void* y, void* saved,
+                           void* ws, size_t ws_bytes, void* stream) {
+  Geometry g;
+  elsaa_status why;
+  if (!make_geometry(p, &g, &why)) return why;
+  if (!q || !k || !v || !lambda || !y || !ws) return ELSAA_ERR_INVALID_ARG;
+  if ((g.sort_bits > 0 && !r_sort) || (g.kr > 0 && !r_race)) return ELSAA_ERR_INVALID_ARG;
+  if (!g.gate_fixed && (!gate_w || !gate_b)) return ELSAA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, y, r_sort, r_race, gate_w, gate_b, saved};
+  for (const void* x : ptrs)
+    if (x && !aligned(x, 16)) return ELSAA_ERR_INVALID_ARG;
+  if (!aligned(ws, 256) || (saved && !aligned(saved, 256))) return ELSAA_ERR_INVALID_ARG;
+  const WorkLayout wl = work_layout(g);
+  if (ws_bytes < wl.total) return ELSAA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  char* w = (char*)ws;
+  char* sv = saved ? (char*)saved : w + wl.saved;
+  const SavedLayout sl = saved_layout(g);
+  const size_t bhn = (size_t)g.BH * g.N;
+  uint16_t* code = (uint16_t*)(sv + sl.code);
+  int32_t* perm = (int32_t*)(sv + sl.perm);
+  char* rcode = sv + sl.rcode;
+  char* rcode_k = rcode + bhn * g.L * g.rcode_bytes;
+  int32_t* counts = (int32_t*)(sv + sl.race_count);
+  float* sums = (float*)(sv + sl.race_sum);
+  float* lse = (float*)(sv + sl.lse);
+  void* o_sp = sv + sl.o_sp;
+  uint32_t* err = (uint32_t*)(w + wl.err);
+  ELSAA_TRY(cudaMemsetAsync(err, 0, sizeof(uint32_t), s));
+
+  // 1. SimHash codes of Q and K
+  if (g.tc_hash)
+    ELSAA_TRY(launch_hash_tc(g, q, k, r_sort, r_race, code, rcode, nullptr, err, s));
+  else
+    ELSAA_TRY(launch_hash_simt(g, q, k, r_sort, r_race, code, rcode, s));
+  // 2. Sort-LSH order of Q and K
+  ELSAA_TRY(launch_sort(g, code, perm, (int32_t*)(w + wl.sort_hist), (int32_t*)(w + wl.sort_tmp),
+                        s));
+  // 3. RACE tables from the keys
+  ELSAA_TRY(launch_race_build(g, rcode_k, v, false, sums, counts, s));
+  // 4. exact sparse branch
+  if (g.tc_attn)
+    ELSAA_TRY(launch_attn_fwd_tc(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s));
+  else
+    ELSAA_TRY(launch_attn_fwd_simt(g, q, k, v, perm, perm + bhn, o_sp, lse, s));
+  // 5. RACE gather, gates, multiplier and output
+  ELSAA_TRY(launch_race_fuse_fwd(g, q, rcode, sums, counts, o_sp, lse, gate_w, gate_b, lambda, y,
+                                 saved ? sv + sl.o_race : nullptr,
+                                 saved ? (int32_t*)(sv + sl.ctot) : nullptr, s));
+  return ELSAA_OK;
+}
+
+elsaa_status elsaa_backward(const elsaa_params* p, const void* q, const void* k, const void* v,
+                            const void* r_sort, const void* r_race, const float* gate_w,
+                            const float* gate_b, const float* lambda, const void* saved,
+                            const void* dy, void* dq, void* dk, void* dv, float* dgate_w,
+                            float* dgate_b, float* dlambda, void* ws, size_t ws_bytes,
+                            void* stream) {
+  (void)r_sort;
+  (void)r_race;
+  Geometry g;
+  elsaa_status why;
+  if (!make_geometry(p, &g, &why)) return why;
+  if (!q || !k || !v || !lambda || !saved || !dy || !dq || !dk || !dv || !dlambda || !ws)
+    return ELSAA_ERR_INVALID_ARG;
+  if (!g.gate_fixed && (!gate_w || !gate_b)) return ELSAA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, dy, dq, dk, dv};
+  for (const void* x : ptrs)
+    if (!aligned(x, 16)) return ELSAA_ERR_INVALID_ARG;
+  if (!aligned(ws, 256) || !aligned(saved, 256)) return ELSAA_ERR_INVALID_ARG;
+  const WorkLayout wl = work_layout(g);
+  if (ws_bytes < wl.total) return ELSAA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  char* w = (char*)ws;
+  const char* sv = (const char*)saved;
+  const SavedLayout sl = saved_layout(g);
+  const size_t bhn = (size_t)g.BH * g.N;
+  const int32_t* perm = (const int32_t*)(sv + sl.perm);
+  const char* rcode = sv + sl.rcode;
+  const char* rcode_k = rcode + bhn * g.L * g.rcode_bytes;
+  const float* lse = (const float*)(sv + sl.lse);
+  const void* o_sp = sv + sl.o_sp;
+  const void* o_race = sv + sl.o_race;
+  const int32_t* ctot = (const int32_t*)(sv + sl.ctot);
+  void* d_o = w + wl.d_o;
+  float* dprime = (float*)(w + wl.dprime);
+  float* dq_acc = (float*)(w + wl.dq_acc);
+  float* dk_acc = (float*)(w + wl.dk_acc);
+  float* dv_acc = (float*)(w + wl.dv_acc);
+  float* dor = (float*)(w + wl.dor);
+  float* d_t = (float*)(w + wl.d_t);
+  float* partials = (float*)(w + wl.partials);
+  ELSAA_TRY(cudaMemsetAsync(w + wl.err, 0, sizeof(uint32_t), s));
+
+  // 1. fusion and gate backward: dO_sp, D', dq from the gates, g_r dy / Ctot
+  ELSAA_TRY(launch_fuse_bwd(g, q, dy, o_sp, o_race, lse, ctot, gate_w, gate_b, lambda, d_o,
+                            dprime, dq_acc, dor, partials, s));
+  // 2. RACE backward: scatter into the table gradient by query code, gather by key code
+  ELSAA_TRY(launch_race_build(g, rcode, dor, true, d_t, nullptr, s));
+  ELSAA_TRY(launch_race_gather_sum(g, rcode_k, d_t, dv_acc, s));
+  // 3. sparse branch backward
+  ELSAA_TRY(cudaMemsetAsync(dk_acc, 0, bhn * g.d * 4, s));
+  ELSAA_TRY(launch_attn_bwd_simt(g, q, k, v, perm, perm + bhn, d_o, lse, dprime, dq_acc, dk_acc,
+                                 dv_acc, s));
+  // 4. outputs
+  ELSAA_TRY(launch_cast_out(g, dq_acc, dq, s));
+  ELSAA_TRY(launch_cast_out(g, dk_acc, dk, s));
+  ELSAA_TRY(launch_cast_out(g, dv_acc, dv, s));
+  ELSAA_TRY(launch_param_reduce(g, partials, dgate_w, dgate_b, dlambda, s));
+  return ELSAA_OK;
+}
+
+elsaa_status elsaa_check(void* ws, void* stream) {
+  if (!ws) return ELSAA_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ELSAA_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return ELSAA_ERR_CUDA;
+  if (word == 0) return ELSAA_OK;
+  if (cudaMemset(ws, 0, sizeof(word)) != cudaSuccess) return ELSAA_ERR_CUDA;
+  return (word & ERR_TIMEOUT) ? ELSAA_ERR_DEVICE_TIMEOUT : ELSAA_ERR_DEVICE_CHECK;
+}
+
+const char* elsaa_status_str(elsaa_status st) {
+  switch (st) {
+    case ELSAA_OK: return "ok";
+    case ELSAA_ERR_INVALID_ARG: return "invalid argument";
+    case ELSAA_ERR_UNSUPPORTED: return "unsupported problem";
+    case ELSAA_ERR_WORKSPACE: return "workspace too small";
+    case ELSAA_ERR_CUDA: return "CUDA error";
+    case ELSAA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case ELSAA_ERR_DEVICE_CHECK: return "device index check failed";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

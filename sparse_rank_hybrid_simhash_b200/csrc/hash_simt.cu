@@ -1,0 +1,99 @@
+// SimHash codes on CUDA cores.
+//
+// "ELSAA: Efficient Low-Rank and Sparse Attention Approximation for Training
+// Transformers" (overview) selects the sparse branch by LSH, and the RACE
+// branch of "Two Efficient Attentions, One Denominator Problem" buckets
+// tokens by hash.  Both use SimHash: bit j of row x is [x . r_j > 0], bit j
+// weighs 2^j.  One warp per row; each lane owns one hyperplane of a group of
+// 32 and accumulates the dot product in fp64 (products of fp32 / bf16 inputs
+// are exact in fp64), so a code differs from an exact evaluation only when a
+// projection is within fp64 rounding of zero.  This kernel serves fp32 data
+// and head dims the tensor-core hash does not tile.
+#include "common.cuh"
+#include "internal.h"
+
+namespace elsaa {
+namespace {
+
+template <typename T, typename CodeT>
+__global__ void __launch_bounds__(256)
+hash_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                 const T* __restrict__ r_sort, const T* __restrict__ r_race,
+                 int64_t rows_per_tensor, int d, int sort_bits, int L, int kr,
+                 uint16_t* __restrict__ code, CodeT* __restrict__ rcode) {
+  extern __shared__ float smem[];
+  const int warps = blockDim.x >> 5;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int P = sort_bits + L * kr;
+  const int nwords = (P + 31) >> 5;
+  float* xs = smem + w * d;
+  uint32_t* words = reinterpret_cast<uint32_t*>(smem + warps * d) + w * nwords;
+  const int64_t total = 2 * rows_per_tensor;
+  for (int64_t row = (int64_t)blockIdx.x * warps + w; row < total;
+       row += (int64_t)gridDim.x * warps) {
+    const T* src = row < rows_per_tensor ? q + row * d : k + (row - rows_per_tensor) * d;
+    for (int t = lane; t < d; t += 32) xs[t] = to_f32(src[t]);
+    __syncwarp();
+    for (int j0 = 0; j0 < P; j0 += 32) {
+      const int j = j0 + lane;
+      bool bit = false;
+      if (j < P) {
+        const T* r = j < sort_bits ? r_sort + (size_t)j * d
+                                   : r_race + (size_t)(j - sort_bits) * d;
+        double acc = 0.0;
+        for (int t = 0; t < d; ++t) acc += (double)xs[t] * (double)to_f32(r[t]);
+        bit = acc > 0.0;
+      }
+      const uint32_t m = __ballot_sync(0xffffffffu, bit);
+      if (lane == 0) words[j0 >> 5] = m;
+    }
+    __syncwarp();
+    auto field = [&](int start, int n) -> uint32_t {
+      uint32_t v = 0;
+      for (int b = 0; b < n; ++b) {
+        const int p = start + b;
+        v |= ((words[p >> 5] >> (p & 31)) & 1u) << b;
+      }
+      return v;
+    };
+    if (lane == 0) code[row] = (uint16_t)field(0, sort_bits);
+    for (int l = lane; l < L; l += 32) rcode[row * L + l] = (CodeT)field(sort_bits + l * kr, kr);
+    __syncwarp();
+  }
+}
+
+template <typename T, typename CodeT>
+cudaError_t run(const Geometry& g, const void* q, const void* k, const void* r_sort,
+                const void* r_race, uint16_t* code, void* rcode, cudaStream_t s) {
+  const int threads = 256, warps = threads / 32;
+  const int P = g.sort_bits + g.L * g.kr;
+  const size_t smem = (size_t)warps * g.d * sizeof(float) + (size_t)warps * ((P + 31) / 32) * 4;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(hash_simt_kernel<T, CodeT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t rows = (int64_t)g.BH * g.N;
+  const int64_t blocks = (2 * rows + warps - 1) / warps;
+  const int grid = (int)(blocks < 148 * 64 ? blocks : 148 * 64);
+  hash_simt_kernel<T, CodeT><<<grid, threads, smem, s>>>(
+      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(r_sort),
+      static_cast<const T*>(r_race), rows, g.d, g.sort_bits, g.L, g.kr, code,
+      static_cast<CodeT*>(rcode));
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_hash_simt(const Geometry& g, const void* q, const void* k, const void* r_sort,
+                             const void* r_race, uint16_t* code, void* rcode, cudaStream_t s) {
+  if (g.bf16) {
+    return g.rcode_bytes == 1
+               ? run<__nv_bfloat16, uint8_t>(g, q, k, r_sort, r_race, code, rcode, s)
+               : run<__nv_bfloat16, uint16_t>(g, q, k, r_sort, r_race, code, rcode, s);
+  }
+  return g.rcode_bytes == 1 ? run<float, uint8_t>(g, q, k, r_sort, r_race, code, rcode, s)
+                            : run<float, uint16_t>(g, q, k, r_sort, r_race, code, rcode, s);
+}
+
+}  // namespace elsaa

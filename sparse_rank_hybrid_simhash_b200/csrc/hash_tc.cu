@@ -1,0 +1,252 @@
+// SimHash codes on tcgen05 tensor cores (bf16 data, d in {64, 128}).
+//
+// "ELSAA: Efficient Low-Rank and Sparse Attention Approximation for Training
+// Transformers" (overview) selects the sparse branch by LSH; the RACE branch
+// ("Two Efficient Attentions, One Denominator Problem") buckets tokens by hash.
+// Bit j of a row x is [x . r_j > 0] with weight 2^j inside its code.  For one
+// row that is a product with every hyperplane: P = sort_bits + L * race_bits
+// columns, a GEMM of (2 B H N) x d by d x P.
+//
+// Products of bf16 values are exact in fp32, so a code can differ from an
+// exact evaluation only where a projection lies within fp32 accumulation
+// error of zero.
+//
+// Persistent CTAs of 128 threads.  The hyperplanes (padded to a multiple of
+// 16 columns with zero rows) stay resident in shared memory; 128-row tiles of
+// Q then K stream in by cp.async (double-buffered when shared memory allows).
+// Per tile the columns go through TMEM in passes of 128: thread t reads the 32
+// projections of row t per tcgen05.ld, turns their signs into a 32-bit mask,
+// appends it to a bit stream and emits every complete code (sort code first,
+// then RACE table 0, 1, ...).
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace elsaa {
+namespace {
+
+using namespace tc;
+
+constexpr int kTile = 128;
+constexpr int kThreads = 128;
+constexpr int kPass = 128;            // TMEM columns per pass
+constexpr uint32_t kTmemCols = 128;
+constexpr int kSmemLimit = 227 * 1024;
+
+struct HashShape {
+  int P, P16, nbuf;
+  uint32_t r_bytes, a_bytes, dyn;
+};
+
+HashShape hash_shape(const Geometry& g) {
+  HashShape h;
+  h.P = g.sort_bits + g.L * g.kr;
+  h.P16 = (h.P + 15) / 16 * 16;
+  h.r_bytes = (uint32_t)h.P16 * g.d * 2;
+  h.a_bytes = (uint32_t)kTile * g.d * 2;
+  h.nbuf = (h.r_bytes + 2 * h.a_bytes + 64 <= (uint32_t)kSmemLimit) ? 2 : 1;
+  h.dyn = h.r_bytes + h.nbuf * h.a_bytes + 64;
+  return h;
+}
+
+template <int D>
+ELSAA_DEV void load_tile(uint32_t dst, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                         int64_t rows_per_tensor, int64_t tile) {
+  constexpr int kChunks = D / 8;
+  const int64_t total = 2 * rows_per_tensor;
+  for (int i = threadIdx.x; i < kTile * kChunks; i += kThreads) {
+    const int row = i / kChunks, ch = i % kChunks;
+    const int64_t grow = tile * kTile + row;
+    const bool valid = grow < total;
+    const int64_t g = valid ? grow : 0;
+    const __nv_bfloat16* src =
+        (g < rows_per_tensor ? q + g * D : k + (g - rows_per_tensor) * D) + ch * 8;
+    cp_async16(dst + (ch >> 3) * (kTile * 128) + sw128_off(row, ch & 7), src, valid ? 16 : 0);
+  }
+}
+
+template <int D, typename CodeT>
+__global__ void __launch_bounds__(kThreads)
+hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+               const __nv_bfloat16* __restrict__ r_sort, const __nv_bfloat16* __restrict__ r_race,
+               int64_t rows_per_tensor, int sort_bits, int L, int kr, int P, int P16, int nbuf,
+               uint16_t* __restrict__ code, CodeT* __restrict__ rcode, uint32_t* __restrict__ err) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t r_bytes = (uint32_t)P16 * D * 2;
+  const uint32_t a_bytes = kTile * D * 2;
+  const uint32_t s_r = sbase, s_a = sbase + r_bytes;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + r_bytes + nbuf * a_bytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  if ((sbase & 1023u) != 0) {   // the swizzled tiles need a 1024-byte aligned base
+    if (tid == 0) raise_error(err, ERR_CHECK);
+    return;
+  }
+  const int64_t tiles = (2 * rows_per_tensor + kTile - 1) / kTile;
+  if ((int64_t)blockIdx.x >= tiles) return;
+
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  // resident hyperplanes: rows [0, sort_bits) from r_sort, then L*kr from r_race, zero padding
+  {
+    constexpr int kChunks = D / 8;
+    for (int i = tid; i < P16 * kChunks; i += kThreads) {
+      const int j = i / kChunks, ch = i % kChunks;
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (j < sort_bits)
+        val = *reinterpret_cast<const uint4*>(r_sort + (size_t)j * D + ch * 8);
+      else if (j < P)
+        val = *reinterpret_cast<const uint4*>(r_race + (size_t)(j - sort_bits) * D + ch * 8);
+      *reinterpret_cast<uint4*>(smem + (ch >> 3) * (P16 * 128) + sw128_off(j, ch & 7)) = val;
+    }
+  }
+  load_tile<D>(s_a, q, k, rows_per_tensor, blockIdx.x);
+  cp_async_commit();
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int npass = (P16 + kPass - 1) / kPass;
+  const int nslots = 1 + L;
+  uint32_t phase = 0;
+  bool ok = true;
+  int it = 0;
+  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
+    const uint32_t buf = nbuf == 2 ? (uint32_t)(it & 1) : 0u;
+    const int64_t next = tile + gridDim.x;
+    if (nbuf == 2 && next < tiles) {
+      load_tile<D>(s_a + (buf ^ 1u) * a_bytes, q, k, rows_per_tensor, next);
+      cp_async_commit();
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      cp_async_wait_all();
+    }
+    fence_async_smem();
+    __syncthreads();
+    const int64_t row = tile * kTile + tid;
+    const bool row_ok = row < 2 * rows_per_tensor;
+    uint64_t acc = 0;
+    int nacc = 0, slot = 0;
+    for (int p = 0; p < npass; ++p) {
+      const int ncol = min(kPass, P16 - p * kPass);
+      if (tid == 0) {
+        fence_after();
+        const uint32_t idesc = idesc_bf16(128, ncol, false, false);
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s) {
+          const uint32_t koff = (s >> 2) * (kTile * 128) + (s & 3) * 32;
+          const uint32_t roff = (s >> 2) * (P16 * 128) + p * kPass * 128 + (s & 3) * 32;
+          mma_bf16_ss(tmem, sw128_desc(s_a + buf * a_bytes + koff, 16, 1024),
+                      sw128_desc(s_r + roff, 16, 1024), idesc, s > 0);
+        }
+        mma_commit(bar);
+      }
+      ok = mbar_wait(bar, phase & 1, err);
+      ++phase;
+      if (__syncthreads_or(!ok)) break;
+      fence_after();
+      for (int c0 = 0; c0 < ncol; c0 += 32) {
+        const int valid = min(32, P - (p * kPass + c0));
+        float v[32];
+        tmem_ld32(tmem + lane_off + c0, v);
+        tmem_ld_wait();
+        if (valid <= 0) continue;
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) m |= (v[i] > 0.f ? 1u : 0u) << i;
+        if (valid < 32) m &= (1u << valid) - 1u;
+        acc |= (uint64_t)m << nacc;
+        nacc += valid;
+        while (slot < nslots) {
+          const int bits = slot == 0 ? sort_bits : kr;
+          if (nacc < bits) break;
+          const uint32_t val = (uint32_t)(acc & ((1ull << bits) - 1ull));
+          acc >>= bits;
+          nacc -= bits;
+          if (row_ok) {
+            if (slot == 0) code[row] = (uint16_t)val;
+            else rcode[row * L + slot - 1] = (CodeT)val;
+          }
+          ++slot;
+        }
+      }
+      fence_before();
+      __syncthreads();
+    }
+    if (!ok) break;
+    // zero-bit codes at the end of the stream
+    while (slot < nslots) {
+      if (row_ok) {
+        if (slot == 0) code[row] = 0;
+        else rcode[row * L + slot - 1] = 0;
+      }
+      ++slot;
+    }
+    if (nbuf == 1 && next < tiles) {
+      load_tile<D>(s_a, q, k, rows_per_tensor, next);
+      cp_async_commit();
+    }
+  }
+  cp_async_wait_all();
+  fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D, typename CodeT>
+cudaError_t run(const Geometry& g, const void* q, const void* k, const void* r_sort,
+                const void* r_race, uint16_t* code, void* rcode, uint32_t* err, cudaStream_t s) {
+  const HashShape h = hash_shape(g);
+  cudaError_t e = cudaFuncSetAttribute(hash_tc_kernel<D, CodeT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)h.dyn);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, hash_tc_kernel<D, CodeT>, kThreads,
+                                                    h.dyn);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);   // TMEM: 4 x 128 columns per SM
+  const int64_t rows = (int64_t)g.BH * g.N;
+  const int64_t tiles = (2 * rows + kTile - 1) / kTile;
+  const int64_t want = (int64_t)sms * per_sm;
+  const int grid = (int)(tiles < want ? tiles : want);
+  hash_tc_kernel<D, CodeT><<<grid, kThreads, h.dyn, s>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+      static_cast<const __nv_bfloat16*>(r_sort), static_cast<const __nv_bfloat16*>(r_race), rows,
+      g.sort_bits, g.L, g.kr, h.P, h.P16, h.nbuf, code, static_cast<CodeT*>(rcode), err);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool hash_tc_supported(const Geometry& g) {
+  if (!g.bf16 || (g.d != 64 && g.d != 128)) return false;
+  const HashShape h = hash_shape(g);
+  return h.P > 0 && h.dyn <= (uint32_t)kSmemLimit;
+}
+
+size_t hash_tc_scratch_bytes(const Geometry&) { return 0; }
+
+cudaError_t launch_hash_tc(const Geometry& g, const void* q, const void* k, const void* r_sort,
+                           const void* r_race, uint16_t* code, void* rcode, void*,
+                           uint32_t* err, cudaStream_t s) {
+  if (g.d == 64)
+    return g.rcode_bytes == 1 ? run<64, uint8_t>(g, q, k, r_sort, r_race, code, rcode, err, s)
+                              : run<64, uint16_t>(g, q, k, r_sort, r_race, code, rcode, err, s);
+  return g.rcode_bytes == 1 ? run<128, uint8_t>(g, q, k, r_sort, r_race, code, rcode, err, s)
+                            : run<128, uint16_t>(g, q, k, r_sort, r_race, code, rcode, err, s);
+}
+
+}  // namespace elsaa

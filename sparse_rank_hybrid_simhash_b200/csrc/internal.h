@@ -1,0 +1,117 @@
+// Host-side layout of the saved state and workspace, and the kernel
+// launchers each .cu file provides.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/elsaa.h"
+
+namespace elsaa {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+
+// Sort-LSH radix pass geometry: digit of at most 8 bits, tiles of kSortTile keys.
+constexpr int kSortTile = 2048;
+constexpr int kSortThreads = 256;
+
+struct Geometry {
+  int B, H, N, d, BH;
+  bool bf16;
+  int esz;            // bytes per element of q/k/v
+  int sort_bits, chunk, L, kr, NB;   // NB = 2^kr buckets
+  int rcode_bytes;    // 1 or 2
+  float scale;
+  int gate_fixed;      // nonzero: constant gates gate_s, gate_r
+  float gate_s, gate_r;
+  int sort_passes, sort_digit_bits, sort_bins, sort_tiles;
+  bool tc_hash;       // tcgen05 kernel for the SimHash codes
+  bool tc_attn;       // tcgen05 kernels for the sparse branch
+};
+
+// Byte offsets inside the saved buffer.
+struct SavedLayout {
+  size_t code, perm, rcode, race_count, race_sum, lse, o_sp, o_race, ctot, total;
+  // code = [2][BH][N] u16 (queries then keys); perm = [2][BH][N] i32;
+  // rcode = [2][BH][N][L] (u8 or u16)
+};
+
+// Byte offsets inside the workspace.
+struct WorkLayout {
+  size_t err;                // 256 bytes: uint32 error word and spare
+  size_t sort_hist;          // [2][BH][bins][tiles] i32
+  size_t sort_tmp;           // [2][BH][N] i32 (intermediate order of a 2-pass sort)
+  size_t saved;              // a SavedLayout used when the forward has no saved buffer
+  size_t d_o;                // [BH][N][d] dtype: dO_sp
+  size_t dprime;             // [BH][N] f32: D' = dO_sp . O_sp - dlse
+  size_t dq_acc, dk_acc, dv_acc;   // [BH][N][d] f32
+  size_t dor;                // [BH][N][d] f32: g_r dy / Ctot
+  size_t d_t;                // [BH][L][NB][d] f32: RACE table gradient
+  size_t partials;           // [kParamBlocks][2d+3] f32
+  size_t total;
+};
+
+constexpr int kParamBlocks = 592;   // 4 x 148 SMs; fixed so the reduction order is fixed
+
+bool make_geometry(const elsaa_params* p, Geometry* g, elsaa_status* why);
+SavedLayout saved_layout(const Geometry& g);
+WorkLayout work_layout(const Geometry& g);
+
+// ---- launchers (each returns cudaGetLastError() after enqueueing) ----------
+
+// SimHash codes of Q and K on CUDA cores (fp64 accumulation of exact products).
+cudaError_t launch_hash_simt(const Geometry& g, const void* q, const void* k, const void* r_sort,
+                             const void* r_race, uint16_t* code, void* rcode, cudaStream_t s);
+// SimHash codes on tcgen05 tensor cores (bf16 products, fp32 accumulation).
+cudaError_t launch_hash_tc(const Geometry& g, const void* q, const void* k, const void* r_sort,
+                           const void* r_race, uint16_t* code, void* rcode, void* scratch,
+                           uint32_t* err, cudaStream_t s);
+size_t hash_tc_scratch_bytes(const Geometry& g);
+bool hash_tc_supported(const Geometry& g);
+
+// Stable Sort-LSH order of the 2*BH code segments.
+cudaError_t launch_sort(const Geometry& g, const uint16_t* code, int32_t* perm, int32_t* hist,
+                        int32_t* tmp, cudaStream_t s);
+
+// RACE tables: sums[bh][l][b][:] = sum of vals rows whose code in table l is b;
+// counts (optional) likewise.  vals_f32 selects fp32 values instead of dtype.
+cudaError_t launch_race_build(const Geometry& g, const void* codes, const void* vals,
+                              bool vals_f32, float* sums, int32_t* counts, cudaStream_t s);
+// out[bh][i][:] = sum_l tables[bh][l][codes[bh][i][l]][:]  (f32, overwritten)
+cudaError_t launch_race_gather_sum(const Geometry& g, const void* codes, const float* tables,
+                                   float* out, cudaStream_t s);
+// Forward RACE gather fused with the gates, the multiplier and the output.
+cudaError_t launch_race_fuse_fwd(const Geometry& g, const void* q, const void* rcode_q,
+                                 const float* sums, const int32_t* counts, const void* o_sp,
+                                 const float* lse, const float* gate_w, const float* gate_b,
+                                 const float* lam, void* y, void* o_race, int32_t* ctot,
+                                 cudaStream_t s);
+
+// Sparse branch, CUDA-core kernels.
+cudaError_t launch_attn_fwd_simt(const Geometry& g, const void* q, const void* k, const void* v,
+                                 const int32_t* perm_q, const int32_t* perm_k, void* o_sp,
+                                 float* lse, cudaStream_t s);
+cudaError_t launch_attn_bwd_simt(const Geometry& g, const void* q, const void* k, const void* v,
+                                 const int32_t* perm_q, const int32_t* perm_k, const void* d_o,
+                                 const float* lse, const float* dprime, float* dq_acc,
+                                 float* dk_acc, float* dv_acc, cudaStream_t s);
+// Sparse branch, tcgen05 kernels.
+cudaError_t launch_attn_fwd_tc(const Geometry& g, const void* q, const void* k, const void* v,
+                               const int32_t* perm_q, const int32_t* perm_k, void* o_sp,
+                               float* lse, uint32_t* err, cudaStream_t s);
+bool attn_tc_supported(const Geometry& g);
+
+// Backward of the fusion and gates (per query), then the parameter reduction
+// and the final casts.
+cudaError_t launch_fuse_bwd(const Geometry& g, const void* q, const void* dy, const void* o_sp,
+                            const void* o_race, const float* lse, const int32_t* ctot,
+                            const float* gate_w, const float* gate_b, const float* lam,
+                            void* d_o, float* dprime, float* dq_acc, float* dor,
+                            float* partials, cudaStream_t s);
+cudaError_t launch_param_reduce(const Geometry& g, const float* partials, float* dgate_w,
+                                float* dgate_b, float* dlambda, cudaStream_t s);
+cudaError_t launch_cast_out(const Geometry& g, const float* src, void* dst, cudaStream_t s);
+
+}  // namespace elsaa

@@ -1,0 +1,152 @@
+// Sort-LSH ordering: a stable LSD radix sort of the sort codes of every
+// (tensor, batch, head) segment, ties kept in token order.
+//
+// The Sort-LSH hybrid of "Two Efficient Attentions, One Denominator Problem"
+// (section "The ablation isolates the actual contribution") orders tokens by
+// hash code so that a chunk of consecutive sorted tokens holds similar ones.
+// Each pass sorts by a digit of at most 8 bits in three launches:
+//   1. per-tile digit histograms (tiles of kSortTile keys, shared-memory counts);
+//   2. per-segment exclusive scan over (digit, tile), digit-major, so a tile's
+//      keys of one digit land after every earlier tile's keys of that digit;
+//   3. a stable scatter: warps own consecutive runs of the tile, count their
+//      digits, take per-warp bases, then rank equal digits within each
+//      32-key round with __match_any_sync.
+// Codes of up to 16 bits take two passes (the second reads the first's order).
+#include "common.cuh"
+#include "internal.h"
+
+namespace elsaa {
+namespace {
+
+constexpr int kWarps = kSortThreads / 32;
+constexpr int kPerWarp = kSortTile / kWarps;   // 256 keys, 8 rounds of 32
+
+__global__ void __launch_bounds__(kSortThreads)
+sort_hist_kernel(const uint16_t* __restrict__ code, const int32_t* __restrict__ order_in,
+                 int N, int shift, int mask, int bins, int tiles, int32_t* __restrict__ hist) {
+  __shared__ int h[256];
+  for (int i = threadIdx.x; i < bins; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  const int seg = blockIdx.y, tile = blockIdx.x;
+  const uint16_t* c = code + (size_t)seg * N;
+  const int32_t* oin = order_in ? order_in + (size_t)seg * N : nullptr;
+  const int p0 = tile * kSortTile, p1 = min(N, p0 + kSortTile);
+  for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
+    const int idx = oin ? oin[p] : p;
+    atomicAdd(&h[(c[idx] >> shift) & mask], 1);
+  }
+  __syncthreads();
+  for (int b = threadIdx.x; b < bins; b += blockDim.x)
+    hist[((size_t)seg * bins + b) * tiles + tile] = h[b];
+}
+
+// In-place exclusive scan of n counts per segment (one block per segment).
+__global__ void __launch_bounds__(1024) sort_scan_kernel(int32_t* __restrict__ hist, int n) {
+  __shared__ int warp_tot[32];
+  int32_t* a = hist + (size_t)blockIdx.x * n;
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int lo = threadIdx.x * per, hi = min(n, lo + per);
+  int local = 0;
+  for (int i = lo; i < hi; ++i) local += a[i];
+  // block exclusive scan of `local`
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) warp_tot[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int v = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += t;
+    }
+    warp_tot[lane] = v;   // inclusive over warps
+  }
+  __syncthreads();
+  int run = incl - local + (w > 0 ? warp_tot[w - 1] : 0);
+  for (int i = lo; i < hi; ++i) {
+    const int t = a[i];
+    a[i] = run;
+    run += t;
+  }
+}
+
+__global__ void __launch_bounds__(kSortThreads)
+sort_scatter_kernel(const uint16_t* __restrict__ code, const int32_t* __restrict__ order_in,
+                    int N, int shift, int mask, int bins, int tiles,
+                    const int32_t* __restrict__ offs, int32_t* __restrict__ order_out) {
+  __shared__ int cnt[kWarps][256];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int seg = blockIdx.y, tile = blockIdx.x;
+  const uint16_t* c = code + (size_t)seg * N;
+  const int32_t* oin = order_in ? order_in + (size_t)seg * N : nullptr;
+  int32_t* out = order_out + (size_t)seg * N;
+  for (int i = threadIdx.x; i < kWarps * 256; i += blockDim.x) (&cnt[0][0])[i] = 0;
+  __syncthreads();
+  const int base_p = tile * kSortTile + w * kPerWarp;
+  const unsigned lt = (1u << lane) - 1u;
+  // pass A: digit counts of this warp's run
+  for (int r = 0; r < kPerWarp / 32; ++r) {
+    const int p = base_p + r * 32 + lane;
+    const bool valid = p < N;
+    const int idx = valid ? (oin ? oin[p] : p) : 0;
+    const int key = valid ? ((c[idx] >> shift) & mask) : (bins + lane);
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    if (valid && lane == __ffs(peers) - 1) cnt[w][key] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // per-warp bases: the tile's global offset for the digit plus earlier warps' counts
+  for (int b = threadIdx.x; b < bins; b += blockDim.x) {
+    int run = offs[((size_t)seg * bins + b) * tiles + tile];
+    for (int ww = 0; ww < kWarps; ++ww) {
+      const int t = cnt[ww][b];
+      cnt[ww][b] = run;
+      run += t;
+    }
+  }
+  __syncthreads();
+  // pass B: stable ranks inside each round, rounds in token order
+  for (int r = 0; r < kPerWarp / 32; ++r) {
+    const int p = base_p + r * 32 + lane;
+    const bool valid = p < N;
+    const int idx = valid ? (oin ? oin[p] : p) : 0;
+    const int key = valid ? ((c[idx] >> shift) & mask) : (bins + lane);
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    int pos = 0;
+    if (valid) pos = cnt[w][key] + __popc(peers & lt);
+    __syncwarp();
+    if (valid) {
+      out[pos] = idx;
+      if (lane == __ffs(peers) - 1) cnt[w][key] += __popc(peers);
+    }
+    __syncwarp();
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_sort(const Geometry& g, const uint16_t* code, int32_t* perm, int32_t* hist,
+                        int32_t* tmp, cudaStream_t s) {
+  const int segs = 2 * g.BH;
+  const dim3 grid(g.sort_tiles, segs);
+  const int mask = g.sort_bins - 1;
+  for (int pass = 0; pass < g.sort_passes; ++pass) {
+    const int shift = pass * g.sort_digit_bits;
+    const int32_t* in = pass == 0 ? nullptr : tmp;
+    int32_t* out = (pass == g.sort_passes - 1) ? perm : tmp;
+    sort_hist_kernel<<<grid, kSortThreads, 0, s>>>(code, in, g.N, shift, mask, g.sort_bins,
+                                                   g.sort_tiles, hist);
+    sort_scan_kernel<<<segs, 1024, 0, s>>>(hist, g.sort_bins * g.sort_tiles);
+    sort_scatter_kernel<<<grid, kSortThreads, 0, s>>>(code, in, g.N, shift, mask, g.sort_bins,
+                                                      g.sort_tiles, hist, out);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace elsaa

@@ -1,0 +1,125 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol,
+and its host-side validation and sizing behave as include/elsaa.h states."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_rank_hybrid_simhash_b200 import binding as B
+from sparse_rank_hybrid_simhash_b200.workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "elsaa.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(elsaa_[a-z_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = B.lib()
+    names = declared_functions()
+    assert "elsaa_forward" in names and "elsaa_backward" in names
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(B.EXPORTS) <= set(names)
+
+
+def test_params_struct_matches_header_field_order():
+    text = open(HEADER).read()
+    body = text[text.index("typedef struct {"):text.index("} elsaa_params;")]
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = []
+    for decl in body.split(";"):
+        decl = decl.replace("typedef struct {", "").strip()
+        if not decl:
+            continue
+        names = decl.split(None, 1)[1]
+        fields += [n.strip() for n in names.split(",")]
+    assert fields == [f[0] for f in B.Params._fields_]
+
+
+def test_status_strings():
+    lib = B.lib()
+    for code, text in B.STATUS.items():
+        assert lib.elsaa_status_str(code).decode() == text
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_workloads_validate_and_size(name):
+    w = WORKLOADS[name]
+    p = B.Params.from_workload(w)
+    assert B.validate(p) == 0
+    bhn = w.B * w.H * w.N
+    esz = 2 if w.dtype == "bf16" else 4
+    saved = B.saved_bytes(p)
+    # codes, perms, RACE codes, tables, lse, O_sp, O_race, Ctot
+    expect = (2 * bhn * 2 + 2 * bhn * 4 + 2 * bhn * w.race_tables * (1 if w.race_bits <= 8 else 2)
+              + w.B * w.H * w.race_tables * (1 << w.race_bits) * (4 + 4 * w.d)
+              + bhn * 4 * 2 + 2 * bhn * w.d * esz)
+    assert expect <= saved <= expect + 256 * 16
+    assert B.workspace_bytes(p) >= saved
+
+
+def test_validation_rejects_bad_problems():
+    good = B.Params.make(1, 2, 256, 64, "bf16", 4, 64, 8, 6)
+    assert B.validate(good) == 0
+    cases = [
+        dict(N=250),                 # N not a multiple of the chunk
+        dict(chunk=0),
+        dict(d=0),
+        dict(sort_bits=17),
+        dict(race_bits=17),
+        dict(race_tables=0),
+        dict(dtype=7),
+    ]
+    for c in cases:
+        p = B.Params.make(1, 2, 256, 64, "bf16", 4, 64, 8, 6)
+        for k, v in c.items():
+            setattr(p, k, v)
+        assert B.validate(p) == 1, c
+        assert B.workspace_bytes(p) == 0 and B.saved_bytes(p) == 0
+    p = B.Params.make(1, 2, 256, 48, "bf16", 4, 64, 8, 6)   # head dim not a multiple of 32
+    assert B.validate(p) == 2
+
+
+def test_null_pointers_are_rejected_before_any_launch():
+    p = B.Params.make(1, 1, 256, 64, "bf16", 4, 64, 8, 6)
+    lib = B.lib()
+    null = ctypes.c_void_p(None)
+    code = lib.elsaa_forward(ctypes.byref(p), *([null] * 10), null, 0, null)
+    assert code == 1
+    code = lib.elsaa_backward(ctypes.byref(p), *([null] * 17), 0, null)
+    assert code == 1
+    assert lib.elsaa_check(null, null) == 1
+
+
+def test_workspace_too_small_is_reported():
+    p = B.Params.make(1, 1, 256, 64, "bf16", 4, 64, 8, 6, gate_fixed=True)
+    lib = B.lib()
+    fake = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced: validation fails first
+    args = [fake] * 5 + [ctypes.c_void_p(None)] * 2 + [fake, fake, ctypes.c_void_p(None)]
+    code = lib.elsaa_forward(ctypes.byref(p), *args, fake, B.workspace_bytes(p) - 256,
+                             ctypes.c_void_p(None))
+    assert code == 3
+
+
+def test_misaligned_buffers_are_rejected():
+    p = B.Params.make(1, 1, 256, 64, "bf16", 4, 64, 8, 6, gate_fixed=True)
+    lib = B.lib()
+    good, bad = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 20) + 8)
+    args = [bad] + [good] * 4 + [ctypes.c_void_p(None)] * 2 + [good, good, ctypes.c_void_p(None)]
+    code = lib.elsaa_forward(ctypes.byref(p), *args, good, B.workspace_bytes(p),
+                             ctypes.c_void_p(None))
+    assert code == 1
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_tensor_core_path_selection(name):
+    w = WORKLOADS[name]
+    expect = w.dtype == "bf16"   # every bf16 workload tiles onto the tcgen05 kernels
+    assert B.uses_tensor_cores(B.Params.from_workload(w)) == expect

@@ -332,3 +332,12 @@ def test_interaction_count_example_order_of_magnitude():
     cnt = O.interaction_count(32768, 128, 64)
     per_query = cnt["total"] / 32768
     assert abs(per_query - gold["elsaa_interactions"] / n) < 1.0
+
+
+def test_zero_race_bits_through_forward_head():
+    # K_r = 0: one bucket per table, every key collides with every query
+    q, k, v, rs, _, gw, gb = _unit(32, 4, 8, 2, 3, 2, seed=80)
+    rr = torch.zeros(3, 0, 4, dtype=F64)
+    out = O.forward_head(q, k, v, rs, rr, 8, None, gw, gb, lam=1.0)
+    assert (out["ctot"] == 3 * 32).all()
+    assert torch.allclose(out["o_race"], v.mean(0).expand(32, 4), atol=1e-12)
