@@ -1,0 +1,423 @@
+"""Benchmark of the ELSAA attention operator (libelsaa) on B200.
+
+One step = one forward and one backward of the whole operator (SimHash codes,
+Sort-LSH order, RACE build, sparse branch, RACE gather + fusion, and their
+backward) over one batch of the text-32k workload: B2 H12 N32768 d64 bf16,
+7-bit Sort-LSH, chunk 128, RACE 32 x 8-bit, learned gates.  Inputs are seeded
+synthetic tensors resident in HBM before the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch (weak
+scaling, different seed per rank); the shared gate and lambda gradients are
+summed across ranks with one NCCL all-reduce inside the step.  Time is device
+time (CUDA events on the launching stream), max over ranks.  Rank 0 prints one
+JSON line.
+
+``--impl reference`` times the fp64 CPU oracle (the reference arm: there is no
+runnable reference implementation) on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from sparse_rank_hybrid_simhash_b200 import binding as B  # noqa: E402
+from sparse_rank_hybrid_simhash_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "ELSAA attn tokens/s fwd and fwd+bwd at N=32K,d=64 bf16; % of roofline"
+WORKLOAD = "text-32k"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "sm_max_mhz": p.get("sm_max_mhz", 1965.0), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per stage (what the method must do, not what a kernel does)
+# ---------------------------------------------------------------------------
+
+def window_keys(N: int, c: int) -> int:
+    """sum over queries of the keys in their Sort-LSH window (own + previous chunk)."""
+    return sum(c * (min((j + 1) * c, N) - max(0, (j - 1) * c)) for j in range(N // c))
+
+
+def stage_work(w):
+    BH, N, d, L, NB = w.B * w.H, w.N, w.d, w.race_tables, 1 << w.race_bits
+    e = 2 if w.dtype == "bf16" else 4
+    rb = 1 if w.race_bits <= 8 else 2
+    P = w.sort_bits + L * w.race_bits
+    wk = window_keys(N, w.chunk) * BH       # query-key pairs of the sparse branch
+    rows = BH * N
+    return {
+        # bound, amount, unit
+        "hash": ("tensor", 2.0 * 2 * rows * d * P, "flop"),
+        "sort": ("hbm", 2 * rows * (2 + 4) * 1.0, "byte"),
+        "race_build": ("alu", 1.0 * rows * L * d, "add"),
+        "sparse_fwd": ("tensor", 4.0 * wk * d, "flop"),
+        "race_fuse": ("hbm", 1.0 * rows * (L * rb + 4 * d * e + 8 + 4), "byte"),
+        "fuse_bwd": ("hbm", 1.0 * rows * (4 * d * e + d * e + 8 * d + 12), "byte"),
+        "race_bwd": ("alu", 2.0 * rows * L * d, "add"),
+        "sparse_bwd": ("tensor", 10.0 * wk * d, "flop"),
+        "finish": ("hbm", 1.0 * rows * d * (4 + e), "byte"),
+    }
+
+
+def operator_roofline(w, peaks):
+    """The whole operator's roofline: max(flops / tensor peak, bytes / HBM peak)."""
+    BH, N, d = w.B * w.H, w.N, w.d
+    e = 2 if w.dtype == "bf16" else 4
+    P = w.sort_bits + w.race_tables * w.race_bits
+    wk = window_keys(N, w.chunk) * BH
+    rows = BH * N
+    f_fwd = 2.0 * 2 * rows * d * P + 4.0 * wk * d
+    f_bwd = 10.0 * wk * d
+    b_fwd = 4.0 * rows * d * e
+    b_all = b_fwd + 2 * (rows * d * e + 8 * rows) + 7.0 * rows * d * e
+    tf, hb = peaks["bf16_tflops"] * 1e12, peaks["hbm_gbs"] * 1e9
+    return {"fwd_us": 1e6 * max(f_fwd / tf, b_fwd / hb),
+            "fwdbwd_us": 1e6 * max((f_fwd + f_bwd) / tf, b_all / hb),
+            "flops_fwd": f_fwd, "flops_fwdbwd": f_fwd + f_bwd, "bytes_fwd": b_fwd,
+            "bytes_fwdbwd": b_all}
+
+
+def alu_peak_adds_per_s(peaks):
+    """Shared-memory fp32 atomic adds per second: 148 SMs x 32 lanes per clock
+    (one conflict-free warp-wide shared atomic per SM per clock) at max SM clock."""
+    return 148 * 32 * peaks["sm_max_mhz"] * 1e6
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.proc = None
+        self.index = index
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out = ""
+        return False
+
+    def summary(self):
+        rows = [r.split(",") for r in self.out.strip().splitlines() if r.count(",") >= 7]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[0]) for r in rows if r[0].strip().replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if r[4 + i].strip().lower() == "active"})
+        loaded = [s for s in sm if s > 0.5 * max(sm)] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    p = B.Params.from_workload(w)
+    inp = make_inputs(w, seed=w.seed + rank, with_dy=True)
+    d = {k: t.to(dev) for k, t in inp.items()}
+    saved = B.alloc_saved(p, dev)
+    ws = B.alloc_workspace(p, dev)
+    y = torch.empty_like(d["q"])
+    grads = [torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"]),
+             torch.empty(2, w.d, dtype=torch.float32, device=dev),
+             torch.empty(2, dtype=torch.float32, device=dev),
+             torch.empty(1, dtype=torch.float32, device=dev)]
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    nf, nb = len(B.FWD_STAGES), len(B.BWD_STAGES)
+
+    def step(ev_f=None, ev_b=None):
+        B.forward(p, d["q"], d["k"], d["v"], d["r_sort"], d["r_race"], d["gate_w"], d["gate_b"],
+                  d["lam"], y=y, saved=saved, ws=ws, events=ev_f)
+        B.backward(p, d["q"], d["k"], d["v"], d["r_sort"], d["r_race"], d["gate_w"],
+                   d["gate_b"], d["lam"], saved, d["dy"], *grads, ws=ws, events=ev_b)
+        if world > 1:
+            pg = torch.cat([grads[3].view(-1), grads[4].view(-1), grads[5].view(-1)])
+            torch.distributed.all_reduce(pg)
+            n = grads[3].numel()
+            grads[3].view(-1).copy_(pg[:n])
+            grads[4].copy_(pg[n:n + 2])
+            grads[5].copy_(pg[n + 2:])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    B.check(ws)
+
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    evs = [([mk() for _ in range(nf + 1)], [mk() for _ in range(nb + 1)], mk())
+           for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)            # L2 flush between timed steps, outside the events
+            ef, eb, end = evs[i]
+            step(ef, eb)
+            end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    B.check(ws)
+    step_ms = [ef[0].elapsed_time(end) for ef, eb, end in evs]
+    fwd_ms = [ef[0].elapsed_time(ef[-1]) for ef, eb, end in evs]
+    stage_ms = {}
+    for j, name in enumerate(B.FWD_STAGES):
+        stage_ms[name] = statistics.mean(ef[j].elapsed_time(ef[j + 1]) for ef, eb, end in evs)
+    for j, name in enumerate(B.BWD_STAGES):
+        stage_ms[name] = statistics.mean(eb[j].elapsed_time(eb[j + 1]) for ef, eb, end in evs)
+    total_ms = sum(step_ms)
+    fwd_total = sum(fwd_ms)
+    if world > 1:
+        t = torch.tensor([total_ms, fwd_total], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms, fwd_total = t.tolist()
+
+    # end to end through the public API with host buffers
+    e2e = run_e2e(args, w, p, inp, dev, world)
+    return w, p, total_ms, fwd_total, stage_ms, clk.summary(), e2e
+
+
+def run_e2e(args, w, p, inp, dev, world):
+    host = {k: inp[k].pin_memory() for k in ("q", "k", "v", "dy")}
+    outs = {k: torch.empty_like(host[k], pin_memory=True) for k in ("q", "k", "v", "dy")}
+    pg_host = torch.empty(2 * w.d + 3, dtype=torch.float32, pin_memory=True)
+    small = {k: inp[k].to(dev) for k in ("r_sort", "r_race", "gate_w", "gate_b", "lam")}
+    dq = {k: torch.empty(host[k].shape, dtype=host[k].dtype, device=dev) for k in host}
+    saved = B.alloc_saved(p, dev)
+    ws = B.alloc_workspace(p, dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for k in host:
+            dq[k].copy_(host[k], non_blocking=True)
+        y = B.forward(p, dq["q"], dq["k"], dq["v"], small["r_sort"], small["r_race"],
+                      small["gate_w"], small["gate_b"], small["lam"], saved=saved, ws=ws)
+        g = B.backward(p, dq["q"], dq["k"], dq["v"], small["r_sort"], small["r_race"],
+                       small["gate_w"], small["gate_b"], small["lam"], saved, dq["dy"], ws=ws)
+        pg = torch.cat([g[3].view(-1), g[4].view(-1), g[5].view(-1)])
+        if world > 1:
+            torch.distributed.all_reduce(pg)
+        outs["q"].copy_(g[0], non_blocking=True)
+        outs["k"].copy_(g[1], non_blocking=True)
+        outs["v"].copy_(g[2], non_blocking=True)
+        outs["dy"].copy_(y, non_blocking=True)
+        pg_host.copy_(pg, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    n = max(1, min(args.steps, 3))
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    start.record(stream)
+    for _ in range(n):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = t.item()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs.values()) + pg_host.numel() * 4
+    return {"value": world * n * w.tokens / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n}
+
+
+# ---------------------------------------------------------------------------
+# the oracle as CPU baseline and as the reference arm
+# ---------------------------------------------------------------------------
+
+def oracle_unit_seconds(w, inp, units):
+    import oracle as O
+    t0 = time.perf_counter()
+    for (b, h) in units:
+        args = (inp["q"][b, h], inp["k"][b, h], inp["v"][b, h], inp["r_sort"], inp["r_race"],
+                w.chunk)
+        O.grads_head(*args, inp["dy"][b, h], None, inp["gate_w"], inp["gate_b"],
+                     float(inp["lam"][0]))
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, units=8):
+    cores = len(os.sched_getaffinity(0))
+    torch.set_num_threads(cores)
+    inp = make_inputs(w, with_dy=True)
+    sel = [(i // w.H % w.B, i % w.H) for i in range(units)]
+    secs = oracle_unit_seconds(w, inp, sel)
+    # one (batch, head) unit is N / H token-equivalents of the B x N-token step
+    value = units * w.N / w.H / secs
+    return {"value": value, "unit": "tokens/s", "cores": torch.get_num_threads(),
+            "kind": "oracle",
+            "sample": f"{units} of {w.B * w.H} (batch, head) units of {w.name}, forward+backward "
+                      f"in fp64 ({secs:.1f} s), scaled to the whole step"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    cores = len(os.sched_getaffinity(0))
+    torch.set_num_threads(cores)
+    inp = make_inputs(w, with_dy=True)
+    per_step = 2
+    units = [(i // w.H % w.B, i % w.H) for i in range(w.B * w.H)]
+    for i in range(args.warmup):
+        oracle_unit_seconds(w, inp, units[:1])
+    secs = []
+    for i in range(args.steps):
+        sel = [units[(i * per_step + j) % len(units)] for j in range(per_step)]
+        secs.append(oracle_unit_seconds(w, inp, sel))
+    total = sum(secs)
+    value = args.steps * per_step * w.N / w.H / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps * (w.B * w.H / per_step),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; stands in for the ArXiv 32K text task)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "sort_bits": w.sort_bits, "chunk": w.chunk, "race_tables": w.race_tables,
+                   "race_bits": w.race_bits, "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": torch.get_num_threads(),
+                         "kind": "oracle",
+                         "sample": f"{per_step} of {w.B * w.H} (batch, head) units per step, "
+                                   "forward+backward in fp64, scaled to the whole step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    w, p, total_ms, fwd_ms, stage_ms, clocks, e2e = run_ours(args, rank, world, local_rank)
+    peaks = load_peaks()
+    if rank == 0:
+        K = args.steps
+        value = world * K * w.tokens / (total_ms / 1e3)
+        fwd_value = world * K * w.tokens / (fwd_ms / 1e3)
+        work = stage_work(w)
+        dom = max(stage_ms, key=lambda s: stage_ms[s])
+        bound, amount, unit = work[dom]
+        sec = stage_ms[dom] / 1e3
+        if bound == "tensor":
+            ach, peak, u = amount / sec / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
+        elif bound == "hbm":
+            ach, peak, u = amount / sec / 1e9, peaks["hbm_gbs"], "GB/s"
+        else:
+            ach, peak, u = amount / sec / 1e9, alu_peak_adds_per_s(peaks) / 1e9, "Gadd/s"
+        roof = operator_roofline(w, peaks)
+        fwd_launch, bwd_launch = B.kernel_launches(p)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; stands in for the ArXiv 32K text task)",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                       "sort_bits": w.sort_bits, "chunk": w.chunk,
+                       "race_tables": w.race_tables, "race_bits": w.race_bits,
+                       "global_batch": world * w.B, "seq_len": w.N,
+                       "parallelism": f"dp{world}",
+                       "l2": "256 MB flush between timed steps; inputs 0.4 GB > L2"},
+            "fwd_tokens_per_s": fwd_value,
+            "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+            "roofline": {"bound": bound, "kernel": dom, "achieved": ach, "peak": peak,
+                         "unit": u, "frac": ach / peak, "traffic": None,
+                         "peak_source": peaks["source"] + (" sustained" if bound == "tensor"
+                                                           else "")},
+            "operator_roofline": {
+                "fwd_us": roof["fwd_us"], "fwdbwd_us": roof["fwdbwd_us"],
+                "frac_fwd": roof["fwd_us"] / (1e3 * fwd_ms / K),
+                "frac_fwdbwd": roof["fwdbwd_us"] / (1e3 * total_ms / K)},
+            "gpu_launches": K * (fwd_launch + bwd_launch),
+            "clocks": clocks,
+            "e2e": e2e,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

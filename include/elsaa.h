@@ -135,6 +135,33 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* q, const void* k,
                             float* dgate_b, float* dlambda, void* ws, size_t ws_bytes,
                             void* stream);
 
+/* Stages of one call, for per-kernel timing: elsaa_forward_staged and
+ * elsaa_backward_staged take `events`, an array of ELSAA_*_STAGES + 1
+ * cudaEvent_t handles (passed as void*; any entry may be NULL) created by the
+ * caller; events[0] is recorded on `stream` before the first stage and
+ * events[i + 1] after stage i.  Forward stages: SimHash codes, Sort-LSH
+ * order, RACE build, sparse branch, RACE gather + fusion.  Backward stages:
+ * fusion/gate backward, RACE backward, sparse backward, final casts and the
+ * parameter-gradient reduction.  Otherwise identical to elsaa_forward and
+ * elsaa_backward (which are these calls with events = NULL). */
+#define ELSAA_FWD_STAGES 5
+#define ELSAA_BWD_STAGES 4
+elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const void* k,
+                                  const void* v, const void* r_sort, const void* r_race,
+                                  const float* gate_w, const float* gate_b, const float* lambda,
+                                  void* y, void* saved, void* ws, size_t ws_bytes, void* stream,
+                                  void* const* events);
+elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const void* k,
+                                   const void* v, const void* r_sort, const void* r_race,
+                                   const float* gate_w, const float* gate_b, const float* lambda,
+                                   const void* saved, const void* dy, void* dq, void* dk, void* dv,
+                                   float* dgate_w, float* dgate_b, float* dlambda, void* ws,
+                                   size_t ws_bytes, void* stream, void* const* events);
+
+/* Number of kernels one elsaa_forward (fwd) and one elsaa_backward (bwd)
+ * enqueue for `p` (memsets excluded). */
+elsaa_status elsaa_kernel_launches(const elsaa_params* p, int32_t* fwd, int32_t* bwd);
+
 /* Fills `out` with device pointers into `saved` (no device access). */
 elsaa_status elsaa_saved_views(const elsaa_params* p, const void* saved, elsaa_views* out);
 

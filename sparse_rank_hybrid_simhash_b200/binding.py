@@ -66,8 +66,11 @@ class Views(ctypes.Structure):
 
 
 EXPORTS = ("elsaa_validate", "elsaa_workspace_bytes", "elsaa_saved_bytes", "elsaa_forward",
-           "elsaa_backward", "elsaa_saved_views", "elsaa_check", "elsaa_status_str",
+           "elsaa_backward", "elsaa_forward_staged", "elsaa_backward_staged",
+           "elsaa_kernel_launches", "elsaa_saved_views", "elsaa_check", "elsaa_status_str",
            "elsaa_uses_tensor_cores")
+FWD_STAGES = ("hash", "sort", "race_build", "sparse_fwd", "race_fuse")
+BWD_STAGES = ("fuse_bwd", "race_bwd", "sparse_bwd", "finish")
 
 _lib = None
 
@@ -91,6 +94,13 @@ def lib() -> ctypes.CDLL:
     L.elsaa_forward.restype = st
     L.elsaa_backward.argtypes = [P] + [vp] * 17 + [sz, vp]
     L.elsaa_backward.restype = st
+    L.elsaa_forward_staged.argtypes = [P] + [vp] * 10 + [vp, sz, vp, vp]
+    L.elsaa_forward_staged.restype = st
+    L.elsaa_backward_staged.argtypes = [P] + [vp] * 17 + [sz, vp, vp]
+    L.elsaa_backward_staged.restype = st
+    L.elsaa_kernel_launches.argtypes = [P, ctypes.POINTER(ctypes.c_int32),
+                                        ctypes.POINTER(ctypes.c_int32)]
+    L.elsaa_kernel_launches.restype = st
     L.elsaa_saved_views.argtypes = [P, vp, ctypes.POINTER(Views)]
     L.elsaa_saved_views.restype = st
     L.elsaa_check.argtypes, L.elsaa_check.restype = [vp, vp], st
@@ -129,6 +139,29 @@ def uses_tensor_cores(p: Params) -> bool:
     return bool(lib().elsaa_uses_tensor_cores(ctypes.byref(p)))
 
 
+def kernel_launches(p: Params):
+    """(kernels per forward, kernels per backward) for ``p``."""
+    f, b = ctypes.c_int32(), ctypes.c_int32()
+    _ok("elsaa_kernel_launches", lib().elsaa_kernel_launches(ctypes.byref(p), ctypes.byref(f),
+                                                            ctypes.byref(b)))
+    return f.value, b.value
+
+
+def _events(events):
+    """ctypes array of cudaEvent_t handles from torch.cuda.Event objects (or None)."""
+    if events is None:
+        return None
+    handles = []
+    for e in events:
+        if e is None:
+            handles.append(None)
+            continue
+        if e.cuda_event == 0:      # torch creates the event on first record
+            e.record()
+        handles.append(e.cuda_event)
+    return (ctypes.c_void_p * len(handles))(*handles)
+
+
 def alloc_workspace(p: Params, device) -> torch.Tensor:
     return torch.empty(max(workspace_bytes(p), 256), dtype=torch.uint8, device=device)
 
@@ -138,21 +171,25 @@ def alloc_saved(p: Params, device) -> torch.Tensor:
 
 
 def forward(p: Params, q, k, v, r_sort, r_race, gate_w, gate_b, lam, y=None, saved=None,
-            ws=None, stream=None) -> torch.Tensor:
-    """y = ELSAA(q, k, v); writes the saved state into ``saved`` when given."""
+            ws=None, stream=None, events=None) -> torch.Tensor:
+    """y = ELSAA(q, k, v); writes the saved state into ``saved`` when given.
+    ``events``: optional list of len(FWD_STAGES) + 1 torch.cuda.Event recorded
+    around each stage."""
     if y is None:
         y = torch.empty_like(q)
     if ws is None:
         ws = alloc_workspace(p, q.device)
-    code = lib().elsaa_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(r_sort),
-                               _ptr(r_race), _ptr(gate_w), _ptr(gate_b), _ptr(lam), _ptr(y),
-                               _ptr(saved), _ptr(ws), ws.numel(), _stream(stream))
+    code = lib().elsaa_forward_staged(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(r_sort),
+                                      _ptr(r_race), _ptr(gate_w), _ptr(gate_b), _ptr(lam),
+                                      _ptr(y), _ptr(saved), _ptr(ws), ws.numel(),
+                                      _stream(stream), _events(events))
     _ok("elsaa_forward", code)
     return y
 
 
 def backward(p: Params, q, k, v, r_sort, r_race, gate_w, gate_b, lam, saved, dy, dq=None,
-             dk=None, dv=None, dgate_w=None, dgate_b=None, dlam=None, ws=None, stream=None):
+             dk=None, dv=None, dgate_w=None, dgate_b=None, dlam=None, ws=None, stream=None,
+             events=None):
     """Gradients of sum(y * dy): (dq, dk, dv, dgate_w, dgate_b, dlambda)."""
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
@@ -163,11 +200,11 @@ def backward(p: Params, q, k, v, r_sort, r_race, gate_w, gate_b, lam, saved, dy,
     dlam = torch.empty(1, dtype=torch.float32, device=dev) if dlam is None else dlam
     if ws is None:
         ws = alloc_workspace(p, dev)
-    code = lib().elsaa_backward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(r_sort),
-                                _ptr(r_race), _ptr(gate_w), _ptr(gate_b), _ptr(lam),
-                                _ptr(saved), _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv),
-                                _ptr(dgate_w), _ptr(dgate_b), _ptr(dlam), _ptr(ws), ws.numel(),
-                                _stream(stream))
+    code = lib().elsaa_backward_staged(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(r_sort),
+                                       _ptr(r_race), _ptr(gate_w), _ptr(gate_b), _ptr(lam),
+                                       _ptr(saved), _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv),
+                                       _ptr(dgate_w), _ptr(dgate_b), _ptr(dlam), _ptr(ws),
+                                       ws.numel(), _stream(stream), _events(events))
     _ok("elsaa_backward", code)
     return dq, dk, dv, dgate_w, dgate_b, dlam
 

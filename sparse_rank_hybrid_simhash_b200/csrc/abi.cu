@@ -101,6 +101,11 @@ namespace {
 
 inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
+inline cudaError_t mark(void* const* events, int i, cudaStream_t s) {
+  if (!events || !events[i]) return cudaSuccess;
+  return cudaEventRecord((cudaEvent_t)events[i], s);
+}
+
 #define ELSAA_TRY(expr)                               \
   do {                                                \
     if ((expr) != cudaSuccess) return ELSAA_ERR_CUDA; \
@@ -162,10 +167,11 @@ elsaa_status elsaa_saved_views(const elsaa_params* p, const void* saved, elsaa_v
   return ELSAA_OK;
 }
 
-elsaa_status elsaa_forward(const elsaa_params* p, const void* q, const void* k, const void* v,
-                           const void* r_sort, const void* r_race, const float* gate_w,
-                           const float* gate_b, const float* lambda, void* y, void* saved,
-                           void* ws, size_t ws_bytes, void* stream) {
+elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const void* k,
+                                  const void* v, const void* r_sort, const void* r_race,
+                                  const float* gate_w, const float* gate_b, const float* lambda,
+                                  void* y, void* saved, void* ws, size_t ws_bytes, void* stream,
+                                  void* const* events) {
   Geometry g;
   elsaa_status why;
   if (!make_geometry(p, &g, &why)) return why;
@@ -193,35 +199,49 @@ elsaa_status elsaa_forward(const elsaa_params* p, const void* q, const void* k, 
   void* o_sp = sv + sl.o_sp;
   uint32_t* err = (uint32_t*)(w + wl.err);
   ELSAA_TRY(cudaMemsetAsync(err, 0, sizeof(uint32_t), s));
+  ELSAA_TRY(mark(events, 0, s));
 
   // 1. SimHash codes of Q and K
   if (g.tc_hash)
     ELSAA_TRY(launch_hash_tc(g, q, k, r_sort, r_race, code, rcode, nullptr, err, s));
   else
     ELSAA_TRY(launch_hash_simt(g, q, k, r_sort, r_race, code, rcode, s));
+  ELSAA_TRY(mark(events, 1, s));
   // 2. Sort-LSH order of Q and K
   ELSAA_TRY(launch_sort(g, code, perm, (int32_t*)(w + wl.sort_hist), (int32_t*)(w + wl.sort_tmp),
                         s));
+  ELSAA_TRY(mark(events, 2, s));
   // 3. RACE tables from the keys
   ELSAA_TRY(launch_race_build(g, rcode_k, v, false, sums, counts, s));
+  ELSAA_TRY(mark(events, 3, s));
   // 4. exact sparse branch
   if (g.tc_attn)
     ELSAA_TRY(launch_attn_fwd_tc(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s));
   else
     ELSAA_TRY(launch_attn_fwd_simt(g, q, k, v, perm, perm + bhn, o_sp, lse, s));
+  ELSAA_TRY(mark(events, 4, s));
   // 5. RACE gather, gates, multiplier and output
   ELSAA_TRY(launch_race_fuse_fwd(g, q, rcode, sums, counts, o_sp, lse, gate_w, gate_b, lambda, y,
                                  saved ? sv + sl.o_race : nullptr,
                                  saved ? (int32_t*)(sv + sl.ctot) : nullptr, s));
+  ELSAA_TRY(mark(events, 5, s));
   return ELSAA_OK;
 }
 
-elsaa_status elsaa_backward(const elsaa_params* p, const void* q, const void* k, const void* v,
-                            const void* r_sort, const void* r_race, const float* gate_w,
-                            const float* gate_b, const float* lambda, const void* saved,
-                            const void* dy, void* dq, void* dk, void* dv, float* dgate_w,
-                            float* dgate_b, float* dlambda, void* ws, size_t ws_bytes,
-                            void* stream) {
+elsaa_status elsaa_forward(const elsaa_params* p, const void* q, const void* k, const void* v,
+                           const void* r_sort, const void* r_race, const float* gate_w,
+                           const float* gate_b, const float* lambda, void* y, void* saved,
+                           void* ws, size_t ws_bytes, void* stream) {
+  return elsaa_forward_staged(p, q, k, v, r_sort, r_race, gate_w, gate_b, lambda, y, saved, ws,
+                              ws_bytes, stream, nullptr);
+}
+
+elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const void* k,
+                                   const void* v, const void* r_sort, const void* r_race,
+                                   const float* gate_w, const float* gate_b, const float* lambda,
+                                   const void* saved, const void* dy, void* dq, void* dk, void* dv,
+                                   float* dgate_w, float* dgate_b, float* dlambda, void* ws,
+                                   size_t ws_bytes, void* stream, void* const* events) {
   (void)r_sort;
   (void)r_race;
   Geometry g;
@@ -257,22 +277,55 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* q, const void* k,
   float* d_t = (float*)(w + wl.d_t);
   float* partials = (float*)(w + wl.partials);
   ELSAA_TRY(cudaMemsetAsync(w + wl.err, 0, sizeof(uint32_t), s));
+  ELSAA_TRY(mark(events, 0, s));
 
   // 1. fusion and gate backward: dO_sp, D', dq from the gates, g_r dy / Ctot
   ELSAA_TRY(launch_fuse_bwd(g, q, dy, o_sp, o_race, lse, ctot, gate_w, gate_b, lambda, d_o,
                             dprime, dq_acc, dor, partials, s));
+  ELSAA_TRY(mark(events, 1, s));
   // 2. RACE backward: scatter into the table gradient by query code, gather by key code
   ELSAA_TRY(launch_race_build(g, rcode, dor, true, d_t, nullptr, s));
   ELSAA_TRY(launch_race_gather_sum(g, rcode_k, d_t, dv_acc, s));
-  // 3. sparse branch backward
-  ELSAA_TRY(cudaMemsetAsync(dk_acc, 0, bhn * g.d * 4, s));
-  ELSAA_TRY(launch_attn_bwd_simt(g, q, k, v, perm, perm + bhn, d_o, lse, dprime, dq_acc, dk_acc,
-                                 dv_acc, s));
-  // 4. outputs
-  ELSAA_TRY(launch_cast_out(g, dq_acc, dq, s));
-  ELSAA_TRY(launch_cast_out(g, dk_acc, dk, s));
-  ELSAA_TRY(launch_cast_out(g, dv_acc, dv, s));
+  ELSAA_TRY(mark(events, 2, s));
+  // 3. sparse branch backward, 4. outputs
+  if (g.tc_attn) {
+    ELSAA_TRY(launch_attn_bwd_tc(g, q, k, v, perm, perm + bhn, d_o, lse, dprime, dv_acc, dq_acc,
+                                 dk, dv, (uint32_t*)(w + wl.err), s));
+    ELSAA_TRY(mark(events, 3, s));
+    ELSAA_TRY(launch_cast_out(g, dq_acc, dq, s));
+  } else {
+    ELSAA_TRY(cudaMemsetAsync(dk_acc, 0, bhn * g.d * 4, s));
+    ELSAA_TRY(launch_attn_bwd_simt(g, q, k, v, perm, perm + bhn, d_o, lse, dprime, dq_acc,
+                                   dk_acc, dv_acc, s));
+    ELSAA_TRY(mark(events, 3, s));
+    ELSAA_TRY(launch_cast_out(g, dq_acc, dq, s));
+    ELSAA_TRY(launch_cast_out(g, dk_acc, dk, s));
+    ELSAA_TRY(launch_cast_out(g, dv_acc, dv, s));
+  }
   ELSAA_TRY(launch_param_reduce(g, partials, dgate_w, dgate_b, dlambda, s));
+  ELSAA_TRY(mark(events, 4, s));
+  return ELSAA_OK;
+}
+
+elsaa_status elsaa_backward(const elsaa_params* p, const void* q, const void* k, const void* v,
+                            const void* r_sort, const void* r_race, const float* gate_w,
+                            const float* gate_b, const float* lambda, const void* saved,
+                            const void* dy, void* dq, void* dk, void* dv, float* dgate_w,
+                            float* dgate_b, float* dlambda, void* ws, size_t ws_bytes,
+                            void* stream) {
+  return elsaa_backward_staged(p, q, k, v, r_sort, r_race, gate_w, gate_b, lambda, saved, dy, dq,
+                               dk, dv, dgate_w, dgate_b, dlambda, ws, ws_bytes, stream, nullptr);
+}
+
+elsaa_status elsaa_kernel_launches(const elsaa_params* p, int32_t* fwd, int32_t* bwd) {
+  Geometry g;
+  elsaa_status why;
+  if (!make_geometry(p, &g, &why)) return why;
+  if (!fwd || !bwd) return ELSAA_ERR_INVALID_ARG;
+  // hash 1, sort 3 per pass, RACE build 1, sparse 1, RACE gather + fusion 1
+  *fwd = 1 + 3 * g.sort_passes + 1 + 1 + 1;
+  // fusion backward 1, RACE build 1 + gather 1, sparse 1 (+ casts), reduction 1
+  *bwd = 1 + 2 + (g.tc_attn ? 1 + 1 : 1 + 3) + 1;
   return ELSAA_OK;
 }
 

@@ -1,0 +1,303 @@
+// Backward of the exact sparse branch on tcgen05 tensor cores (bf16, d in {64, 128}).
+//
+// The sparse branch ("Two Efficient Attentions, One Denominator Problem",
+// section "Two efficient branches can still be mis-scaled") is softmax
+// attention over each query's Sort-LSH window; its row mass also feeds the
+// fusion multiplier, so its log-mass lse carries a gradient of its own.  With
+// P = exp(scale s - lse), dP = dO V^T and D' = rowsum(dO * O) - dlse:
+//   dS = P (dP - D'),  dV = P^T dO,  dK = scale dS^T Q,  dQ = scale dS K.
+//
+// Key-major CTAs: one CTA owns 128 consecutive sorted keys (the MMA's M) and
+// walks, in blocks of up to 128, the sorted queries whose window holds them
+// (query chunk j sees key chunks j-1 and j, so key chunk i is seen by query
+// chunks i and i+1):
+//   S^T  = K Q_b^T,  dP^T = V dO_b^T          tcgen05 (SS) -> TMEM
+//   P^T, dS^T (bf16)                           thread t = key row t -> shared memory
+//   dV += P^T dO_b,  dK += dS^T Q_b            tcgen05, accumulated in TMEM
+//   dQ_b = dS K                                tcgen05 with dS^T read as an
+//                                              MN-major operand; added to the
+//                                              fp32 dq accumulator with atomics
+// dK and dV (plus the RACE branch's dv) are written once, in bf16, at the
+// keys' token indices.  Every wait is bounded.
+#include <math.h>
+
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace elsaa {
+namespace {
+
+using namespace tc;
+
+constexpr int kTile = 128;
+constexpr int kThreads = 128;
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct BwdLayout {
+  static constexpr int kSub = D / 64;
+  static constexpr uint32_t kSubBytes = 128 * 128;
+  static constexpr uint32_t kK = 0;
+  static constexpr uint32_t kV = kK + kSub * kSubBytes;
+  static constexpr uint32_t kQ = kV + kSub * kSubBytes;
+  static constexpr uint32_t kDO = kQ + kSub * kSubBytes;
+  static constexpr uint32_t kPT = kDO + kSub * kSubBytes;    // 128 keys x 128 queries bf16
+  static constexpr uint32_t kDST = kPT + 2 * kSubBytes;
+  static constexpr uint32_t kLse = kDST + 2 * kSubBytes;     // 128 floats
+  static constexpr uint32_t kDpr = kLse + 128 * 4;           // 128 floats
+  static constexpr uint32_t kBar = kDpr + 128 * 4;
+  static constexpr uint32_t kDyn = kBar + 64;
+  // TMEM columns
+  static constexpr uint32_t kTS = 0, kTdP = 128, kTdV = 256, kTdK = 256 + D, kTdQ = 0;
+};
+
+template <int D>
+ELSAA_DEV void gather_rows(uint32_t dst, const __nv_bfloat16* src_base, const int32_t* perm,
+                           int rows) {
+  constexpr int kChunks = D / 8;
+  for (int i = threadIdx.x; i < rows * kChunks; i += kThreads) {
+    const int row = i / kChunks, ch = i % kChunks;
+    const __nv_bfloat16* src = src_base + (size_t)perm[row] * D + ch * 8;
+    cp_async16(dst + (ch >> 3) * (128 * 128) + sw128_off(row, ch & 7), src, 16);
+  }
+}
+
+ELSAA_DEV uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                   const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ perm_q,
+                   const int32_t* __restrict__ perm_k, const __nv_bfloat16* __restrict__ d_o,
+                   const float* __restrict__ lse, const float* __restrict__ dprime,
+                   const float* __restrict__ dv_race, int N, int chunk, float scale,
+                   float scale_log2, float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk,
+                   __nv_bfloat16* __restrict__ dv, uint32_t* __restrict__ err) {
+  using Lay = BwdLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bar_a = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
+  uint64_t* bar_b = bar_a + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_a + 2);
+  float* s_lse = reinterpret_cast<float*>(smem + Lay::kLse);
+  float* s_dpr = reinterpret_cast<float*>(smem + Lay::kDpr);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  if ((sbase & 1023u) != 0) {
+    if (tid == 0) raise_error(err, ERR_CHECK);
+    return;
+  }
+  const int bh = blockIdx.y;
+  const int k0 = blockIdx.x * kTile;
+  const size_t unit = (size_t)bh * N;
+  const int32_t* pq = perm_q + unit;
+  const int32_t* pk = perm_k + unit;
+  // queries whose window holds a key of this tile: chunks chunk(k0) .. chunk(k0+127)+1
+  const int qbase = (k0 / chunk) * chunk;
+  const int qend = min(N, ((k0 + kTile - 1) / chunk + 2) * chunk);
+  const int nqb = (qend - qbase + kTile - 1) / kTile;
+  const int key_chunk = (k0 + tid) / chunk;
+
+  if (tid == 0) {
+    mbar_init(bar_a, 1);
+    mbar_init(bar_b, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  gather_rows<D>(sbase + Lay::kK, k + unit * D, pk + k0, kTile);
+  gather_rows<D>(sbase + Lay::kV, v + unit * D, pk + k0, kTile);
+  cp_async_commit();
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  bool ok = true;
+
+  for (int b = 0; b < nqb; ++b) {
+    const int qb0 = qbase + b * kTile;
+    const int nq = min(kTile, qend - qb0);
+    gather_rows<D>(sbase + Lay::kQ, q + unit * D, pq + qb0, nq);
+    gather_rows<D>(sbase + Lay::kDO, d_o + unit * D, pq + qb0, nq);
+    cp_async_commit();
+    if (tid < nq) {
+      const int i = pq[qb0 + tid];
+      s_lse[tid] = lse[unit + i] * 1.4426950408889634f;
+      s_dpr[tid] = dprime[unit + i];
+    }
+    cp_async_wait_all();
+    fence_async_smem();
+    fence_before();
+    __syncthreads();
+    // S^T = K Q_b^T and dP^T = V dO_b^T
+    if (tid == 0) {
+      fence_after();
+      const uint32_t idesc = idesc_bf16(128, nq, false, false);
+#pragma unroll
+      for (int s = 0; s < D / 16; ++s) {
+        const uint32_t off = (s >> 2) * Lay::kSubBytes + (s & 3) * 32;
+        mma_bf16_ss(tmem + Lay::kTS, sw128_desc(sbase + Lay::kK + off, 16, 1024),
+                    sw128_desc(sbase + Lay::kQ + off, 16, 1024), idesc, s > 0);
+      }
+#pragma unroll
+      for (int s = 0; s < D / 16; ++s) {
+        const uint32_t off = (s >> 2) * Lay::kSubBytes + (s & 3) * 32;
+        mma_bf16_ss(tmem + Lay::kTdP, sw128_desc(sbase + Lay::kV + off, 16, 1024),
+                    sw128_desc(sbase + Lay::kDO + off, 16, 1024), idesc, s > 0);
+      }
+      mma_commit(bar_a);
+    }
+    ok = mbar_wait(bar_a, b & 1, err);
+    if (__syncthreads_or(!ok)) break;
+    fence_after();
+    // P^T and dS^T rows of this thread's key; a query in chunk jq sees this key
+    // iff jq - key_chunk is 0 or 1
+    for (int c0 = 0; c0 < nq; c0 += 32) {
+      float sv[32], dp[32];
+      tmem_ld32(tmem + Lay::kTS + lane_off + c0, sv);
+      tmem_ld32(tmem + Lay::kTdP + lane_off + c0, dp);
+      tmem_ld_wait();
+      uint32_t pp[16], dd[16];
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        float p[2], ds[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int col = c0 + i + e;
+          const int dj = (qb0 + col) / chunk - key_chunk;
+          p[e] = 0.f;
+          ds[e] = 0.f;
+          if (col < nq && (dj == 0 || dj == 1)) {
+            p[e] = exp2f(sv[i + e] * scale_log2 - s_lse[col]);
+            ds[e] = scale * p[e] * (dp[i + e] - s_dpr[col]);
+          }
+        }
+        pp[i >> 1] = pack_bf16(p[0], p[1]);
+        dd[i >> 1] = pack_bf16(ds[0], ds[1]);
+      }
+#pragma unroll
+      for (int q8 = 0; q8 < 4; ++q8) {
+        const int col = c0 + q8 * 8;
+        if (col < nq) {
+          const uint32_t off = (col >> 6) * Lay::kSubBytes + sw128_off(tid, (col & 63) >> 3);
+          *reinterpret_cast<uint4*>(smem + Lay::kPT + off) =
+              make_uint4(pp[q8 * 4], pp[q8 * 4 + 1], pp[q8 * 4 + 2], pp[q8 * 4 + 3]);
+          *reinterpret_cast<uint4*>(smem + Lay::kDST + off) =
+              make_uint4(dd[q8 * 4], dd[q8 * 4 + 1], dd[q8 * 4 + 2], dd[q8 * 4 + 3]);
+        }
+      }
+    }
+    fence_async_smem();
+    fence_before();
+    __syncthreads();
+    // dV += P^T dO_b, dK += dS^T Q_b, dQ_b = dS K
+    if (tid == 0) {
+      fence_after();
+      const uint32_t id_kv = idesc_bf16(128, D, false, true);
+      for (int s = 0; s < nq / 16; ++s) {
+        const uint32_t aoff = (s >> 2) * Lay::kSubBytes + (s & 3) * 32;
+        const uint32_t acc = (b > 0 || s > 0) ? 1u : 0u;
+        mma_bf16_ss(tmem + Lay::kTdV, sw128_desc(sbase + Lay::kPT + aoff, 16, 1024),
+                    sw128_desc(sbase + Lay::kDO + s * 2048, Lay::kSubBytes, 1024), id_kv, acc);
+        mma_bf16_ss(tmem + Lay::kTdK, sw128_desc(sbase + Lay::kDST + aoff, 16, 1024),
+                    sw128_desc(sbase + Lay::kQ + s * 2048, Lay::kSubBytes, 1024), id_kv, acc);
+      }
+      const uint32_t id_q = idesc_bf16(128, D, true, true);
+#pragma unroll
+      for (int s = 0; s < kTile / 16; ++s) {
+        mma_bf16_ss(tmem + Lay::kTdQ,
+                    sw128_desc(sbase + Lay::kDST + s * 2048, Lay::kSubBytes, 1024),
+                    sw128_desc(sbase + Lay::kK + s * 2048, Lay::kSubBytes, 1024), id_q, s > 0);
+      }
+      mma_commit(bar_b);
+    }
+    ok = mbar_wait(bar_b, b & 1, err);
+    if (__syncthreads_or(!ok)) break;
+    fence_after();
+    // dQ rows of this block: TMEM lane t = query qb0 + t
+    {
+      const bool mine = tid < nq;
+      float* dst = dq_acc + (unit + (mine ? pq[qb0 + tid] : 0)) * D;
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        float g[32];
+        tmem_ld32(tmem + Lay::kTdQ + lane_off + c0, g);
+        tmem_ld_wait();
+        if (mine) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) atomicAdd(dst + c0 + i, g[i]);
+        }
+      }
+    }
+    fence_before();
+    __syncthreads();
+  }
+  if (ok) {
+    fence_after();
+    const int i = pk[k0 + tid];
+    const float* dvr = dv_race + (unit + i) * D;
+    __nv_bfloat16* dvo = dv + (unit + i) * D;
+    __nv_bfloat16* dko = dk + (unit + i) * D;
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      float gv[32], gk[32];
+      tmem_ld32(tmem + Lay::kTdV + lane_off + c0, gv);
+      tmem_ld32(tmem + Lay::kTdK + lane_off + c0, gk);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q8 = 0; q8 < 4; ++q8) {
+        uint32_t wv[4], wk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = q8 * 8 + 2 * e;
+          wv[e] = pack_bf16(gv[c] + dvr[c0 + c], gv[c + 1] + dvr[c0 + c + 1]);
+          wk[e] = pack_bf16(gk[c], gk[c + 1]);
+        }
+        *reinterpret_cast<uint4*>(dvo + c0 + q8 * 8) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        *reinterpret_cast<uint4*>(dko + c0 + q8 * 8) = make_uint4(wk[0], wk[1], wk[2], wk[3]);
+      }
+    }
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D>
+cudaError_t bwd(const Geometry& g, const void* q, const void* k, const void* v,
+                const int32_t* perm_q, const int32_t* perm_k, const void* d_o, const float* lse,
+                const float* dprime, const float* dv_race, float* dq_acc, void* dk, void* dv,
+                uint32_t* err, cudaStream_t s) {
+  using Lay = BwdLayout<D>;
+  cudaError_t e = cudaFuncSetAttribute(attn_bwd_tc_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kDyn);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(g.N / kTile, g.BH);
+  attn_bwd_tc_kernel<D><<<grid, kThreads, Lay::kDyn, s>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+      static_cast<const __nv_bfloat16*>(v), perm_q, perm_k,
+      static_cast<const __nv_bfloat16*>(d_o), lse, dprime, dv_race, g.N, g.chunk, g.scale,
+      g.scale * 1.4426950408889634f, dq_acc, static_cast<__nv_bfloat16*>(dk),
+      static_cast<__nv_bfloat16*>(dv), err);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd_tc(const Geometry& g, const void* q, const void* k, const void* v,
+                               const int32_t* perm_q, const int32_t* perm_k, const void* d_o,
+                               const float* lse, const float* dprime, const float* dv_race,
+                               float* dq_acc, void* dk, void* dv, uint32_t* err, cudaStream_t s) {
+  return g.d == 64 ? bwd<64>(g, q, k, v, perm_q, perm_k, d_o, lse, dprime, dv_race, dq_acc, dk,
+                             dv, err, s)
+                   : bwd<128>(g, q, k, v, perm_q, perm_k, d_o, lse, dprime, dv_race, dq_acc, dk,
+                              dv, err, s);
+}
+
+}  // namespace elsaa

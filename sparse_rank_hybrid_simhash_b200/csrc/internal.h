@@ -102,6 +102,11 @@ cudaError_t launch_attn_fwd_tc(const Geometry& g, const void* q, const void* k, 
                                const int32_t* perm_q, const int32_t* perm_k, void* o_sp,
                                float* lse, uint32_t* err, cudaStream_t s);
 bool attn_tc_supported(const Geometry& g);
+// tcgen05 backward: dq_acc += dQ (fp32 atomics); dk, dv written (dv adds dv_race).
+cudaError_t launch_attn_bwd_tc(const Geometry& g, const void* q, const void* k, const void* v,
+                               const int32_t* perm_q, const int32_t* perm_k, const void* d_o,
+                               const float* lse, const float* dprime, const float* dv_race,
+                               float* dq_acc, void* dk, void* dv, uint32_t* err, cudaStream_t s);
 
 // Backward of the fusion and gates (per query), then the parameter reduction
 // and the final casts.
