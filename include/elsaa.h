@@ -162,6 +162,29 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
  * enqueue for `p` (memsets excluded). */
 elsaa_status elsaa_kernel_launches(const elsaa_params* p, int32_t* fwd, int32_t* bwd);
 
+/* Sort-LSH order of given sort codes, using no memory the caller or the
+ * library allocates.  The paper has no counterpart: this exists for callers
+ * that cannot provide scratch memory, such as a serving process whose pool
+ * already holds all device memory, or a framework that forbids cudaMalloc and
+ * cudaFree (which synchronise the device) during a step.
+ * code: device [2][B,H,N] uint16, the sort codes of the queries followed by
+ * those of the keys (elsaa_views.code_q is the start of both); perm: device
+ * [2][B,H,N] int32 output, the token index at each sorted rank, equal to the
+ * permutations elsaa_forward saves.  Both 16-byte aligned.  Only p->B, H, N
+ * and sort_bits matter, but p must validate.
+ * The radix sort's scratch sits in one fixed device array of
+ * ELSAA_NOALLOC_SCRATCH_BYTES that every device loading the library keeps
+ * until exit.  The first call on a device looks up that array's device
+ * address (with the device current), so make it before any stream capture.
+ * Returns ELSAA_ERR_WORKSPACE if the problem needs more scratch than that
+ * (2 B H 2^digit_bits ceil(N/2048) ints, plus 2 B H N ints when sort_bits > 8).
+ * All calls share the array: calls that may overlap on the GPU (other
+ * streams, other host threads on the same device) race and must be ordered
+ * by the caller.  No part of the array needs to start cleared. */
+#define ELSAA_NOALLOC_SCRATCH_BYTES (4u << 20)
+elsaa_status elsaa_sort_codes_noalloc(const elsaa_params* p, const uint16_t* code, int32_t* perm,
+                                      void* stream);
+
 /* Fills `out` with device pointers into `saved` (no device access). */
 elsaa_status elsaa_saved_views(const elsaa_params* p, const void* saved, elsaa_views* out);
 

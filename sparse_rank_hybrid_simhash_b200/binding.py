@@ -68,7 +68,7 @@ class Views(ctypes.Structure):
 EXPORTS = ("elsaa_validate", "elsaa_workspace_bytes", "elsaa_saved_bytes", "elsaa_forward",
            "elsaa_backward", "elsaa_forward_staged", "elsaa_backward_staged",
            "elsaa_kernel_launches", "elsaa_saved_views", "elsaa_check", "elsaa_status_str",
-           "elsaa_uses_tensor_cores")
+           "elsaa_uses_tensor_cores", "elsaa_sort_codes_noalloc")
 FWD_STAGES = ("hash", "sort", "race_build", "sparse_fwd", "race_fuse")
 BWD_STAGES = ("fuse_bwd", "race_bwd", "sparse_bwd", "finish")
 
@@ -101,6 +101,8 @@ def lib() -> ctypes.CDLL:
     L.elsaa_kernel_launches.argtypes = [P, ctypes.POINTER(ctypes.c_int32),
                                         ctypes.POINTER(ctypes.c_int32)]
     L.elsaa_kernel_launches.restype = st
+    L.elsaa_sort_codes_noalloc.argtypes = [P, vp, vp, vp]
+    L.elsaa_sort_codes_noalloc.restype = st
     L.elsaa_saved_views.argtypes = [P, vp, ctypes.POINTER(Views)]
     L.elsaa_saved_views.restype = st
     L.elsaa_check.argtypes, L.elsaa_check.restype = [vp, vp], st
@@ -207,6 +209,15 @@ def backward(p: Params, q, k, v, r_sort, r_race, gate_w, gate_b, lam, saved, dy,
                                        ws.numel(), _stream(stream), _events(events))
     _ok("elsaa_backward", code)
     return dq, dk, dv, dgate_w, dgate_b, dlam
+
+
+def sort_codes_noalloc(p: Params, code: torch.Tensor, perm: torch.Tensor, stream=None) -> None:
+    """Sort-LSH permutations of ``code`` ([2, B, H, N] int16 view of the uint16
+    sort codes, queries then keys) into ``perm`` ([2, B, H, N] int32) with no
+    scratch from the caller: for callers that cannot allocate device memory
+    while they run (see elsaa_sort_codes_noalloc in include/elsaa.h)."""
+    _ok("elsaa_sort_codes_noalloc", lib().elsaa_sort_codes_noalloc(
+        ctypes.byref(p), _ptr(code), _ptr(perm), _stream(stream)))
 
 
 def check(ws: torch.Tensor, stream=None) -> None:

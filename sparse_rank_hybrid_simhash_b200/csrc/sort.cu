@@ -12,6 +12,8 @@
 //      digits, take per-warp bases, then rank equal digits within each
 //      32-key round with __match_any_sync.
 // Codes of up to 16 bits take two passes (the second reads the first's order).
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -150,3 +152,71 @@ cudaError_t launch_sort(const Geometry& g, const uint16_t* code, int32_t* perm, 
 }
 
 }  // namespace elsaa
+
+// ---------------------------------------------------------------------------
+// Sort-LSH order without any device allocation (elsaa_sort_codes_noalloc).
+//
+// Some callers cannot hand the library scratch memory: a serving process whose
+// memory pool has already reserved all device memory at start-up, or a host
+// framework whose allocator contract forbids cudaMalloc/cudaFree inside a step
+// (both synchronise the device).  For them the radix sort's scratch (per-tile
+// digit histograms and, for codes of more than 8 bits, the order after the
+// first pass) lives in one fixed array in device memory that the library
+// itself owns.  Every device that loads the library keeps these bytes until
+// the process exits.
+// ---------------------------------------------------------------------------
+
+namespace elsaa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+constexpr int kMaxDevices = 64;
+
+__device__ __align__(256) unsigned char g_sort_scratch[kNoAllocScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_sort_scratch on the current device, looked up once per
+// device (the host-side symbol is only a stand-in and must never reach a kernel).
+cudaError_t scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_sort_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace elsaa
+
+extern "C" elsaa_status elsaa_sort_codes_noalloc(const elsaa_params* p, const uint16_t* code,
+                                                 int32_t* perm, void* stream) {
+  using namespace elsaa;
+  Geometry g;
+  elsaa_status why;
+  if (!make_geometry(p, &g, &why)) return why;
+  if (!code || !perm) return ELSAA_ERR_INVALID_ARG;
+  if (((uintptr_t)code % 16) != 0 || ((uintptr_t)perm % 16) != 0) return ELSAA_ERR_INVALID_ARG;
+  const size_t hist = align_up((size_t)2 * g.BH * g.sort_bins * g.sort_tiles * 4);
+  const size_t tmp = g.sort_passes > 1 ? (size_t)2 * g.BH * g.N * 4 : 0;
+  if (hist + tmp > kNoAllocScratchBytes) return ELSAA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (scratch_address(&scratch) != cudaSuccess) return ELSAA_ERR_CUDA;
+  char* base = static_cast<char*>(scratch);
+  // every histogram slot and the intermediate order are fully written before
+  // they are read, so nothing left from an earlier call needs clearing
+  if (launch_sort(g, code, perm, reinterpret_cast<int32_t*>(base),
+                  reinterpret_cast<int32_t*>(base + hist), (cudaStream_t)stream) != cudaSuccess)
+    return ELSAA_ERR_CUDA;
+  return ELSAA_OK;
+}
+
