@@ -126,7 +126,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -357,7 +357,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override B (small cases for ncu captures; not a bench line)")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override H (small cases for ncu captures; not a bench line)")
     args = ap.parse_args()
+    if args.batch or args.heads:
+        w0 = WORKLOADS[args.workload]
+        WORKLOADS[args.workload] = w0.replace(B=args.batch or w0.B, H=args.heads or w0.H)
     if args.impl == "reference":
         run_reference(args)
         return
