@@ -75,6 +75,7 @@ WorkLayout work_layout(const Geometry& g) {
   w.err = take(256);
   w.sort_hist = take((size_t)2 * g.BH * g.sort_bins * g.sort_tiles * 4);
   w.sort_tmp = take(2 * bhn * 4);
+  w.absmax = take((size_t)2 * g.BH * 4);
   const size_t shared_base = off;
   // forward without a saved buffer: the saved layout lives here
   w.saved = take(saved_layout(g).total);
@@ -212,7 +213,9 @@ elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const vo
                         s));
   ELSAA_TRY(mark(events, 2, s));
   // 3. RACE tables from the keys
-  ELSAA_TRY(launch_race_build(g, rcode_k, v, false, sums, counts, s));
+  float* absmax = (float*)(w + wl.absmax);
+  ELSAA_TRY(launch_unit_absmax(g, v, false, absmax, s));
+  ELSAA_TRY(launch_race_build(g, rcode_k, v, false, absmax, sums, counts, err, s));
   ELSAA_TRY(mark(events, 3, s));
   // 4. exact sparse branch
   if (g.tc_attn)
@@ -280,11 +283,13 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
   ELSAA_TRY(mark(events, 0, s));
 
   // 1. fusion and gate backward: dO_sp, D', dq from the gates, g_r dy / Ctot
+  float* absmax = (float*)(w + wl.absmax) + g.BH;
   ELSAA_TRY(launch_fuse_bwd(g, q, dy, o_sp, o_race, lse, ctot, gate_w, gate_b, lambda, d_o,
-                            dprime, dq_acc, dor, partials, s));
+                            dprime, dq_acc, dor, absmax, partials, s));
   ELSAA_TRY(mark(events, 1, s));
   // 2. RACE backward: scatter into the table gradient by query code, gather by key code
-  ELSAA_TRY(launch_race_build(g, rcode, dor, true, d_t, nullptr, s));
+  ELSAA_TRY(launch_race_build(g, rcode, dor, true, absmax, d_t, nullptr,
+                              (uint32_t*)(w + wl.err), s));
   ELSAA_TRY(launch_race_gather_sum(g, rcode_k, d_t, dv_acc, s));
   ELSAA_TRY(mark(events, 2, s));
   // 3. sparse branch backward, 4. outputs
@@ -322,8 +327,8 @@ elsaa_status elsaa_kernel_launches(const elsaa_params* p, int32_t* fwd, int32_t*
   elsaa_status why;
   if (!make_geometry(p, &g, &why)) return why;
   if (!fwd || !bwd) return ELSAA_ERR_INVALID_ARG;
-  // hash 1, sort 3 per pass, RACE build 1, sparse 1, RACE gather + fusion 1
-  *fwd = 1 + 3 * g.sort_passes + 1 + 1 + 1;
+  // hash 1, sort 3 per pass, |V| max 1 + RACE build 1, sparse 1, RACE gather + fusion 1
+  *fwd = 1 + 3 * g.sort_passes + 2 + 1 + 1;
   // fusion backward 1, RACE build 1 + gather 1, sparse 1 (+ casts), reduction 1
   *bwd = 1 + 2 + (g.tc_attn ? 1 + 1 : 1 + 3) + 1;
   return ELSAA_OK;

@@ -24,61 +24,104 @@
 namespace elsaa {
 namespace {
 
-template <typename T, int VEC>
+template <typename T>
+ELSAA_DEV void ld4(const T* p, float* v);
+template <>
+ELSAA_DEV void ld4<float>(const float* p, float* v) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+}
+template <>
+ELSAA_DEV void ld4<__nv_bfloat16>(const __nv_bfloat16* p, float* v) {
+  const uint2 raw = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
+// Rounds 4 values to T, stores them, and returns the rounded values in v.
+template <typename T>
+ELSAA_DEV void st4_round(T* p, float* v);
+template <>
+ELSAA_DEV void st4_round<float>(float* p, float* v) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+template <>
+ELSAA_DEV void st4_round<__nv_bfloat16>(__nv_bfloat16* p, float* v) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+  const __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+  uint2 raw;
+  raw.x = *reinterpret_cast<const uint32_t*>(&a);
+  raw.y = *reinterpret_cast<const uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = raw;
+  const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+  v[0] = fa.x; v[1] = fa.y; v[2] = fb.x; v[3] = fb.y;
+}
+
+template <int QL>
+ELSAA_DEV float gsum(float v) {
+#pragma unroll
+  for (int o = QL / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// QL = d / 4 lanes per query (4 consecutive values each, 16-byte accesses),
+// 32 / QL queries per warp.
+template <typename T, int QL>
 __global__ void __launch_bounds__(256)
 fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __restrict__ o_sp,
                 const T* __restrict__ o_race, const float* __restrict__ lse,
                 const int32_t* __restrict__ ctot, const float* __restrict__ gate_w,
                 const float* __restrict__ gate_b, int gate_fixed, float gs_fixed, float gr_fixed,
-                const float* __restrict__ lam, int64_t rows, int L, int d, T* __restrict__ d_o,
-                float* __restrict__ dprime, float* __restrict__ dq_acc, float* __restrict__ dor,
-                float* __restrict__ partials) {
+                const float* __restrict__ lam, int64_t rows, int N, int L, int d,
+                T* __restrict__ d_o, float* __restrict__ dprime, float* __restrict__ dq_acc,
+                float* __restrict__ dor, float* __restrict__ absmax, float* __restrict__ partials) {
+  constexpr int QW = 32 / QL;
   __shared__ float red[8][2 * 128 + 3];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int ql = lane % QL, sub = lane / QL;
   const float lam_v = *lam;
-  float pws[VEC], pwr[VEC], pbs = 0.f, pbr = 0.f, plam = 0.f;
-#pragma unroll
-  for (int i = 0; i < VEC; ++i) pws[i] = pwr[i] = 0.f;
-  float ws_[VEC], wr_[VEC];
-#pragma unroll
-  for (int i = 0; i < VEC; ++i) ws_[i] = wr_[i] = 0.f;
+  float pws[4] = {0.f, 0.f, 0.f, 0.f}, pwr[4] = {0.f, 0.f, 0.f, 0.f};
+  float pbs = 0.f, pbr = 0.f, plam = 0.f;
+  float ws4[4] = {0.f, 0.f, 0.f, 0.f}, wr4[4] = {0.f, 0.f, 0.f, 0.f};
   float bs = 0.f, br = 0.f;
   if (!gate_fixed) {
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) {
-      ws_[i] = gate_w[lane * VEC + i];
-      wr_[i] = gate_w[d + lane * VEC + i];
-    }
+    ld4<float>(gate_w + ql * 4, ws4);
+    ld4<float>(gate_w + d + ql * 4, wr4);
     bs = gate_b[0];
     br = gate_b[1];
   }
-  for (int64_t r = (int64_t)blockIdx.x * nw + w; r < rows; r += (int64_t)gridDim.x * nw) {
-    const size_t base = (size_t)r * d + lane * VEC;
-    float qv[VEC], g[VEC], os[VEC], orc[VEC];
+  int64_t cur_bh = -1;   // unit whose largest |g_r dy / Ctot| this lane holds (lanes ql == 0)
+  float cur_max = 0.f;
+  const int64_t first = ((int64_t)blockIdx.x * nw + w) * QW;
+  const int64_t stride = (int64_t)gridDim.x * nw * QW;
+  for (int64_t r0 = first; r0 < rows; r0 += stride) {
+    const int64_t r = r0 + sub;
+    const bool valid = r < rows;
+    const int64_t rr = valid ? r : rows - 1;
+    const size_t base = (size_t)rr * d + ql * 4;
+    float qv[4], g[4], os[4], orc[4];
+    ld4<T>(q + base, qv);
+    ld4<T>(dy + base, g);
+    ld4<T>(o_sp + base, os);
+    ld4<T>(o_race + base, orc);
     float dyo = 0.f, dyr = 0.f, as = 0.f, ar = 0.f;
 #pragma unroll
-    for (int i = 0; i < VEC; ++i) {
-      qv[i] = to_f32(q[base + i]);
-      g[i] = to_f32(dy[base + i]);
-      os[i] = to_f32(o_sp[base + i]);
-      orc[i] = to_f32(o_race[base + i]);
+    for (int i = 0; i < 4; ++i) {
       dyo += g[i] * os[i];
       dyr += g[i] * orc[i];
-      if (!gate_fixed) {
-        as += qv[i] * ws_[i];
-        ar += qv[i] * wr_[i];
-      }
+      as += qv[i] * ws4[i];
+      ar += qv[i] * wr4[i];
     }
-    dyo = warp_sum(dyo);
-    dyr = warp_sum(dyr);
+    dyo = gsum<QL>(dyo);
+    dyr = gsum<QL>(dyr);
     float gs = gs_fixed, gr = gr_fixed;
     if (!gate_fixed) {
-      gs = 1.0f / (1.0f + expf(-(warp_sum(as) + bs)));
-      gr = 1.0f / (1.0f + expf(-(warp_sum(ar) + br)));
+      gs = 1.0f / (1.0f + expf(-(gsum<QL>(as) + bs)));
+      gr = 1.0f / (1.0f + expf(-(gsum<QL>(ar) + br)));
     }
-    const int c = ctot[r];
+    const int c = ctot[rr];
     const float zr = (float)c / (float)L;
-    const float l = lse[r];
+    const float l = lse[rr];
     const float lz = lam_v * zr;
     const float m = lz > 0.f ? 1.0f / (1.0f + expf(logf(lz) - l)) : 1.0f;
     const float dm = gs * dyo;
@@ -90,38 +133,72 @@ fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __re
       da_r = dyr * gr * (1.0f - gr);
     }
     const float inv_c = c > 0 ? 1.0f / (float)c : 0.f;
-    float dd = 0.f;
+    float dov[4], dqv[4], drv[4];
+    float vmax = 0.f;
 #pragma unroll
-    for (int i = 0; i < VEC; ++i) {
-      const T dov = from_f32<T>(gs * m * g[i]);
-      d_o[base + i] = dov;
-      dd += to_f32(dov) * os[i];
-      dq_acc[base + i] = gate_fixed ? 0.f : da_s * ws_[i] + da_r * wr_[i];
-      dor[base + i] = gr * g[i] * inv_c;
-      if (!gate_fixed) {
+    for (int i = 0; i < 4; ++i) {
+      dov[i] = gs * m * g[i];
+      dqv[i] = da_s * ws4[i] + da_r * wr4[i];
+      drv[i] = gr * g[i] * inv_c;
+      vmax = fmaxf(vmax, fabsf(drv[i]));
+    }
+    vmax = fmaxf(vmax, 0.f);
+#pragma unroll
+    for (int o = QL / 2; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    float dd = 0.f;
+    if (valid) {
+      st4_round<T>(d_o + base, dov);   // dov now holds the stored (rounded) values
+      *reinterpret_cast<float4*>(dq_acc + base) = make_float4(dqv[0], dqv[1], dqv[2], dqv[3]);
+      *reinterpret_cast<float4*>(dor + base) = make_float4(drv[0], drv[1], drv[2], drv[3]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        dd += dov[i] * os[i];
         pws[i] += da_s * qv[i];
         pwr[i] += da_r * qv[i];
       }
     }
-    dd = warp_sum(dd);
-    if (lane == 0) {
-      dprime[r] = dd - dlse;
+    dd = gsum<QL>(dd);
+    if (valid && ql == 0) {
+      dprime[rr] = dd - dlse;
       pbs += da_s;
       pbr += da_r;
       plam += dlam;
+      const int64_t bh = rr / N;
+      if (bh != cur_bh) {
+        if (cur_bh >= 0) atomicMax(reinterpret_cast<int*>(absmax) + cur_bh, __float_as_int(cur_max));
+        cur_bh = bh;
+        cur_max = 0.f;
+      }
+      cur_max = fmaxf(cur_max, vmax);
     }
   }
-  // block reduction of the partial parameter gradients
-  const int P = 2 * d + 3;
+  if (ql == 0 && cur_bh >= 0)
+    atomicMax(reinterpret_cast<int*>(absmax) + cur_bh, __float_as_int(cur_max));
+  // block reduction of the partial parameter gradients: first across the row
+  // groups of a warp, then across warps
 #pragma unroll
-  for (int i = 0; i < VEC; ++i) {
-    red[w][lane * VEC + i] = pws[i];
-    red[w][d + lane * VEC + i] = pwr[i];
+  for (int o = QL; o < 32; o <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      pws[i] += __shfl_xor_sync(0xffffffffu, pws[i], o);
+      pwr[i] += __shfl_xor_sync(0xffffffffu, pwr[i], o);
+    }
+    pbs += __shfl_xor_sync(0xffffffffu, pbs, o);
+    pbr += __shfl_xor_sync(0xffffffffu, pbr, o);
+    plam += __shfl_xor_sync(0xffffffffu, plam, o);
   }
-  if (lane == 0) {
-    red[w][2 * d] = pbs;
-    red[w][2 * d + 1] = pbr;
-    red[w][2 * d + 2] = plam;
+  const int P = 2 * d + 3;
+  if (sub == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      red[w][ql * 4 + i] = pws[i];
+      red[w][d + ql * 4 + i] = pwr[i];
+    }
+    if (ql == 0) {
+      red[w][2 * d] = pbs;
+      red[w][2 * d + 1] = pbr;
+      red[w][2 * d + 2] = plam;
+    }
   }
   __syncthreads();
   for (int e = threadIdx.x; e < P; e += blockDim.x) {
@@ -159,17 +236,21 @@ template <typename T>
 cudaError_t fuse_bwd(const Geometry& g, const void* q, const void* dy, const void* o_sp,
                      const void* o_race, const float* lse, const int32_t* ctot,
                      const float* gate_w, const float* gate_b, const float* lam, void* d_o,
-                     float* dprime, float* dq_acc, float* dor, float* partials, cudaStream_t s) {
+                     float* dprime, float* dq_acc, float* dor, float* absmax, float* partials,
+                     cudaStream_t s) {
   const int64_t rows = (int64_t)g.BH * g.N;
+  cudaError_t e = cudaMemsetAsync(absmax, 0, (size_t)g.BH * sizeof(float), s);
+  if (e != cudaSuccess) return e;
 #define ELSAA_FB(VEC)                                                                          \
   fuse_bwd_kernel<T, VEC><<<kParamBlocks, 256, 0, s>>>(                                        \
       static_cast<const T*>(q), static_cast<const T*>(dy), static_cast<const T*>(o_sp),        \
       static_cast<const T*>(o_race), lse, ctot, gate_w, gate_b, g.gate_fixed, g.gate_s,        \
-      g.gate_r, lam, rows, g.L, g.d, static_cast<T*>(d_o), dprime, dq_acc, dor, partials)
-  switch (g.d / 32) {
-    case 1: ELSAA_FB(1); break;
-    case 2: ELSAA_FB(2); break;
-    default: ELSAA_FB(4); break;
+      g.gate_r, lam, rows, g.N, g.L, g.d, static_cast<T*>(d_o), dprime, dq_acc, dor, absmax,  \
+      partials)
+  switch (g.d) {
+    case 32: ELSAA_FB(8); break;
+    case 64: ELSAA_FB(16); break;
+    default: ELSAA_FB(32); break;
   }
 #undef ELSAA_FB
   return cudaGetLastError();
@@ -181,11 +262,11 @@ cudaError_t launch_fuse_bwd(const Geometry& g, const void* q, const void* dy, co
                             const void* o_race, const float* lse, const int32_t* ctot,
                             const float* gate_w, const float* gate_b, const float* lam,
                             void* d_o, float* dprime, float* dq_acc, float* dor,
-                            float* partials, cudaStream_t s) {
+                            float* absmax, float* partials, cudaStream_t s) {
   return g.bf16 ? fuse_bwd<__nv_bfloat16>(g, q, dy, o_sp, o_race, lse, ctot, gate_w, gate_b, lam,
-                                          d_o, dprime, dq_acc, dor, partials, s)
+                                          d_o, dprime, dq_acc, dor, absmax, partials, s)
                 : fuse_bwd<float>(g, q, dy, o_sp, o_race, lse, ctot, gate_w, gate_b, lam, d_o,
-                                  dprime, dq_acc, dor, partials, s);
+                                  dprime, dq_acc, dor, absmax, partials, s);
 }
 
 cudaError_t launch_param_reduce(const Geometry& g, const float* partials, float* dgate_w,

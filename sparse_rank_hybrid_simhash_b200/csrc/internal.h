@@ -43,6 +43,7 @@ struct WorkLayout {
   size_t err;                // 256 bytes: uint32 error word and spare
   size_t sort_hist;          // [2][BH][bins][tiles] i32
   size_t sort_tmp;           // [2][BH][N] i32 (intermediate order of a 2-pass sort)
+  size_t absmax;             // [2][BH] f32: largest |value| per unit (forward V, backward g_r dy / Ctot)
   size_t saved;              // a SavedLayout used when the forward has no saved buffer
   size_t d_o;                // [BH][N][d] dtype: dO_sp
   size_t dprime;             // [BH][N] f32: D' = dO_sp . O_sp - dlse
@@ -75,10 +76,16 @@ bool hash_tc_supported(const Geometry& g);
 cudaError_t launch_sort(const Geometry& g, const uint16_t* code, int32_t* perm, int32_t* hist,
                         int32_t* tmp, cudaStream_t s);
 
+// Largest |value| of every unit (zeroes absmax first); the fixed-point scale
+// of the RACE build is derived from it.
+cudaError_t launch_unit_absmax(const Geometry& g, const void* vals, bool vals_f32, float* absmax,
+                               cudaStream_t s);
 // RACE tables: sums[bh][l][b][:] = sum of vals rows whose code in table l is b;
-// counts (optional) likewise.  vals_f32 selects fp32 values instead of dtype.
+// counts (optional) likewise.  vals_f32 selects fp32 values instead of dtype;
+// absmax[bh] must bound |vals| of unit bh.
 cudaError_t launch_race_build(const Geometry& g, const void* codes, const void* vals,
-                              bool vals_f32, float* sums, int32_t* counts, cudaStream_t s);
+                              bool vals_f32, const float* absmax, float* sums, int32_t* counts,
+                              uint32_t* err, cudaStream_t s);
 // out[bh][i][:] = sum_l tables[bh][l][codes[bh][i][l]][:]  (f32, overwritten)
 cudaError_t launch_race_gather_sum(const Geometry& g, const void* codes, const float* tables,
                                    float* out, cudaStream_t s);
@@ -110,11 +117,12 @@ cudaError_t launch_attn_bwd_tc(const Geometry& g, const void* q, const void* k, 
 
 // Backward of the fusion and gates (per query), then the parameter reduction
 // and the final casts.
+// absmax[bh] (zeroed by the launcher) receives the largest |g_r dy / Ctot| of unit bh.
 cudaError_t launch_fuse_bwd(const Geometry& g, const void* q, const void* dy, const void* o_sp,
                             const void* o_race, const float* lse, const int32_t* ctot,
                             const float* gate_w, const float* gate_b, const float* lam,
                             void* d_o, float* dprime, float* dq_acc, float* dor,
-                            float* partials, cudaStream_t s);
+                            float* absmax, float* partials, cudaStream_t s);
 cudaError_t launch_param_reduce(const Geometry& g, const float* partials, float* dgate_w,
                                 float* dgate_b, float* dlambda, cudaStream_t s);
 cudaError_t launch_cast_out(const Geometry& g, const float* src, void* dst, cudaStream_t s);

@@ -9,10 +9,10 @@
 //   Ctot = sum_l C[l][h_l(q)],  O_race = sum_l T[l][h_l(q)] / Ctot  (0 if Ctot = 0),
 //   Z_race = Ctot / L.
 //
-// Build: one block owns a slab of tables x a slice of d in shared memory and
-// streams every key of its unit through it (shared-memory fp32 atomics; the
-// slab is written once, so global memory sees no atomics).  Tables too large
-// for shared memory take a global-atomic variant.
+// Build: one block owns a slab of tables x a 32-wide slice of d in shared
+// memory and streams every key of its unit through it (shared-memory fp32
+// atomics; the slab is written once, so global memory sees no atomics).
+// Tables too large for shared memory take a global-atomic variant.
 // Gather: one warp per query, lanes across d, codes broadcast by shuffle.
 // The forward gather is fused with the gates, the multiplier and the output.
 #include "common.cuh"
@@ -20,51 +20,191 @@
 
 namespace elsaa {
 namespace {
+ELSAA_DEV uint32_t smem_addr32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+}  // namespace
+}  // namespace elsaa
 
-constexpr int kBuildSmemBudget = 200 * 1024;
+namespace elsaa {
+namespace {
+
+constexpr int kBuildSmemBudget = 226 * 1024;
+
+// One CTA owns tables [l0, l0 + nt) restricted to a 32-wide slice of d and
+// streams every key of its unit through them in tiles of kBuildKT keys (loaded
+// into registers one tile ahead, staged in shared memory).
+//
+// Sums accumulate in 32-bit fixed point: on B200 a warp-wide 32-bit integer
+// shared-memory reduction runs about 4x faster than an fp32 (or 64-bit) one.
+// A first pass counts the keys of every bucket (C); with C_max the largest
+// count and vmax the unit's largest |value|, the scale 2^S is the largest power
+// of two with C_max * (vmax 2^S + 1/2) < 2^31, so no partial sum can overflow.
+// Each value is rounded once to a multiple of 2^-S; integer sums are exact and
+// order-independent, so every table entry is within count * 2^-(S+1) of the
+// exact sum of its values, and the result does not depend on thread timing.
+constexpr int kBuildThreads = 1024;
+constexpr int kBuildKT = 256;
+constexpr int kDsl = 32;
+constexpr int kValsPerThread = kBuildKT * kDsl / kBuildThreads;   // 8
+constexpr int kCodesPerThreadMax = 8;                             // nt <= 32 over 4 threads per key
+
+struct BuildShape {
+  int nt, groups, nds, ntp;
+  size_t smem;
+};
+
+template <typename TV>
+ELSAA_DEV void load_vals8(const TV* src, float* dst);
+template <>
+ELSAA_DEV void load_vals8<__nv_bfloat16>(const __nv_bfloat16* src, float* dst) {
+  const uint4 raw = *reinterpret_cast<const uint4*>(src);   // 8 bf16
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    dst[2 * i] = f.x;
+    dst[2 * i + 1] = f.y;
+  }
+}
+template <>
+ELSAA_DEV void load_vals8<float>(const float* src, float* dst) {
+  const float4 a = *reinterpret_cast<const float4*>(src);
+  const float4 b = *reinterpret_cast<const float4*>(src + 4);
+  dst[0] = a.x; dst[1] = a.y; dst[2] = a.z; dst[3] = a.w;
+  dst[4] = b.x; dst[5] = b.y; dst[6] = b.z; dst[7] = b.w;
+}
+
+ELSAA_DEV void red_shared_add_u32(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 
 template <typename TV, typename CodeT>
-__global__ void __launch_bounds__(512)
-race_build_smem_kernel(const CodeT* __restrict__ codes, const TV* __restrict__ vals, int N,
-                       int L, int NB, int d, int tabs, int dsl, float* __restrict__ sums,
-                       int32_t* __restrict__ counts) {
-  extern __shared__ float tab[];
+__global__ void __launch_bounds__(kBuildThreads)
+race_build_tiled_kernel(const CodeT* __restrict__ codes, const TV* __restrict__ vals, int N,
+                        int L, int NB, int d, int nt_max, int ntp,
+                        const float* __restrict__ absmax, float* __restrict__ sums,
+                        int32_t* __restrict__ counts, uint32_t* __restrict__ err) {
+  extern __shared__ int32_t smi[];
+  __shared__ int s_cmax;
+  const int tid = threadIdx.x;
   const int bh = blockIdx.y;
-  const int nds = d / dsl;
-  const int tgroup = blockIdx.x / nds, dpart = blockIdx.x % nds;
-  const int l0 = tgroup * tabs, nt = min(L, l0 + tabs) - l0;
-  const int d0 = dpart * dsl;
-  const bool do_counts = counts != nullptr && dpart == 0;
-  int* cnt = reinterpret_cast<int*>(tab + (size_t)tabs * NB * dsl);
-  for (int i = threadIdx.x; i < nt * NB * dsl; i += blockDim.x) tab[i] = 0.f;
-  for (int i = threadIdx.x; i < nt * NB; i += blockDim.x) cnt[i] = 0;
+  const int nds = d / kDsl;
+  const int tg = blockIdx.x / nds, dsl = blockIdx.x % nds;
+  const int l0 = tg * nt_max, nt = min(L, l0 + nt_max) - l0;
+  const int d0 = dsl * kDsl;
+  int32_t* tab = smi;                                              // [nt_max][NB][32]
+  int32_t* cnt = tab + (size_t)nt_max * NB * kDsl;                 // [nt_max][NB]
+  float* vst = reinterpret_cast<float*>(cnt + (((size_t)nt_max * NB + 3) & ~(size_t)3));
+  uint16_t* cst = reinterpret_cast<uint16_t*>(vst + kBuildKT * kDsl);   // [KT][ntp]
+  for (int i = tid; i < nt * NB * kDsl; i += kBuildThreads) tab[i] = 0;
+  for (int i = tid; i < nt * NB; i += kBuildThreads) cnt[i] = 0;
+  if (tid == 0) s_cmax = 0;
   __syncthreads();
-  const CodeT* cb = codes + (size_t)bh * N * L;
-  const TV* vb = vals + (size_t)bh * N * d;
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  const int per_lane = dsl >> 5;   // 1..4
-  for (int j = w; j < N; j += nw) {
-    float x[4];
+  const CodeT* cb = codes + (size_t)bh * N * L + l0;
+  const TV* vb = vals + (size_t)bh * N * d + d0;
+
+  // pass 1: bucket counts of this CTA's tables (one thread per key)
+  for (int key = tid; key < N; key += kBuildThreads) {
+    const CodeT* kc = cb + (size_t)key * L;
+    for (int t = 0; t < nt; ++t) atomicAdd(cnt + t * NB + (int)kc[t], 1);
+  }
+  __syncthreads();
+  int cm = 0;
+  for (int i = tid; i < nt * NB; i += kBuildThreads) cm = max(cm, cnt[i]);
+  atomicMax(&s_cmax, cm);
+  __syncthreads();
+  const float vmax = absmax[bh];
+  if (!(vmax < 3.0e38f)) {   // inf or nan among the values
+    if (tid == 0) raise_error(err, ERR_CHECK);
+    return;
+  }
+  int S = 100;
+  if (s_cmax > 0 && vmax > 0.f) {
+    S = (int)floorf(log2f(2147483000.0f / ((float)s_cmax * vmax))) - 1;
+    S = max(-100, min(100, S));
+  }
+  const float scale = ldexpf(1.0f, S), inv_scale = ldexpf(1.0f, -S);
+
+  // pass 2: fixed-point sums.  Thread tid stages key tid / 4: values [voff, voff + 8)
+  // of the d-slice and codes [cq, cq + ncode) of its tables.
+  const int vkey = tid >> 2, voff = (tid & 3) * 8;
+  const int nq4 = (nt + 3) >> 2, cq = (tid & 3) * nq4;
+  const int ncode = max(0, min(nq4, nt - cq));
+  float pv[kValsPerThread];
+  uint16_t pc[kCodesPerThreadMax];
+  auto prefetch = [&](int tile) {
+    const int j = tile * kBuildKT + vkey;
+    if (j < N) {
+      load_vals8<TV>(vb + (size_t)j * d + voff, pv);
+      const CodeT* kc = cb + (size_t)j * L + cq;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      x[i] = i < per_lane ? to_f32(vb[(size_t)j * d + d0 + lane + 32 * i]) : 0.f;
-    for (int t = 0; t < nt; ++t) {
-      const int b = (int)cb[(size_t)j * L + l0 + t];
-      float* row = tab + ((size_t)t * NB + b) * dsl;
+      for (int c = 0; c < kCodesPerThreadMax; ++c)
+        if (c < ncode) pc[c] = (uint16_t)kc[c];
+    }
+  };
+  const int ntiles = (N + kBuildKT - 1) / kBuildKT;
+  prefetch(0);
+  const int w = tid >> 5, lane = tid & 31;
+  const uint32_t tab_lane = smem_addr32(tab) + lane * 4;   // this lane's column
+  const uint32_t table_bytes = (uint32_t)NB * kDsl * 4;
+  for (int tile = 0; tile < ntiles; ++tile) {
+    const int kcount = min(kBuildKT, N - tile * kBuildKT);
+    __syncthreads();   // the previous tile is fully consumed
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (i < per_lane) atomicAdd(row + lane + 32 * i, x[i]);
-      if (do_counts && lane == 0) atomicAdd(cnt + t * NB + b, 1);
+    for (int i = 0; i < kValsPerThread; i += 4)
+      *reinterpret_cast<float4*>(vst + vkey * kDsl + voff + i) =
+          make_float4(pv[i], pv[i + 1], pv[i + 2], pv[i + 3]);
+#pragma unroll
+    for (int c = 0; c < kCodesPerThreadMax; ++c)
+      if (c < ncode) cst[vkey * ntp + cq + c] = pc[c];
+    __syncthreads();
+    if (tile + 1 < ntiles) prefetch(tile + 1);
+    // warp w: keys [w * 8, w * 8 + 8) of the tile, two at a time, one row per reduction
+    constexpr int kPerWarp = kBuildKT / (kBuildThreads / 32);
+    const int kbeg = w * kPerWarp, kend = min(kbeg + kPerWarp, kcount);
+    for (int key = kbeg; key < kend; key += 2) {
+      const bool two_keys = key + 1 < kend;
+      const uint32_t xa = (uint32_t)__float2int_rn(vst[key * kDsl + lane] * scale);
+      const uint32_t xb =
+          two_keys ? (uint32_t)__float2int_rn(vst[(key + 1) * kDsl + lane] * scale) : 0u;
+      const uint16_t* ka = cst + key * ntp;
+      const uint16_t* kb2 = cst + (two_keys ? key + 1 : key) * ntp;
+      uint32_t tbase = tab_lane;
+      for (int t = 0; t < nt; ++t, tbase += table_bytes) {
+        const uint32_t ca = ka[t], cbk = kb2[t];
+        red_shared_add_u32(tbase + ca * (kDsl * 4), xa);
+        if (two_keys) red_shared_add_u32(tbase + cbk * (kDsl * 4), xb);
+      }
     }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < nt * NB * dsl; i += blockDim.x) {
-    const int t = i / (NB * dsl), rem = i % (NB * dsl), b = rem / dsl, e = rem % dsl;
-    sums[(((size_t)bh * L + l0 + t) * NB + b) * d + d0 + e] = tab[i];
+  for (int i = tid; i < nt * NB * kDsl; i += kBuildThreads) {
+    const int tb = i / kDsl, e = i % kDsl;
+    sums[((size_t)bh * L + l0) * NB * d + (size_t)tb * d + d0 + e] = (float)tab[i] * inv_scale;
   }
-  if (do_counts)
-    for (int i = threadIdx.x; i < nt * NB; i += blockDim.x)
+  if (counts != nullptr && dsl == 0)
+    for (int i = tid; i < nt * NB; i += kBuildThreads)
       counts[((size_t)bh * L + l0) * NB + i] = cnt[i];
+}
+
+// Largest |value| of every unit (an upper bound for the fixed-point scale):
+// absmax must be zeroed; non-negative floats order like their bit patterns.
+template <typename TV>
+__global__ void __launch_bounds__(256)
+unit_absmax_kernel(const TV* __restrict__ vals, int64_t per_unit, float* __restrict__ absmax) {
+  const int bh = blockIdx.y;
+  const TV* v = vals + (size_t)bh * per_unit;
+  float m = 0.f;
+  for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; i < per_unit;
+       i += (int64_t)gridDim.x * blockDim.x * 8) {
+    float x[8];
+    load_vals8<TV>(v + i, x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(x[e]));
+  }
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0) atomicMax(reinterpret_cast<int*>(absmax) + bh, __float_as_int(m));
 }
 
 // Large tables: fp32 atomics straight into zeroed global tables.
@@ -85,33 +225,82 @@ race_build_global_kernel(const CodeT* __restrict__ codes, const TV* __restrict__
   }
 }
 
-template <typename CodeT, int VEC>
+// Gathers: QL = d / 4 lanes per query (each lane owns 4 consecutive values and
+// loads 16 bytes per table row), 32 / QL queries per warp.  The query's codes
+// are loaded QL at a time, one per lane, and broadcast inside the lane group.
+template <int QL>
+ELSAA_DEV float group_sum(float v) {
+#pragma unroll
+  for (int o = QL / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+template <int QL>
+ELSAA_DEV int group_sum_i(int v) {
+#pragma unroll
+  for (int o = QL / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <typename CodeT, int QL>
 __global__ void __launch_bounds__(256)
 race_gather_sum_kernel(const CodeT* __restrict__ codes, const float* __restrict__ tables,
                        int64_t rows, int N, int L, int NB, int d, float* __restrict__ out) {
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  for (int64_t r = (int64_t)blockIdx.x * nw + w; r < rows; r += (int64_t)gridDim.x * nw) {
-    const int64_t bh = r / N;
-    float acc[VEC];
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) acc[i] = 0.f;
-    for (int t0 = 0; t0 < L; t0 += 32) {
-      const int mycode = t0 + lane < L ? (int)codes[r * L + t0 + lane] : 0;
-      const int nt = min(32, L - t0);
+  constexpr int QW = 32 / QL;
+  const int lane = threadIdx.x & 31, ql = lane % QL, gbase = lane - ql;
+  const int64_t first = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * QW;
+  const int64_t stride = (int64_t)gridDim.x * (blockDim.x >> 5) * QW;
+  for (int64_t r0 = first; r0 < rows; r0 += stride) {
+    const int64_t r = r0 + lane / QL;
+    const bool valid = r < rows;
+    const int64_t rr = valid ? r : rows - 1;
+    const int64_t bh = rr / N;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int t0 = 0; t0 < L; t0 += QL) {
+      const int mycode = t0 + ql < L ? (int)codes[rr * L + t0 + ql] : 0;
+      const int nt = min(QL, L - t0);
+#pragma unroll 8
       for (int t = 0; t < nt; ++t) {
-        const int b = __shfl_sync(0xffffffffu, mycode, t);
-        const float* row = tables + ((bh * L + t0 + t) * NB + b) * d + lane * VEC;
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) acc[i] += row[i];
+        const int b = __shfl_sync(0xffffffffu, mycode, gbase + t);
+        const float4 v = *reinterpret_cast<const float4*>(
+            tables + ((bh * L + t0 + t) * NB + b) * d + ql * 4);
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
       }
     }
-    float* o = out + r * d + lane * VEC;
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) o[i] = acc[i];
+    if (valid) *reinterpret_cast<float4*>(out + rr * d + ql * 4) = acc;
   }
 }
 
-template <typename T, typename CodeT, int VEC>
+template <typename T>
+ELSAA_DEV void load4(const T* p, float* v);
+template <>
+ELSAA_DEV void load4<float>(const float* p, float* v) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+}
+template <>
+ELSAA_DEV void load4<__nv_bfloat16>(const __nv_bfloat16* p, float* v) {
+  const uint2 raw = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
+template <typename T>
+ELSAA_DEV void store4(T* p, const float* v);
+template <>
+ELSAA_DEV void store4<float>(float* p, const float* v) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+template <>
+ELSAA_DEV void store4<__nv_bfloat16>(__nv_bfloat16* p, const float* v) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+  const __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+  uint2 raw;
+  raw.x = *reinterpret_cast<const uint32_t*>(&a);
+  raw.y = *reinterpret_cast<const uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = raw;
+}
+
+template <typename T, typename CodeT, int QL>
 __global__ void __launch_bounds__(256)
 race_fuse_fwd_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q,
                      const float* __restrict__ sums, const int32_t* __restrict__ counts,
@@ -120,58 +309,69 @@ race_fuse_fwd_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q,
                      int gate_fixed, float gs_fixed, float gr_fixed,
                      const float* __restrict__ lam, int64_t rows, int N, int L, int NB, int d,
                      T* __restrict__ y, T* __restrict__ o_race, int32_t* __restrict__ ctot_out) {
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  constexpr int QW = 32 / QL;
+  const int lane = threadIdx.x & 31, ql = lane % QL, gbase = lane - ql;
   const float lam_v = *lam;
-  for (int64_t r = (int64_t)blockIdx.x * nw + w; r < rows; r += (int64_t)gridDim.x * nw) {
-    const int64_t bh = r / N;
-    float acc[VEC];
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) acc[i] = 0.f;
+  float ws4[4] = {0.f, 0.f, 0.f, 0.f}, wr4[4] = {0.f, 0.f, 0.f, 0.f};
+  float bs = 0.f, br = 0.f;
+  if (!gate_fixed) {
+    load4<float>(gate_w + ql * 4, ws4);
+    load4<float>(gate_w + d + ql * 4, wr4);
+    bs = gate_b[0];
+    br = gate_b[1];
+  }
+  const int64_t first = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * QW;
+  const int64_t stride = (int64_t)gridDim.x * (blockDim.x >> 5) * QW;
+  for (int64_t r0 = first; r0 < rows; r0 += stride) {
+    const int64_t r = r0 + lane / QL;
+    const bool valid = r < rows;
+    const int64_t rr = valid ? r : rows - 1;
+    const int64_t bh = rr / N;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     int ctot = 0;
-    for (int t0 = 0; t0 < L; t0 += 32) {
-      const int mycode = t0 + lane < L ? (int)rcode_q[r * L + t0 + lane] : 0;
-      if (t0 + lane < L) ctot += counts[(bh * L + t0 + lane) * NB + mycode];
-      const int nt = min(32, L - t0);
+    for (int t0 = 0; t0 < L; t0 += QL) {
+      const int mycode = t0 + ql < L ? (int)rcode_q[rr * L + t0 + ql] : 0;
+      if (t0 + ql < L) ctot += counts[(bh * L + t0 + ql) * NB + mycode];
+      const int nt = min(QL, L - t0);
+#pragma unroll 8
       for (int t = 0; t < nt; ++t) {
-        const int b = __shfl_sync(0xffffffffu, mycode, t);
-        const float* row = sums + ((bh * L + t0 + t) * NB + b) * d + lane * VEC;
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) acc[i] += row[i];
+        const int b = __shfl_sync(0xffffffffu, mycode, gbase + t);
+        const float4 v = *reinterpret_cast<const float4*>(
+            sums + ((bh * L + t0 + t) * NB + b) * d + ql * 4);
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ctot += __shfl_xor_sync(0xffffffffu, ctot, o);
+    ctot = group_sum_i<QL>(ctot);
     const float inv = ctot > 0 ? 1.0f / (float)ctot : 0.f;
-    float qv[VEC], os[VEC], orc[VEC];
-    const size_t base = (size_t)r * d + lane * VEC;
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) {
-      qv[i] = to_f32(q[base + i]);
-      os[i] = to_f32(o_sp[base + i]);
-      orc[i] = acc[i] * inv;
-    }
+    const size_t base = (size_t)rr * d + ql * 4;
+    float qv[4], os[4];
+    load4<T>(q + base, qv);
+    load4<T>(o_sp + base, os);
+    const float orc[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
     float gs = gs_fixed, gr = gr_fixed;
     if (!gate_fixed) {
       float as = 0.f, ar = 0.f;
 #pragma unroll
-      for (int i = 0; i < VEC; ++i) {
-        as += qv[i] * gate_w[lane * VEC + i];
-        ar += qv[i] * gate_w[d + lane * VEC + i];
+      for (int i = 0; i < 4; ++i) {
+        as += qv[i] * ws4[i];
+        ar += qv[i] * wr4[i];
       }
-      as = warp_sum(as) + gate_b[0];
-      ar = warp_sum(ar) + gate_b[1];
+      as = group_sum<QL>(as) + bs;
+      ar = group_sum<QL>(ar) + br;
       gs = 1.0f / (1.0f + expf(-as));
       gr = 1.0f / (1.0f + expf(-ar));
     }
     // m = Z_sp / (Z_sp + lambda Z_race) = 1 / (1 + exp(log(lambda Z_race) - lse))
     const float lz = lam_v * (float)ctot / (float)L;
-    const float m = lz > 0.f ? 1.0f / (1.0f + expf(logf(lz) - lse[r])) : 1.0f;
+    const float m = lz > 0.f ? 1.0f / (1.0f + expf(logf(lz) - lse[rr])) : 1.0f;
+    if (valid) {
+      float yv[4];
 #pragma unroll
-    for (int i = 0; i < VEC; ++i) {
-      y[base + i] = from_f32<T>(gs * m * os[i] + gr * orc[i]);
-      if (o_race) o_race[base + i] = from_f32<T>(orc[i]);
+      for (int i = 0; i < 4; ++i) yv[i] = gs * m * os[i] + gr * orc[i];
+      store4<T>(y + base, yv);
+      if (o_race) store4<T>(o_race + base, orc);
+      if (ctot_out && ql == 0) ctot_out[rr] = ctot;
     }
-    if (ctot_out && lane == 0) ctot_out[r] = ctot;
   }
 }
 
@@ -180,14 +380,44 @@ int grid_for_rows(int64_t rows, int warps_per_block) {
   return (int)(b < 148 * 32 ? b : 148 * 32);
 }
 
+BuildShape build_shape(const Geometry& g) {
+  BuildShape b;
+  const size_t stage = (size_t)kBuildKT * kDsl * 4;
+  const size_t per_table = (size_t)g.NB * (kDsl + 1) * 4 + (size_t)kBuildKT * 2;
+  const size_t budget = (size_t)kBuildSmemBudget - stage - 64;
+  int nt_max = (int)(budget / per_table);
+  if (nt_max > g.L) nt_max = g.L;
+  if (nt_max > 4 * kCodesPerThreadMax) nt_max = 4 * kCodesPerThreadMax;   // codes per thread bound
+  b.nds = g.d / kDsl;
+  // Choose the tables per CTA: every CTA streams all N keys, paying about one
+  // pass over its values plus two cycles per table reduction per key; CTAs run
+  // one per SM in waves of 148, so minimise waves x (2 nt + 1).
+  int best = nt_max;
+  long long best_cost = -1;
+  for (int nt = nt_max; nt >= 1; --nt) {
+    const long long ctas = (long long)((g.L + nt - 1) / nt) * b.nds * g.BH;
+    const long long waves = (ctas + 147) / 148;
+    const long long cost = waves * (2 * nt + 1);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = nt;
+    }
+  }
+  const int nt = nt_max >= 1 ? best : 0;
+  b.nt = nt;
+  b.groups = nt > 0 ? (g.L + nt - 1) / nt : 0;
+  b.ntp = (nt + 1) & ~1;
+  b.smem = (size_t)nt * g.NB * kDsl * 4 + (((size_t)nt * g.NB + 3) & ~(size_t)3) * 4 + stage +
+           (size_t)kBuildKT * b.ntp * 2 + 16;
+  return b;
+}
+
 template <typename TV, typename CodeT>
-cudaError_t build(const Geometry& g, const void* codes, const void* vals, float* sums,
-                  int32_t* counts, cudaStream_t s) {
-  // slab: `tabs` tables x a d-slice of `dsl` (a multiple of 32) in shared memory
-  int dsl = g.d;
-  while (dsl > 32 && (size_t)g.NB * (dsl + 1) * 4 > (size_t)kBuildSmemBudget) dsl >>= 1;
-  const size_t per_table = (size_t)g.NB * (dsl + 1) * 4;
-  if (per_table > (size_t)kBuildSmemBudget) {
+cudaError_t build(const Geometry& g, const void* codes, const void* vals, const float* absmax,
+                  float* sums, int32_t* counts, uint32_t* err, cudaStream_t s) {
+  const BuildShape b = build_shape(g);
+  if (b.nt < 1) {
+    // tables too large for shared memory even one at a time: global atomics
     cudaError_t e = cudaMemsetAsync(sums, 0, (size_t)g.BH * g.L * g.NB * g.d * 4, s);
     if (e != cudaSuccess) return e;
     if (counts) {
@@ -200,17 +430,13 @@ cudaError_t build(const Geometry& g, const void* codes, const void* vals, float*
         g.d, sums, counts);
     return cudaGetLastError();
   }
-  int tabs = (int)(kBuildSmemBudget / per_table);
-  if (tabs > g.L) tabs = g.L;
-  const int groups = (g.L + tabs - 1) / tabs;
-  const size_t smem = (size_t)tabs * g.NB * dsl * 4 + (size_t)tabs * g.NB * 4;
-  cudaError_t e = cudaFuncSetAttribute(race_build_smem_kernel<TV, CodeT>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(race_build_tiled_kernel<TV, CodeT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)b.smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(groups * (g.d / dsl), g.BH);
-  race_build_smem_kernel<TV, CodeT><<<grid, 512, smem, s>>>(
-      static_cast<const CodeT*>(codes), static_cast<const TV*>(vals), g.N, g.L, g.NB, g.d, tabs,
-      dsl, sums, counts);
+  const dim3 grid(b.groups * b.nds, g.BH);
+  race_build_tiled_kernel<TV, CodeT><<<grid, kBuildThreads, b.smem, s>>>(
+      static_cast<const CodeT*>(codes), static_cast<const TV*>(vals), g.N, g.L, g.NB, g.d, b.nt,
+      b.ntp, absmax, sums, counts, err);
   return cudaGetLastError();
 }
 
@@ -218,12 +444,12 @@ template <typename CodeT>
 cudaError_t gather_sum(const Geometry& g, const void* codes, const float* tables, float* out,
                        cudaStream_t s) {
   const int64_t rows = (int64_t)g.BH * g.N;
-  const int grid = grid_for_rows(rows, 8);
+  const int grid = grid_for_rows((rows * g.d / 4 + 31) / 32, 8);
   const CodeT* c = static_cast<const CodeT*>(codes);
-  switch (g.d / 32) {
-    case 1: race_gather_sum_kernel<CodeT, 1><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
-    case 2: race_gather_sum_kernel<CodeT, 2><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
-    default: race_gather_sum_kernel<CodeT, 4><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
+  switch (g.d) {
+    case 32: race_gather_sum_kernel<CodeT, 8><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
+    case 64: race_gather_sum_kernel<CodeT, 16><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
+    default: race_gather_sum_kernel<CodeT, 32><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
   }
   return cudaGetLastError();
 }
@@ -235,16 +461,16 @@ cudaError_t fuse_fwd(const Geometry& g, const void* q, const void* rcode_q, cons
                      void* o_race, int32_t* ctot, cudaStream_t s, int gate_fixed, float gs,
                      float gr) {
   const int64_t rows = (int64_t)g.BH * g.N;
-  const int grid = grid_for_rows(rows, 8);
+  const int grid = grid_for_rows((rows * g.d / 4 + 31) / 32, 8);
 #define ELSAA_FUSE(VEC)                                                                        \
   race_fuse_fwd_kernel<T, CodeT, VEC><<<grid, 256, 0, s>>>(                                    \
       static_cast<const T*>(q), static_cast<const CodeT*>(rcode_q), sums, counts,              \
       static_cast<const T*>(o_sp), lse, gate_w, gate_b, gate_fixed, gs, gr, lam, rows, g.N,    \
       g.L, g.NB, g.d, static_cast<T*>(y), static_cast<T*>(o_race), ctot)
-  switch (g.d / 32) {
-    case 1: ELSAA_FUSE(1); break;
-    case 2: ELSAA_FUSE(2); break;
-    default: ELSAA_FUSE(4); break;
+  switch (g.d) {
+    case 32: ELSAA_FUSE(8); break;
+    case 64: ELSAA_FUSE(16); break;
+    default: ELSAA_FUSE(32); break;
   }
 #undef ELSAA_FUSE
   return cudaGetLastError();
@@ -252,13 +478,32 @@ cudaError_t fuse_fwd(const Geometry& g, const void* q, const void* rcode_q, cons
 
 }  // namespace
 
-cudaError_t launch_race_build(const Geometry& g, const void* codes, const void* vals,
-                              bool vals_f32, float* sums, int32_t* counts, cudaStream_t s) {
+cudaError_t launch_unit_absmax(const Geometry& g, const void* vals, bool vals_f32, float* absmax,
+                               cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(absmax, 0, (size_t)g.BH * sizeof(float), s);
+  if (e != cudaSuccess) return e;
+  const int64_t per_unit = (int64_t)g.N * g.d;
+  const int64_t want = (per_unit / 8 + 255) / 256;
+  const dim3 grid((unsigned)(want < 64 ? want : 64), g.BH);
   if (vals_f32 || !g.bf16)
-    return g.rcode_bytes == 1 ? build<float, uint8_t>(g, codes, vals, sums, counts, s)
-                              : build<float, uint16_t>(g, codes, vals, sums, counts, s);
-  return g.rcode_bytes == 1 ? build<__nv_bfloat16, uint8_t>(g, codes, vals, sums, counts, s)
-                            : build<__nv_bfloat16, uint16_t>(g, codes, vals, sums, counts, s);
+    unit_absmax_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(vals), per_unit,
+                                                    absmax);
+  else
+    unit_absmax_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(vals), per_unit, absmax);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_race_build(const Geometry& g, const void* codes, const void* vals,
+                              bool vals_f32, const float* absmax, float* sums, int32_t* counts,
+                              uint32_t* err, cudaStream_t s) {
+  if (vals_f32 || !g.bf16)
+    return g.rcode_bytes == 1
+               ? build<float, uint8_t>(g, codes, vals, absmax, sums, counts, err, s)
+               : build<float, uint16_t>(g, codes, vals, absmax, sums, counts, err, s);
+  return g.rcode_bytes == 1
+             ? build<__nv_bfloat16, uint8_t>(g, codes, vals, absmax, sums, counts, err, s)
+             : build<__nv_bfloat16, uint16_t>(g, codes, vals, absmax, sums, counts, err, s);
 }
 
 cudaError_t launch_race_gather_sum(const Geometry& g, const void* codes, const float* tables,
