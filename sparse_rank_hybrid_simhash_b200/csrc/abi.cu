@@ -76,6 +76,7 @@ WorkLayout work_layout(const Geometry& g) {
   w.sort_hist = take((size_t)2 * g.BH * g.sort_bins * g.sort_tiles * 4);
   w.sort_tmp = take(2 * bhn * 4);
   w.absmax = take((size_t)2 * g.BH * 4);
+  w.gtab = take((size_t)g.BH * g.L * g.NB * g.d * 2);
   const size_t shared_base = off;
   // forward without a saved buffer: the saved layout lives here
   w.saved = take(saved_layout(g).total);
@@ -215,16 +216,22 @@ elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const vo
   // 3. RACE tables from the keys
   float* absmax = (float*)(w + wl.absmax);
   ELSAA_TRY(launch_unit_absmax(g, v, false, absmax, s));
-  ELSAA_TRY(launch_race_build(g, rcode_k, v, false, absmax, sums, counts, err, s));
+  // gathers read tables in the data dtype: a bf16 copy, or the fp32 sums themselves
+  __nv_bfloat16* gtab = g.bf16 ? (__nv_bfloat16*)(w + wl.gtab) : nullptr;
+  const void* gather_tables = g.bf16 ? (const void*)gtab : (const void*)sums;
+  ELSAA_TRY(launch_race_build(g, rcode_k, v, false, absmax, sums, true, gtab, counts, err, s));
   ELSAA_TRY(mark(events, 3, s));
   // 4. exact sparse branch
-  if (g.tc_attn)
+  if (g.tc_attn && attn_pipe_supported(g))
+    ELSAA_TRY(launch_attn_fwd_pipe(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s));
+  else if (g.tc_attn)
     ELSAA_TRY(launch_attn_fwd_tc(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s));
   else
     ELSAA_TRY(launch_attn_fwd_simt(g, q, k, v, perm, perm + bhn, o_sp, lse, s));
   ELSAA_TRY(mark(events, 4, s));
   // 5. RACE gather, gates, multiplier and output
-  ELSAA_TRY(launch_race_fuse_fwd(g, q, rcode, sums, counts, o_sp, lse, gate_w, gate_b, lambda, y,
+  ELSAA_TRY(launch_race_fuse_fwd(g, q, rcode, gather_tables, counts, o_sp, lse, gate_w, gate_b,
+                                 lambda, y,
                                  saved ? sv + sl.o_race : nullptr,
                                  saved ? (int32_t*)(sv + sl.ctot) : nullptr, s));
   ELSAA_TRY(mark(events, 5, s));
@@ -288,9 +295,11 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
                             dprime, dq_acc, dor, absmax, partials, s));
   ELSAA_TRY(mark(events, 1, s));
   // 2. RACE backward: scatter into the table gradient by query code, gather by key code
-  ELSAA_TRY(launch_race_build(g, rcode, dor, true, absmax, d_t, nullptr,
+  __nv_bfloat16* gtab = g.bf16 ? (__nv_bfloat16*)(w + wl.gtab) : nullptr;
+  ELSAA_TRY(launch_race_build(g, rcode, dor, true, absmax, d_t, !g.bf16, gtab, nullptr,
                               (uint32_t*)(w + wl.err), s));
-  ELSAA_TRY(launch_race_gather_sum(g, rcode_k, d_t, dv_acc, s));
+  ELSAA_TRY(launch_race_gather_sum(g, rcode_k, g.bf16 ? (const void*)gtab : (const void*)d_t,
+                                   dv_acc, s));
   ELSAA_TRY(mark(events, 2, s));
   // 3. sparse branch backward, 4. outputs
   if (g.tc_attn) {

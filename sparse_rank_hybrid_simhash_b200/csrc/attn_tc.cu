@@ -41,17 +41,21 @@ struct FwdLayout {
   static constexpr uint32_t kP = kV0 + 2 * kSub * kSubBytes;
   static constexpr uint32_t kBar = kP + 2 * kSubBytes;      // P: 128 x 128 bf16 in 2 sub-tiles
   static constexpr uint32_t kDyn = kBar + 64;
+  // Token indices of the rows being gathered live in the P buffer, which is
+  // idle whenever a gather is issued.
+  static constexpr uint32_t kIdx = kP;
 };
 
-// Gathers `rows` rows (by `perm`) of a [*, D] bf16 matrix into a swizzled tile.
+// Gathers `rows` rows of a [*, D] bf16 matrix into a swizzled tile; the token
+// index of each row comes from shared memory (staged by one coalesced load).
 template <int D>
-ELSAA_DEV void gather_rows(uint32_t dst, const __nv_bfloat16* src_base, const int32_t* perm,
+ELSAA_DEV void gather_rows(uint32_t dst, const __nv_bfloat16* src_base, const int32_t* idx,
                            int rows) {
   constexpr int kChunks = D / 8;   // 16-byte chunks per row
   for (int i = threadIdx.x; i < rows * kChunks; i += kThreads) {
     const int row = i / kChunks, ch = i % kChunks;
     const int sub = ch >> 3, c8 = ch & 7;
-    const __nv_bfloat16* src = src_base + (size_t)perm[row] * D + ch * 8;
+    const __nv_bfloat16* src = src_base + (size_t)idx[row] * D + ch * 8;
     cp_async16(dst + sub * (128 * 128) + sw128_off(row, c8), src, 16);
   }
 }
@@ -69,6 +73,8 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
   uint64_t* bar_s = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
   uint64_t* bar_o = bar_s + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_s + 2);
+  int32_t* qidx = reinterpret_cast<int32_t*>(smem + Lay::kIdx);   // [128], prologue only
+  int32_t* kidx = qidx + 128;                                     // [2][128]
 
   const int tid = threadIdx.x, warp = tid >> 5;
   if ((sbase & 1023u) != 0) {   // the swizzled tiles need a 1024-byte aligned base
@@ -102,12 +108,17 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  // prologue loads: Q tile and the first two key blocks
-  gather_rows<D>(sbase + Lay::kQ, qb, pq + r0, kTile);
+  // prologue loads: token indices, then the Q tile and the first two key blocks
+  const int my_token = pq[r0 + tid];   // this thread's query row, kept for the epilogue
+  qidx[tid] = my_token;
+  for (int b = 0; b < nkb && b < 2; ++b)
+    if (tid < kend - kbase - b * kKB) kidx[b * 128 + tid] = pk[kbase + b * kKB + tid];
+  __syncthreads();
+  gather_rows<D>(sbase + Lay::kQ, qb, qidx, kTile);
   for (int b = 0; b < nkb && b < 2; ++b) {
     const int nb = min(kKB, kend - kbase - b * kKB);
-    gather_rows<D>(sbase + Lay::kK0 + b * Lay::kSub * Lay::kSubBytes, kb, pk + kbase + b * kKB, nb);
-    gather_rows<D>(sbase + Lay::kV0 + b * Lay::kSub * Lay::kSubBytes, vb, pk + kbase + b * kKB, nb);
+    gather_rows<D>(sbase + Lay::kK0 + b * Lay::kSub * Lay::kSubBytes, kb, kidx + b * 128, nb);
+    gather_rows<D>(sbase + Lay::kV0 + b * Lay::kSub * Lay::kSubBytes, vb, kidx + b * 128, nb);
   }
   cp_async_commit();
   cp_async_wait_all();
@@ -130,8 +141,11 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
       fence_after();
     }
     if (b >= 2) {
-      gather_rows<D>(sbase + Lay::kK0 + slot, kb, pk + kbase + b * kKB, nb);
-      gather_rows<D>(sbase + Lay::kV0 + slot, vb, pk + kbase + b * kKB, nb);
+      int32_t* ki = kidx + (b & 1) * 128;
+      if (tid < nb) ki[tid] = pk[kbase + b * kKB + tid];
+      __syncthreads();
+      gather_rows<D>(sbase + Lay::kK0 + slot, kb, ki, nb);
+      gather_rows<D>(sbase + Lay::kV0 + slot, vb, ki, nb);
       cp_async_commit();
       cp_async_wait_all();
       fence_async_smem();
@@ -229,7 +243,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
   }
   if (ok) {
     fence_after();
-    const int i = pq[r];
+    const int i = my_token;
     const float inv = 1.0f / l_run;
     __nv_bfloat16* orow = o_sp + (unit + i) * D;
     for (int c0 = 0; c0 < D; c0 += 32) {

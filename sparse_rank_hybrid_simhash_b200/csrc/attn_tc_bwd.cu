@@ -45,21 +45,31 @@ struct BwdLayout {
   static constexpr uint32_t kDST = kPT + 2 * kSubBytes;
   static constexpr uint32_t kLse = kDST + 2 * kSubBytes;     // 128 floats
   static constexpr uint32_t kDpr = kLse + 128 * 4;           // 128 floats
-  static constexpr uint32_t kBar = kDpr + 128 * 4;
+  static constexpr uint32_t kIdx = kDpr + 128 * 4;           // token indices: keys, queries
+  static constexpr uint32_t kBar = kIdx + 2 * 128 * 4;
+  static constexpr uint32_t kDQ = kPT;   // dQ staging (fp32, 128 x D) reuses P^T and dS^T
   static constexpr uint32_t kDyn = kBar + 64;
   // TMEM columns
   static constexpr uint32_t kTS = 0, kTdP = 128, kTdV = 256, kTdK = 256 + D, kTdQ = 0;
 };
 
+// Gathers `rows` rows of a [*, D] bf16 matrix into a swizzled tile; the token
+// index of each row comes from shared memory.
 template <int D>
-ELSAA_DEV void gather_rows(uint32_t dst, const __nv_bfloat16* src_base, const int32_t* perm,
+ELSAA_DEV void gather_rows(uint32_t dst, const __nv_bfloat16* src_base, const int32_t* idx,
                            int rows) {
   constexpr int kChunks = D / 8;
   for (int i = threadIdx.x; i < rows * kChunks; i += kThreads) {
     const int row = i / kChunks, ch = i % kChunks;
-    const __nv_bfloat16* src = src_base + (size_t)perm[row] * D + ch * 8;
+    const __nv_bfloat16* src = src_base + (size_t)idx[row] * D + ch * 8;
     cp_async16(dst + (ch >> 3) * (128 * 128) + sw128_off(row, ch & 7), src, 16);
   }
+}
+
+ELSAA_DEV void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
 }
 
 ELSAA_DEV uint32_t pack_bf16(float a, float b) {
@@ -84,6 +94,9 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_a + 2);
   float* s_lse = reinterpret_cast<float*>(smem + Lay::kLse);
   float* s_dpr = reinterpret_cast<float*>(smem + Lay::kDpr);
+  int32_t* kidx = reinterpret_cast<int32_t*>(smem + Lay::kIdx);   // [128] keys of the tile
+  int32_t* qidx = kidx + 128;                                      // [128] queries of the block
+  float* s_dq = reinterpret_cast<float*>(smem + Lay::kDQ);         // [128][D], chunk-rotated
   const int tid = threadIdx.x, warp = tid >> 5;
   if ((sbase & 1023u) != 0) {
     if (tid == 0) raise_error(err, ERR_CHECK);
@@ -109,8 +122,10 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  gather_rows<D>(sbase + Lay::kK, k + unit * D, pk + k0, kTile);
-  gather_rows<D>(sbase + Lay::kV, v + unit * D, pk + k0, kTile);
+  kidx[tid] = pk[k0 + tid];
+  __syncthreads();
+  gather_rows<D>(sbase + Lay::kK, k + unit * D, kidx, kTile);
+  gather_rows<D>(sbase + Lay::kV, v + unit * D, kidx, kTile);
   cp_async_commit();
   fence_before();
   __syncthreads();
@@ -122,11 +137,13 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
   for (int b = 0; b < nqb; ++b) {
     const int qb0 = qbase + b * kTile;
     const int nq = min(kTile, qend - qb0);
-    gather_rows<D>(sbase + Lay::kQ, q + unit * D, pq + qb0, nq);
-    gather_rows<D>(sbase + Lay::kDO, d_o + unit * D, pq + qb0, nq);
+    if (tid < nq) qidx[tid] = pq[qb0 + tid];
+    __syncthreads();
+    gather_rows<D>(sbase + Lay::kQ, q + unit * D, qidx, nq);
+    gather_rows<D>(sbase + Lay::kDO, d_o + unit * D, qidx, nq);
     cp_async_commit();
     if (tid < nq) {
-      const int i = pq[qb0 + tid];
+      const int i = qidx[tid];
       s_lse[tid] = lse[unit + i] * 1.4426950408889634f;
       s_dpr[tid] = dprime[unit + i];
     }
@@ -219,18 +236,30 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
     ok = mbar_wait(bar_b, b & 1, err);
     if (__syncthreads_or(!ok)) break;
     fence_after();
-    // dQ rows of this block: TMEM lane t = query qb0 + t
-    {
-      const bool mine = tid < nq;
-      float* dst = dq_acc + (unit + (mine ? pq[qb0 + tid] : 0)) * D;
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        float g[32];
-        tmem_ld32(tmem + Lay::kTdQ + lane_off + c0, g);
-        tmem_ld_wait();
-        if (mine) {
+    // dQ rows of this block: TMEM lane t = query qb0 + t.  Stage them in shared
+    // memory (16-byte chunk c of row t at chunk position (c + t) mod D/4, so
+    // neither the column writes nor the row reads conflict), then add whole
+    // rows to the fp32 accumulator with 16-byte vector reductions.
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      float g[32];
+      tmem_ld32(tmem + Lay::kTdQ + lane_off + c0, g);
+      tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) atomicAdd(dst + c0 + i, g[i]);
-        }
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const int chunk = (c0 / 4 + q4 + tid) % (D / 4);
+        *reinterpret_cast<float4*>(s_dq + tid * D + chunk * 4) =
+            make_float4(g[q4 * 4], g[q4 * 4 + 1], g[q4 * 4 + 2], g[q4 * 4 + 3]);
+      }
+    }
+    __syncthreads();
+    {
+      constexpr int kRowLanes = D / 4;               // lanes per row
+      constexpr int kRowsPerIter = kThreads / kRowLanes;
+      const int c = tid % kRowLanes;
+      for (int row = tid / kRowLanes; row < nq; row += kRowsPerIter) {
+        const float4 val =
+            *reinterpret_cast<const float4*>(s_dq + row * D + ((c + row) % kRowLanes) * 4);
+        red_add_v4(dq_acc + (unit + qidx[row]) * D + c * 4, val.x, val.y, val.z, val.w);
       }
     }
     fence_before();
@@ -238,7 +267,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
   }
   if (ok) {
     fence_after();
-    const int i = pk[k0 + tid];
+    const int i = kidx[tid];
     const float* dvr = dv_race + (unit + i) * D;
     __nv_bfloat16* dvo = dv + (unit + i) * D;
     __nv_bfloat16* dko = dk + (unit + i) * D;

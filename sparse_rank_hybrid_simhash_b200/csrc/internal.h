@@ -2,6 +2,7 @@
 // launchers each .cu file provides.  Not part of the public ABI.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -44,6 +45,7 @@ struct WorkLayout {
   size_t sort_hist;          // [2][BH][bins][tiles] i32
   size_t sort_tmp;           // [2][BH][N] i32 (intermediate order of a 2-pass sort)
   size_t absmax;             // [2][BH] f32: largest |value| per unit (forward V, backward g_r dy / Ctot)
+  size_t gtab;               // [BH][L][NB][d] bf16: the table copy the RACE gathers read
   size_t saved;              // a SavedLayout used when the forward has no saved buffer
   size_t d_o;                // [BH][N][d] dtype: dO_sp
   size_t dprime;             // [BH][N] f32: D' = dO_sp . O_sp - dlse
@@ -80,21 +82,24 @@ cudaError_t launch_sort(const Geometry& g, const uint16_t* code, int32_t* perm, 
 // of the RACE build is derived from it.
 cudaError_t launch_unit_absmax(const Geometry& g, const void* vals, bool vals_f32, float* absmax,
                                cudaStream_t s);
-// RACE tables: sums[bh][l][b][:] = sum of vals rows whose code in table l is b;
-// counts (optional) likewise.  vals_f32 selects fp32 values instead of dtype;
-// absmax[bh] must bound |vals| of unit bh.
+// RACE tables: sums[bh][l][b][:] = sum of vals rows whose code in table l is b,
+// counts (optional) likewise, and (gtab non-null) a bf16 copy for the gathers.
+// vals_f32 selects fp32 values instead of dtype; absmax[bh] must bound |vals|
+// of unit bh; keep_sums = false leaves `sums` as scratch only.
 cudaError_t launch_race_build(const Geometry& g, const void* codes, const void* vals,
-                              bool vals_f32, const float* absmax, float* sums, int32_t* counts,
-                              uint32_t* err, cudaStream_t s);
-// out[bh][i][:] = sum_l tables[bh][l][codes[bh][i][l]][:]  (f32, overwritten)
-cudaError_t launch_race_gather_sum(const Geometry& g, const void* codes, const float* tables,
+                              bool vals_f32, const float* absmax, float* sums, bool keep_sums,
+                              __nv_bfloat16* gtab, int32_t* counts, uint32_t* err,
+                              cudaStream_t s);
+// out[bh][i][:] = sum_l tables[bh][l][codes[bh][i][l]][:]  (f32, overwritten);
+// tables in the data dtype (bf16 copy, or the fp32 sums for fp32 data).
+cudaError_t launch_race_gather_sum(const Geometry& g, const void* codes, const void* tables,
                                    float* out, cudaStream_t s);
 // Forward RACE gather fused with the gates, the multiplier and the output.
 cudaError_t launch_race_fuse_fwd(const Geometry& g, const void* q, const void* rcode_q,
-                                 const float* sums, const int32_t* counts, const void* o_sp,
-                                 const float* lse, const float* gate_w, const float* gate_b,
-                                 const float* lam, void* y, void* o_race, int32_t* ctot,
-                                 cudaStream_t s);
+                                 const void* tables, const int32_t* counts,
+                                 const void* o_sp, const float* lse, const float* gate_w,
+                                 const float* gate_b, const float* lam, void* y, void* o_race,
+                                 int32_t* ctot, cudaStream_t s);
 
 // Sparse branch, CUDA-core kernels.
 cudaError_t launch_attn_fwd_simt(const Geometry& g, const void* q, const void* k, const void* v,
@@ -109,6 +114,11 @@ cudaError_t launch_attn_fwd_tc(const Geometry& g, const void* q, const void* k, 
                                const int32_t* perm_q, const int32_t* perm_k, void* o_sp,
                                float* lse, uint32_t* err, cudaStream_t s);
 bool attn_tc_supported(const Geometry& g);
+// Persistent warp-specialized forward (d = 64, chunk <= 128 dividing 128).
+bool attn_pipe_supported(const Geometry& g);
+cudaError_t launch_attn_fwd_pipe(const Geometry& g, const void* q, const void* k, const void* v,
+                                 const int32_t* perm_q, const int32_t* perm_k, void* o_sp,
+                                 float* lse, uint32_t* err, cudaStream_t s);
 // tcgen05 backward: dq_acc += dQ (fp32 atomics); dk, dv written (dv adds dv_race).
 cudaError_t launch_attn_bwd_tc(const Geometry& g, const void* q, const void* k, const void* v,
                                const int32_t* perm_q, const int32_t* perm_k, const void* d_o,

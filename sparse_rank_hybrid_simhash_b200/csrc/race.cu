@@ -84,7 +84,8 @@ __global__ void __launch_bounds__(kBuildThreads)
 race_build_tiled_kernel(const CodeT* __restrict__ codes, const TV* __restrict__ vals, int N,
                         int L, int NB, int d, int nt_max, int ntp,
                         const float* __restrict__ absmax, float* __restrict__ sums,
-                        int32_t* __restrict__ counts, uint32_t* __restrict__ err) {
+                        __nv_bfloat16* __restrict__ gtab, int32_t* __restrict__ counts,
+                        uint32_t* __restrict__ err) {
   extern __shared__ int32_t smi[];
   __shared__ int s_cmax;
   const int tid = threadIdx.x;
@@ -181,7 +182,10 @@ race_build_tiled_kernel(const CodeT* __restrict__ codes, const TV* __restrict__ 
   __syncthreads();
   for (int i = tid; i < nt * NB * kDsl; i += kBuildThreads) {
     const int tb = i / kDsl, e = i % kDsl;
-    sums[((size_t)bh * L + l0) * NB * d + (size_t)tb * d + d0 + e] = (float)tab[i] * inv_scale;
+    const size_t o = ((size_t)bh * L + l0) * NB * d + (size_t)tb * d + d0 + e;
+    const float val = (float)tab[i] * inv_scale;
+    if (sums) sums[o] = val;
+    if (gtab) gtab[o] = __float2bfloat16_rn(val);
   }
   if (counts != nullptr && dsl == 0)
     for (int i = tid; i < nt * NB; i += kBuildThreads)
@@ -225,9 +229,10 @@ race_build_global_kernel(const CodeT* __restrict__ codes, const TV* __restrict__
   }
 }
 
-// Gathers: QL = d / 4 lanes per query (each lane owns 4 consecutive values and
-// loads 16 bytes per table row), 32 / QL queries per warp.  The query's codes
-// are loaded QL at a time, one per lane, and broadcast inside the lane group.
+// Gathers read bf16 copies of the tables: QL = d / 8 lanes per query (each
+// lane owns 8 consecutive values and loads 16 bytes per table row), 32 / QL
+// queries per warp.  The query's codes are loaded QL at a time, one per lane,
+// and broadcast inside the lane group.
 template <int QL>
 ELSAA_DEV float group_sum(float v) {
 #pragma unroll
@@ -241,11 +246,56 @@ ELSAA_DEV int group_sum_i(int v) {
   return v;
 }
 
-template <typename CodeT, int QL>
+// Adds the 16 bytes at `row` (8 bf16 or 4 fp32 values) to acc.
+ELSAA_DEV void acc_row(float* acc, const __nv_bfloat16* row) {
+  const uint4 raw = *reinterpret_cast<const uint4*>(row);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    acc[2 * i] += f.x;
+    acc[2 * i + 1] += f.y;
+  }
+}
+ELSAA_DEV void acc_row(float* acc, const float* row) {
+  const float4 f = *reinterpret_cast<const float4*>(row);
+  acc[0] += f.x; acc[1] += f.y; acc[2] += f.z; acc[3] += f.w;
+}
+
+
+
+// EL consecutive values (EL = 8 for bf16 tables, 4 for fp32) to T storage.
+template <typename T, int EL>
+ELSAA_DEV void store_el(T* p, const float* v) {
+#pragma unroll
+  for (int i = 0; i < EL; ++i) p[i] = from_f32<T>(v[i]);
+}
+template <>
+ELSAA_DEV void store_el<__nv_bfloat16, 8>(__nv_bfloat16* p, const float* v) {
+  uint4 raw;
+  uint32_t* w = reinterpret_cast<uint32_t*>(&raw);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    w[i] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  *reinterpret_cast<uint4*>(p) = raw;
+}
+template <>
+ELSAA_DEV void store_el<float, 4>(float* p, const float* v) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+template <>
+ELSAA_DEV void store_el<float, 8>(float* p, const float* v) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+template <typename TT, typename CodeT, int QL>
 __global__ void __launch_bounds__(256)
-race_gather_sum_kernel(const CodeT* __restrict__ codes, const float* __restrict__ tables,
+race_gather_sum_kernel(const CodeT* __restrict__ codes, const TT* __restrict__ tables,
                        int64_t rows, int N, int L, int NB, int d, float* __restrict__ out) {
-  constexpr int QW = 32 / QL;
+  constexpr int QW = 32 / QL, EL = 16 / sizeof(TT);
   const int lane = threadIdx.x & 31, ql = lane % QL, gbase = lane - ql;
   const int64_t first = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * QW;
   const int64_t stride = (int64_t)gridDim.x * (blockDim.x >> 5) * QW;
@@ -254,69 +304,80 @@ race_gather_sum_kernel(const CodeT* __restrict__ codes, const float* __restrict_
     const bool valid = r < rows;
     const int64_t rr = valid ? r : rows - 1;
     const int64_t bh = rr / N;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int t0 = 0; t0 < L; t0 += QL) {
       const int mycode = t0 + ql < L ? (int)codes[rr * L + t0 + ql] : 0;
       const int nt = min(QL, L - t0);
 #pragma unroll 8
       for (int t = 0; t < nt; ++t) {
         const int b = __shfl_sync(0xffffffffu, mycode, gbase + t);
-        const float4 v = *reinterpret_cast<const float4*>(
-            tables + ((bh * L + t0 + t) * NB + b) * d + ql * 4);
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        acc_row(acc, tables + ((bh * L + t0 + t) * NB + b) * d + ql * EL);
       }
     }
-    if (valid) *reinterpret_cast<float4*>(out + rr * d + ql * 4) = acc;
+    if (valid) store_el<float, EL>(out + rr * d + ql * EL, acc);
   }
 }
 
 template <typename T>
-ELSAA_DEV void load4(const T* p, float* v);
+ELSAA_DEV void load8(const T* p, float* v);
 template <>
-ELSAA_DEV void load4<float>(const float* p, float* v) {
+ELSAA_DEV void load8<float>(const float* p, float* v) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0];
+  const float4 b = reinterpret_cast<const float4*>(p)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+template <>
+ELSAA_DEV void load8<__nv_bfloat16>(const __nv_bfloat16* p, float* v) {
+  const uint4 raw = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
+template <typename T, int EL>
+ELSAA_DEV void load_el(const T* p, float* v) {
+#pragma unroll
+  for (int i = 0; i < EL; ++i) v[i] = to_f32(p[i]);
+}
+template <>
+ELSAA_DEV void load_el<__nv_bfloat16, 8>(const __nv_bfloat16* p, float* v) {
+  load8<__nv_bfloat16>(p, v);
+}
+template <>
+ELSAA_DEV void load_el<float, 8>(const float* p, float* v) {
+  load8<float>(p, v);
+}
+template <>
+ELSAA_DEV void load_el<float, 4>(const float* p, float* v) {
   const float4 a = *reinterpret_cast<const float4*>(p);
   v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
 }
-template <>
-ELSAA_DEV void load4<__nv_bfloat16>(const __nv_bfloat16* p, float* v) {
-  const uint2 raw = *reinterpret_cast<const uint2*>(p);
-  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
-  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
-  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
-}
-template <typename T>
-ELSAA_DEV void store4(T* p, const float* v);
-template <>
-ELSAA_DEV void store4<float>(float* p, const float* v) {
-  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-}
-template <>
-ELSAA_DEV void store4<__nv_bfloat16>(__nv_bfloat16* p, const float* v) {
-  const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
-  const __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
-  uint2 raw;
-  raw.x = *reinterpret_cast<const uint32_t*>(&a);
-  raw.y = *reinterpret_cast<const uint32_t*>(&b);
-  *reinterpret_cast<uint2*>(p) = raw;
-}
 
+// T: data type; the tables have the data type too (bf16 copy or fp32 sums).
 template <typename T, typename CodeT, int QL>
 __global__ void __launch_bounds__(256)
 race_fuse_fwd_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q,
-                     const float* __restrict__ sums, const int32_t* __restrict__ counts,
+                     const T* __restrict__ tables, const int32_t* __restrict__ counts,
                      const T* __restrict__ o_sp, const float* __restrict__ lse,
                      const float* __restrict__ gate_w, const float* __restrict__ gate_b,
                      int gate_fixed, float gs_fixed, float gr_fixed,
                      const float* __restrict__ lam, int64_t rows, int N, int L, int NB, int d,
                      T* __restrict__ y, T* __restrict__ o_race, int32_t* __restrict__ ctot_out) {
-  constexpr int QW = 32 / QL;
+  constexpr int QW = 32 / QL, EL = 16 / sizeof(T);
   const int lane = threadIdx.x & 31, ql = lane % QL, gbase = lane - ql;
   const float lam_v = *lam;
-  float ws4[4] = {0.f, 0.f, 0.f, 0.f}, wr4[4] = {0.f, 0.f, 0.f, 0.f};
+  float ws8[EL], wr8[EL];
+#pragma unroll
+  for (int i = 0; i < EL; ++i) ws8[i] = wr8[i] = 0.f;
   float bs = 0.f, br = 0.f;
   if (!gate_fixed) {
-    load4<float>(gate_w + ql * 4, ws4);
-    load4<float>(gate_w + d + ql * 4, wr4);
+    load_el<float, EL>(gate_w + ql * EL, ws8);
+    load_el<float, EL>(gate_w + d + ql * EL, wr8);
     bs = gate_b[0];
     br = gate_b[1];
   }
@@ -327,7 +388,7 @@ race_fuse_fwd_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q,
     const bool valid = r < rows;
     const int64_t rr = valid ? r : rows - 1;
     const int64_t bh = rr / N;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     int ctot = 0;
     for (int t0 = 0; t0 < L; t0 += QL) {
       const int mycode = t0 + ql < L ? (int)rcode_q[rr * L + t0 + ql] : 0;
@@ -336,25 +397,24 @@ race_fuse_fwd_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q,
 #pragma unroll 8
       for (int t = 0; t < nt; ++t) {
         const int b = __shfl_sync(0xffffffffu, mycode, gbase + t);
-        const float4 v = *reinterpret_cast<const float4*>(
-            sums + ((bh * L + t0 + t) * NB + b) * d + ql * 4);
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        acc_row(acc, tables + ((bh * L + t0 + t) * NB + b) * d + ql * EL);
       }
     }
     ctot = group_sum_i<QL>(ctot);
     const float inv = ctot > 0 ? 1.0f / (float)ctot : 0.f;
-    const size_t base = (size_t)rr * d + ql * 4;
-    float qv[4], os[4];
-    load4<T>(q + base, qv);
-    load4<T>(o_sp + base, os);
-    const float orc[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+    const size_t base = (size_t)rr * d + ql * EL;
+    float qv[EL], os[EL], orc[EL];
+    load_el<T, EL>(q + base, qv);
+    load_el<T, EL>(o_sp + base, os);
+#pragma unroll
+    for (int i = 0; i < EL; ++i) orc[i] = acc[i] * inv;
     float gs = gs_fixed, gr = gr_fixed;
     if (!gate_fixed) {
       float as = 0.f, ar = 0.f;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        as += qv[i] * ws4[i];
-        ar += qv[i] * wr4[i];
+      for (int i = 0; i < EL; ++i) {
+        as += qv[i] * ws8[i];
+        ar += qv[i] * wr8[i];
       }
       as = group_sum<QL>(as) + bs;
       ar = group_sum<QL>(ar) + br;
@@ -365,14 +425,21 @@ race_fuse_fwd_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q,
     const float lz = lam_v * (float)ctot / (float)L;
     const float m = lz > 0.f ? 1.0f / (1.0f + expf(logf(lz) - lse[rr])) : 1.0f;
     if (valid) {
-      float yv[4];
+      float yv[EL];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) yv[i] = gs * m * os[i] + gr * orc[i];
-      store4<T>(y + base, yv);
-      if (o_race) store4<T>(o_race + base, orc);
+      for (int i = 0; i < EL; ++i) yv[i] = gs * m * os[i] + gr * orc[i];
+      store_el<T, EL>(y + base, yv);
+      if (o_race) store_el<T, EL>(o_race + base, orc);
       if (ctot_out && ql == 0) ctot_out[rr] = ctot;
     }
   }
+}
+
+__global__ void to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+                               int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    dst[i] = __float2bfloat16_rn(src[i]);
 }
 
 int grid_for_rows(int64_t rows, int warps_per_block) {
@@ -414,11 +481,14 @@ BuildShape build_shape(const Geometry& g) {
 
 template <typename TV, typename CodeT>
 cudaError_t build(const Geometry& g, const void* codes, const void* vals, const float* absmax,
-                  float* sums, int32_t* counts, uint32_t* err, cudaStream_t s) {
+                  float* sums, bool keep_sums, __nv_bfloat16* gtab, int32_t* counts,
+                  uint32_t* err, cudaStream_t s) {
   const BuildShape b = build_shape(g);
   if (b.nt < 1) {
-    // tables too large for shared memory even one at a time: global atomics
-    cudaError_t e = cudaMemsetAsync(sums, 0, (size_t)g.BH * g.L * g.NB * g.d * 4, s);
+    // tables too large for shared memory even one at a time: global fp32
+    // atomics into `sums`, then the bf16 copy
+    const size_t n = (size_t)g.BH * g.L * g.NB * g.d;
+    cudaError_t e = cudaMemsetAsync(sums, 0, n * 4, s);
     if (e != cudaSuccess) return e;
     if (counts) {
       e = cudaMemsetAsync(counts, 0, (size_t)g.BH * g.L * g.NB * 4, s);
@@ -428,6 +498,7 @@ cudaError_t build(const Geometry& g, const void* codes, const void* vals, const 
     race_build_global_kernel<TV, CodeT><<<grid_for_rows(rows, 8), 256, 0, s>>>(
         static_cast<const CodeT*>(codes), static_cast<const TV*>(vals), rows, g.N, g.L, g.NB,
         g.d, sums, counts);
+    if (gtab) to_bf16_kernel<<<148 * 8, 256, 0, s>>>(sums, gtab, (int64_t)n);
     return cudaGetLastError();
   }
   cudaError_t e = cudaFuncSetAttribute(race_build_tiled_kernel<TV, CodeT>,
@@ -436,40 +507,45 @@ cudaError_t build(const Geometry& g, const void* codes, const void* vals, const 
   const dim3 grid(b.groups * b.nds, g.BH);
   race_build_tiled_kernel<TV, CodeT><<<grid, kBuildThreads, b.smem, s>>>(
       static_cast<const CodeT*>(codes), static_cast<const TV*>(vals), g.N, g.L, g.NB, g.d, b.nt,
-      b.ntp, absmax, sums, counts, err);
+      b.ntp, absmax, keep_sums ? sums : nullptr, gtab, counts, err);
   return cudaGetLastError();
 }
 
-template <typename CodeT>
-cudaError_t gather_sum(const Geometry& g, const void* codes, const float* tables, float* out,
+template <typename TT, typename CodeT>
+cudaError_t gather_sum(const Geometry& g, const void* codes, const TT* tables, float* out,
                        cudaStream_t s) {
+  constexpr int EL = 16 / sizeof(TT);
   const int64_t rows = (int64_t)g.BH * g.N;
-  const int grid = grid_for_rows((rows * g.d / 4 + 31) / 32, 8);
+  const int grid = grid_for_rows((rows * g.d / EL + 31) / 32, 8);
   const CodeT* c = static_cast<const CodeT*>(codes);
-  switch (g.d) {
-    case 32: race_gather_sum_kernel<CodeT, 8><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
-    case 64: race_gather_sum_kernel<CodeT, 16><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
-    default: race_gather_sum_kernel<CodeT, 32><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
+  switch (g.d / EL) {
+    case 4: race_gather_sum_kernel<TT, CodeT, 4><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
+    case 8: race_gather_sum_kernel<TT, CodeT, 8><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
+    case 16: race_gather_sum_kernel<TT, CodeT, 16><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
+    default: race_gather_sum_kernel<TT, CodeT, 32><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
   }
   return cudaGetLastError();
 }
 
 template <typename T, typename CodeT>
-cudaError_t fuse_fwd(const Geometry& g, const void* q, const void* rcode_q, const float* sums,
-                     const int32_t* counts, const void* o_sp, const float* lse,
-                     const float* gate_w, const float* gate_b, const float* lam, void* y,
-                     void* o_race, int32_t* ctot, cudaStream_t s, int gate_fixed, float gs,
+cudaError_t fuse_fwd(const Geometry& g, const void* q, const void* rcode_q,
+                     const void* tables, const int32_t* counts, const void* o_sp,
+                     const float* lse, const float* gate_w, const float* gate_b, const float* lam,
+                     void* y, void* o_race, int32_t* ctot, cudaStream_t s, int gate_fixed, float gs,
                      float gr) {
+  constexpr int EL = 16 / sizeof(T);
   const int64_t rows = (int64_t)g.BH * g.N;
-  const int grid = grid_for_rows((rows * g.d / 4 + 31) / 32, 8);
-#define ELSAA_FUSE(VEC)                                                                        \
-  race_fuse_fwd_kernel<T, CodeT, VEC><<<grid, 256, 0, s>>>(                                    \
-      static_cast<const T*>(q), static_cast<const CodeT*>(rcode_q), sums, counts,              \
+  const int grid = grid_for_rows((rows * g.d / EL + 31) / 32, 8);
+#define ELSAA_FUSE(QL)                                                                         \
+  race_fuse_fwd_kernel<T, CodeT, QL><<<grid, 256, 0, s>>>(                                     \
+      static_cast<const T*>(q), static_cast<const CodeT*>(rcode_q),                            \
+      static_cast<const T*>(tables), counts,                                                    \
       static_cast<const T*>(o_sp), lse, gate_w, gate_b, gate_fixed, gs, gr, lam, rows, g.N,    \
       g.L, g.NB, g.d, static_cast<T*>(y), static_cast<T*>(o_race), ctot)
-  switch (g.d) {
-    case 32: ELSAA_FUSE(8); break;
-    case 64: ELSAA_FUSE(16); break;
+  switch (g.d / EL) {
+    case 4: ELSAA_FUSE(4); break;
+    case 8: ELSAA_FUSE(8); break;
+    case 16: ELSAA_FUSE(16); break;
     default: ELSAA_FUSE(32); break;
   }
 #undef ELSAA_FUSE
@@ -495,41 +571,51 @@ cudaError_t launch_unit_absmax(const Geometry& g, const void* vals, bool vals_f3
 }
 
 cudaError_t launch_race_build(const Geometry& g, const void* codes, const void* vals,
-                              bool vals_f32, const float* absmax, float* sums, int32_t* counts,
-                              uint32_t* err, cudaStream_t s) {
+                              bool vals_f32, const float* absmax, float* sums, bool keep_sums,
+                              __nv_bfloat16* gtab, int32_t* counts, uint32_t* err,
+                              cudaStream_t s) {
   if (vals_f32 || !g.bf16)
     return g.rcode_bytes == 1
-               ? build<float, uint8_t>(g, codes, vals, absmax, sums, counts, err, s)
-               : build<float, uint16_t>(g, codes, vals, absmax, sums, counts, err, s);
+               ? build<float, uint8_t>(g, codes, vals, absmax, sums, keep_sums, gtab, counts, err, s)
+               : build<float, uint16_t>(g, codes, vals, absmax, sums, keep_sums, gtab, counts, err,
+                                        s);
   return g.rcode_bytes == 1
-             ? build<__nv_bfloat16, uint8_t>(g, codes, vals, absmax, sums, counts, err, s)
-             : build<__nv_bfloat16, uint16_t>(g, codes, vals, absmax, sums, counts, err, s);
+             ? build<__nv_bfloat16, uint8_t>(g, codes, vals, absmax, sums, keep_sums, gtab, counts,
+                                             err, s)
+             : build<__nv_bfloat16, uint16_t>(g, codes, vals, absmax, sums, keep_sums, gtab,
+                                              counts, err, s);
 }
 
-cudaError_t launch_race_gather_sum(const Geometry& g, const void* codes, const float* tables,
+cudaError_t launch_race_gather_sum(const Geometry& g, const void* codes, const void* tables,
                                    float* out, cudaStream_t s) {
-  return g.rcode_bytes == 1 ? gather_sum<uint8_t>(g, codes, tables, out, s)
-                            : gather_sum<uint16_t>(g, codes, tables, out, s);
+  if (g.bf16) {
+    const __nv_bfloat16* t = static_cast<const __nv_bfloat16*>(tables);
+    return g.rcode_bytes == 1 ? gather_sum<__nv_bfloat16, uint8_t>(g, codes, t, out, s)
+                              : gather_sum<__nv_bfloat16, uint16_t>(g, codes, t, out, s);
+  }
+  const float* t = static_cast<const float*>(tables);
+  return g.rcode_bytes == 1 ? gather_sum<float, uint8_t>(g, codes, t, out, s)
+                            : gather_sum<float, uint16_t>(g, codes, t, out, s);
 }
 
 cudaError_t launch_race_fuse_fwd(const Geometry& g, const void* q, const void* rcode_q,
-                                 const float* sums, const int32_t* counts, const void* o_sp,
-                                 const float* lse, const float* gate_w, const float* gate_b,
-                                 const float* lam, void* y, void* o_race, int32_t* ctot,
-                                 cudaStream_t s) {
+                                 const void* tables, const int32_t* counts,
+                                 const void* o_sp, const float* lse, const float* gate_w,
+                                 const float* gate_b, const float* lam, void* y, void* o_race,
+                                 int32_t* ctot, cudaStream_t s) {
   const float gs = g.gate_s, gr = g.gate_r;
   const int fixed = g.gate_fixed;
   if (g.bf16)
     return g.rcode_bytes == 1
-               ? fuse_fwd<__nv_bfloat16, uint8_t>(g, q, rcode_q, sums, counts, o_sp, lse, gate_w,
+               ? fuse_fwd<__nv_bfloat16, uint8_t>(g, q, rcode_q, tables, counts, o_sp, lse, gate_w,
                                                   gate_b, lam, y, o_race, ctot, s, fixed, gs, gr)
-               : fuse_fwd<__nv_bfloat16, uint16_t>(g, q, rcode_q, sums, counts, o_sp, lse,
+               : fuse_fwd<__nv_bfloat16, uint16_t>(g, q, rcode_q, tables, counts, o_sp, lse,
                                                    gate_w, gate_b, lam, y, o_race, ctot, s, fixed,
                                                    gs, gr);
   return g.rcode_bytes == 1
-             ? fuse_fwd<float, uint8_t>(g, q, rcode_q, sums, counts, o_sp, lse, gate_w, gate_b,
+             ? fuse_fwd<float, uint8_t>(g, q, rcode_q, tables, counts, o_sp, lse, gate_w, gate_b,
                                         lam, y, o_race, ctot, s, fixed, gs, gr)
-             : fuse_fwd<float, uint16_t>(g, q, rcode_q, sums, counts, o_sp, lse, gate_w, gate_b,
+             : fuse_fwd<float, uint16_t>(g, q, rcode_q, tables, counts, o_sp, lse, gate_w, gate_b,
                                          lam, y, o_race, ctot, s, fixed, gs, gr);
 }
 

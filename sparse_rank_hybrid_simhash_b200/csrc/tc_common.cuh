@@ -63,6 +63,10 @@ ELSAA_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+ELSAA_DEV void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // Waits for the phase with the given parity to complete; gives up after
 // kMaxSpin polls, records ERR_TIMEOUT and returns false.
 ELSAA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
