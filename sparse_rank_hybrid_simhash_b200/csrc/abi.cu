@@ -302,7 +302,12 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
                                    dv_acc, s));
   ELSAA_TRY(mark(events, 2, s));
   // 3. sparse branch backward, 4. outputs
-  if (g.tc_attn) {
+  if (g.tc_attn && attn_bwd2_supported(g)) {
+    ELSAA_TRY(launch_attn_bwd2(g, q, k, v, perm, perm + bhn, d_o, lse, dprime, dv_acc, dq_acc,
+                               dk, dv, (uint32_t*)(w + wl.err), s));
+    ELSAA_TRY(mark(events, 3, s));
+    ELSAA_TRY(launch_cast_out(g, dq_acc, dq, s));
+  } else if (g.tc_attn) {
     ELSAA_TRY(launch_attn_bwd_tc(g, q, k, v, perm, perm + bhn, d_o, lse, dprime, dv_acc, dq_acc,
                                  dk, dv, (uint32_t*)(w + wl.err), s));
     ELSAA_TRY(mark(events, 3, s));

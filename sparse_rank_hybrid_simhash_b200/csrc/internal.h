@@ -114,6 +114,12 @@ cudaError_t launch_attn_fwd_tc(const Geometry& g, const void* q, const void* k, 
                                const int32_t* perm_q, const int32_t* perm_k, void* o_sp,
                                float* lse, uint32_t* err, cudaStream_t s);
 bool attn_tc_supported(const Geometry& g);
+// Overlapped backward (d = 64, chunk 64 or 128).
+bool attn_bwd2_supported(const Geometry& g);
+cudaError_t launch_attn_bwd2(const Geometry& g, const void* q, const void* k, const void* v,
+                             const int32_t* perm_q, const int32_t* perm_k, const void* d_o,
+                             const float* lse, const float* dprime, const float* dv_race,
+                             float* dq_acc, void* dk, void* dv, uint32_t* err, cudaStream_t s);
 // Persistent warp-specialized forward (d = 64, chunk <= 128 dividing 128).
 bool attn_pipe_supported(const Geometry& g);
 cudaError_t launch_attn_fwd_pipe(const Geometry& g, const void* q, const void* k, const void* v,

@@ -192,6 +192,166 @@ race_build_tiled_kernel(const CodeT* __restrict__ codes, const TV* __restrict__ 
       counts[((size_t)bh * L + l0) * NB + i] = cnt[i];
 }
 
+// The same build with the key stream as a 4-stage cp.async pipeline: tiles of
+// kPipeKT keys (raw values of the CTA's d-slice and the codes of its tables)
+// land in a ring of shared-memory stages while earlier tiles are reduced, with
+// one barrier per tile.  Keys past N are zero-filled and add nothing.  Needs
+// the codes of a CTA's tables to be 4-byte aligned per key.
+constexpr int kPipeKT = 128;
+constexpr int kPipeStages = 4;
+
+ELSAA_DEV void cp_async4(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+ELSAA_DEV void cp_async16b(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+
+// NT > 0 fixes the tables per CTA at compile time (unrolled, table bases hoisted).
+template <typename TV, typename CodeT, int NT>
+__global__ void __launch_bounds__(kBuildThreads)
+race_build_pipe_kernel(const CodeT* __restrict__ codes, const TV* __restrict__ vals, int N,
+                       int L, int NB, int d, int nt_max, const float* __restrict__ absmax,
+                       float* __restrict__ sums, __nv_bfloat16* __restrict__ gtab,
+                       int32_t* __restrict__ counts, uint32_t* __restrict__ err) {
+  constexpr int VB = kDsl * (int)sizeof(TV);   // value bytes of one key's d-slice
+  extern __shared__ int32_t smi[];
+  __shared__ int s_cmax;
+  const int tid = threadIdx.x;
+  const int bh = blockIdx.y;
+  const int nds = d / kDsl;
+  const int tg = blockIdx.x / nds, dsl = blockIdx.x % nds;
+  const int l0 = tg * nt_max, nt = min(L, l0 + nt_max) - l0;
+  const int d0 = dsl * kDsl;
+  const int CB = nt_max * (int)sizeof(CodeT);    // code bytes of one key (multiple of 4)
+  int32_t* tab = smi;                                              // [nt_max][NB][32]
+  int32_t* cnt = tab + (size_t)nt_max * NB * kDsl;                 // [nt_max][NB]
+  uint8_t* stages = reinterpret_cast<uint8_t*>(cnt + (((size_t)nt_max * NB + 3) & ~(size_t)3));
+  const int stage_bytes = kPipeKT * (VB + CB);
+  for (int i = tid; i < nt * NB * kDsl; i += kBuildThreads) tab[i] = 0;
+  for (int i = tid; i < nt * NB; i += kBuildThreads) cnt[i] = 0;
+  if (tid == 0) s_cmax = 0;
+  __syncthreads();
+  const CodeT* cb = codes + (size_t)bh * N * L + l0;
+  const TV* vb = vals + (size_t)bh * N * d + d0;
+
+  // pass 1: bucket counts of this CTA's tables (one thread per key)
+  for (int key = tid; key < N; key += kBuildThreads) {
+    const CodeT* kc = cb + (size_t)key * L;
+    for (int t = 0; t < nt; ++t) atomicAdd(cnt + t * NB + (int)kc[t], 1);
+  }
+  __syncthreads();
+  int cm = 0;
+  for (int i = tid; i < nt * NB; i += kBuildThreads) cm = max(cm, cnt[i]);
+  atomicMax(&s_cmax, cm);
+  __syncthreads();
+  const float vmax = absmax[bh];
+  if (!(vmax < 3.0e38f)) {
+    if (tid == 0) raise_error(err, ERR_CHECK);
+    return;
+  }
+  int S = 100;
+  if (s_cmax > 0 && vmax > 0.f) {
+    S = (int)floorf(log2f(2147483000.0f / ((float)s_cmax * vmax))) - 1;
+    S = max(-100, min(100, S));
+  }
+  const float scale = ldexpf(1.0f, S), inv_scale = ldexpf(1.0f, -S);
+
+  // pass 2: fixed-point sums over a cp.async ring of key tiles
+  const uint32_t st0 = smem_addr32(stages);
+  const int ntiles = (N + kPipeKT - 1) / kPipeKT;
+  auto issue = [&](int tile, int slot) {
+    const int k0 = tile * kPipeKT;
+    const uint32_t sv = st0 + slot * stage_bytes;
+    for (int c = tid; c < kPipeKT * (VB / 16); c += kBuildThreads) {
+      const int key = c / (VB / 16), part = c % (VB / 16);
+      const int j = k0 + key;
+      const bool in = j < N;
+      cp_async16b(sv + key * VB + part * 16,
+                  vb + (size_t)(in ? j : 0) * d + part * (16 / (int)sizeof(TV)), in ? 16 : 0);
+    }
+    for (int c = tid; c < kPipeKT * (CB / 4); c += kBuildThreads) {
+      const int key = c / (CB / 4), part = c % (CB / 4);
+      const int j = k0 + key;
+      const bool in = j < N;
+      cp_async4(sv + kPipeKT * VB + key * CB + part * 4,
+                reinterpret_cast<const uint8_t*>(cb + (size_t)(in ? j : 0) * L) + part * 4,
+                in ? 4 : 0);
+    }
+  };
+  for (int t = 0; t < kPipeStages - 1; ++t) {
+    if (t < ntiles) issue(t, t);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  const int w = tid >> 5, lane = tid & 31;
+  const uint32_t tab_lane = smem_addr32(tab) + lane * 4;
+  const uint32_t table_bytes = (uint32_t)NB * kDsl * 4;
+  for (int t = 0; t < ntiles; ++t) {
+    asm volatile("cp.async.wait_group %0;" ::"n"(kPipeStages - 2) : "memory");
+    __syncthreads();   // tile t is in; every thread is done with tile t - 1
+    {
+      const int tn = t + kPipeStages - 1;
+      if (tn < ntiles) issue(tn, tn % kPipeStages);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    const uint8_t* sv = stages + (t % kPipeStages) * stage_bytes;
+    // warp w: keys w and w + 32 of each 64-key half, two keys in flight
+    for (int key = w; key < kPipeKT; key += 2 * (kBuildThreads / 32)) {
+      const int key2 = key + kBuildThreads / 32;
+      const float xa = to_f32(reinterpret_cast<const TV*>(sv + key * VB)[lane]);
+      const float xb = to_f32(reinterpret_cast<const TV*>(sv + key2 * VB)[lane]);
+      const uint32_t qa = (uint32_t)__float2int_rn(xa * scale);
+      const uint32_t qb = (uint32_t)__float2int_rn(xb * scale);
+      // codes in 32-bit words: 4 u8 codes or 2 u16 codes per load; a code is
+      // pulled out with one byte permute and scaled into an address with one
+      // multiply-add
+      constexpr int PER = 4 / (int)sizeof(CodeT);
+      const uint32_t* ka = reinterpret_cast<const uint32_t*>(sv + kPipeKT * VB + key * CB);
+      const uint32_t* kb2 = reinterpret_cast<const uint32_t*>(sv + kPipeKT * VB + key2 * CB);
+      if constexpr (NT > 0) {
+#pragma unroll
+        for (int tw = 0; tw < NT; tw += PER) {
+          const uint32_t wa = ka[tw / PER], wb = kb2[tw / PER];
+#pragma unroll
+          for (int e = 0; e < PER; ++e) {
+            const uint32_t sel = sizeof(CodeT) == 1 ? (0x4440u | e) : (e ? 0x4432u : 0x4410u);
+            const uint32_t tb = tab_lane + (uint32_t)(tw + e) * table_bytes;
+            red_shared_add_u32(tb + __byte_perm(wa, 0, sel) * (kDsl * 4), qa);
+            red_shared_add_u32(tb + __byte_perm(wb, 0, sel) * (kDsl * 4), qb);
+          }
+        }
+      } else {
+        uint32_t tbase = tab_lane;
+        for (int tw = 0; tw < nt; tw += PER) {   // nt is a multiple of PER
+          const uint32_t wa = ka[tw / PER], wb = kb2[tw / PER];
+#pragma unroll
+          for (int e = 0; e < PER; ++e, tbase += table_bytes) {
+            const uint32_t sel = sizeof(CodeT) == 1 ? (0x4440u | e) : (e ? 0x4432u : 0x4410u);
+            red_shared_add_u32(tbase + __byte_perm(wa, 0, sel) * (kDsl * 4), qa);
+            red_shared_add_u32(tbase + __byte_perm(wb, 0, sel) * (kDsl * 4), qb);
+          }
+        }
+      }
+    }
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+  for (int i = tid; i < nt * NB * kDsl; i += kBuildThreads) {
+    const int tb = i / kDsl, e = i % kDsl;
+    const size_t o = ((size_t)bh * L + l0) * NB * d + (size_t)tb * d + d0 + e;
+    const float val = (float)tab[i] * inv_scale;
+    if (sums) sums[o] = val;
+    if (gtab) gtab[o] = __float2bfloat16_rn(val);
+  }
+  if (counts != nullptr && dsl == 0)
+    for (int i = tid; i < nt * NB; i += kBuildThreads)
+      counts[((size_t)bh * L + l0) * NB + i] = cnt[i];
+}
+
 // Largest |value| of every unit (an upper bound for the fixed-point scale):
 // absmax must be zeroed; non-negative floats order like their bit patterns.
 template <typename TV>
@@ -500,6 +660,41 @@ cudaError_t build(const Geometry& g, const void* codes, const void* vals, const 
         g.d, sums, counts);
     if (gtab) to_bf16_kernel<<<148 * 8, 256, 0, s>>>(sums, gtab, (int64_t)n);
     return cudaGetLastError();
+  }
+  // pipelined variant: tables per CTA dividing L, codes 4-byte aligned per key
+  if ((g.L * (int)sizeof(CodeT)) % 4 == 0) {
+    const int esz_v = (int)sizeof(TV), rb = (int)sizeof(CodeT), step = 4 / rb;
+    auto smem_for = [&](int nt) {
+      return (size_t)nt * g.NB * kDsl * 4 + (((size_t)nt * g.NB + 3) & ~(size_t)3) * 4 +
+             (size_t)kPipeStages * kPipeKT * (kDsl * esz_v + nt * rb) + 16;
+    };
+    int best = 0;
+    long long best_cost = -1;
+    for (int nt = step; nt <= g.L && smem_for(nt) <= (size_t)kBuildSmemBudget; nt += step) {
+      if (g.L % nt != 0) continue;
+      const long long ctas = (long long)(g.L / nt) * b.nds * g.BH;
+      const long long cost = (ctas + 147) / 148 * (2 * nt + 1);
+      if (best_cost < 0 || cost <= best_cost) {
+        best_cost = cost;
+        best = nt;
+      }
+    }
+    if (best > 0) {
+      const size_t smem = smem_for(best);
+      const dim3 grid(g.L / best * b.nds, g.BH);
+      auto go = [&](auto kernel) -> cudaError_t {
+        cudaError_t e =
+            cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kernel<<<grid, kBuildThreads, smem, s>>>(
+            static_cast<const CodeT*>(codes), static_cast<const TV*>(vals), g.N, g.L, g.NB, g.d,
+            best, absmax, keep_sums ? sums : nullptr, gtab, counts, err);
+        return cudaGetLastError();
+      };
+      if (best == 4) return go(race_build_pipe_kernel<TV, CodeT, 4>);
+      if (best == 8) return go(race_build_pipe_kernel<TV, CodeT, 8>);
+      return go(race_build_pipe_kernel<TV, CodeT, 0>);
+    }
   }
   cudaError_t e = cudaFuncSetAttribute(race_build_tiled_kernel<TV, CodeT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)b.smem);
