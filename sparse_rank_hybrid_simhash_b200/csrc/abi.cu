@@ -88,7 +88,7 @@ WorkLayout work_layout(const Geometry& g) {
   w.dq_acc = take(bhn * g.d * 4);
   w.dk_acc = take(bhn * g.d * 4);
   w.dv_acc = take(bhn * g.d * 4);
-  w.dor = take(bhn * g.d * 4);
+  w.dor = take(bhn * g.d * g.esz);
   w.d_t = take((size_t)g.BH * g.L * g.NB * g.d * 4);
   w.partials = take((size_t)kParamBlocks * (2 * g.d + 3) * 4);
   w.total = off > fwd_end ? off : fwd_end;
@@ -283,7 +283,7 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
   float* dq_acc = (float*)(w + wl.dq_acc);
   float* dk_acc = (float*)(w + wl.dk_acc);
   float* dv_acc = (float*)(w + wl.dv_acc);
-  float* dor = (float*)(w + wl.dor);
+  void* dor = w + wl.dor;
   float* d_t = (float*)(w + wl.d_t);
   float* partials = (float*)(w + wl.partials);
   ELSAA_TRY(cudaMemsetAsync(w + wl.err, 0, sizeof(uint32_t), s));
@@ -296,7 +296,7 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
   ELSAA_TRY(mark(events, 1, s));
   // 2. RACE backward: scatter into the table gradient by query code, gather by key code
   __nv_bfloat16* gtab = g.bf16 ? (__nv_bfloat16*)(w + wl.gtab) : nullptr;
-  ELSAA_TRY(launch_race_build(g, rcode, dor, true, absmax, d_t, !g.bf16, gtab, nullptr,
+  ELSAA_TRY(launch_race_build(g, rcode, dor, false, absmax, d_t, !g.bf16, gtab, nullptr,
                               (uint32_t*)(w + wl.err), s));
   ELSAA_TRY(launch_race_gather_sum(g, rcode_k, g.bf16 ? (const void*)gtab : (const void*)d_t,
                                    dv_acc, s));

@@ -67,14 +67,14 @@ ELSAA_DEV float gsum(float v) {
 // QL = d / 4 lanes per query (4 consecutive values each, 16-byte accesses),
 // 32 / QL queries per warp.
 template <typename T, int QL>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __restrict__ o_sp,
                 const T* __restrict__ o_race, const float* __restrict__ lse,
                 const int32_t* __restrict__ ctot, const float* __restrict__ gate_w,
                 const float* __restrict__ gate_b, int gate_fixed, float gs_fixed, float gr_fixed,
                 const float* __restrict__ lam, int64_t rows, int N, int L, int d,
                 T* __restrict__ d_o, float* __restrict__ dprime, float* __restrict__ dq_acc,
-                float* __restrict__ dor, float* __restrict__ absmax, float* __restrict__ partials) {
+                T* __restrict__ dor, float* __restrict__ absmax, float* __restrict__ partials) {
   constexpr int QW = 32 / QL;
   __shared__ float red[8][2 * 128 + 3];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
@@ -149,7 +149,7 @@ fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __re
     if (valid) {
       st4_round<T>(d_o + base, dov);   // dov now holds the stored (rounded) values
       *reinterpret_cast<float4*>(dq_acc + base) = make_float4(dqv[0], dqv[1], dqv[2], dqv[3]);
-      *reinterpret_cast<float4*>(dor + base) = make_float4(drv[0], drv[1], drv[2], drv[3]);
+      st4_round<T>(dor + base, drv);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         dd += dov[i] * os[i];
@@ -236,7 +236,7 @@ template <typename T>
 cudaError_t fuse_bwd(const Geometry& g, const void* q, const void* dy, const void* o_sp,
                      const void* o_race, const float* lse, const int32_t* ctot,
                      const float* gate_w, const float* gate_b, const float* lam, void* d_o,
-                     float* dprime, float* dq_acc, float* dor, float* absmax, float* partials,
+                     float* dprime, float* dq_acc, void* dor, float* absmax, float* partials,
                      cudaStream_t s) {
   const int64_t rows = (int64_t)g.BH * g.N;
   cudaError_t e = cudaMemsetAsync(absmax, 0, (size_t)g.BH * sizeof(float), s);
@@ -245,7 +245,8 @@ cudaError_t fuse_bwd(const Geometry& g, const void* q, const void* dy, const voi
   fuse_bwd_kernel<T, VEC><<<kParamBlocks, 256, 0, s>>>(                                        \
       static_cast<const T*>(q), static_cast<const T*>(dy), static_cast<const T*>(o_sp),        \
       static_cast<const T*>(o_race), lse, ctot, gate_w, gate_b, g.gate_fixed, g.gate_s,        \
-      g.gate_r, lam, rows, g.N, g.L, g.d, static_cast<T*>(d_o), dprime, dq_acc, dor, absmax,  \
+      g.gate_r, lam, rows, g.N, g.L, g.d, static_cast<T*>(d_o), dprime, dq_acc,               \
+      static_cast<T*>(dor), absmax,                                                            \
       partials)
   switch (g.d) {
     case 32: ELSAA_FB(8); break;
@@ -261,7 +262,7 @@ cudaError_t fuse_bwd(const Geometry& g, const void* q, const void* dy, const voi
 cudaError_t launch_fuse_bwd(const Geometry& g, const void* q, const void* dy, const void* o_sp,
                             const void* o_race, const float* lse, const int32_t* ctot,
                             const float* gate_w, const float* gate_b, const float* lam,
-                            void* d_o, float* dprime, float* dq_acc, float* dor,
+                            void* d_o, float* dprime, float* dq_acc, void* dor,
                             float* absmax, float* partials, cudaStream_t s) {
   return g.bf16 ? fuse_bwd<__nv_bfloat16>(g, q, dy, o_sp, o_race, lse, ctot, gate_w, gate_b, lam,
                                           d_o, dprime, dq_acc, dor, absmax, partials, s)

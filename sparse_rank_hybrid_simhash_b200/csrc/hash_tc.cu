@@ -34,7 +34,7 @@ constexpr int kSmemLimit = 227 * 1024;
 
 struct HashShape {
   int P, P16, nbuf;
-  uint32_t r_bytes, a_bytes, dyn;
+  uint32_t r_bytes, a_bytes, code_bytes, dyn;
 };
 
 HashShape hash_shape(const Geometry& g) {
@@ -43,8 +43,10 @@ HashShape hash_shape(const Geometry& g) {
   h.P16 = (h.P + 15) / 16 * 16;
   h.r_bytes = (uint32_t)h.P16 * g.d * 2;
   h.a_bytes = (uint32_t)kTile * g.d * 2;
-  h.nbuf = (h.r_bytes + 2 * h.a_bytes + 64 <= (uint32_t)kSmemLimit) ? 2 : 1;
-  h.dyn = h.r_bytes + h.nbuf * h.a_bytes + 64;
+  // per-tile staging of the codes: 128 sort codes (u16) then 128 rows of L RACE codes
+  h.code_bytes = (uint32_t)((kTile * 2 + kTile * g.L * g.rcode_bytes + 15) / 16 * 16);
+  h.nbuf = (h.r_bytes + 2 * h.a_bytes + h.code_bytes + 64 <= (uint32_t)kSmemLimit) ? 2 : 1;
+  h.dyn = h.r_bytes + h.nbuf * h.a_bytes + h.code_bytes + 64;
   return h;
 }
 
@@ -75,7 +77,13 @@ hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
   const uint32_t r_bytes = (uint32_t)P16 * D * 2;
   const uint32_t a_bytes = kTile * D * 2;
   const uint32_t s_r = sbase, s_a = sbase + r_bytes;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + r_bytes + nbuf * a_bytes);
+  // code staging: the tile's sort codes, then its rows of RACE codes, written
+  // to global memory as one contiguous block per tile
+  uint16_t* st_code = reinterpret_cast<uint16_t*>(smem + r_bytes + nbuf * a_bytes);
+  CodeT* st_rcode = reinterpret_cast<CodeT*>(st_code + kTile);
+  const uint32_t code_bytes =
+      (uint32_t)((kTile * 2 + kTile * L * (int)sizeof(CodeT) + 15) / 16 * 16);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + r_bytes + nbuf * a_bytes + code_bytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
   const int tid = threadIdx.x, warp = tid >> 5;
   if ((sbase & 1023u) != 0) {   // the swizzled tiles need a 1024-byte aligned base
@@ -130,8 +138,6 @@ hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     }
     fence_async_smem();
     __syncthreads();
-    const int64_t row = tile * kTile + tid;
-    const bool row_ok = row < 2 * rows_per_tensor;
     uint64_t acc = 0;
     int nacc = 0, slot = 0;
     for (int p = 0; p < npass; ++p) {
@@ -170,10 +176,8 @@ hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
           const uint32_t val = (uint32_t)(acc & ((1ull << bits) - 1ull));
           acc >>= bits;
           nacc -= bits;
-          if (row_ok) {
-            if (slot == 0) code[row] = (uint16_t)val;
-            else rcode[row * L + slot - 1] = (CodeT)val;
-          }
+          if (slot == 0) st_code[tid] = (uint16_t)val;
+          else st_rcode[tid * L + slot - 1] = (CodeT)val;
           ++slot;
         }
       }
@@ -183,11 +187,23 @@ hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     if (!ok) break;
     // zero-bit codes at the end of the stream
     while (slot < nslots) {
-      if (row_ok) {
-        if (slot == 0) code[row] = 0;
-        else rcode[row * L + slot - 1] = 0;
-      }
+      if (slot == 0) st_code[tid] = 0;
+      else st_rcode[tid * L + slot - 1] = 0;
       ++slot;
+    }
+    __syncthreads();
+    {
+      // the tile's rows are consecutive: copy its codes as contiguous blocks
+      const int64_t row0 = tile * kTile;
+      const int nrows = (int)min((int64_t)kTile, 2 * rows_per_tensor - row0);
+      const int rbytes = nrows * L * (int)sizeof(CodeT);
+      uint8_t* gdst = reinterpret_cast<uint8_t*>(rcode + row0 * L);
+      const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(st_rcode);
+      const int nvec = rbytes / 16;
+      for (int i = tid; i < nvec; i += kThreads)
+        reinterpret_cast<uint4*>(gdst)[i] = reinterpret_cast<const uint4*>(ssrc)[i];
+      for (int i = nvec * 16 + tid; i < rbytes; i += kThreads) gdst[i] = ssrc[i];
+      for (int i = tid; i < nrows; i += kThreads) code[row0 + i] = st_code[i];
     }
     if (nbuf == 1 && next < tiles) {
       load_tile<D>(s_a, q, k, rows_per_tensor, next);
@@ -210,14 +226,18 @@ cudaError_t run(const Geometry& g, const void* q, const void* k, const void* r_s
   cudaError_t e = cudaFuncSetAttribute(hash_tc_kernel<D, CodeT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)h.dyn);
   if (e != cudaSuccess) return e;
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, hash_tc_kernel<D, CodeT>, kThreads,
-                                                    h.dyn);
+  // let shared memory take the whole carveout so several CTAs fit per SM
+  e = cudaFuncSetAttribute(hash_tc_kernel<D, CodeT>,
+                           cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);   // TMEM: 4 x 128 columns per SM
+  // CTAs per SM: shared memory (228 KB per SM, 1 KB reserved per CTA) and
+  // TMEM (4 x 128 columns)
+  int per_sm = (int)((228u * 1024u) / (h.dyn + 1024u));
+  per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
   const int64_t rows = (int64_t)g.BH * g.N;
   const int64_t tiles = (2 * rows + kTile - 1) / kTile;
   const int64_t want = (int64_t)sms * per_sm;

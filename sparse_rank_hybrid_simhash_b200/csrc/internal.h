@@ -50,13 +50,13 @@ struct WorkLayout {
   size_t d_o;                // [BH][N][d] dtype: dO_sp
   size_t dprime;             // [BH][N] f32: D' = dO_sp . O_sp - dlse
   size_t dq_acc, dk_acc, dv_acc;   // [BH][N][d] f32
-  size_t dor;                // [BH][N][d] f32: g_r dy / Ctot
+  size_t dor;                // [BH][N][d] dtype: g_r dy / Ctot
   size_t d_t;                // [BH][L][NB][d] f32: RACE table gradient
   size_t partials;           // [kParamBlocks][2d+3] f32
   size_t total;
 };
 
-constexpr int kParamBlocks = 592;   // 4 x 148 SMs; fixed so the reduction order is fixed
+constexpr int kParamBlocks = 592;   // one wave of 4 x 148 SMs; fixed so the reduction order is fixed
 
 bool make_geometry(const elsaa_params* p, Geometry* g, elsaa_status* why);
 SavedLayout saved_layout(const Geometry& g);
@@ -137,7 +137,7 @@ cudaError_t launch_attn_bwd_tc(const Geometry& g, const void* q, const void* k, 
 cudaError_t launch_fuse_bwd(const Geometry& g, const void* q, const void* dy, const void* o_sp,
                             const void* o_race, const float* lse, const int32_t* ctot,
                             const float* gate_w, const float* gate_b, const float* lam,
-                            void* d_o, float* dprime, float* dq_acc, float* dor,
+                            void* d_o, float* dprime, float* dq_acc, void* dor,
                             float* absmax, float* partials, cudaStream_t s);
 cudaError_t launch_param_reduce(const Geometry& g, const float* partials, float* dgate_w,
                                 float* dgate_b, float* dlambda, cudaStream_t s);

@@ -452,7 +452,7 @@ ELSAA_DEV void store_el<float, 8>(float* p, const float* v) {
 }
 
 template <typename TT, typename CodeT, int QL>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 race_gather_sum_kernel(const CodeT* __restrict__ codes, const TT* __restrict__ tables,
                        int64_t rows, int N, int L, int NB, int d, float* __restrict__ out) {
   constexpr int QW = 32 / QL, EL = 16 / sizeof(TT);
@@ -468,7 +468,7 @@ race_gather_sum_kernel(const CodeT* __restrict__ codes, const TT* __restrict__ t
     for (int t0 = 0; t0 < L; t0 += QL) {
       const int mycode = t0 + ql < L ? (int)codes[rr * L + t0 + ql] : 0;
       const int nt = min(QL, L - t0);
-#pragma unroll 8
+#pragma unroll 16
       for (int t = 0; t < nt; ++t) {
         const int b = __shfl_sync(0xffffffffu, mycode, gbase + t);
         acc_row(acc, tables + ((bh * L + t0 + t) * NB + b) * d + ql * EL);
@@ -520,7 +520,7 @@ ELSAA_DEV void load_el<float, 4>(const float* p, float* v) {
 
 // T: data type; the tables have the data type too (bf16 copy or fp32 sums).
 template <typename T, typename CodeT, int QL>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 race_fuse_fwd_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q,
                      const T* __restrict__ tables, const int32_t* __restrict__ counts,
                      const T* __restrict__ o_sp, const float* __restrict__ lse,
@@ -554,7 +554,7 @@ race_fuse_fwd_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q,
       const int mycode = t0 + ql < L ? (int)rcode_q[rr * L + t0 + ql] : 0;
       if (t0 + ql < L) ctot += counts[(bh * L + t0 + ql) * NB + mycode];
       const int nt = min(QL, L - t0);
-#pragma unroll 8
+#pragma unroll 16
       for (int t = 0; t < nt; ++t) {
         const int b = __shfl_sync(0xffffffffu, mycode, gbase + t);
         acc_row(acc, tables + ((bh * L + t0 + t) * NB + b) * d + ql * EL);
