@@ -36,6 +36,7 @@ sys.path.insert(0, ROOT)
 import torch  # noqa: E402
 
 from sparse_rank_hybrid_simhash_b200 import binding as B  # noqa: E402
+from sparse_rank_hybrid_simhash_b200 import distributed as DP  # noqa: E402
 from sparse_rank_hybrid_simhash_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "ELSAA attn tokens/s fwd and fwd+bwd at N=32K,d=64 bf16; % of roofline"
@@ -167,7 +168,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     w = WORKLOADS[args.workload]
     p = B.Params.from_workload(w)
-    inp = make_inputs(w, seed=w.seed + rank, with_dy=True)
+    inp = make_inputs(w, seed=DP.rank_seed(w.seed, rank), with_dy=True)
     d = {k: t.to(dev) for k, t in inp.items()}
     saved = B.alloc_saved(p, dev)
     ws = B.alloc_workspace(p, dev)
@@ -186,12 +187,7 @@ def run_ours(args, rank, world, local_rank):
         B.backward(p, d["q"], d["k"], d["v"], d["r_sort"], d["r_race"], d["gate_w"],
                    d["gate_b"], d["lam"], saved, d["dy"], *grads, ws=ws, events=ev_b)
         if world > 1:
-            pg = torch.cat([grads[3].view(-1), grads[4].view(-1), grads[5].view(-1)])
-            torch.distributed.all_reduce(pg)
-            n = grads[3].numel()
-            grads[3].view(-1).copy_(pg[:n])
-            grads[4].copy_(pg[n:n + 2])
-            grads[5].copy_(pg[n + 2:])
+            DP.allreduce_param_grads(grads[3], grads[4], grads[5])
 
     for _ in range(args.warmup):
         step()
@@ -224,9 +220,7 @@ def run_ours(args, rank, world, local_rank):
     total_ms = sum(step_ms)
     fwd_total = sum(fwd_ms)
     if world > 1:
-        t = torch.tensor([total_ms, fwd_total], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms, fwd_total = t.tolist()
+        total_ms, fwd_total = DP.max_over_ranks([total_ms, fwd_total], dev)
 
     # end to end through the public API with host buffers
     e2e = run_e2e(args, w, p, inp, dev, world)
@@ -250,9 +244,9 @@ def run_e2e(args, w, p, inp, dev, world):
                       small["gate_w"], small["gate_b"], small["lam"], saved=saved, ws=ws)
         g = B.backward(p, dq["q"], dq["k"], dq["v"], small["r_sort"], small["r_race"],
                        small["gate_w"], small["gate_b"], small["lam"], saved, dq["dy"], ws=ws)
-        pg = torch.cat([g[3].view(-1), g[4].view(-1), g[5].view(-1)])
         if world > 1:
-            torch.distributed.all_reduce(pg)
+            DP.allreduce_param_grads(g[3], g[4], g[5])
+        pg = torch.cat([g[3].view(-1), g[4].view(-1), g[5].view(-1)])
         outs["q"].copy_(g[0], non_blocking=True)
         outs["k"].copy_(g[1], non_blocking=True)
         outs["v"].copy_(g[2], non_blocking=True)
@@ -272,9 +266,7 @@ def run_e2e(args, w, p, inp, dev, world):
     torch.cuda.synchronize()
     ms = start.elapsed_time(end)
     if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = t.item()
+        ms = DP.max_over_ranks([ms], dev)[0]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = sum(t.numel() * t.element_size() for t in outs.values()) + pg_host.numel() * 4
     return {"value": world * n * w.tokens / (ms / 1e3), "unit": "tokens/s",
