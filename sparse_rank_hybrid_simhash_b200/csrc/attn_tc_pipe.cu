@@ -5,25 +5,30 @@
 // section "Two efficient branches can still be mis-scaled") is exact softmax
 // attention over each query's Sort-LSH window: the query at sorted rank r
 // (chunk j = r / c) sees the keys at sorted ranks [max(0,(j-1)c), (j+1)c).
-// A tile of 128 sorted queries starting at r0 sees the keys [r0 - c, r0 + 128)
-// (r0 = 0: [0, 128)), at most 256, so its scores fit in 256 TMEM columns and
-// the softmax is exact in one pass (row max first, then exp).
 //
-// Roles (320 threads, one CTA per SM, tiles strided over the grid):
-//   warp 0      producer: stages the tile's token indices, then gathers the Q,
-//               K and V rows with cp.async into a two-stage ring of
-//               128B-swizzled tiles; completion arrives on full[stage]
+// Work unit: a tile of 128 sorted queries (rank r0 = 128 tb).  Its keys lie in
+// two 128-key blocks of the sorted order: block tb - 1 (only its last c keys
+// are seen; none when tb = 0) and block tb.  Each CTA takes a contiguous run
+// of tiles, so consecutive tiles share a key block: every block is gathered
+// once (plus one extra at the start of the run) and kept in a four-slot ring.
+// Scores fit in 256 TMEM columns (block tb - 1 in [0, 128), block tb in
+// [128, 256)); the softmax is exact in one pass (row max first, then exp).
+//
+// Roles (320 threads, one CTA per SM):
+//   warp 0      producer: token indices (prefetched one tile ahead, held in
+//               registers and broadcast by shuffles), cp.async gathers of Q
+//               tiles (two-slot ring) and K/V blocks (four-slot ring) into
+//               128B-swizzled tiles; completion arrives on full_q / full_kv
 //   warp 1      MMA issuer (one thread) and TMEM owner:
-//                 S = Q K^T            -> TMEM [0, 256)
-//                 O = P V              -> TMEM [256, 320) or [320, 384)
+//                 O(j-1) = P V        as soon as P of tile j-1 is written
+//                 S(j)   = Q K^T      -> TMEM [0, 256)
+//               and releases Q and K/V slots through tcgen05.commit
 //   warps 2..9  softmax and epilogue: warp w reaches TMEM lanes (query rows)
-//               32 (w % 4) .. +31 and takes half of the key columns (warps 2..5
-//               the first half, 6..9 the second); row max and row sum are
-//               combined through shared memory; p = exp2(scale log2e s - m)
-//               (masked to the row's own window when c < 128), P (bf16) to
-//               shared memory, then O / l and the log-mass to the query's
-//               token index
-// Barriers: full/empty per stage, s_full, p_full, o_full/o_free per O buffer.
+//               32 (w % 4) .. +31 and takes one of two column ranges; row max
+//               and row sum are combined through shared memory;
+//               p = exp2(scale log2e s - m) masked to the row's own window,
+//               P (bf16) to shared memory, then O / l and the log-mass to the
+//               query's token index
 // Every wait is bounded; a timeout records ERR_TIMEOUT and every role leaves
 // its loop, frees TMEM and returns.
 #include <math.h>
@@ -38,25 +43,54 @@ using namespace tc;
 
 constexpr int D = 64;
 constexpr int kTile = 128;
-constexpr int kMaxKeys = 256;
 constexpr int kThreads = 320;
 constexpr int kSoftmaxThreads = 256;
+constexpr int kKvSlots = 4;
+constexpr int kQSlots = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTS = 0, kTO = 256;   // S: 256 columns, O: 2 x 64 columns
 
 struct PipeLayout {
-  static constexpr uint32_t kQ = 128 * 128;           // one stage: Q 128 rows
-  static constexpr uint32_t kKV = kMaxKeys * 128;     // K or V: 256 rows
-  static constexpr uint32_t kStage = kQ + 2 * kKV;    // 80 KB
-  static constexpr uint32_t kP = 2 * kStage;          // P: 128 x 256 bf16, 4 sub-tiles of 64 keys
-  static constexpr uint32_t kRed = kP + 4 * 128 * 128;   // row max and sum: [2 halves][128 rows] x2
+  static constexpr uint32_t kTileBytes = 128 * 128;              // 128 rows x 64 bf16
+  static constexpr uint32_t kKv = 0;                             // [4][K | V]
+  static constexpr uint32_t kKvSlot = 2 * kTileBytes;
+  static constexpr uint32_t kQ = kKv + kKvSlots * kKvSlot;       // [2][Q]
+  static constexpr uint32_t kP = kQ + kQSlots * kTileBytes;      // 128 x 256 bf16, 4 sub-tiles
+  static constexpr uint32_t kRed = kP + 4 * kTileBytes;          // row max and sum [2][2][128]
   static constexpr uint32_t kBar = kRed + 2 * 2 * 128 * 4;
-  static constexpr uint32_t kDyn = kBar + 128;
+  static constexpr uint32_t kDyn = kBar + 256;
 };
 
 struct Bars {
-  uint64_t full[2], empty[2], s_full, p_full, o_full[2], o_free[2];
+  uint64_t full_q[kQSlots], empty_q[kQSlots], full_kv[kKvSlots], empty_kv[kKvSlots];
+  uint64_t s_full, p_full, o_full[2], o_free[2];
   uint32_t tmem;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block");
+
+// Geometry of tile j of this CTA's run.
+struct TileInfo {
+  int bh, tb;          // unit and tile within the unit (r0 = 128 tb)
+  bool has_prev;       // block tb - 1 is part of the window
+  int64_t own, prev;   // ring sequence numbers of blocks tb and tb - 1
+  bool own_last;       // block tb is not used by the next tile
+};
+
+struct Run {
+  int64_t begin, count;
+  int tiles_per_unit;
+  int extra;           // 1 if the run starts with the previous block of its first tile
+  ELSAA_DEV TileInfo tile(int64_t j) const {
+    TileInfo ti;
+    const int64_t t = begin + j;
+    ti.bh = (int)(t / tiles_per_unit);
+    ti.tb = (int)(t % tiles_per_unit);
+    ti.has_prev = ti.tb > 0;
+    ti.own = j + extra;
+    ti.prev = ti.own - 1;
+    ti.own_last = (j + 1 == count) || (ti.tb + 1 == tiles_per_unit);
+    return ti;
+  }
 };
 
 ELSAA_DEV void cp_async_arrive(uint64_t* bar) {
@@ -74,9 +108,36 @@ ELSAA_DEV float ex2(float x) {
 // Barrier among the softmax warps only.
 ELSAA_DEV void softmax_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory"); }
 
-ELSAA_DEV void tile_of(int64_t t, int tiles_per_unit, int* bh, int* r0) {
-  *bh = (int)(t / tiles_per_unit);
-  *r0 = (int)(t % tiles_per_unit) * kTile;
+// Barrier among the softmax warps that also ANDs a flag over them, so that a
+// bounded wait that gave up in one thread makes all of them leave together.
+ELSAA_DEV bool softmax_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kSoftmaxThreads)
+      : "memory");
+  return r != 0;
+}
+
+// Column ranges of a tile's scores: live columns [col_lo, ncols); the two
+// softmax halves take [col_lo & ~31, mid) and [mid, ncols).
+struct Cols {
+  int col0;            // sorted rank of column 0
+  int col_lo, ncols, mid;
+};
+ELSAA_DEV Cols tile_cols(const TileInfo& ti, int chunk) {
+  Cols c;
+  const int r0 = ti.tb * kTile;
+  c.col0 = ti.has_prev ? r0 - kTile : r0;
+  c.col_lo = ti.has_prev ? kTile - chunk : 0;
+  c.ncols = ti.has_prev ? 2 * kTile : kTile;
+  const int lo32 = c.col_lo & ~31;
+  c.mid = ((lo32 + c.ncols) >> 1) & ~31;
+  return c;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -94,16 +155,25 @@ attn_fwd_pipe_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     if (tid == 0) raise_error(err, ERR_CHECK);
     return;
   }
-  const int tiles_per_unit = N / kTile;
-  const int64_t ntiles = (int64_t)BH * tiles_per_unit;
-  // tiles handled by this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...
-  const int64_t my_count =
-      ntiles > blockIdx.x ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  Run run;
+  run.tiles_per_unit = N / kTile;
+  {
+    const int64_t ntiles = (int64_t)BH * run.tiles_per_unit;
+    run.begin = ntiles * blockIdx.x / gridDim.x;
+    run.count = ntiles * (blockIdx.x + 1) / gridDim.x - run.begin;
+    run.extra = (run.count > 0 && run.begin % run.tiles_per_unit != 0) ? 1 : 0;
+  }
 
   if (tid == 0) {
+    for (int s = 0; s < kQSlots; ++s) {
+      mbar_init(&bars->full_q[s], 32);
+      mbar_init(&bars->empty_q[s], 1);
+    }
+    for (int s = 0; s < kKvSlots; ++s) {
+      mbar_init(&bars->full_kv[s], 32);
+      mbar_init(&bars->empty_kv[s], 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars->full[s], 32);
-      mbar_init(&bars->empty[s], 1);
       mbar_init(&bars->o_full[s], 1);
       mbar_init(&bars->o_free[s], kSoftmaxThreads);
     }
@@ -123,97 +193,141 @@ attn_fwd_pipe_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    // Token indices stay in registers (lane j holds rows j, j + 32, ...) and
-    // are broadcast with shuffles while the cp.async gathers are issued.
-    for (int64_t i = 0; i < my_count && ok; ++i) {
-      const int s = (int)(i & 1);
-      if (i >= 2) ok = mbar_wait(&bars->empty[s], (uint32_t)(((i >> 1) - 1) & 1), err);
-      if (!ok) break;
-      int bh, r0;
-      tile_of(blockIdx.x + i * gridDim.x, tiles_per_unit, &bh, &r0);
-      const size_t unit = (size_t)bh * N;
-      const int kbase = max(0, r0 - chunk);
-      const int nk = r0 + kTile - kbase;
-      int qr[kTile / 32], kr[kMaxKeys / 32];
+    // Lane l holds the token indices of rows l, l + 32, l + 64, l + 96 of the
+    // next Q tile and K/V block; a block's rows are gathered 4 per warp
+    // instruction (8 lanes per row, one 16-byte chunk each).
+    const int ch = lane & 7;
+    auto load_idx = [&](const int32_t* perm, size_t base, int (&idx)[4]) {
 #pragma unroll
-      for (int j = 0; j < kTile / 32; ++j) qr[j] = perm_q[unit + r0 + lane + 32 * j];
-#pragma unroll
-      for (int j = 0; j < kMaxKeys / 32; ++j)
-        kr[j] = lane + 32 * j < nk ? perm_k[unit + kbase + lane + 32 * j] : 0;
-      const uint32_t st = sbase + s * Lay::kStage;
-      const __nv_bfloat16* qb = q + unit * D;
+      for (int j = 0; j < 4; ++j) idx[j] = perm[base + lane + 32 * j];
+    };
+    auto issue_kv = [&](int64_t n, size_t unit, const int (&idx)[4]) -> bool {
+      const int s = (int)(n % kKvSlots);
+      if (n >= kKvSlots &&
+          !__all_sync(0xffffffffu,
+                      mbar_wait(&bars->empty_kv[s], (uint32_t)(((n / kKvSlots) - 1) & 1), err)))
+        return false;
+      const uint32_t kst = sbase + Lay::kKv + s * Lay::kKvSlot;
       const __nv_bfloat16* kb = k + unit * D;
       const __nv_bfloat16* vb = v + unit * D;
-      const int ch = lane & 7;
-      // 4 rows per iteration (8 lanes per row, one 16-byte chunk each)
 #pragma unroll
       for (int it = 0; it < kTile / 4; ++it) {
         const int row = 4 * it + (lane >> 3);
-        const int tok = __shfl_sync(0xffffffffu, qr[it >> 3], row & 31);
-        cp_async16(st + sw128_off(row, ch), qb + (size_t)tok * D + ch * 8, 16);
+        const int tok = __shfl_sync(0xffffffffu, idx[it >> 3], row & 31);
+        const size_t src = (size_t)tok * D + ch * 8;
+        cp_async16(kst + sw128_off(row, ch), kb + src, 16);
+        cp_async16(kst + Lay::kTileBytes + sw128_off(row, ch), vb + src, 16);
       }
+      cp_async_arrive(&bars->full_kv[s]);
+      return true;
+    };
+    auto issue_q = [&](int64_t j, size_t unit, const int (&idx)[4]) -> bool {
+      const int s = (int)(j % kQSlots);
+      if (j >= kQSlots &&
+          !__all_sync(0xffffffffu,
+                      mbar_wait(&bars->empty_q[s], (uint32_t)(((j / kQSlots) - 1) & 1), err)))
+        return false;
+      const uint32_t qst = sbase + Lay::kQ + s * Lay::kTileBytes;
+      const __nv_bfloat16* qb = q + unit * D;
 #pragma unroll
-      for (int it = 0; it < kMaxKeys / 4; ++it) {
-        if (4 * it < nk) {   // nk is a multiple of 16: whole iterations only
-          const int row = 4 * it + (lane >> 3);
-          const int tok = __shfl_sync(0xffffffffu, kr[it >> 3], row & 31);
-          const size_t src = (size_t)tok * D + ch * 8;
-          cp_async16(st + Lay::kQ + sw128_off(row, ch), kb + src, 16);
-          cp_async16(st + Lay::kQ + Lay::kKV + sw128_off(row, ch), vb + src, 16);
-        }
+      for (int it = 0; it < kTile / 4; ++it) {
+        const int row = 4 * it + (lane >> 3);
+        const int tok = __shfl_sync(0xffffffffu, idx[it >> 3], row & 31);
+        cp_async16(qst + sw128_off(row, ch), qb + (size_t)tok * D + ch * 8, 16);
       }
-      cp_async_arrive(&bars->full[s]);
+      cp_async_arrive(&bars->full_q[s]);
+      return true;
+    };
+    int qi[4], ki[4];
+    if (run.count > 0) {
+      const TileInfo t0 = run.tile(0);
+      const size_t unit = (size_t)t0.bh * N;
+      if (run.extra) {
+        int pi[4];
+        load_idx(perm_k, unit + (size_t)(t0.tb - 1) * kTile, pi);
+        ok = issue_kv(0, unit, pi);
+      }
+      load_idx(perm_q, unit + (size_t)t0.tb * kTile, qi);
+      load_idx(perm_k, unit + (size_t)t0.tb * kTile, ki);
+    }
+    for (int64_t j = 0; j < run.count && ok; ++j) {
+      const TileInfo ti = run.tile(j);
+      const size_t unit = (size_t)ti.bh * N;
+      ok = issue_q(j, unit, qi) && issue_kv(ti.own, unit, ki);
+      if (!ok) break;
+      if (j + 1 < run.count) {   // prefetch the next tile's indices
+        const TileInfo tn = run.tile(j + 1);
+        const size_t un = (size_t)tn.bh * N;
+        load_idx(perm_q, un + (size_t)tn.tb * kTile, qi);
+        load_idx(perm_k, un + (size_t)tn.tb * kTile, ki);
+      }
     }
     cp_async_wait_all();
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t id_pv = idesc_bf16(128, D, false, true);
+      const uint32_t id_s = idesc_bf16(128, kTile, false, false);
+      auto kv_slot = [&](int64_t n) -> uint32_t {
+        return sbase + Lay::kKv + (uint32_t)(n % kKvSlots) * Lay::kKvSlot;
+      };
       auto issue_pv = [&](int64_t j) -> bool {
-        // O[j % 2] = P V_j ; needs P (p_full) and a free O buffer
+        // O[j % 2] = P V over the live key columns; needs a free O buffer
         const int o = (int)(j & 1);
         if (j >= 2 && !mbar_wait(&bars->o_free[o], (uint32_t)(((j >> 1) - 1) & 1), err))
           return false;
         fence_after();
-        int bh, r0;
-        tile_of(blockIdx.x + j * gridDim.x, tiles_per_unit, &bh, &r0);
-        const int nk = r0 + kTile - max(0, r0 - chunk);
-        const uint32_t vst = sbase + (uint32_t)(j & 1) * Lay::kStage + Lay::kQ + Lay::kKV;
-        for (int s = 0; s < nk / 16; ++s) {
-          const uint32_t poff = (s >> 2) * (128 * 128) + (s & 3) * 32;
+        const TileInfo ti = run.tile(j);
+        const Cols cc = tile_cols(ti, chunk);
+        for (int x = cc.col_lo; x < cc.ncols; x += 16) {
+          const bool in_prev = ti.has_prev && x < kTile;
+          const uint32_t vst = kv_slot(in_prev ? ti.prev : ti.own) + Lay::kTileBytes;
+          const int row = in_prev ? x : (ti.has_prev ? x - kTile : x);
+          const int s = x >> 4;
+          const uint32_t poff = (s >> 2) * Lay::kTileBytes + (s & 3) * 32;
           mma_bf16_ss(tmem + kTO + o * D, sw128_desc(sbase + Lay::kP + poff, 16, 1024),
-                      sw128_desc(vst + s * 2048, 128 * 128, 1024), id_pv, s > 0 ? 1u : 0u);
+                      sw128_desc(vst + (row >> 4) * 2048, Lay::kTileBytes, 1024), id_pv,
+                      x > cc.col_lo ? 1u : 0u);
         }
         mma_commit(&bars->o_full[o]);
-        mma_commit(&bars->empty[j & 1]);
+        if (ti.has_prev) mma_commit(&bars->empty_kv[ti.prev % kKvSlots]);
+        if (ti.own_last) mma_commit(&bars->empty_kv[ti.own % kKvSlots]);
         return true;
       };
-      for (int64_t i = 0; i < my_count && ok; ++i) {
-        const int s = (int)(i & 1);
-        ok = mbar_wait(&bars->full[s], (uint32_t)((i >> 1) & 1), err);
-        if (!ok) break;
-        fence_async_smem();   // cp.async data -> tensor core
-        if (i >= 1) {
-          ok = mbar_wait(&bars->p_full, (uint32_t)((i - 1) & 1), err);
+      int64_t kv_ready = 0;   // blocks whose arrival this thread has seen
+      for (int64_t j = 0; j < run.count && ok; ++j) {
+        if (j >= 1) {
+          ok = mbar_wait(&bars->p_full, (uint32_t)((j - 1) & 1), err);
           if (!ok) break;
-          ok = issue_pv(i - 1);
+          ok = issue_pv(j - 1);
           if (!ok) break;
         }
-        int bh, r0;
-        tile_of(blockIdx.x + i * gridDim.x, tiles_per_unit, &bh, &r0);
-        const int nk = r0 + kTile - max(0, r0 - chunk);
-        const uint32_t st = sbase + s * Lay::kStage;
-        const uint32_t id_s = idesc_bf16(128, nk, false, false);
+        const TileInfo ti = run.tile(j);
+        ok = mbar_wait(&bars->full_q[j % kQSlots], (uint32_t)((j / kQSlots) & 1), err);
+        for (; ok && kv_ready <= ti.own; ++kv_ready)
+          ok = mbar_wait(&bars->full_kv[kv_ready % kKvSlots],
+                         (uint32_t)((kv_ready / kKvSlots) & 1), err);
+        if (!ok) break;
+        fence_async_smem();   // cp.async data -> tensor core
         fence_after();
+        const uint32_t qst = sbase + Lay::kQ + (uint32_t)(j % kQSlots) * Lay::kTileBytes;
+        if (ti.has_prev) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ss(tmem + kTS, sw128_desc(qst + kk * 32, 16, 1024),
+                        sw128_desc(kv_slot(ti.prev) + kk * 32, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+        }
+        const uint32_t own_col = ti.has_prev ? (uint32_t)kTile : 0u;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(tmem + kTS, sw128_desc(st + kk * 32, 16, 1024),
-                      sw128_desc(st + Lay::kQ + kk * 32, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+          mma_bf16_ss(tmem + kTS + own_col, sw128_desc(qst + kk * 32, 16, 1024),
+                      sw128_desc(kv_slot(ti.own) + kk * 32, 16, 1024), id_s, kk > 0 ? 1u : 0u);
         mma_commit(&bars->s_full);
+        mma_commit(&bars->empty_q[j % kQSlots]);
       }
-      if (ok && my_count > 0) {
-        ok = mbar_wait(&bars->p_full, (uint32_t)((my_count - 1) & 1), err);
-        if (ok) ok = issue_pv(my_count - 1);
+      if (ok && run.count > 0) {
+        ok = mbar_wait(&bars->p_full, (uint32_t)((run.count - 1) & 1), err);
+        if (ok) ok = issue_pv(run.count - 1);
       }
     }
     __syncwarp();
@@ -225,21 +339,21 @@ attn_fwd_pipe_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     float* red_m = reinterpret_cast<float*>(smem + Lay::kRed);   // [2][128]
     float* red_l = red_m + 2 * 128;                              // [2][128]
     const bool masked = chunk < kTile;
-    for (int64_t i = 0; i < my_count; ++i) {
-      int bh, r0;
-      tile_of(blockIdx.x + i * gridDim.x, tiles_per_unit, &bh, &r0);
-      const size_t unit = (size_t)bh * N;
+    for (int64_t j = 0; j < run.count; ++j) {
+      const TileInfo ti = run.tile(j);
+      const size_t unit = (size_t)ti.bh * N;
+      const int r0 = ti.tb * kTile;
       const int token = perm_q[unit + r0 + row];
-      const int kbase = max(0, r0 - chunk);
-      const int nk = r0 + kTile - kbase;
-      const int cw = nk >> 1, cbeg = half * cw;          // this warp's key columns
+      const Cols cc = tile_cols(ti, chunk);
+      const int cbeg = half ? cc.mid : (cc.col_lo & ~31);
+      const int cend = half ? cc.ncols : cc.mid;
       const int jr = (r0 + row) / chunk;
-      const int lo = max(0, (jr - 1) * chunk) - kbase, hi = (jr + 1) * chunk - kbase;
-      ok = mbar_wait(&bars->s_full, (uint32_t)(i & 1), err);
+      const int lo = max(0, (jr - 1) * chunk) - cc.col0, hi = (jr + 1) * chunk - cc.col0;
+      ok = softmax_all(mbar_wait(&bars->s_full, (uint32_t)(j & 1), err));
       if (!ok) break;
       fence_after();
       float m = -INFINITY;
-      for (int c0 = cbeg; c0 < cbeg + cw; c0 += 32) {
+      for (int c0 = cbeg; c0 < cend; c0 += 32) {
         float sv[32];
         tmem_ld32(tmem + kTS + lane_off + c0, sv);
         tmem_ld_wait();
@@ -256,7 +370,7 @@ attn_fwd_pipe_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       softmax_sync();
       m = fmaxf(m, red_m[(half ^ 1) * 128 + row]) * scale_log2;   // scale > 0
       float l = 0.f;
-      for (int c0 = cbeg; c0 < cbeg + cw; c0 += 32) {
+      for (int c0 = cbeg; c0 < cend; c0 += 32) {
         float sv[32];
         tmem_ld32(tmem + kTS + lane_off + c0, sv);
         tmem_ld_wait();
@@ -276,7 +390,7 @@ attn_fwd_pipe_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
           const int key = c0 + q8 * 8;
-          uint8_t* dst = smem + Lay::kP + (key >> 6) * (128 * 128) + sw128_off(row, (key & 63) >> 3);
+          uint8_t* dst = smem + Lay::kP + (key >> 6) * Lay::kTileBytes + sw128_off(row, (key & 63) >> 3);
           *reinterpret_cast<uint4*>(dst) =
               make_uint4(packed[q8 * 4], packed[q8 * 4 + 1], packed[q8 * 4 + 2], packed[q8 * 4 + 3]);
         }
@@ -288,8 +402,8 @@ attn_fwd_pipe_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       softmax_sync();
       l += red_l[(half ^ 1) * 128 + row];
       // epilogue: O of this tile; each warp of the pair writes 32 of the 64 columns
-      const int o = (int)(i & 1);
-      ok = mbar_wait(&bars->o_full[o], (uint32_t)((i >> 1) & 1), err);
+      const int o = (int)(j & 1);
+      ok = softmax_all(mbar_wait(&bars->o_full[o], (uint32_t)((j >> 1) & 1), err));
       if (!ok) break;
       fence_after();
       const float inv = 1.0f / l;

@@ -39,6 +39,36 @@ ELSAA_DEV double warp_sum_d(double v) {
 
 ELSAA_DEV float sigmoidf_(float x) { return 1.0f / (1.0f + __expf(-x)); }
 
+// ---- cache-policy hints for 16-byte accesses --------------------------------
+
+// An L2 policy that keeps the lines it touches in preference to others: used
+// for small tables that every row gathers from many times.
+ELSAA_DEV uint64_t l2_keep_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+ELSAA_DEV uint4 ld16_keep(const void* p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+// Streaming (read once) load and store: evict-first in both caches.
+ELSAA_DEV uint4 ld16_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.cs.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+ELSAA_DEV void st16_stream(void* p, uint4 v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+
 ELSAA_DEV void raise_error(uint32_t* err, uint32_t bit) {
   if (err) atomicOr(err, bit);
 }

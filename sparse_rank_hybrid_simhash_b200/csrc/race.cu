@@ -406,32 +406,21 @@ ELSAA_DEV int group_sum_i(int v) {
   return v;
 }
 
-// Adds the 16 bytes at `row` (8 bf16 or 4 fp32 values) to acc.
-ELSAA_DEV void acc_row(float* acc, const __nv_bfloat16* row) {
-  const uint4 raw = *reinterpret_cast<const uint4*>(row);
+// 16 bytes as 8 bf16 or 4 fp32 values, and back.
+ELSAA_DEV void unpack16(uint4 raw, float* v, const __nv_bfloat16*) {
   const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const float2 f = __bfloat1622float2(h[i]);
-    acc[2 * i] += f.x;
-    acc[2 * i + 1] += f.y;
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
   }
 }
-ELSAA_DEV void acc_row(float* acc, const float* row) {
-  const float4 f = *reinterpret_cast<const float4*>(row);
-  acc[0] += f.x; acc[1] += f.y; acc[2] += f.z; acc[3] += f.w;
+ELSAA_DEV void unpack16(uint4 raw, float* v, const float*) {
+  v[0] = __uint_as_float(raw.x); v[1] = __uint_as_float(raw.y);
+  v[2] = __uint_as_float(raw.z); v[3] = __uint_as_float(raw.w);
 }
-
-
-
-// EL consecutive values (EL = 8 for bf16 tables, 4 for fp32) to T storage.
-template <typename T, int EL>
-ELSAA_DEV void store_el(T* p, const float* v) {
-#pragma unroll
-  for (int i = 0; i < EL; ++i) p[i] = from_f32<T>(v[i]);
-}
-template <>
-ELSAA_DEV void store_el<__nv_bfloat16, 8>(__nv_bfloat16* p, const float* v) {
+ELSAA_DEV uint4 pack16(const float* v, const __nv_bfloat16*) {
   uint4 raw;
   uint32_t* w = reinterpret_cast<uint32_t*>(&raw);
 #pragma unroll
@@ -439,17 +428,29 @@ ELSAA_DEV void store_el<__nv_bfloat16, 8>(__nv_bfloat16* p, const float* v) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
     w[i] = *reinterpret_cast<const uint32_t*>(&h);
   }
-  *reinterpret_cast<uint4*>(p) = raw;
+  return raw;
 }
-template <>
-ELSAA_DEV void store_el<float, 4>(float* p, const float* v) {
-  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+ELSAA_DEV uint4 pack16(const float* v, const float*) {
+  return make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
+                    __float_as_uint(v[3]));
 }
-template <>
-ELSAA_DEV void store_el<float, 8>(float* p, const float* v) {
-  reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
-  reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+
+// Adds the 16 bytes at `row` (8 bf16 or 4 fp32 values) to acc; the table line
+// is read with the keep-in-L2 policy `pol`.
+template <typename TT>
+ELSAA_DEV void acc_row(float* acc, const TT* row, uint64_t pol) {
+  constexpr int EL = 16 / sizeof(TT);
+  float f[EL];
+  unpack16(ld16_keep(row, pol), f, row);
+#pragma unroll
+  for (int i = 0; i < EL; ++i) acc[i] += f[i];
 }
+
+// Streaming 16-byte load / store of EL = 16 / sizeof(T) values.
+template <typename T>
+ELSAA_DEV void load16_stream(const T* p, float* v) { unpack16(ld16_stream(p), v, p); }
+template <typename T>
+ELSAA_DEV void store16_stream(T* p, const float* v) { st16_stream(p, pack16(v, p)); }
 
 template <typename TT, typename CodeT, int QL>
 __global__ void __launch_bounds__(256, 4)
@@ -457,6 +458,7 @@ race_gather_sum_kernel(const CodeT* __restrict__ codes, const TT* __restrict__ t
                        int64_t rows, int N, int L, int NB, int d, float* __restrict__ out) {
   constexpr int QW = 32 / QL, EL = 16 / sizeof(TT);
   const int lane = threadIdx.x & 31, ql = lane % QL, gbase = lane - ql;
+  const uint64_t pol = l2_keep_policy();
   const int64_t first = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * QW;
   const int64_t stride = (int64_t)gridDim.x * (blockDim.x >> 5) * QW;
   for (int64_t r0 = first; r0 < rows; r0 += stride) {
@@ -471,10 +473,14 @@ race_gather_sum_kernel(const CodeT* __restrict__ codes, const TT* __restrict__ t
 #pragma unroll 16
       for (int t = 0; t < nt; ++t) {
         const int b = __shfl_sync(0xffffffffu, mycode, gbase + t);
-        acc_row(acc, tables + ((bh * L + t0 + t) * NB + b) * d + ql * EL);
+        acc_row(acc, tables + ((bh * L + t0 + t) * NB + b) * d + ql * EL, pol);
       }
     }
-    if (valid) store_el<float, EL>(out + rr * d + ql * EL, acc);
+    if (valid) {
+      float* o = out + rr * d + ql * EL;
+#pragma unroll
+      for (int i = 0; i < EL; i += 4) store16_stream(o + i, acc + i);
+    }
   }
 }
 
@@ -530,6 +536,7 @@ race_fuse_fwd_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q,
                      T* __restrict__ y, T* __restrict__ o_race, int32_t* __restrict__ ctot_out) {
   constexpr int QW = 32 / QL, EL = 16 / sizeof(T);
   const int lane = threadIdx.x & 31, ql = lane % QL, gbase = lane - ql;
+  const uint64_t pol = l2_keep_policy();
   const float lam_v = *lam;
   float ws8[EL], wr8[EL];
 #pragma unroll
@@ -557,15 +564,15 @@ race_fuse_fwd_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q,
 #pragma unroll 16
       for (int t = 0; t < nt; ++t) {
         const int b = __shfl_sync(0xffffffffu, mycode, gbase + t);
-        acc_row(acc, tables + ((bh * L + t0 + t) * NB + b) * d + ql * EL);
+        acc_row(acc, tables + ((bh * L + t0 + t) * NB + b) * d + ql * EL, pol);
       }
     }
     ctot = group_sum_i<QL>(ctot);
     const float inv = ctot > 0 ? 1.0f / (float)ctot : 0.f;
     const size_t base = (size_t)rr * d + ql * EL;
     float qv[EL], os[EL], orc[EL];
-    load_el<T, EL>(q + base, qv);
-    load_el<T, EL>(o_sp + base, os);
+    load16_stream(q + base, qv);
+    load16_stream(o_sp + base, os);
 #pragma unroll
     for (int i = 0; i < EL; ++i) orc[i] = acc[i] * inv;
     float gs = gs_fixed, gr = gr_fixed;
@@ -588,10 +595,183 @@ race_fuse_fwd_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q,
       float yv[EL];
 #pragma unroll
       for (int i = 0; i < EL; ++i) yv[i] = gs * m * os[i] + gr * orc[i];
-      store_el<T, EL>(y + base, yv);
-      if (o_race) store_el<T, EL>(o_race + base, orc);
+      store16_stream(y + base, yv);
+      if (o_race) store16_stream(o_race + base, orc);
       if (ctot_out && ql == 0) ctot_out[rr] = ctot;
     }
+  }
+}
+
+// ---- row-pipelined gathers ---------------------------------------------------
+//
+// Used when a row's codes are whole 32-bit words (L * code bytes % 4 == 0).
+// A row is served by QL lanes; lane ql of the group holds the row's code
+// words ql, ql + QL, ... (WPL at most), loaded with one access each, and the
+// next row's words are fetched while this row's table lines are gathered, so
+// every gather of a row is independent of any load issued in the same pass.
+
+template <typename CodeT, int QL, int WPL>
+ELSAA_DEV void load_row_codes(const CodeT* row, int W, int ql, uint32_t (&w)[WPL]) {
+  const uint32_t* p = reinterpret_cast<const uint32_t*>(row);
+#pragma unroll
+  for (int i = 0; i < WPL; ++i) {
+    const int wi = ql + i * QL;
+    w[i] = wi < W ? __ldcs(p + wi) : 0u;
+  }
+}
+
+template <typename CodeT>
+ELSAA_DEV int code_of(uint32_t word, int e) {
+  return sizeof(CodeT) == 1 ? (int)((word >> (8 * e)) & 0xFFu) : (int)((word >> (16 * e)) & 0xFFFFu);
+}
+
+// acc += sum over tables t of tab[t][code_t][ql * EL ...], tab = this unit's
+// tables offset by the lane's column slice.
+template <typename TT, typename CodeT, int QL, int WPL>
+ELSAA_DEV void gather_row(const TT* tab, const uint32_t (&w)[WPL], int L, int NB, int d,
+                          int gbase, uint64_t pol, float* acc) {
+  constexpr int PER = 4 / (int)sizeof(CodeT);
+#pragma unroll
+  for (int i = 0; i < WPL; ++i) {
+#pragma unroll
+    for (int sl = 0; sl < QL; ++sl) {
+      const int t0 = (i * QL + sl) * PER;
+      if (t0 < L) {
+        const uint32_t word = __shfl_sync(0xffffffffu, w[i], gbase + sl);
+#pragma unroll
+        for (int e = 0; e < PER; ++e)
+          acc_row(acc, tab + ((size_t)(t0 + e) * NB + code_of<CodeT>(word, e)) * d, pol);
+      }
+    }
+  }
+}
+
+template <typename TT, typename CodeT, int QL, int WPL>
+__global__ void __launch_bounds__(256, 4)
+race_gather_rows_kernel(const CodeT* __restrict__ codes, const TT* __restrict__ tables,
+                        int64_t rows, int N, int L, int NB, int d, float* __restrict__ out) {
+  constexpr int QW = 32 / QL, EL = 16 / sizeof(TT);
+  const int lane = threadIdx.x & 31, ql = lane % QL, gbase = lane - ql;
+  const uint64_t pol = l2_keep_policy();
+  const int W = L * (int)sizeof(CodeT) / 4;
+  const int64_t first = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * QW;
+  const int64_t stride = (int64_t)gridDim.x * (blockDim.x >> 5) * QW;
+  uint32_t w[WPL];
+  {
+    const int64_t r = min(first + lane / QL, rows - 1);
+    load_row_codes<CodeT, QL, WPL>(codes + r * L, W, ql, w);
+  }
+  for (int64_t r0 = first; r0 < rows; r0 += stride) {
+    const int64_t r = r0 + lane / QL;
+    const bool valid = r < rows;
+    const int64_t rr = valid ? r : rows - 1;
+    const int64_t bh = rr / N;
+    uint32_t wn[WPL];
+    load_row_codes<CodeT, QL, WPL>(codes + min(r + stride, rows - 1) * L, W, ql, wn);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    gather_row<TT, CodeT, QL, WPL>(tables + (size_t)bh * L * NB * d + ql * EL, w, L, NB, d,
+                                   gbase, pol, acc);
+    if (valid) {
+      float* o = out + rr * d + ql * EL;
+#pragma unroll
+      for (int i = 0; i < EL; i += 4) store16_stream(o + i, acc + i);
+    }
+#pragma unroll
+    for (int i = 0; i < WPL; ++i) w[i] = wn[i];
+  }
+}
+
+template <typename T, typename CodeT, int QL, int WPL>
+__global__ void __launch_bounds__(256, 4)
+race_fuse_rows_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q,
+                      const T* __restrict__ tables, const int32_t* __restrict__ counts,
+                      const T* __restrict__ o_sp, const float* __restrict__ lse,
+                      const float* __restrict__ gate_w, const float* __restrict__ gate_b,
+                      int gate_fixed, float gs_fixed, float gr_fixed,
+                      const float* __restrict__ lam, int64_t rows, int N, int L, int NB, int d,
+                      T* __restrict__ y, T* __restrict__ o_race, int32_t* __restrict__ ctot_out) {
+  constexpr int QW = 32 / QL, EL = 16 / sizeof(T);
+  constexpr int PER = 4 / (int)sizeof(CodeT);
+  const int lane = threadIdx.x & 31, ql = lane % QL, gbase = lane - ql;
+  const uint64_t pol = l2_keep_policy();
+  const int W = L * (int)sizeof(CodeT) / 4;
+  const float lam_v = *lam;
+  float ws8[EL], wr8[EL];
+#pragma unroll
+  for (int i = 0; i < EL; ++i) ws8[i] = wr8[i] = 0.f;
+  float bs = 0.f, br = 0.f;
+  if (!gate_fixed) {
+    load_el<float, EL>(gate_w + ql * EL, ws8);
+    load_el<float, EL>(gate_w + d + ql * EL, wr8);
+    bs = gate_b[0];
+    br = gate_b[1];
+  }
+  const int64_t first = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * QW;
+  const int64_t stride = (int64_t)gridDim.x * (blockDim.x >> 5) * QW;
+  uint32_t w[WPL];
+  {
+    const int64_t r = min(first + lane / QL, rows - 1);
+    load_row_codes<CodeT, QL, WPL>(rcode_q + r * L, W, ql, w);
+  }
+  for (int64_t r0 = first; r0 < rows; r0 += stride) {
+    const int64_t r = r0 + lane / QL;
+    const bool valid = r < rows;
+    const int64_t rr = valid ? r : rows - 1;
+    const int64_t bh = rr / N;
+    const size_t base = (size_t)rr * d + ql * EL;
+    // this row's streams and the next row's codes go out before the gathers
+    const uint4 q_raw = ld16_stream(q + base);
+    const uint4 os_raw = ld16_stream(o_sp + base);
+    const float lse_r = lse[rr];
+    uint32_t wn[WPL];
+    load_row_codes<CodeT, QL, WPL>(rcode_q + min(r + stride, rows - 1) * L, W, ql, wn);
+    // Ctot: this lane's words' bucket counts
+    int ctot = 0;
+    const int32_t* cnt = counts + (size_t)bh * L * NB;
+#pragma unroll
+    for (int i = 0; i < WPL; ++i) {
+      const int wi = ql + i * QL;
+      if (wi < W) {
+#pragma unroll
+        for (int e = 0; e < PER; ++e) ctot += cnt[(size_t)(wi * PER + e) * NB + code_of<CodeT>(w[i], e)];
+      }
+    }
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    gather_row<T, CodeT, QL, WPL>(tables + (size_t)bh * L * NB * d + ql * EL, w, L, NB, d, gbase,
+                                  pol, acc);
+    ctot = group_sum_i<QL>(ctot);
+    const float inv = ctot > 0 ? 1.0f / (float)ctot : 0.f;
+    float qv[EL], os[EL], orc[EL];
+    unpack16(q_raw, qv, q);
+    unpack16(os_raw, os, o_sp);
+#pragma unroll
+    for (int i = 0; i < EL; ++i) orc[i] = acc[i] * inv;
+    float gs = gs_fixed, gr = gr_fixed;
+    if (!gate_fixed) {
+      float as = 0.f, ar = 0.f;
+#pragma unroll
+      for (int i = 0; i < EL; ++i) {
+        as += qv[i] * ws8[i];
+        ar += qv[i] * wr8[i];
+      }
+      as = group_sum<QL>(as) + bs;
+      ar = group_sum<QL>(ar) + br;
+      gs = 1.0f / (1.0f + expf(-as));
+      gr = 1.0f / (1.0f + expf(-ar));
+    }
+    // m = Z_sp / (Z_sp + lambda Z_race) = 1 / (1 + exp(log(lambda Z_race) - lse))
+    const float lz = lam_v * (float)ctot / (float)L;
+    const float m = lz > 0.f ? 1.0f / (1.0f + expf(logf(lz) - lse_r)) : 1.0f;
+    if (valid) {
+      float yv[EL];
+#pragma unroll
+      for (int i = 0; i < EL; ++i) yv[i] = gs * m * os[i] + gr * orc[i];
+      store16_stream(y + base, yv);
+      if (o_race) store16_stream(o_race + base, orc);
+      if (ctot_out && ql == 0) ctot_out[rr] = ctot;
+    }
+#pragma unroll
+    for (int i = 0; i < WPL; ++i) w[i] = wn[i];
   }
 }
 
@@ -706,18 +886,53 @@ cudaError_t build(const Geometry& g, const void* codes, const void* vals, const 
   return cudaGetLastError();
 }
 
+// Words per lane of the row-pipelined gathers (0: not applicable).
+int row_wpl(const Geometry& g, int QL) {
+  if ((g.L * g.rcode_bytes) % 4 != 0) return 0;
+  const int W = g.L * g.rcode_bytes / 4;
+  const int wpl = (W + QL - 1) / QL;
+  return wpl <= 1 ? 1 : wpl <= 2 ? 2 : wpl <= 4 ? 4 : 0;
+}
+
+int rows_grid(int64_t rows, int QL) {
+  const int64_t warps = (rows * QL + 31) / 32;
+  const int64_t b = (warps + 7) / 8;
+  return (int)(b < 148 * 4 ? b : 148 * 4);
+}
+
 template <typename TT, typename CodeT>
 cudaError_t gather_sum(const Geometry& g, const void* codes, const TT* tables, float* out,
                        cudaStream_t s) {
   constexpr int EL = 16 / sizeof(TT);
   const int64_t rows = (int64_t)g.BH * g.N;
-  const int grid = grid_for_rows((rows * g.d / EL + 31) / 32, 8);
+  const int QLr = g.d / EL;
   const CodeT* c = static_cast<const CodeT*>(codes);
-  switch (g.d / EL) {
-    case 4: race_gather_sum_kernel<TT, CodeT, 4><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
-    case 8: race_gather_sum_kernel<TT, CodeT, 8><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
-    case 16: race_gather_sum_kernel<TT, CodeT, 16><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
-    default: race_gather_sum_kernel<TT, CodeT, 32><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
+  const int wpl = row_wpl(g, QLr);
+  if (wpl > 0) {
+    const int grid = rows_grid(rows, QLr);
+#define ELSAA_GROWS(QL, WPL)                                                                   \
+  race_gather_rows_kernel<TT, CodeT, QL, WPL><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L,  \
+                                                                    g.NB, g.d, out)
+#define ELSAA_GROWS_W(QL)                                                                      \
+  switch (wpl) {                                                                               \
+    case 1: ELSAA_GROWS(QL, 1); break;                                                         \
+    case 2: ELSAA_GROWS(QL, 2); break;                                                         \
+    default: ELSAA_GROWS(QL, 4); break;                                                        \
+  }
+    switch (g.d) {   // QL = d / EL for d in {32, 64, 128}
+      case 32: ELSAA_GROWS_W(32 / EL); break;
+      case 64: ELSAA_GROWS_W(64 / EL); break;
+      default: ELSAA_GROWS_W(128 / EL); break;
+    }
+#undef ELSAA_GROWS_W
+#undef ELSAA_GROWS
+    return cudaGetLastError();
+  }
+  const int grid = grid_for_rows((rows * g.d / EL + 31) / 32, 8);
+  switch (g.d) {
+    case 32: race_gather_sum_kernel<TT, CodeT, 32 / EL><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
+    case 64: race_gather_sum_kernel<TT, CodeT, 64 / EL><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
+    default: race_gather_sum_kernel<TT, CodeT, 128 / EL><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
   }
   return cudaGetLastError();
 }
@@ -730,6 +945,31 @@ cudaError_t fuse_fwd(const Geometry& g, const void* q, const void* rcode_q,
                      float gr) {
   constexpr int EL = 16 / sizeof(T);
   const int64_t rows = (int64_t)g.BH * g.N;
+  const int QLr = g.d / EL;
+  const int wpl = row_wpl(g, QLr);
+  if (wpl > 0) {
+    const int grid = rows_grid(rows, QLr);
+#define ELSAA_FROWS(QL, WPL)                                                                   \
+  race_fuse_rows_kernel<T, CodeT, QL, WPL><<<grid, 256, 0, s>>>(                               \
+      static_cast<const T*>(q), static_cast<const CodeT*>(rcode_q),                            \
+      static_cast<const T*>(tables), counts, static_cast<const T*>(o_sp), lse, gate_w, gate_b, \
+      gate_fixed, gs, gr, lam, rows, g.N, g.L, g.NB, g.d, static_cast<T*>(y),                  \
+      static_cast<T*>(o_race), ctot)
+#define ELSAA_FROWS_W(QL)                                                                      \
+  switch (wpl) {                                                                               \
+    case 1: ELSAA_FROWS(QL, 1); break;                                                         \
+    case 2: ELSAA_FROWS(QL, 2); break;                                                         \
+    default: ELSAA_FROWS(QL, 4); break;                                                        \
+  }
+    switch (g.d) {   // QL = d / EL for d in {32, 64, 128}
+      case 32: ELSAA_FROWS_W(32 / EL); break;
+      case 64: ELSAA_FROWS_W(64 / EL); break;
+      default: ELSAA_FROWS_W(128 / EL); break;
+    }
+#undef ELSAA_FROWS_W
+#undef ELSAA_FROWS
+    return cudaGetLastError();
+  }
   const int grid = grid_for_rows((rows * g.d / EL + 31) / 32, 8);
 #define ELSAA_FUSE(QL)                                                                         \
   race_fuse_fwd_kernel<T, CodeT, QL><<<grid, 256, 0, s>>>(                                     \
@@ -737,11 +977,10 @@ cudaError_t fuse_fwd(const Geometry& g, const void* q, const void* rcode_q,
       static_cast<const T*>(tables), counts,                                                    \
       static_cast<const T*>(o_sp), lse, gate_w, gate_b, gate_fixed, gs, gr, lam, rows, g.N,    \
       g.L, g.NB, g.d, static_cast<T*>(y), static_cast<T*>(o_race), ctot)
-  switch (g.d / EL) {
-    case 4: ELSAA_FUSE(4); break;
-    case 8: ELSAA_FUSE(8); break;
-    case 16: ELSAA_FUSE(16); break;
-    default: ELSAA_FUSE(32); break;
+  switch (g.d) {
+    case 32: ELSAA_FUSE(32 / EL); break;
+    case 64: ELSAA_FUSE(64 / EL); break;
+    default: ELSAA_FUSE(128 / EL); break;
   }
 #undef ELSAA_FUSE
   return cudaGetLastError();
