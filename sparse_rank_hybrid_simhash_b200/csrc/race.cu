@@ -602,6 +602,211 @@ race_fuse_fwd_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q,
   }
 }
 
+// ---- bucket-sorted build --------------------------------------------------------
+//
+// One CTA per (unit, table).  The table's codes are cached in shared memory
+// and counted; a counting sort lists the keys bucket by bucket; then lane
+// groups walk equal shares of that list, gather each key's value row from
+// global memory (L2-resident for the unit) and add it into a register
+// accumulator until the bucket changes, when the run total goes to the
+// shared table with one integer add per column.
+//
+// Exactness and determinism: every value is rounded once to the fixed-point
+// grid 2^-S, with |v| 2^S < 2^21 and C_max vmax 2^S < 2^30, so every partial
+// and every bucket total fits in int32 and integer addition makes the result
+// independent of the order in which keys reach a bucket.  The rounding uses
+// the float-add trick: for |x| < 2^22, the bits of fmaf(v, 2^S, 1.5 * 2^23)
+// are 0x4B400000 plus x rounded to the nearest integer (ties to even, as the
+// add rounds), so a run of n rows sums to its integer total plus n * 0x4B400000
+// modulo 2^32.
+
+constexpr int kSortedThreads = 1024;
+constexpr uint32_t kMagicBits = 0x4B400000u;   // bits of 1.5 * 2^23
+constexpr float kMagic = 12582912.0f;           // 1.5 * 2^23
+
+struct SortedSmem {
+  size_t list, codes, tab, cnt, cur, misc, total;
+};
+__host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
+__host__ __device__ inline SortedSmem sorted_smem(int N, int NB, int d, int code_bytes) {
+  SortedSmem m;
+  m.tab = 0;
+  m.list = align16(m.tab + (size_t)NB * d * 4);
+  m.codes = align16(m.list + (size_t)N * 2);
+  m.cnt = align16(m.codes + (size_t)N * code_bytes);
+  m.cur = align16(m.cnt + (size_t)NB * 4);
+  m.misc = align16(m.cur + (size_t)NB * 4);
+  m.total = m.misc + 256;   // [0] C_max, [1] bad code, [16..48) warp sums of the scan
+  return m;
+}
+
+template <typename TV>
+ELSAA_DEV void add_fixed(uint32_t* acc, uint4 raw, float scale, const TV*) {
+  float v[16 / sizeof(TV)];
+  unpack16(raw, v, static_cast<const TV*>(nullptr));
+#pragma unroll
+  for (int i = 0; i < (int)(16 / sizeof(TV)); ++i)
+    acc[i] += __float_as_uint(fmaf(v[i], scale, kMagic));
+}
+
+template <typename TV, typename CodeT>
+__global__ void __launch_bounds__(kSortedThreads, 1)
+race_build_sorted_kernel(const CodeT* __restrict__ codes, const TV* __restrict__ vals, int N,
+                         int L, int NB, int d, const float* __restrict__ absmax,
+                         float* __restrict__ sums, __nv_bfloat16* __restrict__ gtab,
+                         int32_t* __restrict__ counts, uint32_t* __restrict__ err) {
+  constexpr int EL = 16 / (int)sizeof(TV);
+  extern __shared__ __align__(16) uint8_t sm[];
+  const SortedSmem lay = sorted_smem(N, NB, d, (int)sizeof(CodeT));
+  int32_t* tab = reinterpret_cast<int32_t*>(sm + lay.tab);          // [NB][d] fixed point
+  uint16_t* list = reinterpret_cast<uint16_t*>(sm + lay.list);      // keys, bucket by bucket
+  CodeT* csm = reinterpret_cast<CodeT*>(sm + lay.codes);            // [N] this table's codes
+  int32_t* cnt = reinterpret_cast<int32_t*>(sm + lay.cnt);          // [NB]
+  int32_t* cur = reinterpret_cast<int32_t*>(sm + lay.cur);          // [NB] scatter cursors
+  int32_t* misc = reinterpret_cast<int32_t*>(sm + lay.misc);        // [0] C_max, [1] bad code
+  int32_t* wsum = misc + 16;                                        // [32] scan warp sums
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t = blockIdx.x, bh = blockIdx.y;
+
+  for (int i = tid; i < NB * d; i += kSortedThreads) tab[i] = 0;
+  for (int i = tid; i < NB; i += kSortedThreads) cnt[i] = 0;
+  if (tid < 2) misc[tid] = 0;
+  __syncthreads();
+
+  // codes of table t and their bucket counts
+  const CodeT* cb = codes + (size_t)bh * N * L + t;
+  for (int j = tid; j < N; j += kSortedThreads) {
+    int c = (int)cb[(size_t)j * L];
+    if (c >= NB) {
+      misc[1] = 1;
+      c = 0;
+    }
+    csm[j] = (CodeT)c;
+    atomicAdd(cnt + c, 1);
+  }
+  __syncthreads();
+
+  // exclusive scan of the counts (NB <= 1024: one bucket per thread)
+  {
+    const int c = tid < NB ? cnt[tid] : 0;
+    int x = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31 && warp * 32 < NB) wsum[warp] = x;
+    int cm = c;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cm = max(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+    if (lane == 0) atomicMax(misc, cm);
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp && w * 32 < NB; ++w) before += wsum[w];
+    __syncthreads();
+    if (tid < NB) {
+      cur[tid] = before + x - c;
+      if (counts) counts[((size_t)bh * L + t) * NB + tid] = c;
+    }
+  }
+  __syncthreads();
+  if (misc[1] != 0) {
+    if (tid == 0) raise_error(err, ERR_CHECK);
+    return;
+  }
+  // keys to their buckets' slots (order inside a bucket does not matter)
+  for (int j = tid; j < N; j += kSortedThreads) {
+    const int c = (int)csm[j];
+    list[atomicAdd(cur + c, 1)] = (uint16_t)j;
+  }
+  const float vmax = absmax[bh];
+  if (!(vmax < 3.0e38f)) {
+    if (tid == 0) raise_error(err, ERR_CHECK);
+    return;
+  }
+  __syncthreads();
+  const int cmax = misc[0];
+  int S = 0;
+  if (cmax > 0 && vmax > 0.f) {
+    const int s1 = (int)floorf(log2f(1073741824.0f / ((float)cmax * vmax)));
+    const int s2 = (int)floorf(log2f(2097152.0f / vmax));
+    S = max(-100, min(100, min(s1, s2)));
+  }
+  const float scale = ldexpf(1.0f, S), inv_scale = ldexpf(1.0f, -S);
+
+  // lane groups of QL lanes walk equal shares of the list
+  const int QL = d / EL;
+  const int groups = kSortedThreads / QL;
+  const int g = tid / QL, ql = tid % QL;
+  const int p0 = (int)((int64_t)N * g / groups), p1 = (int)((int64_t)N * (g + 1) / groups);
+  const TV* vb = vals + (size_t)bh * N * d + ql * EL;
+  uint32_t acc[EL];
+#pragma unroll
+  for (int e = 0; e < EL; ++e) acc[e] = 0u;
+  int run_code = -1, run_n = 0;
+  auto flush = [&]() {
+    if (run_n > 0) {
+      const uint32_t bias = (uint32_t)run_n * kMagicBits;
+      int32_t* dst = tab + (size_t)run_code * d + ql * EL;
+#pragma unroll
+      for (int e = 0; e < EL; ++e) {
+        atomicAdd(reinterpret_cast<uint32_t*>(dst + e), acc[e] - bias);
+        acc[e] = 0u;
+      }
+    }
+    run_n = 0;
+  };
+  constexpr int U = 4;
+  int p = p0;
+  for (; p + U <= p1; p += U) {
+    int key[U], code[U];
+    uint4 raw[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      key[u] = list[p + u];
+      code[u] = (int)csm[key[u]];
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) raw[u] = __ldg(reinterpret_cast<const uint4*>(vb + (size_t)key[u] * d));
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (code[u] != run_code) {
+        flush();
+        run_code = code[u];
+      }
+      add_fixed(acc, raw[u], scale, vb);
+      ++run_n;
+    }
+  }
+  for (; p < p1; ++p) {
+    const int k1 = list[p], c1 = (int)csm[k1];
+    const uint4 r1 = __ldg(reinterpret_cast<const uint4*>(vb + (size_t)k1 * d));
+    if (c1 != run_code) {
+      flush();
+      run_code = c1;
+    }
+    add_fixed(acc, r1, scale, vb);
+    ++run_n;
+  }
+  flush();
+  __syncthreads();
+
+  const size_t o0 = ((size_t)bh * L + t) * NB * d;
+  for (int i = tid * 4; i < NB * d; i += kSortedThreads * 4) {
+    const int4 v4 = *reinterpret_cast<const int4*>(tab + i);
+    const float f0 = (float)v4.x * inv_scale, f1 = (float)v4.y * inv_scale;
+    const float f2 = (float)v4.z * inv_scale, f3 = (float)v4.w * inv_scale;
+    if (sums) *reinterpret_cast<float4*>(sums + o0 + i) = make_float4(f0, f1, f2, f3);
+    if (gtab) {
+      const __nv_bfloat162 h0 = __floats2bfloat162_rn(f0, f1), h1 = __floats2bfloat162_rn(f2, f3);
+      uint2 w2;
+      w2.x = *reinterpret_cast<const uint32_t*>(&h0);
+      w2.y = *reinterpret_cast<const uint32_t*>(&h1);
+      *reinterpret_cast<uint2*>(gtab + o0 + i) = w2;
+    }
+  }
+}
+
 // ---- row-pipelined gathers ---------------------------------------------------
 //
 // Used when a row's codes are whole 32-bit words (L * code bytes % 4 == 0).
@@ -823,6 +1028,22 @@ template <typename TV, typename CodeT>
 cudaError_t build(const Geometry& g, const void* codes, const void* vals, const float* absmax,
                   float* sums, bool keep_sums, __nv_bfloat16* gtab, int32_t* counts,
                   uint32_t* err, cudaStream_t s) {
+  {
+    // bucket-sorted build: key indices fit u16, one bucket per thread in the
+    // scan, and the whole table plus the key list fit in shared memory
+    const SortedSmem m = sorted_smem(g.N, g.NB, g.d, (int)sizeof(CodeT));
+    if (g.N <= 65536 && g.NB <= kSortedThreads && m.total <= (size_t)kBuildSmemBudget &&
+        g.d % (16 / (int)sizeof(TV)) == 0) {
+      auto kernel = race_build_sorted_kernel<TV, CodeT>;
+      cudaError_t e =
+          cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)m.total);
+      if (e != cudaSuccess) return e;
+      kernel<<<dim3(g.L, g.BH), kSortedThreads, m.total, s>>>(
+          static_cast<const CodeT*>(codes), static_cast<const TV*>(vals), g.N, g.L, g.NB, g.d,
+          absmax, keep_sums ? sums : nullptr, gtab, counts, err);
+      return cudaGetLastError();
+    }
+  }
   const BuildShape b = build_shape(g);
   if (b.nt < 1) {
     // tables too large for shared memory even one at a time: global fp32
