@@ -57,6 +57,7 @@ SavedLayout saved_layout(const Geometry& g) {
   s.code = take(2 * bhn * 2);
   s.perm = take(2 * bhn * 4);
   s.rcode = take(2 * bhn * g.L * g.rcode_bytes);
+  s.rcode_t = take(2 * bhn * g.L * g.rcode_bytes);
   s.race_count = take((size_t)g.BH * g.L * g.NB * 4);
   s.race_sum = take((size_t)g.BH * g.L * g.NB * g.d * 4);
   s.lse = take(bhn * 4);
@@ -195,6 +196,8 @@ elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const vo
   int32_t* perm = (int32_t*)(sv + sl.perm);
   char* rcode = sv + sl.rcode;
   char* rcode_k = rcode + bhn * g.L * g.rcode_bytes;
+  char* rcode_t = sv + sl.rcode_t;   // table-major: queries, then keys
+  char* rcode_tk = rcode_t + bhn * g.L * g.rcode_bytes;
   int32_t* counts = (int32_t*)(sv + sl.race_count);
   float* sums = (float*)(sv + sl.race_sum);
   float* lse = (float*)(sv + sl.lse);
@@ -205,9 +208,9 @@ elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const vo
 
   // 1. SimHash codes of Q and K
   if (g.tc_hash)
-    ELSAA_TRY(launch_hash_tc(g, q, k, r_sort, r_race, code, rcode, nullptr, err, s));
+    ELSAA_TRY(launch_hash_tc(g, q, k, r_sort, r_race, code, rcode, rcode_t, err, s));
   else
-    ELSAA_TRY(launch_hash_simt(g, q, k, r_sort, r_race, code, rcode, s));
+    ELSAA_TRY(launch_hash_simt(g, q, k, r_sort, r_race, code, rcode, rcode_t, s));
   ELSAA_TRY(mark(events, 1, s));
   // 2. Sort-LSH order of Q and K
   ELSAA_TRY(launch_sort(g, code, perm, (int32_t*)(w + wl.sort_hist), (int32_t*)(w + wl.sort_tmp),
@@ -219,7 +222,7 @@ elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const vo
   // gathers read tables in the data dtype: a bf16 copy, or the fp32 sums themselves
   __nv_bfloat16* gtab = g.bf16 ? (__nv_bfloat16*)(w + wl.gtab) : nullptr;
   const void* gather_tables = g.bf16 ? (const void*)gtab : (const void*)sums;
-  ELSAA_TRY(launch_race_build(g, rcode_k, v, false, absmax, sums, true, gtab, counts, err, s));
+  ELSAA_TRY(launch_race_build(g, rcode_k, rcode_tk, v, false, absmax, sums, true, gtab, counts, err, s));
   ELSAA_TRY(mark(events, 3, s));
   // 4. exact sparse branch
   if (g.tc_attn && attn_pipe_supported(g))
@@ -274,6 +277,7 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
   const int32_t* perm = (const int32_t*)(sv + sl.perm);
   const char* rcode = sv + sl.rcode;
   const char* rcode_k = rcode + bhn * g.L * g.rcode_bytes;
+  const char* rcode_t = sv + sl.rcode_t;   // table-major query codes
   const float* lse = (const float*)(sv + sl.lse);
   const void* o_sp = sv + sl.o_sp;
   const void* o_race = sv + sl.o_race;
@@ -296,7 +300,7 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
   ELSAA_TRY(mark(events, 1, s));
   // 2. RACE backward: scatter into the table gradient by query code, gather by key code
   __nv_bfloat16* gtab = g.bf16 ? (__nv_bfloat16*)(w + wl.gtab) : nullptr;
-  ELSAA_TRY(launch_race_build(g, rcode, dor, false, absmax, d_t, !g.bf16, gtab, nullptr,
+  ELSAA_TRY(launch_race_build(g, rcode, rcode_t, dor, false, absmax, d_t, !g.bf16, gtab, nullptr,
                               (uint32_t*)(w + wl.err), s));
   ELSAA_TRY(launch_race_gather_sum(g, rcode_k, g.bf16 ? (const void*)gtab : (const void*)d_t,
                                    dv_acc, s));

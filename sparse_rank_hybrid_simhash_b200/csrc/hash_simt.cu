@@ -19,8 +19,9 @@ template <typename T, typename CodeT>
 __global__ void __launch_bounds__(256)
 hash_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
                  const T* __restrict__ r_sort, const T* __restrict__ r_race,
-                 int64_t rows_per_tensor, int d, int sort_bits, int L, int kr,
-                 uint16_t* __restrict__ code, CodeT* __restrict__ rcode) {
+                 int64_t rows_per_tensor, int N, int d, int sort_bits, int L, int kr,
+                 uint16_t* __restrict__ code, CodeT* __restrict__ rcode,
+                 CodeT* __restrict__ rcode_t) {
   extern __shared__ float smem[];
   const int warps = blockDim.x >> 5;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -57,14 +58,20 @@ hash_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
       return v;
     };
     if (lane == 0) code[row] = (uint16_t)field(0, sort_bits);
-    for (int l = lane; l < L; l += 32) rcode[row * L + l] = (CodeT)field(sort_bits + l * kr, kr);
+    const int64_t u = row / N;
+    CodeT* tdst = rcode_t + (size_t)u * L * N + (row - u * N);
+    for (int l = lane; l < L; l += 32) {
+      const CodeT c = (CodeT)field(sort_bits + l * kr, kr);
+      rcode[row * L + l] = c;
+      tdst[(size_t)l * N] = c;
+    }
     __syncwarp();
   }
 }
 
 template <typename T, typename CodeT>
 cudaError_t run(const Geometry& g, const void* q, const void* k, const void* r_sort,
-                const void* r_race, uint16_t* code, void* rcode, cudaStream_t s) {
+                const void* r_race, uint16_t* code, void* rcode, void* rcode_t, cudaStream_t s) {
   const int threads = 256, warps = threads / 32;
   const int P = g.sort_bits + g.L * g.kr;
   const size_t smem = (size_t)warps * g.d * sizeof(float) + (size_t)warps * ((P + 31) / 32) * 4;
@@ -78,22 +85,24 @@ cudaError_t run(const Geometry& g, const void* q, const void* k, const void* r_s
   const int grid = (int)(blocks < 148 * 64 ? blocks : 148 * 64);
   hash_simt_kernel<T, CodeT><<<grid, threads, smem, s>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(r_sort),
-      static_cast<const T*>(r_race), rows, g.d, g.sort_bits, g.L, g.kr, code,
-      static_cast<CodeT*>(rcode));
+      static_cast<const T*>(r_race), rows, g.N, g.d, g.sort_bits, g.L, g.kr, code,
+      static_cast<CodeT*>(rcode), static_cast<CodeT*>(rcode_t));
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_hash_simt(const Geometry& g, const void* q, const void* k, const void* r_sort,
-                             const void* r_race, uint16_t* code, void* rcode, cudaStream_t s) {
+                             const void* r_race, uint16_t* code, void* rcode, void* rcode_t,
+                             cudaStream_t s) {
   if (g.bf16) {
     return g.rcode_bytes == 1
-               ? run<__nv_bfloat16, uint8_t>(g, q, k, r_sort, r_race, code, rcode, s)
-               : run<__nv_bfloat16, uint16_t>(g, q, k, r_sort, r_race, code, rcode, s);
+               ? run<__nv_bfloat16, uint8_t>(g, q, k, r_sort, r_race, code, rcode, rcode_t, s)
+               : run<__nv_bfloat16, uint16_t>(g, q, k, r_sort, r_race, code, rcode, rcode_t, s);
   }
-  return g.rcode_bytes == 1 ? run<float, uint8_t>(g, q, k, r_sort, r_race, code, rcode, s)
-                            : run<float, uint16_t>(g, q, k, r_sort, r_race, code, rcode, s);
+  return g.rcode_bytes == 1
+             ? run<float, uint8_t>(g, q, k, r_sort, r_race, code, rcode, rcode_t, s)
+             : run<float, uint16_t>(g, q, k, r_sort, r_race, code, rcode, rcode_t, s);
 }
 
 }  // namespace elsaa

@@ -70,8 +70,9 @@ template <int D, typename CodeT>
 __global__ void __launch_bounds__(kThreads)
 hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                const __nv_bfloat16* __restrict__ r_sort, const __nv_bfloat16* __restrict__ r_race,
-               int64_t rows_per_tensor, int sort_bits, int L, int kr, int P, int P16, int nbuf,
-               uint16_t* __restrict__ code, CodeT* __restrict__ rcode, uint32_t* __restrict__ err) {
+               int64_t rows_per_tensor, int N, int sort_bits, int L, int kr, int P, int P16,
+               int nbuf, uint16_t* __restrict__ code, CodeT* __restrict__ rcode,
+               CodeT* __restrict__ rcode_t, uint32_t* __restrict__ err) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   const uint32_t r_bytes = (uint32_t)P16 * D * 2;
@@ -204,6 +205,14 @@ hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         reinterpret_cast<uint4*>(gdst)[i] = reinterpret_cast<const uint4*>(ssrc)[i];
       for (int i = nvec * 16 + tid; i < rbytes; i += kThreads) gdst[i] = ssrc[i];
       for (int i = tid; i < nrows; i += kThreads) code[row0 + i] = st_code[i];
+      // table-major copy: thread r writes its row's code of every table;
+      // consecutive rows of a unit are consecutive along N
+      if (tid < nrows) {
+        const int64_t gr = row0 + tid;
+        const int64_t u = gr / N;
+        CodeT* dst = rcode_t + (size_t)u * L * N + (gr - u * N);
+        for (int t = 0; t < L; ++t) dst[(size_t)t * N] = st_rcode[tid * L + t];
+      }
     }
     if (nbuf == 1 && next < tiles) {
       load_tile<D>(s_a, q, k, rows_per_tensor, next);
@@ -221,7 +230,8 @@ hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
 
 template <int D, typename CodeT>
 cudaError_t run(const Geometry& g, const void* q, const void* k, const void* r_sort,
-                const void* r_race, uint16_t* code, void* rcode, uint32_t* err, cudaStream_t s) {
+                const void* r_race, uint16_t* code, void* rcode, void* rcode_t, uint32_t* err,
+                cudaStream_t s) {
   const HashShape h = hash_shape(g);
   cudaError_t e = cudaFuncSetAttribute(hash_tc_kernel<D, CodeT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)h.dyn);
@@ -245,7 +255,8 @@ cudaError_t run(const Geometry& g, const void* q, const void* k, const void* r_s
   hash_tc_kernel<D, CodeT><<<grid, kThreads, h.dyn, s>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
       static_cast<const __nv_bfloat16*>(r_sort), static_cast<const __nv_bfloat16*>(r_race), rows,
-      g.sort_bits, g.L, g.kr, h.P, h.P16, h.nbuf, code, static_cast<CodeT*>(rcode), err);
+      g.N, g.sort_bits, g.L, g.kr, h.P, h.P16, h.nbuf, code, static_cast<CodeT*>(rcode),
+      static_cast<CodeT*>(rcode_t), err);
   return cudaGetLastError();
 }
 
@@ -257,16 +268,16 @@ bool hash_tc_supported(const Geometry& g) {
   return h.P > 0 && h.dyn <= (uint32_t)kSmemLimit;
 }
 
-size_t hash_tc_scratch_bytes(const Geometry&) { return 0; }
-
 cudaError_t launch_hash_tc(const Geometry& g, const void* q, const void* k, const void* r_sort,
-                           const void* r_race, uint16_t* code, void* rcode, void*,
+                           const void* r_race, uint16_t* code, void* rcode, void* rcode_t,
                            uint32_t* err, cudaStream_t s) {
   if (g.d == 64)
-    return g.rcode_bytes == 1 ? run<64, uint8_t>(g, q, k, r_sort, r_race, code, rcode, err, s)
-                              : run<64, uint16_t>(g, q, k, r_sort, r_race, code, rcode, err, s);
-  return g.rcode_bytes == 1 ? run<128, uint8_t>(g, q, k, r_sort, r_race, code, rcode, err, s)
-                            : run<128, uint16_t>(g, q, k, r_sort, r_race, code, rcode, err, s);
+    return g.rcode_bytes == 1
+               ? run<64, uint8_t>(g, q, k, r_sort, r_race, code, rcode, rcode_t, err, s)
+               : run<64, uint16_t>(g, q, k, r_sort, r_race, code, rcode, rcode_t, err, s);
+  return g.rcode_bytes == 1
+             ? run<128, uint8_t>(g, q, k, r_sort, r_race, code, rcode, rcode_t, err, s)
+             : run<128, uint16_t>(g, q, k, r_sort, r_race, code, rcode, rcode_t, err, s);
 }
 
 }  // namespace elsaa

@@ -34,9 +34,10 @@ struct Geometry {
 
 // Byte offsets inside the saved buffer.
 struct SavedLayout {
-  size_t code, perm, rcode, race_count, race_sum, lse, o_sp, o_race, ctot, total;
+  size_t code, perm, rcode, rcode_t, race_count, race_sum, lse, o_sp, o_race, ctot, total;
   // code = [2][BH][N] u16 (queries then keys); perm = [2][BH][N] i32;
-  // rcode = [2][BH][N][L] (u8 or u16)
+  // rcode = [2][BH][N][L] (u8 or u16); rcode_t = the same codes table-major,
+  // [2][BH][L][N]
 };
 
 // Byte offsets inside the workspace.
@@ -65,13 +66,14 @@ WorkLayout work_layout(const Geometry& g);
 // ---- launchers (each returns cudaGetLastError() after enqueueing) ----------
 
 // SimHash codes of Q and K on CUDA cores (fp64 accumulation of exact products).
+// Codes go out twice: row-major (rcode) and table-major (rcode_t).
 cudaError_t launch_hash_simt(const Geometry& g, const void* q, const void* k, const void* r_sort,
-                             const void* r_race, uint16_t* code, void* rcode, cudaStream_t s);
+                             const void* r_race, uint16_t* code, void* rcode, void* rcode_t,
+                             cudaStream_t s);
 // SimHash codes on tcgen05 tensor cores (bf16 products, fp32 accumulation).
 cudaError_t launch_hash_tc(const Geometry& g, const void* q, const void* k, const void* r_sort,
-                           const void* r_race, uint16_t* code, void* rcode, void* scratch,
+                           const void* r_race, uint16_t* code, void* rcode, void* rcode_t,
                            uint32_t* err, cudaStream_t s);
-size_t hash_tc_scratch_bytes(const Geometry& g);
 bool hash_tc_supported(const Geometry& g);
 
 // Stable Sort-LSH order of the 2*BH code segments.
@@ -86,7 +88,9 @@ cudaError_t launch_unit_absmax(const Geometry& g, const void* vals, bool vals_f3
 // counts (optional) likewise, and (gtab non-null) a bf16 copy for the gathers.
 // vals_f32 selects fp32 values instead of dtype; absmax[bh] must bound |vals|
 // of unit bh; keep_sums = false leaves `sums` as scratch only.
-cudaError_t launch_race_build(const Geometry& g, const void* codes, const void* vals,
+// codes: [BH][N][L] row-major; codes_t: the same codes [BH][L][N] table-major.
+cudaError_t launch_race_build(const Geometry& g, const void* codes, const void* codes_t,
+                              const void* vals,
                               bool vals_f32, const float* absmax, float* sums, bool keep_sums,
                               __nv_bfloat16* gtab, int32_t* counts, uint32_t* err,
                               cudaStream_t s);

@@ -604,28 +604,25 @@ race_fuse_fwd_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q,
 
 // ---- bucket-sorted build --------------------------------------------------------
 //
-// One CTA per (unit, table).  The table's codes are cached in shared memory
-// and counted; a counting sort lists the keys bucket by bucket; then lane
-// groups walk equal shares of that list, gather each key's value row from
-// global memory (L2-resident for the unit) and add it into a register
-// accumulator until the bucket changes, when the run total goes to the
-// shared table with one integer add per column.
+// One CTA per (unit, table).  A counting sort lists the table's keys bucket
+// by bucket: each warp counts its contiguous share of the keys, a scan gives
+// every (warp, bucket) its slot range, and the warp scatters its keys through
+// its own cursors.  Lane groups then walk equal shares of the list, gather
+// each key's value row from global memory (L2-resident for the unit) and add
+// it in fp32 until the bucket changes, when the run total goes to the shared
+// table as one fixed-point integer per column.
 //
-// Exactness and determinism: every value is rounded once to the fixed-point
-// grid 2^-S, with |v| 2^S < 2^21 and C_max vmax 2^S < 2^30, so every partial
-// and every bucket total fits in int32 and integer addition makes the result
-// independent of the order in which keys reach a bucket.  The rounding uses
-// the float-add trick: for |x| < 2^22, the bits of fmaf(v, 2^S, 1.5 * 2^23)
-// are 0x4B400000 plus x rounded to the nearest integer (ties to even, as the
-// add rounds), so a run of n rows sums to its integer total plus n * 0x4B400000
-// modulo 2^32.
+// Determinism: a cursor is shared only by the lanes of one warp instruction,
+// whose conflicting shared-memory atomics the SM applies in a fixed order, so
+// the list is the same on every run and so is every run's fp32 total; run
+// totals are rounded once to the grid 2^-S (C_max vmax 2^S <= 2^30, so every
+// total fits in int32) and summed as integers, whose order does not matter.
 
 constexpr int kSortedThreads = 1024;
-constexpr uint32_t kMagicBits = 0x4B400000u;   // bits of 1.5 * 2^23
-constexpr float kMagic = 12582912.0f;           // 1.5 * 2^23
+constexpr int kSortedWarps = kSortedThreads / 32;
 
 struct SortedSmem {
-  size_t list, codes, tab, cnt, cur, misc, total;
+  size_t tab, list, codes, whist, bend, misc, total;   // whist: u32 [warps][NB]
 };
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
 __host__ __device__ inline SortedSmem sorted_smem(int N, int NB, int d, int code_bytes) {
@@ -633,25 +630,39 @@ __host__ __device__ inline SortedSmem sorted_smem(int N, int NB, int d, int code
   m.tab = 0;
   m.list = align16(m.tab + (size_t)NB * d * 4);
   m.codes = align16(m.list + (size_t)N * 2);
-  m.cnt = align16(m.codes + (size_t)N * code_bytes);
-  m.cur = align16(m.cnt + (size_t)NB * 4);
-  m.misc = align16(m.cur + (size_t)NB * 4);
+  m.whist = align16(m.codes + (size_t)N * code_bytes);
+  m.bend = align16(m.whist + (size_t)kSortedWarps * NB * 4);
+  m.misc = align16(m.bend + (size_t)NB * 4);
   m.total = m.misc + 256;   // [0] C_max, [1] bad code, [16..48) warp sums of the scan
   return m;
 }
 
-template <typename TV>
-ELSAA_DEV void add_fixed(uint32_t* acc, uint4 raw, float scale, const TV*) {
-  float v[16 / sizeof(TV)];
-  unpack16(raw, v, static_cast<const TV*>(nullptr));
+// a += b on two fp32 lanes at once
+ELSAA_DEV void add_f32x2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 x, y;\n\t"
+      "mov.b64 x, {%0, %1};\n\t"
+      "mov.b64 y, {%2, %3};\n\t"
+      "add.rn.f32x2 x, x, y;\n\t"
+      "mov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1));
+}
+ELSAA_DEV void add_row(float* acc, uint4 raw, const __nv_bfloat16*) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-  for (int i = 0; i < (int)(16 / sizeof(TV)); ++i)
-    acc[i] += __float_as_uint(fmaf(v[i], scale, kMagic));
+  for (int i = 0; i < 4; ++i)
+    add_f32x2(acc[2 * i], acc[2 * i + 1], __uint_as_float(w[i] << 16),
+              __uint_as_float(w[i] & 0xFFFF0000u));
+}
+ELSAA_DEV void add_row(float* acc, uint4 raw, const float*) {
+  add_f32x2(acc[0], acc[1], __uint_as_float(raw.x), __uint_as_float(raw.y));
+  add_f32x2(acc[2], acc[3], __uint_as_float(raw.z), __uint_as_float(raw.w));
 }
 
+// codes_t: table-major codes [BH][L][N]; grid (L, BH); NB buckets.
 template <typename TV, typename CodeT>
 __global__ void __launch_bounds__(kSortedThreads, 1)
-race_build_sorted_kernel(const CodeT* __restrict__ codes, const TV* __restrict__ vals, int N,
+race_build_sorted_kernel(const CodeT* __restrict__ codes_t, const TV* __restrict__ vals, int N,
                          int L, int NB, int d, const float* __restrict__ absmax,
                          float* __restrict__ sums, __nv_bfloat16* __restrict__ gtab,
                          int32_t* __restrict__ counts, uint32_t* __restrict__ err) {
@@ -661,51 +672,69 @@ race_build_sorted_kernel(const CodeT* __restrict__ codes, const TV* __restrict__
   int32_t* tab = reinterpret_cast<int32_t*>(sm + lay.tab);          // [NB][d] fixed point
   uint16_t* list = reinterpret_cast<uint16_t*>(sm + lay.list);      // keys, bucket by bucket
   CodeT* csm = reinterpret_cast<CodeT*>(sm + lay.codes);            // [N] this table's codes
-  int32_t* cnt = reinterpret_cast<int32_t*>(sm + lay.cnt);          // [NB]
-  int32_t* cur = reinterpret_cast<int32_t*>(sm + lay.cur);          // [NB] scatter cursors
+  uint32_t* whist = reinterpret_cast<uint32_t*>(sm + lay.whist);    // [warps][NB]
+  int32_t* bend = reinterpret_cast<int32_t*>(sm + lay.bend);        // [NB] end of each bucket
   int32_t* misc = reinterpret_cast<int32_t*>(sm + lay.misc);        // [0] C_max, [1] bad code
   int32_t* wsum = misc + 16;                                        // [32] scan warp sums
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t = blockIdx.x, bh = blockIdx.y;
+  const CodeT* ct = codes_t + ((size_t)bh * L + t) * N;
+  // warp w owns keys [k0, k1)
+  const int k0 = (int)((int64_t)N * warp / kSortedWarps);
+  const int k1 = (int)((int64_t)N * (warp + 1) / kSortedWarps);
+  uint32_t* wh = whist + (size_t)warp * NB;
 
+  // the table's codes to shared memory (16-byte copies when aligned)
+  {
+    const size_t bytes = (size_t)N * sizeof(CodeT);
+    if (((reinterpret_cast<uintptr_t>(ct) | bytes) & 15u) == 0) {
+      const uint4* src = reinterpret_cast<const uint4*>(ct);
+      uint4* dst = reinterpret_cast<uint4*>(csm);
+      for (int i = tid; i < (int)(bytes / 16); i += kSortedThreads) dst[i] = __ldcs(src + i);
+    } else {
+      for (int i = tid; i < N; i += kSortedThreads) csm[i] = ct[i];
+    }
+  }
   for (int i = tid; i < NB * d; i += kSortedThreads) tab[i] = 0;
-  for (int i = tid; i < NB; i += kSortedThreads) cnt[i] = 0;
+  for (int i = tid; i < kSortedWarps * NB; i += kSortedThreads) whist[i] = 0;
   if (tid < 2) misc[tid] = 0;
   __syncthreads();
 
-  // codes of table t and their bucket counts
-  const CodeT* cb = codes + (size_t)bh * N * L + t;
-  for (int j = tid; j < N; j += kSortedThreads) {
-    int c = (int)cb[(size_t)j * L];
-    if (c >= NB) {
-      misc[1] = 1;
-      c = 0;
-    }
-    csm[j] = (CodeT)c;
-    atomicAdd(cnt + c, 1);
+  // per-warp bucket counts (warp-private counters)
+  for (int j = k0 + lane; j < k1; j += 32) {
+    const int c = (int)csm[j];
+    if (c < NB) atomicAdd(wh + c, 1u);
+    else misc[1] = 1;
   }
   __syncthreads();
 
-  // exclusive scan of the counts (NB <= 1024: one bucket per thread)
+  // bucket totals, their exclusive scan, and each warp's starting slot
   {
-    const int c = tid < NB ? cnt[tid] : 0;
+    int c = 0;
+    if (tid < NB)
+      for (int w = 0; w < kSortedWarps; ++w) c += (int)whist[w * NB + tid];
     int x = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, x, o);
       if (lane >= o) x += y;
     }
-    if (lane == 31 && warp * 32 < NB) wsum[warp] = x;
+    if (lane == 31) wsum[warp] = x;
     int cm = c;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) cm = max(cm, __shfl_xor_sync(0xffffffffu, cm, o));
     if (lane == 0) atomicMax(misc, cm);
     __syncthreads();
     int before = 0;
-    for (int w = 0; w < warp && w * 32 < NB; ++w) before += wsum[w];
-    __syncthreads();
+    for (int w = 0; w < warp; ++w) before += wsum[w];
     if (tid < NB) {
-      cur[tid] = before + x - c;
+      uint32_t run = (uint32_t)(before + x - c);
+      bend[tid] = before + x;
+      for (int w = 0; w < kSortedWarps; ++w) {
+        const uint32_t h = whist[w * NB + tid];
+        whist[w * NB + tid] = run;
+        run += h;
+      }
       if (counts) counts[((size_t)bh * L + t) * NB + tid] = c;
     }
   }
@@ -714,11 +743,9 @@ race_build_sorted_kernel(const CodeT* __restrict__ codes, const TV* __restrict__
     if (tid == 0) raise_error(err, ERR_CHECK);
     return;
   }
-  // keys to their buckets' slots (order inside a bucket does not matter)
-  for (int j = tid; j < N; j += kSortedThreads) {
-    const int c = (int)csm[j];
-    list[atomicAdd(cur + c, 1)] = (uint16_t)j;
-  }
+  // scatter through the warp-private cursors: only lanes of one warp
+  // instruction share a cursor
+  for (int j = k0 + lane; j < k1; j += 32) list[atomicAdd(wh + (int)csm[j], 1u)] = (uint16_t)j;
   const float vmax = absmax[bh];
   if (!(vmax < 3.0e38f)) {
     if (tid == 0) raise_error(err, ERR_CHECK);
@@ -727,67 +754,64 @@ race_build_sorted_kernel(const CodeT* __restrict__ codes, const TV* __restrict__
   __syncthreads();
   const int cmax = misc[0];
   int S = 0;
-  if (cmax > 0 && vmax > 0.f) {
-    const int s1 = (int)floorf(log2f(1073741824.0f / ((float)cmax * vmax)));
-    const int s2 = (int)floorf(log2f(2097152.0f / vmax));
-    S = max(-100, min(100, min(s1, s2)));
-  }
+  if (cmax > 0 && vmax > 0.f)
+    S = max(-100, min(100, (int)floorf(log2f(1073741824.0f / ((float)cmax * vmax)))));
   const float scale = ldexpf(1.0f, S), inv_scale = ldexpf(1.0f, -S);
 
-  // lane groups of QL lanes walk equal shares of the list
+  // lane groups of QL lanes walk equal shares [p0, p1) of the list
   const int QL = d / EL;
   const int groups = kSortedThreads / QL;
   const int g = tid / QL, ql = tid % QL;
   const int p0 = (int)((int64_t)N * g / groups), p1 = (int)((int64_t)N * (g + 1) / groups);
   const TV* vb = vals + (size_t)bh * N * d + ql * EL;
-  uint32_t acc[EL];
+  float acc[EL];
 #pragma unroll
-  for (int e = 0; e < EL; ++e) acc[e] = 0u;
-  int run_code = -1, run_n = 0;
+  for (int e = 0; e < EL; ++e) acc[e] = 0.f;
+  // the bucket holding position p0: the first b with bend[b] > p0
+  int b = 0;
+  if (p0 < p1) {
+    int lo = 0, hi = NB - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (bend[mid] > p0) hi = mid;
+      else lo = mid + 1;
+    }
+    b = lo;
+  }
+  int b_end = p0 < p1 ? bend[b] : 0;
+  bool any = false;
   auto flush = [&]() {
-    if (run_n > 0) {
-      const uint32_t bias = (uint32_t)run_n * kMagicBits;
-      int32_t* dst = tab + (size_t)run_code * d + ql * EL;
+    if (any) {
+      uint32_t* dst = reinterpret_cast<uint32_t*>(tab + (size_t)b * d + ql * EL);
 #pragma unroll
       for (int e = 0; e < EL; ++e) {
-        atomicAdd(reinterpret_cast<uint32_t*>(dst + e), acc[e] - bias);
-        acc[e] = 0u;
+        atomicAdd(dst + e, (uint32_t)__float2int_rn(acc[e] * scale));
+        acc[e] = 0.f;
       }
     }
-    run_n = 0;
+    any = false;
   };
-  constexpr int U = 4;
-  int p = p0;
-  for (; p + U <= p1; p += U) {
-    int key[U], code[U];
-    uint4 raw[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      key[u] = list[p + u];
-      code[u] = (int)csm[key[u]];
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) raw[u] = __ldg(reinterpret_cast<const uint4*>(vb + (size_t)key[u] * d));
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (code[u] != run_code) {
-        flush();
-        run_code = code[u];
-      }
-      add_fixed(acc, raw[u], scale, vb);
-      ++run_n;
-    }
-  }
-  for (; p < p1; ++p) {
-    const int k1 = list[p], c1 = (int)csm[k1];
-    const uint4 r1 = __ldg(reinterpret_cast<const uint4*>(vb + (size_t)k1 * d));
-    if (c1 != run_code) {
+  auto step = [&](int pos, uint4 raw) {
+    if (pos >= b_end) {
       flush();
-      run_code = c1;
+      do b_end = bend[++b]; while (pos >= b_end);
     }
-    add_fixed(acc, r1, scale, vb);
-    ++run_n;
+    add_row(acc, raw, vb);
+    any = true;
+  };
+  auto row = [&](int key) { return __ldg(reinterpret_cast<const uint4*>(vb + (size_t)key * d)); };
+  int p = p0;
+  for (; p < p1 && (p & 3) != 0; ++p) step(p, row(list[p]));
+  for (; p + 4 <= p1; p += 4) {
+    const uint2 k4 = *reinterpret_cast<const uint2*>(list + p);   // four u16 keys
+    const uint4 r0 = row((int)(k4.x & 0xFFFFu)), r1 = row((int)(k4.x >> 16));
+    const uint4 r2 = row((int)(k4.y & 0xFFFFu)), r3 = row((int)(k4.y >> 16));
+    step(p, r0);
+    step(p + 1, r1);
+    step(p + 2, r2);
+    step(p + 3, r3);
   }
+  for (; p < p1; ++p) step(p, row(list[p]));
   flush();
   __syncthreads();
 
@@ -1025,7 +1049,8 @@ BuildShape build_shape(const Geometry& g) {
 }
 
 template <typename TV, typename CodeT>
-cudaError_t build(const Geometry& g, const void* codes, const void* vals, const float* absmax,
+cudaError_t build(const Geometry& g, const void* codes, const void* codes_t, const void* vals,
+                  const float* absmax,
                   float* sums, bool keep_sums, __nv_bfloat16* gtab, int32_t* counts,
                   uint32_t* err, cudaStream_t s) {
   {
@@ -1039,7 +1064,7 @@ cudaError_t build(const Geometry& g, const void* codes, const void* vals, const 
           cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)m.total);
       if (e != cudaSuccess) return e;
       kernel<<<dim3(g.L, g.BH), kSortedThreads, m.total, s>>>(
-          static_cast<const CodeT*>(codes), static_cast<const TV*>(vals), g.N, g.L, g.NB, g.d,
+          static_cast<const CodeT*>(codes_t), static_cast<const TV*>(vals), g.N, g.L, g.NB, g.d,
           absmax, keep_sums ? sums : nullptr, gtab, counts, err);
       return cudaGetLastError();
     }
@@ -1225,19 +1250,20 @@ cudaError_t launch_unit_absmax(const Geometry& g, const void* vals, bool vals_f3
   return cudaGetLastError();
 }
 
-cudaError_t launch_race_build(const Geometry& g, const void* codes, const void* vals,
+cudaError_t launch_race_build(const Geometry& g, const void* codes, const void* codes_t,
+                              const void* vals,
                               bool vals_f32, const float* absmax, float* sums, bool keep_sums,
                               __nv_bfloat16* gtab, int32_t* counts, uint32_t* err,
                               cudaStream_t s) {
   if (vals_f32 || !g.bf16)
     return g.rcode_bytes == 1
-               ? build<float, uint8_t>(g, codes, vals, absmax, sums, keep_sums, gtab, counts, err, s)
-               : build<float, uint16_t>(g, codes, vals, absmax, sums, keep_sums, gtab, counts, err,
+               ? build<float, uint8_t>(g, codes, codes_t, vals, absmax, sums, keep_sums, gtab, counts, err, s)
+               : build<float, uint16_t>(g, codes, codes_t, vals, absmax, sums, keep_sums, gtab, counts, err,
                                         s);
   return g.rcode_bytes == 1
-             ? build<__nv_bfloat16, uint8_t>(g, codes, vals, absmax, sums, keep_sums, gtab, counts,
+             ? build<__nv_bfloat16, uint8_t>(g, codes, codes_t, vals, absmax, sums, keep_sums, gtab, counts,
                                              err, s)
-             : build<__nv_bfloat16, uint16_t>(g, codes, vals, absmax, sums, keep_sums, gtab,
+             : build<__nv_bfloat16, uint16_t>(g, codes, codes_t, vals, absmax, sums, keep_sums, gtab,
                                               counts, err, s);
 }
 

@@ -57,8 +57,8 @@ def test_workloads_validate_and_size(name):
     bhn = w.B * w.H * w.N
     esz = 2 if w.dtype == "bf16" else 4
     saved = B.saved_bytes(p)
-    # codes, perms, RACE codes, tables, lse, O_sp, O_race, Ctot
-    expect = (2 * bhn * 2 + 2 * bhn * 4 + 2 * bhn * w.race_tables * (1 if w.race_bits <= 8 else 2)
+    # codes, perms, RACE codes (row-major and table-major), tables, lse, O_sp, O_race, Ctot
+    expect = (2 * bhn * 2 + 2 * bhn * 4 + 4 * bhn * w.race_tables * (1 if w.race_bits <= 8 else 2)
               + w.B * w.H * w.race_tables * (1 << w.race_bits) * (4 + 4 * w.d)
               + bhn * 4 * 2 + 2 * bhn * w.d * esz)
     assert expect <= saved <= expect + 256 * 16

@@ -74,3 +74,18 @@ def test_two_pass_sort_and_wide_race_codes(cuda_device):
 def test_zero_race_bits(cuda_device):
     w = WORKLOADS["iid-4k"].replace(B=1, H=1, N=512, race_bits=0, chunk=64)
     _run(w, backward=True)
+
+
+@pytest.mark.parametrize("name", ["text-32k", "vision-16k"])
+def test_bitwise_reproducible(cuda_device, name):
+    """Two runs on the same inputs give identical bits: every reduction in the
+    path (table builds, sums, atomics into accumulators) has a fixed order or
+    is exact."""
+    w = small(WORKLOADS[name], B=1, H=2, N=4096)
+    inp = make_inputs(w, with_dy=True)
+    a = run_gpu(w, inp, backward=True)
+    b = run_gpu(w, inp, backward=True)
+    for key in ("y", "dq", "dk", "dv", "dgate_w", "dgate_b", "dlambda"):
+        assert torch.equal(a[key], b[key]), key
+    for key in ("race_sum", "race_count", "lse_sp", "o_sp", "o_race"):
+        assert torch.equal(a["views"][key], b["views"][key]), key
