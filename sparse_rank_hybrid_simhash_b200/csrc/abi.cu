@@ -306,7 +306,12 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
                                    dv_acc, s));
   ELSAA_TRY(mark(events, 2, s));
   // 3. sparse branch backward, 4. outputs
-  if (g.tc_attn && attn_bwd2_supported(g)) {
+  if (g.tc_attn && attn_bwd3_supported(g)) {
+    // writes dq itself: gate part (dq_acc) + sparse part, in the data dtype
+    ELSAA_TRY(launch_attn_bwd3(g, q, k, v, perm, perm + bhn, d_o, lse, dprime, dv_acc, dq_acc,
+                               dq, dk, dv, (uint32_t*)(w + wl.err), s));
+    ELSAA_TRY(mark(events, 3, s));
+  } else if (g.tc_attn && attn_bwd2_supported(g)) {
     ELSAA_TRY(launch_attn_bwd2(g, q, k, v, perm, perm + bhn, d_o, lse, dprime, dv_acc, dq_acc,
                                dk, dv, (uint32_t*)(w + wl.err), s));
     ELSAA_TRY(mark(events, 3, s));
@@ -348,7 +353,8 @@ elsaa_status elsaa_kernel_launches(const elsaa_params* p, int32_t* fwd, int32_t*
   // hash 1, sort 3 per pass, |V| max 1 + RACE build 1, sparse 1, RACE gather + fusion 1
   *fwd = 1 + 3 * g.sort_passes + 2 + 1 + 1;
   // fusion backward 1, RACE build 1 + gather 1, sparse 1 (+ casts), reduction 1
-  *bwd = 1 + 2 + (g.tc_attn ? 1 + 1 : 1 + 3) + 1;
+  const int sparse = g.tc_attn ? (attn_bwd3_supported(g) ? 1 : 1 + 1) : 1 + 3;
+  *bwd = 1 + 2 + sparse + 1;
   return ELSAA_OK;
 }
 

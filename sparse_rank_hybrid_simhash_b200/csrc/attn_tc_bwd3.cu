@@ -1,0 +1,569 @@
+// Backward of the exact sparse branch as a persistent warp-specialized tcgen05
+// pipeline (bf16, d = 64, chunk c <= 128 with 128 % c == 0).
+//
+// Mathematics ("Two Efficient Attentions, One Denominator Problem", section
+// "Two efficient branches can still be mis-scaled": the sparse branch is exact
+// attention over each query's Sort-LSH window, and its log-mass feeds the
+// fusion):
+//   P = exp(scale s - lse), dS = P (dO V^T - D'),
+//   dV = P^T dO,  dK = scale dS^T Q,  dQ = scale dS K.
+//
+// Work: key tiles of 128 sorted keys, key tile kb covering keys [128 kb,
+// 128 kb + 128).  The keys of tile kb are seen by the queries of query block
+// kb ("own") and by the first c queries of block kb + 1 ("next").  Each CTA
+// takes a contiguous run of key tiles, so consecutive tiles share a query
+// block.  The dQ of block qb has two contributions, from tiles qb - 1 and
+// qb; both are accumulated in TMEM by the CTA that owns tile qb and written
+// once, in bf16, together with the gate part of dQ already in dq_gate.  For
+// the first tile of a run the contribution of tile qb - 1 belongs to another
+// CTA; this CTA recomputes it (a "pre" pair: dQ only), and the CTA owning
+// tile qb - 1 skips the dQ of its last "next" pair.  No atomics, and every
+// output element is written by exactly one thread.
+//
+// Roles (320 threads, one CTA per SM):
+//   warp 0      producer: cp.async gathers of K/V key tiles (two-slot ring)
+//               and Q/dO query blocks with their lse and D' (two-slot ring)
+//   warp 1      MMA issuer (one thread) and TMEM owner; for pair p it issues
+//               S^T/dP^T of pair p + 1 as soon as P^T/dS^T of pair p are in
+//               shared memory, then dV, dK, dQ of pair p
+//   warps 2..9  elementwise: warp w reaches TMEM lanes 32 (w % 4) .. +31 and
+//               takes half of the query columns; P^T and dS^T (bf16) to
+//               shared memory; then the dQ flush of a finished query block
+//               and the dV / dK write-out of a finished key tile
+// TMEM: S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384),
+//       dQ [384,448) and [448,512) for alternating query blocks.
+// Every wait is bounded; a timeout records ERR_TIMEOUT and every role leaves
+// its loop, frees TMEM and returns.
+#include <math.h>
+
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace elsaa {
+namespace {
+
+using namespace tc;
+
+constexpr int D = 64;
+constexpr int kTile = 128;
+constexpr int kThreads = 320;
+constexpr int kEwThreads = 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTS = 0, kTdP = 128, kTdV = 256, kTdK = 320, kTdQ = 384;
+
+struct Lay3 {
+  static constexpr uint32_t kSub = 128 * 128;               // 128 rows x 64 bf16
+  static constexpr uint32_t kKv = 0;                        // [2][K | V]
+  static constexpr uint32_t kKvSlot = 2 * kSub;
+  static constexpr uint32_t kQ = kKv + 2 * kKvSlot;         // [2][Q | dO]
+  static constexpr uint32_t kQSlot = 2 * kSub;
+  static constexpr uint32_t kPT = kQ + 2 * kQSlot;          // P^T  [128 keys][128 queries]
+  static constexpr uint32_t kDST = kPT + 2 * kSub;          // dS^T [128 keys][128 queries]
+  static constexpr uint32_t kKidx = kDST + 2 * kSub;        // [2][128] key tokens
+  static constexpr uint32_t kQidx = kKidx + 2 * 128 * 4;    // [2][128] query tokens
+  static constexpr uint32_t kLse = kQidx + 2 * 128 * 4;     // [2][128] lse (log2 units once used)
+  static constexpr uint32_t kDpr = kLse + 2 * 128 * 4;      // [2][128] D'
+  static constexpr uint32_t kBar = kDpr + 2 * 128 * 4;
+  static constexpr uint32_t kDyn = kBar + 256;
+};
+
+struct Bars3 {
+  uint64_t full_kv[2], empty_kv[2], full_q[2], empty_q[2];
+  uint64_t s_full, p_full, pd_free, kvacc_full, dq_full[2];
+  uint32_t tmem;
+};
+static_assert(sizeof(Bars3) <= 256, "barrier block");
+
+// One (key tile, query block) pair of the run.
+struct Pair {
+  int bh, kb, qb;
+  int64_t kvs, qs;       // ring sequence numbers of the key tile and the query block
+  int64_t tile;          // tile index in the run (-1: pre pair)
+  int nq;                // query columns that can see the tile
+  bool kv, dq, dq_acc;   // adds to dV/dK; adds to dQ; dQ adds to an earlier contribution
+  bool flush;            // the query block's dQ is complete after this pair
+  bool first_of_tile, last_of_tile, release_kv, release_q, q_first;
+};
+
+struct Run3 {
+  int64_t begin, count;
+  int T, chunk;
+  int extra;   // 1: the run starts with a pre pair
+  ELSAA_DEV int bh_of(int64_t j) const { return (int)((begin + j) / T); }
+  ELSAA_DEV int kb_of(int64_t j) const { return (int)((begin + j) % T); }
+  ELSAA_DEV bool has_next(int64_t j) const { return kb_of(j) + 1 < T; }
+};
+
+// Enumerates the run's pairs: [pre], then per tile own and (if any) next.
+struct PairIter {
+  const Run3* r;
+  int64_t j;
+  int kind;   // 0 pre, 1 own, 2 next
+  ELSAA_DEV void init(const Run3* run) {
+    r = run;
+    j = 0;
+    kind = run->extra ? 0 : 1;
+  }
+  ELSAA_DEV bool done() const { return j >= r->count; }
+  ELSAA_DEV void advance() {
+    if (kind == 0) kind = 1;
+    else if (kind == 1 && r->has_next(j)) kind = 2;
+    else { ++j; kind = 1; }
+  }
+  ELSAA_DEV Pair get() const {
+    Pair p;
+    p.bh = r->bh_of(j);
+    const int kb = r->kb_of(j);
+    if (kind == 0) {
+      p.kb = kb - 1; p.qb = kb; p.kvs = 0; p.qs = 0; p.tile = -1; p.nq = r->chunk;
+      p.kv = false; p.dq = true; p.dq_acc = false; p.flush = false;
+      p.first_of_tile = true; p.last_of_tile = true; p.release_kv = true; p.release_q = false;
+      p.q_first = true;
+    } else if (kind == 1) {
+      p.kb = kb; p.qb = kb; p.kvs = j + r->extra; p.qs = j; p.tile = j; p.nq = kTile;
+      p.kv = true; p.dq = true;
+      p.dq_acc = j == 0 ? r->extra != 0 : r->has_next(j - 1);
+      p.flush = true;
+      p.first_of_tile = true; p.last_of_tile = !r->has_next(j);
+      p.release_kv = p.last_of_tile; p.release_q = true;
+      p.q_first = j == 0 ? r->extra == 0 : !r->has_next(j - 1);
+    } else {
+      p.kb = kb; p.qb = kb + 1; p.kvs = j + r->extra; p.qs = j + 1; p.tile = j; p.nq = r->chunk;
+      p.kv = true; p.dq = j + 1 < r->count; p.dq_acc = false; p.flush = false;
+      p.first_of_tile = false; p.last_of_tile = true; p.release_kv = true;
+      p.release_q = j + 1 == r->count; p.q_first = true;
+    }
+    return p;
+  }
+};
+
+ELSAA_DEV uint32_t pack2(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+ELSAA_DEV float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+ELSAA_DEV void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+
+ELSAA_DEV void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+ELSAA_DEV void ew_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEwThreads) : "memory"); }
+
+// Barrier among the elementwise warps that ANDs a flag over them.
+ELSAA_DEV bool ew_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kEwThreads)
+      : "memory");
+  return r != 0;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                 const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ perm_q,
+                 const int32_t* __restrict__ perm_k, const __nv_bfloat16* __restrict__ d_o,
+                 const float* __restrict__ lse, const float* __restrict__ dprime,
+                 const float* __restrict__ dv_race, const float* __restrict__ dq_gate, int BH,
+                 int N, int chunk, float scale, float scale_log2, __nv_bfloat16* __restrict__ dq,
+                 __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+                 uint32_t* __restrict__ err) {
+  using Lay = Lay3;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  Bars3* bars = reinterpret_cast<Bars3*>(smem + Lay::kBar);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if ((sbase & 1023u) != 0) {
+    if (tid == 0) raise_error(err, ERR_CHECK);
+    return;
+  }
+  Run3 run;
+  run.T = N / kTile;
+  run.chunk = chunk;
+  {
+    const int64_t ntiles = (int64_t)BH * run.T;
+    run.begin = ntiles * blockIdx.x / gridDim.x;
+    run.count = ntiles * (blockIdx.x + 1) / gridDim.x - run.begin;
+    run.extra = (run.count > 0 && run.begin % run.T != 0) ? 1 : 0;
+  }
+  int32_t* s_kidx = reinterpret_cast<int32_t*>(smem + Lay::kKidx);
+  int32_t* s_qidx = reinterpret_cast<int32_t*>(smem + Lay::kQidx);
+  float* s_lse = reinterpret_cast<float*>(smem + Lay::kLse);
+  float* s_dpr = reinterpret_cast<float*>(smem + Lay::kDpr);
+
+  if (tid == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->full_kv[s], 64);   // 32 cp.async arrivals + 32 plain arrivals
+      mbar_init(&bars->empty_kv[s], 1);
+      mbar_init(&bars->full_q[s], 64);
+      mbar_init(&bars->empty_q[s], 1);
+      mbar_init(&bars->dq_full[s], 1);
+    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->p_full, kEwThreads);
+    mbar_init(&bars->pd_free, 1);
+    mbar_init(&bars->kvacc_full, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem, kTmemCols);
+    tmem_relinquish();
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = bars->tmem;
+  bool ok = true;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    // Lane l handles rows l, l + 32, l + 64, l + 96 of a tile or block; rows
+    // are gathered 4 per warp instruction (8 lanes per row, 16 bytes each).
+    const int ch = lane & 7;
+    auto load_kv = [&](int64_t n, int bh, int kb) -> bool {
+      const size_t unit = (size_t)bh * N;
+      int idx[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) idx[j] = perm_k[unit + (size_t)kb * kTile + lane + 32 * j];
+      const int s = (int)(n & 1);
+      if (n >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars->empty_kv[s],
+                                                      (uint32_t)(((n >> 1) - 1) & 1), err)))
+        return false;
+      const uint32_t kst = sbase + Lay::kKv + s * Lay::kKvSlot;
+      const __nv_bfloat16* kb_ = k + unit * D;
+      const __nv_bfloat16* vb_ = v + unit * D;
+#pragma unroll
+      for (int it = 0; it < kTile / 4; ++it) {
+        const int row = 4 * it + (lane >> 3);
+        const int tok = __shfl_sync(0xffffffffu, idx[it >> 3], row & 31);
+        const size_t src = (size_t)tok * D + ch * 8;
+        cp_async16(kst + sw128_off(row, ch), kb_ + src, 16);
+        cp_async16(kst + Lay::kSub + sw128_off(row, ch), vb_ + src, 16);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s_kidx[s * 128 + lane + 32 * j] = idx[j];
+      cp_async_arrive(&bars->full_kv[s]);
+      mbar_arrive(&bars->full_kv[s]);
+      return true;
+    };
+    auto load_q = [&](int64_t n, int bh, int qb) -> bool {
+      const size_t unit = (size_t)bh * N;
+      int idx[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) idx[j] = perm_q[unit + (size_t)qb * kTile + lane + 32 * j];
+      const int s = (int)(n & 1);
+      if (n >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars->empty_q[s],
+                                                      (uint32_t)(((n >> 1) - 1) & 1), err)))
+        return false;
+      const uint32_t qst = sbase + Lay::kQ + s * Lay::kQSlot;
+      const __nv_bfloat16* qb_ = q + unit * D;
+      const __nv_bfloat16* ob_ = d_o + unit * D;
+#pragma unroll
+      for (int it = 0; it < kTile / 4; ++it) {
+        const int row = 4 * it + (lane >> 3);
+        const int tok = __shfl_sync(0xffffffffu, idx[it >> 3], row & 31);
+        const size_t src = (size_t)tok * D + ch * 8;
+        cp_async16(qst + sw128_off(row, ch), qb_ + src, 16);
+        cp_async16(qst + Lay::kSub + sw128_off(row, ch), ob_ + src, 16);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = lane + 32 * j;
+        cp_async4(smem_u32(s_lse + s * 128 + r), lse + unit + idx[j]);
+        cp_async4(smem_u32(s_dpr + s * 128 + r), dprime + unit + idx[j]);
+        s_qidx[s * 128 + r] = idx[j];
+      }
+      cp_async_arrive(&bars->full_q[s]);
+      mbar_arrive(&bars->full_q[s]);
+      return true;
+    };
+    if (run.count > 0) {
+      const int bh0 = run.bh_of(0), kb0 = run.kb_of(0);
+      if (run.extra) ok = load_kv(0, bh0, kb0 - 1);
+      if (ok) ok = load_q(0, bh0, kb0);
+      const int64_t nq_blocks = run.count + (run.has_next(run.count - 1) ? 1 : 0);
+      for (int64_t j = 0; j < run.count && ok; ++j) {
+        ok = load_kv(j + run.extra, run.bh_of(j), run.kb_of(j));
+        if (!ok) break;
+        if (j + 1 < nq_blocks) {
+          // query block j + 1: the own block of tile j + 1, or the next block of the last tile
+          const bool last = j + 1 == run.count;
+          ok = load_q(j + 1, last ? run.bh_of(j) : run.bh_of(j + 1),
+                      last ? run.kb_of(j) + 1 : run.kb_of(j + 1));
+        }
+      }
+    }
+    cp_async_wait_all();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0 && run.count > 0) {
+      int64_t kv_seen = 0, q_seen = 0;
+      auto wait_data = [&](const Pair& p) -> bool {
+        for (; kv_seen <= p.kvs; ++kv_seen)
+          if (!mbar_wait(&bars->full_kv[kv_seen & 1], (uint32_t)((kv_seen >> 1) & 1), err))
+            return false;
+        for (; q_seen <= p.qs; ++q_seen)
+          if (!mbar_wait(&bars->full_q[q_seen & 1], (uint32_t)((q_seen >> 1) & 1), err))
+            return false;
+        fence_async_smem();   // cp.async data -> tensor core
+        fence_after();
+        return true;
+      };
+      auto kv_slot = [&](int64_t n) { return sbase + Lay::kKv + (uint32_t)(n & 1) * Lay::kKvSlot; };
+      auto q_slot = [&](int64_t n) { return sbase + Lay::kQ + (uint32_t)(n & 1) * Lay::kQSlot; };
+      auto issue_s = [&](const Pair& p) {   // S^T = K Q^T, dP^T = V dO^T
+        const uint32_t idesc = idesc_bf16(128, p.nq, false, false);
+        const uint32_t ks = kv_slot(p.kvs), qs = q_slot(p.qs);
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s)
+          mma_bf16_ss(tmem + kTS, sw128_desc(ks + s * 32, 16, 1024),
+                      sw128_desc(qs + s * 32, 16, 1024), idesc, s > 0);
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s)
+          mma_bf16_ss(tmem + kTdP, sw128_desc(ks + Lay::kSub + s * 32, 16, 1024),
+                      sw128_desc(qs + Lay::kSub + s * 32, 16, 1024), idesc, s > 0);
+        mma_commit(&bars->s_full);
+      };
+      PairIter it;
+      it.init(&run);
+      Pair cur = it.get();
+      ok = wait_data(cur);
+      if (ok) issue_s(cur);
+      for (int64_t pi = 0; ok; ++pi) {
+        ok = mbar_wait(&bars->p_full, (uint32_t)(pi & 1), err);
+        if (!ok) break;
+        fence_after();
+        PairIter nx = it;
+        nx.advance();
+        const bool more = !nx.done();
+        Pair nxt;
+        if (more) {
+          nxt = nx.get();
+          ok = wait_data(nxt);
+          if (!ok) break;
+          issue_s(nxt);
+        }
+        const uint32_t ks = kv_slot(cur.kvs), qs = q_slot(cur.qs);
+        if (cur.kv) {
+          const uint32_t id_kv = idesc_bf16(128, D, false, true);
+          for (int s = 0; s < cur.nq / 16; ++s) {
+            const uint32_t aoff = (s >> 2) * Lay::kSub + (s & 3) * 32;
+            const uint32_t acc = (!cur.first_of_tile || s > 0) ? 1u : 0u;
+            mma_bf16_ss(tmem + kTdV, sw128_desc(sbase + Lay::kPT + aoff, 16, 1024),
+                        sw128_desc(qs + Lay::kSub + s * 2048, Lay::kSub, 1024), id_kv, acc);
+            mma_bf16_ss(tmem + kTdK, sw128_desc(sbase + Lay::kDST + aoff, 16, 1024),
+                        sw128_desc(qs + s * 2048, Lay::kSub, 1024), id_kv, acc);
+          }
+        }
+        if (cur.dq) {
+          const uint32_t id_q = idesc_bf16(128, D, true, true);
+          const uint32_t dqc = kTdQ + (uint32_t)(cur.qs & 1) * D;
+#pragma unroll
+          for (int s = 0; s < kTile / 16; ++s)
+            mma_bf16_ss(tmem + dqc, sw128_desc(sbase + Lay::kDST + s * 2048, Lay::kSub, 1024),
+                        sw128_desc(ks + s * 2048, Lay::kSub, 1024), id_q,
+                        (cur.dq_acc || s > 0) ? 1u : 0u);
+        }
+        mma_commit(&bars->pd_free);
+        if (cur.release_kv) mma_commit(&bars->empty_kv[cur.kvs & 1]);
+        if (cur.release_q) mma_commit(&bars->empty_q[cur.qs & 1]);
+        if (cur.kv && cur.last_of_tile) mma_commit(&bars->kvacc_full);
+        if (cur.flush) mma_commit(&bars->dq_full[cur.qs & 1]);
+        if (!more) break;
+        it = nx;
+        cur = nxt;
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- elementwise + epilogues
+    const int ew = tid - 64;                           // 0 .. 255
+    const int quarter = warp & 3, half = (warp - 2) >> 2;
+    const int row = 32 * quarter + lane;               // TMEM lane
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    const bool masked = chunk < kTile;
+    int lc = 0;
+    while ((1 << lc) < chunk) ++lc;
+    uint32_t flush_parity = 0u;   // bit b: parity of the next completion of dQ buffer b
+    int64_t ntile = 0;
+    int key_tok = 0, flush_tok = 0;
+    PairIter it;
+    it.init(&run);
+    for (int64_t pi = 0; run.count > 0 && !it.done(); ++pi, it.advance()) {
+      const Pair p = it.get();
+      const size_t unit = (size_t)p.bh * N;
+      const int qslot = (int)(p.qs & 1), kslot = (int)(p.kvs & 1);
+      ok = ew_all(mbar_wait(&bars->s_full, (uint32_t)(pi & 1), err) &&
+                  mbar_wait(&bars->full_q[qslot], (uint32_t)((p.qs >> 1) & 1), err) &&
+                  mbar_wait(&bars->full_kv[kslot], (uint32_t)((p.kvs >> 1) & 1), err));
+      if (!ok) break;
+      fence_after();
+      float* ls = s_lse + qslot * 128;
+      const float* dps = s_dpr + qslot * 128;
+      if (p.q_first) {   // the block's lse to log2 units, once per block
+        if (ew < 128) ls[ew] *= 1.4426950408889634f;
+        ew_sync();
+      }
+      if (p.first_of_tile && p.kv) key_tok = s_kidx[kslot * 128 + row];
+      if (p.flush) flush_tok = s_qidx[qslot * 128 + row];
+      // visible query columns of this key row: ranks [i c, (i + 2) c)
+      const int key_chunk = (p.kb * kTile + row) >> lc;
+      const int lo = (key_chunk << lc) - p.qb * kTile, hi = lo + 2 * chunk;
+      const int cend = min(hi, p.nq);
+      uint32_t pw[2][16], dw[2][16];
+#pragma unroll
+      for (int cb = 0; cb < 2; ++cb) {
+        const int c0 = half * 64 + cb * 32;
+        float sv[32], dp[32];
+        tmem_ld32(tmem + kTS + lane_off + c0, sv);
+        tmem_ld32(tmem + kTdP + lane_off + c0, dp);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float2 l2 = *reinterpret_cast<const float2*>(ls + c0 + i);
+          const float2 d2 = *reinterpret_cast<const float2*>(dps + c0 + i);
+          float p0 = ex2(fmaf(sv[i], scale_log2, -l2.x));
+          float p1 = ex2(fmaf(sv[i + 1], scale_log2, -l2.y));
+          if (masked || p.nq < kTile) {
+            const int col = c0 + i;
+            p0 = (col >= lo && col < cend) ? p0 : 0.f;
+            p1 = (col + 1 >= lo && col + 1 < cend) ? p1 : 0.f;
+          }
+          pw[cb][i >> 1] = pack2(p0, p1);
+          dw[cb][i >> 1] = pack2(p0 * (dp[i] - d2.x), p1 * (dp[i + 1] - d2.y));
+        }
+      }
+      if (pi >= 1) {   // the MMAs of the previous pair are done with P^T / dS^T
+        ok = ew_all(mbar_wait(&bars->pd_free, (uint32_t)((pi - 1) & 1), err));
+        if (!ok) break;
+      }
+#pragma unroll
+      for (int cb = 0; cb < 2; ++cb) {
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          const int col = half * 64 + cb * 32 + q8 * 8;
+          const uint32_t off = (col >> 6) * Lay::kSub + sw128_off(row, (col & 63) >> 3);
+          if (p.kv)
+            *reinterpret_cast<uint4*>(smem + Lay::kPT + off) =
+                make_uint4(pw[cb][q8 * 4], pw[cb][q8 * 4 + 1], pw[cb][q8 * 4 + 2], pw[cb][q8 * 4 + 3]);
+          *reinterpret_cast<uint4*>(smem + Lay::kDST + off) =
+              make_uint4(dw[cb][q8 * 4], dw[cb][q8 * 4 + 1], dw[cb][q8 * 4 + 2], dw[cb][q8 * 4 + 3]);
+        }
+      }
+      fence_async_smem();
+      fence_before();
+      mbar_arrive(&bars->p_full);
+
+      if (p.flush) {
+        // dQ of query block qb: TMEM lane = query row, this warp's 32 columns
+        const int b = (int)(p.qs & 1);
+        const float* gate = dq_gate + (unit + flush_tok) * D + half * 32;
+        float4 g4[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) g4[i] = reinterpret_cast<const float4*>(gate)[i];
+        ok = ew_all(mbar_wait(&bars->dq_full[b], (flush_parity >> b) & 1u, err));
+        if (!ok) break;
+        flush_parity ^= 1u << b;
+        fence_after();
+        float g[32];
+        tmem_ld32(tmem + kTdQ + b * D + lane_off + half * 32, g);
+        tmem_ld_wait();
+        __nv_bfloat16* out = dq + (unit + flush_tok) * D + half * 32;
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          const float4 a = g4[2 * q8], c = g4[2 * q8 + 1];
+          const float* x = g + q8 * 8;
+          *reinterpret_cast<uint4*>(out + q8 * 8) =
+              make_uint4(pack2(a.x + scale * x[0], a.y + scale * x[1]),
+                         pack2(a.z + scale * x[2], a.w + scale * x[3]),
+                         pack2(c.x + scale * x[4], c.y + scale * x[5]),
+                         pack2(c.z + scale * x[6], c.w + scale * x[7]));
+        }
+        fence_before();
+      }
+      if (p.kv && p.last_of_tile) {
+        // dV (+ the RACE branch's dv) from half 0, dK from half 1, of this key row
+        ok = ew_all(mbar_wait(&bars->kvacc_full, (uint32_t)(ntile & 1), err));
+        if (!ok) break;
+        ++ntile;
+        fence_after();
+        const uint32_t col = half == 0 ? kTdV : kTdK;
+        __nv_bfloat16* out = (half == 0 ? dv : dk) + (unit + key_tok) * D;
+        const float* add = dv_race + (unit + key_tok) * D;
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          float gv[32];
+          tmem_ld32(tmem + col + lane_off + c0, gv);
+          tmem_ld_wait();
+          if (half == 0) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const float4 a = *reinterpret_cast<const float4*>(add + c0 + e);
+              gv[e] += a.x; gv[e + 1] += a.y; gv[e + 2] += a.z; gv[e + 3] += a.w;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) gv[e] *= scale;
+          }
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8)
+            *reinterpret_cast<uint4*>(out + c0 + q8 * 8) =
+                make_uint4(pack2(gv[q8 * 8], gv[q8 * 8 + 1]), pack2(gv[q8 * 8 + 2], gv[q8 * 8 + 3]),
+                           pack2(gv[q8 * 8 + 4], gv[q8 * 8 + 5]), pack2(gv[q8 * 8 + 6], gv[q8 * 8 + 7]));
+        }
+        fence_before();
+      }
+    }
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+bool attn_bwd3_supported(const Geometry& g) {
+  return g.bf16 && g.d == D && g.N % kTile == 0 && g.chunk >= 16 && g.chunk <= kTile &&
+         kTile % g.chunk == 0;
+}
+
+cudaError_t launch_attn_bwd3(const Geometry& g, const void* q, const void* k, const void* v,
+                             const int32_t* perm_q, const int32_t* perm_k, const void* d_o,
+                             const float* lse, const float* dprime, const float* dv_race,
+                             const float* dq_gate, void* dq, void* dk, void* dv, uint32_t* err,
+                             cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(attn_bwd3_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Lay3::kDyn);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t ntiles = (int64_t)g.BH * (g.N / kTile);
+  const int grid = (int)(ntiles < sms ? ntiles : sms);
+  attn_bwd3_kernel<<<grid, kThreads, Lay3::kDyn, s>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+      static_cast<const __nv_bfloat16*>(v), perm_q, perm_k,
+      static_cast<const __nv_bfloat16*>(d_o), lse, dprime, dv_race, dq_gate, g.BH, g.N, g.chunk,
+      g.scale, g.scale * 1.4426950408889634f, static_cast<__nv_bfloat16*>(dq),
+      static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), err);
+  return cudaGetLastError();
+}
+
+}  // namespace elsaa

@@ -119,6 +119,14 @@ cudaError_t launch_attn_fwd_tc(const Geometry& g, const void* q, const void* k, 
                                float* lse, uint32_t* err, cudaStream_t s);
 bool attn_tc_supported(const Geometry& g);
 // Overlapped backward (d = 64, chunk 64 or 128).
+// Persistent backward (d = 64, bf16, chunk dividing 128): writes dq (gate part
+// from dq_gate plus the sparse part), dk and dv (plus dv_race) directly.
+bool attn_bwd3_supported(const Geometry& g);
+cudaError_t launch_attn_bwd3(const Geometry& g, const void* q, const void* k, const void* v,
+                             const int32_t* perm_q, const int32_t* perm_k, const void* d_o,
+                             const float* lse, const float* dprime, const float* dv_race,
+                             const float* dq_gate, void* dq, void* dk, void* dv, uint32_t* err,
+                             cudaStream_t s);
 bool attn_bwd2_supported(const Geometry& g);
 cudaError_t launch_attn_bwd2(const Geometry& g, const void* q, const void* k, const void* v,
                              const int32_t* perm_q, const int32_t* perm_k, const void* d_o,

@@ -63,6 +63,13 @@ def test_single_chunk_and_ragged_lengths(cuda_device, N, chunk):
     _run(w, backward=True)
 
 
+@pytest.mark.parametrize("chunk", [16, 32])
+def test_small_chunks(cuda_device, chunk):
+    # windows narrower than the 128-row tiles: the attention kernels mask by chunk
+    w = WORKLOADS["iid-4k"].replace(B=1, H=2, N=1024, chunk=chunk)
+    _run(w, backward=True)
+
+
 def test_two_pass_sort_and_wide_race_codes(cuda_device):
     # 12 sort bits take two radix passes; 11 RACE bits give uint16 codes and
     # 2048-bucket tables (the global-atomic build)
