@@ -293,24 +293,31 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
   ELSAA_TRY(cudaMemsetAsync(w + wl.err, 0, sizeof(uint32_t), s));
   ELSAA_TRY(mark(events, 0, s));
 
-  // 1. fusion and gate backward: dO_sp, D', dq from the gates, g_r dy / Ctot
-  float* absmax = (float*)(w + wl.absmax) + g.BH;
-  ELSAA_TRY(launch_fuse_bwd(g, q, dy, o_sp, o_race, lse, ctot, gate_w, gate_b, lambda, d_o,
-                            dprime, dq_acc, dor, absmax, partials, s));
-  ELSAA_TRY(mark(events, 1, s));
-  // 2. RACE backward: scatter into the table gradient by query code, gather by key code
+  // The persistent sparse backward writes dq, dk and dv itself; the RACE
+  // branch's dv is then added in place by the key-code gather.
+  const bool direct = g.tc_attn && attn_bwd3_supported(g) && race_gather_add_supported(g);
   __nv_bfloat16* gtab = g.bf16 ? (__nv_bfloat16*)(w + wl.gtab) : nullptr;
+  const void* race_grad = g.bf16 ? (const void*)gtab : (const void*)d_t;
+  // 1. fusion and gate backward: dO_sp, D', the gate part of dq, g_r dy / Ctot
+  float* absmax = (float*)(w + wl.absmax) + g.BH;
+  float2* da = reinterpret_cast<float2*>(dq_acc);   // direct path: (da_s, da_r) per row
+  ELSAA_TRY(launch_fuse_bwd(g, q, dy, o_sp, o_race, lse, ctot, gate_w, gate_b, lambda, d_o,
+                            dprime, direct ? nullptr : dq_acc, direct ? da : nullptr, dor,
+                            absmax, partials, s));
+  ELSAA_TRY(mark(events, 1, s));
+  // 2. RACE backward: scatter into the table gradient by query code (and, off
+  // the direct path, gather by key code into dv_acc)
   ELSAA_TRY(launch_race_build(g, rcode, rcode_t, dor, false, absmax, d_t, !g.bf16, gtab, nullptr,
                               (uint32_t*)(w + wl.err), s));
-  ELSAA_TRY(launch_race_gather_sum(g, rcode_k, g.bf16 ? (const void*)gtab : (const void*)d_t,
-                                   dv_acc, s));
+  if (!direct) ELSAA_TRY(launch_race_gather_sum(g, rcode_k, race_grad, dv_acc, s));
   ELSAA_TRY(mark(events, 2, s));
   // 3. sparse branch backward, 4. outputs
-  if (g.tc_attn && attn_bwd3_supported(g)) {
-    // writes dq itself: gate part (dq_acc) + sparse part, in the data dtype
-    ELSAA_TRY(launch_attn_bwd3(g, q, k, v, perm, perm + bhn, d_o, lse, dprime, dv_acc, dq_acc,
-                               dq, dk, dv, (uint32_t*)(w + wl.err), s));
+  if (direct) {
+    ELSAA_TRY(launch_attn_bwd3(g, q, k, v, perm, perm + bhn, d_o, lse, dprime, da,
+                               g.gate_fixed ? nullptr : gate_w, dq, dk, dv,
+                               (uint32_t*)(w + wl.err), s));
     ELSAA_TRY(mark(events, 3, s));
+    ELSAA_TRY(launch_race_gather_add(g, rcode_k, race_grad, dv, s));
   } else if (g.tc_attn && attn_bwd2_supported(g)) {
     ELSAA_TRY(launch_attn_bwd2(g, q, k, v, perm, perm + bhn, d_o, lse, dprime, dv_acc, dq_acc,
                                dk, dv, (uint32_t*)(w + wl.err), s));
@@ -353,7 +360,9 @@ elsaa_status elsaa_kernel_launches(const elsaa_params* p, int32_t* fwd, int32_t*
   // hash 1, sort 3 per pass, |V| max 1 + RACE build 1, sparse 1, RACE gather + fusion 1
   *fwd = 1 + 3 * g.sort_passes + 2 + 1 + 1;
   // fusion backward 1, RACE build 1 + gather 1, sparse 1 (+ casts), reduction 1
-  const int sparse = g.tc_attn ? (attn_bwd3_supported(g) ? 1 : 1 + 1) : 1 + 3;
+  // (direct path: the sparse kernel writes dq itself and the gather adds into dv)
+  const bool direct = g.tc_attn && attn_bwd3_supported(g) && race_gather_add_supported(g);
+  const int sparse = direct ? 1 : g.tc_attn ? 1 + 1 : 1 + 3;
   *bwd = 1 + 2 + sparse + 1;
   return ELSAA_OK;
 }

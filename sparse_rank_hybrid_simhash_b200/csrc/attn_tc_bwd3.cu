@@ -14,22 +14,26 @@
 // takes a contiguous run of key tiles, so consecutive tiles share a query
 // block.  The dQ of block qb has two contributions, from tiles qb - 1 and
 // qb; both are accumulated in TMEM by the CTA that owns tile qb and written
-// once, in bf16, together with the gate part of dQ already in dq_gate.  For
+// once, in bf16, together with the gate part of dQ, da_s w_s + da_r w_r (the
+// per-row pair (da_s, da_r) comes from the fusion backward).  For
 // the first tile of a run the contribution of tile qb - 1 belongs to another
 // CTA; this CTA recomputes it (a "pre" pair: dQ only), and the CTA owning
 // tile qb - 1 skips the dQ of its last "next" pair.  No atomics, and every
-// output element is written by exactly one thread.
+// output element is written by exactly one thread.  dv holds the sparse part
+// only; the RACE branch's part is added afterwards.
 //
 // Roles (320 threads, one CTA per SM):
 //   warp 0      producer: cp.async gathers of K/V key tiles (two-slot ring)
-//               and Q/dO query blocks with their lse and D' (two-slot ring)
+//               and Q/dO query blocks with their lse, D' and (da_s, da_r)
+//               (two-slot ring)
 //   warp 1      MMA issuer (one thread) and TMEM owner; for pair p it issues
 //               S^T/dP^T of pair p + 1 as soon as P^T/dS^T of pair p are in
 //               shared memory, then dV, dK, dQ of pair p
 //   warps 2..9  elementwise: warp w reaches TMEM lanes 32 (w % 4) .. +31 and
 //               takes half of the query columns; P^T and dS^T (bf16) to
-//               shared memory; then the dQ flush of a finished query block
-//               and the dV / dK write-out of a finished key tile
+//               shared memory; one pair after a query block's dQ is complete
+//               they write it out (its MMA has finished by then), and after
+//               a key tile's last pair they write out dV and dK
 // TMEM: S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384),
 //       dQ [384,448) and [448,512) for alternating query blocks.
 // Every wait is bounded; a timeout records ERR_TIMEOUT and every role leaves
@@ -63,7 +67,9 @@ struct Lay3 {
   static constexpr uint32_t kQidx = kKidx + 2 * 128 * 4;    // [2][128] query tokens
   static constexpr uint32_t kLse = kQidx + 2 * 128 * 4;     // [2][128] lse (log2 units once used)
   static constexpr uint32_t kDpr = kLse + 2 * 128 * 4;      // [2][128] D'
-  static constexpr uint32_t kBar = kDpr + 2 * 128 * 4;
+  static constexpr uint32_t kDa = kDpr + 2 * 128 * 4;       // [2][128] (da_s, da_r)
+  static constexpr uint32_t kW = kDa + 2 * 128 * 8;         // [2][64] w_s, w_r
+  static constexpr uint32_t kBar = kW + 2 * 64 * 4;
   static constexpr uint32_t kDyn = kBar + 256;
 };
 
@@ -151,6 +157,9 @@ ELSAA_DEV float ex2(float x) {
 ELSAA_DEV void cp_async4(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
+ELSAA_DEV void cp_async8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
 
 ELSAA_DEV void cp_async_arrive(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
@@ -178,7 +187,7 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
                  const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ perm_q,
                  const int32_t* __restrict__ perm_k, const __nv_bfloat16* __restrict__ d_o,
                  const float* __restrict__ lse, const float* __restrict__ dprime,
-                 const float* __restrict__ dv_race, const float* __restrict__ dq_gate, int BH,
+                 const float2* __restrict__ da, const float* __restrict__ gate_w, int BH,
                  int N, int chunk, float scale, float scale_log2, __nv_bfloat16* __restrict__ dq,
                  __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
                  uint32_t* __restrict__ err) {
@@ -204,6 +213,9 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
   int32_t* s_qidx = reinterpret_cast<int32_t*>(smem + Lay::kQidx);
   float* s_lse = reinterpret_cast<float*>(smem + Lay::kLse);
   float* s_dpr = reinterpret_cast<float*>(smem + Lay::kDpr);
+  float2* s_da = reinterpret_cast<float2*>(smem + Lay::kDa);
+  float* s_w = reinterpret_cast<float*>(smem + Lay::kW);
+  for (int i = tid; i < 2 * D; i += kThreads) s_w[i] = gate_w ? gate_w[i] : 0.f;
 
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -285,6 +297,7 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         const int r = lane + 32 * j;
         cp_async4(smem_u32(s_lse + s * 128 + r), lse + unit + idx[j]);
         cp_async4(smem_u32(s_dpr + s * 128 + r), dprime + unit + idx[j]);
+        cp_async8(smem_u32(s_da + s * 128 + r), da + unit + idx[j]);
         s_qidx[s * 128 + r] = idx[j];
       }
       cp_async_arrive(&bars->full_q[s]);
@@ -400,7 +413,39 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     while ((1 << lc) < chunk) ++lc;
     uint32_t flush_parity = 0u;   // bit b: parity of the next completion of dQ buffer b
     int64_t ntile = 0;
-    int key_tok = 0, flush_tok = 0;
+    int key_tok = 0;
+    // the query block whose dQ is written out one pair later
+    bool pend = false;
+    int pend_buf = 0, pend_tok = 0;
+    size_t pend_unit = 0;
+    float2 pend_da = make_float2(0.f, 0.f);
+    const float* wsv = s_w + half * 32;        // this thread's 32 columns of w_s
+    const float* wrv = s_w + D + half * 32;    // and of w_r
+    auto flush = [&]() -> bool {
+      // dQ of the pending block: TMEM lane = query row, this warp's 32 columns
+      const int b = pend_buf;
+      if (!ew_all(mbar_wait(&bars->dq_full[b], (flush_parity >> b) & 1u, err))) return false;
+      flush_parity ^= 1u << b;
+      fence_after();
+      float g[32];
+      tmem_ld32(tmem + kTdQ + b * D + lane_off + half * 32, g);
+      tmem_ld_wait();
+      __nv_bfloat16* out = dq + (pend_unit + pend_tok) * D + half * 32;
+#pragma unroll
+      for (int q8 = 0; q8 < 4; ++q8) {
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int c = q8 * 8 + e;
+          x[e] = fmaf(pend_da.x, wsv[c], fmaf(pend_da.y, wrv[c], scale * g[c]));
+        }
+        *reinterpret_cast<uint4*>(out + q8 * 8) =
+            make_uint4(pack2(x[0], x[1]), pack2(x[2], x[3]), pack2(x[4], x[5]), pack2(x[6], x[7]));
+      }
+      fence_before();
+      pend = false;
+      return true;
+    };
     PairIter it;
     it.init(&run);
     for (int64_t pi = 0; run.count > 0 && !it.done(); ++pi, it.advance()) {
@@ -419,7 +464,12 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         ew_sync();
       }
       if (p.first_of_tile && p.kv) key_tok = s_kidx[kslot * 128 + row];
-      if (p.flush) flush_tok = s_qidx[qslot * 128 + row];
+      int flush_tok = 0;
+      float2 flush_da = make_float2(0.f, 0.f);
+      if (p.flush) {
+        flush_tok = s_qidx[qslot * 128 + row];
+        flush_da = s_da[qslot * 128 + row];
+      }
       // visible query columns of this key row: ranks [i c, (i + 2) c)
       const int key_chunk = (p.kb * kTile + row) >> lc;
       const int lo = (key_chunk << lc) - p.qb * kTile, hi = lo + 2 * chunk;
@@ -468,32 +518,16 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
       fence_before();
       mbar_arrive(&bars->p_full);
 
-      if (p.flush) {
-        // dQ of query block qb: TMEM lane = query row, this warp's 32 columns
-        const int b = (int)(p.qs & 1);
-        const float* gate = dq_gate + (unit + flush_tok) * D + half * 32;
-        float4 g4[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) g4[i] = reinterpret_cast<const float4*>(gate)[i];
-        ok = ew_all(mbar_wait(&bars->dq_full[b], (flush_parity >> b) & 1u, err));
+      if (pend) {
+        ok = flush();
         if (!ok) break;
-        flush_parity ^= 1u << b;
-        fence_after();
-        float g[32];
-        tmem_ld32(tmem + kTdQ + b * D + lane_off + half * 32, g);
-        tmem_ld_wait();
-        __nv_bfloat16* out = dq + (unit + flush_tok) * D + half * 32;
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-          const float4 a = g4[2 * q8], c = g4[2 * q8 + 1];
-          const float* x = g + q8 * 8;
-          *reinterpret_cast<uint4*>(out + q8 * 8) =
-              make_uint4(pack2(a.x + scale * x[0], a.y + scale * x[1]),
-                         pack2(a.z + scale * x[2], a.w + scale * x[3]),
-                         pack2(c.x + scale * x[4], c.y + scale * x[5]),
-                         pack2(c.z + scale * x[6], c.w + scale * x[7]));
-        }
-        fence_before();
+      }
+      if (p.flush) {
+        pend = true;
+        pend_buf = (int)(p.qs & 1);
+        pend_tok = flush_tok;
+        pend_unit = unit;
+        pend_da = flush_da;
       }
       if (p.kv && p.last_of_tile) {
         // dV (+ the RACE branch's dv) from half 0, dK from half 1, of this key row
@@ -502,22 +536,14 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         ++ntile;
         fence_after();
         const uint32_t col = half == 0 ? kTdV : kTdK;
+        const float mul = half == 0 ? 1.0f : scale;
         __nv_bfloat16* out = (half == 0 ? dv : dk) + (unit + key_tok) * D;
-        const float* add = dv_race + (unit + key_tok) * D;
         for (int c0 = 0; c0 < D; c0 += 32) {
           float gv[32];
           tmem_ld32(tmem + col + lane_off + c0, gv);
           tmem_ld_wait();
-          if (half == 0) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              const float4 a = *reinterpret_cast<const float4*>(add + c0 + e);
-              gv[e] += a.x; gv[e + 1] += a.y; gv[e + 2] += a.z; gv[e + 3] += a.w;
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) gv[e] *= scale;
-          }
+          for (int e = 0; e < 32; ++e) gv[e] *= mul;
 #pragma unroll
           for (int q8 = 0; q8 < 4; ++q8)
             *reinterpret_cast<uint4*>(out + c0 + q8 * 8) =
@@ -527,6 +553,7 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         fence_before();
       }
     }
+    if (ok && pend) ok = flush();
   }
   fence_before();
   __syncthreads();
@@ -545,8 +572,8 @@ bool attn_bwd3_supported(const Geometry& g) {
 
 cudaError_t launch_attn_bwd3(const Geometry& g, const void* q, const void* k, const void* v,
                              const int32_t* perm_q, const int32_t* perm_k, const void* d_o,
-                             const float* lse, const float* dprime, const float* dv_race,
-                             const float* dq_gate, void* dq, void* dk, void* dv, uint32_t* err,
+                             const float* lse, const float* dprime, const float2* da,
+                             const float* gate_w, void* dq, void* dk, void* dv, uint32_t* err,
                              cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(attn_bwd3_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -560,7 +587,7 @@ cudaError_t launch_attn_bwd3(const Geometry& g, const void* q, const void* k, co
   attn_bwd3_kernel<<<grid, kThreads, Lay3::kDyn, s>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
       static_cast<const __nv_bfloat16*>(v), perm_q, perm_k,
-      static_cast<const __nv_bfloat16*>(d_o), lse, dprime, dv_race, dq_gate, g.BH, g.N, g.chunk,
+      static_cast<const __nv_bfloat16*>(d_o), lse, dprime, da, gate_w, g.BH, g.N, g.chunk,
       g.scale, g.scale * 1.4426950408889634f, static_cast<__nv_bfloat16*>(dq),
       static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), err);
   return cudaGetLastError();

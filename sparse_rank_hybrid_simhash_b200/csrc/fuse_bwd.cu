@@ -13,6 +13,8 @@
 //   dq_gate = da_s w_s + da_r w_r,  dw += da q,  db += da
 //   dO_sp = g_s m dy,  D' = dO_sp . O_sp - dlse  (the sparse backward's row term)
 //   dO_race / Ctot = g_r dy / Ctot  (scattered into the RACE table gradient)
+// dq_gate goes out either as fp32 rows (dq_acc) or as the pair (da_s, da_r)
+// per row (da_out) for a consumer that forms da_s w_s + da_r w_r itself.
 // One warp per query; per-block partial sums of (dw_s, dw_r, db_s, db_r,
 // dlambda) go to a fixed number of slots and are reduced in a fixed order, so
 // the parameter gradients are deterministic.
@@ -74,7 +76,8 @@ fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __re
                 const float* __restrict__ gate_b, int gate_fixed, float gs_fixed, float gr_fixed,
                 const float* __restrict__ lam, int64_t rows, int N, int L, int d,
                 T* __restrict__ d_o, float* __restrict__ dprime, float* __restrict__ dq_acc,
-                T* __restrict__ dor, float* __restrict__ absmax, float* __restrict__ partials) {
+                float2* __restrict__ da_out, T* __restrict__ dor, float* __restrict__ absmax,
+                float* __restrict__ partials) {
   constexpr int QW = 32 / QL;
   __shared__ float red[8][2 * 128 + 3];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
@@ -148,7 +151,8 @@ fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __re
     float dd = 0.f;
     if (valid) {
       st4_round<T>(d_o + base, dov);   // dov now holds the stored (rounded) values
-      *reinterpret_cast<float4*>(dq_acc + base) = make_float4(dqv[0], dqv[1], dqv[2], dqv[3]);
+      if (dq_acc)
+        *reinterpret_cast<float4*>(dq_acc + base) = make_float4(dqv[0], dqv[1], dqv[2], dqv[3]);
       st4_round<T>(dor + base, drv);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -160,6 +164,7 @@ fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __re
     dd = gsum<QL>(dd);
     if (valid && ql == 0) {
       dprime[rr] = dd - dlse;
+      if (da_out) da_out[rr] = make_float2(da_s, da_r);
       pbs += da_s;
       pbr += da_r;
       plam += dlam;
@@ -236,8 +241,8 @@ template <typename T>
 cudaError_t fuse_bwd(const Geometry& g, const void* q, const void* dy, const void* o_sp,
                      const void* o_race, const float* lse, const int32_t* ctot,
                      const float* gate_w, const float* gate_b, const float* lam, void* d_o,
-                     float* dprime, float* dq_acc, void* dor, float* absmax, float* partials,
-                     cudaStream_t s) {
+                     float* dprime, float* dq_acc, float2* da_out, void* dor, float* absmax,
+                     float* partials, cudaStream_t s) {
   const int64_t rows = (int64_t)g.BH * g.N;
   cudaError_t e = cudaMemsetAsync(absmax, 0, (size_t)g.BH * sizeof(float), s);
   if (e != cudaSuccess) return e;
@@ -245,7 +250,7 @@ cudaError_t fuse_bwd(const Geometry& g, const void* q, const void* dy, const voi
   fuse_bwd_kernel<T, VEC><<<kParamBlocks, 256, 0, s>>>(                                        \
       static_cast<const T*>(q), static_cast<const T*>(dy), static_cast<const T*>(o_sp),        \
       static_cast<const T*>(o_race), lse, ctot, gate_w, gate_b, g.gate_fixed, g.gate_s,        \
-      g.gate_r, lam, rows, g.N, g.L, g.d, static_cast<T*>(d_o), dprime, dq_acc,               \
+      g.gate_r, lam, rows, g.N, g.L, g.d, static_cast<T*>(d_o), dprime, dq_acc, da_out,       \
       static_cast<T*>(dor), absmax,                                                            \
       partials)
   switch (g.d) {
@@ -262,12 +267,12 @@ cudaError_t fuse_bwd(const Geometry& g, const void* q, const void* dy, const voi
 cudaError_t launch_fuse_bwd(const Geometry& g, const void* q, const void* dy, const void* o_sp,
                             const void* o_race, const float* lse, const int32_t* ctot,
                             const float* gate_w, const float* gate_b, const float* lam,
-                            void* d_o, float* dprime, float* dq_acc, void* dor,
+                            void* d_o, float* dprime, float* dq_acc, float2* da_out, void* dor,
                             float* absmax, float* partials, cudaStream_t s) {
   return g.bf16 ? fuse_bwd<__nv_bfloat16>(g, q, dy, o_sp, o_race, lse, ctot, gate_w, gate_b, lam,
-                                          d_o, dprime, dq_acc, dor, absmax, partials, s)
+                                          d_o, dprime, dq_acc, da_out, dor, absmax, partials, s)
                 : fuse_bwd<float>(g, q, dy, o_sp, o_race, lse, ctot, gate_w, gate_b, lam, d_o,
-                                  dprime, dq_acc, dor, absmax, partials, s);
+                                  dprime, dq_acc, da_out, dor, absmax, partials, s);
 }
 
 cudaError_t launch_param_reduce(const Geometry& g, const float* partials, float* dgate_w,

@@ -96,6 +96,11 @@ cudaError_t launch_race_build(const Geometry& g, const void* codes, const void* 
                               cudaStream_t s);
 // out[bh][i][:] = sum_l tables[bh][l][codes[bh][i][l]][:]  (f32, overwritten);
 // tables in the data dtype (bf16 copy, or the fp32 sums for fp32 data).
+// dst[bh][i][:] += sum_l tables[bh][l][codes[bh][i][l]][:], dst in the data dtype
+// (row-pipelined gather only: race_gather_add_supported).
+bool race_gather_add_supported(const Geometry& g);
+cudaError_t launch_race_gather_add(const Geometry& g, const void* codes, const void* tables,
+                                   void* dst, cudaStream_t s);
 cudaError_t launch_race_gather_sum(const Geometry& g, const void* codes, const void* tables,
                                    float* out, cudaStream_t s);
 // Forward RACE gather fused with the gates, the multiplier and the output.
@@ -119,13 +124,14 @@ cudaError_t launch_attn_fwd_tc(const Geometry& g, const void* q, const void* k, 
                                float* lse, uint32_t* err, cudaStream_t s);
 bool attn_tc_supported(const Geometry& g);
 // Overlapped backward (d = 64, chunk 64 or 128).
-// Persistent backward (d = 64, bf16, chunk dividing 128): writes dq (gate part
-// from dq_gate plus the sparse part), dk and dv (plus dv_race) directly.
+// Persistent backward (d = 64, bf16, chunk dividing 128): writes dq (the gate
+// part da_s w_s + da_r w_r from the per-row pair da, plus the sparse part),
+// dk, and dv (sparse part only) directly.  gate_w may be NULL (fixed gates).
 bool attn_bwd3_supported(const Geometry& g);
 cudaError_t launch_attn_bwd3(const Geometry& g, const void* q, const void* k, const void* v,
                              const int32_t* perm_q, const int32_t* perm_k, const void* d_o,
-                             const float* lse, const float* dprime, const float* dv_race,
-                             const float* dq_gate, void* dq, void* dk, void* dv, uint32_t* err,
+                             const float* lse, const float* dprime, const float2* da,
+                             const float* gate_w, void* dq, void* dk, void* dv, uint32_t* err,
                              cudaStream_t s);
 bool attn_bwd2_supported(const Geometry& g);
 cudaError_t launch_attn_bwd2(const Geometry& g, const void* q, const void* k, const void* v,
@@ -149,7 +155,7 @@ cudaError_t launch_attn_bwd_tc(const Geometry& g, const void* q, const void* k, 
 cudaError_t launch_fuse_bwd(const Geometry& g, const void* q, const void* dy, const void* o_sp,
                             const void* o_race, const float* lse, const int32_t* ctot,
                             const float* gate_w, const float* gate_b, const float* lam,
-                            void* d_o, float* dprime, float* dq_acc, void* dor,
+                            void* d_o, float* dprime, float* dq_acc, float2* da_out, void* dor,
                             float* absmax, float* partials, cudaStream_t s);
 cudaError_t launch_param_reduce(const Geometry& g, const float* partials, float* dgate_w,
                                 float* dgate_b, float* dlambda, cudaStream_t s);

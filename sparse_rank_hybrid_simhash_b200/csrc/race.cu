@@ -878,7 +878,8 @@ ELSAA_DEV void gather_row(const TT* tab, const uint32_t (&w)[WPL], int L, int NB
 template <typename TT, typename CodeT, int QL, int WPL>
 __global__ void __launch_bounds__(256, 4)
 race_gather_rows_kernel(const CodeT* __restrict__ codes, const TT* __restrict__ tables,
-                        int64_t rows, int N, int L, int NB, int d, float* __restrict__ out) {
+                        int64_t rows, int N, int L, int NB, int d, float* __restrict__ out,
+                        TT* __restrict__ add_out) {
   constexpr int QW = 32 / QL, EL = 16 / sizeof(TT);
   const int lane = threadIdx.x & 31, ql = lane % QL, gbase = lane - ql;
   const uint64_t pol = l2_keep_policy();
@@ -901,9 +902,18 @@ race_gather_rows_kernel(const CodeT* __restrict__ codes, const TT* __restrict__ 
     gather_row<TT, CodeT, QL, WPL>(tables + (size_t)bh * L * NB * d + ql * EL, w, L, NB, d,
                                    gbase, pol, acc);
     if (valid) {
-      float* o = out + rr * d + ql * EL;
+      if (add_out) {   // add_out[row] += sum, in the data dtype
+        TT* o = add_out + rr * d + ql * EL;
+        float cur[EL];
+        unpack16(*reinterpret_cast<const uint4*>(o), cur, o);
 #pragma unroll
-      for (int i = 0; i < EL; i += 4) store16_stream(o + i, acc + i);
+        for (int i = 0; i < EL; ++i) cur[i] += acc[i];
+        *reinterpret_cast<uint4*>(o) = pack16(cur, o);
+      } else {
+        float* o = out + rr * d + ql * EL;
+#pragma unroll
+        for (int i = 0; i < EL; i += 4) store16_stream(o + i, acc + i);
+      }
     }
 #pragma unroll
     for (int i = 0; i < WPL; ++i) w[i] = wn[i];
@@ -1148,7 +1158,7 @@ int rows_grid(int64_t rows, int QL) {
 
 template <typename TT, typename CodeT>
 cudaError_t gather_sum(const Geometry& g, const void* codes, const TT* tables, float* out,
-                       cudaStream_t s) {
+                       TT* add_out, cudaStream_t s) {
   constexpr int EL = 16 / sizeof(TT);
   const int64_t rows = (int64_t)g.BH * g.N;
   const int QLr = g.d / EL;
@@ -1158,7 +1168,7 @@ cudaError_t gather_sum(const Geometry& g, const void* codes, const TT* tables, f
     const int grid = rows_grid(rows, QLr);
 #define ELSAA_GROWS(QL, WPL)                                                                   \
   race_gather_rows_kernel<TT, CodeT, QL, WPL><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L,  \
-                                                                    g.NB, g.d, out)
+                                                                    g.NB, g.d, out, add_out)
 #define ELSAA_GROWS_W(QL)                                                                      \
   switch (wpl) {                                                                               \
     case 1: ELSAA_GROWS(QL, 1); break;                                                         \
@@ -1174,6 +1184,7 @@ cudaError_t gather_sum(const Geometry& g, const void* codes, const TT* tables, f
 #undef ELSAA_GROWS
     return cudaGetLastError();
   }
+  if (add_out) return cudaErrorNotSupported;   // callers check race_gather_add_supported
   const int grid = grid_for_rows((rows * g.d / EL + 31) / 32, 8);
   switch (g.d) {
     case 32: race_gather_sum_kernel<TT, CodeT, 32 / EL><<<grid, 256, 0, s>>>(c, tables, rows, g.N, g.L, g.NB, g.d, out); break;
@@ -1271,12 +1282,30 @@ cudaError_t launch_race_gather_sum(const Geometry& g, const void* codes, const v
                                    float* out, cudaStream_t s) {
   if (g.bf16) {
     const __nv_bfloat16* t = static_cast<const __nv_bfloat16*>(tables);
-    return g.rcode_bytes == 1 ? gather_sum<__nv_bfloat16, uint8_t>(g, codes, t, out, s)
-                              : gather_sum<__nv_bfloat16, uint16_t>(g, codes, t, out, s);
+    return g.rcode_bytes == 1 ? gather_sum<__nv_bfloat16, uint8_t>(g, codes, t, out, nullptr, s)
+                              : gather_sum<__nv_bfloat16, uint16_t>(g, codes, t, out, nullptr, s);
   }
   const float* t = static_cast<const float*>(tables);
-  return g.rcode_bytes == 1 ? gather_sum<float, uint8_t>(g, codes, t, out, s)
-                            : gather_sum<float, uint16_t>(g, codes, t, out, s);
+  return g.rcode_bytes == 1 ? gather_sum<float, uint8_t>(g, codes, t, out, nullptr, s)
+                            : gather_sum<float, uint16_t>(g, codes, t, out, nullptr, s);
+}
+
+bool race_gather_add_supported(const Geometry& g) {
+  return row_wpl(g, g.d / (g.bf16 ? 8 : 4)) > 0;
+}
+
+cudaError_t launch_race_gather_add(const Geometry& g, const void* codes, const void* tables,
+                                   void* dst, cudaStream_t s) {
+  if (g.bf16) {
+    const __nv_bfloat16* t = static_cast<const __nv_bfloat16*>(tables);
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(dst);
+    return g.rcode_bytes == 1 ? gather_sum<__nv_bfloat16, uint8_t>(g, codes, t, nullptr, o, s)
+                              : gather_sum<__nv_bfloat16, uint16_t>(g, codes, t, nullptr, o, s);
+  }
+  const float* t = static_cast<const float*>(tables);
+  float* o = static_cast<float*>(dst);
+  return g.rcode_bytes == 1 ? gather_sum<float, uint8_t>(g, codes, t, nullptr, o, s)
+                            : gather_sum<float, uint16_t>(g, codes, t, nullptr, o, s);
 }
 
 cudaError_t launch_race_fuse_fwd(const Geometry& g, const void* q, const void* rcode_q,
