@@ -855,11 +855,27 @@ ELSAA_DEV int code_of(uint32_t word, int e) {
 }
 
 // acc += sum over tables t of tab[t][code_t][ql * EL ...], tab = this unit's
-// tables offset by the lane's column slice.
+// tables offset by the lane's column slice.  Offsets are 32-bit (a unit's
+// tables are far below 4 GB): table t starts t * table_bytes in, and a
+// bucket's row is code << row_shift further.
+ELSAA_DEV void add_lines(float* acc, uint4 raw, const __nv_bfloat16*) {
+  const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    add_f32x2(acc[2 * i], acc[2 * i + 1], __uint_as_float(w4[i] << 16),
+              __uint_as_float(w4[i] & 0xFFFF0000u));
+}
+ELSAA_DEV void add_lines(float* acc, uint4 raw, const float*) {
+  add_f32x2(acc[0], acc[1], __uint_as_float(raw.x), __uint_as_float(raw.y));
+  add_f32x2(acc[2], acc[3], __uint_as_float(raw.z), __uint_as_float(raw.w));
+}
+
 template <typename TT, typename CodeT, int QL, int WPL>
-ELSAA_DEV void gather_row(const TT* tab, const uint32_t (&w)[WPL], int L, int NB, int d,
-                          int gbase, uint64_t pol, float* acc) {
+ELSAA_DEV void gather_row(const TT* tab, const uint32_t (&w)[WPL], int L, uint32_t table_bytes,
+                          int row_shift, int gbase, uint64_t pol, float* acc) {
   constexpr int PER = 4 / (int)sizeof(CodeT);
+  const char* base = reinterpret_cast<const char*>(tab);
+  uint32_t toff = 0;
 #pragma unroll
   for (int i = 0; i < WPL; ++i) {
 #pragma unroll
@@ -868,8 +884,13 @@ ELSAA_DEV void gather_row(const TT* tab, const uint32_t (&w)[WPL], int L, int NB
       if (t0 < L) {
         const uint32_t word = __shfl_sync(0xffffffffu, w[i], gbase + sl);
 #pragma unroll
-        for (int e = 0; e < PER; ++e)
-          acc_row(acc, tab + ((size_t)(t0 + e) * NB + code_of<CodeT>(word, e)) * d, pol);
+        for (int e = 0; e < PER; ++e) {
+          const uint32_t code =
+              sizeof(CodeT) == 1 ? __byte_perm(word, 0, 0x4440u | (uint32_t)e)
+                                 : __byte_perm(word, 0, e ? 0x4432u : 0x4410u);
+          add_lines(acc, ld16_keep(base + toff + (code << row_shift), pol), tab);
+          toff += table_bytes;
+        }
       }
     }
   }
@@ -884,6 +905,8 @@ race_gather_rows_kernel(const CodeT* __restrict__ codes, const TT* __restrict__ 
   const int lane = threadIdx.x & 31, ql = lane % QL, gbase = lane - ql;
   const uint64_t pol = l2_keep_policy();
   const int W = L * (int)sizeof(CodeT) / 4;
+  const uint32_t table_bytes = (uint32_t)NB * (uint32_t)d * (uint32_t)sizeof(TT);
+  const int row_shift = 31 - __clz(d * (int)sizeof(TT));   // d * sizeof is a power of two
   const int64_t first = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * QW;
   const int64_t stride = (int64_t)gridDim.x * (blockDim.x >> 5) * QW;
   uint32_t w[WPL];
@@ -899,8 +922,8 @@ race_gather_rows_kernel(const CodeT* __restrict__ codes, const TT* __restrict__ 
     uint32_t wn[WPL];
     load_row_codes<CodeT, QL, WPL>(codes + min(r + stride, rows - 1) * L, W, ql, wn);
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    gather_row<TT, CodeT, QL, WPL>(tables + (size_t)bh * L * NB * d + ql * EL, w, L, NB, d,
-                                   gbase, pol, acc);
+    gather_row<TT, CodeT, QL, WPL>(tables + (size_t)bh * L * NB * d + ql * EL, w, L, table_bytes,
+                                   row_shift, gbase, pol, acc);
     if (valid) {
       if (add_out) {   // add_out[row] += sum, in the data dtype
         TT* o = add_out + rr * d + ql * EL;
@@ -934,6 +957,8 @@ race_fuse_rows_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q
   const int lane = threadIdx.x & 31, ql = lane % QL, gbase = lane - ql;
   const uint64_t pol = l2_keep_policy();
   const int W = L * (int)sizeof(CodeT) / 4;
+  const uint32_t table_bytes = (uint32_t)NB * (uint32_t)d * (uint32_t)sizeof(T);
+  const int row_shift = 31 - __clz(d * (int)sizeof(T));   // d * sizeof is a power of two
   const float lam_v = *lam;
   float ws8[EL], wr8[EL];
 #pragma unroll
@@ -976,8 +1001,8 @@ race_fuse_rows_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q
       }
     }
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    gather_row<T, CodeT, QL, WPL>(tables + (size_t)bh * L * NB * d + ql * EL, w, L, NB, d, gbase,
-                                  pol, acc);
+    gather_row<T, CodeT, QL, WPL>(tables + (size_t)bh * L * NB * d + ql * EL, w, L, table_bytes,
+                                  row_shift, gbase, pol, acc);
     ctot = group_sum_i<QL>(ctot);
     const float inv = ctot > 0 ? 1.0f / (float)ctot : 0.f;
     float qv[EL], os[EL], orc[EL];
