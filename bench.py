@@ -22,6 +22,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import hashlib
 import json
 import math
 import os
@@ -66,24 +67,71 @@ def window_keys(N: int, c: int) -> int:
 
 
 def stage_work(w):
+    """Algorithmic work of each stage: (tensor-core flops, HBM bytes).  Bytes
+    count what the method must move (inputs read once, outputs written once),
+    not what a kernel happens to move; the RACE stages' gathers through L2
+    (L d values per row and pass) are not HBM traffic and are not counted."""
     BH, N, d, L, NB = w.B * w.H, w.N, w.d, w.race_tables, 1 << w.race_bits
     e = 2 if w.dtype == "bf16" else 4
     rb = 1 if w.race_bits <= 8 else 2
     P = w.sort_bits + L * w.race_bits
     wk = window_keys(N, w.chunk) * BH       # query-key pairs of the sparse branch
     rows = BH * N
+    tables = BH * L * NB
     return {
-        # bound, amount, unit
-        "hash": ("tensor", 2.0 * 2 * rows * d * P, "flop"),
-        "sort": ("hbm", 2 * rows * (2 + 4) * 1.0, "byte"),
-        "race_build": ("alu", 1.0 * rows * L * d, "add"),
-        "sparse_fwd": ("tensor", 4.0 * wk * d, "flop"),
-        "race_fuse": ("hbm", 1.0 * rows * (L * rb + 4 * d * e + 8 + 4), "byte"),
-        "fuse_bwd": ("hbm", 1.0 * rows * (4 * d * e + d * e + 8 * d + 12), "byte"),
-        "race_bwd": ("alu", 2.0 * rows * L * d, "add"),
-        "sparse_bwd": ("tensor", 10.0 * wk * d, "flop"),
-        "finish": ("hbm", 1.0 * rows * d * (4 + e), "byte"),
+        "hash": (4.0 * rows * d * P, 2.0 * rows * d * e + 2 * rows * (2 + L * rb)),
+        "sort": (0.0, 2.0 * rows * (2 + 4)),
+        "race_build": (0.0, rows * (d * e + L * rb) + tables * (4.0 * d + 4)),
+        "sparse_fwd": (4.0 * wk * d, rows * (4.0 * d * e + 4 + 8)),
+        "race_fuse": (0.0, rows * (4.0 * d * e + L * rb + 8)),
+        "fuse_bwd": (0.0, rows * (6.0 * d * e + 24)),
+        "race_bwd": (0.0, rows * (d * e + L * rb) + tables * (1.0 * d * e)),
+        "sparse_bwd": (10.0 * wk * d, rows * (7.0 * d * e + 24 + 8)),
+        "finish": (0.0, rows * (2.0 * d * e + L * rb)),
     }
+
+
+def stage_roofline(flops, nbytes, sec, peaks):
+    """Bound = the resource with the longer ideal time; the tensor peak is the
+    sustained one (every stage runs inside a long step)."""
+    tf = peaks["bf16_tflops_sustained"] * 1e12
+    hb = peaks["hbm_gbs"] * 1e9
+    if flops / tf > nbytes / hb:
+        ach, peak, unit, bound = flops / sec / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s", "tensor"
+    else:
+        ach, peak, unit, bound = nbytes / sec / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
+    return {"bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
+            "ideal_us": 1e6 * max(flops / tf, nbytes / hb)}
+
+
+# DRAM bytes (read + write) of one launch of a stage's main kernel, from an
+# ncu capture of the same source (sha1 of the kernel file), scaled to the full
+# workload by the number of units; reported only while that file is unchanged.
+RECORDED_TRAFFIC = {
+    # stage: (kernel source, its sha1 at capture, bytes per full-size launch)
+    "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "9628a6a95e0435f02fdb79d609702aed00e31da4", 2.444e+08),
+    "race_build": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "d71bdb58cc88f62b77ee364f69f39b401eda6744", 1.368e+08),
+    "sparse_fwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_pipe.cu", "3a62fd41f041ed04cb99948b9f4c1fb587d46f41", 3.727e+08),
+    "race_fuse": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "d71bdb58cc88f62b77ee364f69f39b401eda6744", 3.564e+08),
+    "fuse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/fuse_bwd.cu", "b39e9fcf002feed95044d88de883f3eca4907efd", 5.719e+08),
+    "race_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "d71bdb58cc88f62b77ee364f69f39b401eda6744", 1.324e+08),
+    "sparse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_bwd3.cu", "41207b576a5dab9665cc1ed634181525c66ec267", 6.626e+08),
+    "finish": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "d71bdb58cc88f62b77ee364f69f39b401eda6744", 1.58e+08),
+}
+
+
+def recorded_traffic(stage):
+    rec = RECORDED_TRAFFIC.get(stage)
+    if rec is None:
+        return None
+    src, sha, nbytes = rec
+    try:
+        with open(os.path.join(ROOT, src), "rb") as f:
+            if hashlib.sha1(f.read()).hexdigest() != sha:
+                return None
+    except OSError:
+        return None
+    return nbytes
 
 
 def operator_roofline(w, peaks):
@@ -104,26 +152,58 @@ def operator_roofline(w, peaks):
             "bytes_fwdbwd": b_all}
 
 
-def alu_peak_adds_per_s(peaks):
-    """Shared-memory fp32 atomic adds per second: 148 SMs x 32 lanes per clock
-    (one conflict-free warp-wide shared atomic per SM per clock) at max SM clock."""
-    return 148 * 32 * peaks["sm_max_mhz"] * 1e6
-
-
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
+    """SM clock and clock-event reasons during the timed region: NVML polled
+    every 2 ms from a thread (reading only; nothing is set), else nvidia-smi
+    at its 50 ms floor."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
     def __init__(self, index: int):
         self.proc = None
         self.index = index
+        self.samples = []
+        self.nvml = None
+        self.thread = None
+        self.stop = None
+        self.out = ""
+
+    def _poll(self):
+        nv, h = self.nvml
+        while not self.stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((sm, mx, rs))
+            except Exception:   # a failed read leaves the sample out
+                pass
+            time.sleep(0.002)
 
     def __enter__(self):
+        try:
+            import pynvml as nv
+            import threading
+            nv.nvmlInit()
+            try:
+                idx = torch.cuda._get_nvml_device_index(self.index)
+            except Exception:
+                idx = self.index
+            self.nvml = (nv, nv.nvmlDeviceGetHandleByIndex(idx))
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
@@ -134,7 +214,9 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
-        self.out = ""
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -145,6 +227,13 @@ class ClockSampler:
         return False
 
     def summary(self):
+        if self.samples:
+            sm = [float(x[0]) for x in self.samples]
+            loaded = [v for v in sm if v > 0.5 * max(sm)]
+            reasons = sorted({name for x in self.samples for bit, name in self.REASONS.items()
+                              if x[2] & bit})
+            return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(x[1] for x in self.samples),
+                    "reasons": reasons, "samples": len(self.samples), "source": "nvml 2 ms"}
         rows = [r.split(",") for r in self.out.strip().splitlines() if r.count(",") >= 7]
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
@@ -153,10 +242,10 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4)
                           if r[4 + i].strip().lower() == "active"})
-        loaded = [s for s in sm if s > 0.5 * max(sm)] if sm else []
+        loaded = [v for v in sm if v > 0.5 * max(sm)] if sm else []
         return {"sm_mhz": statistics.median(loaded) if loaded else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(rows), "source": "nvidia-smi 50 ms"}
 
 
 # ---------------------------------------------------------------------------
@@ -374,15 +463,11 @@ def main():
         value = world * K * w.tokens / (total_ms / 1e3)
         fwd_value = world * K * w.tokens / (fwd_ms / 1e3)
         work = stage_work(w)
-        dom = max(stage_ms, key=lambda s: stage_ms[s])
-        bound, amount, unit = work[dom]
-        sec = stage_ms[dom] / 1e3
-        if bound == "tensor":
-            ach, peak, u = amount / sec / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
-        elif bound == "hbm":
-            ach, peak, u = amount / sec / 1e9, peaks["hbm_gbs"], "GB/s"
-        else:
-            ach, peak, u = amount / sec / 1e9, alu_peak_adds_per_s(peaks) / 1e9, "Gadd/s"
+        per_stage = {st: stage_roofline(*work[st], stage_ms[st] / 1e3, peaks)
+                     for st in stage_ms}
+        dom = max(stage_ms, key=lambda st: stage_ms[st])
+        rl = per_stage[dom]
+        traffic = recorded_traffic(dom)
         roof = operator_roofline(w, peaks)
         fwd_launch, bwd_launch = B.kernel_launches(p)
         line = {
@@ -398,10 +483,13 @@ def main():
                        "l2": "256 MB flush between timed steps; inputs 0.4 GB > L2"},
             "fwd_tokens_per_s": fwd_value,
             "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
-            "roofline": {"bound": bound, "kernel": dom, "achieved": ach, "peak": peak,
-                         "unit": u, "frac": ach / peak, "traffic": None,
-                         "peak_source": peaks["source"] + (" sustained" if bound == "tensor"
+            "roofline": {"bound": rl["bound"], "kernel": dom, "achieved": rl["achieved"],
+                         "peak": rl["peak"], "unit": rl["unit"], "frac": rl["frac"],
+                         "traffic": traffic,
+                         "peak_source": peaks["source"] + (" sustained" if rl["bound"] == "tensor"
                                                            else "")},
+            "stage_roofline": {st: {k: (round(v, 4) if isinstance(v, float) else v)
+                                    for k, v in r.items()} for st, r in per_stage.items()},
             "operator_roofline": {
                 "fwd_us": roof["fwd_us"], "fwdbwd_us": roof["fwdbwd_us"],
                 "frac_fwd": roof["fwd_us"] / (1e3 * fwd_ms / K),
