@@ -954,38 +954,45 @@ race_fuse_rows_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q
                       T* __restrict__ y, T* __restrict__ o_race, int32_t* __restrict__ ctot_out) {
   constexpr int QW = 32 / QL, EL = 16 / sizeof(T);
   constexpr int PER = 4 / (int)sizeof(CodeT);
-  const int lane = threadIdx.x & 31, ql = lane % QL, gbase = lane - ql;
+  // gate weights, and a two-row staging ring per warp for the q and O_sp
+  // chunks (each lane copies its own 16-byte chunks and reads them back), so
+  // neither sits in registers while the table lines are in flight
+  __shared__ float s_w[2 * 128];
+  __shared__ __align__(16) uint4 s_stage[8][2][2][32];
+  const int lane = threadIdx.x & 31, ql = lane % QL, gbase = lane - ql, wi = threadIdx.x >> 5;
   const uint64_t pol = l2_keep_policy();
   const int W = L * (int)sizeof(CodeT) / 4;
   const uint32_t table_bytes = (uint32_t)NB * (uint32_t)d * (uint32_t)sizeof(T);
   const int row_shift = 31 - __clz(d * (int)sizeof(T));   // d * sizeof is a power of two
   const float lam_v = *lam;
-  float ws8[EL], wr8[EL];
-#pragma unroll
-  for (int i = 0; i < EL; ++i) ws8[i] = wr8[i] = 0.f;
-  float bs = 0.f, br = 0.f;
-  if (!gate_fixed) {
-    load_el<float, EL>(gate_w + ql * EL, ws8);
-    load_el<float, EL>(gate_w + d + ql * EL, wr8);
-    bs = gate_b[0];
-    br = gate_b[1];
-  }
-  const int64_t first = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * QW;
+  for (int i = threadIdx.x; i < 2 * d; i += blockDim.x) s_w[i] = gate_fixed ? 0.f : gate_w[i];
+  const float bs = gate_fixed ? 0.f : gate_b[0], br = gate_fixed ? 0.f : gate_b[1];
+  __syncthreads();
+  const int64_t first = ((int64_t)blockIdx.x * (blockDim.x >> 5) + wi) * QW;
   const int64_t stride = (int64_t)gridDim.x * (blockDim.x >> 5) * QW;
+  auto stage = [&](int64_t r0, int buf) {
+    const int64_t rr = min(r0 + lane / QL, rows - 1);
+    const size_t base = (size_t)rr * d + ql * EL;
+    cp_async16b(smem_addr32(&s_stage[wi][buf][0][lane]), q + base, 16);
+    cp_async16b(smem_addr32(&s_stage[wi][buf][1][lane]), o_sp + base, 16);
+  };
   uint32_t w[WPL];
   {
     const int64_t r = min(first + lane / QL, rows - 1);
     load_row_codes<CodeT, QL, WPL>(rcode_q + r * L, W, ql, w);
   }
-  for (int64_t r0 = first; r0 < rows; r0 += stride) {
+  if (first < rows) stage(first, 0);
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  int buf = 0;
+  for (int64_t r0 = first; r0 < rows; r0 += stride, buf ^= 1) {
     const int64_t r = r0 + lane / QL;
     const bool valid = r < rows;
     const int64_t rr = valid ? r : rows - 1;
     const int64_t bh = rr / N;
     const size_t base = (size_t)rr * d + ql * EL;
-    // this row's streams and the next row's codes go out before the gathers
-    const uint4 q_raw = ld16_stream(q + base);
-    const uint4 os_raw = ld16_stream(o_sp + base);
+    // the next row's q / O_sp chunks and codes go out before this row's gathers
+    if (r0 + stride < rows) stage(r0 + stride, buf ^ 1);
+    asm volatile("cp.async.commit_group;" ::: "memory");
     const float lse_r = lse[rr];
     uint32_t wn[WPL];
     load_row_codes<CodeT, QL, WPL>(rcode_q + min(r + stride, rows - 1) * L, W, ql, wn);
@@ -994,10 +1001,10 @@ race_fuse_rows_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q
     const int32_t* cnt = counts + (size_t)bh * L * NB;
 #pragma unroll
     for (int i = 0; i < WPL; ++i) {
-      const int wi = ql + i * QL;
-      if (wi < W) {
+      const int wd = ql + i * QL;
+      if (wd < W) {
 #pragma unroll
-        for (int e = 0; e < PER; ++e) ctot += cnt[(size_t)(wi * PER + e) * NB + code_of<CodeT>(w[i], e)];
+        for (int e = 0; e < PER; ++e) ctot += cnt[(size_t)(wd * PER + e) * NB + code_of<CodeT>(w[i], e)];
       }
     }
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -1005,9 +1012,10 @@ race_fuse_rows_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q
                                   row_shift, gbase, pol, acc);
     ctot = group_sum_i<QL>(ctot);
     const float inv = ctot > 0 ? 1.0f / (float)ctot : 0.f;
+    asm volatile("cp.async.wait_group 1;" ::: "memory");   // this row's chunks are in
     float qv[EL], os[EL], orc[EL];
-    unpack16(q_raw, qv, q);
-    unpack16(os_raw, os, o_sp);
+    unpack16(s_stage[wi][buf][0][lane], qv, q);
+    unpack16(s_stage[wi][buf][1][lane], os, o_sp);
 #pragma unroll
     for (int i = 0; i < EL; ++i) orc[i] = acc[i] * inv;
     float gs = gs_fixed, gr = gr_fixed;
@@ -1015,8 +1023,8 @@ race_fuse_rows_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q
       float as = 0.f, ar = 0.f;
 #pragma unroll
       for (int i = 0; i < EL; ++i) {
-        as += qv[i] * ws8[i];
-        ar += qv[i] * wr8[i];
+        as += qv[i] * s_w[ql * EL + i];
+        ar += qv[i] * s_w[d + ql * EL + i];
       }
       as = group_sum<QL>(as) + bs;
       ar = group_sum<QL>(ar) + br;
@@ -1037,6 +1045,7 @@ race_fuse_rows_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q
 #pragma unroll
     for (int i = 0; i < WPL; ++i) w[i] = wn[i];
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 __global__ void to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst,
