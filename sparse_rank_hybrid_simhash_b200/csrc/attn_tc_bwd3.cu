@@ -22,18 +22,21 @@
 // output element is written by exactly one thread.  dv holds the sparse part
 // only; the RACE branch's part is added afterwards.
 //
-// Roles (320 threads, one CTA per SM):
-//   warp 0      producer: cp.async gathers of K/V key tiles (two-slot ring)
-//               and Q/dO query blocks with their lse, D' and (da_s, da_r)
-//               (two-slot ring)
+// Roles (448 threads, one CTA per SM):
+//   warp 0      producer: TMA row gathers (four rows per instruction, into
+//               128B-swizzled tiles) of K/V key tiles (two-slot ring) and Q/dO
+//               query blocks (two-slot ring), with the blocks' lse, D' and
+//               (da_s, da_r) by cp.async
 //   warp 1      MMA issuer (one thread) and TMEM owner; for pair p it issues
 //               S^T/dP^T of pair p + 1 as soon as P^T/dS^T of pair p are in
 //               shared memory, then dV, dK, dQ of pair p
 //   warps 2..9  elementwise: warp w reaches TMEM lanes 32 (w % 4) .. +31 and
 //               takes half of the query columns; P^T and dS^T (bf16) to
-//               shared memory; one pair after a query block's dQ is complete
-//               they write it out (its MMA has finished by then), and after
-//               a key tile's last pair they write out dV and dK
+//               shared memory, one 32-column chunk at a time; they also stage
+//               the token indices (and gate pairs) the epilogue needs
+//   warps 10-13 epilogue: a finished query block's dQ (+ gate part) and a
+//               finished key tile's dV and dK from TMEM to bf16 rows; TMEM is
+//               released as soon as it has been read, before the stores
 // TMEM: S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384),
 //       dQ [384,448) and [448,512) for alternating query blocks.
 // Every wait is bounded; a timeout records ERR_TIMEOUT and every role leaves
@@ -50,8 +53,9 @@ using namespace tc;
 
 constexpr int D = 64;
 constexpr int kTile = 128;
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 constexpr int kEwThreads = 256;
+constexpr int kEpThreads = 128;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTS = 0, kTdP = 128, kTdV = 256, kTdK = 320, kTdQ = 384;
 
@@ -69,13 +73,22 @@ struct Lay3 {
   static constexpr uint32_t kDpr = kLse + 2 * 128 * 4;      // [2][128] D'
   static constexpr uint32_t kDa = kDpr + 2 * 128 * 4;       // [2][128] (da_s, da_r)
   static constexpr uint32_t kW = kDa + 2 * 128 * 8;         // [2][64] w_s, w_r
-  static constexpr uint32_t kBar = kW + 2 * 64 * 4;
+  static constexpr uint32_t kFtok = kW + 2 * 64 * 4;        // [2][128] flush: query tokens
+  static constexpr uint32_t kFda = kFtok + 2 * 128 * 4;     // [2][128] flush: (da_s, da_r)
+  static constexpr uint32_t kKtok = kFda + 2 * 128 * 8;     // [2][128] write-out: key tokens
+  static constexpr uint32_t kBar = kKtok + 2 * 128 * 4;
   static constexpr uint32_t kDyn = kBar + 256;
+};
+
+// TMA maps of Q, K, V and dO as [B H N, 64] row matrices.
+struct RowMaps {
+  CUtensorMap q, k, v, o;
 };
 
 struct Bars3 {
   uint64_t full_kv[2], empty_kv[2], full_q[2], empty_q[2];
   uint64_t s_full, p_full, pd_free, kvacc_full, dq_full[2];
+  uint64_t dq_free[2], kvacc_free[2], fl_ready[2], key_ready[2];
   uint32_t tmem;
 };
 static_assert(sizeof(Bars3) <= 256, "barrier block");
@@ -183,10 +196,8 @@ ELSAA_DEV bool ew_all(bool v) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                 const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ perm_q,
-                 const int32_t* __restrict__ perm_k, const __nv_bfloat16* __restrict__ d_o,
-                 const float* __restrict__ lse, const float* __restrict__ dprime,
+attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict__ perm_q,
+                 const int32_t* __restrict__ perm_k, const float* __restrict__ lse, const float* __restrict__ dprime,
                  const float2* __restrict__ da, const float* __restrict__ gate_w, int BH,
                  int N, int chunk, float scale, float scale_log2, __nv_bfloat16* __restrict__ dq,
                  __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
@@ -219,11 +230,17 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars->full_kv[s], 64);   // 32 cp.async arrivals + 32 plain arrivals
+      // full: the producer's byte-count arrival, 32 plain arrivals (token
+      // indices) and, for query blocks, 32 cp.async arrivals (lse, D', da)
+      mbar_init(&bars->full_kv[s], 1 + 32);
       mbar_init(&bars->empty_kv[s], 1);
-      mbar_init(&bars->full_q[s], 64);
+      mbar_init(&bars->full_q[s], 1 + 32 + 32);
       mbar_init(&bars->empty_q[s], 1);
       mbar_init(&bars->dq_full[s], 1);
+      mbar_init(&bars->dq_free[s], kEpThreads);
+      mbar_init(&bars->kvacc_free[s], kEpThreads);
+      mbar_init(&bars->fl_ready[s], 128);   // elementwise threads of half 0
+      mbar_init(&bars->key_ready[s], 128);
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->p_full, kEwThreads);
@@ -243,63 +260,49 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    // Lane l handles rows l, l + 32, l + 64, l + 96 of a tile or block; rows
-    // are gathered 4 per warp instruction (8 lanes per row, 16 bytes each).
-    const int ch = lane & 7;
+    // Lane l handles rows 4 l .. 4 l + 3 of a tile or block: one 16-byte load
+    // of their token indices, one TMA gather of the four rows per matrix.
     auto load_kv = [&](int64_t n, int bh, int kb) -> bool {
       const size_t unit = (size_t)bh * N;
-      int idx[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) idx[j] = perm_k[unit + (size_t)kb * kTile + lane + 32 * j];
+      const int4 t4 = *reinterpret_cast<const int4*>(perm_k + unit + (size_t)kb * kTile + 4 * lane);
       const int s = (int)(n & 1);
       if (n >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars->empty_kv[s],
                                                       (uint32_t)(((n >> 1) - 1) & 1), err)))
         return false;
-      const uint32_t kst = sbase + Lay::kKv + s * Lay::kKvSlot;
-      const __nv_bfloat16* kb_ = k + unit * D;
-      const __nv_bfloat16* vb_ = v + unit * D;
-#pragma unroll
-      for (int it = 0; it < kTile / 4; ++it) {
-        const int row = 4 * it + (lane >> 3);
-        const int tok = __shfl_sync(0xffffffffu, idx[it >> 3], row & 31);
-        const size_t src = (size_t)tok * D + ch * 8;
-        cp_async16(kst + sw128_off(row, ch), kb_ + src, 16);
-        cp_async16(kst + Lay::kSub + sw128_off(row, ch), vb_ + src, 16);
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) s_kidx[s * 128 + lane + 32 * j] = idx[j];
-      cp_async_arrive(&bars->full_kv[s]);
+      if (lane == 0) mbar_arrive_expect_tx(&bars->full_kv[s], 2u * kTile * 128u);
+      __syncwarp();
+      const uint32_t kst = sbase + Lay::kKv + s * Lay::kKvSlot + lane * 512;
+      const int u = (int)unit;
+      tma_gather4(kst, &maps.k, u + t4.x, u + t4.y, u + t4.z, u + t4.w, &bars->full_kv[s]);
+      tma_gather4(kst + Lay::kSub, &maps.v, u + t4.x, u + t4.y, u + t4.z, u + t4.w,
+                  &bars->full_kv[s]);
+      *reinterpret_cast<int4*>(s_kidx + s * 128 + 4 * lane) = t4;
       mbar_arrive(&bars->full_kv[s]);
       return true;
     };
     auto load_q = [&](int64_t n, int bh, int qb) -> bool {
       const size_t unit = (size_t)bh * N;
-      int idx[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) idx[j] = perm_q[unit + (size_t)qb * kTile + lane + 32 * j];
+      const int4 t4 = *reinterpret_cast<const int4*>(perm_q + unit + (size_t)qb * kTile + 4 * lane);
       const int s = (int)(n & 1);
       if (n >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars->empty_q[s],
                                                       (uint32_t)(((n >> 1) - 1) & 1), err)))
         return false;
-      const uint32_t qst = sbase + Lay::kQ + s * Lay::kQSlot;
-      const __nv_bfloat16* qb_ = q + unit * D;
-      const __nv_bfloat16* ob_ = d_o + unit * D;
-#pragma unroll
-      for (int it = 0; it < kTile / 4; ++it) {
-        const int row = 4 * it + (lane >> 3);
-        const int tok = __shfl_sync(0xffffffffu, idx[it >> 3], row & 31);
-        const size_t src = (size_t)tok * D + ch * 8;
-        cp_async16(qst + sw128_off(row, ch), qb_ + src, 16);
-        cp_async16(qst + Lay::kSub + sw128_off(row, ch), ob_ + src, 16);
-      }
+      if (lane == 0) mbar_arrive_expect_tx(&bars->full_q[s], 2u * kTile * 128u);
+      __syncwarp();
+      const uint32_t qst = sbase + Lay::kQ + s * Lay::kQSlot + lane * 512;
+      const int u = (int)unit;
+      tma_gather4(qst, &maps.q, u + t4.x, u + t4.y, u + t4.z, u + t4.w, &bars->full_q[s]);
+      tma_gather4(qst + Lay::kSub, &maps.o, u + t4.x, u + t4.y, u + t4.z, u + t4.w,
+                  &bars->full_q[s]);
+      const int tk[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int r = lane + 32 * j;
-        cp_async4(smem_u32(s_lse + s * 128 + r), lse + unit + idx[j]);
-        cp_async4(smem_u32(s_dpr + s * 128 + r), dprime + unit + idx[j]);
-        cp_async8(smem_u32(s_da + s * 128 + r), da + unit + idx[j]);
-        s_qidx[s * 128 + r] = idx[j];
+        const int r = 4 * lane + j;
+        cp_async4(smem_u32(s_lse + s * 128 + r), lse + unit + tk[j]);
+        cp_async4(smem_u32(s_dpr + s * 128 + r), dprime + unit + tk[j]);
+        cp_async8(smem_u32(s_da + s * 128 + r), da + unit + tk[j]);
       }
+      *reinterpret_cast<int4*>(s_qidx + s * 128 + 4 * lane) = t4;
       cp_async_arrive(&bars->full_q[s]);
       mbar_arrive(&bars->full_q[s]);
       return true;
@@ -354,6 +357,8 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
       PairIter it;
       it.init(&run);
       Pair cur = it.get();
+      // per dQ buffer b (bit b): has it been flushed yet; parity of its flush count
+      uint32_t fl_any = 0u, fl_par = 0u;
       ok = wait_data(cur);
       if (ok) issue_s(cur);
       for (int64_t pi = 0; ok; ++pi) {
@@ -371,6 +376,19 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
           issue_s(nxt);
         }
         const uint32_t ks = kv_slot(cur.kvs), qs = q_slot(cur.qs);
+        if (cur.kv && cur.first_of_tile && cur.tile >= 1) {
+          // the epilogue has read the previous tile's dV / dK
+          ok = mbar_wait(&bars->kvacc_free[(cur.tile - 1) & 1],
+                         (uint32_t)(((cur.tile - 1) >> 1) & 1), err);
+          if (!ok) break;
+        }
+        if (cur.dq && !cur.dq_acc && ((fl_any >> (cur.qs & 1)) & 1u)) {
+          // the epilogue has read this dQ buffer's previous block
+          const int b = (int)(cur.qs & 1);
+          ok = mbar_wait(&bars->dq_free[b], ((fl_par >> b) & 1u) ^ 1u, err);
+          if (!ok) break;
+        }
+        fence_after();
         if (cur.kv) {
           const uint32_t id_kv = idesc_bf16(128, D, false, true);
           for (int s = 0; s < cur.nq / 16; ++s) {
@@ -395,15 +413,19 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         if (cur.release_kv) mma_commit(&bars->empty_kv[cur.kvs & 1]);
         if (cur.release_q) mma_commit(&bars->empty_q[cur.qs & 1]);
         if (cur.kv && cur.last_of_tile) mma_commit(&bars->kvacc_full);
-        if (cur.flush) mma_commit(&bars->dq_full[cur.qs & 1]);
+        if (cur.flush) {
+          mma_commit(&bars->dq_full[cur.qs & 1]);
+          fl_any |= 1u << (cur.qs & 1);
+          fl_par ^= 1u << (cur.qs & 1);
+        }
         if (!more) break;
         it = nx;
         cur = nxt;
       }
     }
     __syncwarp();
-  } else {
-    // ---------------------------------------------------------------- elementwise + epilogues
+  } else if (warp < 10) {
+    // ---------------------------------------------------------------- elementwise
     const int ew = tid - 64;                           // 0 .. 255
     const int quarter = warp & 3, half = (warp - 2) >> 2;
     const int row = 32 * quarter + lane;               // TMEM lane
@@ -411,46 +433,14 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     const bool masked = chunk < kTile;
     int lc = 0;
     while ((1 << lc) < chunk) ++lc;
-    uint32_t flush_parity = 0u;   // bit b: parity of the next completion of dQ buffer b
-    int64_t ntile = 0;
-    int key_tok = 0;
-    // the query block whose dQ is written out one pair later
-    bool pend = false;
-    int pend_buf = 0, pend_tok = 0;
-    size_t pend_unit = 0;
-    float2 pend_da = make_float2(0.f, 0.f);
-    const float* wsv = s_w + half * 32;        // this thread's 32 columns of w_s
-    const float* wrv = s_w + D + half * 32;    // and of w_r
-    auto flush = [&]() -> bool {
-      // dQ of the pending block: TMEM lane = query row, this warp's 32 columns
-      const int b = pend_buf;
-      if (!ew_all(mbar_wait(&bars->dq_full[b], (flush_parity >> b) & 1u, err))) return false;
-      flush_parity ^= 1u << b;
-      fence_after();
-      float g[32];
-      tmem_ld32(tmem + kTdQ + b * D + lane_off + half * 32, g);
-      tmem_ld_wait();
-      __nv_bfloat16* out = dq + (pend_unit + pend_tok) * D + half * 32;
-#pragma unroll
-      for (int q8 = 0; q8 < 4; ++q8) {
-        float x[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int c = q8 * 8 + e;
-          x[e] = fmaf(pend_da.x, wsv[c], fmaf(pend_da.y, wrv[c], scale * g[c]));
-        }
-        *reinterpret_cast<uint4*>(out + q8 * 8) =
-            make_uint4(pack2(x[0], x[1]), pack2(x[2], x[3]), pack2(x[4], x[5]), pack2(x[6], x[7]));
-      }
-      fence_before();
-      pend = false;
-      return true;
-    };
+    uint32_t fl_any = 0u, fl_par = 0u;   // per dQ buffer b (bit b): staged yet; parity of count
+    int32_t* s_ftok = reinterpret_cast<int32_t*>(smem + Lay::kFtok);
+    float2* s_fda = reinterpret_cast<float2*>(smem + Lay::kFda);
+    int32_t* s_ktok = reinterpret_cast<int32_t*>(smem + Lay::kKtok);
     PairIter it;
     it.init(&run);
     for (int64_t pi = 0; run.count > 0 && !it.done(); ++pi, it.advance()) {
       const Pair p = it.get();
-      const size_t unit = (size_t)p.bh * N;
       const int qslot = (int)(p.qs & 1), kslot = (int)(p.kvs & 1);
       ok = ew_all(mbar_wait(&bars->s_full, (uint32_t)(pi & 1), err) &&
                   mbar_wait(&bars->full_q[qslot], (uint32_t)((p.qs >> 1) & 1), err) &&
@@ -463,18 +453,38 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         if (ew < 128) ls[ew] *= 1.4426950408889634f;
         ew_sync();
       }
-      if (p.first_of_tile && p.kv) key_tok = s_kidx[kslot * 128 + row];
-      int flush_tok = 0;
-      float2 flush_da = make_float2(0.f, 0.f);
+      // stage the epilogue's inputs (key tokens of a new tile; query tokens
+      // and gate pairs of a block whose dQ completes with this pair), once
+      // the epilogue is done with the buffer's previous contents
+      if (p.kv && p.first_of_tile) {
+        const int par = (int)(p.tile & 1);
+        if (p.tile >= 2) {
+          ok = ew_all(mbar_wait(&bars->kvacc_free[par], (uint32_t)(((p.tile >> 1) - 1) & 1), err));
+          if (!ok) break;
+        }
+        if (half == 0) {
+          s_ktok[par * 128 + row] = s_kidx[kslot * 128 + row];
+          mbar_arrive(&bars->key_ready[par]);
+        }
+      }
       if (p.flush) {
-        flush_tok = s_qidx[qslot * 128 + row];
-        flush_da = s_da[qslot * 128 + row];
+        const int b = qslot;
+        if ((fl_any >> b) & 1u) {
+          ok = ew_all(mbar_wait(&bars->dq_free[b], ((fl_par >> b) & 1u) ^ 1u, err));
+          if (!ok) break;
+        }
+        fl_any |= 1u << b;
+        fl_par ^= 1u << b;
+        if (half == 0) {
+          s_ftok[b * 128 + row] = s_qidx[qslot * 128 + row];
+          s_fda[b * 128 + row] = s_da[qslot * 128 + row];
+          mbar_arrive(&bars->fl_ready[b]);
+        }
       }
       // visible query columns of this key row: ranks [i c, (i + 2) c)
       const int key_chunk = (p.kb * kTile + row) >> lc;
       const int lo = (key_chunk << lc) - p.qb * kTile, hi = lo + 2 * chunk;
       const int cend = min(hi, p.nq);
-      uint32_t pw[2][16], dw[2][16];
 #pragma unroll
       for (int cb = 0; cb < 2; ++cb) {
         const int c0 = half * 64 + cb * 32;
@@ -482,6 +492,7 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         tmem_ld32(tmem + kTS + lane_off + c0, sv);
         tmem_ld32(tmem + kTdP + lane_off + c0, dp);
         tmem_ld_wait();
+        uint32_t pw[16], dw[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
           const float2 l2 = *reinterpret_cast<const float2*>(ls + c0 + i);
@@ -493,67 +504,106 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
             p0 = (col >= lo && col < cend) ? p0 : 0.f;
             p1 = (col + 1 >= lo && col + 1 < cend) ? p1 : 0.f;
           }
-          pw[cb][i >> 1] = pack2(p0, p1);
-          dw[cb][i >> 1] = pack2(p0 * (dp[i] - d2.x), p1 * (dp[i + 1] - d2.y));
+          pw[i >> 1] = pack2(p0, p1);
+          dw[i >> 1] = pack2(p0 * (dp[i] - d2.x), p1 * (dp[i + 1] - d2.y));
         }
-      }
-      if (pi >= 1) {   // the MMAs of the previous pair are done with P^T / dS^T
-        ok = ew_all(mbar_wait(&bars->pd_free, (uint32_t)((pi - 1) & 1), err));
-        if (!ok) break;
-      }
-#pragma unroll
-      for (int cb = 0; cb < 2; ++cb) {
+        if (cb == 0 && pi >= 1) {   // the MMAs of the previous pair are done with P^T / dS^T
+          ok = ew_all(mbar_wait(&bars->pd_free, (uint32_t)((pi - 1) & 1), err));
+          if (!ok) break;
+        }
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
-          const int col = half * 64 + cb * 32 + q8 * 8;
+          const int col = c0 + q8 * 8;
           const uint32_t off = (col >> 6) * Lay::kSub + sw128_off(row, (col & 63) >> 3);
           if (p.kv)
             *reinterpret_cast<uint4*>(smem + Lay::kPT + off) =
-                make_uint4(pw[cb][q8 * 4], pw[cb][q8 * 4 + 1], pw[cb][q8 * 4 + 2], pw[cb][q8 * 4 + 3]);
+                make_uint4(pw[q8 * 4], pw[q8 * 4 + 1], pw[q8 * 4 + 2], pw[q8 * 4 + 3]);
           *reinterpret_cast<uint4*>(smem + Lay::kDST + off) =
-              make_uint4(dw[cb][q8 * 4], dw[cb][q8 * 4 + 1], dw[cb][q8 * 4 + 2], dw[cb][q8 * 4 + 3]);
+              make_uint4(dw[q8 * 4], dw[q8 * 4 + 1], dw[q8 * 4 + 2], dw[q8 * 4 + 3]);
         }
       }
+      if (!ok) break;
       fence_async_smem();
       fence_before();
       mbar_arrive(&bars->p_full);
-
-      if (pend) {
-        ok = flush();
-        if (!ok) break;
-      }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    // warp w reaches TMEM lanes 32 (w % 4) .. +31: row = query row of a dQ
+    // buffer or key row of dV / dK
+    const int row = 32 * (warp & 3) + lane;
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const int32_t* s_ftok = reinterpret_cast<const int32_t*>(smem + Lay::kFtok);
+    const float2* s_fda = reinterpret_cast<const float2*>(smem + Lay::kFda);
+    const int32_t* s_ktok = reinterpret_cast<const int32_t*>(smem + Lay::kKtok);
+    uint32_t fl_par = 0u;   // bit b: parity of the next flush of dQ buffer b
+    int64_t ntile = 0;
+    PairIter it;
+    it.init(&run);
+    for (; run.count > 0 && !it.done() && ok; it.advance()) {
+      const Pair p = it.get();
+      const size_t unit = (size_t)p.bh * N;
       if (p.flush) {
-        pend = true;
-        pend_buf = (int)(p.qs & 1);
-        pend_tok = flush_tok;
-        pend_unit = unit;
-        pend_da = flush_da;
+        const int b = (int)(p.qs & 1);
+        const uint32_t par = (fl_par >> b) & 1u;
+        ok = mbar_wait(&bars->fl_ready[b], par, err) && mbar_wait(&bars->dq_full[b], par, err);
+        if (!ok) break;
+        fl_par ^= 1u << b;
+        fence_after();
+        float g[64];
+        tmem_ld32(tmem + kTdQ + b * D + lane_off, g);
+        tmem_ld32(tmem + kTdQ + b * D + lane_off + 32, g + 32);
+        tmem_ld_wait();
+        const int tok = s_ftok[b * 128 + row];
+        const float2 da2 = s_fda[b * 128 + row];
+        fence_before();
+        mbar_arrive(&bars->dq_free[b]);
+        __nv_bfloat16* out = dq + (unit + tok) * D;
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) {
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int c = q8 * 8 + e;
+            x[e] = fmaf(da2.x, s_w[c], fmaf(da2.y, s_w[D + c], scale * g[c]));
+          }
+          *reinterpret_cast<uint4*>(out + q8 * 8) =
+              make_uint4(pack2(x[0], x[1]), pack2(x[2], x[3]), pack2(x[4], x[5]), pack2(x[6], x[7]));
+        }
       }
       if (p.kv && p.last_of_tile) {
-        // dV (+ the RACE branch's dv) from half 0, dK from half 1, of this key row
-        ok = ew_all(mbar_wait(&bars->kvacc_full, (uint32_t)(ntile & 1), err));
+        const int par = (int)(ntile & 1);
+        ok = mbar_wait(&bars->key_ready[par], (uint32_t)((ntile >> 1) & 1), err) &&
+             mbar_wait(&bars->kvacc_full, (uint32_t)(ntile & 1), err);
         if (!ok) break;
-        ++ntile;
         fence_after();
-        const uint32_t col = half == 0 ? kTdV : kTdK;
-        const float mul = half == 0 ? 1.0f : scale;
-        __nv_bfloat16* out = (half == 0 ? dv : dk) + (unit + key_tok) * D;
+        uint32_t vw[32], kw[32];
         for (int c0 = 0; c0 < D; c0 += 32) {
-          float gv[32];
-          tmem_ld32(tmem + col + lane_off + c0, gv);
+          float gv[32], gk[32];
+          tmem_ld32(tmem + kTdV + lane_off + c0, gv);
+          tmem_ld32(tmem + kTdK + lane_off + c0, gk);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) gv[e] *= mul;
-#pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8)
-            *reinterpret_cast<uint4*>(out + c0 + q8 * 8) =
-                make_uint4(pack2(gv[q8 * 8], gv[q8 * 8 + 1]), pack2(gv[q8 * 8 + 2], gv[q8 * 8 + 3]),
-                           pack2(gv[q8 * 8 + 4], gv[q8 * 8 + 5]), pack2(gv[q8 * 8 + 6], gv[q8 * 8 + 7]));
+          for (int e = 0; e < 32; e += 2) {
+            vw[(c0 + e) >> 1] = pack2(gv[e], gv[e + 1]);
+            kw[(c0 + e) >> 1] = pack2(scale * gk[e], scale * gk[e + 1]);
+          }
         }
+        const int tok = s_ktok[par * 128 + row];
         fence_before();
+        mbar_arrive(&bars->kvacc_free[par]);
+        ++ntile;
+        __nv_bfloat16* ov = dv + (unit + tok) * D;
+        __nv_bfloat16* ok_ = dk + (unit + tok) * D;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          *reinterpret_cast<uint4*>(ov + q * 8) =
+              make_uint4(vw[4 * q], vw[4 * q + 1], vw[4 * q + 2], vw[4 * q + 3]);
+          *reinterpret_cast<uint4*>(ok_ + q * 8) =
+              make_uint4(kw[4 * q], kw[4 * q + 1], kw[4 * q + 2], kw[4 * q + 3]);
+        }
       }
     }
-    if (ok && pend) ok = flush();
   }
   fence_before();
   __syncthreads();
@@ -566,8 +616,9 @@ attn_bwd3_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 }  // namespace
 
 bool attn_bwd3_supported(const Geometry& g) {
+  // TMA row coordinates are 32-bit
   return g.bf16 && g.d == D && g.N % kTile == 0 && g.chunk >= 16 && g.chunk <= kTile &&
-         kTile % g.chunk == 0;
+         kTile % g.chunk == 0 && (int64_t)g.BH * g.N < (int64_t)1 << 31;
 }
 
 cudaError_t launch_attn_bwd3(const Geometry& g, const void* q, const void* k, const void* v,
@@ -579,15 +630,19 @@ cudaError_t launch_attn_bwd3(const Geometry& g, const void* q, const void* k, co
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Lay3::kDyn);
   if (e != cudaSuccess) return e;
+  RowMaps maps;
+  const uint64_t rows = (uint64_t)g.BH * g.N;
+  if ((e = make_row_map(&maps.q, q, rows)) != cudaSuccess) return e;
+  if ((e = make_row_map(&maps.k, k, rows)) != cudaSuccess) return e;
+  if ((e = make_row_map(&maps.v, v, rows)) != cudaSuccess) return e;
+  if ((e = make_row_map(&maps.o, d_o, rows)) != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t ntiles = (int64_t)g.BH * (g.N / kTile);
   const int grid = (int)(ntiles < sms ? ntiles : sms);
   attn_bwd3_kernel<<<grid, kThreads, Lay3::kDyn, s>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-      static_cast<const __nv_bfloat16*>(v), perm_q, perm_k,
-      static_cast<const __nv_bfloat16*>(d_o), lse, dprime, da, gate_w, g.BH, g.N, g.chunk,
+      maps, perm_q, perm_k, lse, dprime, da, gate_w, g.BH, g.N, g.chunk,
       g.scale, g.scale * 1.4426950408889634f, static_cast<__nv_bfloat16*>(dq),
       static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), err);
   return cudaGetLastError();

@@ -15,10 +15,10 @@
 // [128, 256)); the softmax is exact in one pass (row max first, then exp).
 //
 // Roles (320 threads, one CTA per SM):
-//   warp 0      producer: token indices (prefetched one tile ahead, held in
-//               registers and broadcast by shuffles), cp.async gathers of Q
-//               tiles (two-slot ring) and K/V blocks (four-slot ring) into
-//               128B-swizzled tiles; completion arrives on full_q / full_kv
+//   warp 0      producer: token indices (prefetched one tile ahead), TMA row
+//               gathers (four rows per instruction) of Q tiles (two-slot
+//               ring) and K/V blocks (four-slot ring) into 128B-swizzled
+//               tiles; completion counted in bytes on full_q / full_kv
 //   warp 1      MMA issuer (one thread) and TMEM owner:
 //                 O(j-1) = P V        as soon as P of tile j-1 is written
 //                 S(j)   = Q K^T      -> TMEM [0, 256)
@@ -61,6 +61,11 @@ struct PipeLayout {
   static constexpr uint32_t kDyn = kBar + 256;
 };
 
+// TMA maps of Q, K and V as [B H N, 64] row matrices.
+struct FwdMaps {
+  CUtensorMap q, k, v;
+};
+
 struct Bars {
   uint64_t full_q[kQSlots], empty_q[kQSlots], full_kv[kKvSlots], empty_kv[kKvSlots];
   uint64_t s_full, p_full, o_full[2], o_free[2];
@@ -92,11 +97,6 @@ struct Run {
     return ti;
   }
 };
-
-ELSAA_DEV void cp_async_arrive(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
 
 // 2^x on the special-function unit (approximate, flushes denormals).
 ELSAA_DEV float ex2(float x) {
@@ -141,8 +141,7 @@ ELSAA_DEV Cols tile_cols(const TileInfo& ti, int chunk) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-attn_fwd_pipe_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                     const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ perm_q,
+attn_fwd_pipe_kernel(const __grid_constant__ FwdMaps maps, const int32_t* __restrict__ perm_q,
                      const int32_t* __restrict__ perm_k, int BH, int N, int chunk,
                      float scale_log2, __nv_bfloat16* __restrict__ o_sp, float* __restrict__ lse,
                      uint32_t* __restrict__ err) {
@@ -166,11 +165,11 @@ attn_fwd_pipe_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
 
   if (tid == 0) {
     for (int s = 0; s < kQSlots; ++s) {
-      mbar_init(&bars->full_q[s], 32);
+      mbar_init(&bars->full_q[s], 1);   // the producer's byte-count arrival
       mbar_init(&bars->empty_q[s], 1);
     }
     for (int s = 0; s < kKvSlots; ++s) {
-      mbar_init(&bars->full_kv[s], 32);
+      mbar_init(&bars->full_kv[s], 1);
       mbar_init(&bars->empty_kv[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -193,62 +192,48 @@ attn_fwd_pipe_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    // Lane l holds the token indices of rows l, l + 32, l + 64, l + 96 of the
-    // next Q tile and K/V block; a block's rows are gathered 4 per warp
-    // instruction (8 lanes per row, one 16-byte chunk each).
-    const int ch = lane & 7;
-    auto load_idx = [&](const int32_t* perm, size_t base, int (&idx)[4]) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) idx[j] = perm[base + lane + 32 * j];
+    // Lane l handles rows 4 l .. 4 l + 3 of the next Q tile and K/V block: its
+    // four token indices arrive in one 16-byte load (prefetched one tile
+    // ahead) and each matrix's four rows in one TMA gather; lane 0 first
+    // arms the slot's barrier with the tile's byte count.
+    auto load_idx = [&](const int32_t* perm, size_t base) {
+      return *reinterpret_cast<const int4*>(perm + base + 4 * lane);
     };
-    auto issue_kv = [&](int64_t n, size_t unit, const int (&idx)[4]) -> bool {
+    auto issue_kv = [&](int64_t n, size_t unit, int4 t4) -> bool {
       const int s = (int)(n % kKvSlots);
       if (n >= kKvSlots &&
           !__all_sync(0xffffffffu,
                       mbar_wait(&bars->empty_kv[s], (uint32_t)(((n / kKvSlots) - 1) & 1), err)))
         return false;
-      const uint32_t kst = sbase + Lay::kKv + s * Lay::kKvSlot;
-      const __nv_bfloat16* kb = k + unit * D;
-      const __nv_bfloat16* vb = v + unit * D;
-#pragma unroll
-      for (int it = 0; it < kTile / 4; ++it) {
-        const int row = 4 * it + (lane >> 3);
-        const int tok = __shfl_sync(0xffffffffu, idx[it >> 3], row & 31);
-        const size_t src = (size_t)tok * D + ch * 8;
-        cp_async16(kst + sw128_off(row, ch), kb + src, 16);
-        cp_async16(kst + Lay::kTileBytes + sw128_off(row, ch), vb + src, 16);
-      }
-      cp_async_arrive(&bars->full_kv[s]);
+      if (lane == 0) mbar_arrive_expect_tx(&bars->full_kv[s], 2u * kTile * 128u);
+      __syncwarp();
+      const uint32_t kst = sbase + Lay::kKv + s * Lay::kKvSlot + lane * 512;
+      const int u = (int)unit;
+      tma_gather4(kst, &maps.k, u + t4.x, u + t4.y, u + t4.z, u + t4.w, &bars->full_kv[s]);
+      tma_gather4(kst + Lay::kTileBytes, &maps.v, u + t4.x, u + t4.y, u + t4.z, u + t4.w,
+                  &bars->full_kv[s]);
       return true;
     };
-    auto issue_q = [&](int64_t j, size_t unit, const int (&idx)[4]) -> bool {
+    auto issue_q = [&](int64_t j, size_t unit, int4 t4) -> bool {
       const int s = (int)(j % kQSlots);
       if (j >= kQSlots &&
           !__all_sync(0xffffffffu,
                       mbar_wait(&bars->empty_q[s], (uint32_t)(((j / kQSlots) - 1) & 1), err)))
         return false;
-      const uint32_t qst = sbase + Lay::kQ + s * Lay::kTileBytes;
-      const __nv_bfloat16* qb = q + unit * D;
-#pragma unroll
-      for (int it = 0; it < kTile / 4; ++it) {
-        const int row = 4 * it + (lane >> 3);
-        const int tok = __shfl_sync(0xffffffffu, idx[it >> 3], row & 31);
-        cp_async16(qst + sw128_off(row, ch), qb + (size_t)tok * D + ch * 8, 16);
-      }
-      cp_async_arrive(&bars->full_q[s]);
+      if (lane == 0) mbar_arrive_expect_tx(&bars->full_q[s], kTile * 128u);
+      __syncwarp();
+      const uint32_t qst = sbase + Lay::kQ + s * Lay::kTileBytes + lane * 512;
+      const int u = (int)unit;
+      tma_gather4(qst, &maps.q, u + t4.x, u + t4.y, u + t4.z, u + t4.w, &bars->full_q[s]);
       return true;
     };
-    int qi[4], ki[4];
+    int4 qi = make_int4(0, 0, 0, 0), ki = make_int4(0, 0, 0, 0);
     if (run.count > 0) {
       const TileInfo t0 = run.tile(0);
       const size_t unit = (size_t)t0.bh * N;
-      if (run.extra) {
-        int pi[4];
-        load_idx(perm_k, unit + (size_t)(t0.tb - 1) * kTile, pi);
-        ok = issue_kv(0, unit, pi);
-      }
-      load_idx(perm_q, unit + (size_t)t0.tb * kTile, qi);
-      load_idx(perm_k, unit + (size_t)t0.tb * kTile, ki);
+      if (run.extra) ok = issue_kv(0, unit, load_idx(perm_k, unit + (size_t)(t0.tb - 1) * kTile));
+      qi = load_idx(perm_q, unit + (size_t)t0.tb * kTile);
+      ki = load_idx(perm_k, unit + (size_t)t0.tb * kTile);
     }
     for (int64_t j = 0; j < run.count && ok; ++j) {
       const TileInfo ti = run.tile(j);
@@ -258,11 +243,11 @@ attn_fwd_pipe_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       if (j + 1 < run.count) {   // prefetch the next tile's indices
         const TileInfo tn = run.tile(j + 1);
         const size_t un = (size_t)tn.bh * N;
-        load_idx(perm_q, un + (size_t)tn.tb * kTile, qi);
-        load_idx(perm_k, un + (size_t)tn.tb * kTile, ki);
+        qi = load_idx(perm_q, un + (size_t)tn.tb * kTile);
+        ki = load_idx(perm_k, un + (size_t)tn.tb * kTile);
       }
     }
-    cp_async_wait_all();
+
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
@@ -308,7 +293,6 @@ attn_fwd_pipe_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
           ok = mbar_wait(&bars->full_kv[kv_ready % kKvSlots],
                          (uint32_t)((kv_ready / kKvSlots) & 1), err);
         if (!ok) break;
-        fence_async_smem();   // cp.async data -> tensor core
         fence_after();
         const uint32_t qst = sbase + Lay::kQ + (uint32_t)(j % kQSlots) * Lay::kTileBytes;
         if (ti.has_prev) {
@@ -441,8 +425,9 @@ attn_fwd_pipe_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
 }  // namespace
 
 bool attn_pipe_supported(const Geometry& g) {
+  // TMA row coordinates are 32-bit
   return g.bf16 && g.d == 64 && g.N % kTile == 0 && g.chunk % 16 == 0 && g.chunk <= kTile &&
-         kTile % g.chunk == 0;
+         kTile % g.chunk == 0 && (int64_t)g.BH * g.N < (int64_t)1 << 31;
 }
 
 cudaError_t launch_attn_fwd_pipe(const Geometry& g, const void* q, const void* k, const void* v,
@@ -457,9 +442,13 @@ cudaError_t launch_attn_fwd_pipe(const Geometry& g, const void* q, const void* k
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t ntiles = (int64_t)g.BH * (g.N / kTile);
   const int grid_x = (int)(ntiles < sms ? ntiles : sms);
+  FwdMaps maps;
+  const uint64_t rows = (uint64_t)g.BH * g.N;
+  if ((e = make_row_map(&maps.q, q, rows)) != cudaSuccess) return e;
+  if ((e = make_row_map(&maps.k, k, rows)) != cudaSuccess) return e;
+  if ((e = make_row_map(&maps.v, v, rows)) != cudaSuccess) return e;
   attn_fwd_pipe_kernel<<<grid_x, kThreads, PipeLayout::kDyn, s>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-      static_cast<const __nv_bfloat16*>(v), perm_q, perm_k, g.BH, g.N, g.chunk,
+      maps, perm_q, perm_k, g.BH, g.N, g.chunk,
       g.scale * 1.4426950408889634f, static_cast<__nv_bfloat16*>(o_sp), lse, err);
   return cudaGetLastError();
 }

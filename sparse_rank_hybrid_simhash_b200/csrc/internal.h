@@ -2,6 +2,7 @@
 // launchers each .cu file provides.  Not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -160,5 +161,9 @@ cudaError_t launch_fuse_bwd(const Geometry& g, const void* q, const void* dy, co
 cudaError_t launch_param_reduce(const Geometry& g, const float* partials, float* dgate_w,
                                 float* dgate_b, float* dlambda, cudaStream_t s);
 cudaError_t launch_cast_out(const Geometry& g, const float* src, void* dst, cudaStream_t s);
+
+// 2-D TMA map over a [rows, 64] bf16 matrix: one 128-byte row per box,
+// 128-byte swizzle; the row gathers of the tcgen05 attention kernels use it.
+cudaError_t make_row_map(CUtensorMap* map, const void* base, uint64_t rows);
 
 }  // namespace elsaa

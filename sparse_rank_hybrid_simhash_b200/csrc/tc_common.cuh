@@ -153,6 +153,27 @@ ELSAA_DEV void mma_commit(uint64_t* bar) {
       : "memory");
 }
 
+// ---- TMA ------------------------------------------------------------------
+
+// Arrives on `bar` and adds `bytes` to the transaction count its phase waits for.
+ELSAA_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// Four rows of a 2-D tensor map (box: one row of 64 bf16 = 128 bytes) at row
+// coordinates r0..r3 into 512 consecutive bytes of shared memory at `dst`
+// (128B-swizzled by the map); completion is counted on `bar` in bytes.
+ELSAA_DEV void tma_gather4(uint32_t dst, const void* map, int r0, int r1, int r2, int r3,
+                           uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(map), "r"(0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // ---- cp.async --------------------------------------------------------------
 
 // 16-byte global -> shared copy; src_bytes = 0 zero-fills the destination.
