@@ -69,8 +69,8 @@ struct Lay3 {
   static constexpr uint32_t kDST = kPT + 2 * kSub;          // dS^T [128 keys][128 queries]
   static constexpr uint32_t kKidx = kDST + 2 * kSub;        // [2][128] key tokens
   static constexpr uint32_t kQidx = kKidx + 2 * 128 * 4;    // [2][128] query tokens
-  static constexpr uint32_t kLse = kQidx + 2 * 128 * 4;     // [2][128] lse (log2 units once used)
-  static constexpr uint32_t kDpr = kLse + 2 * 128 * 4;      // [2][128] D'
+  static constexpr uint32_t kLse = kQidx + 2 * 128 * 4;     // [2][128] lse (-log2 units once used)
+  static constexpr uint32_t kDpr = kLse + 2 * 128 * 4;      // [2][128] D' (negated once used)
   static constexpr uint32_t kDa = kDpr + 2 * 128 * 4;       // [2][128] (da_s, da_r)
   static constexpr uint32_t kW = kDa + 2 * 128 * 8;         // [2][64] w_s, w_r
   static constexpr uint32_t kFtok = kW + 2 * 64 * 4;        // [2][128] flush: query tokens
@@ -341,17 +341,26 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
       };
       auto kv_slot = [&](int64_t n) { return sbase + Lay::kKv + (uint32_t)(n & 1) * Lay::kKvSlot; };
       auto q_slot = [&](int64_t n) { return sbase + Lay::kQ + (uint32_t)(n & 1) * Lay::kQSlot; };
+      // descriptors of slot 0's tiles, K-major (a K step adds 32 bytes) and
+      // MN-major (LBO = one tile; a 16-row K step adds 2048 bytes); slot 1 is
+      // one slot size further on
+      const uint64_t kd0 = sw128_desc(kv_slot(0), 16, 1024), qd0 = sw128_desc(q_slot(0), 16, 1024);
+      const uint64_t kn0 = sw128_desc(kv_slot(0), Lay::kSub, 1024);
+      const uint64_t qn0 = sw128_desc(q_slot(0), Lay::kSub, 1024);
+      const uint64_t pt_d = sw128_desc(sbase + Lay::kPT, 16, 1024);
+      const uint64_t ds_d = sw128_desc(sbase + Lay::kDST, 16, 1024);
+      const uint64_t ds_n = sw128_desc(sbase + Lay::kDST, Lay::kSub, 1024);
       auto issue_s = [&](const Pair& p) {   // S^T = K Q^T, dP^T = V dO^T
         const uint32_t idesc = idesc_bf16(128, p.nq, false, false);
-        const uint32_t ks = kv_slot(p.kvs), qs = q_slot(p.qs);
+        const uint64_t kd = desc_add(kd0, (uint32_t)(p.kvs & 1) * Lay::kKvSlot);
+        const uint64_t qd = desc_add(qd0, (uint32_t)(p.qs & 1) * Lay::kQSlot);
 #pragma unroll
         for (int s = 0; s < D / 16; ++s)
-          mma_bf16_ss(tmem + kTS, sw128_desc(ks + s * 32, 16, 1024),
-                      sw128_desc(qs + s * 32, 16, 1024), idesc, s > 0);
+          mma_bf16_ss(tmem + kTS, desc_add(kd, s * 32), desc_add(qd, s * 32), idesc, s > 0);
 #pragma unroll
         for (int s = 0; s < D / 16; ++s)
-          mma_bf16_ss(tmem + kTdP, sw128_desc(ks + Lay::kSub + s * 32, 16, 1024),
-                      sw128_desc(qs + Lay::kSub + s * 32, 16, 1024), idesc, s > 0);
+          mma_bf16_ss(tmem + kTdP, desc_add(kd, Lay::kSub + s * 32),
+                      desc_add(qd, Lay::kSub + s * 32), idesc, s > 0);
         mma_commit(&bars->s_full);
       };
       PairIter it;
@@ -375,7 +384,8 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
           if (!ok) break;
           issue_s(nxt);
         }
-        const uint32_t ks = kv_slot(cur.kvs), qs = q_slot(cur.qs);
+        const uint64_t kn = desc_add(kn0, (uint32_t)(cur.kvs & 1) * Lay::kKvSlot);
+        const uint64_t qn = desc_add(qn0, (uint32_t)(cur.qs & 1) * Lay::kQSlot);
         if (cur.kv && cur.first_of_tile && cur.tile >= 1) {
           // the epilogue has read the previous tile's dV / dK
           ok = mbar_wait(&bars->kvacc_free[(cur.tile - 1) & 1],
@@ -394,10 +404,9 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
           for (int s = 0; s < cur.nq / 16; ++s) {
             const uint32_t aoff = (s >> 2) * Lay::kSub + (s & 3) * 32;
             const uint32_t acc = (!cur.first_of_tile || s > 0) ? 1u : 0u;
-            mma_bf16_ss(tmem + kTdV, sw128_desc(sbase + Lay::kPT + aoff, 16, 1024),
-                        sw128_desc(qs + Lay::kSub + s * 2048, Lay::kSub, 1024), id_kv, acc);
-            mma_bf16_ss(tmem + kTdK, sw128_desc(sbase + Lay::kDST + aoff, 16, 1024),
-                        sw128_desc(qs + s * 2048, Lay::kSub, 1024), id_kv, acc);
+            mma_bf16_ss(tmem + kTdV, desc_add(pt_d, aoff), desc_add(qn, Lay::kSub + s * 2048),
+                        id_kv, acc);
+            mma_bf16_ss(tmem + kTdK, desc_add(ds_d, aoff), desc_add(qn, s * 2048), id_kv, acc);
           }
         }
         if (cur.dq) {
@@ -405,8 +414,7 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
           const uint32_t dqc = kTdQ + (uint32_t)(cur.qs & 1) * D;
 #pragma unroll
           for (int s = 0; s < kTile / 16; ++s)
-            mma_bf16_ss(tmem + dqc, sw128_desc(sbase + Lay::kDST + s * 2048, Lay::kSub, 1024),
-                        sw128_desc(ks + s * 2048, Lay::kSub, 1024), id_q,
+            mma_bf16_ss(tmem + dqc, desc_add(ds_n, s * 2048), desc_add(kn, s * 2048), id_q,
                         (cur.dq_acc || s > 0) ? 1u : 0u);
         }
         mma_commit(&bars->pd_free);
@@ -448,9 +456,12 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
       if (!ok) break;
       fence_after();
       float* ls = s_lse + qslot * 128;
-      const float* dps = s_dpr + qslot * 128;
-      if (p.q_first) {   // the block's lse to log2 units, once per block
-        if (ew < 128) ls[ew] *= 1.4426950408889634f;
+      float* dps = s_dpr + qslot * 128;
+      if (p.q_first) {   // once per block: -lse in log2 units and -D'
+        if (ew < 128) {
+          ls[ew] *= -1.4426950408889634f;
+          dps[ew] = -dps[ew];
+        }
         ew_sync();
       }
       // stage the epilogue's inputs (key tokens of a new tile; query tokens
@@ -493,19 +504,31 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
         tmem_ld32(tmem + kTdP + lane_off + c0, dp);
         tmem_ld_wait();
         uint32_t pw[16], dw[16];
+        const bool edge = masked || p.nq < kTile;
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float2 l2 = *reinterpret_cast<const float2*>(ls + c0 + i);
-          const float2 d2 = *reinterpret_cast<const float2*>(dps + c0 + i);
-          float p0 = ex2(fmaf(sv[i], scale_log2, -l2.x));
-          float p1 = ex2(fmaf(sv[i + 1], scale_log2, -l2.y));
-          if (masked || p.nq < kTile) {
+        for (int i = 0; i < 32; i += 4) {
+          const float4 nl = *reinterpret_cast<const float4*>(ls + c0 + i);    // -lse log2 e
+          const float4 nd = *reinterpret_cast<const float4*>(dps + c0 + i);   // -D'
+          float a0 = sv[i], a1 = sv[i + 1], a2 = sv[i + 2], a3 = sv[i + 3];
+          fma2(a0, a1, scale_log2, scale_log2, nl.x, nl.y);
+          fma2(a2, a3, scale_log2, scale_log2, nl.z, nl.w);
+          float p0 = ex2(a0), p1 = ex2(a1), p2 = ex2(a2), p3 = ex2(a3);
+          if (edge) {
             const int col = c0 + i;
             p0 = (col >= lo && col < cend) ? p0 : 0.f;
             p1 = (col + 1 >= lo && col + 1 < cend) ? p1 : 0.f;
+            p2 = (col + 2 >= lo && col + 2 < cend) ? p2 : 0.f;
+            p3 = (col + 3 >= lo && col + 3 < cend) ? p3 : 0.f;
           }
+          float g0 = dp[i], g1 = dp[i + 1], g2 = dp[i + 2], g3 = dp[i + 3];
+          add2(g0, g1, nd.x, nd.y);
+          add2(g2, g3, nd.z, nd.w);
+          mul2(g0, g1, p0, p1);
+          mul2(g2, g3, p2, p3);
           pw[i >> 1] = pack2(p0, p1);
-          dw[i >> 1] = pack2(p0 * (dp[i] - d2.x), p1 * (dp[i + 1] - d2.y));
+          pw[(i >> 1) + 1] = pack2(p2, p3);
+          dw[i >> 1] = pack2(g0, g1);
+          dw[(i >> 1) + 1] = pack2(g2, g3);
         }
         if (cb == 0 && pi >= 1) {   // the MMAs of the previous pair are done with P^T / dS^T
           ok = ew_all(mbar_wait(&bars->pd_free, (uint32_t)((pi - 1) & 1), err));

@@ -256,6 +256,16 @@ attn_fwd_pipe_kernel(const __grid_constant__ FwdMaps maps, const int32_t* __rest
       auto kv_slot = [&](int64_t n) -> uint32_t {
         return sbase + Lay::kKv + (uint32_t)(n % kKvSlots) * Lay::kKvSlot;
       };
+      // descriptors of every slot's tile, built once: K-major (K step +32
+      // bytes) for Q and K, MN-major (16-row K step +2048 bytes) for V, and
+      // the K-major P tile
+      const uint64_t q_d0 = sw128_desc(sbase + Lay::kQ, 16, 1024);
+      const uint64_t k_d0 = sw128_desc(kv_slot(0), 16, 1024);
+      const uint64_t v_n0 = sw128_desc(kv_slot(0) + Lay::kTileBytes, Lay::kTileBytes, 1024);
+      const uint64_t p_d = sw128_desc(sbase + Lay::kP, 16, 1024);
+      auto qk = [&](int64_t j) { return desc_add(q_d0, (uint32_t)(j % kQSlots) * Lay::kTileBytes); };
+      auto kk_d = [&](int64_t n) { return desc_add(k_d0, (uint32_t)(n % kKvSlots) * Lay::kKvSlot); };
+      auto vn = [&](int64_t n) { return desc_add(v_n0, (uint32_t)(n % kKvSlots) * Lay::kKvSlot); };
       auto issue_pv = [&](int64_t j) -> bool {
         // O[j % 2] = P V over the live key columns; needs a free O buffer
         const int o = (int)(j & 1);
@@ -266,13 +276,12 @@ attn_fwd_pipe_kernel(const __grid_constant__ FwdMaps maps, const int32_t* __rest
         const Cols cc = tile_cols(ti, chunk);
         for (int x = cc.col_lo; x < cc.ncols; x += 16) {
           const bool in_prev = ti.has_prev && x < kTile;
-          const uint32_t vst = kv_slot(in_prev ? ti.prev : ti.own) + Lay::kTileBytes;
+          const uint64_t vd = vn(in_prev ? ti.prev : ti.own);
           const int row = in_prev ? x : (ti.has_prev ? x - kTile : x);
           const int s = x >> 4;
           const uint32_t poff = (s >> 2) * Lay::kTileBytes + (s & 3) * 32;
-          mma_bf16_ss(tmem + kTO + o * D, sw128_desc(sbase + Lay::kP + poff, 16, 1024),
-                      sw128_desc(vst + (row >> 4) * 2048, Lay::kTileBytes, 1024), id_pv,
-                      x > cc.col_lo ? 1u : 0u);
+          mma_bf16_ss(tmem + kTO + o * D, desc_add(p_d, poff), desc_add(vd, (row >> 4) * 2048),
+                      id_pv, x > cc.col_lo ? 1u : 0u);
         }
         mma_commit(&bars->o_full[o]);
         if (ti.has_prev) mma_commit(&bars->empty_kv[ti.prev % kKvSlots]);
@@ -294,18 +303,20 @@ attn_fwd_pipe_kernel(const __grid_constant__ FwdMaps maps, const int32_t* __rest
                          (uint32_t)((kv_ready / kKvSlots) & 1), err);
         if (!ok) break;
         fence_after();
-        const uint32_t qst = sbase + Lay::kQ + (uint32_t)(j % kQSlots) * Lay::kTileBytes;
+        const uint64_t qd = qk(j);
         if (ti.has_prev) {
+          const uint64_t kd = kk_d(ti.prev);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_bf16_ss(tmem + kTS, sw128_desc(qst + kk * 32, 16, 1024),
-                        sw128_desc(kv_slot(ti.prev) + kk * 32, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+            mma_bf16_ss(tmem + kTS, desc_add(qd, kk * 32), desc_add(kd, kk * 32), id_s,
+                        kk > 0 ? 1u : 0u);
         }
         const uint32_t own_col = ti.has_prev ? (uint32_t)kTile : 0u;
+        const uint64_t kd = kk_d(ti.own);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(tmem + kTS + own_col, sw128_desc(qst + kk * 32, 16, 1024),
-                      sw128_desc(kv_slot(ti.own) + kk * 32, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+          mma_bf16_ss(tmem + kTS + own_col, desc_add(qd, kk * 32), desc_add(kd, kk * 32), id_s,
+                      kk > 0 ? 1u : 0u);
         mma_commit(&bars->s_full);
         mma_commit(&bars->empty_q[j % kQSlots]);
       }
@@ -359,18 +370,21 @@ attn_fwd_pipe_kernel(const __grid_constant__ FwdMaps maps, const int32_t* __rest
         tmem_ld32(tmem + kTS + lane_off + c0, sv);
         tmem_ld_wait();
         uint32_t packed[16];
+        float l0 = 0.f, l1 = 0.f;
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          float p0 = ex2(fmaf(sv[e], scale_log2, -m));
-          float p1 = ex2(fmaf(sv[e + 1], scale_log2, -m));
+          float a0 = sv[e], a1 = sv[e + 1];
+          fma2(a0, a1, scale_log2, scale_log2, -m, -m);
+          float p0 = ex2(a0), p1 = ex2(a1);
           if (masked) {
             p0 = (c0 + e >= lo && c0 + e < hi) ? p0 : 0.f;
             p1 = (c0 + e + 1 >= lo && c0 + e + 1 < hi) ? p1 : 0.f;
           }
-          l += p0 + p1;
+          add2(l0, l1, p0, p1);
           const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
           packed[e >> 1] = *reinterpret_cast<const uint32_t*>(&h);
         }
+        l += l0 + l1;
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
           const int key = c0 + q8 * 8;
