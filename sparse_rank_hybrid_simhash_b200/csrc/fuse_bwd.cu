@@ -213,20 +213,25 @@ fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __re
   }
 }
 
+// One warp per parameter: lane l sums partial blocks l, l + 32, ... in fp64,
+// then the lanes combine in a fixed butterfly order (deterministic).
 __global__ void param_reduce_kernel(const float* __restrict__ partials, int blocks, int d,
                                     float* __restrict__ dgate_w, float* __restrict__ dgate_b,
                                     float* __restrict__ dlambda) {
   const int P = 2 * d + 3;
-  for (int e = threadIdx.x; e < P; e += blockDim.x) {
-    double s = 0.0;
-    for (int b = 0; b < blocks; ++b) s += (double)partials[(size_t)b * P + e];
-    if (e < 2 * d) {
-      if (dgate_w) dgate_w[e] = (float)s;
-    } else if (e < 2 * d + 2) {
-      if (dgate_b) dgate_b[e - 2 * d] = (float)s;
-    } else {
-      *dlambda = (float)s;
-    }
+  const int e = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
+  if (e >= P) return;
+  double s = 0.0;
+  for (int b = lane; b < blocks; b += 32) s += (double)partials[(size_t)b * P + e];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane != 0) return;
+  if (e < 2 * d) {
+    if (dgate_w) dgate_w[e] = (float)s;
+  } else if (e < 2 * d + 2) {
+    if (dgate_b) dgate_b[e - 2 * d] = (float)s;
+  } else {
+    *dlambda = (float)s;
   }
 }
 
@@ -277,7 +282,9 @@ cudaError_t launch_fuse_bwd(const Geometry& g, const void* q, const void* dy, co
 
 cudaError_t launch_param_reduce(const Geometry& g, const float* partials, float* dgate_w,
                                 float* dgate_b, float* dlambda, cudaStream_t s) {
-  param_reduce_kernel<<<1, 256, 0, s>>>(partials, kParamBlocks, g.d, dgate_w, dgate_b, dlambda);
+  const int P = 2 * g.d + 3;
+  param_reduce_kernel<<<(P * 32 + 255) / 256, 256, 0, s>>>(partials, kParamBlocks, g.d, dgate_w,
+                                                           dgate_b, dlambda);
   return cudaGetLastError();
 }
 
