@@ -79,7 +79,13 @@ fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __re
                 float2* __restrict__ da_out, T* __restrict__ dor, float* __restrict__ absmax,
                 float* __restrict__ partials) {
   constexpr int QW = 32 / QL;
+  constexpr int CB = 4 * (int)sizeof(T);   // bytes of one lane's 4 values
   __shared__ float red[8][2 * 128 + 3];
+  // per warp, two rows in flight: each lane copies its own chunks of q, dy,
+  // O_sp, O_race (and its row's lse, Ctot) for the next row by cp.async and
+  // reads them back when that row comes up
+  __shared__ __align__(16) uint8_t s_stage[8][2][4][32 * CB];
+  __shared__ __align__(16) uint32_t s_scal[8][2][2][32];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   const int ql = lane % QL, sub = lane / QL;
   const float lam_v = *lam;
@@ -97,16 +103,41 @@ fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __re
   float cur_max = 0.f;
   const int64_t first = ((int64_t)blockIdx.x * nw + w) * QW;
   const int64_t stride = (int64_t)gridDim.x * nw * QW;
-  for (int64_t r0 = first; r0 < rows; r0 += stride) {
+  auto stage = [&](int64_t r0, int buf) {
+    const int64_t rr = min(r0 + sub, rows - 1);
+    const size_t base = (size_t)rr * d + ql * 4;
+    const T* src[4] = {q + base, dy + base, o_sp + base, o_race + base};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(&s_stage[w][buf][t][lane * CB]));
+      if (CB == 8)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src[t]) : "memory");
+      else
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src[t]) : "memory");
+    }
+    const uint32_t d0 = static_cast<uint32_t>(__cvta_generic_to_shared(&s_scal[w][buf][0][lane]));
+    const uint32_t d1 = static_cast<uint32_t>(__cvta_generic_to_shared(&s_scal[w][buf][1][lane]));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d0), "l"(lse + rr) : "memory");
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d1), "l"(ctot + rr) : "memory");
+  };
+  if (first < rows) stage(first, 0);
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  int buf = 0;
+  for (int64_t r0 = first; r0 < rows; r0 += stride, buf ^= 1) {
     const int64_t r = r0 + sub;
     const bool valid = r < rows;
     const int64_t rr = valid ? r : rows - 1;
     const size_t base = (size_t)rr * d + ql * 4;
+    if (r0 + stride < rows) stage(r0 + stride, buf ^ 1);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 1;" ::: "memory");   // this row's chunks are in
     float qv[4], g[4], os[4], orc[4];
-    ld4<T>(q + base, qv);
-    ld4<T>(dy + base, g);
-    ld4<T>(o_sp + base, os);
-    ld4<T>(o_race + base, orc);
+    ld4<T>(reinterpret_cast<const T*>(&s_stage[w][buf][0][lane * CB]), qv);
+    ld4<T>(reinterpret_cast<const T*>(&s_stage[w][buf][1][lane * CB]), g);
+    ld4<T>(reinterpret_cast<const T*>(&s_stage[w][buf][2][lane * CB]), os);
+    ld4<T>(reinterpret_cast<const T*>(&s_stage[w][buf][3][lane * CB]), orc);
+    const float l = __uint_as_float(s_scal[w][buf][0][lane]);
+    const int c = (int)s_scal[w][buf][1][lane];
     float dyo = 0.f, dyr = 0.f, as = 0.f, ar = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -122,9 +153,7 @@ fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __re
       gs = 1.0f / (1.0f + expf(-(gsum<QL>(as) + bs)));
       gr = 1.0f / (1.0f + expf(-(gsum<QL>(ar) + br)));
     }
-    const int c = ctot[rr];
     const float zr = (float)c / (float)L;
-    const float l = lse[rr];
     const float lz = lam_v * zr;
     const float m = lz > 0.f ? 1.0f / (1.0f + expf(logf(lz) - l)) : 1.0f;
     const float dm = gs * dyo;
@@ -177,6 +206,7 @@ fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __re
       cur_max = fmaxf(cur_max, vmax);
     }
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
   if (ql == 0 && cur_bh >= 0)
     atomicMax(reinterpret_cast<int*>(absmax) + cur_bh, __float_as_int(cur_max));
   // block reduction of the partial parameter gradients: first across the row
