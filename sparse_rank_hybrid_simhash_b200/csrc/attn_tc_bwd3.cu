@@ -156,6 +156,21 @@ struct PairIter {
   }
 };
 
+// Waits for this thread's TMEM loads, with the 32 destination registers of
+// the two 16-column loads tied to the wait so that no use of them is
+// scheduled above it.
+ELSAA_DEV void tmem_wait_hold(float* a, float* b) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+f"(a[0]), "+f"(a[1]), "+f"(a[2]), "+f"(a[3]), "+f"(a[4]), "+f"(a[5]),
+                 "+f"(a[6]), "+f"(a[7]), "+f"(a[8]), "+f"(a[9]), "+f"(a[10]), "+f"(a[11]),
+                 "+f"(a[12]), "+f"(a[13]), "+f"(a[14]), "+f"(a[15]), "+f"(b[0]), "+f"(b[1]),
+                 "+f"(b[2]), "+f"(b[3]), "+f"(b[4]), "+f"(b[5]), "+f"(b[6]), "+f"(b[7]),
+                 "+f"(b[8]), "+f"(b[9]), "+f"(b[10]), "+f"(b[11]), "+f"(b[12]), "+f"(b[13]),
+                 "+f"(b[14]), "+f"(b[15])
+               :
+               : "memory");
+}
+
 ELSAA_DEV uint32_t pack2(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -496,17 +511,26 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
       const int key_chunk = (p.kb * kTile + row) >> lc;
       const int lo = (key_chunk << lc) - p.qb * kTile, hi = lo + 2 * chunk;
       const int cend = min(hi, p.nq);
+      // four 16-column chunks of S and dP per thread; the next chunk's TMEM
+      // loads are in flight while this one is computed
+      const int cbase = half * 64;
+      const bool edge = masked || p.nq < kTile;
+      float sv0[16], dp0[16], sv1[16], dp1[16];
+      tmem_ld16(tmem + kTS + lane_off + cbase, sv0);
+      tmem_ld16(tmem + kTdP + lane_off + cbase, dp0);
 #pragma unroll
-      for (int cb = 0; cb < 2; ++cb) {
-        const int c0 = half * 64 + cb * 32;
-        float sv[32], dp[32];
-        tmem_ld32(tmem + kTS + lane_off + c0, sv);
-        tmem_ld32(tmem + kTdP + lane_off + c0, dp);
-        tmem_ld_wait();
-        uint32_t pw[16], dw[16];
-        const bool edge = masked || p.nq < kTile;
+      for (int jc = 0; jc < 4; ++jc) {
+        float* sv = (jc & 1) ? sv1 : sv0;
+        float* dp = (jc & 1) ? dp1 : dp0;
+        tmem_wait_hold(sv, dp);
+        if (jc + 1 < 4) {
+          tmem_ld16(tmem + kTS + lane_off + cbase + (jc + 1) * 16, (jc & 1) ? sv0 : sv1);
+          tmem_ld16(tmem + kTdP + lane_off + cbase + (jc + 1) * 16, (jc & 1) ? dp0 : dp1);
+        }
+        const int c0 = cbase + jc * 16;
+        uint32_t pw[8], dw[8];
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
+        for (int i = 0; i < 16; i += 4) {
           const float4 nl = *reinterpret_cast<const float4*>(ls + c0 + i);    // -lse log2 e
           const float4 nd = *reinterpret_cast<const float4*>(dps + c0 + i);   // -D'
           float a0 = sv[i], a1 = sv[i + 1], a2 = sv[i + 2], a3 = sv[i + 3];
@@ -530,12 +554,15 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
           dw[i >> 1] = pack2(g0, g1);
           dw[(i >> 1) + 1] = pack2(g2, g3);
         }
-        if (cb == 0 && pi >= 1) {   // the MMAs of the previous pair are done with P^T / dS^T
+        if (jc == 0 && pi >= 1) {   // the MMAs of the previous pair are done with P^T / dS^T
           ok = ew_all(mbar_wait(&bars->pd_free, (uint32_t)((pi - 1) & 1), err));
-          if (!ok) break;
+          if (!ok) {
+            tmem_ld_wait();
+            break;
+          }
         }
 #pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
+        for (int q8 = 0; q8 < 2; ++q8) {
           const int col = c0 + q8 * 8;
           const uint32_t off = (col >> 6) * Lay::kSub + sw128_off(row, (col & 63) >> 3);
           if (p.kv)
