@@ -20,15 +20,16 @@
 //               ring) and K/V blocks (four-slot ring) into 128B-swizzled
 //               tiles; completion counted in bytes on full_q / full_kv
 //   warp 1      MMA issuer (one thread) and TMEM owner:
-//                 O(j-1) = P V        as soon as P of tile j-1 is written
+//                 O(j-1) = P V        as soon as P of tile j-1 is written,
+//                                     P read from TMEM as the A operand
 //                 S(j)   = Q K^T      -> TMEM [0, 256)
 //               and releases Q and K/V slots through tcgen05.commit
 //   warps 2..9  softmax and epilogue: warp w reaches TMEM lanes (query rows)
 //               32 (w % 4) .. +31 and takes one of two column ranges; row max
 //               and row sum are combined through shared memory;
 //               p = exp2(scale log2e s - m) masked to the row's own window,
-//               P (bf16) to shared memory, then O / l and the log-mass to the
-//               query's token index
+//               P (bf16 pairs) to TMEM [384, 512), then O / l and the
+//               log-mass to the query's token index
 // Every wait is bounded; a timeout records ERR_TIMEOUT and every role leaves
 // its loop, frees TMEM and returns.
 #include <math.h>
@@ -49,14 +50,14 @@ constexpr int kKvSlots = 4;
 constexpr int kQSlots = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTS = 0, kTO = 256;   // S: 256 columns, O: 2 x 64 columns
+constexpr uint32_t kTP = 384;            // P: 128 columns, two bf16 per column
 
 struct PipeLayout {
   static constexpr uint32_t kTileBytes = 128 * 128;              // 128 rows x 64 bf16
   static constexpr uint32_t kKv = 0;                             // [4][K | V]
   static constexpr uint32_t kKvSlot = 2 * kTileBytes;
   static constexpr uint32_t kQ = kKv + kKvSlots * kKvSlot;       // [2][Q]
-  static constexpr uint32_t kP = kQ + kQSlots * kTileBytes;      // 128 x 256 bf16, 4 sub-tiles
-  static constexpr uint32_t kRed = kP + 4 * kTileBytes;          // row max and sum [2][2][128]
+  static constexpr uint32_t kRed = kQ + kQSlots * kTileBytes;    // row max and sum [2][2][128]
   static constexpr uint32_t kBar = kRed + 2 * 2 * 128 * 4;
   static constexpr uint32_t kDyn = kBar + 256;
 };
@@ -262,7 +263,6 @@ attn_fwd_pipe_kernel(const __grid_constant__ FwdMaps maps, const int32_t* __rest
       const uint64_t q_d0 = sw128_desc(sbase + Lay::kQ, 16, 1024);
       const uint64_t k_d0 = sw128_desc(kv_slot(0), 16, 1024);
       const uint64_t v_n0 = sw128_desc(kv_slot(0) + Lay::kTileBytes, Lay::kTileBytes, 1024);
-      const uint64_t p_d = sw128_desc(sbase + Lay::kP, 16, 1024);
       auto qk = [&](int64_t j) { return desc_add(q_d0, (uint32_t)(j % kQSlots) * Lay::kTileBytes); };
       auto kk_d = [&](int64_t n) { return desc_add(k_d0, (uint32_t)(n % kKvSlots) * Lay::kKvSlot); };
       auto vn = [&](int64_t n) { return desc_add(v_n0, (uint32_t)(n % kKvSlots) * Lay::kKvSlot); };
@@ -278,10 +278,8 @@ attn_fwd_pipe_kernel(const __grid_constant__ FwdMaps maps, const int32_t* __rest
           const bool in_prev = ti.has_prev && x < kTile;
           const uint64_t vd = vn(in_prev ? ti.prev : ti.own);
           const int row = in_prev ? x : (ti.has_prev ? x - kTile : x);
-          const int s = x >> 4;
-          const uint32_t poff = (s >> 2) * Lay::kTileBytes + (s & 3) * 32;
-          mma_bf16_ss(tmem + kTO + o * D, desc_add(p_d, poff), desc_add(vd, (row >> 4) * 2048),
-                      id_pv, x > cc.col_lo ? 1u : 0u);
+          mma_bf16_ts(tmem + kTO + o * D, tmem + kTP + (uint32_t)(x >> 1),
+                      desc_add(vd, (row >> 4) * 2048), id_pv, x > cc.col_lo ? 1u : 0u);
         }
         mma_commit(&bars->o_full[o]);
         if (ti.has_prev) mma_commit(&bars->empty_kv[ti.prev % kKvSlots]);
@@ -385,16 +383,11 @@ attn_fwd_pipe_kernel(const __grid_constant__ FwdMaps maps, const int32_t* __rest
           packed[e >> 1] = *reinterpret_cast<const uint32_t*>(&h);
         }
         l += l0 + l1;
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-          const int key = c0 + q8 * 8;
-          uint8_t* dst = smem + Lay::kP + (key >> 6) * Lay::kTileBytes + sw128_off(row, (key & 63) >> 3);
-          *reinterpret_cast<uint4*>(dst) =
-              make_uint4(packed[q8 * 4], packed[q8 * 4 + 1], packed[q8 * 4 + 2], packed[q8 * 4 + 3]);
-        }
+        // the row's P values of keys c0 .. c0 + 31 into TMEM columns c0 / 2 ..
+        tmem_st16(tmem + kTP + lane_off + (uint32_t)(c0 >> 1), packed);
       }
+      tmem_st_wait();
       red_l[half * 128 + row] = l;
-      fence_async_smem();
       fence_before();
       mbar_arrive(&bars->p_full);
       softmax_sync();
