@@ -965,6 +965,7 @@ race_fuse_rows_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q
   const uint32_t table_bytes = (uint32_t)NB * (uint32_t)d * (uint32_t)sizeof(T);
   const int row_shift = 31 - __clz(d * (int)sizeof(T));   // d * sizeof is a power of two
   const float lam_v = *lam;
+  const float inv_L = 1.0f / (float)L;
   for (int i = threadIdx.x; i < 2 * d; i += blockDim.x) s_w[i] = gate_fixed ? 0.f : gate_w[i];
   const float bs = gate_fixed ? 0.f : gate_b[0], br = gate_fixed ? 0.f : gate_b[1];
   __syncthreads();
@@ -1011,7 +1012,7 @@ race_fuse_rows_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q
     gather_row<T, CodeT, QL, WPL>(tables + (size_t)bh * L * NB * d + ql * EL, w, L, table_bytes,
                                   row_shift, gbase, pol, acc);
     ctot = group_sum_i<QL>(ctot);
-    const float inv = ctot > 0 ? 1.0f / (float)ctot : 0.f;
+    const float inv = ctot > 0 ? __fdividef(1.0f, (float)ctot) : 0.f;
     asm volatile("cp.async.wait_group 1;" ::: "memory");   // this row's chunks are in
     float qv[EL], os[EL], orc[EL];
     unpack16(s_stage[wi][buf][0][lane], qv, q);
@@ -1028,12 +1029,12 @@ race_fuse_rows_kernel(const T* __restrict__ q, const CodeT* __restrict__ rcode_q
       }
       as = group_sum<QL>(as) + bs;
       ar = group_sum<QL>(ar) + br;
-      gs = 1.0f / (1.0f + expf(-as));
-      gr = 1.0f / (1.0f + expf(-ar));
+      gs = __fdividef(1.0f, 1.0f + __expf(-as));
+      gr = __fdividef(1.0f, 1.0f + __expf(-ar));
     }
     // m = Z_sp / (Z_sp + lambda Z_race) = 1 / (1 + exp(log(lambda Z_race) - lse))
-    const float lz = lam_v * (float)ctot / (float)L;
-    const float m = lz > 0.f ? 1.0f / (1.0f + expf(logf(lz) - lse_r)) : 1.0f;
+    const float lz = lam_v * (float)ctot * inv_L;
+    const float m = lz > 0.f ? __fdividef(1.0f, 1.0f + __expf(__logf(lz) - lse_r)) : 1.0f;
     if (valid) {
       float yv[EL];
 #pragma unroll
