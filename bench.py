@@ -109,14 +109,14 @@ def stage_roofline(flops, nbytes, sec, peaks):
 # workload by the number of units; reported only while that file is unchanged.
 RECORDED_TRAFFIC = {
     # stage: (kernel source, its sha1 at capture, bytes per full-size launch)
-    "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "9628a6a95e0435f02fdb79d609702aed00e31da4", 2.444e+08),
-    "race_build": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "d71bdb58cc88f62b77ee364f69f39b401eda6744", 1.368e+08),
-    "sparse_fwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_pipe.cu", "3a62fd41f041ed04cb99948b9f4c1fb587d46f41", 3.727e+08),
-    "race_fuse": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "d71bdb58cc88f62b77ee364f69f39b401eda6744", 3.564e+08),
-    "fuse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/fuse_bwd.cu", "b39e9fcf002feed95044d88de883f3eca4907efd", 5.719e+08),
-    "race_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "d71bdb58cc88f62b77ee364f69f39b401eda6744", 1.324e+08),
-    "sparse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_bwd3.cu", "41207b576a5dab9665cc1ed634181525c66ec267", 6.626e+08),
-    "finish": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "d71bdb58cc88f62b77ee364f69f39b401eda6744", 1.58e+08),
+    "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "803a7fe621006eabe5ce0f2c498653ba03e4da75", 2.432e+08),
+    "race_build": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "c074d833a8677a22349643ee291b65fc403659e5", 1.369e+08),
+    "sparse_fwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_pipe.cu", "91a31d0c88874e37ef33ed4bb443baabc0c07369", 3.728e+08),
+    "race_fuse": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "c074d833a8677a22349643ee291b65fc403659e5", 3.733e+08),
+    "fuse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/fuse_bwd.cu", "b2b1538c8f47145cb34db05fe72d360dcc260381", 5.688e+08),
+    "race_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "c074d833a8677a22349643ee291b65fc403659e5", 1.317e+08),
+    "sparse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_bwd3.cu", "5530f1537a8b0a387b2bc31b36e8aaece4caa2c4", 6.643e+08),
+    "finish": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "c074d833a8677a22349643ee291b65fc403659e5", 1.583e+08),
 }
 
 
@@ -377,12 +377,17 @@ def oracle_unit_seconds(w, inp, units):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w, units=8):
+def cpu_baseline(w, min_seconds=10.0):
+    """The oracle on the host cores over (batch, head) units of the workload,
+    one after another until at least min_seconds of CPU work (or every unit)."""
     cores = len(os.sched_getaffinity(0))
     torch.set_num_threads(cores)
     inp = make_inputs(w, with_dy=True)
-    sel = [(i // w.H % w.B, i % w.H) for i in range(units)]
-    secs = oracle_unit_seconds(w, inp, sel)
+    all_units = [(i // w.H % w.B, i % w.H) for i in range(w.B * w.H)]
+    secs, units = 0.0, 0
+    while units < len(all_units) and secs < min_seconds:
+        secs += oracle_unit_seconds(w, inp, all_units[units:units + 1])
+        units += 1
     # one (batch, head) unit is N / H token-equivalents of the B x N-token step
     value = units * w.N / w.H / secs
     return {"value": value, "unit": "tokens/s", "cores": torch.get_num_threads(),
