@@ -87,7 +87,7 @@ struct RowMaps {
 
 struct Bars3 {
   uint64_t full_kv[2], empty_kv[2], full_q[2], empty_q[2];
-  uint64_t s_full, p_full, pd_free, kvacc_full, dq_full[2];
+  uint64_t s_full, s_free, p_full, pd_free, kvacc_full, dq_full[2];
   uint64_t dq_free[2], kvacc_free[2], fl_ready[2], key_ready[2];
   uint32_t tmem;
 };
@@ -258,6 +258,7 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
       mbar_init(&bars->key_ready[s], 128);
     }
     mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_free, kEwThreads);
     mbar_init(&bars->p_full, kEwThreads);
     mbar_init(&bars->pd_free, 1);
     mbar_init(&bars->kvacc_full, 1);
@@ -386,7 +387,10 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
       ok = wait_data(cur);
       if (ok) issue_s(cur);
       for (int64_t pi = 0; ok; ++pi) {
-        ok = mbar_wait(&bars->p_full, (uint32_t)(pi & 1), err);
+        // the next pair's S and dP go out as soon as every elementwise thread
+        // has read this pair's S and dP from TMEM; its gradients once P^T and
+        // dS^T are in shared memory
+        ok = mbar_wait(&bars->s_free, (uint32_t)(pi & 1), err);
         if (!ok) break;
         fence_after();
         PairIter nx = it;
@@ -399,6 +403,9 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
           if (!ok) break;
           issue_s(nxt);
         }
+        ok = mbar_wait(&bars->p_full, (uint32_t)(pi & 1), err);
+        if (!ok) break;
+        fence_after();
         const uint64_t kn = desc_add(kn0, (uint32_t)(cur.kvs & 1) * Lay::kKvSlot);
         const uint64_t qn = desc_add(qn0, (uint32_t)(cur.qs & 1) * Lay::kQSlot);
         if (cur.kv && cur.first_of_tile && cur.tile >= 1) {
@@ -523,6 +530,10 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
         float* sv = (jc & 1) ? sv1 : sv0;
         float* dp = (jc & 1) ? dp1 : dp0;
         tmem_wait_hold(sv, dp);
+        if (jc == 3) {   // this pair's S and dP are read: TMEM may take the next pair's
+          fence_before();
+          mbar_arrive(&bars->s_free);
+        }
         if (jc + 1 < 4) {
           tmem_ld16(tmem + kTS + lane_off + cbase + (jc + 1) * 16, (jc & 1) ? sv0 : sv1);
           tmem_ld16(tmem + kTdP + lane_off + cbase + (jc + 1) * 16, (jc & 1) ? dp0 : dp1);
