@@ -87,7 +87,7 @@ struct RowMaps {
 
 struct Bars3 {
   uint64_t full_kv[2], empty_kv[2], full_q[2], empty_q[2];
-  uint64_t s_full, s_free, p_full, pd_free, kvacc_full, dq_full[2];
+  uint64_t s_full, s_free, p_full, pt_free, pd_free, kvacc_full, dq_full[2];
   uint64_t dq_free[2], kvacc_free[2], fl_ready[2], key_ready[2];
   uint32_t tmem;
 };
@@ -260,6 +260,7 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->s_free, kEwThreads);
     mbar_init(&bars->p_full, kEwThreads);
+    mbar_init(&bars->pt_free, 1);
     mbar_init(&bars->pd_free, 1);
     mbar_init(&bars->kvacc_full, 1);
     fence_mbar_init();
@@ -421,13 +422,21 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
           if (!ok) break;
         }
         fence_after();
+        // dV first: its completion frees P^T for the next pair's stores
+        const uint32_t id_kv = idesc_bf16(128, D, false, true);
         if (cur.kv) {
-          const uint32_t id_kv = idesc_bf16(128, D, false, true);
           for (int s = 0; s < cur.nq / 16; ++s) {
             const uint32_t aoff = (s >> 2) * Lay::kSub + (s & 3) * 32;
             const uint32_t acc = (!cur.first_of_tile || s > 0) ? 1u : 0u;
             mma_bf16_ss(tmem + kTdV, desc_add(pt_d, aoff), desc_add(qn, Lay::kSub + s * 2048),
                         id_kv, acc);
+          }
+        }
+        mma_commit(&bars->pt_free);
+        if (cur.kv) {
+          for (int s = 0; s < cur.nq / 16; ++s) {
+            const uint32_t aoff = (s >> 2) * Lay::kSub + (s & 3) * 32;
+            const uint32_t acc = (!cur.first_of_tile || s > 0) ? 1u : 0u;
             mma_bf16_ss(tmem + kTdK, desc_add(ds_d, aoff), desc_add(qn, s * 2048), id_kv, acc);
           }
         }
@@ -519,10 +528,13 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
       const int lo = (key_chunk << lc) - p.qb * kTile, hi = lo + 2 * chunk;
       const int cend = min(hi, p.nq);
       // four 16-column chunks of S and dP per thread; the next chunk's TMEM
-      // loads are in flight while this one is computed
+      // loads are in flight while this one is computed. P^T goes out chunk by
+      // chunk once the previous pair's dV has read it; dS^T is held and goes
+      // out once the previous pair's dK and dQ have read theirs.
       const int cbase = half * 64;
       const bool edge = masked || p.nq < kTile;
       float sv0[16], dp0[16], sv1[16], dp1[16];
+      uint32_t dw[4][8];
       tmem_ld16(tmem + kTS + lane_off + cbase, sv0);
       tmem_ld16(tmem + kTdP + lane_off + cbase, dp0);
 #pragma unroll
@@ -539,7 +551,7 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
           tmem_ld16(tmem + kTdP + lane_off + cbase + (jc + 1) * 16, (jc & 1) ? dp0 : dp1);
         }
         const int c0 = cbase + jc * 16;
-        uint32_t pw[8], dw[8];
+        uint32_t pw[8];
 #pragma unroll
         for (int i = 0; i < 16; i += 4) {
           const float4 nl = *reinterpret_cast<const float4*>(ls + c0 + i);    // -lse log2 e
@@ -562,25 +574,39 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
           mul2(g2, g3, p2, p3);
           pw[i >> 1] = pack2(p0, p1);
           pw[(i >> 1) + 1] = pack2(p2, p3);
-          dw[i >> 1] = pack2(g0, g1);
-          dw[(i >> 1) + 1] = pack2(g2, g3);
+          dw[jc][i >> 1] = pack2(g0, g1);
+          dw[jc][(i >> 1) + 1] = pack2(g2, g3);
         }
-        if (jc == 0 && pi >= 1) {   // the MMAs of the previous pair are done with P^T / dS^T
-          ok = ew_all(mbar_wait(&bars->pd_free, (uint32_t)((pi - 1) & 1), err));
+        if (jc == 0 && pi >= 1) {   // the previous pair's dV is done with P^T
+          ok = ew_all(mbar_wait(&bars->pt_free, (uint32_t)((pi - 1) & 1), err));
           if (!ok) {
             tmem_ld_wait();
             break;
           }
         }
+        if (p.kv) {
 #pragma unroll
-        for (int q8 = 0; q8 < 2; ++q8) {
-          const int col = c0 + q8 * 8;
-          const uint32_t off = (col >> 6) * Lay::kSub + sw128_off(row, (col & 63) >> 3);
-          if (p.kv)
+          for (int q8 = 0; q8 < 2; ++q8) {
+            const int col = c0 + q8 * 8;
+            const uint32_t off = (col >> 6) * Lay::kSub + sw128_off(row, (col & 63) >> 3);
             *reinterpret_cast<uint4*>(smem + Lay::kPT + off) =
                 make_uint4(pw[q8 * 4], pw[q8 * 4 + 1], pw[q8 * 4 + 2], pw[q8 * 4 + 3]);
+          }
+        }
+      }
+      if (!ok) break;
+      if (pi >= 1) {   // the previous pair's dK and dQ are done with dS^T
+        ok = ew_all(mbar_wait(&bars->pd_free, (uint32_t)((pi - 1) & 1), err));
+        if (!ok) break;
+      }
+#pragma unroll
+      for (int jc = 0; jc < 4; ++jc) {
+#pragma unroll
+        for (int q8 = 0; q8 < 2; ++q8) {
+          const int col = cbase + jc * 16 + q8 * 8;
+          const uint32_t off = (col >> 6) * Lay::kSub + sw128_off(row, (col & 63) >> 3);
           *reinterpret_cast<uint4*>(smem + Lay::kDST + off) =
-              make_uint4(dw[q8 * 4], dw[q8 * 4 + 1], dw[q8 * 4 + 2], dw[q8 * 4 + 3]);
+              make_uint4(dw[jc][q8 * 4], dw[jc][q8 * 4 + 1], dw[jc][q8 * 4 + 2], dw[jc][q8 * 4 + 3]);
         }
       }
       if (!ok) break;
