@@ -89,16 +89,16 @@ fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __re
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   const int ql = lane % QL, sub = lane / QL;
   const float lam_v = *lam;
+  // gate weights (w_s then w_r) in shared memory, zero for fixed gates; the
+  // row chunks are read from the staging ring where they are used, so few
+  // values stay live across the row
+  __shared__ __align__(16) float s_w[2 * 128];
+  for (int i = threadIdx.x; i < 2 * d; i += blockDim.x) s_w[i] = gate_fixed ? 0.f : gate_w[i];
+  const float* ws4 = s_w + ql * 4;
+  const float* wr4 = s_w + d + ql * 4;
   float pws[4] = {0.f, 0.f, 0.f, 0.f}, pwr[4] = {0.f, 0.f, 0.f, 0.f};
   float pbs = 0.f, pbr = 0.f, plam = 0.f;
-  float ws4[4] = {0.f, 0.f, 0.f, 0.f}, wr4[4] = {0.f, 0.f, 0.f, 0.f};
-  float bs = 0.f, br = 0.f;
-  if (!gate_fixed) {
-    ld4<float>(gate_w + ql * 4, ws4);
-    ld4<float>(gate_w + d + ql * 4, wr4);
-    bs = gate_b[0];
-    br = gate_b[1];
-  }
+  const float bs = gate_fixed ? 0.f : gate_b[0], br = gate_fixed ? 0.f : gate_b[1];
   int64_t cur_bh = -1;   // unit whose largest |g_r dy / Ctot| this lane holds (lanes ql == 0)
   float cur_max = 0.f;
   const int64_t first = ((int64_t)blockIdx.x * nw + w) * QW;
@@ -122,6 +122,7 @@ fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __re
   };
   if (first < rows) stage(first, 0);
   asm volatile("cp.async.commit_group;" ::: "memory");
+  __syncthreads();   // s_w
   int buf = 0;
   for (int64_t r0 = first; r0 < rows; r0 += stride, buf ^= 1) {
     const int64_t r = r0 + sub;
@@ -131,20 +132,34 @@ fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __re
     if (r0 + stride < rows) stage(r0 + stride, buf ^ 1);
     asm volatile("cp.async.commit_group;" ::: "memory");
     asm volatile("cp.async.wait_group 1;" ::: "memory");   // this row's chunks are in
-    float qv[4], g[4], os[4], orc[4];
-    ld4<T>(reinterpret_cast<const T*>(&s_stage[w][buf][0][lane * CB]), qv);
-    ld4<T>(reinterpret_cast<const T*>(&s_stage[w][buf][1][lane * CB]), g);
-    ld4<T>(reinterpret_cast<const T*>(&s_stage[w][buf][2][lane * CB]), os);
-    ld4<T>(reinterpret_cast<const T*>(&s_stage[w][buf][3][lane * CB]), orc);
+    const T* st_q = reinterpret_cast<const T*>(&s_stage[w][buf][0][lane * CB]);
+    const T* st_g = reinterpret_cast<const T*>(&s_stage[w][buf][1][lane * CB]);
+    const T* st_os = reinterpret_cast<const T*>(&s_stage[w][buf][2][lane * CB]);
+    const T* st_or = reinterpret_cast<const T*>(&s_stage[w][buf][3][lane * CB]);
     const float l = __uint_as_float(s_scal[w][buf][0][lane]);
     const int c = (int)s_scal[w][buf][1][lane];
     float dyo = 0.f, dyr = 0.f, as = 0.f, ar = 0.f;
+    {
+      float g[4], os[4], orc[4];
+      ld4<T>(st_g, g);
+      ld4<T>(st_os, os);
+      ld4<T>(st_or, orc);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      dyo += g[i] * os[i];
-      dyr += g[i] * orc[i];
-      as += qv[i] * ws4[i];
-      ar += qv[i] * wr4[i];
+      for (int i = 0; i < 4; ++i) {
+        dyo += g[i] * os[i];
+        dyr += g[i] * orc[i];
+      }
+    }
+    if (!gate_fixed) {
+      float qv[4], w4s[4], w4r[4];
+      ld4<T>(st_q, qv);
+      ld4<float>(ws4, w4s);
+      ld4<float>(wr4, w4r);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        as += qv[i] * w4s[i];
+        ar += qv[i] * w4r[i];
+      }
     }
     dyo = gsum<QL>(dyo);
     dyr = gsum<QL>(dyr);
@@ -165,14 +180,17 @@ fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __re
       da_r = dyr * gr * (1.0f - gr);
     }
     const float inv_c = c > 0 ? 1.0f / (float)c : 0.f;
-    float dov[4], dqv[4], drv[4];
+    float dov[4], drv[4];
     float vmax = 0.f;
+    {
+      float g[4];
+      ld4<T>(st_g, g);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      dov[i] = gs * m * g[i];
-      dqv[i] = da_s * ws4[i] + da_r * wr4[i];
-      drv[i] = gr * g[i] * inv_c;
-      vmax = fmaxf(vmax, fabsf(drv[i]));
+      for (int i = 0; i < 4; ++i) {
+        dov[i] = gs * m * g[i];
+        drv[i] = gr * g[i] * inv_c;
+        vmax = fmaxf(vmax, fabsf(drv[i]));
+      }
     }
     vmax = fmaxf(vmax, 0.f);
 #pragma unroll
@@ -180,14 +198,27 @@ fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __re
     float dd = 0.f;
     if (valid) {
       st4_round<T>(d_o + base, dov);   // dov now holds the stored (rounded) values
-      if (dq_acc)
-        *reinterpret_cast<float4*>(dq_acc + base) = make_float4(dqv[0], dqv[1], dqv[2], dqv[3]);
+      if (dq_acc) {
+        float w4s[4], w4r[4];
+        ld4<float>(ws4, w4s);
+        ld4<float>(wr4, w4r);
+        *reinterpret_cast<float4*>(dq_acc + base) =
+            make_float4(da_s * w4s[0] + da_r * w4r[0], da_s * w4s[1] + da_r * w4r[1],
+                        da_s * w4s[2] + da_r * w4r[2], da_s * w4s[3] + da_r * w4r[3]);
+      }
       st4_round<T>(dor + base, drv);
+      float os[4];
+      ld4<T>(st_os, os);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        dd += dov[i] * os[i];
-        pws[i] += da_s * qv[i];
-        pwr[i] += da_r * qv[i];
+      for (int i = 0; i < 4; ++i) dd += dov[i] * os[i];
+      if (!gate_fixed) {
+        float qv[4];
+        ld4<T>(st_q, qv);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          pws[i] += da_s * qv[i];
+          pwr[i] += da_r * qv[i];
+        }
       }
     }
     dd = gsum<QL>(dd);

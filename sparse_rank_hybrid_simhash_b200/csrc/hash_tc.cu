@@ -56,8 +56,17 @@ HashShape hash_shape(const Geometry& g) {
   h.a_bytes = (uint32_t)kTile * g.d * 2;
   // per-tile staging: 128 rows of RACE code words, then 128 sort codes (u16)
   h.code_bytes = (uint32_t)((kTile * h.S * 4 + kTile * 2 + 15) / 16 * 16);
-  h.nbuf = (h.r_bytes + 2 * h.a_bytes + h.code_bytes + 64 <= (uint32_t)kSmemLimit) ? 2 : 1;
-  h.dyn = h.r_bytes + h.nbuf * h.a_bytes + h.code_bytes + 64;
+  // two A buffers overlap a tile's load with the previous tile's passes; one
+  // buffer wins where it lets one more CTA onto each SM (measured: 4 CTAs with
+  // one buffer beat 3 with two at text-32k sizes)
+  const uint32_t dyn1 = h.r_bytes + h.a_bytes + h.code_bytes + 64;
+  const uint32_t dyn2 = dyn1 + h.a_bytes;
+  auto per_sm = [](uint32_t dyn) {
+    const int n = (int)((228u * 1024u) / (dyn + 1024u));
+    return n > 4 ? 4 : n;
+  };
+  h.nbuf = (dyn2 <= (uint32_t)kSmemLimit && per_sm(dyn2) >= per_sm(dyn1)) ? 2 : 1;
+  h.dyn = h.nbuf == 2 ? dyn2 : dyn1;
   return h;
 }
 
