@@ -360,8 +360,19 @@ unit_absmax_kernel(const TV* __restrict__ vals, int64_t per_unit, float* __restr
   const int bh = blockIdx.y;
   const TV* v = vals + (size_t)bh * per_unit;
   float m = 0.f;
-  for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; i < per_unit;
-       i += (int64_t)gridDim.x * blockDim.x * 8) {
+  const int64_t step = (int64_t)gridDim.x * blockDim.x * 8;
+  int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  // four independent 8-value loads in flight per thread
+  for (; i + 3 * step < per_unit; i += 4 * step) {
+    float x[4][8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) load_vals8<TV>(v + i + u * step, x[u]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(x[u][e]));
+  }
+  for (; i < per_unit; i += step) {
     float x[8];
     load_vals8<TV>(v + i, x);
 #pragma unroll
