@@ -109,14 +109,14 @@ def stage_roofline(flops, nbytes, sec, peaks):
 # workload by the number of units; reported only while that file is unchanged.
 RECORDED_TRAFFIC = {
     # stage: (kernel source, its sha1 at capture, bytes per full-size launch)
-    "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "803a7fe621006eabe5ce0f2c498653ba03e4da75", 2.432e+08),
-    "race_build": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "c074d833a8677a22349643ee291b65fc403659e5", 1.369e+08),
-    "sparse_fwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_pipe.cu", "91a31d0c88874e37ef33ed4bb443baabc0c07369", 3.728e+08),
-    "race_fuse": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "c074d833a8677a22349643ee291b65fc403659e5", 3.733e+08),
-    "fuse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/fuse_bwd.cu", "b2b1538c8f47145cb34db05fe72d360dcc260381", 5.688e+08),
-    "race_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "c074d833a8677a22349643ee291b65fc403659e5", 1.317e+08),
-    "sparse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_bwd3.cu", "5530f1537a8b0a387b2bc31b36e8aaece4caa2c4", 6.643e+08),
-    "finish": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "c074d833a8677a22349643ee291b65fc403659e5", 1.583e+08),
+    "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "69efc768d31fb28fcd4a8ec01551bf7466f6ee92", 2.459e+08),
+    "race_build": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "9ff8ca9fd3724573a561d5ad5f1319a4dafe1fd0", 1.372e+08),
+    "sparse_fwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_pipe.cu", "91a31d0c88874e37ef33ed4bb443baabc0c07369", 3.735e+08),
+    "race_fuse": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "9ff8ca9fd3724573a561d5ad5f1319a4dafe1fd0", 3.717e+08),
+    "fuse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/fuse_bwd.cu", "c1e06a2a9098db4377026b2d34cb6b9937a690b7", 5.621e+08),
+    "race_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "9ff8ca9fd3724573a561d5ad5f1319a4dafe1fd0", 1.34e+08),
+    "sparse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_bwd3.cu", "86c54fd265fc87d0c79fa35a86c609fe1cdf0c1b", 6.626e+08),
+    "finish": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "9ff8ca9fd3724573a561d5ad5f1319a4dafe1fd0", 1.586e+08),
 }
 
 
