@@ -249,13 +249,83 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# ablation and single-branch modes (same kernels, other gate / lambda settings)
+# ---------------------------------------------------------------------------
+
+# mode: (gate_fixed, gate_s, gate_r, lambda or None to keep the workload's)
+MODES = {
+    "elsaa": None,                          # the workload as drawn: learned gates, lambda = 1
+    "sort_lsh_race": (False, None, None, 0.0),   # sparse multiplier fixed to one (lambda = 0)
+    "race_only": (True, 0.0, 1.0, None),    # y = O_race
+    "sparse_only": (True, 1.0, 0.0, 0.0),   # y = O_sp (Sort-LSH attention alone)
+}
+
+STANDS_IN_FOR = {
+    "text-32k": "synthetic (seeded; stands in for the ArXiv 32K text task)",
+    "vision-16k": "synthetic (seeded; stands in for the 16K image tasks)",
+    "needle-256k": "synthetic (seeded; stands in for needle-in-a-haystack)",
+}
+
+
+def bench_config(w, mode, world, l2):
+    """The config object of a bench line (both arms)."""
+    return {"workload": w.name, "mode": mode, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+            "sort_bits": w.sort_bits, "chunk": w.chunk, "race_tables": w.race_tables,
+            "race_bits": w.race_bits,
+            "gates": "learned" if not w.gate_fixed else f"fixed {w.gate_s}/{w.gate_r}",
+            "lambda": w.lam, "global_batch": world * w.B, "seq_len": w.N,
+            "parallelism": f"dp{world}", "l2": l2}
+
+
+def apply_mode(w, mode):
+    """The workload with the gate / lambda settings of an ablation mode."""
+    m = MODES[mode]
+    if m is None:
+        return w
+    fixed, gs, gr, lam = m
+    kw = {"gate_fixed": fixed}
+    if gs is not None:
+        kw.update(gate_s=gs, gate_r=gr)
+    if lam is not None:
+        kw["lam"] = lam
+    return w.replace(**kw)
+
+
+def time_dense_sdpa(w, d, steps=3, warmup=2):
+    """Dense softmax attention (torch SDPA, its own kernels) forward + backward on
+    the same Q, K, V: context for what the sparse branch replaces, not a path of
+    this library."""
+    import torch.nn.functional as F
+    q = d["q"].detach().clone().requires_grad_(True)
+    k = d["k"].detach().clone().requires_grad_(True)
+    v = d["v"].detach().clone().requires_grad_(True)
+
+    def one():
+        o = F.scaled_dot_product_attention(q, k, v)
+        o.backward(d["dy"])
+
+    for _ in range(warmup):
+        one()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s0.record()
+    for _ in range(steps):
+        one()
+    s1.record()
+    torch.cuda.synchronize()
+    ms = s0.elapsed_time(s1) / steps
+    return {"ms_per_step": ms, "tokens_per_s": w.tokens / (ms / 1e3), "steps": steps,
+            "impl": "torch scaled_dot_product_attention (dense, fwd+bwd)"}
+
+
+# ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 
 def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = WORKLOADS[args.workload]
+    w = apply_mode(WORKLOADS[args.workload], args.mode)
     p = B.Params.from_workload(w)
     inp = make_inputs(w, seed=DP.rank_seed(w.seed, rank), with_dy=True)
     d = {k: t.to(dev) for k, t in inp.items()}
@@ -313,7 +383,8 @@ def run_ours(args, rank, world, local_rank):
 
     # end to end through the public API with host buffers
     e2e = run_e2e(args, w, p, inp, dev, world)
-    return w, p, total_ms, fwd_total, stage_ms, clk.summary(), e2e
+    context = time_dense_sdpa(w, d) if args.dense_context and world == 1 else None
+    return w, p, total_ms, fwd_total, stage_ms, clk.summary(), e2e, context
 
 
 def run_e2e(args, w, p, inp, dev, world):
@@ -400,7 +471,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    w = WORKLOADS[args.workload]
+    w = apply_mode(WORKLOADS[args.workload], args.mode)
     cores = len(os.sched_getaffinity(0))
     torch.set_num_threads(cores)
     inp = make_inputs(w, with_dy=True)
@@ -419,10 +490,8 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps * (w.B * w.H / per_step),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded; stands in for the ArXiv 32K text task)",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                   "sort_bits": w.sort_bits, "chunk": w.chunk, "race_tables": w.race_tables,
-                   "race_bits": w.race_bits, "l2": "n/a (CPU)"},
+        "data": STANDS_IN_FOR.get(w.name, "synthetic (seeded)"),
+        "config": bench_config(w, args.mode, args.gpus, "n/a (CPU)"),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": torch.get_num_threads(),
                          "kind": "oracle",
                          "sample": f"{per_step} of {w.B * w.H} (batch, head) units per step, "
@@ -443,6 +512,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", default="elsaa", choices=sorted(MODES),
+                    help="ablation / single-branch setting of the gates and lambda")
+    ap.add_argument("--dense-context", action="store_true",
+                    help="also time dense torch SDPA fwd+bwd on the same inputs (context)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override B (small cases for ncu captures; not a bench line)")
     ap.add_argument("--heads", type=int, default=None,
@@ -461,7 +534,7 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
-    w, p, total_ms, fwd_ms, stage_ms, clocks, e2e = run_ours(args, rank, world, local_rank)
+    w, p, total_ms, fwd_ms, stage_ms, clocks, e2e, context = run_ours(args, rank, world, local_rank)
     peaks = load_peaks()
     if rank == 0:
         K = args.steps
@@ -479,13 +552,9 @@ def main():
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded; stands in for the ArXiv 32K text task)",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                       "sort_bits": w.sort_bits, "chunk": w.chunk,
-                       "race_tables": w.race_tables, "race_bits": w.race_bits,
-                       "global_batch": world * w.B, "seq_len": w.N,
-                       "parallelism": f"dp{world}",
-                       "l2": "256 MB flush between timed steps; inputs 0.4 GB > L2"},
+            "data": STANDS_IN_FOR.get(w.name, "synthetic (seeded)"),
+            "config": bench_config(w, args.mode, world,
+                                   "256 MB flush between timed steps; inputs 0.4 GB > L2"),
             "fwd_tokens_per_s": fwd_value,
             "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
             "roofline": {"bound": rl["bound"], "kernel": dom, "achieved": rl["achieved"],
@@ -503,6 +572,8 @@ def main():
             "clocks": clocks,
             "e2e": e2e,
         }
+        if context is not None:
+            line["context"] = {"dense_sdpa": context}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)

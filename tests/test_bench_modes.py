@@ -1,0 +1,48 @@
+"""Host logic of the bench's ablation / single-branch modes (no GPU): each
+mode sets the gates and lambda of the method's ablations, and the oracle under
+those settings reduces to the branch the mode names."""
+
+import importlib.util
+import os
+
+import pytest
+import torch
+
+import oracle as O
+from sparse_rank_hybrid_simhash_b200.workloads import WORKLOADS, make_inputs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_mode_settings():
+    bench = _bench()
+    w = WORKLOADS["text-32k"]
+    assert bench.apply_mode(w, "elsaa") == w
+    s = bench.apply_mode(w, "sort_lsh_race")
+    assert (s.gate_fixed, s.lam) == (False, 0.0)
+    r = bench.apply_mode(w, "race_only")
+    assert (r.gate_fixed, r.gate_s, r.gate_r, r.lam) == (True, 0.0, 1.0, w.lam)
+    p = bench.apply_mode(w, "sparse_only")
+    assert (p.gate_fixed, p.gate_s, p.gate_r, p.lam) == (True, 1.0, 0.0, 0.0)
+    cfg = bench.bench_config(p, "sparse_only", 1, "x")
+    assert cfg["mode"] == "sparse_only" and cfg["gates"] == "fixed 1.0/0.0" and cfg["lambda"] == 0.0
+
+
+@pytest.mark.parametrize("mode,branch", [("race_only", "o_race"), ("sparse_only", "o_sp")])
+def test_single_branch_modes_reduce_to_their_branch(mode, branch):
+    bench = _bench()
+    w = bench.apply_mode(WORKLOADS["iid-4k"].replace(B=1, H=1, N=256, chunk=64), mode)
+    inp = make_inputs(w, with_dy=False)
+    gw = None if w.gate_fixed else inp["gate_w"][0]
+    ref = O.forward_head(inp["q"][0, 0], inp["k"][0, 0], inp["v"][0, 0], inp["r_sort"],
+                         inp["r_race"], w.chunk, gate_w=gw, gate_b=inp["gate_b"],
+                         fixed_gates=(w.gate_s, w.gate_r) if w.gate_fixed else None,
+                         lam=float(inp["lam"][0]))
+    assert torch.allclose(ref["y"], ref[branch], rtol=0, atol=1e-12)
