@@ -17,6 +17,11 @@ Parity status of each function (what pins it, see ``tests/test_oracle.py``):
                        angular collision statistics
   stable_sort_perm     pinned: pure-Python sort by (code, index), permutation
                        and ordering properties
+  gray_rank / sort_keys
+                       pinned: inverts the enumerated reflected Gray code,
+                       one-bit steps between neighbouring buckets, brute-force
+                       stable sort by Gray position; local order = token order
+                       with a banded dense mask
   sparse_branch        pinned: one chunk == dense softmax attention, masked dense
                        softmax over the rank mask, one-hot value support test,
                        closed form for Q = 0
@@ -36,6 +41,9 @@ from .elsaa_oracle import (  # noqa: F401
     simhash_projections,
     simhash_codes,
     stable_sort_perm,
+    gray_rank,
+    sort_keys,
+    SORT_ORDERS,
     chunk_window,
     sparse_branch,
     race_build,

@@ -79,6 +79,37 @@ def stable_sort_perm(code: torch.Tensor) -> torch.Tensor:
     return torch.from_numpy(np.argsort(code.numpy(), kind="stable").astype(np.int64))
 
 
+SORT_ORDERS = ("binary", "gray", "local")
+
+
+def gray_rank(code: torch.Tensor) -> torch.Tensor:
+    """Position of each code in the reflected binary Gray sequence, i.e. the
+    b with b ^ (b >> 1) == code (prefix XOR of the code's bits from the top).
+    Ordering buckets this way makes neighbouring buckets differ in one
+    hyperplane; this is an extension of the pages' binary bucket order."""
+    b = code.to(torch.int64).clone()
+    shift = 1
+    while shift < 32:
+        b ^= b >> shift
+        shift <<= 1
+    return b
+
+
+def sort_keys(code: torch.Tensor, order: str = "binary") -> torch.Tensor:
+    """The key Sort-LSH sorts by.  binary: the code itself (the pages' Sort-LSH);
+    gray: the code's Gray-sequence position; local: one key for every token,
+    so the stable order is token order and chunks are local windows of
+    consecutive tokens (the ELSAA overview lists local windows among the
+    sparse patterns)."""
+    if order == "binary":
+        return code
+    if order == "gray":
+        return gray_rank(code)
+    if order == "local":
+        return torch.zeros_like(code)
+    raise ValueError(f"unknown sort order {order!r}")
+
+
 def chunk_window(rank: int, chunk: int) -> tuple:
     """Sorted key ranks [lo, hi) seen by the query at sorted rank ``rank``:
     its own chunk and the previous one (chunk 0 only itself), no wrap-around."""
@@ -188,7 +219,8 @@ def _hash_all(q64, k64, r_sort, r_race):
 
 def forward_head(q, k, v, r_sort, r_race, chunk: int, scale: Optional[float] = None,
                  gate_w=None, gate_b=None, lam=1.0, fixed_gates: Optional[tuple] = None,
-                 codes: Optional[Dict[str, torch.Tensor]] = None) -> Dict[str, torch.Tensor]:
+                 codes: Optional[Dict[str, torch.Tensor]] = None,
+                 sort_order: str = "binary") -> Dict[str, torch.Tensor]:
     """The whole operator on one (batch, head) unit.
 
     q, k, v: [N, d] (any float dtype; upcast to fp64).  r_sort: [b_s, d];
@@ -215,7 +247,8 @@ def forward_head(q, k, v, r_sort, r_race, chunk: int, scale: Optional[float] = N
     else:
         code_q, code_k = codes["code_q"].to(torch.int64), codes["code_k"].to(torch.int64)
         rcode_q, rcode_k = codes["rcode_q"].to(torch.int64), codes["rcode_k"].to(torch.int64)
-    perm_q, perm_k = stable_sort_perm(code_q), stable_sort_perm(code_k)
+    perm_q = stable_sort_perm(sort_keys(code_q, sort_order))
+    perm_k = stable_sort_perm(sort_keys(code_k, sort_order))
     o_sp, lse = sparse_branch(q64, k64, v64, perm_q, perm_k, chunk, scale)
     counts, sums = race_build(rcode_k, v64, 1 << kr)
     ctot, o_race, z_race = race_query(rcode_q, counts, sums)
@@ -233,7 +266,8 @@ def forward_head(q, k, v, r_sort, r_race, chunk: int, scale: Optional[float] = N
 
 def grads_head(q, k, v, r_sort, r_race, chunk: int, dy, scale: Optional[float] = None,
                gate_w=None, gate_b=None, lam=1.0, fixed_gates: Optional[tuple] = None,
-               codes: Optional[Dict[str, torch.Tensor]] = None) -> Dict[str, torch.Tensor]:
+               codes: Optional[Dict[str, torch.Tensor]] = None,
+               sort_order: str = "binary") -> Dict[str, torch.Tensor]:
     """Gradients of sum(y * dy) with the hash codes held constant (codes are
     piecewise constant in q and k), by fp64 autograd through forward_head.
     The pages state that ELSAA is used in training ("ELSAA combines sparsity
@@ -252,10 +286,10 @@ def grads_head(q, k, v, r_sort, r_race, chunk: int, dy, scale: Optional[float] =
         leaves += [gw, gb]
     if codes is None:
         first = forward_head(q, k, v, r_sort, r_race, chunk, scale, gate_w, gate_b, lam,
-                             fixed_gates)
+                             fixed_gates, sort_order=sort_order)
         codes = {name: first[name] for name in ("code_q", "code_k", "rcode_q", "rcode_k")}
     out = forward_head(q64, k64, v64, r_sort, r_race, chunk, scale, gw, gb, lam64,
-                       fixed_gates, codes=codes)
+                       fixed_gates, codes=codes, sort_order=sort_order)
     loss = (out["y"] * dy.to(F64)).sum()
     g = torch.autograd.grad(loss, leaves, allow_unused=True)
     res = {"dq": g[0], "dk": g[1], "dv": g[2], "dlambda": g[3]}
@@ -270,14 +304,14 @@ def grads_head(q, k, v, r_sort, r_race, chunk: int, dy, scale: Optional[float] =
 
 
 def forward_batch(q, k, v, r_sort, r_race, chunk: int, scale=None, gate_w=None,
-                  gate_b=None, lam=1.0, fixed_gates=None, units=None):
+                  gate_b=None, lam=1.0, fixed_gates=None, units=None, sort_order="binary"):
     """forward_head over (batch, head) units of [B, H, N, d] tensors; ``units``
     selects a subset of (b, h) pairs (default all).  Returns {(b, h): dict}."""
     B, H = q.shape[0], q.shape[1]
     if units is None:
         units = [(b, h) for b in range(B) for h in range(H)]
     return {(b, h): forward_head(q[b, h], k[b, h], v[b, h], r_sort, r_race, chunk, scale,
-                                 gate_w, gate_b, lam, fixed_gates)
+                                 gate_w, gate_b, lam, fixed_gates, sort_order=sort_order)
             for (b, h) in units}
 
 

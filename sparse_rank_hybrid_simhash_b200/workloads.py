@@ -55,6 +55,7 @@ class Workload:
     backward: bool = True
     seed: int = 0
     dist: str = "iid"      # iid | clusters | zipf | needle
+    sort_order: str = "binary"   # binary | gray | local (Sort-LSH bucket order)
 
     @property
     def torch_dtype(self):

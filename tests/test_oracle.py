@@ -341,3 +341,76 @@ def test_zero_race_bits_through_forward_head():
     out = O.forward_head(q, k, v, rs, rr, 8, None, gw, gb, lam=1.0)
     assert (out["ctot"] == 3 * 32).all()
     assert torch.allclose(out["o_race"], v.mean(0).expand(32, 4), atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Sort-LSH bucket orders: Gray sequence and local windows
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 5, 8, 16])
+def test_gray_rank_inverts_the_reflected_gray_code(bits):
+    # the reflected binary Gray code of position i is i ^ (i >> 1); its
+    # position must come back from the code
+    n = 1 << bits
+    pos = torch.arange(n, dtype=torch.int64) if bits <= 12 else torch.randint(0, n, (4096,))
+    codes = pos ^ (pos >> 1)
+    assert torch.equal(O.gray_rank(codes), pos)
+
+
+def test_gray_order_neighbours_differ_in_one_bit():
+    bits = 6
+    codes = torch.randint(0, 1 << bits, (500,), generator=torch.Generator().manual_seed(7))
+    perm = O.stable_sort_perm(O.sort_keys(codes, "gray"))
+    distinct = []
+    for t in perm.tolist():
+        c = int(codes[t])
+        if not distinct or distinct[-1] != c:
+            distinct.append(c)
+    assert len(distinct) == len(set(distinct))   # each bucket is one contiguous run
+    full = list(range(1 << bits))
+    seq = [i ^ (i >> 1) for i in full]          # the Gray sequence, enumerated
+    where = {c: i for i, c in enumerate(seq)}
+    assert [where[c] for c in distinct] == sorted(where[c] for c in distinct)
+    for a, b in zip(distinct, distinct[1:]):
+        if where[b] == where[a] + 1:
+            assert bin(a ^ b).count("1") == 1
+
+
+def test_gray_sort_is_stable_brute_force():
+    codes = torch.randint(0, 8, (60,), generator=torch.Generator().manual_seed(8))
+    seq = [i ^ (i >> 1) for i in range(8)]
+    pos = {c: i for i, c in enumerate(seq)}
+    expect = sorted(range(60), key=lambda t: (pos[int(codes[t])], t))
+    assert O.stable_sort_perm(O.sort_keys(codes, "gray")).tolist() == expect
+
+
+def test_local_order_is_token_order_and_a_banded_mask():
+    n, d, c = 48, 5, 8
+    codes = torch.randint(0, 16, (n,), generator=torch.Generator().manual_seed(9))
+    perm = O.stable_sort_perm(O.sort_keys(codes, "local"))
+    assert torch.equal(perm, torch.arange(n))
+    q, k, v = rnd((n, d), 15), rnd((n, d), 16), rnd((n, d), 17)
+    o, lse = O.sparse_branch(q, k, v, perm, perm, c, 0.4)
+    i = torch.arange(n)
+    ci, cj = (i // c)[:, None], (i // c)[None, :]
+    mask = (cj == ci) | (cj == ci - 1)          # own chunk and the previous one, in token order
+    s = (0.4 * q @ k.T).masked_fill(~mask, float("-inf"))
+    assert torch.allclose(o, torch.softmax(s, 1) @ v, atol=1e-12, rtol=0)
+    assert torch.allclose(lse, torch.logsumexp(s, 1), atol=1e-12, rtol=0)
+
+
+def test_sort_order_reaches_the_operator():
+    n, d, c = 64, 8, 16
+    q, k, v = rnd((n, d), 18), rnd((n, d), 19), rnd((n, d), 20)
+    rs = rnd((3, d), 21).float()
+    rr = rnd((2, 3, d), 22).float()
+    outs = {o: O.forward_head(q, k, v, rs, rr, c, None, lam=1.0, fixed_gates=(0.5, 0.5),
+                              sort_order=o) for o in O.SORT_ORDERS}
+    assert torch.equal(outs["local"]["perm_q"], torch.arange(n))
+    assert torch.equal(outs["gray"]["perm_q"],
+                       O.stable_sort_perm(O.gray_rank(outs["gray"]["code_q"])))
+    # the RACE branch does not depend on the order
+    for o in ("gray", "local"):
+        assert torch.allclose(outs[o]["o_race"], outs["binary"]["o_race"], atol=0, rtol=0)
+    with pytest.raises(ValueError):
+        O.sort_keys(outs["binary"]["code_q"], "spiral")
