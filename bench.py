@@ -270,7 +270,8 @@ STANDS_IN_FOR = {
 def bench_config(w, mode, world, l2):
     """The config object of a bench line (both arms)."""
     return {"workload": w.name, "mode": mode, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-            "sort_bits": w.sort_bits, "chunk": w.chunk, "race_tables": w.race_tables,
+            "sort_bits": w.sort_bits, "sort_order": w.sort_order, "chunk": w.chunk,
+            "race_tables": w.race_tables,
             "race_bits": w.race_bits,
             "gates": "learned" if not w.gate_fixed else f"fixed {w.gate_s}/{w.gate_r}",
             "lambda": w.lam, "global_batch": world * w.B, "seq_len": w.N,
@@ -325,7 +326,7 @@ def time_dense_sdpa(w, d, steps=3, warmup=2):
 def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = apply_mode(WORKLOADS[args.workload], args.mode)
+    w = apply_mode(WORKLOADS[args.workload], args.mode).replace(sort_order=args.sort_order)
     p = B.Params.from_workload(w)
     inp = make_inputs(w, seed=DP.rank_seed(w.seed, rank), with_dy=True)
     d = {k: t.to(dev) for k, t in inp.items()}
@@ -443,8 +444,9 @@ def oracle_unit_seconds(w, inp, units):
     for (b, h) in units:
         args = (inp["q"][b, h], inp["k"][b, h], inp["v"][b, h], inp["r_sort"], inp["r_race"],
                 w.chunk)
+        fixed = (w.gate_s, w.gate_r) if w.gate_fixed else None
         O.grads_head(*args, inp["dy"][b, h], None, inp["gate_w"], inp["gate_b"],
-                     float(inp["lam"][0]))
+                     float(inp["lam"][0]), fixed, sort_order=w.sort_order)
     return time.perf_counter() - t0
 
 
@@ -471,7 +473,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    w = apply_mode(WORKLOADS[args.workload], args.mode)
+    w = apply_mode(WORKLOADS[args.workload], args.mode).replace(sort_order=args.sort_order)
     cores = len(os.sched_getaffinity(0))
     torch.set_num_threads(cores)
     inp = make_inputs(w, with_dy=True)
@@ -514,6 +516,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--mode", default="elsaa", choices=sorted(MODES),
                     help="ablation / single-branch setting of the gates and lambda")
+    ap.add_argument("--sort-order", default="binary", choices=["binary", "gray", "local"],
+                    help="Sort-LSH chunk order: code value, Gray sequence, or token order")
     ap.add_argument("--dense-context", action="store_true",
                     help="also time dense torch SDPA fwd+bwd on the same inputs (context)")
     ap.add_argument("--batch", type=int, default=None,

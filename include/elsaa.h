@@ -64,6 +64,16 @@ typedef enum {
 
 typedef enum { ELSAA_BF16 = 0, ELSAA_F32 = 1 } elsaa_dtype;
 
+/* Order of the Sort-LSH chunks ("Two Efficient Attentions, One Denominator
+ * Problem", section "The ablation isolates the actual contribution": tokens
+ * sorted by hash code, consecutive chunks attend).  BINARY sorts by the code
+ * value (the pages' Sort-LSH); GRAY sorts by the code's position in the
+ * reflected binary Gray sequence, so neighbouring buckets differ in one
+ * hyperplane (an extension); LOCAL keeps token order, i.e. local windows of
+ * consecutive tokens (the ELSAA overview lists local windows among the sparse
+ * patterns).  Every order is stable: equal keys keep token order. */
+typedef enum { ELSAA_SORT_BINARY = 0, ELSAA_SORT_GRAY = 1, ELSAA_SORT_LOCAL = 2 } elsaa_sort_order;
+
 typedef struct {
   int32_t B, H, N, d;     /* batch, heads, tokens per unit, head dim d in {32, 64, 128} */
   int32_t dtype;          /* elsaa_dtype of q, k, v, r_sort, r_race, y, dy, dq, dk, dv */
@@ -74,6 +84,7 @@ typedef struct {
   float scale;            /* score scale; <= 0 selects 1/sqrt(d) */
   int32_t gate_fixed;     /* nonzero: gates are the constants gate_s, gate_r */
   float gate_s, gate_r;
+  int32_t sort_order;     /* elsaa_sort_order of the Sort-LSH chunks */
 } elsaa_params;
 
 /* Device views into a forward's saved state (see elsaa_saved_views). */

@@ -18,6 +18,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libelsaa.so")
 
 ELSAA_BF16, ELSAA_F32 = 0, 1
+# elsaa_sort_order: the Sort-LSH chunk order
+SORT_ORDERS = {"binary": 0, "gray": 1, "local": 2}
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported problem", 3: "workspace too small",
           4: "CUDA error", 5: "device wait timed out", 6: "device index check failed"}
 
@@ -35,19 +37,19 @@ class Params(ctypes.Structure):
                 ("chunk", ctypes.c_int32), ("race_tables", ctypes.c_int32),
                 ("race_bits", ctypes.c_int32), ("scale", ctypes.c_float),
                 ("gate_fixed", ctypes.c_int32), ("gate_s", ctypes.c_float),
-                ("gate_r", ctypes.c_float)]
+                ("gate_r", ctypes.c_float), ("sort_order", ctypes.c_int32)]
 
     @classmethod
     def make(cls, B, H, N, d, dtype, sort_bits, chunk, race_tables, race_bits, scale=0.0,
-             gate_fixed=False, gate_s=0.5, gate_r=0.5) -> "Params":
+             gate_fixed=False, gate_s=0.5, gate_r=0.5, sort_order="binary") -> "Params":
         dt = ELSAA_BF16 if dtype in ("bf16", torch.bfloat16) else ELSAA_F32
         return cls(B, H, N, d, dt, sort_bits, chunk, race_tables, race_bits, float(scale),
-                   int(bool(gate_fixed)), float(gate_s), float(gate_r))
+                   int(bool(gate_fixed)), float(gate_s), float(gate_r), SORT_ORDERS[sort_order])
 
     @classmethod
     def from_workload(cls, w) -> "Params":
         return cls.make(w.B, w.H, w.N, w.d, w.dtype, w.sort_bits, w.chunk, w.race_tables,
-                        w.race_bits, 0.0, w.gate_fixed, w.gate_s, w.gate_r)
+                        w.race_bits, 0.0, w.gate_fixed, w.gate_s, w.gate_r, w.sort_order)
 
     @property
     def torch_dtype(self):

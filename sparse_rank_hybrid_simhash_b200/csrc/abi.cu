@@ -15,6 +15,9 @@ bool make_geometry(const elsaa_params* p, Geometry* g, elsaa_status* why) {
   if (p->dtype != ELSAA_BF16 && p->dtype != ELSAA_F32) return false;
   if (p->chunk <= 0 || p->N % p->chunk != 0) return false;
   if (p->sort_bits < 0 || p->sort_bits > 16) return false;
+  if (p->sort_order != ELSAA_SORT_BINARY && p->sort_order != ELSAA_SORT_GRAY &&
+      p->sort_order != ELSAA_SORT_LOCAL)
+    return false;
   if (p->race_tables < 1 || p->race_tables > 4096) return false;
   if (p->race_bits < 0 || p->race_bits > 16) return false;
   if ((int64_t)p->B * p->H * p->N * (p->d > p->race_tables ? p->d : p->race_tables) >
@@ -39,6 +42,7 @@ bool make_geometry(const elsaa_params* p, Geometry* g, elsaa_status* why) {
   g->gate_fixed = p->gate_fixed ? 1 : 0;
   g->gate_s = p->gate_s;
   g->gate_r = p->gate_r;
+  g->sort_order = p->sort_order;
   g->sort_passes = p->sort_bits <= 8 ? 1 : 2;
   g->sort_digit_bits = (p->sort_bits + g->sort_passes - 1) / g->sort_passes;
   g->sort_bins = 1 << g->sort_digit_bits;

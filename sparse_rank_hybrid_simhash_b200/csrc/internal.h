@@ -28,6 +28,7 @@ struct Geometry {
   float scale;
   int gate_fixed;      // nonzero: constant gates gate_s, gate_r
   float gate_s, gate_r;
+  int sort_order;      // elsaa_sort_order
   int sort_passes, sort_digit_bits, sort_bins, sort_tiles;
   bool tc_hash;       // tcgen05 kernel for the SimHash codes
   bool tc_attn;       // tcgen05 kernels for the sparse branch

@@ -12,6 +12,9 @@
 //      digits, take per-warp bases, then rank equal digits within each
 //      32-key round with __match_any_sync.
 // Codes of up to 16 bits take two passes (the second reads the first's order).
+// Gray order sorts by each code's position in the reflected binary Gray
+// sequence (the prefix XOR of its bits from the top), computed where a code is
+// read; local order writes token order without sorting.
 #include <mutex>
 
 #include "common.cuh"
@@ -23,9 +26,22 @@ namespace {
 constexpr int kWarps = kSortThreads / 32;
 constexpr int kPerWarp = kSortTile / kWarps;   // 256 keys, 8 rounds of 32
 
+// The sort key of a code: the code itself, or its Gray-sequence position.
+ELSAA_DEV int sort_key(uint16_t code, int gray) {
+  int b = code;
+  if (gray) {
+    b ^= b >> 1;
+    b ^= b >> 2;
+    b ^= b >> 4;
+    b ^= b >> 8;
+  }
+  return b;
+}
+
 __global__ void __launch_bounds__(kSortThreads)
 sort_hist_kernel(const uint16_t* __restrict__ code, const int32_t* __restrict__ order_in,
-                 int N, int shift, int mask, int bins, int tiles, int32_t* __restrict__ hist) {
+                 int N, int shift, int mask, int bins, int tiles, int gray,
+                 int32_t* __restrict__ hist) {
   __shared__ int h[256];
   for (int i = threadIdx.x; i < bins; i += blockDim.x) h[i] = 0;
   __syncthreads();
@@ -35,7 +51,7 @@ sort_hist_kernel(const uint16_t* __restrict__ code, const int32_t* __restrict__ 
   const int p0 = tile * kSortTile, p1 = min(N, p0 + kSortTile);
   for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
     const int idx = oin ? oin[p] : p;
-    atomicAdd(&h[(c[idx] >> shift) & mask], 1);
+    atomicAdd(&h[(sort_key(c[idx], gray) >> shift) & mask], 1);
   }
   __syncthreads();
   for (int b = threadIdx.x; b < bins; b += blockDim.x)
@@ -80,7 +96,7 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(int32_t* __restrict__ h
 
 __global__ void __launch_bounds__(kSortThreads)
 sort_scatter_kernel(const uint16_t* __restrict__ code, const int32_t* __restrict__ order_in,
-                    int N, int shift, int mask, int bins, int tiles,
+                    int N, int shift, int mask, int bins, int tiles, int gray,
                     const int32_t* __restrict__ offs, int32_t* __restrict__ order_out) {
   __shared__ int cnt[kWarps][256];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -97,7 +113,7 @@ sort_scatter_kernel(const uint16_t* __restrict__ code, const int32_t* __restrict
     const int p = base_p + r * 32 + lane;
     const bool valid = p < N;
     const int idx = valid ? (oin ? oin[p] : p) : 0;
-    const int key = valid ? ((c[idx] >> shift) & mask) : (bins + lane);
+    const int key = valid ? ((sort_key(c[idx], gray) >> shift) & mask) : (bins + lane);
     const unsigned peers = __match_any_sync(0xffffffffu, key);
     if (valid && lane == __ffs(peers) - 1) cnt[w][key] += __popc(peers);
     __syncwarp();
@@ -118,7 +134,7 @@ sort_scatter_kernel(const uint16_t* __restrict__ code, const int32_t* __restrict
     const int p = base_p + r * 32 + lane;
     const bool valid = p < N;
     const int idx = valid ? (oin ? oin[p] : p) : 0;
-    const int key = valid ? ((c[idx] >> shift) & mask) : (bins + lane);
+    const int key = valid ? ((sort_key(c[idx], gray) >> shift) & mask) : (bins + lane);
     const unsigned peers = __match_any_sync(0xffffffffu, key);
     int pos = 0;
     if (valid) pos = cnt[w][key] + __popc(peers & lt);
@@ -131,11 +147,26 @@ sort_scatter_kernel(const uint16_t* __restrict__ code, const int32_t* __restrict
   }
 }
 
+// perm[seg][i] = i: local windows keep token order.
+__global__ void __launch_bounds__(256)
+token_order_kernel(int64_t total, int N, int32_t* __restrict__ perm) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x)
+    perm[i] = (int32_t)(i % N);
+}
+
 }  // namespace
 
 cudaError_t launch_sort(const Geometry& g, const uint16_t* code, int32_t* perm, int32_t* hist,
                         int32_t* tmp, cudaStream_t s) {
   const int segs = 2 * g.BH;
+  if (g.sort_order == ELSAA_SORT_LOCAL) {
+    const int64_t total = (int64_t)segs * g.N;
+    const int64_t want = (total + 255) / 256;
+    token_order_kernel<<<(int)(want < 148 * 8 ? want : 148 * 8), 256, 0, s>>>(total, g.N, perm);
+    return cudaGetLastError();
+  }
+  const int gray = g.sort_order == ELSAA_SORT_GRAY ? 1 : 0;
   const dim3 grid(g.sort_tiles, segs);
   const int mask = g.sort_bins - 1;
   for (int pass = 0; pass < g.sort_passes; ++pass) {
@@ -143,10 +174,10 @@ cudaError_t launch_sort(const Geometry& g, const uint16_t* code, int32_t* perm, 
     const int32_t* in = pass == 0 ? nullptr : tmp;
     int32_t* out = (pass == g.sort_passes - 1) ? perm : tmp;
     sort_hist_kernel<<<grid, kSortThreads, 0, s>>>(code, in, g.N, shift, mask, g.sort_bins,
-                                                   g.sort_tiles, hist);
+                                                   g.sort_tiles, gray, hist);
     sort_scan_kernel<<<segs, 1024, 0, s>>>(hist, g.sort_bins * g.sort_tiles);
     sort_scatter_kernel<<<grid, kSortThreads, 0, s>>>(code, in, g.N, shift, mask, g.sort_bins,
-                                                      g.sort_tiles, hist, out);
+                                                      g.sort_tiles, gray, hist, out);
   }
   return cudaGetLastError();
 }

@@ -76,6 +76,8 @@ def test_validation_rejects_bad_problems():
         dict(race_bits=17),
         dict(race_tables=0),
         dict(dtype=7),
+        dict(sort_order=3),
+        dict(sort_order=-1),
     ]
     for c in cases:
         p = B.Params.make(1, 2, 256, 64, "bf16", 4, 64, 8, 6)
@@ -85,6 +87,8 @@ def test_validation_rejects_bad_problems():
         assert B.workspace_bytes(p) == 0 and B.saved_bytes(p) == 0
     p = B.Params.make(1, 2, 256, 48, "bf16", 4, 64, 8, 6)   # head dim not a multiple of 32
     assert B.validate(p) == 2
+    for order in B.SORT_ORDERS:
+        assert B.validate(B.Params.make(1, 2, 256, 64, "bf16", 4, 64, 8, 6, sort_order=order)) == 0
 
 
 def test_null_pointers_are_rejected_before_any_launch():

@@ -70,6 +70,15 @@ def test_small_chunks(cuda_device, chunk):
     _run(w, backward=True)
 
 
+@pytest.mark.parametrize("order,sort_bits", [("gray", 7), ("gray", 12), ("local", 4)])
+def test_sort_orders(cuda_device, order, sort_bits):
+    # Gray-sequence bucket order (one and two radix passes) and local windows
+    # in token order, through the same attention and RACE kernels
+    w = WORKLOADS["iid-4k"].replace(B=1, H=2, N=1024, chunk=64, sort_bits=sort_bits,
+                                    sort_order=order)
+    _run(w, backward=True)
+
+
 def test_two_pass_sort_and_wide_race_codes(cuda_device):
     # 12 sort bits take two radix passes; 11 RACE bits give uint16 codes and
     # 2048-bucket tables (the global-atomic build)
