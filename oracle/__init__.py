@@ -23,8 +23,8 @@ Parity status of each function (what pins it, see ``tests/test_oracle.py``):
                        stable sort by Gray position; local order = token order
                        with a banded dense mask
   sparse_branch        pinned: one chunk == dense softmax attention, masked dense
-                       softmax over the rank mask, one-hot value support test,
-                       closed form for Q = 0
+                       softmax over the rank mask (lookback 0 to 3 chunks),
+                       one-hot value support test, closed form for Q = 0
   race_build / race_query
                        pinned: per-table sums, K_r = 0 closed form, collision
                        count matrix brute force

@@ -110,18 +110,20 @@ def sort_keys(code: torch.Tensor, order: str = "binary") -> torch.Tensor:
     raise ValueError(f"unknown sort order {order!r}")
 
 
-def chunk_window(rank: int, chunk: int) -> tuple:
+def chunk_window(rank: int, chunk: int, lookback: int = 1) -> tuple:
     """Sorted key ranks [lo, hi) seen by the query at sorted rank ``rank``:
-    its own chunk and the previous one (chunk 0 only itself), no wrap-around."""
+    its own chunk and the previous one (chunk 0 only itself), no wrap-around.
+    ``lookback`` previous chunks instead of one is an extension (0: the own
+    chunk only); the pages' Sort-LSH is lookback = 1."""
     j = rank // chunk
-    return max(0, (j - 1) * chunk), (j + 1) * chunk
+    return max(0, (j - lookback) * chunk), (j + 1) * chunk
 
 
 # ---------------------------------------------------------------------------
 # Step 3: exact sparse branch
 # ---------------------------------------------------------------------------
 
-def sparse_branch(q, k, v, perm_q, perm_k, chunk: int, scale: float):
+def sparse_branch(q, k, v, perm_q, perm_k, chunk: int, scale: float, lookback: int = 1):
     """Exact softmax attention restricted to the Sort-LSH window ("Two
     Efficient Attentions, One Denominator Problem", section "Two efficient
     branches can still be mis-scaled": the sparse branch computes only the
@@ -131,7 +133,7 @@ def sparse_branch(q, k, v, perm_q, perm_k, chunk: int, scale: float):
     qs, ks, vs = q[perm_q], k[perm_k], v[perm_k]
     outs, lses = [], []
     for j in range(n // chunk):
-        lo, hi = chunk_window(j * chunk, chunk)
+        lo, hi = chunk_window(j * chunk, chunk, lookback)
         s = scale * (qs[j * chunk:(j + 1) * chunk] @ ks[lo:hi].T)
         lses.append(torch.logsumexp(s, dim=1))
         outs.append(torch.softmax(s, dim=1) @ vs[lo:hi])
@@ -220,7 +222,7 @@ def _hash_all(q64, k64, r_sort, r_race):
 def forward_head(q, k, v, r_sort, r_race, chunk: int, scale: Optional[float] = None,
                  gate_w=None, gate_b=None, lam=1.0, fixed_gates: Optional[tuple] = None,
                  codes: Optional[Dict[str, torch.Tensor]] = None,
-                 sort_order: str = "binary") -> Dict[str, torch.Tensor]:
+                 sort_order: str = "binary", lookback: int = 1) -> Dict[str, torch.Tensor]:
     """The whole operator on one (batch, head) unit.
 
     q, k, v: [N, d] (any float dtype; upcast to fp64).  r_sort: [b_s, d];
@@ -249,7 +251,7 @@ def forward_head(q, k, v, r_sort, r_race, chunk: int, scale: Optional[float] = N
         rcode_q, rcode_k = codes["rcode_q"].to(torch.int64), codes["rcode_k"].to(torch.int64)
     perm_q = stable_sort_perm(sort_keys(code_q, sort_order))
     perm_k = stable_sort_perm(sort_keys(code_k, sort_order))
-    o_sp, lse = sparse_branch(q64, k64, v64, perm_q, perm_k, chunk, scale)
+    o_sp, lse = sparse_branch(q64, k64, v64, perm_q, perm_k, chunk, scale, lookback)
     counts, sums = race_build(rcode_k, v64, 1 << kr)
     ctot, o_race, z_race = race_query(rcode_q, counts, sums)
     if fixed_gates is None:
@@ -267,7 +269,7 @@ def forward_head(q, k, v, r_sort, r_race, chunk: int, scale: Optional[float] = N
 def grads_head(q, k, v, r_sort, r_race, chunk: int, dy, scale: Optional[float] = None,
                gate_w=None, gate_b=None, lam=1.0, fixed_gates: Optional[tuple] = None,
                codes: Optional[Dict[str, torch.Tensor]] = None,
-               sort_order: str = "binary") -> Dict[str, torch.Tensor]:
+               sort_order: str = "binary", lookback: int = 1) -> Dict[str, torch.Tensor]:
     """Gradients of sum(y * dy) with the hash codes held constant (codes are
     piecewise constant in q and k), by fp64 autograd through forward_head.
     The pages state that ELSAA is used in training ("ELSAA combines sparsity
@@ -286,10 +288,10 @@ def grads_head(q, k, v, r_sort, r_race, chunk: int, dy, scale: Optional[float] =
         leaves += [gw, gb]
     if codes is None:
         first = forward_head(q, k, v, r_sort, r_race, chunk, scale, gate_w, gate_b, lam,
-                             fixed_gates, sort_order=sort_order)
+                             fixed_gates, sort_order=sort_order, lookback=lookback)
         codes = {name: first[name] for name in ("code_q", "code_k", "rcode_q", "rcode_k")}
     out = forward_head(q64, k64, v64, r_sort, r_race, chunk, scale, gw, gb, lam64,
-                       fixed_gates, codes=codes, sort_order=sort_order)
+                       fixed_gates, codes=codes, sort_order=sort_order, lookback=lookback)
     loss = (out["y"] * dy.to(F64)).sum()
     g = torch.autograd.grad(loss, leaves, allow_unused=True)
     res = {"dq": g[0], "dk": g[1], "dv": g[2], "dlambda": g[3]}
@@ -304,14 +306,16 @@ def grads_head(q, k, v, r_sort, r_race, chunk: int, dy, scale: Optional[float] =
 
 
 def forward_batch(q, k, v, r_sort, r_race, chunk: int, scale=None, gate_w=None,
-                  gate_b=None, lam=1.0, fixed_gates=None, units=None, sort_order="binary"):
+                  gate_b=None, lam=1.0, fixed_gates=None, units=None, sort_order="binary",
+                  lookback=1):
     """forward_head over (batch, head) units of [B, H, N, d] tensors; ``units``
     selects a subset of (b, h) pairs (default all).  Returns {(b, h): dict}."""
     B, H = q.shape[0], q.shape[1]
     if units is None:
         units = [(b, h) for b in range(B) for h in range(H)]
     return {(b, h): forward_head(q[b, h], k[b, h], v[b, h], r_sort, r_race, chunk, scale,
-                                 gate_w, gate_b, lam, fixed_gates, sort_order=sort_order)
+                                 gate_w, gate_b, lam, fixed_gates, sort_order=sort_order,
+                                 lookback=lookback)
             for (b, h) in units}
 
 

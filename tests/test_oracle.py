@@ -414,3 +414,34 @@ def test_sort_order_reaches_the_operator():
         assert torch.allclose(outs[o]["o_race"], outs["binary"]["o_race"], atol=0, rtol=0)
     with pytest.raises(ValueError):
         O.sort_keys(outs["binary"]["code_q"], "spiral")
+
+
+@pytest.mark.parametrize("lookback", [0, 2, 3])
+def test_lookback_window_equals_masked_dense_softmax(lookback):
+    n, d, c = 48, 6, 8
+    q, k, v = rnd((n, d), 23), rnd((n, d), 24), rnd((n, d), 25)
+    pq = torch.randperm(n, generator=torch.Generator().manual_seed(26))
+    pk = torch.randperm(n, generator=torch.Generator().manual_seed(27))
+    o, lse = O.sparse_branch(q, k, v, pq, pk, c, 0.5, lookback)
+    rank_q = {int(t): r for r, t in enumerate(pq)}
+    rank_k = {int(t): r for r, t in enumerate(pk)}
+    mask = torch.zeros(n, n, dtype=torch.bool)
+    for i in range(n):
+        for j in range(n):
+            cq, ck = rank_q[i] // c, rank_k[j] // c
+            mask[i, j] = cq - lookback <= ck <= cq
+    s = (0.5 * q @ k.T).masked_fill(~mask, float("-inf"))
+    assert torch.allclose(o, torch.softmax(s, 1) @ v, atol=1e-12, rtol=0)
+    assert torch.allclose(lse, torch.logsumexp(s, 1), atol=1e-12, rtol=0)
+    for i in range(n):   # chunk j sees min(j, lookback) + 1 chunks
+        assert int(mask[i].sum()) == c * (min(rank_q[i] // c, lookback) + 1)
+
+
+def test_lookback_zero_with_one_chunk_is_dense_attention():
+    n, d = 24, 5
+    q, k, v = rnd((n, d), 28), rnd((n, d), 29), rnd((n, d), 30)
+    pq = torch.randperm(n, generator=torch.Generator().manual_seed(31))
+    pk = torch.randperm(n, generator=torch.Generator().manual_seed(32))
+    o, _ = O.sparse_branch(q, k, v, pq, pk, n, 0.7, 0)
+    ref = torch.nn.functional.scaled_dot_product_attention(q[None], k[None], v[None], scale=0.7)[0]
+    assert torch.allclose(o, ref, atol=1e-12, rtol=0)
