@@ -61,9 +61,10 @@ def load_peaks():
 # algorithmic work per stage (what the method must do, not what a kernel does)
 # ---------------------------------------------------------------------------
 
-def window_keys(N: int, c: int) -> int:
-    """sum over queries of the keys in their Sort-LSH window (own + previous chunk)."""
-    return sum(c * (min((j + 1) * c, N) - max(0, (j - 1) * c)) for j in range(N // c))
+def window_keys(N: int, c: int, lookback: int = 1) -> int:
+    """sum over queries of the keys in their Sort-LSH window (own chunk and
+    ``lookback`` previous ones)."""
+    return sum(c * (min((j + 1) * c, N) - max(0, (j - lookback) * c)) for j in range(N // c))
 
 
 def stage_work(w):
@@ -75,7 +76,7 @@ def stage_work(w):
     e = 2 if w.dtype == "bf16" else 4
     rb = 1 if w.race_bits <= 8 else 2
     P = w.sort_bits + L * w.race_bits
-    wk = window_keys(N, w.chunk) * BH       # query-key pairs of the sparse branch
+    wk = window_keys(N, w.chunk, w.lookback) * BH   # query-key pairs of the sparse branch
     rows = BH * N
     tables = BH * L * NB
     return {
@@ -139,7 +140,7 @@ def operator_roofline(w, peaks):
     BH, N, d = w.B * w.H, w.N, w.d
     e = 2 if w.dtype == "bf16" else 4
     P = w.sort_bits + w.race_tables * w.race_bits
-    wk = window_keys(N, w.chunk) * BH
+    wk = window_keys(N, w.chunk, w.lookback) * BH
     rows = BH * N
     f_fwd = 2.0 * 2 * rows * d * P + 4.0 * wk * d
     f_bwd = 10.0 * wk * d
@@ -270,7 +271,8 @@ STANDS_IN_FOR = {
 def bench_config(w, mode, world, l2):
     """The config object of a bench line (both arms)."""
     return {"workload": w.name, "mode": mode, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-            "sort_bits": w.sort_bits, "sort_order": w.sort_order, "chunk": w.chunk,
+            "sort_bits": w.sort_bits, "sort_order": w.sort_order, "lookback": w.lookback,
+            "chunk": w.chunk,
             "race_tables": w.race_tables,
             "race_bits": w.race_bits,
             "gates": "learned" if not w.gate_fixed else f"fixed {w.gate_s}/{w.gate_r}",
@@ -326,7 +328,8 @@ def time_dense_sdpa(w, d, steps=3, warmup=2):
 def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = apply_mode(WORKLOADS[args.workload], args.mode).replace(sort_order=args.sort_order)
+    w = apply_mode(WORKLOADS[args.workload], args.mode).replace(
+        sort_order=args.sort_order, lookback=args.lookback)
     p = B.Params.from_workload(w)
     inp = make_inputs(w, seed=DP.rank_seed(w.seed, rank), with_dy=True)
     d = {k: t.to(dev) for k, t in inp.items()}
@@ -473,7 +476,8 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    w = apply_mode(WORKLOADS[args.workload], args.mode).replace(sort_order=args.sort_order)
+    w = apply_mode(WORKLOADS[args.workload], args.mode).replace(
+        sort_order=args.sort_order, lookback=args.lookback)
     cores = len(os.sched_getaffinity(0))
     torch.set_num_threads(cores)
     inp = make_inputs(w, with_dy=True)
@@ -518,6 +522,8 @@ def main():
                     help="ablation / single-branch setting of the gates and lambda")
     ap.add_argument("--sort-order", default="binary", choices=["binary", "gray", "local"],
                     help="Sort-LSH chunk order: code value, Gray sequence, or token order")
+    ap.add_argument("--lookback", type=int, default=1,
+                    help="previous sorted chunks a query chunk attends (1: own and previous)")
     ap.add_argument("--dense-context", action="store_true",
                     help="also time dense torch SDPA fwd+bwd on the same inputs (context)")
     ap.add_argument("--batch", type=int, default=None,

@@ -85,6 +85,10 @@ typedef struct {
   int32_t gate_fixed;     /* nonzero: gates are the constants gate_s, gate_r */
   float gate_s, gate_r;
   int32_t sort_order;     /* elsaa_sort_order of the Sort-LSH chunks */
+  int32_t lookback;       /* previous sorted chunks a query chunk attends besides its own,
+                           * 0..64 with (lookback + 1) * chunk <= 6144: 1 is the pages'
+                           * Sort-LSH (own and previous chunk); other values are an
+                           * extension served by the CUDA-core attention kernels */
 } elsaa_params;
 
 /* Device views into a forward's saved state (see elsaa_saved_views). */

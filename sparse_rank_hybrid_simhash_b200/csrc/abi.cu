@@ -18,6 +18,7 @@ bool make_geometry(const elsaa_params* p, Geometry* g, elsaa_status* why) {
   if (p->sort_order != ELSAA_SORT_BINARY && p->sort_order != ELSAA_SORT_GRAY &&
       p->sort_order != ELSAA_SORT_LOCAL)
     return false;
+  if (p->lookback < 0 || p->lookback > 64) return false;
   if (p->race_tables < 1 || p->race_tables > 4096) return false;
   if (p->race_bits < 0 || p->race_bits > 16) return false;
   if ((int64_t)p->B * p->H * p->N * (p->d > p->race_tables ? p->d : p->race_tables) >
@@ -25,6 +26,8 @@ bool make_geometry(const elsaa_params* p, Geometry* g, elsaa_status* why) {
     return false;
   *why = ELSAA_ERR_UNSUPPORTED;
   if (p->d != 32 && p->d != 64 && p->d != 128) return false;
+  // the CUDA-core attention keeps a query's window of scores in shared memory
+  if ((int64_t)(p->lookback + 1) * p->chunk > 6144) return false;
   g->B = p->B;
   g->H = p->H;
   g->N = p->N;
@@ -43,6 +46,7 @@ bool make_geometry(const elsaa_params* p, Geometry* g, elsaa_status* why) {
   g->gate_s = p->gate_s;
   g->gate_r = p->gate_r;
   g->sort_order = p->sort_order;
+  g->lookback = p->lookback;
   g->sort_passes = p->sort_bits <= 8 ? 1 : 2;
   g->sort_digit_bits = (p->sort_bits + g->sort_passes - 1) / g->sort_passes;
   g->sort_bins = 1 << g->sort_digit_bits;

@@ -5,7 +5,8 @@
 // branches can still be mis-scaled"): the sparse branch computes only the
 // selected query-key interactions, exactly, and keeps their mass.  The query at
 // sorted rank r (chunk j = r / chunk) attends the keys at sorted ranks
-// [max(0, (j-1) chunk), (j+1) chunk): O_sp = softmax(s) V, lse = log sum exp(s),
+// [max(0, (j-lb) chunk), (j+1) chunk), lb = 1 on the pages (other lookbacks are
+// an extension this kernel serves): O_sp = softmax(s) V, lse = log sum exp(s),
 // s = scale q . k.  One warp per query: lanes over keys for the scores, lanes
 // over d for the output; results land at the query's token index.
 //
@@ -24,11 +25,11 @@ template <typename T>
 __global__ void __launch_bounds__(128)
 attn_fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                      const int32_t* __restrict__ perm_q, const int32_t* __restrict__ perm_k,
-                     int64_t rows, int N, int d, int chunk, float scale, T* __restrict__ o_sp,
-                     float* __restrict__ lse) {
+                     int64_t rows, int N, int d, int chunk, int lookback, float scale,
+                     T* __restrict__ o_sp, float* __restrict__ lse) {
   extern __shared__ float sm[];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  float* qs = sm + (size_t)w * (d + 2 * chunk);
+  float* qs = sm + (size_t)w * (d + (lookback + 1) * chunk);
   float* ps = qs + d;
   for (int64_t row = (int64_t)blockIdx.x * nw + w; row < rows; row += (int64_t)gridDim.x * nw) {
     const int64_t bh = row / N;
@@ -38,7 +39,7 @@ attn_fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
     for (int e = lane; e < d; e += 32) qs[e] = to_f32(qi[e]);
     __syncwarp();
     const int j = r / chunk;
-    const int lo = max(0, (j - 1) * chunk), nk = (j + 1) * chunk - lo;
+    const int lo = max(0, (j - lookback) * chunk), nk = (j + 1) * chunk - lo;
     const int32_t* pk = perm_k + bh * N + lo;
     float mx = -INFINITY;
     for (int t = lane; t < nk; t += 32) {
@@ -75,14 +76,15 @@ attn_bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
                      const int32_t* __restrict__ perm_q, const int32_t* __restrict__ perm_k,
                      const T* __restrict__ d_o, const float* __restrict__ lse,
                      const float* __restrict__ dprime, int64_t rows, int N, int d, int chunk,
-                     float scale, float* __restrict__ dq_acc, float* __restrict__ dk_acc,
-                     float* __restrict__ dv_acc) {
+                     int lookback, float scale, float* __restrict__ dq_acc,
+                     float* __restrict__ dk_acc, float* __restrict__ dv_acc) {
   extern __shared__ float sm[];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  float* qs = sm + (size_t)w * (2 * d + 4 * chunk);
+  const int win = (lookback + 1) * chunk;
+  float* qs = sm + (size_t)w * (2 * d + 2 * win);
   float* dos = qs + d;
   float* ps = dos + d;
-  float* dss = ps + 2 * chunk;
+  float* dss = ps + win;
   for (int64_t row = (int64_t)blockIdx.x * nw + w; row < rows; row += (int64_t)gridDim.x * nw) {
     const int64_t bh = row / N;
     const int r = (int)(row % N);
@@ -94,7 +96,7 @@ attn_bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
     __syncwarp();
     const float l = lse[bh * N + i], dp_i = dprime[bh * N + i];
     const int j = r / chunk;
-    const int lo = max(0, (j - 1) * chunk), nk = (j + 1) * chunk - lo;
+    const int lo = max(0, (j - lookback) * chunk), nk = (j + 1) * chunk - lo;
     const int32_t* pk = perm_k + bh * N + lo;
     for (int t = lane; t < nk; t += 32) {
       const T* kr = k + (bh * N + pk[t]) * d;
@@ -132,7 +134,7 @@ template <typename T>
 cudaError_t fwd(const Geometry& g, const void* q, const void* k, const void* v,
                 const int32_t* perm_q, const int32_t* perm_k, void* o_sp, float* lse,
                 cudaStream_t s) {
-  const size_t smem = 4 * (size_t)(g.d + 2 * g.chunk) * sizeof(float);
+  const size_t smem = 4 * (size_t)(g.d + (g.lookback + 1) * g.chunk) * sizeof(float);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_simt_kernel<T>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -141,7 +143,7 @@ cudaError_t fwd(const Geometry& g, const void* q, const void* k, const void* v,
   const int64_t rows = (int64_t)g.BH * g.N;
   attn_fwd_simt_kernel<T><<<rows_grid(rows, 4), 128, smem, s>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), perm_q,
-      perm_k, rows, g.N, g.d, g.chunk, g.scale, static_cast<T*>(o_sp), lse);
+      perm_k, rows, g.N, g.d, g.chunk, g.lookback, g.scale, static_cast<T*>(o_sp), lse);
   return cudaGetLastError();
 }
 
@@ -150,7 +152,7 @@ cudaError_t bwd(const Geometry& g, const void* q, const void* k, const void* v,
                 const int32_t* perm_q, const int32_t* perm_k, const void* d_o, const float* lse,
                 const float* dprime, float* dq_acc, float* dk_acc, float* dv_acc,
                 cudaStream_t s) {
-  const size_t smem = 4 * (size_t)(2 * g.d + 4 * g.chunk) * sizeof(float);
+  const size_t smem = 4 * (size_t)(2 * g.d + 2 * (g.lookback + 1) * g.chunk) * sizeof(float);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(attn_bwd_simt_kernel<T>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -159,8 +161,8 @@ cudaError_t bwd(const Geometry& g, const void* q, const void* k, const void* v,
   const int64_t rows = (int64_t)g.BH * g.N;
   attn_bwd_simt_kernel<T><<<rows_grid(rows, 4), 128, smem, s>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), perm_q,
-      perm_k, static_cast<const T*>(d_o), lse, dprime, rows, g.N, g.d, g.chunk, g.scale, dq_acc,
-      dk_acc, dv_acc);
+      perm_k, static_cast<const T*>(d_o), lse, dprime, rows, g.N, g.d, g.chunk, g.lookback,
+      g.scale, dq_acc, dk_acc, dv_acc);
   return cudaGetLastError();
 }
 

@@ -29,6 +29,7 @@ struct Geometry {
   int gate_fixed;      // nonzero: constant gates gate_s, gate_r
   float gate_s, gate_r;
   int sort_order;      // elsaa_sort_order
+  int lookback;        // previous chunks a query chunk attends (1: own and previous)
   int sort_passes, sort_digit_bits, sort_bins, sort_tiles;
   bool tc_hash;       // tcgen05 kernel for the SimHash codes
   bool tc_attn;       // tcgen05 kernels for the sparse branch

@@ -56,6 +56,7 @@ class Workload:
     seed: int = 0
     dist: str = "iid"      # iid | clusters | zipf | needle
     sort_order: str = "binary"   # binary | gray | local (Sort-LSH bucket order)
+    lookback: int = 1            # previous sorted chunks a query chunk attends
 
     @property
     def torch_dtype(self):

@@ -66,11 +66,11 @@ def oracle_unit(w: Workload, inp, b: int, h: int, codes=None, backward=False):
     args = (inp["q"][b, h], inp["k"][b, h], inp["v"][b, h], inp["r_sort"], inp["r_race"],
             w.chunk)
     out = O.forward_head(*args, None, inp["gate_w"], inp["gate_b"], lam, fixed, codes=codes,
-                         sort_order=w.sort_order)
+                         sort_order=w.sort_order, lookback=w.lookback)
     if backward:
         c = codes or {n: out[n] for n in ("code_q", "code_k", "rcode_q", "rcode_k")}
         g = O.grads_head(*args, inp["dy"][b, h], None, inp["gate_w"], inp["gate_b"], lam, fixed,
-                         codes=c, sort_order=w.sort_order)
+                         codes=c, sort_order=w.sort_order, lookback=w.lookback)
         out.update({"grad_" + k: v for k, v in g.items()})
     return out
 

@@ -78,6 +78,8 @@ def test_validation_rejects_bad_problems():
         dict(dtype=7),
         dict(sort_order=3),
         dict(sort_order=-1),
+        dict(lookback=-1),
+        dict(lookback=65),
     ]
     for c in cases:
         p = B.Params.make(1, 2, 256, 64, "bf16", 4, 64, 8, 6)
@@ -89,6 +91,11 @@ def test_validation_rejects_bad_problems():
     assert B.validate(p) == 2
     for order in B.SORT_ORDERS:
         assert B.validate(B.Params.make(1, 2, 256, 64, "bf16", 4, 64, 8, 6, sort_order=order)) == 0
+    for lb in (0, 1, 3):
+        assert B.validate(B.Params.make(1, 2, 256, 64, "bf16", 4, 64, 8, 6, lookback=lb)) == 0
+    # the CUDA-core attention keeps (lookback + 1) chunk scores per query in shared memory
+    p = B.Params.make(1, 2, 8192, 64, "bf16", 4, 1024, 8, 6, lookback=6)
+    assert B.validate(p) == 2
 
 
 def test_null_pointers_are_rejected_before_any_launch():

@@ -79,6 +79,13 @@ def test_sort_orders(cuda_device, order, sort_bits):
     _run(w, backward=True)
 
 
+@pytest.mark.parametrize("lookback,dtype", [(0, "bf16"), (2, "bf16"), (3, "f32")])
+def test_lookback(cuda_device, lookback, dtype):
+    # windows of lookback previous chunks plus the own one (CUDA-core attention)
+    w = WORKLOADS["iid-4k"].replace(B=1, H=2, N=512, chunk=32, lookback=lookback, dtype=dtype)
+    _run(w, backward=True)
+
+
 def test_two_pass_sort_and_wide_race_codes(cuda_device):
     # 12 sort bits take two radix passes; 11 RACE bits give uint16 codes and
     # 2048-bucket tables (the global-atomic build)
