@@ -28,12 +28,16 @@
 //               query blocks (two-slot ring), with the blocks' lse, D' and
 //               (da_s, da_r) by cp.async
 //   warp 1      MMA issuer (one thread) and TMEM owner; for pair p it issues
-//               S^T/dP^T of pair p + 1 as soon as P^T/dS^T of pair p are in
-//               shared memory, then dV, dK, dQ of pair p
+//               S^T/dP^T of pair p + 1 as soon as the elementwise warps have
+//               read S^T/dP^T of pair p out of TMEM (s_free), then, once P^T
+//               and dS^T of pair p are in shared memory (p_full), dV of pair p
+//               (its completion frees P^T: pt_free) and dK, dQ (pd_free)
 //   warps 2..9  elementwise: warp w reaches TMEM lanes 32 (w % 4) .. +31 and
-//               takes half of the query columns; P^T and dS^T (bf16) to
-//               shared memory, one 32-column chunk at a time; they also stage
-//               the token indices (and gate pairs) the epilogue needs
+//               takes half of the query columns, read in 16-column chunks with
+//               the next chunk's load in flight; P^T (bf16) goes to shared
+//               memory chunk by chunk after pt_free of the previous pair, dS^T
+//               is held in registers and stored after its pd_free; they also
+//               stage the token indices (and gate pairs) the epilogue needs
 //   warps 10-13 epilogue: a finished query block's dQ (+ gate part) and a
 //               finished key tile's dV and dK from TMEM to bf16 rows; TMEM is
 //               released as soon as it has been read, before the stores
