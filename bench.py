@@ -110,7 +110,7 @@ def stage_roofline(flops, nbytes, sec, peaks):
 # workload by the number of units; reported only while that file is unchanged.
 RECORDED_TRAFFIC = {
     # stage: (kernel source, its sha1 at capture, bytes per full-size launch)
-    "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "69efc768d31fb28fcd4a8ec01551bf7466f6ee92", 2.459e+08),
+    "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "e64b5b0853a47abfb13af9aec16cec6b49568584", 2.459e+08),
     "race_build": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "9ff8ca9fd3724573a561d5ad5f1319a4dafe1fd0", 1.372e+08),
     "sparse_fwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_pipe.cu", "91a31d0c88874e37ef33ed4bb443baabc0c07369", 3.735e+08),
     "race_fuse": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "9ff8ca9fd3724573a561d5ad5f1319a4dafe1fd0", 3.717e+08),

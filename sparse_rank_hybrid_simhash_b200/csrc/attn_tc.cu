@@ -137,7 +137,10 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
     const uint32_t slot = (b & 1) * Lay::kSub * Lay::kSubBytes;
     if (b >= 1) {
       ok = mbar_wait(bar_o, (b - 1) & 1, err);
-      if (__syncthreads_or(!ok)) break;
+      if (__syncthreads_or(!ok)) {  // every thread leaves with ok false
+        ok = false;
+        break;
+      }
       fence_after();
     }
     if (b >= 2) {
@@ -164,7 +167,10 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
       mma_commit(bar_s);
     }
     ok = mbar_wait(bar_s, b & 1, err);
-    if (__syncthreads_or(!ok)) break;
+    if (__syncthreads_or(!ok)) {  // every thread leaves with ok false
+      ok = false;
+      break;
+    }
     fence_after();
     // online softmax over this block, row t of TMEM lane t
     const int c_lo = lo - b * kKB, c_hi = min(hi - b * kKB, nb);

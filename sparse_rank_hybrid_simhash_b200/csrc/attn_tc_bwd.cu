@@ -170,7 +170,10 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
       mma_commit(bar_a);
     }
     ok = mbar_wait(bar_a, b & 1, err);
-    if (__syncthreads_or(!ok)) break;
+    if (__syncthreads_or(!ok)) {  // every thread leaves with ok false
+      ok = false;
+      break;
+    }
     fence_after();
     // P^T and dS^T rows of this thread's key; a query in chunk jq sees this key
     // iff jq - key_chunk is 0 or 1
@@ -234,7 +237,10 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
       mma_commit(bar_b);
     }
     ok = mbar_wait(bar_b, b & 1, err);
-    if (__syncthreads_or(!ok)) break;
+    if (__syncthreads_or(!ok)) {  // every thread leaves with ok false
+      ok = false;
+      break;
+    }
     fence_after();
     // dQ rows of this block: TMEM lane t = query qb0 + t.  Stage them in shared
     // memory (16-byte chunk c of row t at chunk position (c + t) mod D/4, so

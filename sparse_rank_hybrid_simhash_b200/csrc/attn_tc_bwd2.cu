@@ -174,7 +174,10 @@ attn_bwd2_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
   for (int b = 0; b < nqb; ++b) {
     const int qb0 = k0 + b * kTile, nq = min(kTile, qend - qb0), buf = b & 1;
     ok = mbar_wait(bar_s, b & 1, err);
-    if (__syncthreads_or(!ok)) break;
+    if (__syncthreads_or(!ok)) {  // every thread leaves with ok false
+      ok = false;
+      break;
+    }
     fence_after();
     // P^T and dS^T: this thread's key row, half of the query columns
     {
@@ -239,7 +242,10 @@ attn_bwd2_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
       if (b + 1 < nqb) issue_sdp(b + 1);
     }
     ok = mbar_wait(bar_g, b & 1, err);
-    if (__syncthreads_or(!ok)) break;
+    if (__syncthreads_or(!ok)) {  // every thread leaves with ok false
+      ok = false;
+      break;
+    }
     fence_after();
     // dQ of block b: TMEM lane = query row, this warp's 32 columns; staged with
     // chunk c of row r at position (c + r) mod 16 so neither pass conflicts

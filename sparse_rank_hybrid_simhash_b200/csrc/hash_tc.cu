@@ -197,7 +197,10 @@ hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
       ok = mbar_wait(bar, phase & 1, err);
       ++phase;
-      if (__syncthreads_or(!ok)) break;
+      if (__syncthreads_or(!ok)) {  // every thread leaves with ok false
+        ok = false;
+        break;
+      }
       fence_after();
       for (int c0 = 0; c0 < ncol; c0 += 32) {
         const int w = (p * kPass + c0) >> 5;
@@ -388,7 +391,10 @@ hash_tc_stream_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
       }
       ok = mbar_wait(bar, phase & 1, err);
       ++phase;
-      if (__syncthreads_or(!ok)) break;
+      if (__syncthreads_or(!ok)) {  // every thread leaves with ok false
+        ok = false;
+        break;
+      }
       fence_after();
       for (int c0 = 0; c0 < ncol; c0 += 32) {
         const int valid = min(32, P - (p * kPass + c0));
