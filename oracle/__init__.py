@@ -28,6 +28,9 @@ Parity status of each function (what pins it, see ``tests/test_oracle.py``):
   race_build / race_query
                        pinned: per-table sums, K_r = 0 closed form, collision
                        count matrix brute force
+  race_query_causal    pinned: pure-Python loop over (query, table, key j <= i),
+                       last token equals the full read-out, causal dense
+                       identities through forward_head
   gates / fuse         pinned: lambda = 0 ablation (m == 1), single-branch gate
                        settings, Z_race = 0, closed form for Q = 0
   forward_head         pinned through the pieces above and the Q = 0 closed form
@@ -48,6 +51,7 @@ from .elsaa_oracle import (  # noqa: F401
     sparse_branch,
     race_build,
     race_query,
+    race_query_causal,
     gates,
     fuse,
     forward_head,

@@ -123,20 +123,37 @@ def chunk_window(rank: int, chunk: int, lookback: int = 1) -> tuple:
 # Step 3: exact sparse branch
 # ---------------------------------------------------------------------------
 
-def sparse_branch(q, k, v, perm_q, perm_k, chunk: int, scale: float, lookback: int = 1):
+def sparse_branch(q, k, v, perm_q, perm_k, chunk: int, scale: float, lookback: int = 1,
+                  causal: bool = False):
     """Exact softmax attention restricted to the Sort-LSH window ("Two
     Efficient Attentions, One Denominator Problem", section "Two efficient
     branches can still be mis-scaled": the sparse branch computes only the
     selected interactions, exactly).  Returns (O_sp [N, d], lse [N]) in token
-    order; Z_sp = exp(lse) is the unshifted attention mass of the window."""
+    order; Z_sp = exp(lse) is the unshifted attention mass of the window.
+
+    ``causal`` (an extension: the pages note that causal use was not
+    evaluated) keeps only the keys of the window whose token index is at most
+    the query's; a query with no such key gets O_sp = 0 and lse = -inf
+    (Z_sp = 0)."""
     n = q.shape[0]
     qs, ks, vs = q[perm_q], k[perm_k], v[perm_k]
     outs, lses = [], []
     for j in range(n // chunk):
         lo, hi = chunk_window(j * chunk, chunk, lookback)
         s = scale * (qs[j * chunk:(j + 1) * chunk] @ ks[lo:hi].T)
-        lses.append(torch.logsumexp(s, dim=1))
-        outs.append(torch.softmax(s, dim=1) @ vs[lo:hi])
+        if not causal:
+            lses.append(torch.logsumexp(s, dim=1))
+            outs.append(torch.softmax(s, dim=1) @ vs[lo:hi])
+            continue
+        allowed = perm_k[lo:hi][None, :] <= perm_q[j * chunk:(j + 1) * chunk][:, None]
+        has = allowed.any(dim=1)
+        # rows without a key take finite stand-in scores so that no NaN
+        # reaches the gradients; their results are replaced below
+        s = torch.where(allowed | ~has[:, None], s, torch.full_like(s, float("-inf")))
+        lse_j = torch.logsumexp(s, dim=1)
+        o_j = torch.softmax(s, dim=1) @ vs[lo:hi]
+        lses.append(torch.where(has, lse_j, torch.full_like(lse_j, float("-inf"))))
+        outs.append(torch.where(has[:, None], o_j, torch.zeros_like(o_j)))
     o_sorted = torch.cat(outs, 0)
     lse_sorted = torch.cat(lses, 0)
     inv = torch.empty_like(perm_q)
@@ -160,6 +177,28 @@ def race_build(rcode_k: torch.Tensor, v: torch.Tensor, nbuckets: int):
         torch.zeros(nbuckets, d, dtype=F64).index_add(0, rcode_k[:, l], v) for l in range(L)
     ])
     return counts, sums
+
+
+def race_query_causal(rcode_q: torch.Tensor, rcode_k: torch.Tensor, v: torch.Tensor):
+    """Causal RACE read-out (an extension): query i reads, in every table, only
+    the keys j <= i of its bucket: Ctot_i = sum_l #{j <= i : h_l(k_j) = h_l(q_i)},
+    O_race_i = sum of those keys' values / Ctot_i (0 when Ctot_i = 0),
+    Z_race_i = Ctot_i / L.  Written as the collision-count matrix restricted to
+    j <= i, a block of queries at a time.  Returns (Ctot, O_race, Z_race)."""
+    n, L = rcode_q.shape
+    ctot = torch.zeros(n, dtype=torch.int64)
+    num = torch.zeros(n, v.shape[1], dtype=F64)
+    for a in range(0, n, 512):
+        b = min(n, a + 512)
+        cnt = torch.zeros(b - a, n, dtype=torch.int64)
+        for l in range(L):
+            cnt += (rcode_q[a:b, l][:, None] == rcode_k[:, l][None, :]).to(torch.int64)
+        cnt *= (torch.arange(n)[None, :] <= torch.arange(a, b)[:, None]).to(torch.int64)
+        ctot[a:b] = cnt.sum(dim=1)
+        num[a:b] = cnt.to(F64) @ v
+    safe = torch.where(ctot > 0, ctot, torch.ones_like(ctot)).to(F64)
+    o_race = torch.where((ctot > 0)[:, None], num / safe[:, None], torch.zeros_like(num))
+    return ctot, o_race, ctot.to(F64) / L
 
 
 def race_query(rcode_q: torch.Tensor, counts: torch.Tensor, sums: torch.Tensor):
@@ -200,7 +239,11 @@ def fuse(o_sp, lse, o_race, z_race, g_s, g_r, lam):
     independently: y = g_s * m * O_sp + g_r * O_race.  With lambda = 0 the
     multiplier is one (the Sort_Lsh_RACE ablation)."""
     z_sp = torch.exp(lse)
-    m = z_sp / (z_sp + lam * z_race)
+    den = z_sp + lam * z_race
+    # m = 1 where both masses vanish (only a causal window can have Z_sp = 0);
+    # the safe denominator keeps NaN out of the unused branch's gradient
+    safe = torch.where(den > 0, den, torch.ones_like(den))
+    m = torch.where(den > 0, z_sp / safe, torch.ones_like(den))
     y = g_s[:, None] * m[:, None] * o_sp + g_r[:, None] * o_race
     return y, m
 
@@ -222,7 +265,8 @@ def _hash_all(q64, k64, r_sort, r_race):
 def forward_head(q, k, v, r_sort, r_race, chunk: int, scale: Optional[float] = None,
                  gate_w=None, gate_b=None, lam=1.0, fixed_gates: Optional[tuple] = None,
                  codes: Optional[Dict[str, torch.Tensor]] = None,
-                 sort_order: str = "binary", lookback: int = 1) -> Dict[str, torch.Tensor]:
+                 sort_order: str = "binary", lookback: int = 1,
+                 causal: bool = False) -> Dict[str, torch.Tensor]:
     """The whole operator on one (batch, head) unit.
 
     q, k, v: [N, d] (any float dtype; upcast to fp64).  r_sort: [b_s, d];
@@ -251,9 +295,12 @@ def forward_head(q, k, v, r_sort, r_race, chunk: int, scale: Optional[float] = N
         rcode_q, rcode_k = codes["rcode_q"].to(torch.int64), codes["rcode_k"].to(torch.int64)
     perm_q = stable_sort_perm(sort_keys(code_q, sort_order))
     perm_k = stable_sort_perm(sort_keys(code_k, sort_order))
-    o_sp, lse = sparse_branch(q64, k64, v64, perm_q, perm_k, chunk, scale, lookback)
+    o_sp, lse = sparse_branch(q64, k64, v64, perm_q, perm_k, chunk, scale, lookback, causal)
     counts, sums = race_build(rcode_k, v64, 1 << kr)
-    ctot, o_race, z_race = race_query(rcode_q, counts, sums)
+    if causal:
+        ctot, o_race, z_race = race_query_causal(rcode_q, rcode_k, v64)
+    else:
+        ctot, o_race, z_race = race_query(rcode_q, counts, sums)
     if fixed_gates is None:
         g_s, g_r = gates(q64, gate_w.to(F64), gate_b.to(F64))
     else:
@@ -269,7 +316,8 @@ def forward_head(q, k, v, r_sort, r_race, chunk: int, scale: Optional[float] = N
 def grads_head(q, k, v, r_sort, r_race, chunk: int, dy, scale: Optional[float] = None,
                gate_w=None, gate_b=None, lam=1.0, fixed_gates: Optional[tuple] = None,
                codes: Optional[Dict[str, torch.Tensor]] = None,
-               sort_order: str = "binary", lookback: int = 1) -> Dict[str, torch.Tensor]:
+               sort_order: str = "binary", lookback: int = 1,
+               causal: bool = False) -> Dict[str, torch.Tensor]:
     """Gradients of sum(y * dy) with the hash codes held constant (codes are
     piecewise constant in q and k), by fp64 autograd through forward_head.
     The pages state that ELSAA is used in training ("ELSAA combines sparsity
@@ -288,10 +336,12 @@ def grads_head(q, k, v, r_sort, r_race, chunk: int, dy, scale: Optional[float] =
         leaves += [gw, gb]
     if codes is None:
         first = forward_head(q, k, v, r_sort, r_race, chunk, scale, gate_w, gate_b, lam,
-                             fixed_gates, sort_order=sort_order, lookback=lookback)
+                             fixed_gates, sort_order=sort_order, lookback=lookback,
+                             causal=causal)
         codes = {name: first[name] for name in ("code_q", "code_k", "rcode_q", "rcode_k")}
     out = forward_head(q64, k64, v64, r_sort, r_race, chunk, scale, gw, gb, lam64,
-                       fixed_gates, codes=codes, sort_order=sort_order, lookback=lookback)
+                       fixed_gates, codes=codes, sort_order=sort_order, lookback=lookback,
+                       causal=causal)
     loss = (out["y"] * dy.to(F64)).sum()
     g = torch.autograd.grad(loss, leaves, allow_unused=True)
     res = {"dq": g[0], "dk": g[1], "dv": g[2], "dlambda": g[3]}

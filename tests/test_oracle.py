@@ -445,3 +445,101 @@ def test_lookback_zero_with_one_chunk_is_dense_attention():
     o, _ = O.sparse_branch(q, k, v, pq, pk, n, 0.7, 0)
     ref = torch.nn.functional.scaled_dot_product_attention(q[None], k[None], v[None], scale=0.7)[0]
     assert torch.allclose(o, ref, atol=1e-12, rtol=0)
+
+
+# ---------------------------------------------------------------------------
+# causal ELSAA (an extension: keys j <= i only, in both branches)
+# ---------------------------------------------------------------------------
+
+def test_causal_one_local_chunk_is_causal_dense_attention():
+    n, d = 20, 6
+    q, k, v = rnd((n, d), 80), rnd((n, d), 81), rnd((n, d), 82)
+    perm = torch.arange(n)
+    o, lse = O.sparse_branch(q, k, v, perm, perm, n, 0.6, 0, causal=True)
+    ref = torch.nn.functional.scaled_dot_product_attention(q[None], k[None], v[None],
+                                                           is_causal=True, scale=0.6)[0]
+    assert torch.allclose(o, ref, atol=1e-12, rtol=0)
+    s = (0.6 * q @ k.T).masked_fill(torch.ones(n, n, dtype=torch.bool).triu(1), float("-inf"))
+    assert torch.allclose(lse, torch.logsumexp(s, 1), atol=1e-12, rtol=0)
+
+
+def test_causal_window_brute_force_and_empty_windows():
+    n, d, c = 32, 5, 8
+    q, k, v = rnd((n, d), 83), rnd((n, d), 84), rnd((n, d), 85)
+    pq = torch.randperm(n, generator=torch.Generator().manual_seed(86))
+    pk = torch.arange(n).flip(0)   # late keys first: early queries find no earlier key
+    o, lse = O.sparse_branch(q, k, v, pq, pk, c, 0.5, 1, causal=True)
+    rank_q = {int(t): r for r, t in enumerate(pq)}
+    rank_k = {int(t): r for r, t in enumerate(pk)}
+    empty = 0
+    for i in range(n):
+        keys = [j for j in range(n)
+                if rank_q[i] // c - 1 <= rank_k[j] // c <= rank_q[i] // c and j <= i]
+        if not keys:
+            empty += 1
+            assert float(lse[i]) == float("-inf") and torch.all(o[i] == 0)
+            continue
+        s = torch.stack([0.5 * q[i] @ k[j] for j in keys])
+        p = torch.softmax(s, 0)
+        assert abs(float(lse[i]) - float(torch.logsumexp(s, 0))) < 1e-12
+        assert torch.allclose(o[i], sum(p[t] * v[j] for t, j in enumerate(keys)), atol=1e-12)
+    assert empty > 0
+    # gradients stay finite through the empty windows
+    qg, kg, vg = (t.clone().requires_grad_(True) for t in (q, k, v))
+    og, lg = O.sparse_branch(qg, kg, vg, pq, pk, c, 0.5, 1, causal=True)
+    (og.sum() + lg[torch.isfinite(lg)].sum()).backward()
+    assert all(torch.isfinite(t.grad).all() for t in (qg, kg, vg))
+
+
+def test_causal_race_brute_force():
+    n, L, nb, d = 24, 3, 4, 3
+    g = torch.Generator().manual_seed(87)
+    rq = torch.randint(0, nb, (n, L), generator=g)
+    rk = torch.randint(0, nb, (n, L), generator=g)
+    v = rnd((n, d), 88)
+    ctot, o_race, z_race = O.race_query_causal(rq, rk, v)
+    for i in range(n):
+        cnt, num = 0, torch.zeros(d, dtype=F64)
+        for l in range(L):
+            for j in range(i + 1):
+                if int(rq[i, l]) == int(rk[j, l]):
+                    cnt += 1
+                    num += v[j]
+        assert int(ctot[i]) == cnt
+        assert abs(float(z_race[i]) - cnt / L) < 1e-15
+        assert torch.allclose(o_race[i], num / cnt if cnt else num, atol=1e-12)
+    # the last token sees every key: the full read-out
+    counts, sums = O.race_build(rk, v, nb)
+    c_full, o_full, _ = O.race_query(rq, counts, sums)
+    assert int(ctot[-1]) == int(c_full[-1])
+    assert torch.allclose(o_race[-1], o_full[-1], atol=1e-12)
+
+
+def test_fusion_with_an_empty_causal_window():
+    n, d = 3, 2
+    o_sp = torch.zeros(n, d, dtype=F64)
+    lse = torch.full((n,), float("-inf"), dtype=F64)
+    o_race = rnd((n, d), 89)
+    z_race = torch.tensor([2.0, 0.0, 1.0], dtype=F64)
+    g_s, g_r = torch.full((n,), 0.4, dtype=F64), torch.full((n,), 0.7, dtype=F64)
+    y, m = O.fuse(o_sp, lse, o_race, z_race, g_s, g_r, 1.0)
+    assert m.tolist() == [0.0, 1.0, 0.0]   # Z_sp = 0: m = 0, or 1 where both masses vanish
+    assert torch.allclose(y, 0.7 * o_race, atol=1e-15)
+
+
+def test_causal_gradients_match_finite_differences():
+    n, d, c, L, kr = 12, 4, 4, 2, 2
+    q, k, v, rs, rr, gw, gb = _unit(n, d, c, 2, L, kr, seed=90)
+    first = O.forward_head(q, k, v, rs, rr, c, None, gw, gb, 0.7, causal=True)
+    codes = {x: first[x] for x in ("code_q", "code_k", "rcode_q", "rcode_k")}
+    dy = rnd((n, d), 91)
+
+    def f(q_, k_, v_, w_, b_, lam_):
+        return O.forward_head(q_, k_, v_, rs, rr, c, None, w_, b_, lam_, codes=codes,
+                              causal=True)["y"]
+
+    args = tuple(t.clone().requires_grad_(True) for t in (q, k, v, gw, gb))
+    lam = torch.tensor(0.7, dtype=F64, requires_grad=True)
+    assert torch.autograd.gradcheck(f, args + (lam,), eps=1e-6, atol=1e-7)
+    g = O.grads_head(q, k, v, rs, rr, c, dy, None, gw, gb, 0.7, codes=codes, causal=True)
+    assert all(torch.isfinite(g[x]).all() for x in ("dq", "dk", "dv", "dlambda"))
