@@ -272,6 +272,7 @@ def bench_config(w, mode, world, l2):
     """The config object of a bench line (both arms)."""
     return {"workload": w.name, "mode": mode, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
             "sort_bits": w.sort_bits, "sort_order": w.sort_order, "lookback": w.lookback,
+            "causal": w.causal,
             "chunk": w.chunk,
             "race_tables": w.race_tables,
             "race_bits": w.race_bits,
@@ -329,7 +330,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = apply_mode(WORKLOADS[args.workload], args.mode).replace(
-        sort_order=args.sort_order, lookback=args.lookback)
+        sort_order=args.sort_order, lookback=args.lookback, causal=args.causal)
     p = B.Params.from_workload(w)
     inp = make_inputs(w, seed=DP.rank_seed(w.seed, rank), with_dy=True)
     d = {k: t.to(dev) for k, t in inp.items()}
@@ -477,7 +478,7 @@ def run_reference(args):
     if rank != 0:
         return
     w = apply_mode(WORKLOADS[args.workload], args.mode).replace(
-        sort_order=args.sort_order, lookback=args.lookback)
+        sort_order=args.sort_order, lookback=args.lookback, causal=args.causal)
     cores = len(os.sched_getaffinity(0))
     torch.set_num_threads(cores)
     inp = make_inputs(w, with_dy=True)
@@ -524,6 +525,8 @@ def main():
                     help="Sort-LSH chunk order: code value, Gray sequence, or token order")
     ap.add_argument("--lookback", type=int, default=1,
                     help="previous sorted chunks a query chunk attends (1: own and previous)")
+    ap.add_argument("--causal", action="store_true",
+                    help="keys j <= i only (CUDA-core attention, RACE token scans)")
     ap.add_argument("--dense-context", action="store_true",
                     help="also time dense torch SDPA fwd+bwd on the same inputs (context)")
     ap.add_argument("--batch", type=int, default=None,

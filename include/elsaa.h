@@ -89,6 +89,12 @@ typedef struct {
                            * 0..64 with (lookback + 1) * chunk <= 6144: 1 is the pages'
                            * Sort-LSH (own and previous chunk); other values are an
                            * extension served by the CUDA-core attention kernels */
+  int32_t causal;         /* nonzero: query i sees only keys j <= i (token index), in the
+                           * sparse window and in the RACE read-out (an extension: the
+                           * pages did not evaluate causal use); a window left without
+                           * keys has Z_sp = 0 (O_sp = 0, lse = -inf).  Runs on the
+                           * CUDA-core attention and a per-table token scan for RACE;
+                           * needs 2^race_bits * (d + 1) * 4 <= 200 KB */
 } elsaa_params;
 
 /* Device views into a forward's saved state (see elsaa_saved_views). */

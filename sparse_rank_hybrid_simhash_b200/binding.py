@@ -38,22 +38,22 @@ class Params(ctypes.Structure):
                 ("race_bits", ctypes.c_int32), ("scale", ctypes.c_float),
                 ("gate_fixed", ctypes.c_int32), ("gate_s", ctypes.c_float),
                 ("gate_r", ctypes.c_float), ("sort_order", ctypes.c_int32),
-                ("lookback", ctypes.c_int32)]
+                ("lookback", ctypes.c_int32), ("causal", ctypes.c_int32)]
 
     @classmethod
     def make(cls, B, H, N, d, dtype, sort_bits, chunk, race_tables, race_bits, scale=0.0,
              gate_fixed=False, gate_s=0.5, gate_r=0.5, sort_order="binary",
-             lookback=1) -> "Params":
+             lookback=1, causal=False) -> "Params":
         dt = ELSAA_BF16 if dtype in ("bf16", torch.bfloat16) else ELSAA_F32
         return cls(B, H, N, d, dt, sort_bits, chunk, race_tables, race_bits, float(scale),
                    int(bool(gate_fixed)), float(gate_s), float(gate_r), SORT_ORDERS[sort_order],
-                   int(lookback))
+                   int(lookback), int(bool(causal)))
 
     @classmethod
     def from_workload(cls, w) -> "Params":
         return cls.make(w.B, w.H, w.N, w.d, w.dtype, w.sort_bits, w.chunk, w.race_tables,
                         w.race_bits, 0.0, w.gate_fixed, w.gate_s, w.gate_r, w.sort_order,
-                        w.lookback)
+                        w.lookback, w.causal)
 
     @property
     def torch_dtype(self):

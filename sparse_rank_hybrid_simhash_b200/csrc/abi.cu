@@ -19,6 +19,7 @@ bool make_geometry(const elsaa_params* p, Geometry* g, elsaa_status* why) {
       p->sort_order != ELSAA_SORT_LOCAL)
     return false;
   if (p->lookback < 0 || p->lookback > 64) return false;
+  if (p->causal != 0 && p->causal != 1) return false;
   if (p->race_tables < 1 || p->race_tables > 4096) return false;
   if (p->race_bits < 0 || p->race_bits > 16) return false;
   if ((int64_t)p->B * p->H * p->N * (p->d > p->race_tables ? p->d : p->race_tables) >
@@ -47,12 +48,14 @@ bool make_geometry(const elsaa_params* p, Geometry* g, elsaa_status* why) {
   g->gate_r = p->gate_r;
   g->sort_order = p->sort_order;
   g->lookback = p->lookback;
+  g->causal = p->causal;
   g->sort_passes = p->sort_bits <= 8 ? 1 : 2;
   g->sort_digit_bits = (p->sort_bits + g->sort_passes - 1) / g->sort_passes;
   g->sort_bins = 1 << g->sort_digit_bits;
   g->sort_tiles = (p->N + kSortTile - 1) / kSortTile;
   g->tc_hash = hash_tc_supported(*g);
   g->tc_attn = attn_tc_supported(*g);
+  if (g->causal && !race_causal_supported(*g)) return false;
   *why = ELSAA_OK;
   return true;
 }
@@ -86,6 +89,7 @@ WorkLayout work_layout(const Geometry& g) {
   w.sort_tmp = take(2 * bhn * 4);
   w.absmax = take((size_t)2 * g.BH * 4);
   w.gtab = take((size_t)g.BH * g.L * g.NB * g.d * 2);
+  w.causal_num = take(g.causal ? bhn * g.d * 4 : 0);
   const size_t shared_base = off;
   // forward without a saved buffer: the saved layout lives here
   w.saved = take(saved_layout(g).total);
@@ -224,6 +228,20 @@ elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const vo
   ELSAA_TRY(launch_sort(g, code, perm, (int32_t*)(w + wl.sort_hist), (int32_t*)(w + wl.sort_tmp),
                         s));
   ELSAA_TRY(mark(events, 2, s));
+  if (g.causal) {
+    // causal: the RACE read-out of query i takes keys j <= i only (a token
+    // scan per table), the sparse window likewise
+    float* num = (float*)(w + wl.causal_num);
+    int32_t* ct = (int32_t*)(sv + sl.ctot);
+    ELSAA_TRY(mark(events, 3, s));   // (no separate build stage)
+    ELSAA_TRY(launch_race_causal_fwd(g, rcode, rcode_k, v, num, ct, sums, counts, s));
+    ELSAA_TRY(launch_attn_fwd_simt(g, q, k, v, perm, perm + bhn, o_sp, lse, s));
+    ELSAA_TRY(mark(events, 4, s));
+    ELSAA_TRY(launch_fuse_causal(g, q, o_sp, lse, num, ct, gate_w, gate_b, lambda, y,
+                                 sv + sl.o_race, s));
+    ELSAA_TRY(mark(events, 5, s));
+    return ELSAA_OK;
+  }
   // 3. RACE tables from the keys
   float* absmax = (float*)(w + wl.absmax);
   ELSAA_TRY(launch_unit_absmax(g, v, false, absmax, s));
@@ -314,10 +332,16 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
                             absmax, partials, s));
   ELSAA_TRY(mark(events, 1, s));
   // 2. RACE backward: scatter into the table gradient by query code (and, off
-  // the direct path, gather by key code into dv_acc)
-  ELSAA_TRY(launch_race_build(g, rcode, rcode_t, dor, false, absmax, d_t, !g.bf16, gtab, nullptr,
-                              (uint32_t*)(w + wl.err), s));
-  if (!direct) ELSAA_TRY(launch_race_gather_sum(g, rcode_k, race_grad, dv_acc, s));
+  // the direct path, gather by key code into dv_acc); causal: one reverse
+  // token scan per table straight into dv_acc
+  if (g.causal) {
+    ELSAA_TRY(cudaMemsetAsync(dv_acc, 0, bhn * g.d * 4, s));
+    ELSAA_TRY(launch_race_causal_bwd(g, rcode, rcode_k, dor, dv_acc, s));
+  } else {
+    ELSAA_TRY(launch_race_build(g, rcode, rcode_t, dor, false, absmax, d_t, !g.bf16, gtab,
+                                nullptr, (uint32_t*)(w + wl.err), s));
+    if (!direct) ELSAA_TRY(launch_race_gather_sum(g, rcode_k, race_grad, dv_acc, s));
+  }
   ELSAA_TRY(mark(events, 2, s));
   // 3. sparse branch backward, 4. outputs
   if (direct) {
@@ -366,12 +390,15 @@ elsaa_status elsaa_kernel_launches(const elsaa_params* p, int32_t* fwd, int32_t*
   if (!make_geometry(p, &g, &why)) return why;
   if (!fwd || !bwd) return ELSAA_ERR_INVALID_ARG;
   // hash 1, sort 3 per pass, |V| max 1 + RACE build 1, sparse 1, RACE gather + fusion 1
-  *fwd = 1 + 3 * g.sort_passes + 2 + 1 + 1;
+  // (local order: one kernel writes token order instead of the radix passes;
+  // causal: one RACE token scan, then the sparse branch and the fusion)
+  const int sort = g.sort_order == ELSAA_SORT_LOCAL ? 1 : 3 * g.sort_passes;
+  *fwd = g.causal ? 1 + sort + 1 + 1 + 1 : 1 + sort + 2 + 1 + 1;
   // fusion backward 1, RACE build 1 + gather 1, sparse 1 (+ casts), reduction 1
   // (direct path: the sparse kernel writes dq itself and the gather adds into dv)
   const bool direct = g.tc_attn && attn_bwd3_supported(g) && race_gather_add_supported(g);
   const int sparse = direct ? 1 : g.tc_attn ? 1 + 1 : 1 + 3;
-  *bwd = 1 + 2 + sparse + 1;
+  *bwd = 1 + (g.causal ? 1 : 2) + sparse + 1;
   return ELSAA_OK;
 }
 

@@ -8,7 +8,9 @@
 // [max(0, (j-lb) chunk), (j+1) chunk), lb = 1 on the pages (other lookbacks are
 // an extension this kernel serves): O_sp = softmax(s) V, lse = log sum exp(s),
 // s = scale q . k.  One warp per query: lanes over keys for the scores, lanes
-// over d for the output; results land at the query's token index.
+// over d for the output; results land at the query's token index.  Causal
+// (an extension): keys whose token index exceeds the query's are left out; a
+// query left with no key gets O_sp = 0 and lse = -inf.
 //
 // Backward (one warp per query, keys' gradients by fp32 atomics):
 //   p = exp(s - lse), dP = dO . v, dS = p (dP - D'),  D' = dO . O - dlse,
@@ -25,8 +27,8 @@ template <typename T>
 __global__ void __launch_bounds__(128)
 attn_fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                      const int32_t* __restrict__ perm_q, const int32_t* __restrict__ perm_k,
-                     int64_t rows, int N, int d, int chunk, int lookback, float scale,
-                     T* __restrict__ o_sp, float* __restrict__ lse) {
+                     int64_t rows, int N, int d, int chunk, int lookback, int causal,
+                     float scale, T* __restrict__ o_sp, float* __restrict__ lse) {
   extern __shared__ float sm[];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   float* qs = sm + (size_t)w * (d + (lookback + 1) * chunk);
@@ -43,29 +45,33 @@ attn_fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
     const int32_t* pk = perm_k + bh * N + lo;
     float mx = -INFINITY;
     for (int t = lane; t < nk; t += 32) {
-      const T* kr = k + (bh * N + pk[t]) * d;
-      float s = 0.f;
-      for (int e = 0; e < d; ++e) s += qs[e] * to_f32(kr[e]);
-      s *= scale;
+      float s = -INFINITY;
+      if (!causal || pk[t] <= i) {
+        const T* kr = k + (bh * N + pk[t]) * d;
+        s = 0.f;
+        for (int e = 0; e < d; ++e) s += qs[e] * to_f32(kr[e]);
+        s *= scale;
+      }
       ps[t] = s;
       mx = fmaxf(mx, s);
     }
     mx = warp_max(mx);
+    const bool any = mx > -INFINITY;   // false only for a causal window without keys
     float sum = 0.f;
     for (int t = lane; t < nk; t += 32) {
-      const float p = expf(ps[t] - mx);
+      const float p = any ? expf(ps[t] - mx) : 0.f;
       ps[t] = p;
       sum += p;
     }
     sum = warp_sum(sum);
     __syncwarp();
-    const float inv = 1.0f / sum;
+    const float inv = any ? 1.0f / sum : 0.f;
     for (int e = lane; e < d; e += 32) {
       float o = 0.f;
       for (int t = 0; t < nk; ++t) o += ps[t] * to_f32(v[(bh * N + pk[t]) * d + e]);
       o_sp[(bh * N + i) * d + e] = from_f32<T>(o * inv);
     }
-    if (lane == 0) lse[bh * N + i] = mx + logf(sum);
+    if (lane == 0) lse[bh * N + i] = any ? mx + logf(sum) : -INFINITY;
     __syncwarp();
   }
 }
@@ -76,7 +82,7 @@ attn_bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
                      const int32_t* __restrict__ perm_q, const int32_t* __restrict__ perm_k,
                      const T* __restrict__ d_o, const float* __restrict__ lse,
                      const float* __restrict__ dprime, int64_t rows, int N, int d, int chunk,
-                     int lookback, float scale, float* __restrict__ dq_acc,
+                     int lookback, int causal, float scale, float* __restrict__ dq_acc,
                      float* __restrict__ dk_acc, float* __restrict__ dv_acc) {
   extern __shared__ float sm[];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
@@ -106,7 +112,7 @@ attn_bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
         s += qs[e] * to_f32(kr[e]);
         dp += dos[e] * to_f32(vr[e]);
       }
-      const float p = expf(s * scale - l);
+      const float p = (!causal || pk[t] <= i) ? expf(s * scale - l) : 0.f;
       ps[t] = p;
       dss[t] = p * (dp - dp_i);
     }
@@ -143,7 +149,7 @@ cudaError_t fwd(const Geometry& g, const void* q, const void* k, const void* v,
   const int64_t rows = (int64_t)g.BH * g.N;
   attn_fwd_simt_kernel<T><<<rows_grid(rows, 4), 128, smem, s>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), perm_q,
-      perm_k, rows, g.N, g.d, g.chunk, g.lookback, g.scale, static_cast<T*>(o_sp), lse);
+      perm_k, rows, g.N, g.d, g.chunk, g.lookback, g.causal, g.scale, static_cast<T*>(o_sp), lse);
   return cudaGetLastError();
 }
 
@@ -162,7 +168,7 @@ cudaError_t bwd(const Geometry& g, const void* q, const void* k, const void* v,
   attn_bwd_simt_kernel<T><<<rows_grid(rows, 4), 128, smem, s>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), perm_q,
       perm_k, static_cast<const T*>(d_o), lse, dprime, rows, g.N, g.d, g.chunk, g.lookback,
-      g.scale, dq_acc, dk_acc, dv_acc);
+      g.causal, g.scale, dq_acc, dk_acc, dv_acc);
   return cudaGetLastError();
 }
 

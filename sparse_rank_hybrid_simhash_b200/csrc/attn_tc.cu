@@ -299,6 +299,7 @@ cudaError_t fwd(const Geometry& g, const void* q, const void* k, const void* v,
 bool attn_tc_supported(const Geometry& g) {
   if (!g.bf16 || (g.d != 64 && g.d != 128)) return false;
   if (g.lookback != 1) return false;   // the tiles hold the own and the previous chunk
+  if (g.causal) return false;
   if (g.N % kTile != 0 || g.chunk % 16 != 0) return false;
   return (kTile % g.chunk == 0) || (g.chunk % kTile == 0);
 }

@@ -173,7 +173,9 @@ fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __re
     const float m = lz > 0.f ? 1.0f / (1.0f + expf(logf(lz) - l)) : 1.0f;
     const float dm = gs * dyo;
     const float dlse = dm * m * (1.0f - m);
-    const float dlam = zr > 0.f ? -dm * m * m * expf(logf(zr) - l) : 0.f;
+    // a causal window without keys (lse = -inf) has Z_sp = 0: m is 0 or 1 and
+    // carries no lambda gradient
+    const float dlam = (zr > 0.f && l > -INFINITY) ? -dm * m * m * expf(logf(zr) - l) : 0.f;
     float da_s = 0.f, da_r = 0.f;
     if (!gate_fixed) {
       da_s = m * dyo * gs * (1.0f - gs);

@@ -30,6 +30,7 @@ struct Geometry {
   float gate_s, gate_r;
   int sort_order;      // elsaa_sort_order
   int lookback;        // previous chunks a query chunk attends (1: own and previous)
+  int causal;          // keys j <= i only (sparse window and RACE read-out)
   int sort_passes, sort_digit_bits, sort_bins, sort_tiles;
   bool tc_hash;       // tcgen05 kernel for the SimHash codes
   bool tc_attn;       // tcgen05 kernels for the sparse branch
@@ -50,6 +51,7 @@ struct WorkLayout {
   size_t sort_tmp;           // [2][BH][N] i32 (intermediate order of a 2-pass sort)
   size_t absmax;             // [2][BH] f32: largest |value| per unit (forward V, backward g_r dy / Ctot)
   size_t gtab;               // [BH][L][NB][d] bf16: the table copy the RACE gathers read
+  size_t causal_num;         // [BH][N][d] f32: causal RACE numerators (0 bytes unless causal)
   size_t saved;              // a SavedLayout used when the forward has no saved buffer
   size_t d_o;                // [BH][N][d] dtype: dO_sp
   size_t dprime;             // [BH][N] f32: D' = dO_sp . O_sp - dlse
@@ -163,6 +165,20 @@ cudaError_t launch_fuse_bwd(const Geometry& g, const void* q, const void* dy, co
 cudaError_t launch_param_reduce(const Geometry& g, const float* partials, float* dgate_w,
                                 float* dgate_b, float* dlambda, cudaStream_t s);
 cudaError_t launch_cast_out(const Geometry& g, const float* src, void* dst, cudaStream_t s);
+
+// Causal RACE (race_causal.cu): per-table token scans and the fusion on their
+// read-out.  num [BH][N][d] fp32 and ctot [BH][N] are zeroed and accumulated;
+// sums / counts receive the full tables.
+bool race_causal_supported(const Geometry& g);
+cudaError_t launch_race_causal_fwd(const Geometry& g, const void* rcode_q, const void* rcode_k,
+                                   const void* v, float* num, int32_t* ctot, float* sums,
+                                   int32_t* counts, cudaStream_t s);
+cudaError_t launch_race_causal_bwd(const Geometry& g, const void* rcode_q, const void* rcode_k,
+                                   const void* dor, float* dv_acc, cudaStream_t s);
+cudaError_t launch_fuse_causal(const Geometry& g, const void* q, const void* o_sp,
+                               const float* lse, const float* num, const int32_t* ctot,
+                               const float* gate_w, const float* gate_b, const float* lam,
+                               void* y, void* o_race, cudaStream_t s);
 
 // 2-D TMA map over a [rows, 64] bf16 matrix: one 128-byte row per box,
 // 128-byte swizzle; the row gathers of the tcgen05 attention kernels use it.

@@ -57,6 +57,7 @@ class Workload:
     dist: str = "iid"      # iid | clusters | zipf | needle
     sort_order: str = "binary"   # binary | gray | local (Sort-LSH bucket order)
     lookback: int = 1            # previous sorted chunks a query chunk attends
+    causal: bool = False         # keys j <= i only
 
     @property
     def torch_dtype(self):

@@ -80,6 +80,7 @@ def test_validation_rejects_bad_problems():
         dict(sort_order=-1),
         dict(lookback=-1),
         dict(lookback=65),
+        dict(causal=2),
     ]
     for c in cases:
         p = B.Params.make(1, 2, 256, 64, "bf16", 4, 64, 8, 6)
@@ -96,6 +97,9 @@ def test_validation_rejects_bad_problems():
     # the CUDA-core attention keeps (lookback + 1) chunk scores per query in shared memory
     p = B.Params.make(1, 2, 8192, 64, "bf16", 4, 1024, 8, 6, lookback=6)
     assert B.validate(p) == 2
+    assert B.validate(B.Params.make(1, 2, 256, 64, "bf16", 4, 64, 8, 8, causal=True)) == 0
+    # the causal RACE scan keeps one table in shared memory
+    assert B.validate(B.Params.make(1, 2, 256, 128, "bf16", 4, 64, 8, 9, causal=True)) == 2
 
 
 def test_null_pointers_are_rejected_before_any_launch():

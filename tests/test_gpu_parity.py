@@ -86,6 +86,16 @@ def test_lookback(cuda_device, lookback, dtype):
     _run(w, backward=True)
 
 
+@pytest.mark.parametrize("dtype,order,gates", [("bf16", "binary", False), ("f32", "local", False),
+                                               ("bf16", "binary", True)])
+def test_causal(cuda_device, dtype, order, gates):
+    # keys j <= i in both branches (CUDA-core attention, per-table RACE token
+    # scans); binary order leaves some early queries with empty windows
+    w = WORKLOADS["iid-4k"].replace(B=1, H=2, N=512, chunk=32, dtype=dtype, sort_order=order,
+                                    causal=True, gate_fixed=gates, gate_s=0.6, gate_r=0.8)
+    _run(w, backward=True)
+
+
 def test_two_pass_sort_and_wide_race_codes(cuda_device):
     # 12 sort bits take two radix passes; 11 RACE bits give uint16 codes and
     # 2048-bucket tables (the global-atomic build)
