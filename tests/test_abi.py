@@ -138,3 +138,14 @@ def test_tensor_core_path_selection(name):
     w = WORKLOADS[name]
     expect = w.dtype == "bf16"   # every bf16 workload tiles onto the tcgen05 kernels
     assert B.uses_tensor_cores(B.Params.from_workload(w)) == expect
+
+
+def test_kernel_launch_counts():
+    # the counts bench.py reports as gpu_launches, per forward and backward
+    w = WORKLOADS["text-32k"]
+    assert B.kernel_launches(B.Params.from_workload(w)) == (8, 5)   # tcgen05 path, one sort pass
+    assert B.kernel_launches(B.Params.from_workload(w.replace(sort_order="local"))) == (6, 5)
+    assert B.kernel_launches(B.Params.from_workload(w.replace(sort_bits=12))) == (11, 5)
+    # causal: token scan instead of |V| max + build; CUDA-core sparse backward + 3 casts
+    c = B.kernel_launches(B.Params.from_workload(w.replace(causal=True)))
+    assert c == (1 + 3 + 1 + 1 + 1, 1 + 1 + 4 + 1)
