@@ -2,9 +2,9 @@
  * libelsaa: the ELSAA attention operator (forward and backward) on NVIDIA B200.
  *
  * ELSAA ("ELSAA: Efficient Low-Rank and Sparse Attention Approximation for
- * Training Transformers", overview) is the non-causal attention applied after
- * the dense Q/K/V projections.  Per (batch, head) unit, with Q, K, V in
- * R^{N x d}:
+ * Training Transformers", overview) is the attention applied after the dense
+ * Q/K/V projections (non-causal on the pages; elsaa_params.causal adds a
+ * causal variant).  Per (batch, head) unit, with Q, K, V in R^{N x d}:
  *
  *   1. SimHash codes: bit j of a row x is [x . r_j > 0].  A sort code of
  *      sort_bits bits from r_sort, and one code of race_bits bits per RACE
@@ -12,6 +12,8 @@
  *   2. Sort-LSH: Q and K are each ordered by their sort code, ties by token
  *      index (stable).  Sorted query chunk j (chunk rows) attends sorted key
  *      chunks j-1 and j (chunk 0 only its own), no wrap-around.
+ *      (elsaa_params.sort_order and lookback select other orders and window
+ *      widths.)
  *   3. Exact sparse branch: O_sp = softmax(scale * q k^T) V over that window
  *      and its unshifted mass Z_sp = exp(lse_sp) ("Two Efficient Attentions,
  *      One Denominator Problem", section "Two efficient branches can still be
@@ -161,7 +163,8 @@ elsaa_status elsaa_backward(const elsaa_params* p, const void* q, const void* k,
  * cudaEvent_t handles (passed as void*; any entry may be NULL) created by the
  * caller; events[0] is recorded on `stream` before the first stage and
  * events[i + 1] after stage i.  Forward stages: SimHash codes, Sort-LSH
- * order, RACE build, sparse branch, RACE gather + fusion.  Backward stages:
+ * order, RACE build, sparse branch, RACE gather + fusion (causal: the RACE
+ * token scan runs in the sparse-branch stage and the build stage is empty).  Backward stages:
  * fusion/gate backward, RACE backward, sparse backward, final casts and the
  * parameter-gradient reduction.  Otherwise identical to elsaa_forward and
  * elsaa_backward (which are these calls with events = NULL). */
@@ -191,8 +194,8 @@ elsaa_status elsaa_kernel_launches(const elsaa_params* p, int32_t* fwd, int32_t*
  * code: device [2][B,H,N] uint16, the sort codes of the queries followed by
  * those of the keys (elsaa_views.code_q is the start of both); perm: device
  * [2][B,H,N] int32 output, the token index at each sorted rank, equal to the
- * permutations elsaa_forward saves.  Both 16-byte aligned.  Only p->B, H, N
- * and sort_bits matter, but p must validate.
+ * permutations elsaa_forward saves.  Both 16-byte aligned.  Only p->B, H, N,
+ * sort_bits and sort_order matter, but p must validate.
  * The radix sort's scratch sits in one fixed device array of
  * ELSAA_NOALLOC_SCRATCH_BYTES that every device loading the library keeps
  * until exit.  The first call on a device looks up that array's device
