@@ -7,6 +7,14 @@ backward) over one batch of the text-32k workload: B2 H12 N32768 d64 bf16,
 synthetic tensors resident in HBM before the timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--mode elsaa|sort_lsh_race|race_only|sparse_only]
+                    [--sort-order binary|gray|local] [--lookback L] [--causal]
+                    [--dense-context] [--no-cpu-baseline]
+
+The modes are the method's ablations on the same kernels (lambda = 0, or one
+branch gated off); sort order, lookback and causal select the extensions of
+the Sort-LSH window; --dense-context adds a timing of dense torch SDPA on the
+same inputs as context.
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch (weak
 scaling, different seed per rank); the shared gate and lambda gradients are
