@@ -57,7 +57,7 @@ extern "C" {
 typedef enum {
   ELSAA_OK = 0,
   ELSAA_ERR_INVALID_ARG = 1,     /* a null pointer, a bad size or misaligned buffer */
-  ELSAA_ERR_UNSUPPORTED = 2,     /* a valid request this build does not implement */
+  ELSAA_ERR_UNSUPPORTED = 2,     /* a valid request this library does not implement */
   ELSAA_ERR_WORKSPACE = 3,       /* ws_bytes smaller than elsaa_workspace_bytes() */
   ELSAA_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed */
   ELSAA_ERR_DEVICE_TIMEOUT = 5,  /* a kernel's bounded wait ran out (elsaa_check) */

@@ -1,6 +1,6 @@
 // Host side of the TMA row gathers: 2-D tensor maps over [rows, 64] bf16
 // matrices (one row per box, 128-byte swizzle), encoded through the driver
-// entry point the runtime resolves (the library links no driver library).
+// entry point the runtime resolves (no direct driver-API calls).
 #include <cudaTypedefs.h>
 #include <mutex>
 
