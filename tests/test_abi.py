@@ -81,6 +81,10 @@ def test_validation_rejects_bad_problems():
         dict(lookback=-1),
         dict(lookback=65),
         dict(causal=2),
+        dict(N=0),                   # empty sequence
+        dict(B=0),
+        dict(H=-1),
+        dict(B=1 << 20, H=1 << 10),  # more than 2^40 elements
     ]
     for c in cases:
         p = B.Params.make(1, 2, 256, 64, "bf16", 4, 64, 8, 6)
