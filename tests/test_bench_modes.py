@@ -46,3 +46,20 @@ def test_single_branch_modes_reduce_to_their_branch(mode, branch):
                          fixed_gates=(w.gate_s, w.gate_r) if w.gate_fixed else None,
                          lam=float(inp["lam"][0]))
     assert torch.allclose(ref["y"], ref[branch], rtol=0, atol=1e-12)
+
+
+def test_operator_roofline_of_the_text_workload():
+    # the operator roofline the bench divides by: fwd 1.04e11 flops / 0.403 GB,
+    # fwd+bwd 2.33e11 flops / 1.32 GB at B2 H12 N32768 d64 bf16, c 128, 7 + 32 x 8 bits
+    bench = _bench()
+    peaks = {"bf16_tflops": 1606.3, "hbm_gbs": 6539.5}
+    r = bench.operator_roofline(WORKLOADS["text-32k"], peaks)
+    n, bh, d = 32768, 24, 64
+    window = 128 * (128 + 255 * 256)          # chunk 0 sees 128 keys, the rest 256
+    assert bench.window_keys(n, 128) == window
+    f_fwd = 2 * 2 * bh * n * d * (7 + 32 * 8) + 4 * bh * window * d
+    assert abs(r["flops_fwd"] - f_fwd) < 1
+    assert abs(r["bytes_fwd"] - 4 * bh * n * d * 2) < 1
+    assert abs(r["fwd_us"] - 65.0) < 0.1 and abs(r["fwdbwd_us"] - 202.0) < 0.1
+    # lookback widens the window: chunk j sees min(j, lb) + 1 chunks
+    assert bench.window_keys(1024, 128, 3) == 128 * 128 * sum(min(j, 3) + 1 for j in range(8))
