@@ -28,6 +28,10 @@ Parity status of each function (what pins it, see ``tests/test_oracle.py``):
   race_build / race_query
                        pinned: per-table sums, K_r = 0 closed form, collision
                        count matrix brute force
+  sparse_branch_rounds / round_perms
+                       pinned: one round equals sparse_branch, a repeated round
+                       adds nothing (keys counted once), pure-Python union of
+                       windows, mass never below any single round's
   race_query_causal    pinned: pure-Python loop over (query, table, key j <= i),
                        last token equals the full read-out, causal dense
                        identities through forward_head
@@ -49,6 +53,8 @@ from .elsaa_oracle import (  # noqa: F401
     SORT_ORDERS,
     chunk_window,
     sparse_branch,
+    sparse_branch_rounds,
+    round_perms,
     race_build,
     race_query,
     race_query_causal,

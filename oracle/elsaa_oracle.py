@@ -161,6 +161,45 @@ def sparse_branch(q, k, v, perm_q, perm_k, chunk: int, scale: float, lookback: i
     return o_sorted[inv], lse_sorted[inv]
 
 
+def sparse_branch_rounds(q, k, v, perms_q, perms_k, chunk: int, scale: float,
+                         lookback: int = 1, causal: bool = False):
+    """Several hash rounds (an extension; the pages use one round): every
+    round t sorts Q and K by its own codes, and a query attends the union of
+    its Sort-LSH windows over the rounds, each key once, with exact softmax.
+    perms_q / perms_k: one permutation per round.  One round is exactly
+    sparse_branch.  Written as a dense N x N mask (test sizes only)."""
+    n = q.shape[0]
+    allowed = torch.zeros(n, n, dtype=torch.bool)
+    for pq, pk in zip(perms_q, perms_k):
+        rank_q = torch.empty_like(pq)
+        rank_q[pq] = torch.arange(n, dtype=pq.dtype)
+        rank_k = torch.empty_like(pk)
+        rank_k[pk] = torch.arange(n, dtype=pk.dtype)
+        cq, ck = (rank_q // chunk)[:, None], (rank_k // chunk)[None, :]
+        allowed |= (ck <= cq) & (ck >= cq - lookback)
+    if causal:
+        allowed &= torch.arange(n)[None, :] <= torch.arange(n)[:, None]
+    has = allowed.any(dim=1)
+    s = scale * (q @ k.T)
+    s = torch.where(allowed | ~has[:, None], s, torch.full_like(s, float("-inf")))
+    lse = torch.logsumexp(s, dim=1)
+    o = torch.softmax(s, dim=1) @ v
+    return (torch.where(has[:, None], o, torch.zeros_like(o)),
+            torch.where(has, lse, torch.full_like(lse, float("-inf"))))
+
+
+def round_perms(q, k, r_sort_rounds, sort_order: str = "binary"):
+    """Sort-LSH permutations of Q and K for each round's hyperplanes
+    (r_sort_rounds: [R, b_s, d]); returns (perms_q, perms_k) lists."""
+    perms_q, perms_k = [], []
+    for planes in r_sort_rounds:
+        cq = simhash_codes(simhash_projections(q.to(F64), planes))
+        ck = simhash_codes(simhash_projections(k.to(F64), planes))
+        perms_q.append(stable_sort_perm(sort_keys(cq, sort_order)))
+        perms_k.append(stable_sort_perm(sort_keys(ck, sort_order)))
+    return perms_q, perms_k
+
+
 # ---------------------------------------------------------------------------
 # Step 4: low-rank RACE branch
 # ---------------------------------------------------------------------------

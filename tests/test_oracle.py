@@ -543,3 +543,54 @@ def test_causal_gradients_match_finite_differences():
     assert torch.autograd.gradcheck(f, args + (lam,), eps=1e-6, atol=1e-7)
     g = O.grads_head(q, k, v, rs, rr, c, dy, None, gw, gb, 0.7, codes=codes, causal=True)
     assert all(torch.isfinite(g[x]).all() for x in ("dq", "dk", "dv", "dlambda"))
+
+
+# ---------------------------------------------------------------------------
+# several hash rounds (an extension): union of the rounds' windows, keys once
+# ---------------------------------------------------------------------------
+
+def test_one_round_is_the_sparse_branch():
+    n, d, c = 48, 6, 8
+    q, k, v = rnd((n, d), 100), rnd((n, d), 101), rnd((n, d), 102)
+    rs = rnd((1, 3, d), 103)
+    pq, pk = O.round_perms(q, k, rs)
+    o1, l1 = O.sparse_branch(q, k, v, pq[0], pk[0], c, 0.4)
+    o2, l2 = O.sparse_branch_rounds(q, k, v, pq, pk, c, 0.4)
+    assert torch.allclose(o1, o2, atol=1e-12, rtol=0)
+    assert torch.allclose(l1, l2, atol=1e-12, rtol=0)
+
+
+def test_a_repeated_round_adds_nothing_and_more_rounds_add_mass():
+    n, d, c = 40, 5, 8
+    q, k, v = rnd((n, d), 104), rnd((n, d), 105), rnd((n, d), 106)
+    rs = rnd((3, 3, d), 107)
+    pq, pk = O.round_perms(q, k, rs)
+    o1, l1 = O.sparse_branch_rounds(q, k, v, pq[:1], pk[:1], c, 0.5)
+    od, ld = O.sparse_branch_rounds(q, k, v, [pq[0], pq[0]], [pk[0], pk[0]], c, 0.5)
+    assert torch.allclose(o1, od, atol=1e-12, rtol=0) and torch.allclose(l1, ld, atol=1e-12, rtol=0)
+    o3, l3 = O.sparse_branch_rounds(q, k, v, pq, pk, c, 0.5)
+    for t in range(3):
+        _, lt = O.sparse_branch_rounds(q, k, v, pq[t:t + 1], pk[t:t + 1], c, 0.5)
+        assert torch.all(l3 >= lt - 1e-12)
+
+
+def test_rounds_union_brute_force():
+    n, d, c = 24, 4, 4
+    q, k, v = rnd((n, d), 108), rnd((n, d), 109), rnd((n, d), 110)
+    g = torch.Generator().manual_seed(111)
+    pq = [torch.randperm(n, generator=g) for _ in range(2)]
+    pk = [torch.randperm(n, generator=g) for _ in range(2)]
+    o, lse = O.sparse_branch_rounds(q, k, v, pq, pk, c, 0.6)
+    for i in range(n):
+        keys = set()
+        for t in range(2):
+            ri = int((pq[t] == i).nonzero()) // c
+            for j in range(n):
+                rj = int((pk[t] == j).nonzero()) // c
+                if ri - 1 <= rj <= ri:
+                    keys.add(j)
+        keys = sorted(keys)
+        s = torch.stack([0.6 * q[i] @ k[j] for j in keys])
+        p = torch.softmax(s, 0)
+        assert abs(float(lse[i]) - float(torch.logsumexp(s, 0))) < 1e-12
+        assert torch.allclose(o[i], sum(p[t] * v[j] for t, j in enumerate(keys)), atol=1e-12)
