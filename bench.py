@@ -122,7 +122,7 @@ RECORDED_TRAFFIC = {
     "race_build": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "9ff8ca9fd3724573a561d5ad5f1319a4dafe1fd0", 1.372e+08),
     "sparse_fwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_pipe.cu", "91a31d0c88874e37ef33ed4bb443baabc0c07369", 3.735e+08),
     "race_fuse": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "9ff8ca9fd3724573a561d5ad5f1319a4dafe1fd0", 3.717e+08),
-    "fuse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/fuse_bwd.cu", "89c43d20c325ca642bd7659d6e92a675de8d3d7b", 5.621e+08),
+    "fuse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/fuse_bwd.cu", "d225c68863731ac35a2126d849af1623d8c512c7", 5.621e+08),
     "race_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "9ff8ca9fd3724573a561d5ad5f1319a4dafe1fd0", 1.34e+08),
     "sparse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_bwd3.cu", "d8764bf2cfd3093b7f01c78d4ad9412897ad1eeb", 6.626e+08),
     "finish": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "9ff8ca9fd3724573a561d5ad5f1319a4dafe1fd0", 1.586e+08),

@@ -15,7 +15,8 @@
 //   dO_race / Ctot = g_r dy / Ctot  (scattered into the RACE table gradient)
 // dq_gate goes out either as fp32 rows (dq_acc) or as the pair (da_s, da_r)
 // per row (da_out) for a consumer that forms da_s w_s + da_r w_r itself.
-// One warp per query; per-block partial sums of (dw_s, dw_r, db_s, db_r,
+// A query takes d / 4 lanes (four values each), so a warp serves 128 / d
+// queries per step; per-block partial sums of (dw_s, dw_r, db_s, db_r,
 // dlambda) go to a fixed number of slots and are reduced in a fixed order, so
 // the parameter gradients are deterministic.
 #include <math.h>
@@ -66,8 +67,8 @@ ELSAA_DEV float gsum(float v) {
   return v;
 }
 
-// QL = d / 4 lanes per query (4 consecutive values each, 16-byte accesses),
-// 32 / QL queries per warp.
+// QL = d / 4 lanes per query (4 consecutive values each: 8-byte accesses for
+// bf16, 16-byte for fp32), 32 / QL queries per warp.
 template <typename T, int QL>
 __global__ void __launch_bounds__(256, 4)
 fuse_bwd_kernel(const T* __restrict__ q, const T* __restrict__ dy, const T* __restrict__ o_sp,
