@@ -118,14 +118,14 @@ def stage_roofline(flops, nbytes, sec, peaks):
 # workload by the number of units; reported only while that file is unchanged.
 RECORDED_TRAFFIC = {
     # stage: (kernel source, its sha1 at capture, bytes per full-size launch)
-    "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "e64b5b0853a47abfb13af9aec16cec6b49568584", 2.459e+08),
-    "race_build": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "9ff8ca9fd3724573a561d5ad5f1319a4dafe1fd0", 1.372e+08),
+    "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "495295df2fda78a4a966636d9641afe4401ac126", 2.459e+08),
+    "race_build": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "0d588b8c632b81b3ffdfb0a8110ff049180f2520", 1.372e+08),
     "sparse_fwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_pipe.cu", "91a31d0c88874e37ef33ed4bb443baabc0c07369", 3.735e+08),
-    "race_fuse": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "9ff8ca9fd3724573a561d5ad5f1319a4dafe1fd0", 3.717e+08),
+    "race_fuse": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "0d588b8c632b81b3ffdfb0a8110ff049180f2520", 3.717e+08),
     "fuse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/fuse_bwd.cu", "d225c68863731ac35a2126d849af1623d8c512c7", 5.621e+08),
-    "race_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "9ff8ca9fd3724573a561d5ad5f1319a4dafe1fd0", 1.34e+08),
+    "race_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "0d588b8c632b81b3ffdfb0a8110ff049180f2520", 1.34e+08),
     "sparse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_bwd3.cu", "d8764bf2cfd3093b7f01c78d4ad9412897ad1eeb", 6.626e+08),
-    "finish": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "9ff8ca9fd3724573a561d5ad5f1319a4dafe1fd0", 1.586e+08),
+    "finish": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "0d588b8c632b81b3ffdfb0a8110ff049180f2520", 1.586e+08),
 }
 
 

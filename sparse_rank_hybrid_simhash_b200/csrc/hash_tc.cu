@@ -19,7 +19,8 @@
 //
 // Persistent CTAs of 128 threads.  The hyperplanes stay resident in shared
 // memory; 128-row tiles of Q then K stream in by cp.async (double-buffered
-// when shared memory allows).  Per tile the columns go through TMEM in passes
+// where that costs no CTA per SM: at text-32k sizes four single-buffered CTAs
+// per SM beat three double-buffered ones).  Per tile the columns go through TMEM in passes
 // of 128: thread t reads the 32 projections of row t per tcgen05.ld and keeps
 // the sign mask.  The tile's codes leave as one contiguous row-major block and,
 // through a 4 x 4 (or 2 x 2) byte transpose across lanes, as 4-byte runs of

@@ -9,12 +9,18 @@
 //   Ctot = sum_l C[l][h_l(q)],  O_race = sum_l T[l][h_l(q)] / Ctot  (0 if Ctot = 0),
 //   Z_race = Ctot / L.
 //
-// Build: one block owns a slab of tables x a 32-wide slice of d in shared
-// memory and streams every key of its unit through it (shared-memory fp32
-// atomics; the slab is written once, so global memory sees no atomics).
-// Tables too large for shared memory take a global-atomic variant.
-// Gather: one warp per query, lanes across d, codes broadcast by shuffle.
-// The forward gather is fused with the gates, the multiplier and the output.
+// Build (race_build_sorted_kernel, described where it is defined): one CTA
+// per (unit, table) bucket-sorts the table's keys in shared memory and sums
+// each bucket's value rows as one run, into a fixed-point table (exact,
+// order-independent).  Shapes it does not fit take a slab build (a block owns
+// tables x a 32-wide slice of d in shared memory and streams every key of its
+// unit through it with shared-memory atomics) or, for tables too large for
+// shared memory, a global-atomic build.
+// Gather (race_gather_rows_kernel, race_fuse_rows_kernel): a row per group of
+// d / 8 lanes with 16-byte table lines, the row's codes as whole words and
+// the next row's codes prefetched; the forward gather is fused with the gates,
+// the multiplier and the output.  Other code widths take a warp-per-query
+// gather with codes broadcast by shuffle.
 #include "common.cuh"
 #include "internal.h"
 
