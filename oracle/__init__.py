@@ -35,7 +35,9 @@ Parity status of each function (what pins it, see ``tests/test_oracle.py``):
   race_query_causal    pinned: pure-Python loop over (query, table, key j <= i),
                        last token equals the full read-out, causal dense
                        identities through forward_head
-  gates / fuse         pinned: lambda = 0 ablation (m == 1), single-branch gate
+  gates / fuse         pinned: hand-worked learned gates (distinct weight rows,
+                       nonzero biases, q != 0, tokens out of sorted order),
+                       lambda = 0 ablation (m == 1), single-branch gate
                        settings, Z_race = 0, closed form for Q = 0
   forward_head         pinned through the pieces above and the Q = 0 closed form
   grads_head           pinned: finite differences (gradcheck) of forward_head,

@@ -262,6 +262,45 @@ def test_hand_worked_four_token_example():
             assert abs(float(out["y"][i, c]) - y[c]) < 1e-13
 
 
+def test_hand_worked_learned_gates():
+    """The learned gates of the same 4-token example written out with scalars:
+    g_s = sigmoid(w_s . q_i + b_s) from row 0 of the gate weights, g_r from row 1,
+    q_i the query in token order (the sort puts the tokens in order 1, 3, 0, 2,
+    so a gate taken at a sorted position would differ), no score scale on the
+    gate logit (ELSAA overview: learned or fixed gates; "Two Efficient
+    Attentions, One Denominator Problem", section "Two efficient branches can
+    still be mis-scaled": independent token-wise gates)."""
+    q = torch.tensor([[1.0, 1.0], [-1.0, 1.0], [0.5, -1.0], [-2.0, -1.0]], dtype=F64)
+    k = torch.tensor([[1.0, 0.0], [-1.0, 1.0], [2.0, -1.0], [0.0, 1.0]], dtype=F64)
+    v = torch.tensor([[1.0, 2.0], [3.0, -1.0], [0.0, 4.0], [-2.0, 1.0]], dtype=F64)
+    rs = torch.tensor([[1.0, 0.0]], dtype=F64)
+    rr = torch.tensor([[[0.0, 1.0]]], dtype=F64)
+    gw = torch.tensor([[0.5, -0.25], [1.0, 0.75]], dtype=F64)   # row 0 sparse, row 1 RACE
+    gb = torch.tensor([0.1, -0.2], dtype=F64)
+    lam = 0.5
+    out = O.forward_head(q, k, v, rs, rr, 2, None, gw, gb, lam=lam)
+    assert out["perm_q"].tolist() == [1, 3, 0, 2]
+    sig = lambda a: 1.0 / (1.0 + math.exp(-a))
+    Q = q.tolist()
+    # logits by hand: token 0: w_s.q = 0.5 - 0.25 = 0.25, w_r.q = 1.0 + 0.75 = 1.75
+    a_s = [0.25, -0.75, 0.5, -0.75]
+    a_r = [1.75, -0.25, -0.25, -2.75]
+    for i in range(4):
+        assert abs(0.5 * Q[i][0] - 0.25 * Q[i][1] - a_s[i]) < 1e-15
+        assert abs(1.0 * Q[i][0] + 0.75 * Q[i][1] - a_r[i]) < 1e-15
+        gs, gr = sig(a_s[i] + 0.1), sig(a_r[i] - 0.2)
+        assert abs(float(out["g_s"][i]) - gs) < 1e-14
+        assert abs(float(out["g_r"][i]) - gr) < 1e-14
+        m = float(out["m"][i])
+        for c in range(2):
+            want = gs * m * float(out["o_sp"][i, c]) + gr * float(out["o_race"][i, c])
+            assert abs(float(out["y"][i, c]) - want) < 1e-13
+    # the two rows are not interchangeable on this example
+    assert abs(float(out["g_s"][0]) - sig(1.75 + 0.1)) > 0.1
+    # token 0 and token 2 swap places in the sorted order: their gates differ
+    assert abs(float(out["g_s"][0]) - float(out["g_s"][2])) > 0.01
+
+
 def test_zero_queries_closed_form():
     n, d, c, L, kr = 64, 6, 16, 5, 3
     k, v = rnd((n, d), 40), rnd((n, d), 41)
