@@ -38,22 +38,23 @@ class Params(ctypes.Structure):
                 ("race_bits", ctypes.c_int32), ("scale", ctypes.c_float),
                 ("gate_fixed", ctypes.c_int32), ("gate_s", ctypes.c_float),
                 ("gate_r", ctypes.c_float), ("sort_order", ctypes.c_int32),
-                ("lookback", ctypes.c_int32), ("causal", ctypes.c_int32)]
+                ("lookback", ctypes.c_int32), ("causal", ctypes.c_int32),
+                ("hash_rounds", ctypes.c_int32)]
 
     @classmethod
     def make(cls, B, H, N, d, dtype, sort_bits, chunk, race_tables, race_bits, scale=0.0,
              gate_fixed=False, gate_s=0.5, gate_r=0.5, sort_order="binary",
-             lookback=1, causal=False) -> "Params":
+             lookback=1, causal=False, hash_rounds=1) -> "Params":
         dt = ELSAA_BF16 if dtype in ("bf16", torch.bfloat16) else ELSAA_F32
         return cls(B, H, N, d, dt, sort_bits, chunk, race_tables, race_bits, float(scale),
                    int(bool(gate_fixed)), float(gate_s), float(gate_r), SORT_ORDERS[sort_order],
-                   int(lookback), int(bool(causal)))
+                   int(lookback), int(bool(causal)), int(hash_rounds))
 
     @classmethod
     def from_workload(cls, w) -> "Params":
         return cls.make(w.B, w.H, w.N, w.d, w.dtype, w.sort_bits, w.chunk, w.race_tables,
                         w.race_bits, 0.0, w.gate_fixed, w.gate_s, w.gate_r, w.sort_order,
-                        w.lookback, w.causal)
+                        w.lookback, w.causal, w.hash_rounds)
 
     @property
     def torch_dtype(self):
@@ -68,7 +69,8 @@ class Views(ctypes.Structure):
                 ("rcode_bytes", ctypes.c_int32), ("race_count", ctypes.c_void_p),
                 ("race_sum", ctypes.c_void_p), ("lse_sp", ctypes.c_void_p),
                 ("o_sp", ctypes.c_void_p), ("o_race", ctypes.c_void_p),
-                ("ctot", ctypes.c_void_p)]
+                ("ctot", ctypes.c_void_p), ("round_code", ctypes.c_void_p),
+                ("round_perm", ctypes.c_void_p), ("hash_rounds", ctypes.c_int32)]
 
 
 EXPORTS = ("elsaa_validate", "elsaa_workspace_bytes", "elsaa_saved_bytes", "elsaa_forward",
@@ -221,7 +223,20 @@ def sort_codes_noalloc(p: Params, code: torch.Tensor, perm: torch.Tensor, stream
     """Sort-LSH permutations of ``code`` ([2, B, H, N] int16 view of the uint16
     sort codes, queries then keys) into ``perm`` ([2, B, H, N] int32) with no
     scratch from the caller: for callers that cannot allocate device memory
-    while they run (see elsaa_sort_codes_noalloc in include/elsaa.h)."""
+    while they run (see elsaa_sort_codes_noalloc in include/elsaa.h).  Both
+    tensors must be contiguous and on the current CUDA device, whose scratch
+    array the call uses."""
+    n = 2 * p.B * p.H * p.N
+    if code.dtype not in (torch.int16, torch.uint16) or perm.dtype != torch.int32:
+        raise TypeError("code must be int16/uint16 and perm int32")
+    if code.numel() != n or perm.numel() != n:
+        raise ValueError(f"code and perm must hold 2*B*H*N = {n} elements")
+    if not (code.is_contiguous() and perm.is_contiguous()):
+        raise ValueError("code and perm must be contiguous")
+    cur = torch.cuda.current_device()
+    for t in (code, perm):
+        if t.device.type != "cuda" or t.device.index != cur:
+            raise ValueError(f"tensors must be on the current device cuda:{cur}")
     _ok("elsaa_sort_codes_noalloc", lib().elsaa_sort_codes_noalloc(
         ctypes.byref(p), _ptr(code), _ptr(perm), _stream(stream)))
 
@@ -260,6 +275,11 @@ def saved_views(p: Params, saved: torch.Tensor) -> Dict[str, torch.Tensor]:
         "o_sp": view(v.o_sp, n * d, dt, (B, H, N, d)),
         "o_race": view(v.o_race, n * d, dt, (B, H, N, d)),
         "ctot": view(v.ctot, n, torch.int32, (B, H, N)),
+        # every hash round: [R, 2 (queries, keys), B, H, N]
+        "round_code": view(v.round_code, v.hash_rounds * 2 * n, torch.int16,
+                           (v.hash_rounds, 2, B, H, N)),
+        "round_perm": view(v.round_perm, v.hash_rounds * 2 * n, torch.int32,
+                           (v.hash_rounds, 2, B, H, N)),
     }
 
 

@@ -201,28 +201,74 @@ namespace elsaa {
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
-constexpr int kMaxDevices = 64;
+constexpr int kMaxContexts = 64;
 
 __device__ __align__(256) unsigned char g_sort_scratch[kNoAllocScratchBytes];
 
+// Device addresses of g_sort_scratch, one per CUDA context that has called in.
+// The address belongs to the module loaded into a context, so the cache is
+// keyed on the context's unique ID (cuCtxGetId: never reused within a
+// process), not on the device index: after cudaDeviceReset, or when the caller
+// makes another context current on the same device, the module is loaded anew
+// and the array can sit elsewhere, and that context looks the address up again.
 std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  void* ptr;
+};
+ScratchEntry g_scratch[kMaxContexts] = {};
+int g_scratch_n = 0;
 
-// Device address of g_sort_scratch on the current device, looked up once per
-// device (the host-side symbol is only a stand-in and must never reach a kernel).
+// cuCtxGetCurrent and cuCtxGetId through the driver entry points the runtime
+// resolves (the library makes no direct driver-API calls).
+struct CtxFns {
+  CUresult (*get_current)(CUcontext*) = nullptr;
+  CUresult (*get_id)(CUcontext, unsigned long long*) = nullptr;
+};
+const CtxFns& ctx_fns() {
+  static CtxFns f;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_current = reinterpret_cast<CUresult (*)(CUcontext*)>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_id = reinterpret_cast<CUresult (*)(CUcontext, unsigned long long*)>(p);
+  });
+  return f;
+}
+
+// Device address of g_sort_scratch in the current context (the host-side
+// symbol is only a stand-in and must never reach a kernel).
 cudaError_t scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_sort_scratch);
+  const CtxFns& f = ctx_fns();
+  if (!f.get_current || !f.get_id) return cudaErrorNotSupported;
+  CUcontext ctx = nullptr;
+  if (f.get_current(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  void* ptr = nullptr;
+  if (ctx == nullptr) {
+    // no context yet: the symbol lookup makes the runtime's primary context current
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_sort_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = ptr;
+    if (f.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorDeviceUninitialized;
   }
-  *out = g_scratch_ptr[dev];
+  unsigned long long id = 0;
+  if (f.get_id(ctx, &id) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  for (int i = 0; i < g_scratch_n; ++i)
+    if (g_scratch[i].ctx_id == id) {
+      *out = g_scratch[i].ptr;
+      return cudaSuccess;
+    }
+  if (ptr == nullptr) {
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_sort_scratch);
+    if (e != cudaSuccess) return e;
+  }
+  if (g_scratch_n < kMaxContexts) g_scratch[g_scratch_n++] = {id, ptr};
+  *out = ptr;
   return cudaSuccess;
 }
 

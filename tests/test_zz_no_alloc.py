@@ -24,6 +24,13 @@ CASES = {
     "text-32k-small": small(WORKLOADS["text-32k"], B=1, H=2, N=1024),
     "two-radix-passes": WORKLOADS["iid-4k"].replace(B=1, H=2, N=1024, sort_bits=12),
     "needle-small": small(WORKLOADS["needle-256k"], B=1, H=2, N=2048),
+    # Gray order transforms the key where the radix sort reads it; 12 bits
+    # take two passes, so both the histograms and the intermediate order sit
+    # in the library's scratch
+    "gray-two-passes": WORKLOADS["iid-4k"].replace(B=1, H=2, N=1024, sort_bits=12,
+                                                   sort_order="gray"),
+    # local order writes token order and touches no scratch
+    "local-order": WORKLOADS["iid-4k"].replace(B=1, H=2, N=1024, sort_order="local"),
 }
 
 
@@ -39,7 +46,8 @@ def test_noalloc_sort_matches_forward_permutations(cuda_device, name):
     B.check(ws)
     views = B.saved_views(p, saved)
     n = w.B * w.H * w.N
-    codes = views["code_q"]            # the query codes, followed in memory by the key codes
+    # the query codes followed by the key codes, as one contiguous [2, B, H, N]
+    codes = torch.cat([views["code_q"].reshape(-1), views["code_k"].reshape(-1)])
     expect = torch.cat([views["perm_q"].reshape(-1), views["perm_k"].reshape(-1)])
     for _ in range(2):                 # the second call sees the first call's scratch
         perm = torch.full((2 * n,), -1, dtype=torch.int32, device=cuda_device)
