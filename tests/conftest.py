@@ -19,3 +19,14 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Print the parameter-gradient errors measured by the parity tests."""
+    stats = sys.modules.get("parity")
+    stats = getattr(stats, "PARAM_GRAD_STATS", None) if stats else None
+    if not stats:
+        return
+    terminalreporter.write_line("parameter gradients: workload name rel_l2 cancellation scaled")
+    for row in stats:
+        terminalreporter.write_line("  %s %s %.3e %.3e %.3e" % row)

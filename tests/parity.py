@@ -68,7 +68,8 @@ def oracle_unit(w: Workload, inp, b: int, h: int, codes=None, backward=False):
     out = O.forward_head(*args, None, inp["gate_w"], inp["gate_b"], lam, fixed, codes=codes,
                          sort_order=w.sort_order, lookback=w.lookback, causal=w.causal)
     if backward:
-        c = codes or {n: out[n] for n in ("code_q", "code_k", "rcode_q", "rcode_k")}
+        c = codes or {n: out[n] for n in ("code_q", "code_k", "rcode_q", "rcode_k",
+                                          "round_code_q", "round_code_k") if n in out}
         g = O.grads_head(*args, inp["dy"][b, h], None, inp["gate_w"], inp["gate_b"], lam, fixed,
                          codes=c, sort_order=w.sort_order, lookback=w.lookback,
                          causal=w.causal)
@@ -102,17 +103,31 @@ def check_unit(w: Workload, inp, gpu, b: int, h: int, backward: bool, report: di
     n_diff += compare_codes(code_k, ref["code_k"], ref["near_code_k"], "sort code k")
     n_diff += compare_codes(rq, ref["rcode_q"], ref["near_rcode_q"], "race code q")
     n_diff += compare_codes(rk, ref["rcode_k"], ref["near_rcode_k"], "race code k")
+    codes = {"code_q": code_q, "code_k": code_k, "rcode_q": rq, "rcode_k": rk}
+    if w.hash_rounds > 1:
+        # every hash round's codes; round 0 is the codes above
+        rc = B.unsigned16(v["round_code"][:, :, b, h])            # [R, 2, N]
+        for t in range(1, w.hash_rounds):
+            n_diff += compare_codes(rc[t, 0], ref["round_code_q"][t],
+                                    ref["near_round_code_q"][t], f"round {t} code q")
+            n_diff += compare_codes(rc[t, 1], ref["round_code_k"][t],
+                                    ref["near_round_code_k"][t], f"round {t} code k")
+        assert torch.equal(rc[0, 0], code_q) and torch.equal(rc[0, 1], code_k)
+        codes.update(round_code_q=rc[:, 0], round_code_k=rc[:, 1])
     report["code_mismatch_near_zero"] = report.get("code_mismatch_near_zero", 0) + n_diff
     if n_diff:
         # several codes are correct where a projection is ~0: re-run the oracle's
         # float steps with the device's codes
-        codes = {"code_q": code_q, "code_k": code_k, "rcode_q": rq, "rcode_k": rk}
         ref = oracle_unit(w, inp, b, h, codes=codes, backward=backward)
     elif backward:
         ref = oracle_unit(w, inp, b, h, backward=True)
     # sort order and table counts are exact
     assert torch.equal(v["perm_q"][b, h].to(torch.int64), ref["perm_q"]), "perm_q"
     assert torch.equal(v["perm_k"][b, h].to(torch.int64), ref["perm_k"]), "perm_k"
+    if w.hash_rounds > 1:
+        rp = v["round_perm"][:, :, b, h].to(torch.int64)
+        assert torch.equal(rp[:, 0], ref["round_perm_q"]), "round perm q"
+        assert torch.equal(rp[:, 1], ref["round_perm_k"]), "round perm k"
     assert torch.equal(v["race_count"][b, h].to(torch.int64), ref["race_count"]), "race_count"
     assert torch.equal(v["ctot"][b, h].to(torch.int64), ref["ctot"]), "ctot"
     assert_close("race_sum", v["race_sum"][b, h], ref["race_sum"], dt, 1e-5, 1e-3)
@@ -130,13 +145,30 @@ def check_unit(w: Workload, inp, gpu, b: int, h: int, backward: bool, report: di
     return ref
 
 
+# Every parameter-gradient comparison made in this process:
+# (workload, name, plain rel-L2, cancellation ratio, error / sum-of-magnitudes)
+PARAM_GRAD_STATS: List[tuple] = []
+
+# Below this cancellation ratio the plain rel-L2 bound is not asserted: the
+# device's error is a bf16-level fraction (about 1e-3 measured) of the summed
+# magnitudes, so the plain ratio error / ||sum|| exceeds 1e-2 once the sum is
+# under a tenth of the magnitudes it was summed from.
+CANCELLATION_FLOOR = 0.1
+
+
 def check_param_grads(w: Workload, gpu, refs: List[dict]):
     """Gate and lambda gradients are sums over every unit: compare when all
-    units were checked.  Their per-unit contributions can cancel, so the
-    error is measured against the size of what was summed:
-    ||got - ref||_2 <= tol * || sum_u |ref_u| ||_2  (for one unit this is the
-    relative L2 error)."""
+    units were checked.  Two measures are taken:
+      plain  = ||got - ref||_2 / ||ref||_2        (the stated rel-L2 bound)
+      scaled = ||got - ref||_2 / || sum_u |ref_u| ||_2
+    where ref_u is unit u's contribution.  The scaled measure is always
+    asserted; the plain one wherever the cancellation ratio
+    ||ref|| / ||sum_u |ref_u||| is at least CANCELLATION_FLOOR (where the parts
+    cancel further, the bf16 error, which scales with the parts and not with
+    their sum, can exceed it).  Every comparison is recorded in
+    PARAM_GRAD_STATS."""
     r0, _ = TOL[w.dtype]
+    out = {}
     for name, key in (("dgate_w", "grad_dgate_w"), ("dgate_b", "grad_dgate_b"),
                       ("dlambda", "grad_dlambda")):
         parts = torch.stack([r[key].reshape(-1) for r in refs])
@@ -144,5 +176,18 @@ def check_param_grads(w: Workload, gpu, refs: List[dict]):
         scale = parts.abs().sum(0).norm().item()
         got = gpu[name].double().reshape(-1)
         err = (got - ref).norm().item()
+        ref_norm = ref.norm().item()
+        if scale == 0.0:   # fixed gates: both sides exactly zero
+            assert err == 0.0, f"{name}: expected exact zeros, ||err|| = {err:.3e}"
+            continue
+        plain = err / ref_norm if ref_norm > 0 else float("inf")
+        ratio = ref_norm / scale
+        tag = f"{w.name}[B{w.B} H{w.H} N{w.N} c{w.chunk} {w.sort_order} lam{w.lam}]"
+        PARAM_GRAD_STATS.append((tag, name, plain, ratio, err / scale))
+        out[name] = {"rel_l2": plain, "cancellation": ratio, "scaled": err / scale}
         assert err <= r0 * scale + 1e-12, \
             f"{name}: ||err|| = {err:.3e}, tol * ||sum_u |parts||| = {r0 * scale:.3e}"
+        if ratio >= CANCELLATION_FLOOR:
+            assert plain <= r0, f"{name}: rel_l2 {plain:.3e} (<= {r0}); cancellation " \
+                                f"ratio {ratio:.3e}"
+    return out
