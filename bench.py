@@ -8,7 +8,8 @@ synthetic tensors resident in HBM before the timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--mode elsaa|sort_lsh_race|race_only|sparse_only]
-                    [--sort-order binary|gray|local] [--lookback L] [--causal]
+                    [--sort-order binary|gray|local] [--lookback L] [--hash-rounds R]
+                    [--causal]
                     [--dense-context] [--no-cpu-baseline]
 
 The modes are the method's ablations on the same kernels (lambda = 0, or one
@@ -280,7 +281,7 @@ def bench_config(w, mode, world, l2):
     """The config object of a bench line (both arms)."""
     return {"workload": w.name, "mode": mode, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
             "sort_bits": w.sort_bits, "sort_order": w.sort_order, "lookback": w.lookback,
-            "causal": w.causal,
+            "causal": w.causal, "hash_rounds": w.hash_rounds,
             "chunk": w.chunk,
             "race_tables": w.race_tables,
             "race_bits": w.race_bits,
@@ -338,7 +339,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = apply_mode(WORKLOADS[args.workload], args.mode).replace(
-        sort_order=args.sort_order, lookback=args.lookback, causal=args.causal)
+        sort_order=args.sort_order, lookback=args.lookback, causal=args.causal,
+        hash_rounds=args.hash_rounds)
     p = B.Params.from_workload(w)
     inp = make_inputs(w, seed=DP.rank_seed(w.seed, rank), with_dy=True)
     d = {k: t.to(dev) for k, t in inp.items()}
@@ -458,7 +460,8 @@ def oracle_unit_seconds(w, inp, units):
                 w.chunk)
         fixed = (w.gate_s, w.gate_r) if w.gate_fixed else None
         O.grads_head(*args, inp["dy"][b, h], None, inp["gate_w"], inp["gate_b"],
-                     float(inp["lam"][0]), fixed, sort_order=w.sort_order)
+                     float(inp["lam"][0]), fixed, sort_order=w.sort_order,
+                     lookback=w.lookback, causal=w.causal)
     return time.perf_counter() - t0
 
 
@@ -486,7 +489,8 @@ def run_reference(args):
     if rank != 0:
         return
     w = apply_mode(WORKLOADS[args.workload], args.mode).replace(
-        sort_order=args.sort_order, lookback=args.lookback, causal=args.causal)
+        sort_order=args.sort_order, lookback=args.lookback, causal=args.causal,
+        hash_rounds=args.hash_rounds)
     cores = len(os.sched_getaffinity(0))
     torch.set_num_threads(cores)
     inp = make_inputs(w, with_dy=True)
@@ -533,6 +537,8 @@ def main():
                     help="Sort-LSH chunk order: code value, Gray sequence, or token order")
     ap.add_argument("--lookback", type=int, default=1,
                     help="previous sorted chunks a query chunk attends (1: own and previous)")
+    ap.add_argument("--hash-rounds", type=int, default=1,
+                    help="Sort-LSH hash rounds; a query attends the union of its windows")
     ap.add_argument("--causal", action="store_true",
                     help="keys j <= i only (CUDA-core attention, RACE token scans)")
     ap.add_argument("--dense-context", action="store_true",

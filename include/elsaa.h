@@ -12,8 +12,8 @@
  *   2. Sort-LSH: Q and K are each ordered by their sort code, ties by token
  *      index (stable).  Sorted query chunk j (chunk rows) attends sorted key
  *      chunks j-1 and j (chunk 0 only its own), no wrap-around.
- *      (elsaa_params.sort_order and lookback select other orders and window
- *      widths.)
+ *      (elsaa_params.sort_order, lookback and hash_rounds select other
+ *      orders, window widths and several hash rounds.)
  *   3. Exact sparse branch: O_sp = softmax(scale * q k^T) V over that window
  *      and its unshifted mass Z_sp = exp(lse_sp) ("Two Efficient Attentions,
  *      One Denominator Problem", section "Two efficient branches can still be
@@ -32,9 +32,11 @@
  *
  * Conventions for every entry point:
  *   - Every pointer named "device" is CUDA device memory owned by the caller.
- *     The library never allocates or frees device or pinned memory and keeps
- *     no mutable global state; calls on different streams with different
- *     workspaces may run concurrently.
+ *     The library never allocates or frees device or pinned memory.  Apart
+ *     from elsaa_sort_codes_noalloc (one fixed device array shared by all of
+ *     its calls, and a cache of that array's address per CUDA context; see
+ *     its comment) it keeps no mutable global state: calls on different
+ *     streams with different workspaces may run concurrently.
  *   - All work is enqueued on `stream` (a cudaStream_t passed as void*; NULL
  *     is the legacy default stream).  Calls return without synchronising;
  *     device-side failures (a bounded wait that ran out) are recorded in the
@@ -97,6 +99,12 @@ typedef struct {
                            * keys has Z_sp = 0 (O_sp = 0, lse = -inf).  Runs on the
                            * CUDA-core attention and a per-table token scan for RACE;
                            * needs 2^race_bits * (d + 1) * 4 <= 200 KB */
+  int32_t hash_rounds;    /* Sort-LSH hash rounds, 0..8 (0 and 1 both mean one round, the
+                           * pages' setting).  With R > 1 rounds every round t sorts Q
+                           * and K by its own sort hyperplanes r_sort[t], and a query
+                           * attends the union of its R windows, each key once, with
+                           * exact softmax (an extension; runs on the CUDA-core
+                           * attention; needs R * (lookback + 1) * chunk <= 6144) */
 } elsaa_params;
 
 /* Device views into a forward's saved state (see elsaa_saved_views). */
@@ -114,6 +122,11 @@ typedef struct {
   void* o_sp;             /* [B,H,N,d] sparse-branch output (dtype), token order */
   void* o_race;           /* [B,H,N,d] RACE-branch output (dtype), token order */
   int32_t* ctot;          /* [B,H,N] Ctot */
+  uint16_t* round_code;   /* [R][2][B,H,N] sort codes of every hash round (queries then keys
+                           * per round); round 0 is code_q / code_k */
+  int32_t* round_perm;    /* [R][2][B,H,N] permutations of every round; round 0 is
+                           * perm_q / perm_k */
+  int32_t hash_rounds;    /* R */
 } elsaa_views;
 
 /* Returns ELSAA_OK if `p` describes a supported problem, else the reason. */
@@ -128,8 +141,8 @@ size_t elsaa_workspace_bytes(const elsaa_params* p);
  * backward reads; 0 if `p` is invalid. */
 size_t elsaa_saved_bytes(const elsaa_params* p);
 
-/* Forward.  q, k, v: device [B,H,N,d]; r_sort: device [sort_bits, d] (may
- * be NULL when sort_bits = 0); r_race: device [L, race_bits, d] (may be NULL
+/* Forward.  q, k, v: device [B,H,N,d]; r_sort: device [R, sort_bits, d] with
+ * R = hash_rounds (may be NULL when sort_bits = 0); r_race: device [L, race_bits, d] (may be NULL
  * when race_bits = 0); hyperplanes are shared by Q and K and by every unit
  * and have the data dtype.  gate_w: device fp32 [2,d] (row 0 sparse, row 1 RACE),
  * gate_b: device fp32 [2]; both ignored (may be NULL) if gate_fixed.
@@ -194,12 +207,15 @@ elsaa_status elsaa_kernel_launches(const elsaa_params* p, int32_t* fwd, int32_t*
  * code: device [2][B,H,N] uint16, the sort codes of the queries followed by
  * those of the keys (elsaa_views.code_q is the start of both); perm: device
  * [2][B,H,N] int32 output, the token index at each sorted rank, equal to the
- * permutations elsaa_forward saves.  Both 16-byte aligned.  Only p->B, H, N,
- * sort_bits and sort_order matter, but p must validate.
+ * permutations elsaa_forward saves (for one hash round: hash_rounds is not
+ * read).  Both 16-byte aligned.  Only p->B, H, N, sort_bits and sort_order
+ * matter, but p must validate.
  * The radix sort's scratch sits in one fixed device array of
  * ELSAA_NOALLOC_SCRATCH_BYTES that every device loading the library keeps
- * until exit.  The first call on a device looks up that array's device
- * address (with the device current), so make it before any stream capture.
+ * until exit.  The first call in a CUDA context looks up that array's device
+ * address in the current context, so make it before any stream capture; a
+ * context created later (after cudaDeviceReset, or another context made
+ * current) repeats the lookup on its first call.
  * Returns ELSAA_ERR_WORKSPACE if the problem needs more scratch than that
  * (2 B H 2^digit_bits ceil(N/2048) ints, plus 2 B H N ints when sort_bits > 8).
  * All calls share the array: calls that may overlap on the GPU (other

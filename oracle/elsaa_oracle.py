@@ -308,20 +308,25 @@ def forward_head(q, k, v, r_sort, r_race, chunk: int, scale: Optional[float] = N
                  causal: bool = False) -> Dict[str, torch.Tensor]:
     """The whole operator on one (batch, head) unit.
 
-    q, k, v: [N, d] (any float dtype; upcast to fp64).  r_sort: [b_s, d];
-    r_race: [L, K_r, d].  ``codes`` may carry precomputed code_q / code_k /
-    rcode_q / rcode_k (used to re-run the float steps with another side's
-    codes where a projection sits within NEAR_ZERO of zero, and to freeze the
-    hash in gradient checks).  Returns every intermediate in token order."""
+    q, k, v: [N, d] (any float dtype; upcast to fp64).  r_sort: [b_s, d] for
+    one Sort-LSH hash round, or [R, b_s, d] for R rounds (several rounds are an
+    extension: sparse_branch_rounds); r_race: [L, K_r, d].  ``codes`` may
+    carry precomputed code_q / code_k / rcode_q / rcode_k (and round_code_q /
+    round_code_k [R, N] for several rounds; used to re-run the float steps with
+    another side's codes where a projection sits within NEAR_ZERO of zero, and
+    to freeze the hash in gradient checks).  Returns every intermediate in
+    token order."""
     q64, k64, v64 = q.to(F64), k.to(F64), v.to(F64)
     n, d = q64.shape
     L, kr, _ = r_race.shape
+    rounds = r_sort.shape[0] if r_sort.dim() == 3 else 1
+    r_sort0 = r_sort[0] if r_sort.dim() == 3 else r_sort
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     out: Dict[str, torch.Tensor] = {}
     if codes is None:
         with torch.no_grad():
-            pq_s, pk_s, pq_r, pk_r = _hash_all(q64.detach(), k64.detach(), r_sort, r_race)
+            pq_s, pk_s, pq_r, pk_r = _hash_all(q64.detach(), k64.detach(), r_sort0, r_race)
         code_q, code_k = simhash_codes(pq_s), simhash_codes(pk_s)
         rcode_q, rcode_k = simhash_codes(pq_r), simhash_codes(pk_r)
         near = [p.abs() < NEAR_ZERO for p in (pq_s, pk_s, pq_r, pk_r)]
@@ -329,12 +334,31 @@ def forward_head(q, k, v, r_sort, r_race, chunk: int, scale: Optional[float] = N
         out["near_code_k"] = near[1].any(dim=-1)
         out["near_rcode_q"] = near[2].any(dim=-1)
         out["near_rcode_k"] = near[3].any(dim=-1)
+        if rounds > 1:
+            with torch.no_grad():
+                proj_q = [simhash_projections(q64.detach(), r_sort[t]) for t in range(rounds)]
+                proj_k = [simhash_projections(k64.detach(), r_sort[t]) for t in range(rounds)]
+            round_code_q = torch.stack([simhash_codes(p) for p in proj_q])
+            round_code_k = torch.stack([simhash_codes(p) for p in proj_k])
+            out["near_round_code_q"] = torch.stack([(p.abs() < NEAR_ZERO).any(-1) for p in proj_q])
+            out["near_round_code_k"] = torch.stack([(p.abs() < NEAR_ZERO).any(-1) for p in proj_k])
     else:
         code_q, code_k = codes["code_q"].to(torch.int64), codes["code_k"].to(torch.int64)
         rcode_q, rcode_k = codes["rcode_q"].to(torch.int64), codes["rcode_k"].to(torch.int64)
+        if rounds > 1:
+            round_code_q = codes["round_code_q"].to(torch.int64)
+            round_code_k = codes["round_code_k"].to(torch.int64)
     perm_q = stable_sort_perm(sort_keys(code_q, sort_order))
     perm_k = stable_sort_perm(sort_keys(code_k, sort_order))
-    o_sp, lse = sparse_branch(q64, k64, v64, perm_q, perm_k, chunk, scale, lookback, causal)
+    if rounds == 1:
+        o_sp, lse = sparse_branch(q64, k64, v64, perm_q, perm_k, chunk, scale, lookback, causal)
+    else:
+        perms_q = [stable_sort_perm(sort_keys(c, sort_order)) for c in round_code_q]
+        perms_k = [stable_sort_perm(sort_keys(c, sort_order)) for c in round_code_k]
+        o_sp, lse = sparse_branch_rounds(q64, k64, v64, perms_q, perms_k, chunk, scale,
+                                         lookback, causal)
+        out.update(round_code_q=round_code_q, round_code_k=round_code_k,
+                   round_perm_q=torch.stack(perms_q), round_perm_k=torch.stack(perms_k))
     counts, sums = race_build(rcode_k, v64, 1 << kr)
     if causal:
         ctot, o_race, z_race = race_query_causal(rcode_q, rcode_k, v64)
@@ -377,7 +401,8 @@ def grads_head(q, k, v, r_sort, r_race, chunk: int, dy, scale: Optional[float] =
         first = forward_head(q, k, v, r_sort, r_race, chunk, scale, gate_w, gate_b, lam,
                              fixed_gates, sort_order=sort_order, lookback=lookback,
                              causal=causal)
-        codes = {name: first[name] for name in ("code_q", "code_k", "rcode_q", "rcode_k")}
+        codes = {name: first[name] for name in ("code_q", "code_k", "rcode_q", "rcode_k",
+                                                "round_code_q", "round_code_k") if name in first}
     out = forward_head(q64, k64, v64, r_sort, r_race, chunk, scale, gw, gb, lam64,
                        fixed_gates, codes=codes, sort_order=sort_order, lookback=lookback,
                        causal=causal)

@@ -20,6 +20,7 @@ bool make_geometry(const elsaa_params* p, Geometry* g, elsaa_status* why) {
     return false;
   if (p->lookback < 0 || p->lookback > 64) return false;
   if (p->causal != 0 && p->causal != 1) return false;
+  if (p->hash_rounds < 0 || p->hash_rounds > kMaxRounds) return false;
   if (p->race_tables < 1 || p->race_tables > 4096) return false;
   if (p->race_bits < 0 || p->race_bits > 16) return false;
   if ((int64_t)p->B * p->H * p->N * (p->d > p->race_tables ? p->d : p->race_tables) >
@@ -27,8 +28,11 @@ bool make_geometry(const elsaa_params* p, Geometry* g, elsaa_status* why) {
     return false;
   *why = ELSAA_ERR_UNSUPPORTED;
   if (p->d != 32 && p->d != 64 && p->d != 128) return false;
-  // the CUDA-core attention keeps a query's window of scores in shared memory
-  if ((int64_t)(p->lookback + 1) * p->chunk > 6144) return false;
+  // the CUDA-core attention keeps a query's windows of scores in shared memory
+  const int rounds = p->hash_rounds > 1 ? p->hash_rounds : 1;
+  if ((int64_t)rounds * (p->lookback + 1) * p->chunk > 6144) return false;
+  // extra rounds' sort codes: (rounds - 1) * sort_bits projections per row
+  if ((rounds - 1) * p->sort_bits > 128) return false;
   g->B = p->B;
   g->H = p->H;
   g->N = p->N;
@@ -49,12 +53,13 @@ bool make_geometry(const elsaa_params* p, Geometry* g, elsaa_status* why) {
   g->sort_order = p->sort_order;
   g->lookback = p->lookback;
   g->causal = p->causal;
+  g->rounds = rounds;
   g->sort_passes = p->sort_bits <= 8 ? 1 : 2;
   g->sort_digit_bits = (p->sort_bits + g->sort_passes - 1) / g->sort_passes;
   g->sort_bins = 1 << g->sort_digit_bits;
   g->sort_tiles = (p->N + kSortTile - 1) / kSortTile;
   g->tc_hash = hash_tc_supported(*g);
-  g->tc_attn = attn_tc_supported(*g);
+  g->tc_attn = attn_tc_supported(*g) && g->rounds == 1;
   if (g->causal && !race_causal_supported(*g)) return false;
   *why = ELSAA_OK;
   return true;
@@ -65,8 +70,8 @@ SavedLayout saved_layout(const Geometry& g) {
   const size_t bhn = (size_t)g.BH * g.N;
   size_t off = 0;
   auto take = [&](size_t bytes) { const size_t o = off; off = align_up(off + bytes); return o; };
-  s.code = take(2 * bhn * 2);
-  s.perm = take(2 * bhn * 4);
+  s.code = take((size_t)g.rounds * 2 * bhn * 2);
+  s.perm = take((size_t)g.rounds * 2 * bhn * 4);
   s.rcode = take(2 * bhn * g.L * g.rcode_bytes);
   s.rcode_t = take(2 * bhn * g.L * g.rcode_bytes);
   s.race_count = take((size_t)g.BH * g.L * g.NB * 4);
@@ -75,6 +80,7 @@ SavedLayout saved_layout(const Geometry& g) {
   s.o_sp = take(bhn * g.d * g.esz);
   s.o_race = take(bhn * g.d * g.esz);
   s.ctot = take(bhn * 4);
+  s.rank = take(g.rounds > 1 ? (size_t)g.rounds * 2 * bhn * 4 : 0);
   s.total = off;
   return s;
 }
@@ -179,6 +185,9 @@ elsaa_status elsaa_saved_views(const elsaa_params* p, const void* saved, elsaa_v
   out->o_sp = b + s.o_sp;
   out->o_race = b + s.o_race;
   out->ctot = (int32_t*)(b + s.ctot);
+  out->round_code = (uint16_t*)(b + s.code);
+  out->round_perm = (int32_t*)(b + s.perm);
+  out->hash_rounds = g.rounds;
   return ELSAA_OK;
 }
 
@@ -223,10 +232,16 @@ elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const vo
     ELSAA_TRY(launch_hash_tc(g, q, k, r_sort, r_race, code, rcode, rcode_t, err, s));
   else
     ELSAA_TRY(launch_hash_simt(g, q, k, r_sort, r_race, code, rcode, rcode_t, s));
+  // several hash rounds: the other rounds' sort codes
+  if (g.rounds > 1) ELSAA_TRY(launch_hash_sort_rounds(g, q, k, r_sort, code, s));
   ELSAA_TRY(mark(events, 1, s));
-  // 2. Sort-LSH order of Q and K
-  ELSAA_TRY(launch_sort(g, code, perm, (int32_t*)(w + wl.sort_hist), (int32_t*)(w + wl.sort_tmp),
-                        s));
+  // 2. Sort-LSH order of Q and K (every round), and with several rounds the
+  // inverse orders the attention uses to count each key once
+  for (int t = 0; t < g.rounds; ++t)
+    ELSAA_TRY(launch_sort(g, code + (size_t)t * 2 * bhn, perm + (size_t)t * 2 * bhn,
+                          (int32_t*)(w + wl.sort_hist), (int32_t*)(w + wl.sort_tmp), s));
+  int32_t* rank = g.rounds > 1 ? (int32_t*)(sv + sl.rank) : nullptr;
+  if (rank) ELSAA_TRY(launch_ranks(g, perm, rank, (int64_t)g.rounds * 2 * g.BH, s));
   ELSAA_TRY(mark(events, 2, s));
   if (g.causal) {
     // causal: the RACE read-out of query i takes keys j <= i only (a token
@@ -235,7 +250,7 @@ elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const vo
     int32_t* ct = (int32_t*)(sv + sl.ctot);
     ELSAA_TRY(mark(events, 3, s));   // (no separate build stage)
     ELSAA_TRY(launch_race_causal_fwd(g, rcode, rcode_k, v, num, ct, sums, counts, s));
-    ELSAA_TRY(launch_attn_fwd_simt(g, q, k, v, perm, perm + bhn, o_sp, lse, s));
+    ELSAA_TRY(launch_attn_fwd_simt(g, q, k, v, perm, perm + bhn, rank, o_sp, lse, s));
     ELSAA_TRY(mark(events, 4, s));
     ELSAA_TRY(launch_fuse_causal(g, q, o_sp, lse, num, ct, gate_w, gate_b, lambda, y,
                                  sv + sl.o_race, s));
@@ -256,7 +271,7 @@ elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const vo
   else if (g.tc_attn)
     ELSAA_TRY(launch_attn_fwd_tc(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s));
   else
-    ELSAA_TRY(launch_attn_fwd_simt(g, q, k, v, perm, perm + bhn, o_sp, lse, s));
+    ELSAA_TRY(launch_attn_fwd_simt(g, q, k, v, perm, perm + bhn, rank, o_sp, lse, s));
   ELSAA_TRY(mark(events, 4, s));
   // 5. RACE gather, gates, multiplier and output
   ELSAA_TRY(launch_race_fuse_fwd(g, q, rcode, gather_tables, counts, o_sp, lse, gate_w, gate_b,
@@ -301,6 +316,7 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
   const SavedLayout sl = saved_layout(g);
   const size_t bhn = (size_t)g.BH * g.N;
   const int32_t* perm = (const int32_t*)(sv + sl.perm);
+  const int32_t* rank = g.rounds > 1 ? (const int32_t*)(sv + sl.rank) : nullptr;
   const char* rcode = sv + sl.rcode;
   const char* rcode_k = rcode + bhn * g.L * g.rcode_bytes;
   const char* rcode_t = sv + sl.rcode_t;   // table-major query codes
@@ -362,8 +378,8 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
     ELSAA_TRY(launch_cast_out(g, dq_acc, dq, s));
   } else {
     ELSAA_TRY(cudaMemsetAsync(dk_acc, 0, bhn * g.d * 4, s));
-    ELSAA_TRY(launch_attn_bwd_simt(g, q, k, v, perm, perm + bhn, d_o, lse, dprime, dq_acc,
-                                   dk_acc, dv_acc, s));
+    ELSAA_TRY(launch_attn_bwd_simt(g, q, k, v, perm, perm + bhn, rank, d_o, lse, dprime,
+                                   dq_acc, dk_acc, dv_acc, s));
     ELSAA_TRY(mark(events, 3, s));
     ELSAA_TRY(launch_cast_out(g, dq_acc, dq, s));
     ELSAA_TRY(launch_cast_out(g, dk_acc, dk, s));
@@ -392,7 +408,10 @@ elsaa_status elsaa_kernel_launches(const elsaa_params* p, int32_t* fwd, int32_t*
   // hash 1, sort 3 per pass, |V| max 1 + RACE build 1, sparse 1, RACE gather + fusion 1
   // (local order: one kernel writes token order instead of the radix passes;
   // causal: one RACE token scan, then the sparse branch and the fusion)
-  const int sort = g.sort_order == ELSAA_SORT_LOCAL ? 1 : 3 * g.sort_passes;
+  // (several hash rounds: one more hash kernel, one sort per round and the
+  // inverse orders; zero-bit extra codes are a memset)
+  const int sort1 = g.sort_order == ELSAA_SORT_LOCAL ? 1 : 3 * g.sort_passes;
+  const int sort = g.rounds * sort1 + (g.rounds > 1 ? 1 + (g.sort_bits > 0 ? 1 : 0) : 0);
   *fwd = g.causal ? 1 + sort + 1 + 1 + 1 : 1 + sort + 2 + 1 + 1;
   // fusion backward 1, RACE build 1 + gather 1, sparse 1 (+ casts), reduction 1
   // (direct path: the sparse kernel writes dq itself and the gather adds into dv)

@@ -90,7 +90,93 @@ cudaError_t run(const Geometry& g, const void* q, const void* k, const void* r_s
   return cudaGetLastError();
 }
 
+// Sort codes of hash rounds 1 .. R-1 (several Sort-LSH rounds, an extension):
+// one warp per Q or K row, lane j of a group of 32 owns projection j of the
+// (R - 1) * sort_bits extra hyperplanes (round 1 + j / sort_bits, bit
+// j % sort_bits), fp64 sums of exact products as above.  code: [R][2 rows].
+template <typename T>
+__global__ void __launch_bounds__(256)
+hash_sort_rounds_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                        const T* __restrict__ r_sort, int64_t rows_per_tensor, int d,
+                        int sort_bits, int rounds, uint16_t* __restrict__ code) {
+  extern __shared__ float smem[];
+  const int warps = blockDim.x >> 5;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int P = (rounds - 1) * sort_bits;   // <= 7 * 16 = 112: at most four words
+  float* xs = smem + w * d;
+  const int64_t total = 2 * rows_per_tensor;
+  for (int64_t row = (int64_t)blockIdx.x * warps + w; row < total;
+       row += (int64_t)gridDim.x * warps) {
+    const T* src = row < rows_per_tensor ? q + row * d : k + (row - rows_per_tensor) * d;
+    for (int t = lane; t < d; t += 32) xs[t] = to_f32(src[t]);
+    __syncwarp();
+    uint32_t words[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int wi = 0; wi < 4; ++wi) {
+      const int j = wi * 32 + lane;
+      bool bit = false;
+      if (j < P) {
+        const T* r = r_sort + (size_t)(sort_bits + j) * d;   // rounds 1.. follow round 0
+        double acc = 0.0;
+        for (int t = 0; t < d; ++t) acc += (double)xs[t] * (double)to_f32(r[t]);
+        bit = acc > 0.0;
+      }
+      words[wi] = __ballot_sync(0xffffffffu, bit);
+    }
+    if (lane < rounds - 1) {
+      uint32_t v = 0;
+      for (int b = 0; b < sort_bits; ++b) {
+        const int p = lane * sort_bits + b;
+        v |= ((words[p >> 5] >> (p & 31)) & 1u) << b;
+      }
+      code[(int64_t)(lane + 1) * total + row] = (uint16_t)v;
+    }
+    __syncwarp();
+  }
+}
+
+// rank[seg][perm[seg][x]] = x
+__global__ void __launch_bounds__(256)
+rank_kernel(const int32_t* __restrict__ perm, int32_t* __restrict__ rank, int64_t total, int N) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t seg = i / N;
+    const int p = perm[i];
+    if (p >= 0 && p < N) rank[seg * N + p] = (int32_t)(i - seg * N);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_hash_sort_rounds(const Geometry& g, const void* q, const void* k,
+                                    const void* r_sort, uint16_t* code, cudaStream_t s) {
+  if (g.rounds <= 1) return cudaSuccess;
+  const int64_t rows = (int64_t)g.BH * g.N;
+  if (g.sort_bits == 0)   // zero-bit codes are all 0
+    return cudaMemsetAsync(code + 2 * rows, 0, (size_t)(g.rounds - 1) * 2 * rows * 2, s);
+  if ((g.rounds - 1) * g.sort_bits > 128) return cudaErrorInvalidValue;
+  const int threads = 256, warps = threads / 32;
+  const size_t smem = (size_t)warps * g.d * sizeof(float);
+  const int64_t blocks = (2 * rows + warps - 1) / warps;
+  const int grid = (int)(blocks < 148 * 64 ? blocks : 148 * 64);
+  if (g.bf16)
+    hash_sort_rounds_kernel<__nv_bfloat16><<<grid, threads, smem, s>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(r_sort), rows, g.d, g.sort_bits, g.rounds, code);
+  else
+    hash_sort_rounds_kernel<float><<<grid, threads, smem, s>>>(
+        static_cast<const float*>(q), static_cast<const float*>(k),
+        static_cast<const float*>(r_sort), rows, g.d, g.sort_bits, g.rounds, code);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ranks(const Geometry& g, const int32_t* perm, int32_t* rank, int64_t segs,
+                         cudaStream_t s) {
+  const int64_t total = segs * g.N;
+  const int64_t want = (total + 255) / 256;
+  rank_kernel<<<(int)(want < 148 * 8 ? want : 148 * 8), 256, 0, s>>>(perm, rank, total, g.N);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_hash_simt(const Geometry& g, const void* q, const void* k, const void* r_sort,
                              const void* r_race, uint16_t* code, void* rcode, void* rcode_t,

@@ -18,6 +18,8 @@ inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a
 // Sort-LSH radix pass geometry: digit of at most 8 bits, tiles of kSortTile keys.
 constexpr int kSortTile = 2048;
 constexpr int kSortThreads = 256;
+// Sort-LSH hash rounds the library serves.
+constexpr int kMaxRounds = 8;
 
 struct Geometry {
   int B, H, N, d, BH;
@@ -31,6 +33,7 @@ struct Geometry {
   int sort_order;      // elsaa_sort_order
   int lookback;        // previous chunks a query chunk attends (1: own and previous)
   int causal;          // keys j <= i only (sparse window and RACE read-out)
+  int rounds;          // Sort-LSH hash rounds R >= 1
   int sort_passes, sort_digit_bits, sort_bins, sort_tiles;
   bool tc_hash;       // tcgen05 kernel for the SimHash codes
   bool tc_attn;       // tcgen05 kernels for the sparse branch
@@ -38,10 +41,11 @@ struct Geometry {
 
 // Byte offsets inside the saved buffer.
 struct SavedLayout {
-  size_t code, perm, rcode, rcode_t, race_count, race_sum, lse, o_sp, o_race, ctot, total;
-  // code = [2][BH][N] u16 (queries then keys); perm = [2][BH][N] i32;
-  // rcode = [2][BH][N][L] (u8 or u16); rcode_t = the same codes table-major,
-  // [2][BH][L][N]
+  size_t code, perm, rcode, rcode_t, race_count, race_sum, lse, o_sp, o_race, ctot, rank, total;
+  // code = [R][2][BH][N] u16 (per hash round: queries then keys); perm =
+  // [R][2][BH][N] i32; rcode = [2][BH][N][L] (u8 or u16); rcode_t = the same
+  // codes table-major, [2][BH][L][N]; rank = the inverse permutations
+  // [R][2][BH][N] i32 (0 bytes for one round)
 };
 
 // Byte offsets inside the workspace.
@@ -81,6 +85,14 @@ cudaError_t launch_hash_tc(const Geometry& g, const void* q, const void* k, cons
                            uint32_t* err, cudaStream_t s);
 bool hash_tc_supported(const Geometry& g);
 
+// Sort codes of hash rounds 1 .. R-1 (round 0 comes with the main hash):
+// code[t][2][BH][N] from r_sort[t] ([R][sort_bits][d]), on CUDA cores.
+cudaError_t launch_hash_sort_rounds(const Geometry& g, const void* q, const void* k,
+                                    const void* r_sort, uint16_t* code, cudaStream_t s);
+// rank[seg][perm[seg][x]] = x over `segs` segments of N.
+cudaError_t launch_ranks(const Geometry& g, const int32_t* perm, int32_t* rank, int64_t segs,
+                         cudaStream_t s);
+
 // Stable Sort-LSH order of the 2*BH code segments.
 cudaError_t launch_sort(const Geometry& g, const uint16_t* code, int32_t* perm, int32_t* hist,
                         int32_t* tmp, cudaStream_t s);
@@ -115,14 +127,17 @@ cudaError_t launch_race_fuse_fwd(const Geometry& g, const void* q, const void* r
                                  const float* gate_b, const float* lam, void* y, void* o_race,
                                  int32_t* ctot, cudaStream_t s);
 
-// Sparse branch, CUDA-core kernels.
+// Sparse branch, CUDA-core kernels.  perm_q / perm_k are round 0's; with
+// g.rounds > 1 round t's permutations sit t * 2 BH N further, and `rank`
+// holds every round's inverse permutations ([R][2][BH][N]; unused for one round).
 cudaError_t launch_attn_fwd_simt(const Geometry& g, const void* q, const void* k, const void* v,
-                                 const int32_t* perm_q, const int32_t* perm_k, void* o_sp,
-                                 float* lse, cudaStream_t s);
+                                 const int32_t* perm_q, const int32_t* perm_k,
+                                 const int32_t* rank, void* o_sp, float* lse, cudaStream_t s);
 cudaError_t launch_attn_bwd_simt(const Geometry& g, const void* q, const void* k, const void* v,
-                                 const int32_t* perm_q, const int32_t* perm_k, const void* d_o,
-                                 const float* lse, const float* dprime, float* dq_acc,
-                                 float* dk_acc, float* dv_acc, cudaStream_t s);
+                                 const int32_t* perm_q, const int32_t* perm_k,
+                                 const int32_t* rank, const void* d_o, const float* lse,
+                                 const float* dprime, float* dq_acc, float* dk_acc,
+                                 float* dv_acc, cudaStream_t s);
 // Sparse branch, tcgen05 kernels.
 cudaError_t launch_attn_fwd_tc(const Geometry& g, const void* q, const void* k, const void* v,
                                const int32_t* perm_q, const int32_t* perm_k, void* o_sp,

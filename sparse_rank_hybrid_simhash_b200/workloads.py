@@ -58,6 +58,7 @@ class Workload:
     sort_order: str = "binary"   # binary | gray | local (Sort-LSH bucket order)
     lookback: int = 1            # previous sorted chunks a query chunk attends
     causal: bool = False         # keys j <= i only
+    hash_rounds: int = 1         # Sort-LSH hash rounds (each with its own hyperplanes)
 
     @property
     def torch_dtype(self):
@@ -121,7 +122,8 @@ def _qk_zipf(rng, B, H, N, d, prototypes=512, s=1.1):
 def make_inputs(w: Workload, seed: Optional[int] = None, with_dy: Optional[bool] = None,
                 device="cpu") -> Dict[str, torch.Tensor]:
     """Draw every input of one workload.  Returns torch tensors:
-    q, k, v [B, H, N, d] and r_sort [b_s, d], r_race [L, K_r, d] in the
+    q, k, v [B, H, N, d] and r_sort [b_s, d] (one hash round; [R, b_s, d] for
+    R rounds, round 0 the same draw as for one round), r_race [L, K_r, d] in the
     workload dtype; gate_w [2, d], gate_b [2], lam [1] in fp32; dy (same shape
     and dtype as q) when the workload has a backward; for the needle workload
     also needle_key [B, H] and needle_query [B, H] (token indices)."""
@@ -160,6 +162,11 @@ def make_inputs(w: Workload, seed: Optional[int] = None, with_dy: Optional[bool]
     if with_dy if with_dy is not None else w.backward:
         out["dy"] = torch.from_numpy(_normal(rng, (B, H, N, d))).to(dt)
     out.update(extra)
+    if w.hash_rounds > 1:
+        # the other rounds' hyperplanes are drawn last, so every other input
+        # keeps its one-round values
+        more = _normal(rng, (w.hash_rounds - 1, w.sort_bits, d))
+        out["r_sort"] = torch.cat([out["r_sort"][None], torch.from_numpy(more).to(dt)], 0)
     if device != "cpu":
         out = {kk: t.to(device) for kk, t in out.items()}
     return out

@@ -81,6 +81,8 @@ def test_validation_rejects_bad_problems():
         dict(lookback=-1),
         dict(lookback=65),
         dict(causal=2),
+        dict(hash_rounds=-1),
+        dict(hash_rounds=9),
         dict(N=0),                   # empty sequence
         dict(B=0),
         dict(H=-1),
@@ -102,6 +104,17 @@ def test_validation_rejects_bad_problems():
     p = B.Params.make(1, 2, 8192, 64, "bf16", 4, 1024, 8, 6, lookback=6)
     assert B.validate(p) == 2
     assert B.validate(B.Params.make(1, 2, 256, 64, "bf16", 4, 64, 8, 8, causal=True)) == 0
+    # several hash rounds: R windows of scores per query in shared memory
+    for r in (0, 1, 2, 8):
+        assert B.validate(B.Params.make(1, 2, 256, 64, "bf16", 4, 64, 8, 6, hash_rounds=r)) == 0
+    assert B.validate(B.Params.make(1, 2, 8192, 64, "bf16", 4, 1024, 8, 6, hash_rounds=4)) == 2
+    # one round: 0 and 1 are the same problem with the same saved layout
+    p0 = B.Params.make(1, 2, 256, 64, "bf16", 4, 64, 8, 6, hash_rounds=0)
+    p1 = B.Params.make(1, 2, 256, 64, "bf16", 4, 64, 8, 6, hash_rounds=1)
+    assert B.saved_bytes(p0) == B.saved_bytes(p1)
+    p3 = B.Params.make(1, 2, 256, 64, "bf16", 4, 64, 8, 6, hash_rounds=3)
+    # codes, orders and inverse orders of two more rounds
+    assert B.saved_bytes(p3) >= B.saved_bytes(p1) + 2 * 2 * 512 * (2 + 4) + 3 * 2 * 512 * 4
     # the causal RACE scan keeps one table in shared memory
     assert B.validate(B.Params.make(1, 2, 256, 128, "bf16", 4, 64, 8, 9, causal=True)) == 2
 
@@ -153,3 +166,7 @@ def test_kernel_launch_counts():
     # causal: token scan instead of |V| max + build; CUDA-core sparse backward + 3 casts
     c = B.kernel_launches(B.Params.from_workload(w.replace(causal=True)))
     assert c == (1 + 3 + 1 + 1 + 1, 1 + 1 + 4 + 1)
+    # three hash rounds: one more hash kernel, three sorts, the inverse orders;
+    # CUDA-core sparse backward + 3 casts
+    r = B.kernel_launches(B.Params.from_workload(w.replace(hash_rounds=3)))
+    assert r == (1 + 1 + 3 * 3 + 1 + 2 + 1 + 1, 1 + 2 + 1 + 3 + 1)

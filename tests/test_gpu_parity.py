@@ -79,6 +79,17 @@ def test_sort_orders(cuda_device, order, sort_bits):
     _run(w, backward=True)
 
 
+@pytest.mark.parametrize("rounds,dtype,order,causal", [(2, "bf16", "binary", False),
+                                                       (3, "bf16", "gray", False),
+                                                       (3, "f32", "binary", True)])
+def test_hash_rounds(cuda_device, rounds, dtype, order, causal):
+    # several Sort-LSH hash rounds: every round's codes and orders, and the
+    # attention over the union of the rounds' windows (each key once)
+    w = WORKLOADS["iid-4k"].replace(B=1, H=2, N=512, chunk=32, dtype=dtype, sort_order=order,
+                                    causal=causal, hash_rounds=rounds)
+    _run(w, backward=True)
+
+
 @pytest.mark.parametrize("lookback,dtype", [(0, "bf16"), (2, "bf16"), (3, "f32")])
 def test_lookback(cuda_device, lookback, dtype):
     # windows of lookback previous chunks plus the own one (CUDA-core attention)

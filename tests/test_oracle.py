@@ -633,3 +633,43 @@ def test_rounds_union_brute_force():
         p = torch.softmax(s, 0)
         assert abs(float(lse[i]) - float(torch.logsumexp(s, 0))) < 1e-12
         assert torch.allclose(o[i], sum(p[t] * v[j] for t, j in enumerate(keys)), atol=1e-12)
+
+
+def test_rounds_through_forward_head():
+    """forward_head with [R, b_s, d] hyperplanes: one round in 3-D form is the
+    2-D one-round operator; a repeated round changes nothing; two distinct
+    rounds give the union-window sparse branch, the same RACE branch and
+    round 0's codes as the one-round call."""
+    n, d, c, L, kr = 64, 6, 16, 3, 2
+    q, k, v, rs, rr, gw, gb = _unit(n, d, c, 3, L, kr, seed=120)
+    one = O.forward_head(q, k, v, rs, rr, c, None, gw, gb, 0.8)
+    one3 = O.forward_head(q, k, v, rs[None], rr, c, None, gw, gb, 0.8)
+    assert torch.equal(one["y"], one3["y"])
+    rep = O.forward_head(q, k, v, torch.stack([rs, rs]), rr, c, None, gw, gb, 0.8)
+    assert torch.allclose(rep["y"], one["y"], atol=1e-13, rtol=0)
+    rs2 = torch.stack([rs, rnd(tuple(rs.shape), 121)])
+    two = O.forward_head(q, k, v, rs2, rr, c, None, gw, gb, 0.8)
+    assert torch.equal(two["code_q"], one["code_q"]) and torch.equal(two["round_code_q"][0],
+                                                                     one["code_q"])
+    assert torch.equal(two["o_race"], one["o_race"])
+    pq, pk = O.round_perms(q, k, rs2)
+    o, lse = O.sparse_branch_rounds(q.to(F64), k.to(F64), v.to(F64), pq, pk, c,
+                                    1 / math.sqrt(d))
+    assert torch.allclose(two["o_sp"], o, atol=1e-13, rtol=0)
+    assert torch.all(two["lse"] >= one["lse"] - 1e-12) and bool((two["lse"] > one["lse"]).any())
+
+
+def test_rounds_gradients_match_finite_differences():
+    n, d, c, L, kr = 16, 4, 4, 2, 2
+    q, k, v, rs, rr, gw, gb = _unit(n, d, c, 2, L, kr, seed=130)
+    rs2 = torch.stack([rs, rnd(tuple(rs.shape), 131)])
+    first = O.forward_head(q, k, v, rs2, rr, c, None, gw, gb, 0.7)
+    codes = {x: first[x] for x in ("code_q", "code_k", "rcode_q", "rcode_k", "round_code_q",
+                                   "round_code_k")}
+
+    def f(q_, k_, v_, w_, b_, lam_):
+        return O.forward_head(q_, k_, v_, rs2, rr, c, None, w_, b_, lam_, codes=codes)["y"]
+
+    args = tuple(t.clone().requires_grad_(True) for t in (q, k, v, gw, gb))
+    lam = torch.tensor(0.7, dtype=F64, requires_grad=True)
+    assert torch.autograd.gradcheck(f, args + (lam,), eps=1e-6, atol=1e-7)
