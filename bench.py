@@ -10,7 +10,7 @@ synthetic tensors resident in HBM before the timed region.
                     [--workload NAME] [--mode elsaa|sort_lsh_race|race_only|sparse_only]
                     [--sort-order binary|gray|local] [--lookback L] [--hash-rounds R]
                     [--causal]
-                    [--dense-context] [--no-cpu-baseline]
+                    [--dense-context] [--no-cpu-baseline] [--no-other-workloads]
 
 The modes are the method's ablations on the same kernels (lambda = 0, or one
 branch gated off); sort order, lookback and causal select the extensions of
@@ -160,6 +160,56 @@ def operator_roofline(w, peaks):
             "fwdbwd_us": 1e6 * max((f_fwd + f_bwd) / tf, b_all / hb),
             "flops_fwd": f_fwd, "flops_fwdbwd": f_fwd + f_bwd, "bytes_fwd": b_fwd,
             "bytes_fwdbwd": b_all}
+
+
+def interaction_count(w):
+    """Query-key and query-bucket interactions one step performs ("Two
+    Efficient Attentions, One Denominator Problem", section "Linear
+    interactions are not yet production economics": the count grows linearly
+    in N; the formula itself is lost, the 32K example survives): every query
+    scores the keys of its Sort-LSH window (own and previous chunk; with R hash
+    rounds at most R windows) and reads one bucket in each of the L RACE
+    tables."""
+    BH, N = w.B * w.H, w.N
+    sparse = window_keys(N, w.chunk, w.lookback) * max(1, w.hash_rounds) / N
+    race = w.race_tables
+    return {"per_query": sparse + race, "sparse_per_query": sparse, "race_per_query": race,
+            "per_step": (sparse + race) * BH * N, "dense_per_query": N,
+            "fraction_of_dense": (sparse + race) / N,
+            "note": "sparse = window keys (upper bound with several hash rounds), race = L"}
+
+
+# Stages whose table lines move through on-chip memory, not HBM: every row
+# reads (or adds) one line of d values per table.  The gathers of the forward
+# read-out and of the value gradient run from shared-memory slabs (where they
+# fit); the table builds sum value rows gathered from L2.
+RACE_ONCHIP = {"race_build": "l2", "race_fuse": "smem", "race_bwd": "l2", "finish": "smem"}
+# measured row-gather rate of an L2-resident table (independent 16-byte loads
+# of random 128-byte rows, 592-1184 CTAs on a B200)
+L2_GATHER_GBS = 20000.0
+
+
+def race_onchip_bound(w, stage_ms, sm_mhz, slab_ok):
+    """Each RACE stage against its on-chip bound: bytes of table lines per
+    pass (rows x L x d x element size of the bf16 tables) over the stage time,
+    against shared-memory bandwidth (148 SMs x 128 B per clock x the sampled
+    SM clock) for the slab gathers, or the measured L2 row-gather rate."""
+    BH, N, d, L = w.B * w.H, w.N, w.d, w.race_tables
+    nbytes = BH * N * L * d * 2.0
+    smem_gbs = 148 * 128 * (sm_mhz or 1965.0) * 1e6 / 1e9
+    out = {}
+    for st, kind in RACE_ONCHIP.items():
+        if st not in stage_ms or stage_ms[st] <= 0:
+            continue
+        if kind == "smem" and not slab_ok:
+            kind = "l2"
+        peak = smem_gbs if kind == "smem" else L2_GATHER_GBS
+        ach = nbytes / (stage_ms[st] / 1e3) / 1e9
+        out[st] = {"onchip_bytes": nbytes, "achieved_GBs": round(ach, 1),
+                   "peak_GBs": round(peak, 1), "frac": round(ach / peak, 4),
+                   "peak_kind": ("shared memory: 148 SMs x 128 B/clk x SM clock" if kind == "smem"
+                                 else "L2 row gather, measured")}
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -396,10 +446,15 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         total_ms, fwd_total = DP.max_over_ranks([total_ms, fwd_total], dev)
 
+    views = B.saved_views(p, saved)
+    dev_unit = {"y": y[0, 0].cpu()}
+    dev_unit.update({k: views[k][0, 0].cpu() for k in ("code_q", "code_k", "rcode_q", "rcode_k")})
+    del saved, ws, grads, flush
+    torch.cuda.empty_cache()
     # end to end through the public API with host buffers
     e2e = run_e2e(args, w, p, inp, dev, world)
     context = time_dense_sdpa(w, d) if args.dense_context and world == 1 else None
-    return w, p, total_ms, fwd_total, stage_ms, clk.summary(), e2e, context
+    return w, p, total_ms, fwd_total, stage_ms, clk.summary(), e2e, context, dev_unit
 
 
 def run_e2e(args, w, p, inp, dev, world):
@@ -449,6 +504,65 @@ def run_e2e(args, w, p, inp, dev, world):
 
 
 # ---------------------------------------------------------------------------
+# the other workloads, device-timed (context for the headline)
+# ---------------------------------------------------------------------------
+
+def time_workload(name, dev, steps=5, warmup=3):
+    """Forward (and forward + backward where the workload has one) of another
+    workload at full size, device-timed with CUDA events and an L2 flush
+    between steps; tokens/s and the operator-roofline fractions."""
+    w = WORKLOADS[name]
+    p = B.Params.from_workload(w)
+    d = {k: t.to(dev) for k, t in make_inputs(w, with_dy=w.backward).items()}
+    saved = B.alloc_saved(p, dev)
+    ws = B.alloc_workspace(p, dev)
+    y = torch.empty_like(d["q"])
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def fwd():
+        B.forward(p, d["q"], d["k"], d["v"], d["r_sort"], d["r_race"], d["gate_w"],
+                  d["gate_b"], d["lam"], y=y, saved=saved, ws=ws)
+
+    def bwd():
+        B.backward(p, d["q"], d["k"], d["v"], d["r_sort"], d["r_race"], d["gate_w"],
+                   d["gate_b"], d["lam"], saved, d["dy"], ws=ws)
+
+    for _ in range(warmup):
+        fwd()
+        if w.backward:
+            bwd()
+    torch.cuda.synchronize()
+    B.check(ws)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for e in ev:
+        flush.fill_(1)
+        e[0].record()
+        fwd()
+        e[1].record()
+        if w.backward:
+            bwd()
+        e[2].record()
+    torch.cuda.synchronize()
+    B.check(ws)
+    peaks = load_peaks()
+    roof = operator_roofline(w, peaks)
+    f_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    out = {"shape": f"B{w.B} H{w.H} N{w.N} d{w.d} {w.dtype}", "fwd_ms": round(f_ms, 4),
+           "fwd_tokens_per_s": w.tokens / (f_ms / 1e3),
+           "fwd_roofline_us": round(roof["fwd_us"], 2),
+           "fwd_roofline_frac": roof["fwd_us"] / (1e3 * f_ms),
+           "path": B.path_flags(p), "steps": steps}
+    if w.backward:
+        fb_ms = statistics.mean(e[0].elapsed_time(e[2]) for e in ev)
+        out.update({"fwdbwd_ms": round(fb_ms, 4), "fwdbwd_tokens_per_s": w.tokens / (fb_ms / 1e3),
+                    "fwdbwd_roofline_us": round(roof["fwdbwd_us"], 2),
+                    "fwdbwd_roofline_frac": roof["fwdbwd_us"] / (1e3 * fb_ms)})
+    del d, saved, ws, y, flush
+    torch.cuda.empty_cache()
+    return out
+
+
+# ---------------------------------------------------------------------------
 # the oracle as CPU baseline and as the reference arm
 # ---------------------------------------------------------------------------
 
@@ -465,9 +579,12 @@ def oracle_unit_seconds(w, inp, units):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w, min_seconds=10.0):
+def cpu_baseline(w, min_seconds=10.0, device_unit=None):
     """The oracle on the host cores over (batch, head) units of the workload,
-    one after another until at least min_seconds of CPU work (or every unit)."""
+    one after another until at least min_seconds of CPU work (or every unit).
+    With ``device_unit`` (unit (0, 0) of the timed device run: y and the
+    codes), the oracle's forward of that unit also gives the parity figures of
+    the bench line (outside the timed oracle calls)."""
     cores = len(os.sched_getaffinity(0))
     torch.set_num_threads(cores)
     inp = make_inputs(w, with_dy=True)
@@ -478,10 +595,34 @@ def cpu_baseline(w, min_seconds=10.0):
         units += 1
     # one (batch, head) unit is N / H token-equivalents of the B x N-token step
     value = units * w.N / w.H / secs
-    return {"value": value, "unit": "tokens/s", "cores": torch.get_num_threads(),
-            "kind": "oracle",
-            "sample": f"{units} of {w.B * w.H} (batch, head) units of {w.name}, forward+backward "
-                      f"in fp64 ({secs:.1f} s), scaled to the whole step"}
+    out = {"value": value, "unit": "tokens/s", "cores": torch.get_num_threads(),
+           "kind": "oracle",
+           "sample": f"{units} of {w.B * w.H} (batch, head) units of {w.name}, forward+backward "
+                     f"in fp64 ({secs:.1f} s), scaled to the whole step"}
+    if device_unit is not None:
+        out["parity_unit"] = parity_sample(w, inp, device_unit)
+    return out
+
+
+def parity_sample(w, inp, dev_unit):
+    """Unit (0, 0) of the timed run against the oracle: code mismatches, codes
+    whose projection lies within rounding of zero, and rel-L2 / max-abs of y."""
+    import oracle as O
+    fixed = (w.gate_s, w.gate_r) if w.gate_fixed else None
+    ref = O.forward_head(inp["q"][0, 0], inp["k"][0, 0], inp["v"][0, 0], inp["r_sort"],
+                         inp["r_race"], w.chunk, None, inp["gate_w"], inp["gate_b"],
+                         float(inp["lam"][0]), fixed, sort_order=w.sort_order,
+                         lookback=w.lookback, causal=w.causal)
+    mism, near, total = 0, 0, 0
+    for key in ("code_q", "code_k", "rcode_q", "rcode_k"):
+        got = dev_unit[key].to(torch.int64) & 0xFFFF
+        mism += int((got != ref[key]).sum())
+        near += int(ref["near_" + key].sum())
+        total += ref[key].numel()
+    y, ry = dev_unit["y"].double(), ref["y"]
+    return {"unit": "(0, 0)", "codes": total, "code_mismatches": mism,
+            "near_zero_projections": near, "y_rel_l2": float((y - ry).norm() / ry.norm()),
+            "y_max_abs": float((y - ry).abs().max())}
 
 
 def run_reference(args):
@@ -531,6 +672,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the device timing of iid-4k, vision-16k and needle-256k")
     ap.add_argument("--mode", default="elsaa", choices=sorted(MODES),
                     help="ablation / single-branch setting of the gates and lambda")
     ap.add_argument("--sort-order", default="binary", choices=["binary", "gray", "local"],
@@ -561,7 +704,8 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
-    w, p, total_ms, fwd_ms, stage_ms, clocks, e2e, context = run_ours(args, rank, world, local_rank)
+    w, p, total_ms, fwd_ms, stage_ms, clocks, e2e, context, dev_unit = run_ours(
+        args, rank, world, local_rank)
     peaks = load_peaks()
     if rank == 0:
         K = args.steps
@@ -599,10 +743,17 @@ def main():
             "clocks": clocks,
             "e2e": e2e,
         }
+        line["interactions"] = interaction_count(w)
+        line["race_onchip"] = race_onchip_bound(w, stage_ms, clocks.get("sm_mhz"),
+                                                B.path_flags(p)["slab_fwd"])
+        line["path"] = B.path_flags(p)
         if context is not None:
             line["context"] = {"dense_sdpa": context}
+        if world == 1 and not args.no_other_workloads and args.workload == WORKLOAD:
+            line["other_workloads"] = {name: time_workload(name, torch.device("cuda", local_rank))
+                                       for name in ("iid-4k", "vision-16k", "needle-256k")}
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(w)
+            line["cpu_baseline"] = cpu_baseline(w, device_unit=dev_unit)
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()

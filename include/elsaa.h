@@ -241,6 +241,17 @@ const char* elsaa_status_str(elsaa_status s);
  * dims other than 64/128, or chunk shapes the tensor kernels do not tile). */
 int32_t elsaa_uses_tensor_cores(const elsaa_params* p);
 
+/* Bit mask of the kernel families elsaa_forward / elsaa_backward take for
+ * `p` (0 if p is invalid): ELSAA_PATH_TC_HASH the tcgen05 SimHash GEMM;
+ * ELSAA_PATH_TC_ATTN the tcgen05 sparse branch; ELSAA_PATH_SLAB_FWD the RACE
+ * read-out from shared-memory table slabs (gate logits from the hash GEMM);
+ * ELSAA_PATH_SLAB_BWD the RACE value gradient from shared-memory slabs. */
+#define ELSAA_PATH_TC_HASH 1
+#define ELSAA_PATH_TC_ATTN 2
+#define ELSAA_PATH_SLAB_FWD 4
+#define ELSAA_PATH_SLAB_BWD 8
+int32_t elsaa_path_flags(const elsaa_params* p);
+
 #ifdef __cplusplus
 }
 #endif

@@ -76,7 +76,9 @@ class Views(ctypes.Structure):
 EXPORTS = ("elsaa_validate", "elsaa_workspace_bytes", "elsaa_saved_bytes", "elsaa_forward",
            "elsaa_backward", "elsaa_forward_staged", "elsaa_backward_staged",
            "elsaa_kernel_launches", "elsaa_saved_views", "elsaa_check", "elsaa_status_str",
-           "elsaa_uses_tensor_cores", "elsaa_sort_codes_noalloc")
+           "elsaa_uses_tensor_cores", "elsaa_sort_codes_noalloc", "elsaa_path_flags")
+# elsaa_path_flags bits
+PATH_FLAGS = {"tc_hash": 1, "tc_attn": 2, "slab_fwd": 4, "slab_bwd": 8}
 FWD_STAGES = ("hash", "sort", "race_build", "sparse_fwd", "race_fuse")
 BWD_STAGES = ("fuse_bwd", "race_bwd", "sparse_bwd", "finish")
 
@@ -98,6 +100,7 @@ def lib() -> ctypes.CDLL:
     L.elsaa_workspace_bytes.argtypes, L.elsaa_workspace_bytes.restype = [P], sz
     L.elsaa_saved_bytes.argtypes, L.elsaa_saved_bytes.restype = [P], sz
     L.elsaa_uses_tensor_cores.argtypes, L.elsaa_uses_tensor_cores.restype = [P], ctypes.c_int32
+    L.elsaa_path_flags.argtypes, L.elsaa_path_flags.restype = [P], ctypes.c_int32
     L.elsaa_forward.argtypes = [P] + [vp] * 10 + [vp, sz, vp]
     L.elsaa_forward.restype = st
     L.elsaa_backward.argtypes = [P] + [vp] * 17 + [sz, vp]
@@ -147,6 +150,12 @@ def saved_bytes(p: Params) -> int:
 
 def uses_tensor_cores(p: Params) -> bool:
     return bool(lib().elsaa_uses_tensor_cores(ctypes.byref(p)))
+
+
+def path_flags(p: Params) -> Dict[str, bool]:
+    """Which kernel families the operator takes for ``p`` (elsaa_path_flags)."""
+    f = lib().elsaa_path_flags(ctypes.byref(p))
+    return {name: bool(f & bit) for name, bit in PATH_FLAGS.items()}
 
 
 def kernel_launches(p: Params):

@@ -95,6 +95,7 @@ WorkLayout work_layout(const Geometry& g) {
   w.sort_tmp = take(2 * bhn * 4);
   w.absmax = take((size_t)2 * g.BH * 4);
   w.gtab = take((size_t)g.BH * g.L * g.NB * g.d * 2);
+  w.gl = take(bhn * sizeof(float2));
   w.causal_num = take(g.causal ? bhn * g.d * 4 : 0);
   const size_t shared_base = off;
   // forward without a saved buffer: the saved layout lives here
@@ -126,6 +127,19 @@ inline cudaError_t mark(void* const* events, int i, cudaStream_t s) {
   if (!events || !events[i]) return cudaSuccess;
   return cudaEventRecord((cudaEvent_t)events[i], s);
 }
+
+// The RACE read-out runs from shared-memory table slabs where they fit; it
+// takes the learned gates' logits from the hash GEMM.
+bool slab_fwd(const Geometry& g) {
+  return g.tc_hash && !g.causal && race_slab_supported(g, true) &&
+         (g.gate_fixed || hash_tc_gate_logits_supported(g));
+}
+// The persistent sparse backward writes dq, dk and dv itself; the RACE
+// branch's dv is then added in place by a key-code gather.
+bool direct_bwd(const Geometry& g) {
+  return g.tc_attn && attn_bwd3_supported(g) && race_gather_add_supported(g);
+}
+bool slab_bwd(const Geometry& g) { return direct_bwd(g) && race_slab_supported(g, false); }
 
 #define ELSAA_TRY(expr)                               \
   do {                                                \
@@ -227,9 +241,11 @@ elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const vo
   ELSAA_TRY(cudaMemsetAsync(err, 0, sizeof(uint32_t), s));
   ELSAA_TRY(mark(events, 0, s));
 
-  // 1. SimHash codes of Q and K
+  const bool slab = slab_fwd(g);
+  float2* gl = (slab && !g.gate_fixed) ? (float2*)(w + wl.gl) : nullptr;
+  // 1. SimHash codes of Q and K (and the gate logits)
   if (g.tc_hash)
-    ELSAA_TRY(launch_hash_tc(g, q, k, r_sort, r_race, code, rcode, rcode_t, err, s));
+    ELSAA_TRY(launch_hash_tc(g, q, k, r_sort, r_race, code, rcode, rcode_t, gate_w, gl, err, s));
   else
     ELSAA_TRY(launch_hash_simt(g, q, k, r_sort, r_race, code, rcode, rcode_t, s));
   // several hash rounds: the other rounds' sort codes
@@ -274,10 +290,15 @@ elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const vo
     ELSAA_TRY(launch_attn_fwd_simt(g, q, k, v, perm, perm + bhn, rank, o_sp, lse, s));
   ELSAA_TRY(mark(events, 4, s));
   // 5. RACE gather, gates, multiplier and output
-  ELSAA_TRY(launch_race_fuse_fwd(g, q, rcode, gather_tables, counts, o_sp, lse, gate_w, gate_b,
-                                 lambda, y,
-                                 saved ? sv + sl.o_race : nullptr,
-                                 saved ? (int32_t*)(sv + sl.ctot) : nullptr, s));
+  if (slab)
+    ELSAA_TRY(launch_race_slab_fuse(g, rcode, gather_tables, counts, o_sp, lse, gl, gate_b,
+                                    lambda, y, saved ? sv + sl.o_race : nullptr,
+                                    saved ? (int32_t*)(sv + sl.ctot) : nullptr, err, s));
+  else
+    ELSAA_TRY(launch_race_fuse_fwd(g, q, rcode, gather_tables, counts, o_sp, lse, gate_w, gate_b,
+                                   lambda, y,
+                                   saved ? sv + sl.o_race : nullptr,
+                                   saved ? (int32_t*)(sv + sl.ctot) : nullptr, s));
   ELSAA_TRY(mark(events, 5, s));
   return ELSAA_OK;
 }
@@ -337,7 +358,7 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
 
   // The persistent sparse backward writes dq, dk and dv itself; the RACE
   // branch's dv is then added in place by the key-code gather.
-  const bool direct = g.tc_attn && attn_bwd3_supported(g) && race_gather_add_supported(g);
+  const bool direct = direct_bwd(g);
   __nv_bfloat16* gtab = g.bf16 ? (__nv_bfloat16*)(w + wl.gtab) : nullptr;
   const void* race_grad = g.bf16 ? (const void*)gtab : (const void*)d_t;
   // 1. fusion and gate backward: dO_sp, D', the gate part of dq, g_r dy / Ctot
@@ -365,7 +386,10 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
                                g.gate_fixed ? nullptr : gate_w, dq, dk, dv,
                                (uint32_t*)(w + wl.err), s));
     ELSAA_TRY(mark(events, 3, s));
-    ELSAA_TRY(launch_race_gather_add(g, rcode_k, race_grad, dv, s));
+    if (slab_bwd(g))
+      ELSAA_TRY(launch_race_slab_add(g, rcode_k, race_grad, dv, (uint32_t*)(w + wl.err), s));
+    else
+      ELSAA_TRY(launch_race_gather_add(g, rcode_k, race_grad, dv, s));
   } else if (g.tc_attn && attn_bwd2_supported(g)) {
     ELSAA_TRY(launch_attn_bwd2(g, q, k, v, perm, perm + bhn, d_o, lse, dprime, dv_acc, dq_acc,
                                dk, dv, (uint32_t*)(w + wl.err), s));
@@ -415,10 +439,18 @@ elsaa_status elsaa_kernel_launches(const elsaa_params* p, int32_t* fwd, int32_t*
   *fwd = g.causal ? 1 + sort + 1 + 1 + 1 : 1 + sort + 2 + 1 + 1;
   // fusion backward 1, RACE build 1 + gather 1, sparse 1 (+ casts), reduction 1
   // (direct path: the sparse kernel writes dq itself and the gather adds into dv)
-  const bool direct = g.tc_attn && attn_bwd3_supported(g) && race_gather_add_supported(g);
+  const bool direct = direct_bwd(g);
   const int sparse = direct ? 1 : g.tc_attn ? 1 + 1 : 1 + 3;
   *bwd = 1 + (g.causal ? 1 : 2) + sparse + 1;
   return ELSAA_OK;
+}
+
+int32_t elsaa_path_flags(const elsaa_params* p) {
+  Geometry g;
+  elsaa_status why;
+  if (!make_geometry(p, &g, &why)) return 0;
+  return (g.tc_hash ? ELSAA_PATH_TC_HASH : 0) | (g.tc_attn ? ELSAA_PATH_TC_ATTN : 0) |
+         (slab_fwd(g) ? ELSAA_PATH_SLAB_FWD : 0) | (slab_bwd(g) ? ELSAA_PATH_SLAB_BWD : 0);
 }
 
 elsaa_status elsaa_check(void* ws, void* stream) {

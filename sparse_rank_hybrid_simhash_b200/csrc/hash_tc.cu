@@ -17,6 +17,13 @@
 // 32-bit word of finished codes: the sign mask of 32 projections is stored as
 // is, with no bit stream to assemble.
 //
+// Learned gates (ELSAA overview: token-wise gates g = sigmoid(w . q_i + b))
+// need w_s . q_i and w_r . q_i for every query row; they ride along as four
+// more columns after the sort code: w_s and w_r each split into a bf16 high
+// part and the bf16 remainder (w - hi), so the two columns' fp32 sum carries
+// w to about 16 significant bits and the products stay exact in fp32.  The
+// read-out writes (w_s . q_i, w_r . q_i) for the query rows.
+//
 // Persistent CTAs of 128 threads.  The hyperplanes stay resident in shared
 // memory; 128-row tiles of Q then K stream in by cp.async (double-buffered
 // where that costs no CTA per SM: at text-32k sizes four single-buffered CTAs
@@ -40,18 +47,18 @@ constexpr uint32_t kTmemCols = 128;
 constexpr int kSmemLimit = 227 * 1024;
 
 struct HashShape {
-  int P16;       // columns: 32 Wr RACE columns, 16 sort columns
+  int P16;       // columns: 32 Wr RACE columns, 16 sort columns (+ 16 with gate columns)
   int cw, Wr;    // bits per RACE code; 32-bit words of RACE codes per row
   int S;         // staging stride in words (odd: conflict-free)
   int nbuf;
   uint32_t r_bytes, a_bytes, code_bytes, dyn;
 };
 
-HashShape hash_shape(const Geometry& g) {
+HashShape hash_shape(const Geometry& g, bool gates) {
   HashShape h;
   h.cw = 8 * g.rcode_bytes;
   h.Wr = g.L * h.cw / 32;
-  h.P16 = 32 * h.Wr + 16;
+  h.P16 = 32 * h.Wr + (gates ? 32 : 16);
   h.S = h.Wr | 1;
   h.r_bytes = (uint32_t)h.P16 * g.d * 2;
   h.a_bytes = (uint32_t)kTile * g.d * 2;
@@ -115,7 +122,8 @@ hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
                const __nv_bfloat16* __restrict__ r_sort, const __nv_bfloat16* __restrict__ r_race,
                int64_t rows_per_tensor, int N, int sort_bits, int L, int kr, int cw, int Wr, int S,
                int P16, int nbuf, uint16_t* __restrict__ code, CodeT* __restrict__ rcode,
-               CodeT* __restrict__ rcode_t, uint32_t* __restrict__ err) {
+               CodeT* __restrict__ rcode_t, const float* __restrict__ gate_w,
+               float2* __restrict__ gl, uint32_t* __restrict__ err) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   const uint32_t r_bytes = (uint32_t)P16 * D * 2;
@@ -155,6 +163,23 @@ hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         if (b < kr) val = *reinterpret_cast<const uint4*>(r_race + (size_t)(t * kr + b) * D + ch * 8);
       } else if (j - race_cols < sort_bits) {
         val = *reinterpret_cast<const uint4*>(r_sort + (size_t)(j - race_cols) * D + ch * 8);
+      } else if (gl != nullptr && j - race_cols >= 16 && j - race_cols < 20) {
+        // gate columns: w_s hi, w_s lo, w_r hi, w_r lo
+        const int gc = j - race_cols - 16;
+        const float* wrow = gate_w + (size_t)(gc >> 1) * D + ch * 8;
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          float x[2] = {wrow[e], wrow[e + 1]};
+#pragma unroll
+          for (int m = 0; m < 2; ++m) {
+            const float hi = __bfloat162float(__float2bfloat16_rn(x[m]));
+            x[m] = (gc & 1) ? x[m] - hi : hi;
+          }
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(x[0], x[1]);
+          pk[e >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        val = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
       *reinterpret_cast<uint4*>(smem + (ch >> 3) * (P16 * 128) + sw128_off(j, ch & 7)) = val;
     }
@@ -212,7 +237,12 @@ hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
 #pragma unroll
         for (int i = 0; i < 32; ++i) m |= (uint32_t)(__float_as_int(v[i]) > 0) << i;
         if (w < Wr) st_w[tid * S + w] = m;
-        else if (w == Wr) st_code[tid] = (uint16_t)(m & 0xFFFFu);
+        else if (w == Wr) {
+          st_code[tid] = (uint16_t)(m & 0xFFFFu);
+          const int64_t grow = tile * kTile + tid;
+          if (gl != nullptr && grow < rows_per_tensor)   // a query row: its gate logits
+            gl[grow] = make_float2(v[16] + v[17], v[18] + v[19]);
+        }
       }
       fence_before();
       __syncthreads();
@@ -271,9 +301,9 @@ hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
 
 template <int D, typename CodeT>
 cudaError_t run(const Geometry& g, const void* q, const void* k, const void* r_sort,
-                const void* r_race, uint16_t* code, void* rcode, void* rcode_t, uint32_t* err,
-                cudaStream_t s) {
-  const HashShape h = hash_shape(g);
+                const void* r_race, uint16_t* code, void* rcode, void* rcode_t,
+                const float* gate_w, float2* gl, uint32_t* err, cudaStream_t s) {
+  const HashShape h = hash_shape(g, gl != nullptr);
   cudaError_t e = cudaFuncSetAttribute(hash_tc_kernel<D, CodeT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)h.dyn);
   if (e != cudaSuccess) return e;
@@ -297,7 +327,7 @@ cudaError_t run(const Geometry& g, const void* q, const void* k, const void* r_s
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
       static_cast<const __nv_bfloat16*>(r_sort), static_cast<const __nv_bfloat16*>(r_race), rows,
       g.N, g.sort_bits, g.L, g.kr, h.cw, h.Wr, h.S, h.P16, h.nbuf, code,
-      static_cast<CodeT*>(rcode), static_cast<CodeT*>(rcode_t), err);
+      static_cast<CodeT*>(rcode), static_cast<CodeT*>(rcode_t), gate_w, gl, err);
   return cudaGetLastError();
 }
 
@@ -498,27 +528,32 @@ cudaError_t run_stream(const Geometry& g, const void* q, const void* k, const vo
   return cudaGetLastError();
 }
 
-bool aligned_layout_fits(const Geometry& g) {
+bool aligned_layout_fits(const Geometry& g, bool gates) {
   // codes fill whole 32-bit words per row; 128-row tiles never straddle units
   if ((g.L * g.rcode_bytes) % 4 != 0 || g.N % kTile != 0 || g.sort_bits > 16) return false;
-  return hash_shape(g).dyn <= (uint32_t)kSmemLimit;
+  return hash_shape(g, gates).dyn <= (uint32_t)kSmemLimit;
 }
 
 }  // namespace
 
+bool hash_tc_gate_logits_supported(const Geometry& g) {
+  return g.bf16 && (g.d == 64 || g.d == 128) && aligned_layout_fits(g, true);
+}
+
 bool hash_tc_supported(const Geometry& g) {
   if (!g.bf16 || (g.d != 64 && g.d != 128)) return false;
-  if (aligned_layout_fits(g)) return true;
+  if (aligned_layout_fits(g, false)) return true;
   const StreamShape h = stream_shape(g);
   return h.P > 0 && h.dyn <= (uint32_t)kSmemLimit;
 }
 
 cudaError_t launch_hash_tc(const Geometry& g, const void* q, const void* k, const void* r_sort,
                            const void* r_race, uint16_t* code, void* rcode, void* rcode_t,
-                           uint32_t* err, cudaStream_t s) {
-  const bool al = aligned_layout_fits(g);
+                           const float* gate_w, float2* gl, uint32_t* err, cudaStream_t s) {
+  if (gl != nullptr && !hash_tc_gate_logits_supported(g)) return cudaErrorInvalidValue;
+  const bool al = aligned_layout_fits(g, gl != nullptr);
 #define ELSAA_HASH(DD, CT)                                                                    \
-  (al ? run<DD, CT>(g, q, k, r_sort, r_race, code, rcode, rcode_t, err, s)                   \
+  (al ? run<DD, CT>(g, q, k, r_sort, r_race, code, rcode, rcode_t, gate_w, gl, err, s)       \
       : run_stream<DD, CT>(g, q, k, r_sort, r_race, code, rcode, rcode_t, err, s))
   if (g.d == 64) return g.rcode_bytes == 1 ? ELSAA_HASH(64, uint8_t) : ELSAA_HASH(64, uint16_t);
   return g.rcode_bytes == 1 ? ELSAA_HASH(128, uint8_t) : ELSAA_HASH(128, uint16_t);

@@ -55,6 +55,7 @@ struct WorkLayout {
   size_t sort_tmp;           // [2][BH][N] i32 (intermediate order of a 2-pass sort)
   size_t absmax;             // [2][BH] f32: largest |value| per unit (forward V, backward g_r dy / Ctot)
   size_t gtab;               // [BH][L][NB][d] bf16: the table copy the RACE gathers read
+  size_t gl;                 // [BH][N] float2: gate logits from the hash (shared-memory gathers)
   size_t causal_num;         // [BH][N][d] f32: causal RACE numerators (0 bytes unless causal)
   size_t saved;              // a SavedLayout used when the forward has no saved buffer
   size_t d_o;                // [BH][N][d] dtype: dO_sp
@@ -80,10 +81,14 @@ cudaError_t launch_hash_simt(const Geometry& g, const void* q, const void* k, co
                              const void* r_race, uint16_t* code, void* rcode, void* rcode_t,
                              cudaStream_t s);
 // SimHash codes on tcgen05 tensor cores (bf16 products, fp32 accumulation).
+// With gl non-null (learned gates) the same GEMM also writes the gate logits
+// gl[row] = (w_s . q_row, w_r . q_row) of every query row, w = gate_w [2][d]
+// fp32 (hash_tc_gate_logits_supported).
 cudaError_t launch_hash_tc(const Geometry& g, const void* q, const void* k, const void* r_sort,
                            const void* r_race, uint16_t* code, void* rcode, void* rcode_t,
-                           uint32_t* err, cudaStream_t s);
+                           const float* gate_w, float2* gl, uint32_t* err, cudaStream_t s);
 bool hash_tc_supported(const Geometry& g);
+bool hash_tc_gate_logits_supported(const Geometry& g);
 
 // Sort codes of hash rounds 1 .. R-1 (round 0 comes with the main hash):
 // code[t][2][BH][N] from r_sort[t] ([R][sort_bits][d]), on CUDA cores.
@@ -120,6 +125,18 @@ cudaError_t launch_race_gather_add(const Geometry& g, const void* codes, const v
                                    void* dst, cudaStream_t s);
 cudaError_t launch_race_gather_sum(const Geometry& g, const void* codes, const void* tables,
                                    float* out, cudaStream_t s);
+// RACE read-out from tables resident in shared memory (race_slab.cu): bf16
+// data, one-byte codes, 16 or 32 tables.  Forward: gathers by query codes
+// fused with the gates (gl from the hash when learned), the multiplier and the
+// output; add: dst[row] += the gathered table rows (the RACE value gradient).
+bool race_slab_supported(const Geometry& g, bool fuse);
+cudaError_t launch_race_slab_fuse(const Geometry& g, const void* rcode_q, const void* tables,
+                                  const int32_t* counts, const void* o_sp, const float* lse,
+                                  const float2* gl, const float* gate_b, const float* lam,
+                                  void* y, void* o_race, int32_t* ctot, uint32_t* err,
+                                  cudaStream_t s);
+cudaError_t launch_race_slab_add(const Geometry& g, const void* codes, const void* tables,
+                                 void* dst, uint32_t* err, cudaStream_t s);
 // Forward RACE gather fused with the gates, the multiplier and the output.
 cudaError_t launch_race_fuse_fwd(const Geometry& g, const void* q, const void* rcode_q,
                                  const void* tables, const int32_t* counts,
@@ -198,5 +215,9 @@ cudaError_t launch_fuse_causal(const Geometry& g, const void* q, const void* o_s
 // 2-D TMA map over a [rows, 64] bf16 matrix: one 128-byte row per box,
 // 128-byte swizzle; the row gathers of the tcgen05 attention kernels use it.
 cudaError_t make_row_map(CUtensorMap* map, const void* base, uint64_t rows);
+// 3-D TMA map over a [units, n, d] bf16 tensor (d contiguous), no swizzle, box
+// of 8 columns x box_rows rows x 1 unit: the RACE slab kernels' row tiles.
+cudaError_t make_slab_map(CUtensorMap* map, const void* base, uint64_t units, uint64_t n,
+                          uint64_t d, uint32_t box_rows);
 
 }  // namespace elsaa

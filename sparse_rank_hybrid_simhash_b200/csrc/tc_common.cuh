@@ -245,6 +245,32 @@ ELSAA_DEV void tma_gather4(uint32_t dst, const void* map, int r0, int r1, int r2
       : "memory");
 }
 
+// One box of a 3-D tensor map at coordinates (x, y, z) into shared memory at
+// `dst`; completion is counted on `bar` in bytes.  x (innermost, in elements)
+// must be a multiple of 16 bytes; out-of-range elements read as zero.
+ELSAA_DEV void tma_load_3d(uint32_t dst, const void* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// One box from shared memory at `src` to a 3-D tensor map at (x, y, z), x a
+// multiple of 16 bytes and every coordinate >= 0; elements outside the
+// tensor are not written.  Completes in the thread's bulk async-group.
+ELSAA_DEV void tma_store_3d(const void* map, int x, int y, int z, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];"
+               ::"l"(map), "r"(x), "r"(y), "r"(z), "r"(src)
+               : "memory");
+}
+ELSAA_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+ELSAA_DEV void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
+template <int N>
+ELSAA_DEV void bulk_wait() { asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory"); }
+
 // ---- cp.async --------------------------------------------------------------
 
 // 16-byte global -> shared copy; src_bytes = 0 zero-fills the destination.

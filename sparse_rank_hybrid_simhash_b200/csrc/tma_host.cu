@@ -1,6 +1,8 @@
-// Host side of the TMA row gathers: 2-D tensor maps over [rows, 64] bf16
-// matrices (one row per box, 128-byte swizzle), encoded through the driver
-// entry point the runtime resolves (no direct driver-API calls).
+// Host side of the TMA copies: 2-D tensor maps over [rows, 64] bf16 matrices
+// (one row per box, 128-byte swizzle) for the attention kernels' row gathers,
+// and 3-D maps over [units, N, d] bf16 with 8-column boxes for the RACE slab
+// kernels; encoded through the driver entry point the runtime resolves (no
+// direct driver-API calls).
 #include <cudaTypedefs.h>
 #include <mutex>
 
@@ -34,6 +36,21 @@ cudaError_t make_row_map(CUtensorMap* map, const void* base, uint64_t rows) {
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                         strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_slab_map(CUtensorMap* map, const void* base, uint64_t units, uint64_t n,
+                          uint64_t d, uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {d, n, units};
+  const cuuint64_t strides[2] = {d * 2, n * d * 2};
+  const cuuint32_t box[3] = {8, box_rows, 1};
+  const cuuint32_t elem[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }

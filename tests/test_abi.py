@@ -170,3 +170,21 @@ def test_kernel_launch_counts():
     # CUDA-core sparse backward + 3 casts
     r = B.kernel_launches(B.Params.from_workload(w.replace(hash_rounds=3)))
     assert r == (1 + 1 + 3 * 3 + 1 + 2 + 1 + 1, 1 + 2 + 1 + 3 + 1)
+
+
+def test_path_flags():
+    # the kernel families each workload takes (what the bench line and the
+    # parity tests rely on)
+    f = {n: B.path_flags(B.Params.from_workload(w)) for n, w in WORKLOADS.items()}
+    assert all(f["text-32k"].values()) and all(f["vision-16k"].values())
+    assert all(f["iid-4k"].values())
+    # 10-bit RACE codes: the tables do not fit a shared-memory slab
+    assert f["needle-256k"]["tc_hash"] and f["needle-256k"]["tc_attn"]
+    assert not f["needle-256k"]["slab_fwd"] and not f["needle-256k"]["slab_bwd"]
+    assert not any(f["tiny-fp32"].values())
+    w = WORKLOADS["text-32k"]
+    assert not B.path_flags(B.Params.from_workload(w.replace(causal=True)))["slab_fwd"]
+    assert not B.path_flags(B.Params.from_workload(w.replace(hash_rounds=2)))["slab_bwd"]
+    assert B.path_flags(B.Params.from_workload(w.replace(hash_rounds=2)))["slab_fwd"]
+    assert B.path_flags(B.Params.make(1, 1, 256, 64, "bf16", 4, 64, 8, 6)) == {
+        "tc_hash": True, "tc_attn": True, "slab_fwd": False, "slab_bwd": False}
