@@ -458,30 +458,27 @@ def run_ours(args, rank, world, local_rank):
 
 
 def run_e2e(args, w, p, inp, dev, world):
+    """The same step end to end through the public API with host buffers: the
+    batch's inputs sit in pinned host memory and its outputs go back there
+    every step, streamed through the device in groups of heads
+    (pipeline.HostStepPipeline: copy-in, compute and copy-out overlap)."""
+    from sparse_rank_hybrid_simhash_b200.pipeline import HostStepPipeline
+    BH = w.B * w.H
+    groups = next(g for g in (4, 3, 2, 1) if BH % g == 0)
     host = {k: inp[k].pin_memory() for k in ("q", "k", "v", "dy")}
-    outs = {k: torch.empty_like(host[k], pin_memory=True) for k in ("q", "k", "v", "dy")}
-    pg_host = torch.empty(2 * w.d + 3, dtype=torch.float32, pin_memory=True)
-    small = {k: inp[k].to(dev) for k in ("r_sort", "r_race", "gate_w", "gate_b", "lam")}
-    dq = {k: torch.empty(host[k].shape, dtype=host[k].dtype, device=dev) for k in host}
-    saved = B.alloc_saved(p, dev)
-    ws = B.alloc_workspace(p, dev)
+    outs = {k: torch.empty_like(host["q"], pin_memory=True) for k in ("y", "dq", "dk", "dv")}
+    pipe = HostStepPipeline(p, groups, dev, inp["r_sort"], inp["r_race"], inp["gate_w"],
+                            inp["gate_b"], inp["lam"])
     stream = torch.cuda.current_stream()
+    pg_dev = torch.empty(2 * w.d + 3, dtype=torch.float32, device=dev)
 
     def step():
-        for k in host:
-            dq[k].copy_(host[k], non_blocking=True)
-        y = B.forward(p, dq["q"], dq["k"], dq["v"], small["r_sort"], small["r_race"],
-                      small["gate_w"], small["gate_b"], small["lam"], saved=saved, ws=ws)
-        g = B.backward(p, dq["q"], dq["k"], dq["v"], small["r_sort"], small["r_race"],
-                       small["gate_w"], small["gate_b"], small["lam"], saved, dq["dy"], ws=ws)
-        if world > 1:
-            DP.allreduce_param_grads(g[3], g[4], g[5])
-        pg = torch.cat([g[3].view(-1), g[4].view(-1), g[5].view(-1)])
-        outs["q"].copy_(g[0], non_blocking=True)
-        outs["k"].copy_(g[1], non_blocking=True)
-        outs["v"].copy_(g[2], non_blocking=True)
-        outs["dy"].copy_(y, non_blocking=True)
-        pg_host.copy_(pg, non_blocking=True)
+        pipe.enqueue(host, outs, stream)
+        if world > 1:   # the shared-parameter gradients, summed over ranks
+            stream.synchronize()
+            gw, gb, gl = pipe.gradients()
+            pg_dev.copy_(torch.cat([gw.view(-1), gb, gl]))
+            torch.distributed.all_reduce(pg_dev)
 
     step()
     torch.cuda.synchronize()
@@ -494,13 +491,15 @@ def run_e2e(args, w, p, inp, dev, world):
         step()
     end.record(stream)
     torch.cuda.synchronize()
+    pipe.gradients()
     ms = start.elapsed_time(end)
     if world > 1:
         ms = DP.max_over_ranks([ms], dev)[0]
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = sum(t.numel() * t.element_size() for t in outs.values()) + pg_host.numel() * 4
+    h2d = pipe.h2d_bytes(host)
+    d2h = sum(t.numel() * t.element_size() for t in outs.values()) + pipe.pg_host.numel() * 4
     return {"value": world * n * w.tokens / (ms / 1e3), "unit": "tokens/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
+            "pipeline": f"{groups} head groups; copy-in, compute and copy-out streams overlap"}
 
 
 # ---------------------------------------------------------------------------
