@@ -96,6 +96,7 @@ WorkLayout work_layout(const Geometry& g) {
   w.absmax = take((size_t)2 * g.BH * 4);
   w.gtab = take((size_t)g.BH * g.L * g.NB * g.d * 2);
   w.gl = take(bhn * sizeof(float2));
+  w.count_scratch = take((size_t)g.BH * g.L * g.NB * 4);
   w.causal_num = take(g.causal ? bhn * g.d * 4 : 0);
   const size_t shared_base = off;
   // forward without a saved buffer: the saved layout lives here
@@ -279,7 +280,8 @@ elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const vo
   // gathers read tables in the data dtype: a bf16 copy, or the fp32 sums themselves
   __nv_bfloat16* gtab = g.bf16 ? (__nv_bfloat16*)(w + wl.gtab) : nullptr;
   const void* gather_tables = g.bf16 ? (const void*)gtab : (const void*)sums;
-  ELSAA_TRY(launch_race_build(g, rcode_k, rcode_tk, v, false, absmax, sums, true, gtab, counts, err, s));
+  ELSAA_TRY(launch_race_build(g, rcode_k, rcode_tk, v, false, absmax, sums, true, gtab, counts,
+                              (int32_t*)(w + wl.count_scratch), err, s));
   ELSAA_TRY(mark(events, 3, s));
   // 4. exact sparse branch
   if (g.tc_attn && attn_pipe_supported(g))
@@ -376,7 +378,8 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
     ELSAA_TRY(launch_race_causal_bwd(g, rcode, rcode_k, dor, dv_acc, s));
   } else {
     ELSAA_TRY(launch_race_build(g, rcode, rcode_t, dor, false, absmax, d_t, !g.bf16, gtab,
-                                nullptr, (uint32_t*)(w + wl.err), s));
+                                nullptr, (int32_t*)(w + wl.count_scratch),
+                                (uint32_t*)(w + wl.err), s));
     if (!direct) ELSAA_TRY(launch_race_gather_sum(g, rcode_k, race_grad, dv_acc, s));
   }
   ELSAA_TRY(mark(events, 2, s));
@@ -436,12 +439,15 @@ elsaa_status elsaa_kernel_launches(const elsaa_params* p, int32_t* fwd, int32_t*
   // inverse orders; zero-bit extra codes are a memset)
   const int sort1 = g.sort_order == ELSAA_SORT_LOCAL ? 1 : 3 * g.sort_passes;
   const int sort = g.rounds * sort1 + (g.rounds > 1 ? 1 + (g.sort_bits > 0 ? 1 : 0) : 0);
-  *fwd = g.causal ? 1 + sort + 1 + 1 + 1 : 1 + sort + 2 + 1 + 1;
+  const int build = race_build_kernels(g, false, g.bf16);
+  *fwd = g.causal ? 1 + sort + 1 + 1 + 1 : 1 + sort + 1 + build + 1 + 1;
   // fusion backward 1, RACE build 1 + gather 1, sparse 1 (+ casts), reduction 1
   // (direct path: the sparse kernel writes dq itself and the gather adds into dv)
   const bool direct = direct_bwd(g);
   const int sparse = direct ? 1 : g.tc_attn ? 1 + 1 : 1 + 3;
-  *bwd = 1 + (g.causal ? 1 : 2) + sparse + 1;
+  // (the RACE backward: the table-gradient build, then, off the direct path, a gather)
+  const int race_bwd = g.causal ? 1 : race_build_kernels(g, false, g.bf16) + (direct ? 0 : 1);
+  *bwd = 1 + race_bwd + sparse + (direct ? 1 : 0) + 1;
   return ELSAA_OK;
 }
 

@@ -56,6 +56,7 @@ struct WorkLayout {
   size_t absmax;             // [2][BH] f32: largest |value| per unit (forward V, backward g_r dy / Ctot)
   size_t gtab;               // [BH][L][NB][d] bf16: the table copy the RACE gathers read
   size_t gl;                 // [BH][N] float2: gate logits from the hash (shared-memory gathers)
+  size_t count_scratch;      // [BH][L][NB] i32: bucket counts of a build that has no counts output
   size_t causal_num;         // [BH][N][d] f32: causal RACE numerators (0 bytes unless causal)
   size_t saved;              // a SavedLayout used when the forward has no saved buffer
   size_t d_o;                // [BH][N][d] dtype: dO_sp
@@ -111,11 +112,15 @@ cudaError_t launch_unit_absmax(const Geometry& g, const void* vals, bool vals_f3
 // vals_f32 selects fp32 values instead of dtype; absmax[bh] must bound |vals|
 // of unit bh; keep_sums = false leaves `sums` as scratch only.
 // codes: [BH][N][L] row-major; codes_t: the same codes [BH][L][N] table-major.
+// count_scratch: [BH][L][NB] int32 the segmented build counts into when
+// `counts` is null (long sequences need the counts to size the fixed-point grid).
+// Kernels one launch_race_build enqueues (memsets excluded).
+int race_build_kernels(const Geometry& g, bool vals_f32, bool gtab);
 cudaError_t launch_race_build(const Geometry& g, const void* codes, const void* codes_t,
                               const void* vals,
                               bool vals_f32, const float* absmax, float* sums, bool keep_sums,
-                              __nv_bfloat16* gtab, int32_t* counts, uint32_t* err,
-                              cudaStream_t s);
+                              __nv_bfloat16* gtab, int32_t* counts, int32_t* count_scratch,
+                              uint32_t* err, cudaStream_t s);
 // out[bh][i][:] = sum_l tables[bh][l][codes[bh][i][l]][:]  (f32, overwritten);
 // tables in the data dtype (bf16 copy, or the fp32 sums for fp32 data).
 // dst[bh][i][:] += sum_l tables[bh][l][codes[bh][i][l]][:], dst in the data dtype

@@ -848,6 +848,248 @@ race_build_sorted_kernel(const CodeT* __restrict__ codes_t, const TV* __restrict
   }
 }
 
+// ---- segmented bucket-sorted build (long sequences, large tables) ------------
+//
+// For shapes whose table or key list does not fit one CTA's shared memory
+// (needle-256k: N = 262144 keys, 1024 buckets x 128 values): one CTA per
+// (unit, table, segment of kSegKeys keys) bucket-sorts its segment's keys the
+// same way (warp-private counters and cursors, so the list is the same on
+// every run), sums each bucket's run of value rows in fp32 registers, rounds
+// the run total to the grid 2^-S and adds it, as an integer, into a zeroed
+// int32 table in global memory (the fp32 table's bytes).  S is chosen from the
+// table's largest bucket count (from a counting pass) and the unit's largest
+// |value| as in the single-CTA build (C_max vmax 2^S <= 2^30): integer sums
+// are exact and order-independent, so the table is the same on every run.  A
+// last pass turns each table into fp32 (and the bf16 copy) in place.
+
+constexpr int kSegThreads = 512;
+constexpr int kSegWarps = kSegThreads / 32;
+constexpr int kSegKeys = 32768;
+
+struct SegSmem {
+  size_t list, codes, whist, bend, misc, total;
+};
+__host__ __device__ inline SegSmem seg_smem(int seg, int NB, int code_bytes) {
+  SegSmem m;
+  m.list = 0;
+  m.codes = align16((size_t)seg * 2);
+  m.whist = align16(m.codes + (size_t)seg * code_bytes);
+  m.bend = align16(m.whist + (size_t)kSegWarps * NB * 4);
+  m.misc = align16(m.bend + (size_t)NB * 4);
+  m.total = m.misc + 256;   // [0] C_max, [1] bad code, [16..32) warp sums of the scan
+  return m;
+}
+
+// counts[bh][t][b] += the segment's keys in bucket b (counts zeroed first)
+template <typename CodeT>
+__global__ void __launch_bounds__(256)
+race_seg_hist_kernel(const CodeT* __restrict__ codes_t, int N, int L, int NB, int seg,
+                     int32_t* __restrict__ counts, uint32_t* __restrict__ err) {
+  extern __shared__ int32_t hist[];
+  const int t = blockIdx.y, bh = blockIdx.z;
+  const int j0 = blockIdx.x * seg, j1 = min(N, j0 + seg);
+  const CodeT* ct = codes_t + ((size_t)bh * L + t) * N;
+  for (int b = threadIdx.x; b < NB; b += blockDim.x) hist[b] = 0;
+  __syncthreads();
+  bool bad = false;
+  for (int j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
+    const int c = (int)ct[j];
+    if (c < NB) atomicAdd(hist + c, 1);
+    else bad = true;
+  }
+  if (bad) raise_error(err, ERR_CHECK);
+  __syncthreads();
+  int32_t* dst = counts + ((size_t)bh * L + t) * NB;
+  for (int b = threadIdx.x; b < NB; b += blockDim.x)
+    if (hist[b]) atomicAdd(dst + b, hist[b]);
+}
+
+// Grid exponent S of one table: C_max vmax 2^S <= 2^30 (every integer total fits int32).
+ELSAA_DEV int seg_grid(int cmax, float vmax) {
+  if (cmax > 0 && vmax > 0.f)
+    return max(-100, min(100, (int)floorf(log2f(1073741824.0f / ((float)cmax * vmax)))));
+  return 0;
+}
+
+template <typename TV, typename CodeT>
+__global__ void __launch_bounds__(kSegThreads, 1)
+race_build_seg_kernel(const CodeT* __restrict__ codes_t, const TV* __restrict__ vals, int N,
+                      int L, int NB, int d, int seg, const float* __restrict__ absmax,
+                      const int32_t* __restrict__ counts, float* __restrict__ sums,
+                      uint32_t* __restrict__ err) {
+  constexpr int EL = 16 / (int)sizeof(TV);
+  extern __shared__ __align__(16) uint8_t sm[];
+  const SegSmem lay = seg_smem(seg, NB, (int)sizeof(CodeT));
+  uint16_t* list = reinterpret_cast<uint16_t*>(sm + lay.list);      // segment keys, by bucket
+  CodeT* csm = reinterpret_cast<CodeT*>(sm + lay.codes);            // the segment's codes
+  uint32_t* whist = reinterpret_cast<uint32_t*>(sm + lay.whist);    // [warps][NB]
+  int32_t* bend = reinterpret_cast<int32_t*>(sm + lay.bend);        // [NB] end of each bucket
+  int32_t* misc = reinterpret_cast<int32_t*>(sm + lay.misc);        // [0] C_max, [1] bad code
+  int32_t* wsum = misc + 16;                                        // [kSegWarps] scan sums
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t = blockIdx.y, bh = blockIdx.z;
+  const int j0 = blockIdx.x * seg, n = min(N, j0 + seg) - j0;   // keys [j0, j0 + n)
+  const CodeT* ct = codes_t + ((size_t)bh * L + t) * N + j0;
+  // warp w owns segment keys [k0, k1)
+  const int k0 = (int)((int64_t)n * warp / kSegWarps);
+  const int k1 = (int)((int64_t)n * (warp + 1) / kSegWarps);
+  uint32_t* wh = whist + (size_t)warp * NB;
+  for (int i = tid; i < n; i += kSegThreads) csm[i] = ct[i];
+  for (int i = tid; i < kSegWarps * NB; i += kSegThreads) whist[i] = 0;
+  if (tid < 2) misc[tid] = 0;
+  __syncthreads();
+  // the table's largest bucket count (all segments), for the grid 2^-S
+  {
+    const int32_t* cnt = counts + ((size_t)bh * L + t) * NB;
+    int cm = 0;
+    for (int b = tid; b < NB; b += kSegThreads) cm = max(cm, cnt[b]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cm = max(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+    if (lane == 0) atomicMax(misc, cm);
+  }
+  for (int j = k0 + lane; j < k1; j += 32) {
+    const int c = (int)csm[j];
+    if (c < NB) atomicAdd(wh + c, 1u);
+    else misc[1] = 1;
+  }
+  __syncthreads();
+  if (misc[1] != 0) {
+    if (tid == 0) raise_error(err, ERR_CHECK);
+    return;
+  }
+  // bucket totals of the segment, their exclusive scan (blocks of 32 buckets
+  // per warp, kSegWarps warps per pass), and each warp's starting slot
+  int carry = 0;
+  for (int b0 = 0; b0 < NB; b0 += kSegThreads) {
+    const int b = b0 + tid;
+    int c = 0;
+    if (b < NB)
+      for (int w = 0; w < kSegWarps; ++w) c += (int)whist[w * NB + b];
+    int x = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    int before = carry;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    int total = 0;
+    for (int w = 0; w < kSegWarps; ++w) total += wsum[w];
+    if (b < NB) {
+      uint32_t run = (uint32_t)(before + x - c);
+      bend[b] = before + x;
+      for (int w = 0; w < kSegWarps; ++w) {
+        const uint32_t h = whist[w * NB + b];
+        whist[w * NB + b] = run;
+        run += h;
+      }
+    }
+    carry += total;
+    __syncthreads();
+  }
+  // scatter through the warp-private cursors
+  for (int j = k0 + lane; j < k1; j += 32) list[atomicAdd(wh + (int)csm[j], 1u)] = (uint16_t)j;
+  const float vmax = absmax[bh];
+  if (!(vmax < 3.0e38f)) {
+    if (tid == 0) raise_error(err, ERR_CHECK);
+    return;
+  }
+  __syncthreads();
+  const float scale = ldexpf(1.0f, seg_grid(misc[0], vmax));
+
+  // lane groups of QL lanes walk equal shares [p0, p1) of the list
+  const int QL = d / EL;
+  const int groups = kSegThreads / QL;
+  const int gi = tid / QL, ql = tid % QL;
+  const int p0 = (int)((int64_t)n * gi / groups), p1 = (int)((int64_t)n * (gi + 1) / groups);
+  const TV* vb = vals + ((size_t)bh * N + j0) * d + ql * EL;
+  // the fp32 table's bytes hold the int32 sums until the finishing pass
+  uint32_t* tb = reinterpret_cast<uint32_t*>(sums + ((size_t)bh * L + t) * NB * d) + ql * EL;
+  float acc[EL];
+#pragma unroll
+  for (int e = 0; e < EL; ++e) acc[e] = 0.f;
+  int b = 0;
+  if (p0 < p1) {
+    int lo = 0, hi = NB - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (bend[mid] > p0) hi = mid;
+      else lo = mid + 1;
+    }
+    b = lo;
+  }
+  int b_end = p0 < p1 ? bend[b] : 0;
+  bool any = false;
+  auto flush = [&]() {
+    if (any) {
+      uint32_t* dst = tb + (size_t)b * d;
+#pragma unroll
+      for (int e = 0; e < EL; ++e) {
+        atomicAdd(dst + e, (uint32_t)__float2int_rn(acc[e] * scale));
+        acc[e] = 0.f;
+      }
+    }
+    any = false;
+  };
+  auto step = [&](int pos, uint4 raw) {
+    if (pos >= b_end) {
+      flush();
+      do b_end = bend[++b]; while (pos >= b_end);
+    }
+    add_row(acc, raw, vb);
+    any = true;
+  };
+  auto row = [&](int key) { return __ldg(reinterpret_cast<const uint4*>(vb + (size_t)key * d)); };
+  int p = p0;
+  for (; p < p1 && (p & 3) != 0; ++p) step(p, row(list[p]));
+  for (; p + 4 <= p1; p += 4) {
+    const uint2 k4 = *reinterpret_cast<const uint2*>(list + p);
+    const uint4 r0 = row((int)(k4.x & 0xFFFFu)), r1 = row((int)(k4.x >> 16));
+    const uint4 r2 = row((int)(k4.y & 0xFFFFu)), r3 = row((int)(k4.y >> 16));
+    step(p, r0);
+    step(p + 1, r1);
+    step(p + 2, r2);
+    step(p + 3, r3);
+  }
+  for (; p < p1; ++p) step(p, row(list[p]));
+  flush();
+}
+
+// One block per (unit, table): the int32 sums become fp32 (scaled by 2^-S of
+// that table) in place, and the bf16 copy is written if gtab is non-null.
+__global__ void __launch_bounds__(256)
+race_seg_finish_kernel(float* __restrict__ sums, __nv_bfloat16* __restrict__ gtab,
+                       const int32_t* __restrict__ counts, const float* __restrict__ absmax,
+                       int L, int NB, int d) {
+  __shared__ int s_cmax;
+  const int t = blockIdx.x, bh = blockIdx.y;
+  if (threadIdx.x == 0) s_cmax = 0;
+  __syncthreads();
+  const int32_t* cnt = counts + ((size_t)bh * L + t) * NB;
+  int cm = 0;
+  for (int b = threadIdx.x; b < NB; b += blockDim.x) cm = max(cm, cnt[b]);
+  cm = __reduce_max_sync(0xffffffffu, cm);
+  if ((threadIdx.x & 31) == 0) atomicMax(&s_cmax, cm);
+  __syncthreads();
+  const float inv_scale = ldexpf(1.0f, -seg_grid(s_cmax, absmax[bh]));
+  const size_t o0 = ((size_t)bh * L + t) * NB * d;
+  for (int i = threadIdx.x * 4; i < NB * d; i += blockDim.x * 4) {
+    const int4 v = *reinterpret_cast<const int4*>(sums + o0 + i);
+    const float f0 = (float)v.x * inv_scale, f1 = (float)v.y * inv_scale;
+    const float f2 = (float)v.z * inv_scale, f3 = (float)v.w * inv_scale;
+    *reinterpret_cast<float4*>(sums + o0 + i) = make_float4(f0, f1, f2, f3);
+    if (gtab) {
+      const __nv_bfloat162 a = __floats2bfloat162_rn(f0, f1), b = __floats2bfloat162_rn(f2, f3);
+      uint2 w;
+      w.x = *reinterpret_cast<const uint32_t*>(&a);
+      w.y = *reinterpret_cast<const uint32_t*>(&b);
+      *reinterpret_cast<uint2*>(gtab + o0 + i) = w;
+    }
+  }
+}
+
 // ---- row-pipelined gathers ---------------------------------------------------
 //
 // Used when a row's codes are whole 32-bit words (L * code bytes % 4 == 0).
@@ -1114,7 +1356,7 @@ template <typename TV, typename CodeT>
 cudaError_t build(const Geometry& g, const void* codes, const void* codes_t, const void* vals,
                   const float* absmax,
                   float* sums, bool keep_sums, __nv_bfloat16* gtab, int32_t* counts,
-                  uint32_t* err, cudaStream_t s) {
+                  int32_t* count_scratch, uint32_t* err, cudaStream_t s) {
   {
     // bucket-sorted build: key indices fit u16, one bucket per thread in the
     // scan, and the whole table plus the key list fit in shared memory
@@ -1128,6 +1370,36 @@ cudaError_t build(const Geometry& g, const void* codes, const void* codes_t, con
       kernel<<<dim3(g.L, g.BH), kSortedThreads, m.total, s>>>(
           static_cast<const CodeT*>(codes_t), static_cast<const TV*>(vals), g.N, g.L, g.NB, g.d,
           absmax, keep_sums ? sums : nullptr, gtab, counts, err);
+      return cudaGetLastError();
+    }
+  }
+  {
+    // segmented bucket-sorted build: counts by a counting pass, then one CTA
+    // per (unit, table, segment) adding exact run totals into the zeroed table
+    const int seg = g.N < kSegKeys ? g.N : kSegKeys;
+    const SegSmem m = seg_smem(seg, g.NB, (int)sizeof(CodeT));
+    if (g.NB <= 1024 && m.total <= (size_t)kBuildSmemBudget &&
+        g.d % (16 / (int)sizeof(TV)) == 0 && (g.d / (16 / (int)sizeof(TV))) <= 32 &&
+        sums != nullptr) {
+      const size_t tab = (size_t)g.BH * g.L * g.NB;
+      // the table's counts (the caller's output, or scratch where it has none)
+      int32_t* cnt = counts != nullptr ? counts : count_scratch;
+      if (cnt == nullptr) return cudaErrorInvalidValue;
+      cudaError_t e = cudaMemsetAsync(cnt, 0, tab * 4, s);
+      if (e != cudaSuccess) return e;
+      e = cudaMemsetAsync(sums, 0, tab * g.d * 4, s);
+      if (e != cudaSuccess) return e;
+      const dim3 grid((g.N + seg - 1) / seg, g.L, g.BH);
+      race_seg_hist_kernel<CodeT><<<grid, 256, g.NB * 4, s>>>(
+          static_cast<const CodeT*>(codes_t), g.N, g.L, g.NB, seg, cnt, err);
+      auto kernel = race_build_seg_kernel<TV, CodeT>;
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)m.total);
+      if (e != cudaSuccess) return e;
+      kernel<<<grid, kSegThreads, m.total, s>>>(static_cast<const CodeT*>(codes_t),
+                                                static_cast<const TV*>(vals), g.N, g.L, g.NB, g.d,
+                                                seg, absmax, cnt, sums, err);
+      race_seg_finish_kernel<<<dim3(g.L, g.BH), 256, 0, s>>>(sums, gtab, cnt, absmax, g.L, g.NB,
+                                                              g.d);
       return cudaGetLastError();
     }
   }
@@ -1313,21 +1585,38 @@ cudaError_t launch_unit_absmax(const Geometry& g, const void* vals, bool vals_f3
   return cudaGetLastError();
 }
 
+int race_build_kernels(const Geometry& g, bool vals_f32, bool gtab) {
+  const int esz = (vals_f32 || !g.bf16) ? 4 : 2;
+  const int cb = g.rcode_bytes;
+  const SortedSmem m = sorted_smem(g.N, g.NB, g.d, cb);
+  if (g.N <= 65536 && g.NB <= kSortedThreads && m.total <= (size_t)kBuildSmemBudget &&
+      g.d % (16 / esz) == 0)
+    return 1;
+  const int seg = g.N < kSegKeys ? g.N : kSegKeys;
+  if (g.NB <= 1024 && seg_smem(seg, g.NB, cb).total <= (size_t)kBuildSmemBudget &&
+      g.d % (16 / esz) == 0 && g.d / (16 / esz) <= 32)
+    return 3;   // counting pass, build, finishing pass
+  const BuildShape b = build_shape(g);
+  if (b.nt < 1) return 1 + (gtab ? 1 : 0);   // global atomics, bf16 copy
+  return 1;
+}
+
 cudaError_t launch_race_build(const Geometry& g, const void* codes, const void* codes_t,
                               const void* vals,
                               bool vals_f32, const float* absmax, float* sums, bool keep_sums,
-                              __nv_bfloat16* gtab, int32_t* counts, uint32_t* err,
-                              cudaStream_t s) {
+                              __nv_bfloat16* gtab, int32_t* counts, int32_t* count_scratch,
+                              uint32_t* err, cudaStream_t s) {
   if (vals_f32 || !g.bf16)
     return g.rcode_bytes == 1
-               ? build<float, uint8_t>(g, codes, codes_t, vals, absmax, sums, keep_sums, gtab, counts, err, s)
-               : build<float, uint16_t>(g, codes, codes_t, vals, absmax, sums, keep_sums, gtab, counts, err,
-                                        s);
+               ? build<float, uint8_t>(g, codes, codes_t, vals, absmax, sums, keep_sums, gtab,
+                                       counts, count_scratch, err, s)
+               : build<float, uint16_t>(g, codes, codes_t, vals, absmax, sums, keep_sums, gtab,
+                                        counts, count_scratch, err, s);
   return g.rcode_bytes == 1
-             ? build<__nv_bfloat16, uint8_t>(g, codes, codes_t, vals, absmax, sums, keep_sums, gtab, counts,
-                                             err, s)
-             : build<__nv_bfloat16, uint16_t>(g, codes, codes_t, vals, absmax, sums, keep_sums, gtab,
-                                              counts, err, s);
+             ? build<__nv_bfloat16, uint8_t>(g, codes, codes_t, vals, absmax, sums, keep_sums,
+                                             gtab, counts, count_scratch, err, s)
+             : build<__nv_bfloat16, uint16_t>(g, codes, codes_t, vals, absmax, sums, keep_sums,
+                                              gtab, counts, count_scratch, err, s);
 }
 
 cudaError_t launch_race_gather_sum(const Geometry& g, const void* codes, const void* tables,
