@@ -241,6 +241,64 @@ const char* elsaa_status_str(elsaa_status s);
  * dims other than 64/128, or chunk shapes the tensor kernels do not tile). */
 int32_t elsaa_uses_tensor_cores(const elsaa_params* p);
 
+/* ---- Pieces of the operator for a sequence split across devices ---------
+ *
+ * A sequence can be split into token shards on several devices (the
+ * package's sharding module): every shard's sort codes are gathered, every
+ * device computes the same global Sort-LSH orders, the rows of each device's
+ * range of sorted chunks (and one chunk before it) are exchanged to it, and
+ * the RACE tables are summed over the shards.  These calls are the device
+ * steps of that scheme; p describes the problem each call runs on (the shard,
+ * or a device's sorted range).  All pointers are device memory; ws is a
+ * workspace of elsaa_workspace_bytes(p).  Sharded problems need one hash
+ * round and no causal mask (p is rejected otherwise where it matters). */
+
+/* Sort codes of q and k ([B,H,N,d]): code [2][B,H,N] uint16 (queries then
+ * keys), as elsaa_forward computes them. */
+elsaa_status elsaa_sort_codes_of(const elsaa_params* p, const void* q, const void* k,
+                                 const void* r_sort, const void* r_race, uint16_t* code,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/* Stable Sort-LSH order (p->sort_order) of given codes [2][B,H,N] uint16:
+ * perm [2][B,H,N] int32, the token index at each sorted rank. */
+elsaa_status elsaa_sort_codes(const elsaa_params* p, const uint16_t* code, int32_t* perm,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/* RACE tables of the keys k and values v ([B,H,N,d]): race_sum [B,H,L,2^K_r,d]
+ * fp32 and race_count [B,H,L,2^K_r] int32 (overwritten).  Tables of several
+ * shards of one sequence add up to the tables of the whole sequence. */
+elsaa_status elsaa_race_tables(const elsaa_params* p, const void* k, const void* v,
+                               const void* r_race, float* race_sum, int32_t* race_count,
+                               void* ws, size_t ws_bytes, void* stream);
+
+/* elsaa_forward with the RACE tables given (race_sum / race_count as above,
+ * e.g. summed over every shard of the sequence) instead of built from k and v.
+ * The tables are copied into the saved state. */
+elsaa_status elsaa_forward_tables(const elsaa_params* p, const void* q, const void* k,
+                                  const void* v, const void* r_sort, const void* r_race,
+                                  const float* gate_w, const float* gate_b, const float* lambda,
+                                  const float* race_sum, const int32_t* race_count, void* y,
+                                  void* saved, void* ws, size_t ws_bytes, void* stream);
+
+/* elsaa_backward of a forward made by elsaa_forward_tables: writes the RACE
+ * table gradient dT = d sum(y dy) / d race_sum of this call's queries into
+ * d_race_sum ([B,H,L,2^K_r,d] fp32, overwritten) and leaves the RACE branch's
+ * value gradient out of dv (dv holds the sparse branch's part only; see
+ * elsaa_race_value_grad). */
+elsaa_status elsaa_backward_tables(const elsaa_params* p, const void* q, const void* k,
+                                   const void* v, const void* r_sort, const void* r_race,
+                                   const float* gate_w, const float* gate_b, const float* lambda,
+                                   const void* saved, const void* dy, void* dq, void* dk, void* dv,
+                                   float* dgate_w, float* dgate_b, float* dlambda,
+                                   float* d_race_sum, void* ws, size_t ws_bytes, void* stream);
+
+/* The RACE branch's value gradient of keys k: dv[j] += sum_l dT[l][h_l(k_j)]
+ * (dv in the data dtype, [B,H,N,d]; d_race_sum as written by
+ * elsaa_backward_tables, summed over the shards). */
+elsaa_status elsaa_race_value_grad(const elsaa_params* p, const void* k, const void* r_race,
+                                   const float* d_race_sum, void* dv, void* ws, size_t ws_bytes,
+                                   void* stream);
+
 /* Bit mask of the kernel families elsaa_forward / elsaa_backward take for
  * `p` (0 if p is invalid): ELSAA_PATH_TC_HASH the tcgen05 SimHash GEMM;
  * ELSAA_PATH_TC_ATTN the tcgen05 sparse branch; ELSAA_PATH_SLAB_FWD the RACE

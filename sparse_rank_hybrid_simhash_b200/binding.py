@@ -76,7 +76,9 @@ class Views(ctypes.Structure):
 EXPORTS = ("elsaa_validate", "elsaa_workspace_bytes", "elsaa_saved_bytes", "elsaa_forward",
            "elsaa_backward", "elsaa_forward_staged", "elsaa_backward_staged",
            "elsaa_kernel_launches", "elsaa_saved_views", "elsaa_check", "elsaa_status_str",
-           "elsaa_uses_tensor_cores", "elsaa_sort_codes_noalloc", "elsaa_path_flags")
+           "elsaa_uses_tensor_cores", "elsaa_sort_codes_noalloc", "elsaa_path_flags",
+           "elsaa_sort_codes_of", "elsaa_sort_codes", "elsaa_race_tables", "elsaa_forward_tables",
+           "elsaa_backward_tables", "elsaa_race_value_grad")
 # elsaa_path_flags bits
 PATH_FLAGS = {"tc_hash": 1, "tc_attn": 2, "slab_fwd": 4, "slab_bwd": 8}
 FWD_STAGES = ("hash", "sort", "race_build", "sparse_fwd", "race_fuse")
@@ -101,6 +103,18 @@ def lib() -> ctypes.CDLL:
     L.elsaa_saved_bytes.argtypes, L.elsaa_saved_bytes.restype = [P], sz
     L.elsaa_uses_tensor_cores.argtypes, L.elsaa_uses_tensor_cores.restype = [P], ctypes.c_int32
     L.elsaa_path_flags.argtypes, L.elsaa_path_flags.restype = [P], ctypes.c_int32
+    L.elsaa_sort_codes_of.argtypes = [P] + [vp] * 6 + [sz, vp]
+    L.elsaa_sort_codes_of.restype = st
+    L.elsaa_sort_codes.argtypes = [P] + [vp] * 3 + [sz, vp]
+    L.elsaa_sort_codes.restype = st
+    L.elsaa_race_tables.argtypes = [P] + [vp] * 6 + [sz, vp]
+    L.elsaa_race_tables.restype = st
+    L.elsaa_forward_tables.argtypes = [P] + [vp] * 13 + [sz, vp]
+    L.elsaa_forward_tables.restype = st
+    L.elsaa_backward_tables.argtypes = [P] + [vp] * 18 + [sz, vp]
+    L.elsaa_backward_tables.restype = st
+    L.elsaa_race_value_grad.argtypes = [P] + [vp] * 5 + [sz, vp]
+    L.elsaa_race_value_grad.restype = st
     L.elsaa_forward.argtypes = [P] + [vp] * 10 + [vp, sz, vp]
     L.elsaa_forward.restype = st
     L.elsaa_backward.argtypes = [P] + [vp] * 17 + [sz, vp]
@@ -248,6 +262,79 @@ def sort_codes_noalloc(p: Params, code: torch.Tensor, perm: torch.Tensor, stream
             raise ValueError(f"tensors must be on the current device cuda:{cur}")
     _ok("elsaa_sort_codes_noalloc", lib().elsaa_sort_codes_noalloc(
         ctypes.byref(p), _ptr(code), _ptr(perm), _stream(stream)))
+
+
+# ---- pieces for a sequence split across devices (shard.py) -------------------
+
+def _tables_shape(p: Params):
+    return (p.B, p.H, p.race_tables, 1 << p.race_bits)
+
+
+def sort_codes_of(p: Params, q, k, r_sort, r_race, ws=None, stream=None) -> torch.Tensor:
+    """Sort codes [2, B, H, N] (int16 view of uint16) of q and k."""
+    ws = alloc_workspace(p, q.device) if ws is None else ws
+    code = torch.empty((2, p.B, p.H, p.N), dtype=torch.int16, device=q.device)
+    _ok("elsaa_sort_codes_of", lib().elsaa_sort_codes_of(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(r_sort), _ptr(r_race), _ptr(code), _ptr(ws),
+        ws.numel(), _stream(stream)))
+    return code
+
+
+def sort_codes(p: Params, code: torch.Tensor, ws=None, stream=None) -> torch.Tensor:
+    """Stable Sort-LSH order [2, B, H, N] int32 of codes [2, B, H, N]."""
+    ws = alloc_workspace(p, code.device) if ws is None else ws
+    perm = torch.empty((2, p.B, p.H, p.N), dtype=torch.int32, device=code.device)
+    _ok("elsaa_sort_codes", lib().elsaa_sort_codes(ctypes.byref(p), _ptr(code), _ptr(perm),
+                                                   _ptr(ws), ws.numel(), _stream(stream)))
+    return perm
+
+
+def race_tables(p: Params, k, v, r_race, ws=None, stream=None):
+    """RACE tables of k, v: (sums [B, H, L, NB, d] fp32, counts [B, H, L, NB] int32)."""
+    ws = alloc_workspace(p, k.device) if ws is None else ws
+    sums = torch.empty(_tables_shape(p) + (p.d,), dtype=torch.float32, device=k.device)
+    counts = torch.empty(_tables_shape(p), dtype=torch.int32, device=k.device)
+    _ok("elsaa_race_tables", lib().elsaa_race_tables(
+        ctypes.byref(p), _ptr(k), _ptr(v), _ptr(r_race), _ptr(sums), _ptr(counts), _ptr(ws),
+        ws.numel(), _stream(stream)))
+    return sums, counts
+
+
+def forward_tables(p: Params, q, k, v, r_sort, r_race, gate_w, gate_b, lam, sums, counts,
+                   y=None, saved=None, ws=None, stream=None) -> torch.Tensor:
+    """elsaa_forward with the RACE tables given."""
+    y = torch.empty_like(q) if y is None else y
+    ws = alloc_workspace(p, q.device) if ws is None else ws
+    _ok("elsaa_forward_tables", lib().elsaa_forward_tables(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(r_sort), _ptr(r_race), _ptr(gate_w),
+        _ptr(gate_b), _ptr(lam), _ptr(sums), _ptr(counts), _ptr(y), _ptr(saved), _ptr(ws),
+        ws.numel(), _stream(stream)))
+    return y
+
+
+def backward_tables(p: Params, q, k, v, r_sort, r_race, gate_w, gate_b, lam, saved, dy, ws,
+                    stream=None):
+    """(dq, dk, dv without the RACE value gradient, dgate_w, dgate_b, dlambda,
+    d_race_sum) of a forward_tables call."""
+    dev = q.device
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dgw = torch.empty(2, p.d, dtype=torch.float32, device=dev)
+    dgb = torch.empty(2, dtype=torch.float32, device=dev)
+    dlam = torch.empty(1, dtype=torch.float32, device=dev)
+    dsums = torch.empty(_tables_shape(p) + (p.d,), dtype=torch.float32, device=dev)
+    _ok("elsaa_backward_tables", lib().elsaa_backward_tables(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(r_sort), _ptr(r_race), _ptr(gate_w),
+        _ptr(gate_b), _ptr(lam), _ptr(saved), _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgw),
+        _ptr(dgb), _ptr(dlam), _ptr(dsums), _ptr(ws), ws.numel(), _stream(stream)))
+    return dq, dk, dv, dgw, dgb, dlam, dsums
+
+
+def race_value_grad(p: Params, k, r_race, d_sums, dv, ws=None, stream=None) -> None:
+    """dv += the RACE branch's value gradient of keys k (in place)."""
+    ws = alloc_workspace(p, k.device) if ws is None else ws
+    _ok("elsaa_race_value_grad", lib().elsaa_race_value_grad(
+        ctypes.byref(p), _ptr(k), _ptr(r_race), _ptr(d_sums), _ptr(dv), _ptr(ws), ws.numel(),
+        _stream(stream)))
 
 
 def check(ws: torch.Tensor, stream=None) -> None:

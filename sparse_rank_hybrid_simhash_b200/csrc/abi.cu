@@ -141,6 +141,8 @@ bool direct_bwd(const Geometry& g) {
   return g.tc_attn && attn_bwd3_supported(g) && race_gather_add_supported(g);
 }
 bool slab_bwd(const Geometry& g) { return direct_bwd(g) && race_slab_supported(g, false); }
+// the shared-memory value-gradient gather on its own (any attention path)
+bool slab_bwd_add(const Geometry& g) { return race_slab_supported(g, false); }
 
 #define ELSAA_TRY(expr)                               \
   do {                                                \
@@ -206,14 +208,26 @@ elsaa_status elsaa_saved_views(const elsaa_params* p, const void* saved, elsaa_v
   return ELSAA_OK;
 }
 
-elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const void* k,
-                                  const void* v, const void* r_sort, const void* r_race,
-                                  const float* gate_w, const float* gate_b, const float* lambda,
-                                  void* y, void* saved, void* ws, size_t ws_bytes, void* stream,
-                                  void* const* events) {
+}  // extern "C"
+
+namespace {
+
+// RACE tables given by the caller instead of built from this call's keys (a
+// sequence shard: the tables are sums over every shard's keys).
+struct ExtTables {
+  const float* sums;       // [BH][L][NB][d] fp32
+  const int32_t* counts;   // [BH][L][NB]
+};
+
+elsaa_status forward_impl(const elsaa_params* p, const void* q, const void* k, const void* v,
+                          const void* r_sort, const void* r_race, const float* gate_w,
+                          const float* gate_b, const float* lambda, void* y, void* saved,
+                          void* ws, size_t ws_bytes, void* stream, void* const* events,
+                          const ExtTables* ext) {
   Geometry g;
   elsaa_status why;
   if (!make_geometry(p, &g, &why)) return why;
+  if (ext && (g.causal || !ext->sums || !ext->counts)) return ELSAA_ERR_INVALID_ARG;
   if (!q || !k || !v || !lambda || !y || !ws) return ELSAA_ERR_INVALID_ARG;
   if ((g.sort_bits > 0 && !r_sort) || (g.kr > 0 && !r_race)) return ELSAA_ERR_INVALID_ARG;
   if (!g.gate_fixed && (!gate_w || !gate_b)) return ELSAA_ERR_INVALID_ARG;
@@ -274,14 +288,21 @@ elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const vo
     ELSAA_TRY(mark(events, 5, s));
     return ELSAA_OK;
   }
-  // 3. RACE tables from the keys
+  // 3. RACE tables from the keys (or the caller's tables)
   float* absmax = (float*)(w + wl.absmax);
-  ELSAA_TRY(launch_unit_absmax(g, v, false, absmax, s));
   // gathers read tables in the data dtype: a bf16 copy, or the fp32 sums themselves
   __nv_bfloat16* gtab = g.bf16 ? (__nv_bfloat16*)(w + wl.gtab) : nullptr;
   const void* gather_tables = g.bf16 ? (const void*)gtab : (const void*)sums;
-  ELSAA_TRY(launch_race_build(g, rcode_k, rcode_tk, v, false, absmax, sums, true, gtab, counts,
-                              (int32_t*)(w + wl.count_scratch), err, s));
+  if (ext) {
+    const size_t tab = (size_t)g.BH * g.L * g.NB;
+    ELSAA_TRY(cudaMemcpyAsync(sums, ext->sums, tab * g.d * 4, cudaMemcpyDeviceToDevice, s));
+    ELSAA_TRY(cudaMemcpyAsync(counts, ext->counts, tab * 4, cudaMemcpyDeviceToDevice, s));
+    if (gtab) ELSAA_TRY(launch_tables_to_bf16(g, sums, gtab, s));
+  } else {
+    ELSAA_TRY(launch_unit_absmax(g, v, false, absmax, s));
+    ELSAA_TRY(launch_race_build(g, rcode_k, rcode_tk, v, false, absmax, sums, true, gtab, counts,
+                                (int32_t*)(w + wl.count_scratch), err, s));
+  }
   ELSAA_TRY(mark(events, 3, s));
   // 4. exact sparse branch
   if (g.tc_attn && attn_pipe_supported(g))
@@ -305,25 +326,15 @@ elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const vo
   return ELSAA_OK;
 }
 
-elsaa_status elsaa_forward(const elsaa_params* p, const void* q, const void* k, const void* v,
-                           const void* r_sort, const void* r_race, const float* gate_w,
-                           const float* gate_b, const float* lambda, void* y, void* saved,
-                           void* ws, size_t ws_bytes, void* stream) {
-  return elsaa_forward_staged(p, q, k, v, r_sort, r_race, gate_w, gate_b, lambda, y, saved, ws,
-                              ws_bytes, stream, nullptr);
-}
-
-elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const void* k,
-                                   const void* v, const void* r_sort, const void* r_race,
-                                   const float* gate_w, const float* gate_b, const float* lambda,
-                                   const void* saved, const void* dy, void* dq, void* dk, void* dv,
-                                   float* dgate_w, float* dgate_b, float* dlambda, void* ws,
-                                   size_t ws_bytes, void* stream, void* const* events) {
-  (void)r_sort;
-  (void)r_race;
+elsaa_status backward_impl(const elsaa_params* p, const void* q, const void* k, const void* v,
+                           const float* gate_w, const float* gate_b, const float* lambda,
+                           const void* saved, const void* dy, void* dq, void* dk, void* dv,
+                           float* dgate_w, float* dgate_b, float* dlambda, void* ws,
+                           size_t ws_bytes, void* stream, void* const* events, float* d_tables) {
   Geometry g;
   elsaa_status why;
   if (!make_geometry(p, &g, &why)) return why;
+  if (d_tables && g.causal) return ELSAA_ERR_INVALID_ARG;
   if (!q || !k || !v || !lambda || !saved || !dy || !dq || !dk || !dv || !dlambda || !ws)
     return ELSAA_ERR_INVALID_ARG;
   if (!g.gate_fixed && (!gate_w || !gate_b)) return ELSAA_ERR_INVALID_ARG;
@@ -376,6 +387,13 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
   if (g.causal) {
     ELSAA_TRY(cudaMemsetAsync(dv_acc, 0, bhn * g.d * 4, s));
     ELSAA_TRY(launch_race_causal_bwd(g, rcode, rcode_k, dor, dv_acc, s));
+  } else if (d_tables) {
+    // the caller's table gradient (fp32); the value gradient of the RACE
+    // branch is left to the caller (elsaa_race_value_grad once dT is summed)
+    ELSAA_TRY(launch_race_build(g, rcode, rcode_t, dor, false, absmax, d_tables, true, nullptr,
+                                nullptr, (int32_t*)(w + wl.count_scratch),
+                                (uint32_t*)(w + wl.err), s));
+    if (!direct) ELSAA_TRY(cudaMemsetAsync(dv_acc, 0, bhn * g.d * 4, s));
   } else {
     ELSAA_TRY(launch_race_build(g, rcode, rcode_t, dor, false, absmax, d_t, !g.bf16, gtab,
                                 nullptr, (int32_t*)(w + wl.count_scratch),
@@ -389,10 +407,13 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
                                g.gate_fixed ? nullptr : gate_w, dq, dk, dv,
                                (uint32_t*)(w + wl.err), s));
     ELSAA_TRY(mark(events, 3, s));
-    if (slab_bwd(g))
+    if (d_tables) {
+      // (the caller adds the RACE value gradient)
+    } else if (slab_bwd(g)) {
       ELSAA_TRY(launch_race_slab_add(g, rcode_k, race_grad, dv, (uint32_t*)(w + wl.err), s));
-    else
+    } else {
       ELSAA_TRY(launch_race_gather_add(g, rcode_k, race_grad, dv, s));
+    }
   } else if (g.tc_attn && attn_bwd2_supported(g)) {
     ELSAA_TRY(launch_attn_bwd2(g, q, k, v, perm, perm + bhn, d_o, lse, dprime, dv_acc, dq_acc,
                                dk, dv, (uint32_t*)(w + wl.err), s));
@@ -417,14 +438,72 @@ elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const v
   return ELSAA_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+elsaa_status elsaa_forward_staged(const elsaa_params* p, const void* q, const void* k,
+                                  const void* v, const void* r_sort, const void* r_race,
+                                  const float* gate_w, const float* gate_b, const float* lambda,
+                                  void* y, void* saved, void* ws, size_t ws_bytes, void* stream,
+                                  void* const* events) {
+  return forward_impl(p, q, k, v, r_sort, r_race, gate_w, gate_b, lambda, y, saved, ws, ws_bytes,
+                      stream, events, nullptr);
+}
+
+elsaa_status elsaa_forward(const elsaa_params* p, const void* q, const void* k, const void* v,
+                           const void* r_sort, const void* r_race, const float* gate_w,
+                           const float* gate_b, const float* lambda, void* y, void* saved,
+                           void* ws, size_t ws_bytes, void* stream) {
+  return forward_impl(p, q, k, v, r_sort, r_race, gate_w, gate_b, lambda, y, saved, ws, ws_bytes,
+                      stream, nullptr, nullptr);
+}
+
+elsaa_status elsaa_forward_tables(const elsaa_params* p, const void* q, const void* k,
+                                  const void* v, const void* r_sort, const void* r_race,
+                                  const float* gate_w, const float* gate_b, const float* lambda,
+                                  const float* race_sum, const int32_t* race_count, void* y,
+                                  void* saved, void* ws, size_t ws_bytes, void* stream) {
+  const ExtTables ext{race_sum, race_count};
+  return forward_impl(p, q, k, v, r_sort, r_race, gate_w, gate_b, lambda, y, saved, ws, ws_bytes,
+                      stream, nullptr, &ext);
+}
+
+elsaa_status elsaa_backward_staged(const elsaa_params* p, const void* q, const void* k,
+                                   const void* v, const void* r_sort, const void* r_race,
+                                   const float* gate_w, const float* gate_b, const float* lambda,
+                                   const void* saved, const void* dy, void* dq, void* dk, void* dv,
+                                   float* dgate_w, float* dgate_b, float* dlambda, void* ws,
+                                   size_t ws_bytes, void* stream, void* const* events) {
+  (void)r_sort;
+  (void)r_race;
+  return backward_impl(p, q, k, v, gate_w, gate_b, lambda, saved, dy, dq, dk, dv, dgate_w,
+                       dgate_b, dlambda, ws, ws_bytes, stream, events, nullptr);
+}
+
 elsaa_status elsaa_backward(const elsaa_params* p, const void* q, const void* k, const void* v,
                             const void* r_sort, const void* r_race, const float* gate_w,
                             const float* gate_b, const float* lambda, const void* saved,
                             const void* dy, void* dq, void* dk, void* dv, float* dgate_w,
                             float* dgate_b, float* dlambda, void* ws, size_t ws_bytes,
                             void* stream) {
-  return elsaa_backward_staged(p, q, k, v, r_sort, r_race, gate_w, gate_b, lambda, saved, dy, dq,
-                               dk, dv, dgate_w, dgate_b, dlambda, ws, ws_bytes, stream, nullptr);
+  (void)r_sort;
+  (void)r_race;
+  return backward_impl(p, q, k, v, gate_w, gate_b, lambda, saved, dy, dq, dk, dv, dgate_w,
+                       dgate_b, dlambda, ws, ws_bytes, stream, nullptr, nullptr);
+}
+
+elsaa_status elsaa_backward_tables(const elsaa_params* p, const void* q, const void* k,
+                                   const void* v, const void* r_sort, const void* r_race,
+                                   const float* gate_w, const float* gate_b, const float* lambda,
+                                   const void* saved, const void* dy, void* dq, void* dk, void* dv,
+                                   float* dgate_w, float* dgate_b, float* dlambda,
+                                   float* d_race_sum, void* ws, size_t ws_bytes, void* stream) {
+  (void)r_sort;
+  (void)r_race;
+  if (!d_race_sum) return ELSAA_ERR_INVALID_ARG;
+  return backward_impl(p, q, k, v, gate_w, gate_b, lambda, saved, dy, dq, dk, dv, dgate_w,
+                       dgate_b, dlambda, ws, ws_bytes, stream, nullptr, d_race_sum);
 }
 
 elsaa_status elsaa_kernel_launches(const elsaa_params* p, int32_t* fwd, int32_t* bwd) {
@@ -448,6 +527,138 @@ elsaa_status elsaa_kernel_launches(const elsaa_params* p, int32_t* fwd, int32_t*
   // (the RACE backward: the table-gradient build, then, off the direct path, a gather)
   const int race_bwd = g.causal ? 1 : race_build_kernels(g, false, g.bf16) + (direct ? 0 : 1);
   *bwd = 1 + race_bwd + sparse + (direct ? 1 : 0) + 1;
+  return ELSAA_OK;
+}
+
+// ---- pieces of the operator for a sequence split across devices ------------
+
+elsaa_status elsaa_sort_codes_of(const elsaa_params* p, const void* q, const void* k,
+                                 const void* r_sort, const void* r_race, uint16_t* code,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  Geometry g;
+  elsaa_status why;
+  if (!make_geometry(p, &g, &why)) return why;
+  if (!q || !k || !code || !ws || (g.sort_bits > 0 && !r_sort) || (g.kr > 0 && !r_race))
+    return ELSAA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(code, 16) || !aligned(ws, 256))
+    return ELSAA_ERR_INVALID_ARG;
+  const WorkLayout wl = work_layout(g);
+  if (ws_bytes < wl.total) return ELSAA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  char* w = (char*)ws;
+  char* sv = w + wl.saved;   // the hash writes into the workspace's saved-state area
+  const SavedLayout sl = saved_layout(g);
+  const size_t bhn = (size_t)g.BH * g.N;
+  uint16_t* c = (uint16_t*)(sv + sl.code);
+  char* rcode = sv + sl.rcode;
+  char* rcode_t = sv + sl.rcode_t;
+  uint32_t* err = (uint32_t*)(w + wl.err);
+  ELSAA_TRY(cudaMemsetAsync(err, 0, sizeof(uint32_t), s));
+  if (g.tc_hash)
+    ELSAA_TRY(launch_hash_tc(g, q, k, r_sort, r_race, c, rcode, rcode_t, nullptr, nullptr, err, s));
+  else
+    ELSAA_TRY(launch_hash_simt(g, q, k, r_sort, r_race, c, rcode, rcode_t, s));
+  ELSAA_TRY(cudaMemcpyAsync(code, c, 2 * bhn * 2, cudaMemcpyDeviceToDevice, s));
+  return ELSAA_OK;
+}
+
+elsaa_status elsaa_sort_codes(const elsaa_params* p, const uint16_t* code, int32_t* perm,
+                              void* ws, size_t ws_bytes, void* stream) {
+  Geometry g;
+  elsaa_status why;
+  if (!make_geometry(p, &g, &why)) return why;
+  if (!code || !perm || !ws) return ELSAA_ERR_INVALID_ARG;
+  if (!aligned(code, 16) || !aligned(perm, 16) || !aligned(ws, 256)) return ELSAA_ERR_INVALID_ARG;
+  const WorkLayout wl = work_layout(g);
+  if (ws_bytes < wl.total) return ELSAA_ERR_WORKSPACE;
+  char* w = (char*)ws;
+  ELSAA_TRY(launch_sort(g, code, perm, (int32_t*)(w + wl.sort_hist), (int32_t*)(w + wl.sort_tmp),
+                        (cudaStream_t)stream));
+  return ELSAA_OK;
+}
+
+elsaa_status elsaa_race_tables(const elsaa_params* p, const void* k, const void* v,
+                               const void* r_race, float* race_sum, int32_t* race_count,
+                               void* ws, size_t ws_bytes, void* stream) {
+  Geometry g;
+  elsaa_status why;
+  if (!make_geometry(p, &g, &why)) return why;
+  if (!k || !v || !race_sum || !race_count || !ws || (g.kr > 0 && !r_race))
+    return ELSAA_ERR_INVALID_ARG;
+  const void* ptrs[] = {k, v, race_sum, race_count};
+  for (const void* x : ptrs)
+    if (!aligned(x, 16)) return ELSAA_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return ELSAA_ERR_INVALID_ARG;
+  const WorkLayout wl = work_layout(g);
+  if (ws_bytes < wl.total) return ELSAA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  char* w = (char*)ws;
+  char* sv = w + wl.saved;
+  const SavedLayout sl = saved_layout(g);
+  const size_t bhn = (size_t)g.BH * g.N;
+  uint16_t* c = (uint16_t*)(sv + sl.code);
+  char* rcode = sv + sl.rcode;
+  char* rcode_t = sv + sl.rcode_t;
+  uint32_t* err = (uint32_t*)(w + wl.err);
+  ELSAA_TRY(cudaMemsetAsync(err, 0, sizeof(uint32_t), s));
+  // the keys' RACE codes (the hash also codes its first operand: the keys
+  // again); no sort hyperplanes are read
+  Geometry gk = g;
+  gk.sort_bits = 0;
+  if (gk.tc_hash)
+    ELSAA_TRY(launch_hash_tc(gk, k, k, nullptr, r_race, c, rcode, rcode_t, nullptr, nullptr, err,
+                             s));
+  else
+    ELSAA_TRY(launch_hash_simt(gk, k, k, nullptr, r_race, c, rcode, rcode_t, s));
+  float* absmax = (float*)(w + wl.absmax);
+  ELSAA_TRY(launch_unit_absmax(g, v, false, absmax, s));
+  ELSAA_TRY(launch_race_build(g, rcode + bhn * g.L * g.rcode_bytes,
+                              rcode_t + bhn * g.L * g.rcode_bytes, v, false, absmax, race_sum,
+                              true, nullptr, race_count, (int32_t*)(w + wl.count_scratch), err,
+                              s));
+  return ELSAA_OK;
+}
+
+elsaa_status elsaa_race_value_grad(const elsaa_params* p, const void* k, const void* r_race,
+                                   const float* d_race_sum, void* dv, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  Geometry g;
+  elsaa_status why;
+  if (!make_geometry(p, &g, &why)) return why;
+  if (!k || !d_race_sum || !dv || !ws || (g.kr > 0 && !r_race)) return ELSAA_ERR_INVALID_ARG;
+  if (!aligned(k, 16) || !aligned(d_race_sum, 16) || !aligned(dv, 16) || !aligned(ws, 256))
+    return ELSAA_ERR_INVALID_ARG;
+  if (!race_gather_add_supported(g)) return ELSAA_ERR_UNSUPPORTED;
+  const WorkLayout wl = work_layout(g);
+  if (ws_bytes < wl.total) return ELSAA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  char* w = (char*)ws;
+  char* sv = w + wl.saved;
+  const SavedLayout sl = saved_layout(g);
+  const size_t bhn = (size_t)g.BH * g.N;
+  uint16_t* c = (uint16_t*)(sv + sl.code);
+  char* rcode = sv + sl.rcode;
+  char* rcode_t = sv + sl.rcode_t;
+  uint32_t* err = (uint32_t*)(w + wl.err);
+  ELSAA_TRY(cudaMemsetAsync(err, 0, sizeof(uint32_t), s));
+  Geometry gk = g;   // RACE codes of the keys only: no sort hyperplanes
+  gk.sort_bits = 0;
+  if (gk.tc_hash)
+    ELSAA_TRY(launch_hash_tc(gk, k, k, nullptr, r_race, c, rcode, rcode_t, nullptr, nullptr, err,
+                             s));
+  else
+    ELSAA_TRY(launch_hash_simt(gk, k, k, nullptr, r_race, c, rcode, rcode_t, s));
+  const char* rcode_k = rcode + bhn * g.L * g.rcode_bytes;
+  const void* tables = d_race_sum;
+  if (g.bf16) {
+    __nv_bfloat16* gtab = (__nv_bfloat16*)(w + wl.gtab);
+    ELSAA_TRY(launch_tables_to_bf16(g, d_race_sum, gtab, s));
+    tables = gtab;
+  }
+  if (slab_bwd_add(g))
+    ELSAA_TRY(launch_race_slab_add(g, rcode_k, tables, dv, err, s));
+  else
+    ELSAA_TRY(launch_race_gather_add(g, rcode_k, tables, dv, s));
   return ELSAA_OK;
 }
 

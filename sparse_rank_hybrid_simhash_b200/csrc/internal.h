@@ -114,6 +114,9 @@ cudaError_t launch_unit_absmax(const Geometry& g, const void* vals, bool vals_f3
 // codes: [BH][N][L] row-major; codes_t: the same codes [BH][L][N] table-major.
 // count_scratch: [BH][L][NB] int32 the segmented build counts into when
 // `counts` is null (long sequences need the counts to size the fixed-point grid).
+// bf16 copy of fp32 tables [BH][L][NB][d] (what the gathers read).
+cudaError_t launch_tables_to_bf16(const Geometry& g, const float* sums, __nv_bfloat16* gtab,
+                                  cudaStream_t s);
 // Kernels one launch_race_build enqueues (memsets excluded).
 int race_build_kernels(const Geometry& g, bool vals_f32, bool gtab);
 cudaError_t launch_race_build(const Geometry& g, const void* codes, const void* codes_t,

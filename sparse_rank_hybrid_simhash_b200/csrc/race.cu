@@ -1619,6 +1619,13 @@ cudaError_t launch_race_build(const Geometry& g, const void* codes, const void* 
                                               gtab, counts, count_scratch, err, s);
 }
 
+cudaError_t launch_tables_to_bf16(const Geometry& g, const float* sums, __nv_bfloat16* gtab,
+                                  cudaStream_t s) {
+  const int64_t n = (int64_t)g.BH * g.L * g.NB * g.d;
+  to_bf16_kernel<<<148 * 8, 256, 0, s>>>(sums, gtab, n);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_race_gather_sum(const Geometry& g, const void* codes, const void* tables,
                                    float* out, cudaStream_t s) {
   if (g.bf16) {

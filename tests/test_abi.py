@@ -188,3 +188,16 @@ def test_path_flags():
     assert B.path_flags(B.Params.from_workload(w.replace(hash_rounds=2)))["slab_fwd"]
     assert B.path_flags(B.Params.make(1, 1, 256, 64, "bf16", 4, 64, 8, 6)) == {
         "tc_hash": True, "tc_attn": True, "slab_fwd": False, "slab_bwd": False}
+
+
+def test_binding_argument_counts_match_the_header():
+    # every bound entry point takes as many arguments as its declaration
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    lib = B.lib()
+    for name in B.EXPORTS:
+        m = re.search(r"\b" + name + r"\s*\(([^)]*)\)\s*;", text)
+        assert m, name
+        params = [x for x in m.group(1).split(",") if x.strip() and x.strip() != "void"]
+        argtypes = getattr(lib, name).argtypes
+        assert argtypes is not None and len(argtypes) == len(params), \
+            f"{name}: {len(argtypes or [])} bound, {len(params)} declared"
