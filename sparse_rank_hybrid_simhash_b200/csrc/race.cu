@@ -664,12 +664,18 @@ ELSAA_DEV void add_f32x2(float& a0, float& a1, float b0, float b1) {
       : "+f"(a0), "+f"(a1)
       : "f"(b0), "f"(b1));
 }
+// acc += a row's 8 bf16 values by mixed-precision adds (bf16 operand, fp32
+// accumulator: the sums of converting first, in fewer instructions)
 ELSAA_DEV void add_row(float* acc, uint4 raw, const __nv_bfloat16*) {
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i)
-    add_f32x2(acc[2 * i], acc[2 * i + 1], __uint_as_float(w[i] << 16),
-              __uint_as_float(w[i] & 0xFFFF0000u));
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "mov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\t"
+        "add.rn.f32.bf16 %1, hi, %1;\n\t}"
+        : "+f"(acc[2 * i]), "+f"(acc[2 * i + 1])
+        : "r"(w[i]));
 }
 ELSAA_DEV void add_row(float* acc, uint4 raw, const float*) {
   add_f32x2(acc[0], acc[1], __uint_as_float(raw.x), __uint_as_float(raw.y));
