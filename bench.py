@@ -11,6 +11,7 @@ synthetic tensors resident in HBM before the timed region.
                     [--sort-order binary|gray|local] [--lookback L] [--hash-rounds R]
                     [--causal]
                     [--dense-context] [--no-cpu-baseline] [--no-other-workloads]
+                    [--seq-shards P]
 
 The modes are the method's ablations on the same kernels (lambda = 0, or one
 branch gated off); sort order, lookback and causal select the extensions of
@@ -22,6 +23,10 @@ scaling, different seed per rank); the shared gate and lambda gradients are
 summed across ranks with one NCCL all-reduce inside the step.  Time is device
 time (CUDA events on the launching stream), max over ranks.  Rank 0 prints one
 JSON line.
+
+``--seq-shards P`` times instead the workload with every unit's sequence split
+into P token shards (shard.py): one per rank under torchrun, or all of them in
+one process on one GPU (an emulation; the line says so).
 
 ``--impl reference`` times the fp64 CPU oracle (the reference arm: there is no
 runnable reference implementation) on a bounded sample of the same workload.
@@ -464,7 +469,8 @@ def run_e2e(args, w, p, inp, dev, world):
     (pipeline.HostStepPipeline: copy-in, compute and copy-out overlap)."""
     from sparse_rank_hybrid_simhash_b200.pipeline import HostStepPipeline
     BH = w.B * w.H
-    groups = next(g for g in (4, 3, 2, 1) if BH % g == 0)
+    # more groups shorten the unoverlapped first copy-in and last copy-out
+    groups = next(g for g in (8, 6, 4, 3, 2, 1) if BH % g == 0)
     host = {k: inp[k].pin_memory() for k in ("q", "k", "v", "dy")}
     outs = {k: torch.empty_like(host["q"], pin_memory=True) for k in ("y", "dq", "dk", "dv")}
     pipe = HostStepPipeline(p, groups, dev, inp["r_sort"], inp["r_race"], inp["gate_w"],
@@ -500,6 +506,72 @@ def run_e2e(args, w, p, inp, dev, world):
     return {"value": world * n * w.tokens / (ms / 1e3), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
             "pipeline": f"{groups} head groups; copy-in, compute and copy-out streams overlap"}
+
+
+# ---------------------------------------------------------------------------
+# a sequence split over ranks (shard.py)
+# ---------------------------------------------------------------------------
+
+def run_seq_shards(args, rank, world, local_rank):
+    """Forward (and backward where the workload has one) of one workload with
+    every unit's sequence split into args.seq_shards token shards: one shard
+    per rank under torchrun (NCCL collectives), or every shard in this process
+    on one GPU (the collectives become device copies: an emulation of the
+    split, all shards' work serialised).  Total work is fixed (strong scaling)."""
+    from sparse_rank_hybrid_simhash_b200.shard import DistComm, LocalComm, ShardedElsaa
+    P = args.seq_shards
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    p = B.Params.from_workload(w)
+    if world > 1:
+        if world != P:
+            raise SystemExit("--seq-shards must equal the number of ranks")
+        comm, mine = DistComm(), [rank]
+    else:
+        comm, mine = LocalComm(P), list(range(P))
+    inp = make_inputs(w, with_dy=w.backward)
+    M = w.N // P
+    sh = {n: [inp[n][:, :, r * M:(r + 1) * M].contiguous().to(dev) for r in mine]
+          for n in (("q", "k", "v", "dy") if w.backward else ("q", "k", "v"))}
+    args_ = tuple(inp[n].to(dev) for n in ("r_sort", "r_race", "gate_w", "gate_b", "lam"))
+    op = ShardedElsaa(p, comm)
+
+    def step():
+        op.forward(sh["q"], sh["k"], sh["v"], *args_)
+        if w.backward:
+            op.backward(sh["dy"], *args_)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(args.steps):
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        ms = DP.max_over_ranks([ms], dev)[0]
+    if rank == 0:
+        line = {
+            "metric": f"ELSAA tokens/s, {w.name} sequence split over {P} shards "
+                      + ("(fwd+bwd)" if w.backward else "(fwd)"),
+            "value": args.steps * w.tokens / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": w.dtype, "data": STANDS_IN_FOR.get(w.name, "synthetic (seeded)"),
+            "config": dict(bench_config(w, "elsaa", world, "inputs > L2"), seq_shards=P,
+                           parallelism=f"sequence split x{P}"),
+            "emulated": world == 1 and P > 1,
+            "note": ("all shards in one process on one GPU: collectives are device copies and "
+                     "the shards' work is serialised" if world == 1 and P > 1 else
+                     "one shard per rank, NCCL all-gather / all-to-all / all-reduce"),
+        }
+        print(json.dumps(line), flush=True)
 
 
 # ---------------------------------------------------------------------------
@@ -685,6 +757,9 @@ def main():
                     help="keys j <= i only (CUDA-core attention, RACE token scans)")
     ap.add_argument("--dense-context", action="store_true",
                     help="also time dense torch SDPA fwd+bwd on the same inputs (context)")
+    ap.add_argument("--seq-shards", type=int, default=0,
+                    help="split every unit's sequence into this many token shards (one per "
+                         "rank under torchrun; all in this process on one GPU)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override B (small cases for ncu captures; not a bench line)")
     ap.add_argument("--heads", type=int, default=None,
@@ -703,6 +778,12 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
+    if args.seq_shards:
+        run_seq_shards(args, rank, world, local_rank)
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
     w, p, total_ms, fwd_ms, stage_ms, clocks, e2e, context, dev_unit = run_ours(
         args, rank, world, local_rank)
     peaks = load_peaks()
