@@ -119,34 +119,42 @@ def stage_roofline(flops, nbytes, sec, peaks):
             "ideal_us": 1e6 * max(flops / tf, nbytes / hb)}
 
 
-# DRAM bytes (read + write) of one launch of a stage's main kernel, from an
-# ncu capture of the same source (sha1 of the kernel file), scaled to the full
-# workload by the number of units; reported only while that file is unchanged.
+# DRAM bytes (read + write) of one launch of a stage's main kernel on the
+# text-32k workload, from an ncu capture at 12 heads (B=1, H=12) of the same
+# source (sha1 of the kernel file); scaled to a launch by the number of
+# (batch, head) units, and reported only while that file is unchanged and the
+# stage runs the captured kernel (the slab kernels where the path flags say so).
+TRAFFIC_WORKLOAD, TRAFFIC_UNITS = "text-32k", 12
 RECORDED_TRAFFIC = {
-    # stage: (kernel source, its sha1 at capture, bytes per full-size launch)
-    "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "495295df2fda78a4a966636d9641afe4401ac126", 2.459e+08),
-    "race_build": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "0d588b8c632b81b3ffdfb0a8110ff049180f2520", 1.372e+08),
-    "sparse_fwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_pipe.cu", "91a31d0c88874e37ef33ed4bb443baabc0c07369", 3.735e+08),
-    "race_fuse": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "0d588b8c632b81b3ffdfb0a8110ff049180f2520", 3.717e+08),
-    "fuse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/fuse_bwd.cu", "d225c68863731ac35a2126d849af1623d8c512c7", 5.621e+08),
-    "race_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "0d588b8c632b81b3ffdfb0a8110ff049180f2520", 1.34e+08),
-    "sparse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_bwd3.cu", "d8764bf2cfd3093b7f01c78d4ad9412897ad1eeb", 6.626e+08),
-    "finish": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "0d588b8c632b81b3ffdfb0a8110ff049180f2520", 1.586e+08),
+    # stage: (kernel source, its sha1 at capture, bytes per 12-unit launch, path flag needed)
+    "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "d38b93c83be7bafa7040797e9a19dce5b2ba90f0", 1.259e+08, "tc_hash"),
+    "race_build": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "15a1fb45c20eb380372ec944794c10506c62861f", 6.91e+07, None),
+    "sparse_fwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_pipe.cu", "91a31d0c88874e37ef33ed4bb443baabc0c07369", 1.87e+08, "tc_attn"),
+    "race_fuse": ("sparse_rank_hybrid_simhash_b200/csrc/race_slab.cu", "5135a962ed6cf3d305d45cb27ffcdf41815cc38e", 1.448e+08, "slab_fwd"),
+    "fuse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/fuse_bwd.cu", "d225c68863731ac35a2126d849af1623d8c512c7", 2.817e+08, None),
+    "race_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "15a1fb45c20eb380372ec944794c10506c62861f", 6.67e+07, None),
+    "sparse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_bwd3.cu", "d8764bf2cfd3093b7f01c78d4ad9412897ad1eeb", 3.321e+08, "tc_attn"),
+    "finish": ("sparse_rank_hybrid_simhash_b200/csrc/race_slab.cu", "5135a962ed6cf3d305d45cb27ffcdf41815cc38e", 7.85e+07, "slab_bwd"),
 }
 
 
-def recorded_traffic(stage):
+def recorded_traffic(w, stage, path):
+    """DRAM bytes of one full launch of the stage's kernel, or None when the
+    capture does not describe what this run launches."""
     rec = RECORDED_TRAFFIC.get(stage)
-    if rec is None:
+    ref = WORKLOADS[TRAFFIC_WORKLOAD]
+    if rec is None or w.replace(B=ref.B, H=ref.H, seed=ref.seed) != ref:
         return None
-    src, sha, nbytes = rec
+    src, sha, nbytes, flag = rec
+    if flag is not None and not path.get(flag, False):
+        return None
     try:
         with open(os.path.join(ROOT, src), "rb") as f:
             if hashlib.sha1(f.read()).hexdigest() != sha:
                 return None
     except OSError:
         return None
-    return nbytes
+    return nbytes * (w.B * w.H) / TRAFFIC_UNITS
 
 
 def operator_roofline(w, peaks):
@@ -796,7 +804,8 @@ def main():
                      for st in stage_ms}
         dom = max(stage_ms, key=lambda st: stage_ms[st])
         rl = per_stage[dom]
-        traffic = recorded_traffic(dom)
+        path = B.path_flags(p)
+        traffic = recorded_traffic(w, dom, path)
         roof = operator_roofline(w, peaks)
         fwd_launch, bwd_launch = B.kernel_launches(p)
         line = {
@@ -813,8 +822,10 @@ def main():
                          "traffic": traffic,
                          "peak_source": peaks["source"] + (" sustained" if rl["bound"] == "tensor"
                                                            else "")},
-            "stage_roofline": {st: {k: (round(v, 4) if isinstance(v, float) else v)
-                                    for k, v in r.items()} for st, r in per_stage.items()},
+            "stage_roofline": {st: dict({k: (round(v, 4) if isinstance(v, float) else v)
+                                         for k, v in r.items()},
+                                        traffic=recorded_traffic(w, st, path))
+                               for st, r in per_stage.items()},
             "operator_roofline": {
                 "fwd_us": roof["fwd_us"], "fwdbwd_us": roof["fwdbwd_us"],
                 "frac_fwd": roof["fwd_us"] / (1e3 * fwd_ms / K),
@@ -825,8 +836,8 @@ def main():
         }
         line["interactions"] = interaction_count(w)
         line["race_onchip"] = race_onchip_bound(w, stage_ms, clocks.get("sm_mhz"),
-                                                B.path_flags(p)["slab_fwd"])
-        line["path"] = B.path_flags(p)
+                                                path["slab_fwd"])
+        line["path"] = path
         if context is not None:
             line["context"] = {"dense_sdpa": context}
         if world == 1 and not args.no_other_workloads and args.workload == WORKLOAD:

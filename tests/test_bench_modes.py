@@ -63,3 +63,18 @@ def test_operator_roofline_of_the_text_workload():
     assert abs(r["fwd_us"] - 65.0) < 0.1 and abs(r["fwdbwd_us"] - 202.0) < 0.1
     # lookback widens the window: chunk j sees min(j, lb) + 1 chunks
     assert bench.window_keys(1024, 128, 3) == 128 * 128 * sum(min(j, 3) + 1 for j in range(8))
+
+
+def test_recorded_traffic_only_describes_the_captured_kernels():
+    # DRAM bytes from a capture at 12 heads scale with the units of the run and
+    # are withheld where the run launches something else
+    bench = _bench()
+    w = WORKLOADS["text-32k"]
+    path = {"tc_hash": True, "tc_attn": True, "slab_fwd": True, "slab_bwd": True}
+    full = bench.recorded_traffic(w, "sparse_bwd", path)
+    assert full is not None and full > 0
+    assert bench.recorded_traffic(w.replace(B=1), "sparse_bwd", path) == full / 2
+    assert bench.recorded_traffic(w, "race_fuse", dict(path, slab_fwd=False)) is None
+    assert bench.recorded_traffic(w.replace(lookback=2), "sparse_bwd", path) is None
+    assert bench.recorded_traffic(WORKLOADS["iid-4k"], "sparse_bwd", path) is None
+    assert bench.recorded_traffic(bench.apply_mode(w, "race_only"), "hash", path) is None
