@@ -303,11 +303,15 @@ elsaa_status elsaa_race_value_grad(const elsaa_params* p, const void* k, const v
  * `p` (0 if p is invalid): ELSAA_PATH_TC_HASH the tcgen05 SimHash GEMM;
  * ELSAA_PATH_TC_ATTN the tcgen05 sparse branch; ELSAA_PATH_SLAB_FWD the RACE
  * read-out from shared-memory table slabs (gate logits from the hash GEMM);
- * ELSAA_PATH_SLAB_BWD the RACE value gradient from shared-memory slabs. */
+ * ELSAA_PATH_SLAB_BWD the RACE value gradient from shared-memory slabs;
+ * ELSAA_PATH_TC_WIN the sparse forward on the tcgen05 kernel that streams
+ * the window in 128-key blocks (d = 128, chunks above 128, lookback other
+ * than 1; the backward of those shapes runs on CUDA cores). */
 #define ELSAA_PATH_TC_HASH 1
 #define ELSAA_PATH_TC_ATTN 2
 #define ELSAA_PATH_SLAB_FWD 4
 #define ELSAA_PATH_SLAB_BWD 8
+#define ELSAA_PATH_TC_WIN 16
 int32_t elsaa_path_flags(const elsaa_params* p);
 
 #ifdef __cplusplus

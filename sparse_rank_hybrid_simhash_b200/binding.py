@@ -80,7 +80,7 @@ EXPORTS = ("elsaa_validate", "elsaa_workspace_bytes", "elsaa_saved_bytes", "elsa
            "elsaa_sort_codes_of", "elsaa_sort_codes", "elsaa_race_tables", "elsaa_forward_tables",
            "elsaa_backward_tables", "elsaa_race_value_grad")
 # elsaa_path_flags bits
-PATH_FLAGS = {"tc_hash": 1, "tc_attn": 2, "slab_fwd": 4, "slab_bwd": 8}
+PATH_FLAGS = {"tc_hash": 1, "tc_attn": 2, "slab_fwd": 4, "slab_bwd": 8, "tc_win": 16}
 FWD_STAGES = ("hash", "sort", "race_build", "sparse_fwd", "race_fuse")
 BWD_STAGES = ("fuse_bwd", "race_bwd", "sparse_bwd", "finish")
 

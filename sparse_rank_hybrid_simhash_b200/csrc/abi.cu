@@ -135,6 +135,12 @@ bool slab_fwd(const Geometry& g) {
   return g.tc_hash && !g.causal && race_slab_supported(g, true) &&
          (g.gate_fixed || hash_tc_gate_logits_supported(g));
 }
+// The sparse forward streams the window in 128-key blocks where the
+// lookback-1 pipeline does not apply (d = 128, chunks above 128, other
+// lookbacks).
+bool win_fwd(const Geometry& g) {
+  return !(g.tc_attn && attn_pipe_supported(g)) && attn_win_supported(g);
+}
 // The persistent sparse backward writes dq, dk and dv itself; the RACE
 // branch's dv is then added in place by a key-code gather.
 bool direct_bwd(const Geometry& g) {
@@ -307,6 +313,8 @@ elsaa_status forward_impl(const elsaa_params* p, const void* q, const void* k, c
   // 4. exact sparse branch
   if (g.tc_attn && attn_pipe_supported(g))
     ELSAA_TRY(launch_attn_fwd_pipe(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s));
+  else if (win_fwd(g))
+    ELSAA_TRY(launch_attn_fwd_win(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s));
   else if (g.tc_attn)
     ELSAA_TRY(launch_attn_fwd_tc(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s));
   else
@@ -667,7 +675,8 @@ int32_t elsaa_path_flags(const elsaa_params* p) {
   elsaa_status why;
   if (!make_geometry(p, &g, &why)) return 0;
   return (g.tc_hash ? ELSAA_PATH_TC_HASH : 0) | (g.tc_attn ? ELSAA_PATH_TC_ATTN : 0) |
-         (slab_fwd(g) ? ELSAA_PATH_SLAB_FWD : 0) | (slab_bwd(g) ? ELSAA_PATH_SLAB_BWD : 0);
+         (slab_fwd(g) ? ELSAA_PATH_SLAB_FWD : 0) | (slab_bwd(g) ? ELSAA_PATH_SLAB_BWD : 0) |
+         (win_fwd(g) ? ELSAA_PATH_TC_WIN : 0);
 }
 
 elsaa_status elsaa_check(void* ws, void* stream) {

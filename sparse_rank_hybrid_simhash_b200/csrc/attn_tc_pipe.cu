@@ -14,17 +14,20 @@
 // Scores fit in 256 TMEM columns (block tb - 1 in [0, 128), block tb in
 // [128, 256)); the softmax is exact in one pass (row max first, then exp).
 //
-// Roles (320 threads, one CTA per SM):
-//   warp 0      producer: token indices (prefetched one tile ahead), TMA row
+// Roles (416 threads, one CTA per SM):
+//   warps 0..3  producers: token indices (prefetched one tile ahead), TMA row
 //               gathers (four rows per instruction) of Q tiles (two-slot
 //               ring) and K/V blocks (four-slot ring) into 128B-swizzled
-//               tiles; completion counted in bytes on full_q / full_kv
-//   warp 1      MMA issuer (one thread) and TMEM owner:
+//               tiles; completion counted in bytes on full_q / full_kv.  A
+//               warp issues its gathers one after another at a few tens of
+//               nanoseconds each, so each 128-row tile is split over four
+//               warps (one per SM sub-partition, 32 rows each)
+//   warp 12     MMA issuer (one thread) and TMEM owner:
 //                 O(j-1) = P V        as soon as P of tile j-1 is written,
 //                                     P read from TMEM as the A operand
 //                 S(j)   = Q K^T      -> TMEM [0, 256)
 //               and releases Q and K/V slots through tcgen05.commit
-//   warps 2..9  softmax and epilogue: warp w reaches TMEM lanes (query rows)
+//   warps 4..11 softmax and epilogue: warp w reaches TMEM lanes (query rows)
 //               32 (w % 4) .. +31 and takes one of two column ranges; row max
 //               and row sum are combined through shared memory;
 //               p = exp2(scale log2e s - m) masked to the row's own window,
@@ -44,7 +47,10 @@ using namespace tc;
 
 constexpr int D = 64;
 constexpr int kTile = 128;
-constexpr int kThreads = 320;
+constexpr int kThreads = 416;
+constexpr int kProducers = 4;            // warps 0..3
+constexpr int kSoftmaxWarp0 = 4;         // warps 4..11
+constexpr int kMmaWarp = 12;
 constexpr int kSoftmaxThreads = 256;
 constexpr int kKvSlots = 4;
 constexpr int kQSlots = 2;
@@ -166,11 +172,11 @@ attn_fwd_pipe_kernel(const __grid_constant__ FwdMaps maps, const int32_t* __rest
 
   if (tid == 0) {
     for (int s = 0; s < kQSlots; ++s) {
-      mbar_init(&bars->full_q[s], 1);   // the producer's byte-count arrival
+      mbar_init(&bars->full_q[s], kProducers);   // each producer warp's byte-count arrival
       mbar_init(&bars->empty_q[s], 1);
     }
     for (int s = 0; s < kKvSlots; ++s) {
-      mbar_init(&bars->full_kv[s], 1);
+      mbar_init(&bars->full_kv[s], kProducers);
       mbar_init(&bars->empty_kv[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -181,7 +187,7 @@ attn_fwd_pipe_kernel(const __grid_constant__ FwdMaps maps, const int32_t* __rest
     mbar_init(&bars->p_full, kSoftmaxThreads);
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&bars->tmem, kTmemCols);
     tmem_relinquish();
   }
@@ -191,14 +197,17 @@ attn_fwd_pipe_kernel(const __grid_constant__ FwdMaps maps, const int32_t* __rest
   const uint32_t tmem = bars->tmem;
   bool ok = true;
 
-  if (warp == 0) {
-    // ---------------------------------------------------------------- producer
-    // Lane l handles rows 4 l .. 4 l + 3 of the next Q tile and K/V block: its
-    // four token indices arrive in one 16-byte load (prefetched one tile
-    // ahead) and each matrix's four rows in one TMA gather; lane 0 first
-    // arms the slot's barrier with the tile's byte count.
+  if (warp < kProducers) {
+    // ---------------------------------------------------------------- producers
+    // Producer warp pw loads rows 32 pw .. 32 pw + 31 of each Q tile and K/V
+    // block: lane l < 8 takes rows 32 pw + 4 l .. + 3, whose four token
+    // indices arrive in one 16-byte load (prefetched one tile ahead) and each
+    // matrix's four rows in one TMA gather; lane 0 first arms the slot's
+    // barrier with this warp's share of the bytes.
+    const bool gl = lane < 8;
+    const int rbase = 32 * warp + 4 * lane;   // first row of this lane
     auto load_idx = [&](const int32_t* perm, size_t base) {
-      return *reinterpret_cast<const int4*>(perm + base + 4 * lane);
+      return gl ? *reinterpret_cast<const int4*>(perm + base + rbase) : make_int4(0, 0, 0, 0);
     };
     auto issue_kv = [&](int64_t n, size_t unit, int4 t4) -> bool {
       const int s = (int)(n % kKvSlots);
@@ -206,13 +215,15 @@ attn_fwd_pipe_kernel(const __grid_constant__ FwdMaps maps, const int32_t* __rest
           !__all_sync(0xffffffffu,
                       mbar_wait(&bars->empty_kv[s], (uint32_t)(((n / kKvSlots) - 1) & 1), err)))
         return false;
-      if (lane == 0) mbar_arrive_expect_tx(&bars->full_kv[s], 2u * kTile * 128u);
+      if (lane == 0) mbar_arrive_expect_tx(&bars->full_kv[s], 2u * kTile * 128u / kProducers);
       __syncwarp();
-      const uint32_t kst = sbase + Lay::kKv + s * Lay::kKvSlot + lane * 512;
+      const uint32_t kst = sbase + Lay::kKv + s * Lay::kKvSlot + (uint32_t)rbase * 128;
       const int u = (int)unit;
-      tma_gather4(kst, &maps.k, u + t4.x, u + t4.y, u + t4.z, u + t4.w, &bars->full_kv[s]);
-      tma_gather4(kst + Lay::kTileBytes, &maps.v, u + t4.x, u + t4.y, u + t4.z, u + t4.w,
-                  &bars->full_kv[s]);
+      if (gl) {
+        tma_gather4(kst, &maps.k, u + t4.x, u + t4.y, u + t4.z, u + t4.w, &bars->full_kv[s]);
+        tma_gather4(kst + Lay::kTileBytes, &maps.v, u + t4.x, u + t4.y, u + t4.z, u + t4.w,
+                    &bars->full_kv[s]);
+      }
       return true;
     };
     auto issue_q = [&](int64_t j, size_t unit, int4 t4) -> bool {
@@ -221,11 +232,11 @@ attn_fwd_pipe_kernel(const __grid_constant__ FwdMaps maps, const int32_t* __rest
           !__all_sync(0xffffffffu,
                       mbar_wait(&bars->empty_q[s], (uint32_t)(((j / kQSlots) - 1) & 1), err)))
         return false;
-      if (lane == 0) mbar_arrive_expect_tx(&bars->full_q[s], kTile * 128u);
+      if (lane == 0) mbar_arrive_expect_tx(&bars->full_q[s], kTile * 128u / kProducers);
       __syncwarp();
-      const uint32_t qst = sbase + Lay::kQ + s * Lay::kTileBytes + lane * 512;
+      const uint32_t qst = sbase + Lay::kQ + s * Lay::kTileBytes + (uint32_t)rbase * 128;
       const int u = (int)unit;
-      tma_gather4(qst, &maps.q, u + t4.x, u + t4.y, u + t4.z, u + t4.w, &bars->full_q[s]);
+      if (gl) tma_gather4(qst, &maps.q, u + t4.x, u + t4.y, u + t4.z, u + t4.w, &bars->full_q[s]);
       return true;
     };
     int4 qi = make_int4(0, 0, 0, 0), ki = make_int4(0, 0, 0, 0);
@@ -249,7 +260,7 @@ attn_fwd_pipe_kernel(const __grid_constant__ FwdMaps maps, const int32_t* __rest
       }
     }
 
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t id_pv = idesc_bf16(128, D, false, true);
@@ -326,7 +337,7 @@ attn_fwd_pipe_kernel(const __grid_constant__ FwdMaps maps, const int32_t* __rest
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
-    const int quarter = warp & 3, half = (warp - 2) >> 2;
+    const int quarter = warp & 3, half = (warp - kSoftmaxWarp0) >> 2;
     const int row = 32 * quarter + lane;               // TMEM lane = query row of the tile
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     float* red_m = reinterpret_cast<float*>(smem + Lay::kRed);   // [2][128]
@@ -423,7 +434,7 @@ attn_fwd_pipe_kernel(const __grid_constant__ FwdMaps maps, const int32_t* __rest
   }
   fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }

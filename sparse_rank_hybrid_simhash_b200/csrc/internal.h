@@ -188,6 +188,12 @@ bool attn_pipe_supported(const Geometry& g);
 cudaError_t launch_attn_fwd_pipe(const Geometry& g, const void* q, const void* k, const void* v,
                                  const int32_t* perm_q, const int32_t* perm_k, void* o_sp,
                                  float* lse, uint32_t* err, cudaStream_t s);
+// Persistent forward over any Sort-LSH window, streamed in 128-key blocks
+// (bf16, d = 64 or 128, one hash round, no causal mask).
+bool attn_win_supported(const Geometry& g);
+cudaError_t launch_attn_fwd_win(const Geometry& g, const void* q, const void* k, const void* v,
+                                const int32_t* perm_q, const int32_t* perm_k, void* o_sp,
+                                float* lse, uint32_t* err, cudaStream_t s);
 // tcgen05 backward: dq_acc += dQ (fp32 atomics); dk, dv written (dv adds dv_race).
 cudaError_t launch_attn_bwd_tc(const Geometry& g, const void* q, const void* k, const void* v,
                                const int32_t* perm_q, const int32_t* perm_k, const void* d_o,
@@ -220,9 +226,10 @@ cudaError_t launch_fuse_causal(const Geometry& g, const void* q, const void* o_s
                                const float* gate_w, const float* gate_b, const float* lam,
                                void* y, void* o_race, cudaStream_t s);
 
-// 2-D TMA map over a [rows, 64] bf16 matrix: one 128-byte row per box,
-// 128-byte swizzle; the row gathers of the tcgen05 attention kernels use it.
-cudaError_t make_row_map(CUtensorMap* map, const void* base, uint64_t rows);
+// 2-D TMA map over a [rows, width] bf16 matrix (width 64 or 128): a box is 64
+// columns of one row (128 bytes), 128-byte swizzle; the row gathers of the
+// tcgen05 attention kernels use it.
+cudaError_t make_row_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t width = 64);
 // 3-D TMA map over a [units, n, d] bf16 tensor (d contiguous), no swizzle, box
 // of 8 columns x box_rows rows x 1 unit: the RACE slab kernels' row tiles.
 cudaError_t make_slab_map(CUtensorMap* map, const void* base, uint64_t units, uint64_t n,

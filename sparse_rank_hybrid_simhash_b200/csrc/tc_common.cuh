@@ -245,6 +245,17 @@ ELSAA_DEV void tma_gather4(uint32_t dst, const void* map, int r0, int r1, int r2
       : "memory");
 }
 
+// The same gather from column x (elements, a multiple of 8) of a wider row
+// matrix: the 64 columns x .. x + 63 of each row.
+ELSAA_DEV void tma_gather4_x(uint32_t dst, const void* map, int x, int r0, int r1, int r2, int r3,
+                             uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(map), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // One box of a 3-D tensor map at coordinates (x, y, z) into shared memory at
 // `dst`; completion is counted on `bar` in bytes.  x (innermost, in elements)
 // must be a multiple of 16 bytes; out-of-range elements read as zero.

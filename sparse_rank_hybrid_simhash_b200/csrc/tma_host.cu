@@ -1,8 +1,8 @@
-// Host side of the TMA copies: 2-D tensor maps over [rows, 64] bf16 matrices
-// (one row per box, 128-byte swizzle) for the attention kernels' row gathers,
-// and 3-D maps over [units, N, d] bf16 with 8-column boxes for the RACE slab
-// kernels; encoded through the driver entry point the runtime resolves (no
-// direct driver-API calls).
+// Host side of the TMA copies: 2-D tensor maps over [rows, 64] or [rows, 128]
+// bf16 matrices (a box of one row of 64 columns, 128-byte swizzle) for the
+// attention kernels' row gathers, and 3-D maps over [units, N, d] bf16 with
+// 8-column boxes for the RACE slab kernels; encoded through the driver entry
+// point the runtime resolves (no direct driver-API calls).
 #include <cudaTypedefs.h>
 #include <mutex>
 
@@ -26,11 +26,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 }  // namespace
 
-cudaError_t make_row_map(CUtensorMap* map, const void* base, uint64_t rows) {
+cudaError_t make_row_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t width) {
   PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
   if (fn == nullptr) return cudaErrorNotSupported;
-  const cuuint64_t dims[2] = {64, rows};
-  const cuuint64_t strides[1] = {64 * 2};
+  const cuuint64_t dims[2] = {width, rows};
+  const cuuint64_t strides[1] = {width * 2};
   const cuuint32_t box[2] = {64, 1};
   const cuuint32_t elem[2] = {1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,

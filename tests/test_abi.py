@@ -176,18 +176,29 @@ def test_path_flags():
     # the kernel families each workload takes (what the bench line and the
     # parity tests rely on)
     f = {n: B.path_flags(B.Params.from_workload(w)) for n, w in WORKLOADS.items()}
-    assert all(f["text-32k"].values()) and all(f["vision-16k"].values())
-    assert all(f["iid-4k"].values())
-    # 10-bit RACE codes: the tables do not fit a shared-memory slab
+    main = ("tc_hash", "tc_attn", "slab_fwd", "slab_bwd")
+    for n in ("text-32k", "vision-16k", "iid-4k"):
+        assert all(f[n][k] for k in main) and not f[n]["tc_win"]
+    # 10-bit RACE codes: the tables do not fit a shared-memory slab; d = 128
+    # and 256-key chunks: the streamed-window forward
     assert f["needle-256k"]["tc_hash"] and f["needle-256k"]["tc_attn"]
     assert not f["needle-256k"]["slab_fwd"] and not f["needle-256k"]["slab_bwd"]
+    assert f["needle-256k"]["tc_win"]
+    for lb in (0, 2, 5):
+        g = B.path_flags(B.Params.from_workload(WORKLOADS["text-32k"].replace(lookback=lb)))
+        assert g["tc_win"] and not g["tc_attn"]
     assert not any(f["tiny-fp32"].values())
     w = WORKLOADS["text-32k"]
     assert not B.path_flags(B.Params.from_workload(w.replace(causal=True)))["slab_fwd"]
     assert not B.path_flags(B.Params.from_workload(w.replace(hash_rounds=2)))["slab_bwd"]
     assert B.path_flags(B.Params.from_workload(w.replace(hash_rounds=2)))["slab_fwd"]
     assert B.path_flags(B.Params.make(1, 1, 256, 64, "bf16", 4, 64, 8, 6)) == {
-        "tc_hash": True, "tc_attn": True, "slab_fwd": False, "slab_bwd": False}
+        "tc_hash": True, "tc_attn": True, "slab_fwd": False, "slab_bwd": False, "tc_win": False}
+    # causal, several hash rounds, fp32 and ragged lengths keep the CUDA-core forward
+    w = WORKLOADS["text-32k"]
+    for x in (w.replace(causal=True), w.replace(hash_rounds=2), w.replace(dtype="f32"),
+              w.replace(N=32768 + 64, chunk=64)):
+        assert not B.path_flags(B.Params.from_workload(x))["tc_win"]
 
 
 def test_binding_argument_counts_match_the_header():

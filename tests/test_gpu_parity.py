@@ -97,6 +97,18 @@ def test_lookback(cuda_device, lookback, dtype):
     _run(w, backward=True)
 
 
+@pytest.mark.parametrize("d,N,chunk,lookback", [(64, 2048, 256, 1), (128, 1024, 128, 1),
+                                                (128, 1024, 64, 3), (64, 1536, 384, 1),
+                                                (64, 1152, 96, 2), (128, 2048, 256, 0)])
+def test_streamed_window_forward(cuda_device, d, N, chunk, lookback):
+    # the tcgen05 forward that streams each tile's window in 128-key blocks:
+    # chunks above 128 (unmasked, several blocks), d = 128, lookback other
+    # than 1, and chunks that neither divide nor are multiples of 128 (masked)
+    w = WORKLOADS["iid-4k"].replace(B=1, H=2, N=N, d=d, chunk=chunk, lookback=lookback)
+    assert B.path_flags(B.Params.from_workload(w))["tc_win"]
+    _run(w, backward=True)
+
+
 @pytest.mark.parametrize("dtype,order,gates", [("bf16", "binary", False), ("f32", "local", False),
                                                ("bf16", "binary", True)])
 def test_causal(cuda_device, dtype, order, gates):
