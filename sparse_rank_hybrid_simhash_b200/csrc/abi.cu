@@ -315,8 +315,6 @@ elsaa_status forward_impl(const elsaa_params* p, const void* q, const void* k, c
     ELSAA_TRY(launch_attn_fwd_pipe(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s));
   else if (win_fwd(g))
     ELSAA_TRY(launch_attn_fwd_win(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s));
-  else if (g.tc_attn)
-    ELSAA_TRY(launch_attn_fwd_tc(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s));
   else
     ELSAA_TRY(launch_attn_fwd_simt(g, q, k, v, perm, perm + bhn, rank, o_sp, lse, s));
   ELSAA_TRY(mark(events, 4, s));

@@ -163,10 +163,9 @@ cudaError_t launch_attn_bwd_simt(const Geometry& g, const void* q, const void* k
                                  const int32_t* rank, const void* d_o, const float* lse,
                                  const float* dprime, float* dq_acc, float* dk_acc,
                                  float* dv_acc, cudaStream_t s);
-// Sparse branch, tcgen05 kernels.
-cudaError_t launch_attn_fwd_tc(const Geometry& g, const void* q, const void* k, const void* v,
-                               const int32_t* perm_q, const int32_t* perm_k, void* o_sp,
-                               float* lse, uint32_t* err, cudaStream_t s);
+// Sparse branch, tcgen05 kernels.  attn_tc_supported: the shapes whose
+// forward and backward both run on them (bf16, d = 64 or 128, N % 128 == 0,
+// any chunk c % 16 == 0 and any lookback, no causal mask).
 bool attn_tc_supported(const Geometry& g);
 // Overlapped backward (d = 64, chunk 64 or 128).
 // Persistent backward (d = 64, bf16, chunk dividing 128): writes dq (the gate
@@ -183,7 +182,8 @@ cudaError_t launch_attn_bwd2(const Geometry& g, const void* q, const void* k, co
                              const int32_t* perm_q, const int32_t* perm_k, const void* d_o,
                              const float* lse, const float* dprime, const float* dv_race,
                              float* dq_acc, void* dk, void* dv, uint32_t* err, cudaStream_t s);
-// Persistent warp-specialized forward (d = 64, chunk <= 128 dividing 128).
+// Persistent warp-specialized forward (d = 64, chunk <= 128 dividing 128,
+// lookback 1).
 bool attn_pipe_supported(const Geometry& g);
 cudaError_t launch_attn_fwd_pipe(const Geometry& g, const void* q, const void* k, const void* v,
                                  const int32_t* perm_q, const int32_t* perm_k, void* o_sp,
@@ -194,7 +194,8 @@ bool attn_win_supported(const Geometry& g);
 cudaError_t launch_attn_fwd_win(const Geometry& g, const void* q, const void* k, const void* v,
                                 const int32_t* perm_q, const int32_t* perm_k, void* o_sp,
                                 float* lse, uint32_t* err, cudaStream_t s);
-// tcgen05 backward: dq_acc += dQ (fp32 atomics); dk, dv written (dv adds dv_race).
+// tcgen05 backward for any window (key-major, one CTA per 128 sorted keys):
+// dq_acc += dQ (fp32 atomics); dk, dv written (dv adds dv_race).
 cudaError_t launch_attn_bwd_tc(const Geometry& g, const void* q, const void* k, const void* v,
                                const int32_t* perm_q, const int32_t* perm_k, const void* d_o,
                                const float* lse, const float* dprime, const float* dv_race,

@@ -184,9 +184,11 @@ def test_path_flags():
     assert f["needle-256k"]["tc_hash"] and f["needle-256k"]["tc_attn"]
     assert not f["needle-256k"]["slab_fwd"] and not f["needle-256k"]["slab_bwd"]
     assert f["needle-256k"]["tc_win"]
+    # other lookbacks: the streamed-window forward and the key-major tcgen05
+    # backward (not the persistent backward, which holds two query blocks)
     for lb in (0, 2, 5):
         g = B.path_flags(B.Params.from_workload(WORKLOADS["text-32k"].replace(lookback=lb)))
-        assert g["tc_win"] and not g["tc_attn"]
+        assert g["tc_win"] and g["tc_attn"] and not g["slab_bwd"]
     assert not any(f["tiny-fp32"].values())
     w = WORKLOADS["text-32k"]
     assert not B.path_flags(B.Params.from_workload(w.replace(causal=True)))["slab_fwd"]

@@ -65,16 +65,23 @@ def test_operator_roofline_of_the_text_workload():
     assert bench.window_keys(1024, 128, 3) == 128 * 128 * sum(min(j, 3) + 1 for j in range(8))
 
 
-def test_recorded_traffic_only_describes_the_captured_kernels():
+def test_recorded_traffic_only_describes_the_captured_kernels(monkeypatch):
     # DRAM bytes from a capture at 12 heads scale with the units of the run and
-    # are withheld where the run launches something else
+    # are withheld where the run launches something else or the kernel's
+    # source has changed since the capture
+    import hashlib
     bench = _bench()
+    src = "sparse_rank_hybrid_simhash_b200/csrc/attn_tc_bwd3.cu"
+    sha = hashlib.sha1(open(os.path.join(ROOT, src), "rb").read()).hexdigest()
+    monkeypatch.setitem(bench.RECORDED_TRAFFIC, "sparse_bwd", (src, sha, 3.0e8, "tc_attn"))
+    monkeypatch.setitem(bench.RECORDED_TRAFFIC, "race_fuse", (src, sha, 1.0e8, "slab_fwd"))
     w = WORKLOADS["text-32k"]
     path = {"tc_hash": True, "tc_attn": True, "slab_fwd": True, "slab_bwd": True}
-    full = bench.recorded_traffic(w, "sparse_bwd", path)
-    assert full is not None and full > 0
-    assert bench.recorded_traffic(w.replace(B=1), "sparse_bwd", path) == full / 2
+    assert bench.recorded_traffic(w, "sparse_bwd", path) == 3.0e8 * 24 / 12
+    assert bench.recorded_traffic(w.replace(B=1), "sparse_bwd", path) == 3.0e8
     assert bench.recorded_traffic(w, "race_fuse", dict(path, slab_fwd=False)) is None
     assert bench.recorded_traffic(w.replace(lookback=2), "sparse_bwd", path) is None
     assert bench.recorded_traffic(WORKLOADS["iid-4k"], "sparse_bwd", path) is None
-    assert bench.recorded_traffic(bench.apply_mode(w, "race_only"), "hash", path) is None
+    assert bench.recorded_traffic(bench.apply_mode(w, "race_only"), "sparse_bwd", path) is None
+    monkeypatch.setitem(bench.RECORDED_TRAFFIC, "sparse_bwd", (src, "0" * 40, 3.0e8, "tc_attn"))
+    assert bench.recorded_traffic(w, "sparse_bwd", path) is None

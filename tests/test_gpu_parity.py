@@ -90,10 +90,15 @@ def test_hash_rounds(cuda_device, rounds, dtype, order, causal):
     _run(w, backward=True)
 
 
-@pytest.mark.parametrize("lookback,dtype", [(0, "bf16"), (2, "bf16"), (3, "f32")])
-def test_lookback(cuda_device, lookback, dtype):
-    # windows of lookback previous chunks plus the own one (CUDA-core attention)
-    w = WORKLOADS["iid-4k"].replace(B=1, H=2, N=512, chunk=32, lookback=lookback, dtype=dtype)
+@pytest.mark.parametrize("lookback,dtype,chunk,N", [(0, "bf16", 32, 512), (2, "bf16", 32, 512),
+                                                    (3, "f32", 32, 512), (2, "bf16", 128, 2048),
+                                                    (4, "bf16", 64, 1024)])
+def test_lookback(cuda_device, lookback, dtype, chunk, N):
+    # windows of lookback previous chunks plus the own one: bf16 on the
+    # streamed-window forward and the key-major tcgen05 backward, fp32 on the
+    # CUDA-core attention
+    w = WORKLOADS["iid-4k"].replace(B=1, H=2, N=N, chunk=chunk, lookback=lookback, dtype=dtype)
+    assert B.path_flags(B.Params.from_workload(w))["tc_attn"] == (dtype == "bf16")
     _run(w, backward=True)
 
 
