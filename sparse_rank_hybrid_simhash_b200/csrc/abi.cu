@@ -287,7 +287,10 @@ elsaa_status forward_impl(const elsaa_params* p, const void* q, const void* k, c
     int32_t* ct = (int32_t*)(sv + sl.ctot);
     ELSAA_TRY(mark(events, 3, s));   // (no separate build stage)
     ELSAA_TRY(launch_race_causal_fwd(g, rcode, rcode_k, v, num, ct, sums, counts, s));
-    ELSAA_TRY(launch_attn_fwd_simt(g, q, k, v, perm, perm + bhn, rank, o_sp, lse, s));
+    if (win_fwd(g))
+      ELSAA_TRY(launch_attn_fwd_win(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s));
+    else
+      ELSAA_TRY(launch_attn_fwd_simt(g, q, k, v, perm, perm + bhn, rank, o_sp, lse, s));
     ELSAA_TRY(mark(events, 4, s));
     ELSAA_TRY(launch_fuse_causal(g, q, o_sp, lse, num, ct, gate_w, gate_b, lambda, y,
                                  sv + sl.o_race, s));

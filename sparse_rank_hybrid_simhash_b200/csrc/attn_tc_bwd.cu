@@ -10,7 +10,8 @@
 // Key-major CTAs: one CTA owns 128 consecutive sorted keys (the MMA's M) and
 // walks, in blocks of up to 128, the sorted queries whose window holds them
 // (query chunk j sees key chunks j - lb .. j, so key chunk i is seen by query
-// chunks i .. i + lb; lb = 1 in the pages), for any chunk c with c % 16 == 0:
+// chunks i .. i + lb; lb = 1 in the pages), for any chunk c with c % 16 == 0,
+// optionally with the causal mask (key token index at most the query's):
 //   S^T  = K Q_b^T,  dP^T = V dO_b^T          tcgen05 (SS) -> TMEM
 //   P^T, dS^T (bf16)                           thread t = key row t -> shared memory
 //   dV += P^T dO_b,  dK += dS^T Q_b            tcgen05, accumulated in TMEM
@@ -83,7 +84,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
                    const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ perm_q,
                    const int32_t* __restrict__ perm_k, const __nv_bfloat16* __restrict__ d_o,
                    const float* __restrict__ lse, const float* __restrict__ dprime,
-                   const float* __restrict__ dv_race, int N, int chunk, int lookback, float scale,
+                   const float* __restrict__ dv_race, int N, int chunk, int lookback, int causal,
+                   float scale,
                    float scale_log2, float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk,
                    __nv_bfloat16* __restrict__ dv, uint32_t* __restrict__ err) {
   using Lay = BwdLayout<D>;
@@ -112,6 +114,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
   const int qend = min(N, ((k0 + kTile - 1) / chunk + 1 + lookback) * chunk);
   const int nqb = (qend - qbase + kTile - 1) / kTile;
   const int key_chunk = (k0 + tid) / chunk;
+  const int my_tok = pk[k0 + tid];
 
   if (tid == 0) {
     mbar_init(bar_a, 1);
@@ -176,7 +179,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
     }
     fence_after();
     // P^T and dS^T rows of this thread's key; a query in chunk jq sees this key
-    // iff 0 <= jq - key_chunk <= lb
+    // iff 0 <= jq - key_chunk <= lb (and, causal, the key's token index is at
+    // most the query's)
     for (int c0 = 0; c0 < nq; c0 += 32) {
       float sv[32], dp[32];
       tmem_ld32(tmem + Lay::kTS + lane_off + c0, sv);
@@ -192,7 +196,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
           const int dj = (qb0 + col) / chunk - key_chunk;
           p[e] = 0.f;
           ds[e] = 0.f;
-          if (col < nq && dj >= 0 && dj <= lookback) {
+          if (col < nq && dj >= 0 && dj <= lookback && (!causal || my_tok <= qidx[col])) {
             p[e] = exp2f(sv[i + e] * scale_log2 - s_lse[col]);
             ds[e] = scale * p[e] * (dp[i + e] - s_dpr[col]);
           }
@@ -318,7 +322,7 @@ cudaError_t bwd(const Geometry& g, const void* q, const void* k, const void* v,
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
       static_cast<const __nv_bfloat16*>(v), perm_q, perm_k,
       static_cast<const __nv_bfloat16*>(d_o), lse, dprime, dv_race, g.N, g.chunk, g.lookback,
-      g.scale,
+      g.causal ? 1 : 0, g.scale,
       g.scale * 1.4426950408889634f, dq_acc, static_cast<__nv_bfloat16*>(dk),
       static_cast<__nv_bfloat16*>(dv), err);
   return cudaGetLastError();
@@ -329,7 +333,7 @@ cudaError_t bwd(const Geometry& g, const void* q, const void* k, const void* v,
 bool attn_tc_supported(const Geometry& g) {
   // the forward of this domain is the streamed-window kernel; TMA row
   // coordinates are 32-bit
-  return g.bf16 && (g.d == 64 || g.d == 128) && !g.causal && g.N % kTile == 0 &&
+  return g.bf16 && (g.d == 64 || g.d == 128) && g.N % kTile == 0 &&
          g.chunk % 16 == 0 && g.lookback >= 0 && (int64_t)g.BH * g.N < (int64_t)1 << 31;
 }
 

@@ -12,6 +12,9 @@
 // covers the 128-key blocks kb_lo .. kb_lo + nb - 1 of the sorted keys; the
 // rows' own windows are applied as a mask (none is needed when c is a multiple
 // of 128: every row of the tile then has the same, block-aligned window).
+// With the causal mask (an extension; the pages did not evaluate causal use)
+// a row also drops the keys whose token index exceeds its own; a row left
+// without keys gets O_sp = 0 and lse = -inf.
 // A window may exceed what TMEM holds next to O, so each tile takes two
 // passes over its blocks: pass 1 computes S = Q K^T block by block for the
 // exact row maximum; pass 2 computes S again, P = exp(scale s - m) (bf16, in
@@ -138,8 +141,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restrict__ perm_q,
                     const int32_t* __restrict__ perm_k, int BH, int N, int chunk, int lookback,
-                    float scale_log2, __nv_bfloat16* __restrict__ o_sp, float* __restrict__ lse,
-                    uint32_t* __restrict__ err) {
+                    int causal, float scale_log2, __nv_bfloat16* __restrict__ o_sp,
+                    float* __restrict__ lse, uint32_t* __restrict__ err) {
   using Lay = WinLayout<D>;
   constexpr int KS = Lay::kKSlots, VS = Lay::kVSlots, OB = Lay::kOBufs;
   constexpr uint32_t kTileBytes = Lay::kTileBytes;
@@ -341,7 +344,7 @@ attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restr
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     float* red_m = reinterpret_cast<float*>(smem + Lay::kRed);   // [2][128]
     float* red_l = red_m + 2 * 128;                              // [2][128]
-    const bool masked = chunk % kTile != 0;
+    const bool masked = causal || chunk % kTile != 0;
     int64_t ns = 0, np = 0;
     for (int64_t j = 0; j < count; ++j) {
       const WinTile w = tile(j);
@@ -353,6 +356,28 @@ attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restr
       const int lo = max(0, (jr - lookback) * chunk) - w.kb_lo * kTile;
       const int hi = (jr + 1) * chunk - w.kb_lo * kTile;
       const int cb = half * 64;   // this thread's 64 columns of every block
+      // bit e: column cb + e of block b is a key of the row (its window and,
+      // with the causal mask, a token index at most the query's)
+      auto allow_bits = [&](int b) -> uint64_t {
+        const int c0 = b * kTile + cb;
+        const int a = max(0, lo - c0), z = min(64, hi - c0);
+        if (a >= z) return 0ull;
+        uint64_t bits = (z == 64 ? ~0ull : (1ull << z) - 1ull) & ~((1ull << a) - 1ull);
+        if (causal) {
+          const int4* kt = reinterpret_cast<const int4*>(
+              perm_k + unit + (size_t)(w.kb_lo + b) * kTile + cb);
+          uint64_t c = 0;
+#pragma unroll 2
+          for (int e4 = 0; e4 < 16; ++e4) {
+            const int4 t = __ldg(kt + e4);
+            c |= ((uint64_t)(t.x <= token) | (uint64_t)(t.y <= token) << 1 |
+                  (uint64_t)(t.z <= token) << 2 | (uint64_t)(t.w <= token) << 3)
+                 << (4 * e4);
+          }
+          bits &= c;
+        }
+        return bits;
+      };
       // pass 1: row maximum
       float m = -INFINITY;
       for (int b = 0; b < w.nb; ++b) {
@@ -367,11 +392,11 @@ attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restr
         fence_before();
         mbar_arrive(&bars->s_free[sb]);
         ++ns;
-        const int c0 = b * kTile + cb;
         if (masked) {
+          const uint64_t al = allow_bits(b);
 #pragma unroll
           for (int e = 0; e < 64; ++e)
-            if (c0 + e >= lo && c0 + e < hi) m = fmaxf(m, sv[e]);
+            if ((al >> e) & 1ull) m = fmaxf(m, sv[e]);
         } else {
 #pragma unroll
           for (int e = 0; e < 64; ++e) m = fmaxf(m, sv[e]);
@@ -389,7 +414,7 @@ attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restr
                          (np < 2 || mbar_wait(&bars->p_free[pb], reuse_parity(np, 2), err)));
         if (!ok) break;
         fence_after();
-        const int c0 = b * kTile + cb;
+        const uint64_t al = masked ? allow_bits(b) : ~0ull;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           float sv[32];
@@ -403,9 +428,8 @@ attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restr
             fma2(a0, a1, scale_log2, scale_log2, -m, -m);
             float p0 = ex2(a0), p1 = ex2(a1);
             if (masked) {
-              const int c = c0 + 32 * h + e;
-              p0 = (c >= lo && c < hi) ? p0 : 0.f;
-              p1 = (c + 1 >= lo && c + 1 < hi) ? p1 : 0.f;
+              p0 = ((al >> (32 * h + e)) & 1ull) ? p0 : 0.f;
+              p1 = ((al >> (32 * h + e + 1)) & 1ull) ? p1 : 0.f;
             }
             add2(l0, l1, p0, p1);
             const __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
@@ -431,7 +455,7 @@ attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restr
       ok = softmax_all(mbar_wait(&bars->o_full[o], use_parity(j, OB), err));
       if (!ok) break;
       fence_after();
-      const float inv = 1.0f / l;
+      const float inv = l > 0.f ? 1.0f / l : 0.f;   // l = 0: a causal row without keys
       __nv_bfloat16* orow = o_sp + (unit + token) * D;
 #pragma unroll
       for (int h = 0; h < D / 64; ++h) {
@@ -451,7 +475,8 @@ attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restr
           *reinterpret_cast<uint4*>(orow + c0 + q8 * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
       }
-      if (half == 0) lse[unit + token] = (m + log2f(l)) * 0.69314718055994531f;
+      if (half == 0)
+        lse[unit + token] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
       fence_before();
       mbar_arrive(&bars->o_free[o]);
     }
@@ -484,7 +509,8 @@ cudaError_t launch(const Geometry& g, const void* q, const void* k, const void* 
   if ((e = make_row_map(&maps.k, k, rows, D)) != cudaSuccess) return e;
   if ((e = make_row_map(&maps.v, v, rows, D)) != cudaSuccess) return e;
   attn_fwd_win_kernel<D><<<grid_x, kThreads, Lay::kDyn, s>>>(
-      maps, perm_q, perm_k, g.BH, g.N, g.chunk, g.lookback, g.scale * 1.4426950408889634f,
+      maps, perm_q, perm_k, g.BH, g.N, g.chunk, g.lookback, g.causal ? 1 : 0,
+      g.scale * 1.4426950408889634f,
       static_cast<__nv_bfloat16*>(o_sp), lse, err);
   return cudaGetLastError();
 }
@@ -492,10 +518,10 @@ cudaError_t launch(const Geometry& g, const void* q, const void* k, const void* 
 }  // namespace
 
 bool attn_win_supported(const Geometry& g) {
-  // TMA row coordinates are 32-bit; the windows are sorted-rank ranges, so a
-  // single hash round and no causal mask
+  // TMA row coordinates are 32-bit; the windows are sorted-rank ranges of a
+  // single hash round
   return g.bf16 && (g.d == 64 || g.d == 128) && g.N % kTile == 0 && g.chunk % 16 == 0 &&
-         g.N % g.chunk == 0 && g.lookback >= 0 && g.rounds == 1 && !g.causal &&
+         g.N % g.chunk == 0 && g.lookback >= 0 && g.rounds == 1 &&
          (int64_t)g.BH * g.N < (int64_t)1 << 31;
 }
 

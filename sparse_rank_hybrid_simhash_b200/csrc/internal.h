@@ -165,7 +165,7 @@ cudaError_t launch_attn_bwd_simt(const Geometry& g, const void* q, const void* k
                                  float* dv_acc, cudaStream_t s);
 // Sparse branch, tcgen05 kernels.  attn_tc_supported: the shapes whose
 // forward and backward both run on them (bf16, d = 64 or 128, N % 128 == 0,
-// any chunk c % 16 == 0 and any lookback, no causal mask).
+// any chunk c % 16 == 0 and any lookback, with or without the causal mask).
 bool attn_tc_supported(const Geometry& g);
 // Overlapped backward (d = 64, chunk 64 or 128).
 // Persistent backward (d = 64, bf16, chunk dividing 128): writes dq (the gate
@@ -189,7 +189,7 @@ cudaError_t launch_attn_fwd_pipe(const Geometry& g, const void* q, const void* k
                                  const int32_t* perm_q, const int32_t* perm_k, void* o_sp,
                                  float* lse, uint32_t* err, cudaStream_t s);
 // Persistent forward over any Sort-LSH window, streamed in 128-key blocks
-// (bf16, d = 64 or 128, one hash round, no causal mask).
+// (bf16, d = 64 or 128, one hash round, optionally causal).
 bool attn_win_supported(const Geometry& g);
 cudaError_t launch_attn_fwd_win(const Geometry& g, const void* q, const void* k, const void* v,
                                 const int32_t* perm_q, const int32_t* perm_k, void* o_sp,

@@ -27,6 +27,7 @@ def pytest_terminal_summary(terminalreporter):
     stats = getattr(stats, "PARAM_GRAD_STATS", None) if stats else None
     if not stats:
         return
-    terminalreporter.write_line("parameter gradients: workload name rel_l2 cancellation scaled")
+    terminalreporter.write_line("parameter gradients: workload name rel_l2 cancellation "
+                                "rounding-sigma/|ref|")
     for row in stats:
         terminalreporter.write_line("  %s %s %.3e %.3e %.3e" % row)

@@ -74,6 +74,7 @@ def oracle_unit(w: Workload, inp, b: int, h: int, codes=None, backward=False):
                          codes=c, sort_order=w.sort_order, lookback=w.lookback,
                          causal=w.causal)
         out.update({"grad_" + k: v for k, v in g.items()})
+        out.update(q_in=inp["q"][b, h], dy_in=inp["dy"][b, h], lam_in=lam)
     return out
 
 
@@ -146,28 +147,74 @@ def check_unit(w: Workload, inp, gpu, b: int, h: int, backward: bool, report: di
 
 
 # Every parameter-gradient comparison made in this process:
-# (workload, name, plain rel-L2, cancellation ratio, error / sum-of-magnitudes)
+# (workload, name, plain rel-L2, cancellation ratio, rounding scale / ||ref||)
 PARAM_GRAD_STATS: List[tuple] = []
 
-# Below this cancellation ratio the plain rel-L2 bound is not asserted: the
-# device's error is a bf16-level fraction (about 1e-3 measured) of the summed
-# magnitudes, so the plain ratio error / ||sum|| exceeds 1e-2 once the sum is
-# under a tenth of the magnitudes it was summed from.
-CANCELLATION_FLOOR = 0.1
+# The gate and lambda gradients are sums over every row of dot products of dy
+# with O_sp and O_race, which the device holds in the data dtype.  Their error
+# model: every element of the stored O carries an independent relative
+# perturbation of one unit in the last place (2^-8 for bf16, 2^-23 for fp32);
+# propagated through the per-row terms, the gradients' error then has the
+# scale  sigma = ulp * sqrt(sum_rows e_row^2),  e_row the row's sensitivity
+# times |dy * O| (param_grads_closed_form).  Measured device errors sit at
+# 0.1 .. 1.2 sigma (bf16 causal and long-chunk cases, where the sums cancel
+# within and across units); the check allows SIGMA_FACTOR sigma on top of the
+# stated tolerance, and asserts the plain rel-L2 bound wherever that allowance
+# is under half of it.
+SIGMA_FACTOR = 4.0
+ULP = {"bf16": 2.0 ** -8, "f32": 2.0 ** -23}
+
+
+def param_grads_closed_form(refs: List[dict]):
+    """Gate and lambda gradients of the fusion from the oracle's forward
+    intermediates ("Two Efficient Attentions, One Denominator Problem",
+    section "Two efficient branches can still be mis-scaled": y = g_s m O_sp +
+    g_r O_race, m = Z_sp / (Z_sp + lambda Z_race), g = sigmoid(w . q + b)):
+      dL/da_s = (dy . m O_sp) g_s (1 - g_s),  dL/da_r = (dy . O_race) g_r (1 - g_r),
+      dL/dlambda = g_s (dy . O_sp) dm/dlambda,  dm/dlambda = -Z_sp Z_race / den^2,
+    summed over rows (times q for the weights).  Returns the gradients and,
+    per gradient element, sum_rows e_row^2 with e_row the row's sensitivity
+    to relative perturbations of the stored O: |coefficient| * ||dy * O||.
+    Fixed gates have no gate gradient (only lambda's applies)."""
+    d = refs[0]["o_sp"].shape[-1]
+    g = {"dgate_w": torch.zeros(2, d, dtype=torch.float64),
+         "dgate_b": torch.zeros(2, dtype=torch.float64),
+         "dlambda": torch.zeros(1, dtype=torch.float64)}
+    var = {k: torch.zeros_like(v) for k, v in g.items()}
+    for r in refs:
+        osp, ora = r["o_sp"], r["o_race"]
+        dy, q = r["dy_in"].double(), r["q_in"].double()
+        g_s, g_r, m = r["g_s"], r["g_r"], r["m"]
+        z_sp, z_r = torch.exp(r["lse"]), r["z_race"]
+        den = z_sp + r["lam_in"] * z_r
+        safe = torch.where(den > 0, den, torch.ones_like(den))
+        dm = torch.where(den > 0, -z_sp * z_r / safe ** 2, torch.zeros_like(den))
+        ys, yr = (dy * osp).sum(-1), (dy * ora).sum(-1)
+        es, er = (dy * osp).norm(dim=-1), (dy * ora).norm(dim=-1)
+        cs, cr = m * g_s * (1 - g_s), g_r * (1 - g_r)
+        g["dgate_w"][0] += ((ys * cs)[:, None] * q).sum(0)
+        g["dgate_w"][1] += ((yr * cr)[:, None] * q).sum(0)
+        var["dgate_w"][0] += (((es * cs)[:, None] * q) ** 2).sum(0)
+        var["dgate_w"][1] += (((er * cr)[:, None] * q) ** 2).sum(0)
+        g["dgate_b"] += torch.stack([(ys * cs).sum(), (yr * cr).sum()])
+        var["dgate_b"] += torch.stack([((es * cs) ** 2).sum(), ((er * cr) ** 2).sum()])
+        g["dlambda"] += (g_s * ys * dm).sum()
+        var["dlambda"] += ((g_s * es * dm) ** 2).sum()
+    return g, var
 
 
 def check_param_grads(w: Workload, gpu, refs: List[dict]):
     """Gate and lambda gradients are sums over every unit: compare when all
-    units were checked.  Two measures are taken:
-      plain  = ||got - ref||_2 / ||ref||_2        (the stated rel-L2 bound)
-      scaled = ||got - ref||_2 / || sum_u |ref_u| ||_2
-    where ref_u is unit u's contribution.  The scaled measure is always
-    asserted; the plain one wherever the cancellation ratio
-    ||ref|| / ||sum_u |ref_u||| is at least CANCELLATION_FLOOR (where the parts
-    cancel further, the bf16 error, which scales with the parts and not with
-    their sum, can exceed it).  Every comparison is recorded in
-    PARAM_GRAD_STATS."""
+    units were checked.  Measured:
+      plain = ||got - ref||_2 / ||ref||_2   (the stated rel-L2 bound)
+      sigma = ulp * ||sqrt(sum_rows e_row^2)||_2   (param_grads_closed_form;
+              its gradients equal the oracle's autograd ones, checked here)
+    Asserted: ||got - ref|| <= tol ||ref|| + SIGMA_FACTOR sigma, and plain <=
+    tol wherever SIGMA_FACTOR sigma <= tol ||ref|| / 2.  Every comparison is
+    recorded in PARAM_GRAD_STATS with the cancellation ratio
+    ||ref|| / ||sum_u |ref_u|||."""
     r0, _ = TOL[w.dtype]
+    closed, var = param_grads_closed_form(refs)
     out = {}
     for name, key in (("dgate_w", "grad_dgate_w"), ("dgate_b", "grad_dgate_b"),
                       ("dlambda", "grad_dlambda")):
@@ -180,14 +227,19 @@ def check_param_grads(w: Workload, gpu, refs: List[dict]):
         if scale == 0.0:   # fixed gates: both sides exactly zero
             assert err == 0.0, f"{name}: expected exact zeros, ||err|| = {err:.3e}"
             continue
+        assert (closed[name].reshape(-1) - ref).norm().item() <= 1e-9 * scale, \
+            f"{name}: closed form != autograd"
+        sigma = ULP[w.dtype] * var[name].reshape(-1).sqrt().norm().item()
         plain = err / ref_norm if ref_norm > 0 else float("inf")
         ratio = ref_norm / scale
-        tag = f"{w.name}[B{w.B} H{w.H} N{w.N} c{w.chunk} {w.sort_order} lam{w.lam}]"
-        PARAM_GRAD_STATS.append((tag, name, plain, ratio, err / scale))
-        out[name] = {"rel_l2": plain, "cancellation": ratio, "scaled": err / scale}
-        assert err <= r0 * scale + 1e-12, \
-            f"{name}: ||err|| = {err:.3e}, tol * ||sum_u |parts||| = {r0 * scale:.3e}"
-        if ratio >= CANCELLATION_FLOOR:
-            assert plain <= r0, f"{name}: rel_l2 {plain:.3e} (<= {r0}); cancellation " \
-                                f"ratio {ratio:.3e}"
+        tag = f"{w.name}[B{w.B} H{w.H} N{w.N} c{w.chunk} {w.sort_order} lam{w.lam}" \
+              f"{' causal' if w.causal else ''}]"
+        rel_sigma = sigma / max(ref_norm, 1e-300)
+        PARAM_GRAD_STATS.append((tag, name, plain, ratio, rel_sigma))
+        out[name] = {"rel_l2": plain, "cancellation": ratio, "sigma": rel_sigma}
+        bound = r0 * ref_norm + SIGMA_FACTOR * sigma + 1e-12
+        assert err <= bound, f"{name}: ||err|| = {err:.3e} > tol ||ref|| + " \
+                             f"{SIGMA_FACTOR} sigma = {bound:.3e} (sigma {sigma:.3e})"
+        if SIGMA_FACTOR * sigma <= 0.5 * r0 * ref_norm:
+            assert plain <= r0, f"{name}: rel_l2 {plain:.3e} (<= {r0}); sigma {sigma:.3e}"
     return out

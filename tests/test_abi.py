@@ -163,8 +163,11 @@ def test_kernel_launch_counts():
     assert B.kernel_launches(B.Params.from_workload(w)) == (8, 5)   # tcgen05 path, one sort pass
     assert B.kernel_launches(B.Params.from_workload(w.replace(sort_order="local"))) == (6, 5)
     assert B.kernel_launches(B.Params.from_workload(w.replace(sort_bits=12))) == (11, 5)
-    # causal: token scan instead of |V| max + build; CUDA-core sparse backward + 3 casts
+    # causal: token scan instead of |V| max + build; the key-major tcgen05
+    # sparse backward + the dq cast (fp32: CUDA-core sparse backward + 3 casts)
     c = B.kernel_launches(B.Params.from_workload(w.replace(causal=True)))
+    assert c == (1 + 3 + 1 + 1 + 1, 1 + 1 + 2 + 1)
+    c = B.kernel_launches(B.Params.from_workload(w.replace(causal=True, dtype="f32")))
     assert c == (1 + 3 + 1 + 1 + 1, 1 + 1 + 4 + 1)
     # three hash rounds: one more hash kernel, three sorts, the inverse orders;
     # CUDA-core sparse backward + 3 casts
@@ -196,11 +199,13 @@ def test_path_flags():
     assert B.path_flags(B.Params.from_workload(w.replace(hash_rounds=2)))["slab_fwd"]
     assert B.path_flags(B.Params.make(1, 1, 256, 64, "bf16", 4, 64, 8, 6)) == {
         "tc_hash": True, "tc_attn": True, "slab_fwd": False, "slab_bwd": False, "tc_win": False}
-    # causal, several hash rounds, fp32 and ragged lengths keep the CUDA-core forward
+    # several hash rounds, fp32 and ragged lengths keep the CUDA-core forward;
+    # causal takes the streamed-window forward and the key-major backward
     w = WORKLOADS["text-32k"]
-    for x in (w.replace(causal=True), w.replace(hash_rounds=2), w.replace(dtype="f32"),
-              w.replace(N=32768 + 64, chunk=64)):
+    for x in (w.replace(hash_rounds=2), w.replace(dtype="f32"), w.replace(N=32768 + 64, chunk=64)):
         assert not B.path_flags(B.Params.from_workload(x))["tc_win"]
+    c = B.path_flags(B.Params.from_workload(w.replace(causal=True)))
+    assert c["tc_win"] and c["tc_attn"] and not c["slab_fwd"] and not c["slab_bwd"]
 
 
 def test_binding_argument_counts_match_the_header():

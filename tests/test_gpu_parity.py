@@ -114,13 +114,19 @@ def test_streamed_window_forward(cuda_device, d, N, chunk, lookback):
     _run(w, backward=True)
 
 
-@pytest.mark.parametrize("dtype,order,gates", [("bf16", "binary", False), ("f32", "local", False),
-                                               ("bf16", "binary", True)])
-def test_causal(cuda_device, dtype, order, gates):
-    # keys j <= i in both branches (CUDA-core attention, per-table RACE token
-    # scans); binary order leaves some early queries with empty windows
-    w = WORKLOADS["iid-4k"].replace(B=1, H=2, N=512, chunk=32, dtype=dtype, sort_order=order,
-                                    causal=True, gate_fixed=gates, gate_s=0.6, gate_r=0.8)
+@pytest.mark.parametrize("dtype,order,gates,d,N,chunk,lookback", [
+    ("bf16", "binary", False, 64, 512, 32, 1), ("f32", "local", False, 64, 512, 32, 1),
+    ("bf16", "binary", True, 64, 512, 32, 1), ("bf16", "gray", False, 64, 2048, 128, 1),
+    ("bf16", "binary", False, 128, 1024, 64, 2), ("bf16", "local", False, 64, 1024, 256, 0)])
+def test_causal(cuda_device, dtype, order, gates, d, N, chunk, lookback):
+    # keys j <= i in both branches (per-table RACE token scans; bf16 on the
+    # streamed-window forward and the key-major tcgen05 backward, fp32 on the
+    # CUDA-core attention); binary order leaves some early queries with empty
+    # windows
+    w = WORKLOADS["iid-4k"].replace(B=1, H=2, N=N, d=d, chunk=chunk, lookback=lookback,
+                                    dtype=dtype, sort_order=order, causal=True,
+                                    gate_fixed=gates, gate_s=0.6, gate_r=0.8)
+    assert B.path_flags(B.Params.from_workload(w))["tc_win"] == (dtype == "bf16")
     _run(w, backward=True)
 
 
