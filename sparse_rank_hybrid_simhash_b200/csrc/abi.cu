@@ -286,7 +286,8 @@ elsaa_status forward_impl(const elsaa_params* p, const void* q, const void* k, c
     float* num = (float*)(w + wl.causal_num);
     int32_t* ct = (int32_t*)(sv + sl.ctot);
     ELSAA_TRY(mark(events, 3, s));   // (no separate build stage)
-    ELSAA_TRY(launch_race_causal_fwd(g, rcode, rcode_k, v, num, ct, sums, counts, s));
+    ELSAA_TRY(launch_race_causal_fwd(g, rcode, rcode_k, rcode_t, rcode_tk, v, num, ct, sums,
+                                     counts, s));
     if (win_fwd(g))
       ELSAA_TRY(launch_attn_fwd_win(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s));
     else
@@ -395,7 +396,8 @@ elsaa_status backward_impl(const elsaa_params* p, const void* q, const void* k, 
   // token scan per table straight into dv_acc
   if (g.causal) {
     ELSAA_TRY(cudaMemsetAsync(dv_acc, 0, bhn * g.d * 4, s));
-    ELSAA_TRY(launch_race_causal_bwd(g, rcode, rcode_k, dor, dv_acc, s));
+    ELSAA_TRY(launch_race_causal_bwd(g, rcode, rcode_k, rcode_t,
+                                     rcode_t + bhn * g.L * g.rcode_bytes, dor, dv_acc, s));
   } else if (d_tables) {
     // the caller's table gradient (fp32); the value gradient of the RACE
     // branch is left to the caller (elsaa_race_value_grad once dT is summed)

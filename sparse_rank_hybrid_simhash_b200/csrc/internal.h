@@ -213,15 +213,19 @@ cudaError_t launch_param_reduce(const Geometry& g, const float* partials, float*
                                 float* dgate_b, float* dlambda, cudaStream_t s);
 cudaError_t launch_cast_out(const Geometry& g, const float* src, void* dst, cudaStream_t s);
 
-// Causal RACE (race_causal.cu): per-table token scans and the fusion on their
-// read-out.  num [BH][N][d] fp32 and ctot [BH][N] are zeroed and accumulated;
-// sums / counts receive the full tables.
+// Causal RACE (race_causal.cu): token walks over the tables and the fusion on
+// their read-out.  Codes row-major (rcode_*) and table-major (rcode_t*).
+// num [BH][N][d] fp32 and ctot [BH][N] receive the prefix read-out, sums /
+// counts the full tables; the backward writes the RACE value gradient into
+// dv_acc (which must be zero on entry).
 bool race_causal_supported(const Geometry& g);
 cudaError_t launch_race_causal_fwd(const Geometry& g, const void* rcode_q, const void* rcode_k,
-                                   const void* v, float* num, int32_t* ctot, float* sums,
-                                   int32_t* counts, cudaStream_t s);
+                                   const void* rcode_tq, const void* rcode_tk, const void* v,
+                                   float* num, int32_t* ctot, float* sums, int32_t* counts,
+                                   cudaStream_t s);
 cudaError_t launch_race_causal_bwd(const Geometry& g, const void* rcode_q, const void* rcode_k,
-                                   const void* dor, float* dv_acc, cudaStream_t s);
+                                   const void* rcode_tq, const void* rcode_tk, const void* dor,
+                                   float* dv_acc, cudaStream_t s);
 cudaError_t launch_fuse_causal(const Geometry& g, const void* q, const void* o_sp,
                                const float* lse, const float* num, const int32_t* ctot,
                                const float* gate_w, const float* gate_b, const float* lam,

@@ -115,8 +115,12 @@ def test_validation_rejects_bad_problems():
     p3 = B.Params.make(1, 2, 256, 64, "bf16", 4, 64, 8, 6, hash_rounds=3)
     # codes, orders and inverse orders of two more rounds
     assert B.saved_bytes(p3) >= B.saved_bytes(p1) + 2 * 2 * 512 * (2 + 4) + 3 * 2 * 512 * 4
-    # the causal RACE scan keeps one table in shared memory
-    assert B.validate(B.Params.make(1, 2, 256, 128, "bf16", 4, 64, 8, 9, causal=True)) == 2
+    # the causal RACE walk keeps a column slab of every table in shared memory
+    # (L dividing 32); other table counts take the per-table scan, which keeps
+    # one whole table there
+    assert B.validate(B.Params.make(1, 2, 256, 128, "bf16", 4, 64, 8, 9, causal=True)) == 0
+    assert B.validate(B.Params.make(1, 2, 256, 128, "bf16", 4, 64, 12, 9, causal=True)) == 2
+    assert B.validate(B.Params.make(1, 2, 256, 128, "bf16", 4, 64, 12, 8, causal=True)) == 0
 
 
 def test_null_pointers_are_rejected_before_any_launch():

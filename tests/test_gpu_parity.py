@@ -130,6 +130,18 @@ def test_causal(cuda_device, dtype, order, gates, d, N, chunk, lookback):
     _run(w, backward=True)
 
 
+@pytest.mark.parametrize("tables,race_bits,N", [(12, 6, 512), (16, 6, 512 + 16), (8, 9, 512),
+                                               (4, 6, 256)])
+def test_causal_race_walks(cuda_device, tables, race_bits, N):
+    # the causal RACE read-out and value gradient: the warp walk over 32-token
+    # groups (4, 8 and 16 tables; 16-bit codes at 9 bits), and the per-table
+    # token scans where the walk does not apply (12 tables; a length that is
+    # not a multiple of 32)
+    w = WORKLOADS["iid-4k"].replace(B=1, H=2, N=N, chunk=16 if N % 32 else 32,
+                                    race_tables=tables, race_bits=race_bits, causal=True)
+    _run(w, backward=True)
+
+
 def test_two_pass_sort_and_wide_race_codes(cuda_device):
     # 12 sort bits take two radix passes; 11 RACE bits give uint16 codes and
     # 2048-bucket tables (the global-atomic build)
