@@ -59,7 +59,7 @@ bool make_geometry(const elsaa_params* p, Geometry* g, elsaa_status* why) {
   g->sort_bins = 1 << g->sort_digit_bits;
   g->sort_tiles = (p->N + kSortTile - 1) / kSortTile;
   g->tc_hash = hash_tc_supported(*g);
-  g->tc_attn = attn_tc_supported(*g) && g->rounds == 1;
+  g->tc_attn = attn_tc_supported(*g);
   if (g->causal && !race_causal_supported(*g)) return false;
   *why = ELSAA_OK;
   return true;
@@ -101,6 +101,10 @@ WorkLayout work_layout(const Geometry& g) {
   const size_t shared_base = off;
   // forward without a saved buffer: the saved layout lives here
   w.saved = take(saved_layout(g).total);
+  // several hash rounds on the tcgen05 forward: each round's partial softmax
+  const bool parts = g.rounds > 1 && g.tc_attn;
+  w.round_o = take(parts ? (size_t)g.rounds * bhn * g.d * 4 : 0);
+  w.round_lse = take(parts ? (size_t)g.rounds * bhn * 4 : 0);
   const size_t fwd_end = off;
   // backward temporaries reuse the same bytes (a backward always has a saved buffer)
   off = shared_base;
@@ -147,6 +151,16 @@ bool direct_bwd(const Geometry& g) {
   return g.tc_attn && attn_bwd3_supported(g) && race_gather_add_supported(g);
 }
 bool slab_bwd(const Geometry& g) { return direct_bwd(g) && race_slab_supported(g, false); }
+// The streamed-window sparse forward: one pass, or one per hash round and the
+// combine of their partial softmaxes.
+cudaError_t sparse_win(const Geometry& g, const void* q, const void* k, const void* v,
+                       const int32_t* perm, const int32_t* rank, char* w, const WorkLayout& wl,
+                       void* o_sp, float* lse, uint32_t* err, cudaStream_t s) {
+  const size_t bhn = (size_t)g.BH * g.N;
+  if (g.rounds == 1) return launch_attn_fwd_win(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s);
+  return launch_attn_fwd_win_rounds(g, q, k, v, perm, rank, (float*)(w + wl.round_o),
+                                    (float*)(w + wl.round_lse), o_sp, lse, err, s);
+}
 // the shared-memory value-gradient gather on its own (any attention path)
 bool slab_bwd_add(const Geometry& g) { return race_slab_supported(g, false); }
 
@@ -289,7 +303,7 @@ elsaa_status forward_impl(const elsaa_params* p, const void* q, const void* k, c
     ELSAA_TRY(launch_race_causal_fwd(g, rcode, rcode_k, rcode_t, rcode_tk, v, num, ct, sums,
                                      counts, s));
     if (win_fwd(g))
-      ELSAA_TRY(launch_attn_fwd_win(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s));
+      ELSAA_TRY(sparse_win(g, q, k, v, perm, rank, w, wl, o_sp, lse, err, s));
     else
       ELSAA_TRY(launch_attn_fwd_simt(g, q, k, v, perm, perm + bhn, rank, o_sp, lse, s));
     ELSAA_TRY(mark(events, 4, s));
@@ -318,7 +332,7 @@ elsaa_status forward_impl(const elsaa_params* p, const void* q, const void* k, c
   if (g.tc_attn && attn_pipe_supported(g))
     ELSAA_TRY(launch_attn_fwd_pipe(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s));
   else if (win_fwd(g))
-    ELSAA_TRY(launch_attn_fwd_win(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s));
+    ELSAA_TRY(sparse_win(g, q, k, v, perm, rank, w, wl, o_sp, lse, err, s));
   else
     ELSAA_TRY(launch_attn_fwd_simt(g, q, k, v, perm, perm + bhn, rank, o_sp, lse, s));
   ELSAA_TRY(mark(events, 4, s));
@@ -430,6 +444,16 @@ elsaa_status backward_impl(const elsaa_params* p, const void* q, const void* k, 
                                dk, dv, (uint32_t*)(w + wl.err), s));
     ELSAA_TRY(mark(events, 3, s));
     ELSAA_TRY(launch_cast_out(g, dq_acc, dq, s));
+  } else if (g.tc_attn && g.rounds > 1) {
+    // one key-major pass per hash round, dk and dv accumulated in fp32 (dv_acc
+    // holds the RACE part)
+    ELSAA_TRY(cudaMemsetAsync(dk_acc, 0, bhn * g.d * 4, s));
+    ELSAA_TRY(launch_attn_bwd_tc_rounds(g, q, k, v, perm, rank, d_o, lse, dprime, dq_acc, dk_acc,
+                                        dv_acc, (uint32_t*)(w + wl.err), s));
+    ELSAA_TRY(mark(events, 3, s));
+    ELSAA_TRY(launch_cast_out(g, dq_acc, dq, s));
+    ELSAA_TRY(launch_cast_out(g, dk_acc, dk, s));
+    ELSAA_TRY(launch_cast_out(g, dv_acc, dv, s));
   } else if (g.tc_attn) {
     ELSAA_TRY(launch_attn_bwd_tc(g, q, k, v, perm, perm + bhn, d_o, lse, dprime, dv_acc, dq_acc,
                                  dk, dv, (uint32_t*)(w + wl.err), s));
@@ -530,11 +554,14 @@ elsaa_status elsaa_kernel_launches(const elsaa_params* p, int32_t* fwd, int32_t*
   const int sort1 = g.sort_order == ELSAA_SORT_LOCAL ? 1 : 3 * g.sort_passes;
   const int sort = g.rounds * sort1 + (g.rounds > 1 ? 1 + (g.sort_bits > 0 ? 1 : 0) : 0);
   const int build = race_build_kernels(g, false, g.bf16);
-  *fwd = g.causal ? 1 + sort + 1 + 1 + 1 : 1 + sort + 1 + build + 1 + 1;
+  // (several rounds on tcgen05: one window pass per round + the combine)
+  const int sparse_fwd = g.rounds > 1 && win_fwd(g) ? g.rounds + 1 : 1;
+  *fwd = g.causal ? 1 + sort + 1 + sparse_fwd + 1 : 1 + sort + 1 + build + sparse_fwd + 1;
   // fusion backward 1, RACE build 1 + gather 1, sparse 1 (+ casts), reduction 1
   // (direct path: the sparse kernel writes dq itself and the gather adds into dv)
   const bool direct = direct_bwd(g);
-  const int sparse = direct ? 1 : g.tc_attn ? 1 + 1 : 1 + 3;
+  // (several rounds on tcgen05: one key-major pass per round + 3 casts)
+  const int sparse = direct ? 1 : g.tc_attn ? (g.rounds > 1 ? g.rounds + 3 : 1 + 1) : 1 + 3;
   // (the RACE backward: the table-gradient build, then, off the direct path, a gather)
   const int race_bwd = g.causal ? 1 : race_build_kernels(g, false, g.bf16) + (direct ? 0 : 1);
   *bwd = 1 + race_bwd + sparse + (direct ? 1 : 0) + 1;

@@ -19,7 +19,11 @@
 //                                              MN-major operand; added to the
 //                                              fp32 dq accumulator with atomics
 // dK and dV (plus the RACE branch's dv) are written once, in bf16, at the
-// keys' token indices.  Every wait is bounded.
+// keys' token indices.  With several hash rounds (an extension: the union of
+// the rounds' windows, each key once) the kernel runs once per round t on that
+// round's orders with the final lse, masks the (key, query) pairs whose key an
+// earlier round's window of the query already holds, and adds dK and dV into
+// fp32 accumulators instead.  Every wait is bounded.
 #include <math.h>
 
 #include "internal.h"
@@ -47,7 +51,8 @@ struct BwdLayout {
   static constexpr uint32_t kLse = kDST + 2 * kSubBytes;     // 128 floats
   static constexpr uint32_t kDpr = kLse + 128 * 4;           // 128 floats
   static constexpr uint32_t kIdx = kDpr + 128 * 4;           // token indices: keys, queries
-  static constexpr uint32_t kBar = kIdx + 2 * 128 * 4;
+  static constexpr uint32_t kWin = kIdx + 2 * 128 * 4;       // earlier rounds' query windows
+  static constexpr uint32_t kBar = kWin + 2 * (kMaxRounds - 1) * 128 * 4;
   static constexpr uint32_t kDQ = kPT;   // dQ staging (fp32, 128 x D) reuses P^T and dS^T
   static constexpr uint32_t kDyn = kBar + 64;
   // TMEM columns
@@ -78,14 +83,17 @@ ELSAA_DEV uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <int D>
+// MR: the largest hash-round count the instance handles (1, or kMaxRounds
+// for the several-round passes).
+template <int D, int MR>
 __global__ void __launch_bounds__(kThreads)
 attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                    const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ perm_q,
                    const int32_t* __restrict__ perm_k, const __nv_bfloat16* __restrict__ d_o,
                    const float* __restrict__ lse, const float* __restrict__ dprime,
                    const float* __restrict__ dv_race, int N, int chunk, int lookback, int causal,
-                   float scale,
+                   const int32_t* __restrict__ rank, int round, float* __restrict__ dk_acc,
+                   float* __restrict__ dv_acc, float scale,
                    float scale_log2, float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk,
                    __nv_bfloat16* __restrict__ dv, uint32_t* __restrict__ err) {
   using Lay = BwdLayout<D>;
@@ -115,6 +123,15 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
   const int nqb = (qend - qbase + kTile - 1) / kTile;
   const int key_chunk = (k0 + tid) / chunk;
   const int my_tok = pk[k0 + tid];
+  // several rounds: this key's ranks in the earlier rounds, and per query
+  // column the query's earlier windows [s_wlo, s_whi)
+  const int64_t rows = (int64_t)gridDim.y * N, rstride = 2 * rows;   // rank: [R][2][BH][N]
+  int my_rank[MR];
+#pragma unroll
+  for (int u = 0; u < MR; ++u)
+    my_rank[u] = u < round ? rank[u * rstride + rows + unit + my_tok] : 0;
+  int32_t* s_wlo = reinterpret_cast<int32_t*>(smem + Lay::kWin);   // [kMaxRounds - 1][128]
+  int32_t* s_whi = s_wlo + (kMaxRounds - 1) * 128;
 
   if (tid == 0) {
     mbar_init(bar_a, 1);
@@ -140,7 +157,14 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
   for (int b = 0; b < nqb; ++b) {
     const int qb0 = qbase + b * kTile;
     const int nq = min(kTile, qend - qb0);
-    if (tid < nq) qidx[tid] = pq[qb0 + tid];
+    if (tid < nq) {
+      qidx[tid] = pq[qb0 + tid];
+      for (int u = 0; u < round; ++u) {
+        const int ju = rank[u * rstride + unit + qidx[tid]] / chunk;
+        s_wlo[u * 128 + tid] = max(0, (ju - lookback) * chunk);
+        s_whi[u * 128 + tid] = min(N, (ju + 1) * chunk);
+      }
+    }
     __syncthreads();
     gather_rows<D>(sbase + Lay::kQ, q + unit * D, qidx, nq);
     gather_rows<D>(sbase + Lay::kDO, d_o + unit * D, qidx, nq);
@@ -196,7 +220,13 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
           const int dj = (qb0 + col) / chunk - key_chunk;
           p[e] = 0.f;
           ds[e] = 0.f;
-          if (col < nq && dj >= 0 && dj <= lookback && (!causal || my_tok <= qidx[col])) {
+          bool seen = false;
+#pragma unroll
+          for (int u = 0; u < MR; ++u)
+            if (u < round && col < nq)
+              seen |= my_rank[u] >= s_wlo[u * 128 + col] && my_rank[u] < s_whi[u * 128 + col];
+          if (col < nq && dj >= 0 && dj <= lookback && (!causal || my_tok <= qidx[col]) &&
+              !seen) {
             p[e] = exp2f(sv[i + e] * scale_log2 - s_lse[col]);
             ds[e] = scale * p[e] * (dp[i + e] - s_dpr[col]);
           }
@@ -286,6 +316,20 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
       tmem_ld32(tmem + Lay::kTdV + lane_off + c0, gv);
       tmem_ld32(tmem + Lay::kTdK + lane_off + c0, gk);
       tmem_ld_wait();
+      if (dk_acc != nullptr) {   // several rounds: one writer per key row and round
+        float* ka = dk_acc + (unit + i) * D + c0;
+        float* va = dv_acc + (unit + i) * D + c0;
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          float4 a = *reinterpret_cast<float4*>(ka + 4 * c4);
+          float4 b = *reinterpret_cast<float4*>(va + 4 * c4);
+          a.x += gk[4 * c4]; a.y += gk[4 * c4 + 1]; a.z += gk[4 * c4 + 2]; a.w += gk[4 * c4 + 3];
+          b.x += gv[4 * c4]; b.y += gv[4 * c4 + 1]; b.z += gv[4 * c4 + 2]; b.w += gv[4 * c4 + 3];
+          *reinterpret_cast<float4*>(ka + 4 * c4) = a;
+          *reinterpret_cast<float4*>(va + 4 * c4) = b;
+        }
+        continue;
+      }
 #pragma unroll
       for (int q8 = 0; q8 < 4; ++q8) {
         uint32_t wv[4], wk[4];
@@ -308,21 +352,22 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
   }
 }
 
-template <int D>
+template <int D, int MR>
 cudaError_t bwd(const Geometry& g, const void* q, const void* k, const void* v,
                 const int32_t* perm_q, const int32_t* perm_k, const void* d_o, const float* lse,
                 const float* dprime, const float* dv_race, float* dq_acc, void* dk, void* dv,
-                uint32_t* err, cudaStream_t s) {
+                const int32_t* rank, int round, float* dk_acc, float* dv_acc, uint32_t* err,
+                cudaStream_t s) {
   using Lay = BwdLayout<D>;
-  cudaError_t e = cudaFuncSetAttribute(attn_bwd_tc_kernel<D>,
+  cudaError_t e = cudaFuncSetAttribute(attn_bwd_tc_kernel<D, MR>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kDyn);
   if (e != cudaSuccess) return e;
   const dim3 grid(g.N / kTile, g.BH);
-  attn_bwd_tc_kernel<D><<<grid, kThreads, Lay::kDyn, s>>>(
+  attn_bwd_tc_kernel<D, MR><<<grid, kThreads, Lay::kDyn, s>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
       static_cast<const __nv_bfloat16*>(v), perm_q, perm_k,
       static_cast<const __nv_bfloat16*>(d_o), lse, dprime, dv_race, g.N, g.chunk, g.lookback,
-      g.causal ? 1 : 0, g.scale,
+      g.causal ? 1 : 0, rank, round, dk_acc, dv_acc, g.scale,
       g.scale * 1.4426950408889634f, dq_acc, static_cast<__nv_bfloat16*>(dk),
       static_cast<__nv_bfloat16*>(dv), err);
   return cudaGetLastError();
@@ -341,10 +386,30 @@ cudaError_t launch_attn_bwd_tc(const Geometry& g, const void* q, const void* k, 
                                const int32_t* perm_q, const int32_t* perm_k, const void* d_o,
                                const float* lse, const float* dprime, const float* dv_race,
                                float* dq_acc, void* dk, void* dv, uint32_t* err, cudaStream_t s) {
-  return g.d == 64 ? bwd<64>(g, q, k, v, perm_q, perm_k, d_o, lse, dprime, dv_race, dq_acc, dk,
-                             dv, err, s)
-                   : bwd<128>(g, q, k, v, perm_q, perm_k, d_o, lse, dprime, dv_race, dq_acc, dk,
-                              dv, err, s);
+  return g.d == 64 ? bwd<64, 1>(g, q, k, v, perm_q, perm_k, d_o, lse, dprime, dv_race, dq_acc,
+                                dk, dv, nullptr, 0, nullptr, nullptr, err, s)
+                   : bwd<128, 1>(g, q, k, v, perm_q, perm_k, d_o, lse, dprime, dv_race, dq_acc,
+                                 dk, dv, nullptr, 0, nullptr, nullptr, err, s);
+}
+
+cudaError_t launch_attn_bwd_tc_rounds(const Geometry& g, const void* q, const void* k,
+                                      const void* v, const int32_t* perm, const int32_t* rank,
+                                      const void* d_o, const float* lse, const float* dprime,
+                                      float* dq_acc, float* dk_acc, float* dv_acc, uint32_t* err,
+                                      cudaStream_t s) {
+  const int64_t rows = (int64_t)g.BH * g.N;
+  for (int t = 0; t < g.rounds; ++t) {
+    const int32_t* pq = perm + (size_t)t * 2 * rows;
+    const cudaError_t e =
+        g.d == 64 ? bwd<64, kMaxRounds - 1>(g, q, k, v, pq, pq + rows, d_o, lse, dprime, nullptr,
+                                            dq_acc, nullptr, nullptr, rank, t, dk_acc, dv_acc,
+                                            err, s)
+                  : bwd<128, kMaxRounds - 1>(g, q, k, v, pq, pq + rows, d_o, lse, dprime,
+                                             nullptr, dq_acc, nullptr, nullptr, rank, t, dk_acc,
+                                             dv_acc, err, s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace elsaa

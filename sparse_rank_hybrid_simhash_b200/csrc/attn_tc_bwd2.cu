@@ -312,7 +312,7 @@ attn_bwd2_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 }  // namespace
 
 bool attn_bwd2_supported(const Geometry& g) {
-  return g.bf16 && g.lookback == 1 && !g.causal && g.d == D && g.N % kTile == 0 &&
+  return g.bf16 && g.lookback == 1 && !g.causal && g.rounds == 1 && g.d == D && g.N % kTile == 0 &&
          (g.chunk == 64 || g.chunk == 128);
 }
 

@@ -708,7 +708,7 @@ attn_bwd3_kernel(const __grid_constant__ RowMaps maps, const int32_t* __restrict
 
 bool attn_bwd3_supported(const Geometry& g) {
   // TMA row coordinates are 32-bit
-  return g.bf16 && g.lookback == 1 && !g.causal && g.d == D && g.N % kTile == 0 &&
+  return g.bf16 && g.lookback == 1 && !g.causal && g.rounds == 1 && g.d == D && g.N % kTile == 0 &&
          g.chunk >= 16 && g.chunk <= kTile &&
          kTile % g.chunk == 0 && (int64_t)g.BH * g.N < (int64_t)1 << 31;
 }

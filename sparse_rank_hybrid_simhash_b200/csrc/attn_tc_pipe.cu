@@ -444,7 +444,7 @@ attn_fwd_pipe_kernel(const __grid_constant__ FwdMaps maps, const int32_t* __rest
 
 bool attn_pipe_supported(const Geometry& g) {
   // TMA row coordinates are 32-bit
-  return g.bf16 && g.lookback == 1 && !g.causal && g.d == 64 && g.N % kTile == 0 &&
+  return g.bf16 && g.lookback == 1 && !g.causal && g.rounds == 1 && g.d == 64 && g.N % kTile == 0 &&
          g.chunk % 16 == 0 && g.chunk <= kTile &&
          kTile % g.chunk == 0 && (int64_t)g.BH * g.N < (int64_t)1 << 31;
 }

@@ -14,7 +14,12 @@
 // of 128: every row of the tile then has the same, block-aligned window).
 // With the causal mask (an extension; the pages did not evaluate causal use)
 // a row also drops the keys whose token index exceeds its own; a row left
-// without keys gets O_sp = 0 and lse = -inf.
+// without keys gets O_sp = 0 and lse = -inf.  With several hash rounds (an
+// extension: a query attends the union of its rounds' windows, each key once)
+// the kernel runs once per round t on that round's orders, drops the keys
+// that lie in the query's window of an earlier round (by the keys' and the
+// query's ranks in that round), and writes the round's partial softmax (O_t
+// normalized by its own mass, in fp32, and lse_t) for round_combine_kernel.
 // A window may exceed what TMEM holds next to O, so each tile takes two
 // passes over its blocks: pass 1 computes S = Q K^T block by block for the
 // exact row maximum; pass 2 computes S again, P = exp(scale s - m) (bf16, in
@@ -137,12 +142,17 @@ ELSAA_DEV bool softmax_all(bool v) {
 ELSAA_DEV uint32_t reuse_parity(int64_t n, int slots) { return (uint32_t)(((n / slots) - 1) & 1); }
 ELSAA_DEV uint32_t use_parity(int64_t n, int slots) { return (uint32_t)((n / slots) & 1); }
 
-template <int D>
+// MR: the largest hash-round count the instance handles (1, or kMaxRounds
+// for the several-round passes; the one-round instance keeps no per-round
+// state in registers).
+template <int D, int MR>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restrict__ perm_q,
                     const int32_t* __restrict__ perm_k, int BH, int N, int chunk, int lookback,
                     int causal, float scale_log2, __nv_bfloat16* __restrict__ o_sp,
-                    float* __restrict__ lse, uint32_t* __restrict__ err) {
+                    float* __restrict__ lse, const int32_t* __restrict__ rank, int round,
+                    int64_t rank_len, float* __restrict__ o_part, float* __restrict__ lse_part,
+                    uint32_t* __restrict__ err) {
   using Lay = WinLayout<D>;
   constexpr int KS = Lay::kKSlots, VS = Lay::kVSlots, OB = Lay::kOBufs;
   constexpr uint32_t kTileBytes = Lay::kTileBytes;
@@ -344,7 +354,8 @@ attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restr
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     float* red_m = reinterpret_cast<float*>(smem + Lay::kRed);   // [2][128]
     float* red_l = red_m + 2 * 128;                              // [2][128]
-    const bool masked = causal || chunk % kTile != 0;
+    const bool masked = causal || round > 0 || chunk % kTile != 0;
+    const int64_t rows = (int64_t)BH * N, rstride = 2 * rows;   // rank: [R][2][BH][N]
     int64_t ns = 0, np = 0;
     for (int64_t j = 0; j < count; ++j) {
       const WinTile w = tile(j);
@@ -356,22 +367,57 @@ attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restr
       const int lo = max(0, (jr - lookback) * chunk) - w.kb_lo * kTile;
       const int hi = (jr + 1) * chunk - w.kb_lo * kTile;
       const int cb = half * 64;   // this thread's 64 columns of every block
-      // bit e: column cb + e of block b is a key of the row (its window and,
-      // with the causal mask, a token index at most the query's)
+      // the query's windows in the earlier rounds (several hash rounds)
+      int wlo[MR], whi[MR];
+#pragma unroll
+      for (int u = 0; u < MR; ++u) {
+        wlo[u] = whi[u] = 0;
+        if (u < round) {
+          const int64_t at = u * rstride + (int64_t)unit + token;
+          if (at < 0 || at >= rank_len || token < 0 || token >= N) {   // checked: never taken
+            raise_error(err, ERR_CHECK);
+            continue;
+          }
+          const int ju = rank[at] / chunk;
+          wlo[u] = max(0, (ju - lookback) * chunk);
+          whi[u] = min(N, (ju + 1) * chunk);
+        }
+      }
+      // a key of this round's window that an earlier round's window of the
+      // query already holds
+      auto seen = [&](int key) {
+        bool in = false;
+#pragma unroll
+        for (int u = 0; u < MR; ++u)
+          if (u < round) {
+            const int64_t at = u * rstride + rows + (int64_t)unit + key;
+            if (at < 0 || at >= rank_len || key < 0 || key >= N) {   // checked: never taken
+              raise_error(err, ERR_CHECK);
+              continue;
+            }
+            const int rk = __ldg(rank + at);
+            in |= rk >= wlo[u] && rk < whi[u];
+          }
+        return in;
+      };
+      // bit e: column cb + e of block b is a key of the row (its window; with
+      // the causal mask, a token index at most the query's; with several
+      // rounds, not seen in an earlier round)
       auto allow_bits = [&](int b) -> uint64_t {
         const int c0 = b * kTile + cb;
         const int a = max(0, lo - c0), z = min(64, hi - c0);
         if (a >= z) return 0ull;
         uint64_t bits = (z == 64 ? ~0ull : (1ull << z) - 1ull) & ~((1ull << a) - 1ull);
-        if (causal) {
+        if (causal || round > 0) {
           const int4* kt = reinterpret_cast<const int4*>(
               perm_k + unit + (size_t)(w.kb_lo + b) * kTile + cb);
+          auto keep = [&](int key) { return (!causal || key <= token) && !(round > 0 && seen(key)); };
           uint64_t c = 0;
 #pragma unroll 2
           for (int e4 = 0; e4 < 16; ++e4) {
             const int4 t = __ldg(kt + e4);
-            c |= ((uint64_t)(t.x <= token) | (uint64_t)(t.y <= token) << 1 |
-                  (uint64_t)(t.z <= token) << 2 | (uint64_t)(t.w <= token) << 3)
+            c |= ((uint64_t)keep(t.x) | (uint64_t)keep(t.y) << 1 | (uint64_t)keep(t.z) << 2 |
+                  (uint64_t)keep(t.w) << 3)
                  << (4 * e4);
           }
           bits &= c;
@@ -455,7 +501,7 @@ attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restr
       ok = softmax_all(mbar_wait(&bars->o_full[o], use_parity(j, OB), err));
       if (!ok) break;
       fence_after();
-      const float inv = l > 0.f ? 1.0f / l : 0.f;   // l = 0: a causal row without keys
+      const float inv = l > 0.f ? 1.0f / l : 0.f;   // l = 0: a row without keys
       __nv_bfloat16* orow = o_sp + (unit + token) * D;
 #pragma unroll
       for (int h = 0; h < D / 64; ++h) {
@@ -463,6 +509,15 @@ attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restr
         float ov[32];
         tmem_ld32(tmem + kTO + (uint32_t)(o * D + c0) + lane_off, ov);
         tmem_ld_wait();
+        if (o_part != nullptr) {   // a round's partial, fp32
+          float* prow = o_part + (unit + token) * D + c0;
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            *reinterpret_cast<float4*>(prow + 4 * q4) =
+                make_float4(ov[4 * q4] * inv, ov[4 * q4 + 1] * inv, ov[4 * q4 + 2] * inv,
+                            ov[4 * q4 + 3] * inv);
+          continue;
+        }
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
           uint32_t w4[4];
@@ -476,7 +531,8 @@ attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restr
         }
       }
       if (half == 0)
-        lse[unit + token] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        (o_part != nullptr ? lse_part : lse)[unit + token] =
+            l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
       fence_before();
       mbar_arrive(&bars->o_free[o]);
     }
@@ -489,12 +545,13 @@ attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restr
   }
 }
 
-template <int D>
+template <int D, int MR>
 cudaError_t launch(const Geometry& g, const void* q, const void* k, const void* v,
                    const int32_t* perm_q, const int32_t* perm_k, void* o_sp, float* lse,
-                   uint32_t* err, cudaStream_t s) {
+                   const int32_t* rank, int round, float* o_part, float* lse_part, uint32_t* err,
+                   cudaStream_t s) {
   using Lay = WinLayout<D>;
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_win_kernel<D>,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_win_kernel<D, MR>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Lay::kDyn);
   if (e != cudaSuccess) return e;
@@ -508,28 +565,84 @@ cudaError_t launch(const Geometry& g, const void* q, const void* k, const void* 
   if ((e = make_row_map(&maps.q, q, rows, D)) != cudaSuccess) return e;
   if ((e = make_row_map(&maps.k, k, rows, D)) != cudaSuccess) return e;
   if ((e = make_row_map(&maps.v, v, rows, D)) != cudaSuccess) return e;
-  attn_fwd_win_kernel<D><<<grid_x, kThreads, Lay::kDyn, s>>>(
+  attn_fwd_win_kernel<D, MR><<<grid_x, kThreads, Lay::kDyn, s>>>(
       maps, perm_q, perm_k, g.BH, g.N, g.chunk, g.lookback, g.causal ? 1 : 0,
-      g.scale * 1.4426950408889634f,
-      static_cast<__nv_bfloat16*>(o_sp), lse, err);
+      g.scale * 1.4426950408889634f, static_cast<__nv_bfloat16*>(o_sp), lse, rank, round,
+      (int64_t)g.rounds * 2 * g.BH * g.N, o_part, lse_part, err);
   return cudaGetLastError();
+}
+
+// O_sp and lse of the union of the rounds' windows from the rounds' partials:
+// lse = log sum_t exp(lse_t), O = sum_t exp(lse_t - lse) O_t (rows without keys
+// in every round: O = 0, lse = -inf).  One warp per row, lanes over d.
+__global__ void __launch_bounds__(256)
+round_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
+                     int R, int64_t rows, int d, __nv_bfloat16* __restrict__ o_sp,
+                     float* __restrict__ lse) {
+  const int lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int64_t r = (int64_t)blockIdx.x * nw + (threadIdx.x >> 5); r < rows;
+       r += (int64_t)gridDim.x * nw) {
+    float m = -INFINITY;
+    for (int t = 0; t < R; ++t) m = fmaxf(m, lse_part[t * rows + r]);
+    if (m == -INFINITY) {
+      for (int e = lane; e < d; e += 32) o_sp[r * d + e] = __float2bfloat16_rn(0.f);
+      if (lane == 0) lse[r] = -INFINITY;
+      continue;
+    }
+    float z = 0.f;
+    for (int t = 0; t < R; ++t) z += expf(lse_part[t * rows + r] - m);
+    const float lz = m + logf(z);
+    for (int e = lane; e < d; e += 32) {
+      float acc = 0.f;
+      for (int t = 0; t < R; ++t) {
+        const float wt = expf(lse_part[t * rows + r] - lz);
+        acc += wt * o_part[(t * rows + r) * d + e];
+      }
+      o_sp[r * d + e] = __float2bfloat16_rn(acc);
+    }
+    if (lane == 0) lse[r] = lz;
+  }
 }
 
 }  // namespace
 
 bool attn_win_supported(const Geometry& g) {
-  // TMA row coordinates are 32-bit; the windows are sorted-rank ranges of a
-  // single hash round
+  // TMA row coordinates are 32-bit
   return g.bf16 && (g.d == 64 || g.d == 128) && g.N % kTile == 0 && g.chunk % 16 == 0 &&
-         g.N % g.chunk == 0 && g.lookback >= 0 && g.rounds == 1 &&
+         g.N % g.chunk == 0 && g.lookback >= 0 && g.rounds >= 1 && g.rounds <= kMaxRounds &&
          (int64_t)g.BH * g.N < (int64_t)1 << 31;
 }
 
 cudaError_t launch_attn_fwd_win(const Geometry& g, const void* q, const void* k, const void* v,
                                 const int32_t* perm_q, const int32_t* perm_k, void* o_sp,
                                 float* lse, uint32_t* err, cudaStream_t s) {
-  return g.d == 64 ? launch<64>(g, q, k, v, perm_q, perm_k, o_sp, lse, err, s)
-                   : launch<128>(g, q, k, v, perm_q, perm_k, o_sp, lse, err, s);
+  return g.d == 64 ? launch<64, 1>(g, q, k, v, perm_q, perm_k, o_sp, lse, nullptr, 0, nullptr,
+                                   nullptr, err, s)
+                   : launch<128, 1>(g, q, k, v, perm_q, perm_k, o_sp, lse, nullptr, 0, nullptr,
+                                    nullptr, err, s);
+}
+
+cudaError_t launch_attn_fwd_win_rounds(const Geometry& g, const void* q, const void* k,
+                                       const void* v, const int32_t* perm, const int32_t* rank,
+                                       float* o_part, float* lse_part, void* o_sp, float* lse,
+                                       uint32_t* err, cudaStream_t s) {
+  const int64_t rows = (int64_t)g.BH * g.N;
+  for (int t = 0; t < g.rounds; ++t) {
+    const int32_t* pq = perm + (size_t)t * 2 * rows;
+    float* op = o_part + (size_t)t * rows * g.d;
+    float* lp = lse_part + (size_t)t * rows;
+    const cudaError_t e =
+        g.d == 64
+            ? launch<64, kMaxRounds>(g, q, k, v, pq, pq + rows, o_sp, lse, rank, t, op, lp, err, s)
+            : launch<128, kMaxRounds>(g, q, k, v, pq, pq + rows, o_sp, lse, rank, t, op, lp, err,
+                                      s);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t want = (rows + 7) / 8;
+  const int grid = (int)(want < 148 * 16 ? want : 148 * 16);
+  round_combine_kernel<<<grid, 256, 0, s>>>(o_part, lse_part, g.rounds, rows, g.d,
+                                            static_cast<__nv_bfloat16*>(o_sp), lse);
+  return cudaGetLastError();
 }
 
 }  // namespace elsaa

@@ -59,6 +59,8 @@ struct WorkLayout {
   size_t count_scratch;      // [BH][L][NB] i32: bucket counts of a build that has no counts output
   size_t causal_num;         // [BH][N][d] f32: causal RACE numerators (0 bytes unless causal)
   size_t saved;              // a SavedLayout used when the forward has no saved buffer
+  size_t round_o, round_lse; // [R][BH][N][d] / [R][BH][N] f32: per-round partial softmax
+                             // (several hash rounds on the tcgen05 forward; else 0 bytes)
   size_t d_o;                // [BH][N][d] dtype: dO_sp
   size_t dprime;             // [BH][N] f32: D' = dO_sp . O_sp - dlse
   size_t dq_acc, dk_acc, dv_acc;   // [BH][N][d] f32
@@ -194,12 +196,27 @@ bool attn_win_supported(const Geometry& g);
 cudaError_t launch_attn_fwd_win(const Geometry& g, const void* q, const void* k, const void* v,
                                 const int32_t* perm_q, const int32_t* perm_k, void* o_sp,
                                 float* lse, uint32_t* err, cudaStream_t s);
+// Several hash rounds: one streamed-window pass per round (perm and rank
+// [R][2][BH][N]), each writing its partial softmax to o_part / lse_part, then
+// their combine into o_sp and lse.
+cudaError_t launch_attn_fwd_win_rounds(const Geometry& g, const void* q, const void* k,
+                                       const void* v, const int32_t* perm, const int32_t* rank,
+                                       float* o_part, float* lse_part, void* o_sp, float* lse,
+                                       uint32_t* err, cudaStream_t s);
 // tcgen05 backward for any window (key-major, one CTA per 128 sorted keys):
 // dq_acc += dQ (fp32 atomics); dk, dv written (dv adds dv_race).
 cudaError_t launch_attn_bwd_tc(const Geometry& g, const void* q, const void* k, const void* v,
                                const int32_t* perm_q, const int32_t* perm_k, const void* d_o,
                                const float* lse, const float* dprime, const float* dv_race,
                                float* dq_acc, void* dk, void* dv, uint32_t* err, cudaStream_t s);
+// Several hash rounds: one key-major pass per round with the final lse,
+// masking keys an earlier round's window of the query holds; dq_acc += dQ,
+// dk_acc += dK, dv_acc += dV (fp32).
+cudaError_t launch_attn_bwd_tc_rounds(const Geometry& g, const void* q, const void* k,
+                                      const void* v, const int32_t* perm, const int32_t* rank,
+                                      const void* d_o, const float* lse, const float* dprime,
+                                      float* dq_acc, float* dk_acc, float* dv_acc, uint32_t* err,
+                                      cudaStream_t s);
 
 // Backward of the fusion and gates (per query), then the parameter reduction
 // and the final casts.

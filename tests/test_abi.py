@@ -173,10 +173,13 @@ def test_kernel_launch_counts():
     assert c == (1 + 3 + 1 + 1 + 1, 1 + 1 + 2 + 1)
     c = B.kernel_launches(B.Params.from_workload(w.replace(causal=True, dtype="f32")))
     assert c == (1 + 3 + 1 + 1 + 1, 1 + 1 + 4 + 1)
-    # three hash rounds: one more hash kernel, three sorts, the inverse orders;
-    # CUDA-core sparse backward + 3 casts
+    # three hash rounds: one more hash kernel, three sorts, the inverse orders,
+    # one streamed-window pass per round and their combine; backward: one
+    # key-major pass per round + 3 casts (fp32: CUDA-core attention both ways)
     r = B.kernel_launches(B.Params.from_workload(w.replace(hash_rounds=3)))
-    assert r == (1 + 1 + 3 * 3 + 1 + 2 + 1 + 1, 1 + 2 + 1 + 3 + 1)
+    assert r == (1 + 1 + 3 * 3 + 1 + 2 + (3 + 1) + 1, 1 + 2 + (3 + 3) + 1)
+    r = B.kernel_launches(B.Params.from_workload(w.replace(hash_rounds=3, dtype="f32")))
+    assert r[1] == 1 + 2 + 1 + 3 + 1
 
 
 def test_path_flags():
@@ -203,11 +206,13 @@ def test_path_flags():
     assert B.path_flags(B.Params.from_workload(w.replace(hash_rounds=2)))["slab_fwd"]
     assert B.path_flags(B.Params.make(1, 1, 256, 64, "bf16", 4, 64, 8, 6)) == {
         "tc_hash": True, "tc_attn": True, "slab_fwd": False, "slab_bwd": False, "tc_win": False}
-    # several hash rounds, fp32 and ragged lengths keep the CUDA-core forward;
-    # causal takes the streamed-window forward and the key-major backward
+    # fp32 and ragged lengths keep the CUDA-core attention; causal and several
+    # hash rounds take the streamed-window forward and the key-major backward
     w = WORKLOADS["text-32k"]
-    for x in (w.replace(hash_rounds=2), w.replace(dtype="f32"), w.replace(N=32768 + 64, chunk=64)):
+    for x in (w.replace(dtype="f32"), w.replace(N=32768 + 64, chunk=64)):
         assert not B.path_flags(B.Params.from_workload(x))["tc_win"]
+    r = B.path_flags(B.Params.from_workload(w.replace(hash_rounds=2)))
+    assert r["tc_win"] and r["tc_attn"] and not r["slab_bwd"]
     c = B.path_flags(B.Params.from_workload(w.replace(causal=True)))
     assert c["tc_win"] and c["tc_attn"] and not c["slab_fwd"] and not c["slab_bwd"]
 

@@ -90,6 +90,20 @@ def test_hash_rounds(cuda_device, rounds, dtype, order, causal):
     _run(w, backward=True)
 
 
+@pytest.mark.parametrize("rounds,d,N,chunk,lookback,causal", [
+    (2, 64, 2048, 128, 1, False), (4, 64, 1024, 64, 2, False), (2, 128, 1024, 256, 0, False),
+    (3, 64, 1024, 32, 1, True), (8, 64, 512, 64, 1, False)])
+def test_hash_rounds_tensor_cores(cuda_device, rounds, d, N, chunk, lookback, causal):
+    # several rounds in bf16: one streamed-window pass per round, keys of an
+    # earlier round's window masked, partial softmaxes combined; backward one
+    # key-major pass per round with the final lse
+    w = WORKLOADS["iid-4k"].replace(B=1, H=2, N=N, d=d, chunk=chunk, lookback=lookback,
+                                    causal=causal, hash_rounds=rounds)
+    f = B.path_flags(B.Params.from_workload(w))
+    assert f["tc_win"] and f["tc_attn"]
+    _run(w, backward=True)
+
+
 @pytest.mark.parametrize("lookback,dtype,chunk,N", [(0, "bf16", 32, 512), (2, "bf16", 32, 512),
                                                     (3, "f32", 32, 512), (2, "bf16", 128, 2048),
                                                     (4, "bf16", 64, 1024)])
