@@ -161,6 +161,10 @@ cudaError_t sparse_win(const Geometry& g, const void* q, const void* k, const vo
   return launch_attn_fwd_win_rounds(g, q, k, v, perm, rank, (float*)(w + wl.round_o),
                                     (float*)(w + wl.round_lse), o_sp, lse, err, s);
 }
+// Several hash rounds: the tcgen05 hash GEMM gives every round's sort codes.
+bool rounds_in_hash(const Geometry& g) {
+  return g.rounds > 1 && g.tc_hash && hash_tc_rounds_supported(g, slab_fwd(g) && !g.gate_fixed);
+}
 // the shared-memory value-gradient gather on its own (any attention path)
 bool slab_bwd_add(const Geometry& g) { return race_slab_supported(g, false); }
 
@@ -280,11 +284,13 @@ elsaa_status forward_impl(const elsaa_params* p, const void* q, const void* k, c
   float2* gl = (slab && !g.gate_fixed) ? (float2*)(w + wl.gl) : nullptr;
   // 1. SimHash codes of Q and K (and the gate logits)
   if (g.tc_hash)
-    ELSAA_TRY(launch_hash_tc(g, q, k, r_sort, r_race, code, rcode, rcode_t, gate_w, gl, err, s));
+    ELSAA_TRY(launch_hash_tc(g, q, k, r_sort, r_race, code, rcode, rcode_t, gate_w, gl,
+                             rounds_in_hash(g) ? g.rounds : 1, err, s));
   else
     ELSAA_TRY(launch_hash_simt(g, q, k, r_sort, r_race, code, rcode, rcode_t, s));
   // several hash rounds: the other rounds' sort codes
-  if (g.rounds > 1) ELSAA_TRY(launch_hash_sort_rounds(g, q, k, r_sort, code, s));
+  if (g.rounds > 1 && !rounds_in_hash(g))
+    ELSAA_TRY(launch_hash_sort_rounds(g, q, k, r_sort, code, s));
   ELSAA_TRY(mark(events, 1, s));
   // 2. Sort-LSH order of Q and K (every round), and with several rounds the
   // inverse orders the attention uses to count each key once
@@ -552,7 +558,8 @@ elsaa_status elsaa_kernel_launches(const elsaa_params* p, int32_t* fwd, int32_t*
   // (several hash rounds: one more hash kernel, one sort per round and the
   // inverse orders; zero-bit extra codes are a memset)
   const int sort1 = g.sort_order == ELSAA_SORT_LOCAL ? 1 : 3 * g.sort_passes;
-  const int sort = g.rounds * sort1 + (g.rounds > 1 ? 1 + (g.sort_bits > 0 ? 1 : 0) : 0);
+  const int sort = g.rounds * sort1 +
+                   (g.rounds > 1 ? 1 + (g.sort_bits > 0 && !rounds_in_hash(g) ? 1 : 0) : 0);
   const int build = race_build_kernels(g, false, g.bf16);
   // (several rounds on tcgen05: one window pass per round + the combine)
   const int sparse_fwd = g.rounds > 1 && win_fwd(g) ? g.rounds + 1 : 1;
@@ -593,7 +600,8 @@ elsaa_status elsaa_sort_codes_of(const elsaa_params* p, const void* q, const voi
   uint32_t* err = (uint32_t*)(w + wl.err);
   ELSAA_TRY(cudaMemsetAsync(err, 0, sizeof(uint32_t), s));
   if (g.tc_hash)
-    ELSAA_TRY(launch_hash_tc(g, q, k, r_sort, r_race, c, rcode, rcode_t, nullptr, nullptr, err, s));
+    ELSAA_TRY(
+        launch_hash_tc(g, q, k, r_sort, r_race, c, rcode, rcode_t, nullptr, nullptr, 1, err, s));
   else
     ELSAA_TRY(launch_hash_simt(g, q, k, r_sort, r_race, c, rcode, rcode_t, s));
   ELSAA_TRY(cudaMemcpyAsync(code, c, 2 * bhn * 2, cudaMemcpyDeviceToDevice, s));
@@ -644,8 +652,8 @@ elsaa_status elsaa_race_tables(const elsaa_params* p, const void* k, const void*
   Geometry gk = g;
   gk.sort_bits = 0;
   if (gk.tc_hash)
-    ELSAA_TRY(launch_hash_tc(gk, k, k, nullptr, r_race, c, rcode, rcode_t, nullptr, nullptr, err,
-                             s));
+    ELSAA_TRY(
+        launch_hash_tc(gk, k, k, nullptr, r_race, c, rcode, rcode_t, nullptr, nullptr, 1, err, s));
   else
     ELSAA_TRY(launch_hash_simt(gk, k, k, nullptr, r_race, c, rcode, rcode_t, s));
   float* absmax = (float*)(w + wl.absmax);
@@ -682,8 +690,8 @@ elsaa_status elsaa_race_value_grad(const elsaa_params* p, const void* k, const v
   Geometry gk = g;   // RACE codes of the keys only: no sort hyperplanes
   gk.sort_bits = 0;
   if (gk.tc_hash)
-    ELSAA_TRY(launch_hash_tc(gk, k, k, nullptr, r_race, c, rcode, rcode_t, nullptr, nullptr, err,
-                             s));
+    ELSAA_TRY(
+        launch_hash_tc(gk, k, k, nullptr, r_race, c, rcode, rcode_t, nullptr, nullptr, 1, err, s));
   else
     ELSAA_TRY(launch_hash_simt(gk, k, k, nullptr, r_race, c, rcode, rcode_t, s));
   const char* rcode_k = rcode + bhn * g.L * g.rcode_bytes;

@@ -24,6 +24,10 @@
 // w to about 16 significant bits and the products stay exact in fp32.  The
 // read-out writes (w_s . q_i, w_r . q_i) for the query rows.
 //
+// Several Sort-LSH hash rounds (an extension): rounds 1 .. R - 1's sort codes
+// take 16 more columns each after that word (two rounds per 32-bit word), so
+// the one GEMM gives every round's codes.
+//
 // Persistent CTAs of 128 threads.  The hyperplanes stay resident in shared
 // memory; 128-row tiles of Q then K stream in by cp.async (double-buffered
 // where that costs no CTA per SM: at text-32k sizes four single-buffered CTAs
@@ -54,11 +58,12 @@ struct HashShape {
   uint32_t r_bytes, a_bytes, code_bytes, dyn;
 };
 
-HashShape hash_shape(const Geometry& g, bool gates) {
+HashShape hash_shape(const Geometry& g, bool gates, int rounds) {
   HashShape h;
   h.cw = 8 * g.rcode_bytes;
   h.Wr = g.L * h.cw / 32;
   h.P16 = 32 * h.Wr + (gates ? 32 : 16);
+  if (rounds > 1) h.P16 = 32 * h.Wr + 32 + 16 * (rounds - 1);
   h.S = h.Wr | 1;
   h.r_bytes = (uint32_t)h.P16 * g.d * 2;
   h.a_bytes = (uint32_t)kTile * g.d * 2;
@@ -121,7 +126,8 @@ __global__ void __launch_bounds__(kThreads)
 hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                const __nv_bfloat16* __restrict__ r_sort, const __nv_bfloat16* __restrict__ r_race,
                int64_t rows_per_tensor, int N, int sort_bits, int L, int kr, int cw, int Wr, int S,
-               int P16, int nbuf, uint16_t* __restrict__ code, CodeT* __restrict__ rcode,
+               int P16, int nbuf, int rounds, uint16_t* __restrict__ code,
+               CodeT* __restrict__ rcode,
                CodeT* __restrict__ rcode_t, const float* __restrict__ gate_w,
                float2* __restrict__ gl, uint32_t* __restrict__ err) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -163,6 +169,12 @@ hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         if (b < kr) val = *reinterpret_cast<const uint4*>(r_race + (size_t)(t * kr + b) * D + ch * 8);
       } else if (j - race_cols < sort_bits) {
         val = *reinterpret_cast<const uint4*>(r_sort + (size_t)(j - race_cols) * D + ch * 8);
+      } else if (j - race_cols >= 32) {
+        // rounds 1 .. R - 1: 16 columns each
+        const int x = j - race_cols - 32, t = 1 + x / 16, b = x % 16;
+        if (t < rounds && b < sort_bits)
+          val = *reinterpret_cast<const uint4*>(r_sort + ((size_t)t * sort_bits + b) * D +
+                                                ch * 8);
       } else if (gl != nullptr && j - race_cols >= 16 && j - race_cols < 20) {
         // gate columns: w_s hi, w_s lo, w_r hi, w_r lo
         const int gc = j - race_cols - 16;
@@ -237,7 +249,13 @@ hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
 #pragma unroll
         for (int i = 0; i < 32; ++i) m |= (uint32_t)(__float_as_int(v[i]) > 0) << i;
         if (w < Wr) st_w[tid * S + w] = m;
-        else if (w == Wr) {
+        else if (w > Wr) {   // rounds 2 (w - Wr) - 1 and 2 (w - Wr)
+          const int t = 2 * (w - Wr) - 1;
+          const int64_t grow = tile * kTile + tid;
+          code[(size_t)t * 2 * rows_per_tensor + grow] = (uint16_t)(m & 0xFFFFu);
+          if (t + 1 < rounds)
+            code[(size_t)(t + 1) * 2 * rows_per_tensor + grow] = (uint16_t)(m >> 16);
+        } else if (w == Wr) {
           st_code[tid] = (uint16_t)(m & 0xFFFFu);
           const int64_t grow = tile * kTile + tid;
           if (gl != nullptr && grow < rows_per_tensor)   // a query row: its gate logits
@@ -302,8 +320,8 @@ hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
 template <int D, typename CodeT>
 cudaError_t run(const Geometry& g, const void* q, const void* k, const void* r_sort,
                 const void* r_race, uint16_t* code, void* rcode, void* rcode_t,
-                const float* gate_w, float2* gl, uint32_t* err, cudaStream_t s) {
-  const HashShape h = hash_shape(g, gl != nullptr);
+                const float* gate_w, float2* gl, int rounds, uint32_t* err, cudaStream_t s) {
+  const HashShape h = hash_shape(g, gl != nullptr, rounds);
   cudaError_t e = cudaFuncSetAttribute(hash_tc_kernel<D, CodeT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)h.dyn);
   if (e != cudaSuccess) return e;
@@ -326,7 +344,7 @@ cudaError_t run(const Geometry& g, const void* q, const void* k, const void* r_s
   hash_tc_kernel<D, CodeT><<<grid, kThreads, h.dyn, s>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
       static_cast<const __nv_bfloat16*>(r_sort), static_cast<const __nv_bfloat16*>(r_race), rows,
-      g.N, g.sort_bits, g.L, g.kr, h.cw, h.Wr, h.S, h.P16, h.nbuf, code,
+      g.N, g.sort_bits, g.L, g.kr, h.cw, h.Wr, h.S, h.P16, h.nbuf, rounds, code,
       static_cast<CodeT*>(rcode), static_cast<CodeT*>(rcode_t), gate_w, gl, err);
   return cudaGetLastError();
 }
@@ -528,10 +546,10 @@ cudaError_t run_stream(const Geometry& g, const void* q, const void* k, const vo
   return cudaGetLastError();
 }
 
-bool aligned_layout_fits(const Geometry& g, bool gates) {
+bool aligned_layout_fits(const Geometry& g, bool gates, int rounds = 1) {
   // codes fill whole 32-bit words per row; 128-row tiles never straddle units
   if ((g.L * g.rcode_bytes) % 4 != 0 || g.N % kTile != 0 || g.sort_bits > 16) return false;
-  return hash_shape(g, gates).dyn <= (uint32_t)kSmemLimit;
+  return hash_shape(g, gates, rounds).dyn <= (uint32_t)kSmemLimit;
 }
 
 }  // namespace
@@ -547,13 +565,19 @@ bool hash_tc_supported(const Geometry& g) {
   return h.P > 0 && h.dyn <= (uint32_t)kSmemLimit;
 }
 
+bool hash_tc_rounds_supported(const Geometry& g, bool gates) {
+  return g.rounds > 1 && hash_tc_supported(g) && aligned_layout_fits(g, gates, g.rounds);
+}
+
 cudaError_t launch_hash_tc(const Geometry& g, const void* q, const void* k, const void* r_sort,
                            const void* r_race, uint16_t* code, void* rcode, void* rcode_t,
-                           const float* gate_w, float2* gl, uint32_t* err, cudaStream_t s) {
+                           const float* gate_w, float2* gl, int rounds, uint32_t* err,
+                           cudaStream_t s) {
   if (gl != nullptr && !hash_tc_gate_logits_supported(g)) return cudaErrorInvalidValue;
-  const bool al = aligned_layout_fits(g, gl != nullptr);
+  if (rounds > 1 && !aligned_layout_fits(g, gl != nullptr, rounds)) return cudaErrorInvalidValue;
+  const bool al = aligned_layout_fits(g, gl != nullptr, rounds);
 #define ELSAA_HASH(DD, CT)                                                                    \
-  (al ? run<DD, CT>(g, q, k, r_sort, r_race, code, rcode, rcode_t, gate_w, gl, err, s)       \
+  (al ? run<DD, CT>(g, q, k, r_sort, r_race, code, rcode, rcode_t, gate_w, gl, rounds, err, s) \
       : run_stream<DD, CT>(g, q, k, r_sort, r_race, code, rcode, rcode_t, err, s))
   if (g.d == 64) return g.rcode_bytes == 1 ? ELSAA_HASH(64, uint8_t) : ELSAA_HASH(64, uint16_t);
   return g.rcode_bytes == 1 ? ELSAA_HASH(128, uint8_t) : ELSAA_HASH(128, uint16_t);

@@ -89,7 +89,11 @@ cudaError_t launch_hash_simt(const Geometry& g, const void* q, const void* k, co
 // fp32 (hash_tc_gate_logits_supported).
 cudaError_t launch_hash_tc(const Geometry& g, const void* q, const void* k, const void* r_sort,
                            const void* r_race, uint16_t* code, void* rcode, void* rcode_t,
-                           const float* gate_w, float2* gl, uint32_t* err, cudaStream_t s);
+                           const float* gate_w, float2* gl, int rounds, uint32_t* err,
+                           cudaStream_t s);
+// The GEMM also gives the sort codes of hash rounds 1 .. R - 1 (rounds = R in
+// launch_hash_tc; code then holds [R][2][BH][N]).
+bool hash_tc_rounds_supported(const Geometry& g, bool gates);
 bool hash_tc_supported(const Geometry& g);
 bool hash_tc_gate_logits_supported(const Geometry& g);
 
