@@ -105,6 +105,7 @@ WorkLayout work_layout(const Geometry& g) {
   const bool parts = g.rounds > 1 && g.tc_attn;
   w.round_o = take(parts ? (size_t)g.rounds * bhn * g.d * 4 : 0);
   w.round_lse = take(parts ? (size_t)g.rounds * bhn * 4 : 0);
+  w.round_kr = take(parts ? (size_t)g.rounds * (g.rounds - 1) / 2 * bhn * 4 : 0);
   const size_t fwd_end = off;
   // backward temporaries reuse the same bytes (a backward always has a saved buffer)
   off = shared_base;
@@ -158,8 +159,9 @@ cudaError_t sparse_win(const Geometry& g, const void* q, const void* k, const vo
                        void* o_sp, float* lse, uint32_t* err, cudaStream_t s) {
   const size_t bhn = (size_t)g.BH * g.N;
   if (g.rounds == 1) return launch_attn_fwd_win(g, q, k, v, perm, perm + bhn, o_sp, lse, err, s);
-  return launch_attn_fwd_win_rounds(g, q, k, v, perm, rank, (float*)(w + wl.round_o),
-                                    (float*)(w + wl.round_lse), o_sp, lse, err, s);
+  return launch_attn_fwd_win_rounds(g, q, k, v, perm, rank, (int32_t*)(w + wl.round_kr),
+                                    (float*)(w + wl.round_o), (float*)(w + wl.round_lse), o_sp,
+                                    lse, err, s);
 }
 // Several hash rounds: the tcgen05 hash GEMM gives every round's sort codes.
 bool rounds_in_hash(const Geometry& g) {
@@ -561,8 +563,9 @@ elsaa_status elsaa_kernel_launches(const elsaa_params* p, int32_t* fwd, int32_t*
   const int sort = g.rounds * sort1 +
                    (g.rounds > 1 ? 1 + (g.sort_bits > 0 && !rounds_in_hash(g) ? 1 : 0) : 0);
   const int build = race_build_kernels(g, false, g.bf16);
-  // (several rounds on tcgen05: one window pass per round + the combine)
-  const int sparse_fwd = g.rounds > 1 && win_fwd(g) ? g.rounds + 1 : 1;
+  // (several rounds on tcgen05: the key ranks, one window pass per round and
+  // the combine)
+  const int sparse_fwd = g.rounds > 1 && win_fwd(g) ? 1 + g.rounds + 1 : 1;
   *fwd = g.causal ? 1 + sort + 1 + sparse_fwd + 1 : 1 + sort + 1 + build + sparse_fwd + 1;
   // fusion backward 1, RACE build 1 + gather 1, sparse 1 (+ casts), reduction 1
   // (direct path: the sparse kernel writes dq itself and the gather adds into dv)

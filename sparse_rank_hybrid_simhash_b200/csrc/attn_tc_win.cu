@@ -18,8 +18,10 @@
 // extension: a query attends the union of its rounds' windows, each key once)
 // the kernel runs once per round t on that round's orders, drops the keys
 // that lie in the query's window of an earlier round (by the keys' and the
-// query's ranks in that round), and writes the round's partial softmax (O_t
-// normalized by its own mass, in fp32, and lse_t) for round_combine_kernel.
+// query's ranks in that round; the keys' earlier ranks come laid out in round
+// t's key order, from round_key_ranks_kernel), and writes the round's partial
+// softmax (O_t normalized by its own mass, in fp32, and lse_t) for
+// round_combine_kernel.
 // A window may exceed what TMEM holds next to O, so each tile takes two
 // passes over its blocks: pass 1 computes S = Q K^T block by block for the
 // exact row maximum; pass 2 computes S again, P = exp(scale s - m) (bf16, in
@@ -151,7 +153,8 @@ attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restr
                     const int32_t* __restrict__ perm_k, int BH, int N, int chunk, int lookback,
                     int causal, float scale_log2, __nv_bfloat16* __restrict__ o_sp,
                     float* __restrict__ lse, const int32_t* __restrict__ rank, int round,
-                    int64_t rank_len, float* __restrict__ o_part, float* __restrict__ lse_part,
+                    int64_t rank_len, const int32_t* __restrict__ kranks,
+                    float* __restrict__ o_part, float* __restrict__ lse_part,
                     uint32_t* __restrict__ err) {
   using Lay = WinLayout<D>;
   constexpr int KS = Lay::kKSlots, VS = Lay::kVSlots, OB = Lay::kOBufs;
@@ -383,44 +386,40 @@ attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restr
           whi[u] = min(N, (ju + 1) * chunk);
         }
       }
-      // a key of this round's window that an earlier round's window of the
-      // query already holds
-      auto seen = [&](int key) {
-        bool in = false;
-#pragma unroll
-        for (int u = 0; u < MR; ++u)
-          if (u < round) {
-            const int64_t at = u * rstride + rows + (int64_t)unit + key;
-            if (at < 0 || at >= rank_len || key < 0 || key >= N) {   // checked: never taken
-              raise_error(err, ERR_CHECK);
-              continue;
-            }
-            const int rk = __ldg(rank + at);
-            in |= rk >= wlo[u] && rk < whi[u];
-          }
-        return in;
-      };
       // bit e: column cb + e of block b is a key of the row (its window; with
       // the causal mask, a token index at most the query's; with several
-      // rounds, not seen in an earlier round)
+      // rounds, not in an earlier round's window of the query)
       auto allow_bits = [&](int b) -> uint64_t {
         const int c0 = b * kTile + cb;
         const int a = max(0, lo - c0), z = min(64, hi - c0);
         if (a >= z) return 0ull;
         uint64_t bits = (z == 64 ? ~0ull : (1ull << z) - 1ull) & ~((1ull << a) - 1ull);
-        if (causal || round > 0) {
-          const int4* kt = reinterpret_cast<const int4*>(
-              perm_k + unit + (size_t)(w.kb_lo + b) * kTile + cb);
-          auto keep = [&](int key) { return (!causal || key <= token) && !(round > 0 && seen(key)); };
+        const size_t pos = unit + (size_t)(w.kb_lo + b) * kTile + cb;   // sorted key position
+        if (causal) {
+          const int4* kt = reinterpret_cast<const int4*>(perm_k + pos);
           uint64_t c = 0;
 #pragma unroll 2
           for (int e4 = 0; e4 < 16; ++e4) {
             const int4 t = __ldg(kt + e4);
-            c |= ((uint64_t)keep(t.x) | (uint64_t)keep(t.y) << 1 | (uint64_t)keep(t.z) << 2 |
-                  (uint64_t)keep(t.w) << 3)
+            c |= ((uint64_t)(t.x <= token) | (uint64_t)(t.y <= token) << 1 |
+                  (uint64_t)(t.z <= token) << 2 | (uint64_t)(t.w <= token) << 3)
                  << (4 * e4);
           }
           bits &= c;
+        }
+#pragma unroll
+        for (int u = 0; u < MR; ++u) {
+          if (u >= round) break;
+          const int4* kr = reinterpret_cast<const int4*>(kranks + u * rows + pos);
+          const int lo_u = wlo[u], hi_u = whi[u];
+          auto in = [&](int x) { return (uint64_t)(x >= lo_u && x < hi_u); };
+          uint64_t sb = 0;
+#pragma unroll 2
+          for (int e4 = 0; e4 < 16; ++e4) {
+            const int4 t = __ldg(kr + e4);
+            sb |= (in(t.x) | in(t.y) << 1 | in(t.z) << 2 | in(t.w) << 3) << (4 * e4);
+          }
+          bits &= ~sb;
         }
         return bits;
       };
@@ -548,8 +547,8 @@ attn_fwd_win_kernel(const __grid_constant__ WinMaps maps, const int32_t* __restr
 template <int D, int MR>
 cudaError_t launch(const Geometry& g, const void* q, const void* k, const void* v,
                    const int32_t* perm_q, const int32_t* perm_k, void* o_sp, float* lse,
-                   const int32_t* rank, int round, float* o_part, float* lse_part, uint32_t* err,
-                   cudaStream_t s) {
+                   const int32_t* rank, int round, const int32_t* kranks, float* o_part,
+                   float* lse_part, uint32_t* err, cudaStream_t s) {
   using Lay = WinLayout<D>;
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_win_kernel<D, MR>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -568,7 +567,7 @@ cudaError_t launch(const Geometry& g, const void* q, const void* k, const void* 
   attn_fwd_win_kernel<D, MR><<<grid_x, kThreads, Lay::kDyn, s>>>(
       maps, perm_q, perm_k, g.BH, g.N, g.chunk, g.lookback, g.causal ? 1 : 0,
       g.scale * 1.4426950408889634f, static_cast<__nv_bfloat16*>(o_sp), lse, rank, round,
-      (int64_t)g.rounds * 2 * g.BH * g.N, o_part, lse_part, err);
+      (int64_t)g.rounds * 2 * g.BH * g.N, kranks, o_part, lse_part, err);
   return cudaGetLastError();
 }
 
@@ -604,6 +603,25 @@ round_combine_kernel(const float* __restrict__ o_part, const float* __restrict__
   }
 }
 
+// For round pairs u < t: the rank in round u of round t's sorted key pos,
+// kranks[(t (t - 1) / 2 + u) rows + unit + pos] = rank_k[u][unit + perm_k[t][unit + pos]]
+// (perm and rank: [R][2][BH][N], token indices within the unit).
+__global__ void __launch_bounds__(256)
+round_key_ranks_kernel(const int32_t* __restrict__ perm, const int32_t* __restrict__ rank,
+                       int R, int64_t rows, int N, int32_t* __restrict__ kranks) {
+  const int64_t total = (int64_t)R * (R - 1) / 2 * rows;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t pair = i / rows, x = i - pair * rows;
+    int t = 1;
+    while ((int64_t)t * (t + 1) / 2 <= pair) ++t;   // pairs t (t - 1) / 2 .. t (t + 1) / 2 - 1
+    const int u = (int)(pair - (int64_t)t * (t - 1) / 2);
+    const int64_t unit = x / N * N;
+    const int key = perm[(int64_t)t * 2 * rows + rows + x];
+    kranks[i] = rank[(int64_t)u * 2 * rows + rows + unit + key];
+  }
+}
+
 }  // namespace
 
 bool attn_win_supported(const Geometry& g) {
@@ -617,29 +635,35 @@ cudaError_t launch_attn_fwd_win(const Geometry& g, const void* q, const void* k,
                                 const int32_t* perm_q, const int32_t* perm_k, void* o_sp,
                                 float* lse, uint32_t* err, cudaStream_t s) {
   return g.d == 64 ? launch<64, 1>(g, q, k, v, perm_q, perm_k, o_sp, lse, nullptr, 0, nullptr,
-                                   nullptr, err, s)
+                                   nullptr, nullptr, err, s)
                    : launch<128, 1>(g, q, k, v, perm_q, perm_k, o_sp, lse, nullptr, 0, nullptr,
-                                    nullptr, err, s);
+                                    nullptr, nullptr, err, s);
 }
 
 cudaError_t launch_attn_fwd_win_rounds(const Geometry& g, const void* q, const void* k,
                                        const void* v, const int32_t* perm, const int32_t* rank,
-                                       float* o_part, float* lse_part, void* o_sp, float* lse,
-                                       uint32_t* err, cudaStream_t s) {
+                                       int32_t* kranks, float* o_part, float* lse_part,
+                                       void* o_sp, float* lse, uint32_t* err, cudaStream_t s) {
   const int64_t rows = (int64_t)g.BH * g.N;
+  const int64_t total = (int64_t)g.rounds * (g.rounds - 1) / 2 * rows;
+  const int64_t want = (total + 255) / 256;
+  round_key_ranks_kernel<<<(int)(want < 148 * 32 ? want : 148 * 32), 256, 0, s>>>(
+      perm, rank, g.rounds, rows, g.N, kranks);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   for (int t = 0; t < g.rounds; ++t) {
     const int32_t* pq = perm + (size_t)t * 2 * rows;
+    const int32_t* kr = kranks + (size_t)t * (t - 1) / 2 * rows;
     float* op = o_part + (size_t)t * rows * g.d;
     float* lp = lse_part + (size_t)t * rows;
-    const cudaError_t e =
-        g.d == 64
-            ? launch<64, kMaxRounds>(g, q, k, v, pq, pq + rows, o_sp, lse, rank, t, op, lp, err, s)
-            : launch<128, kMaxRounds>(g, q, k, v, pq, pq + rows, o_sp, lse, rank, t, op, lp, err,
-                                      s);
+    e = g.d == 64 ? launch<64, kMaxRounds>(g, q, k, v, pq, pq + rows, o_sp, lse, rank, t, kr, op,
+                                           lp, err, s)
+                  : launch<128, kMaxRounds>(g, q, k, v, pq, pq + rows, o_sp, lse, rank, t, kr, op,
+                                            lp, err, s);
     if (e != cudaSuccess) return e;
   }
-  const int64_t want = (rows + 7) / 8;
-  const int grid = (int)(want < 148 * 16 ? want : 148 * 16);
+  const int64_t wc = (rows + 7) / 8;
+  const int grid = (int)(wc < 148 * 16 ? wc : 148 * 16);
   round_combine_kernel<<<grid, 256, 0, s>>>(o_part, lse_part, g.rounds, rows, g.d,
                                             static_cast<__nv_bfloat16*>(o_sp), lse);
   return cudaGetLastError();

@@ -60,6 +60,7 @@ struct WorkLayout {
   size_t causal_num;         // [BH][N][d] f32: causal RACE numerators (0 bytes unless causal)
   size_t saved;              // a SavedLayout used when the forward has no saved buffer
   size_t round_o, round_lse; // [R][BH][N][d] / [R][BH][N] f32: per-round partial softmax
+  size_t round_kr;           // [R (R - 1) / 2][BH][N] i32: keys' earlier-round ranks
                              // (several hash rounds on the tcgen05 forward; else 0 bytes)
   size_t d_o;                // [BH][N][d] dtype: dO_sp
   size_t dprime;             // [BH][N] f32: D' = dO_sp . O_sp - dlse
@@ -200,13 +201,14 @@ bool attn_win_supported(const Geometry& g);
 cudaError_t launch_attn_fwd_win(const Geometry& g, const void* q, const void* k, const void* v,
                                 const int32_t* perm_q, const int32_t* perm_k, void* o_sp,
                                 float* lse, uint32_t* err, cudaStream_t s);
-// Several hash rounds: one streamed-window pass per round (perm and rank
-// [R][2][BH][N]), each writing its partial softmax to o_part / lse_part, then
-// their combine into o_sp and lse.
+// Several hash rounds: the keys' earlier-round ranks in each round's key order
+// (kranks, [R (R - 1) / 2][BH][N] i32), one streamed-window pass per round
+// (perm and rank [R][2][BH][N]), each writing its partial softmax to o_part /
+// lse_part, then their combine into o_sp and lse.
 cudaError_t launch_attn_fwd_win_rounds(const Geometry& g, const void* q, const void* k,
                                        const void* v, const int32_t* perm, const int32_t* rank,
-                                       float* o_part, float* lse_part, void* o_sp, float* lse,
-                                       uint32_t* err, cudaStream_t s);
+                                       int32_t* kranks, float* o_part, float* lse_part,
+                                       void* o_sp, float* lse, uint32_t* err, cudaStream_t s);
 // tcgen05 backward for any window (key-major, one CTA per 128 sorted keys):
 // dq_acc += dQ (fp32 atomics); dk, dv written (dv adds dv_race).
 cudaError_t launch_attn_bwd_tc(const Geometry& g, const void* q, const void* k, const void* v,

@@ -174,11 +174,11 @@ def test_kernel_launch_counts():
     c = B.kernel_launches(B.Params.from_workload(w.replace(causal=True, dtype="f32")))
     assert c == (1 + 3 + 1 + 1 + 1, 1 + 1 + 4 + 1)
     # three hash rounds: every round's sort codes from the one hash GEMM, three
-    # sorts, the inverse orders, one streamed-window pass per round and their
-    # combine; backward: one key-major pass per round + 3 casts (fp32: a second
+    # sorts, the inverse orders, the keys' earlier-round ranks, one
+    # streamed-window pass per round and their combine; backward: one key-major pass per round + 3 casts (fp32: a second
     # hash kernel for the other rounds' codes and CUDA-core attention both ways)
     r = B.kernel_launches(B.Params.from_workload(w.replace(hash_rounds=3)))
-    assert r == (1 + 3 * 3 + 1 + 2 + (3 + 1) + 1, 1 + 2 + (3 + 3) + 1)
+    assert r == (1 + 3 * 3 + 1 + 2 + (1 + 3 + 1) + 1, 1 + 2 + (3 + 3) + 1)
     r = B.kernel_launches(B.Params.from_workload(w.replace(hash_rounds=3, dtype="f32")))
     assert r == (1 + 1 + 3 * 3 + 1 + 2 + 1 + 1, 1 + 2 + 1 + 3 + 1)
 
