@@ -84,14 +84,15 @@ ELSAA_DEV uint32_t pack_bf16(float a, float b) {
 }
 
 // MR: the largest hash-round count the instance handles (1, or kMaxRounds
-// for the several-round passes).
-template <int D, int MR>
+// for the several-round passes); CAUSAL: the causal mask (compile-time, so the
+// element loop of the other instances carries no test for it).
+template <int D, int MR, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads)
 attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                    const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ perm_q,
                    const int32_t* __restrict__ perm_k, const __nv_bfloat16* __restrict__ d_o,
                    const float* __restrict__ lse, const float* __restrict__ dprime,
-                   const float* __restrict__ dv_race, int N, int chunk, int lookback, int causal,
+                   const float* __restrict__ dv_race, int N, int chunk, int lookback,
                    const int32_t* __restrict__ rank, int round, float* __restrict__ dk_acc,
                    float* __restrict__ dv_acc, float scale,
                    float scale_log2, float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk,
@@ -123,15 +124,17 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
   const int nqb = (qend - qbase + kTile - 1) / kTile;
   const int key_chunk = (k0 + tid) / chunk;
   const int my_tok = pk[k0 + tid];
-  // several rounds: this key's ranks in the earlier rounds, and per query
-  // column the query's earlier windows [s_wlo, s_whi)
+  // several rounds: this key's chunk in each earlier round, and per query
+  // column the query's chunk there (a key is in a query's window of round u
+  // when 0 <= query chunk - key chunk <= lookback); s_qc: the columns' chunks
+  // in this round
   const int64_t rows = (int64_t)gridDim.y * N, rstride = 2 * rows;   // rank: [R][2][BH][N]
-  int my_rank[MR];
+  int my_chunk[MR];
 #pragma unroll
   for (int u = 0; u < MR; ++u)
-    my_rank[u] = u < round ? rank[u * rstride + rows + unit + my_tok] : 0;
-  int32_t* s_wlo = reinterpret_cast<int32_t*>(smem + Lay::kWin);   // [kMaxRounds - 1][128]
-  int32_t* s_whi = s_wlo + (kMaxRounds - 1) * 128;
+    my_chunk[u] = u < round ? rank[u * rstride + rows + unit + my_tok] / chunk : 0;
+  int32_t* s_qj = reinterpret_cast<int32_t*>(smem + Lay::kWin);   // [kMaxRounds - 1][128]
+  int32_t* s_qc = s_qj + (kMaxRounds - 1) * 128;                  // [128]
 
   if (tid == 0) {
     mbar_init(bar_a, 1);
@@ -159,11 +162,9 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
     const int nq = min(kTile, qend - qb0);
     if (tid < nq) {
       qidx[tid] = pq[qb0 + tid];
-      for (int u = 0; u < round; ++u) {
-        const int ju = rank[u * rstride + unit + qidx[tid]] / chunk;
-        s_wlo[u * 128 + tid] = max(0, (ju - lookback) * chunk);
-        s_whi[u * 128 + tid] = min(N, (ju + 1) * chunk);
-      }
+      s_qc[tid] = (qb0 + tid) / chunk;
+      for (int u = 0; u < round; ++u)
+        s_qj[u * 128 + tid] = rank[u * rstride + unit + qidx[tid]] / chunk;
     }
     __syncthreads();
     gather_rows<D>(sbase + Lay::kQ, q + unit * D, qidx, nq);
@@ -210,6 +211,30 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
       tmem_ld32(tmem + Lay::kTS + lane_off + c0, sv);
       tmem_ld32(tmem + Lay::kTdP + lane_off + c0, dp);
       tmem_ld_wait();
+      // bit i: column c0 + i is a query of this key (in this round's window,
+      // causal if asked, not in an earlier round's window); the one-round
+      // instance tests each element in place instead
+      uint32_t okb = 0;
+      if constexpr (MR > 1) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int col = c0 + i;
+          const bool in = col < nq && (uint32_t)(s_qc[col] - key_chunk) <= (uint32_t)lookback &&
+                          (!CAUSAL || my_tok <= qidx[col]);
+          okb |= (uint32_t)in << i;
+        }
+#pragma unroll
+        for (int u = 0; u < MR; ++u) {
+          if (u >= round) break;
+          uint32_t sb = 0;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            sb |= (uint32_t)((uint32_t)(s_qj[u * 128 + c0 + i] - my_chunk[u]) <=
+                             (uint32_t)lookback)
+                  << i;
+          okb &= ~sb;
+        }
+      }
       uint32_t pp[16], dd[16];
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {
@@ -217,16 +242,17 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int col = c0 + i + e;
-          const int dj = (qb0 + col) / chunk - key_chunk;
           p[e] = 0.f;
           ds[e] = 0.f;
-          bool seen = false;
-#pragma unroll
-          for (int u = 0; u < MR; ++u)
-            if (u < round && col < nq)
-              seen |= my_rank[u] >= s_wlo[u * 128 + col] && my_rank[u] < s_whi[u * 128 + col];
-          if (col < nq && dj >= 0 && dj <= lookback && (!causal || my_tok <= qidx[col]) &&
-              !seen) {
+          bool ok;
+          if constexpr (MR > 1) {
+            ok = (okb >> (i + e)) & 1u;
+          } else {
+            const int dj = (qb0 + col) / chunk - key_chunk;
+            ok = col < nq && dj >= 0 && dj <= lookback;
+            if constexpr (CAUSAL) ok = ok && my_tok <= qidx[col];
+          }
+          if (ok) {
             p[e] = exp2f(sv[i + e] * scale_log2 - s_lse[col]);
             ds[e] = scale * p[e] * (dp[i + e] - s_dpr[col]);
           }
@@ -352,25 +378,37 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
   }
 }
 
+template <int D, int MR, bool CAUSAL>
+cudaError_t bwd1(const Geometry& g, const void* q, const void* k, const void* v,
+                const int32_t* perm_q, const int32_t* perm_k, const void* d_o, const float* lse,
+                const float* dprime, const float* dv_race, float* dq_acc, void* dk, void* dv,
+                const int32_t* rank, int round, float* dk_acc, float* dv_acc, uint32_t* err,
+                cudaStream_t s) {
+  using Lay = BwdLayout<D>;
+  cudaError_t e = cudaFuncSetAttribute(attn_bwd_tc_kernel<D, MR, CAUSAL>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kDyn);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(g.N / kTile, g.BH);
+  attn_bwd_tc_kernel<D, MR, CAUSAL><<<grid, kThreads, Lay::kDyn, s>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+      static_cast<const __nv_bfloat16*>(v), perm_q, perm_k,
+      static_cast<const __nv_bfloat16*>(d_o), lse, dprime, dv_race, g.N, g.chunk, g.lookback,
+      rank, round, dk_acc, dv_acc, g.scale,
+      g.scale * 1.4426950408889634f, dq_acc, static_cast<__nv_bfloat16*>(dk),
+      static_cast<__nv_bfloat16*>(dv), err);
+  return cudaGetLastError();
+}
+
 template <int D, int MR>
 cudaError_t bwd(const Geometry& g, const void* q, const void* k, const void* v,
                 const int32_t* perm_q, const int32_t* perm_k, const void* d_o, const float* lse,
                 const float* dprime, const float* dv_race, float* dq_acc, void* dk, void* dv,
                 const int32_t* rank, int round, float* dk_acc, float* dv_acc, uint32_t* err,
                 cudaStream_t s) {
-  using Lay = BwdLayout<D>;
-  cudaError_t e = cudaFuncSetAttribute(attn_bwd_tc_kernel<D, MR>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kDyn);
-  if (e != cudaSuccess) return e;
-  const dim3 grid(g.N / kTile, g.BH);
-  attn_bwd_tc_kernel<D, MR><<<grid, kThreads, Lay::kDyn, s>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-      static_cast<const __nv_bfloat16*>(v), perm_q, perm_k,
-      static_cast<const __nv_bfloat16*>(d_o), lse, dprime, dv_race, g.N, g.chunk, g.lookback,
-      g.causal ? 1 : 0, rank, round, dk_acc, dv_acc, g.scale,
-      g.scale * 1.4426950408889634f, dq_acc, static_cast<__nv_bfloat16*>(dk),
-      static_cast<__nv_bfloat16*>(dv), err);
-  return cudaGetLastError();
+  return g.causal ? bwd1<D, MR, true>(g, q, k, v, perm_q, perm_k, d_o, lse, dprime, dv_race,
+                                      dq_acc, dk, dv, rank, round, dk_acc, dv_acc, err, s)
+                  : bwd1<D, MR, false>(g, q, k, v, perm_q, perm_k, d_o, lse, dprime, dv_race,
+                                       dq_acc, dk, dv, rank, round, dk_acc, dv_acc, err, s);
 }
 
 }  // namespace
