@@ -127,14 +127,14 @@ def stage_roofline(flops, nbytes, sec, peaks):
 TRAFFIC_WORKLOAD, TRAFFIC_UNITS = "text-32k", 12
 RECORDED_TRAFFIC = {
     # stage: (kernel source, its sha1 at capture, bytes per 12-unit launch, path flag needed)
-    "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "d38b93c83be7bafa7040797e9a19dce5b2ba90f0", 1.259e+08, "tc_hash"),
-    "race_build": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "15a1fb45c20eb380372ec944794c10506c62861f", 6.91e+07, None),
-    "sparse_fwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_pipe.cu", "91a31d0c88874e37ef33ed4bb443baabc0c07369", 1.87e+08, "tc_attn"),
-    "race_fuse": ("sparse_rank_hybrid_simhash_b200/csrc/race_slab.cu", "5135a962ed6cf3d305d45cb27ffcdf41815cc38e", 1.448e+08, "slab_fwd"),
-    "fuse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/fuse_bwd.cu", "d225c68863731ac35a2126d849af1623d8c512c7", 2.817e+08, None),
-    "race_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "15a1fb45c20eb380372ec944794c10506c62861f", 6.67e+07, None),
-    "sparse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_bwd3.cu", "d8764bf2cfd3093b7f01c78d4ad9412897ad1eeb", 3.321e+08, "tc_attn"),
-    "finish": ("sparse_rank_hybrid_simhash_b200/csrc/race_slab.cu", "5135a962ed6cf3d305d45cb27ffcdf41815cc38e", 7.85e+07, "slab_bwd"),
+    "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "0f6d6d0fa080567b642065af04df9b3345737c4f", 1.2331e+08, "tc_hash"),
+    "race_build": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "15a1fb45c20eb380372ec944794c10506c62861f", 6.874e+07, None),
+    "sparse_fwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_pipe.cu", "b33f474224da484dfb1f6128dd2527644c56625a", 1.8644e+08, "tc_attn"),
+    "race_fuse": ("sparse_rank_hybrid_simhash_b200/csrc/race_slab.cu", "5135a962ed6cf3d305d45cb27ffcdf41815cc38e", 1.4487e+08, "slab_fwd"),
+    "fuse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/fuse_bwd.cu", "d225c68863731ac35a2126d849af1623d8c512c7", 2.8098e+08, None),
+    "race_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "15a1fb45c20eb380372ec944794c10506c62861f", 6.688e+07, None),
+    "sparse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_bwd3.cu", "ffbd2e8b9a9bb8a1a16dfa244ec836a1dc90ccdc", 3.3276e+08, "tc_attn"),
+    "finish": ("sparse_rank_hybrid_simhash_b200/csrc/race_slab.cu", "5135a962ed6cf3d305d45cb27ffcdf41815cc38e", 7.874e+07, "slab_bwd"),
 }
 
 
