@@ -92,19 +92,25 @@ typedef struct {
   int32_t lookback;       /* previous sorted chunks a query chunk attends besides its own,
                            * 0..64 with (lookback + 1) * chunk <= 6144: 1 is the pages'
                            * Sort-LSH (own and previous chunk); other values are an
-                           * extension served by the CUDA-core attention kernels */
+                           * extension (bf16: the streamed-window tcgen05 forward and
+                           * the key-major tcgen05 backward) */
   int32_t causal;         /* nonzero: query i sees only keys j <= i (token index), in the
                            * sparse window and in the RACE read-out (an extension: the
                            * pages did not evaluate causal use); a window left without
-                           * keys has Z_sp = 0 (O_sp = 0, lse = -inf).  Runs on the
-                           * CUDA-core attention and a per-table token scan for RACE;
-                           * needs 2^race_bits * (d + 1) * 4 <= 200 KB */
+                           * keys has Z_sp = 0 (O_sp = 0, lse = -inf).  bf16 runs on
+                           * the tcgen05 window forward and key-major backward with a
+                           * token mask; the RACE read-out walks the tables token by
+                           * token (L in {4, 8, 16, 32} and N % 32 == 0 with
+                           * 2 * 2^race_bits * 128 <= 200 KB, else per-table scans that
+                           * need 2^race_bits * (d + 1) * 4 <= 200 KB) */
   int32_t hash_rounds;    /* Sort-LSH hash rounds, 0..8 (0 and 1 both mean one round, the
                            * pages' setting).  With R > 1 rounds every round t sorts Q
                            * and K by its own sort hyperplanes r_sort[t], and a query
                            * attends the union of its R windows, each key once, with
-                           * exact softmax (an extension; runs on the CUDA-core
-                           * attention; needs R * (lookback + 1) * chunk <= 6144) */
+                           * exact softmax (an extension; bf16: every round's codes from
+                           * the hash GEMM, one tcgen05 window pass per round and a
+                           * combine, one backward pass per round; needs R * (lookback
+                           * + 1) * chunk <= 6144) */
 } elsaa_params;
 
 /* Device views into a forward's saved state (see elsaa_saved_views). */
@@ -238,7 +244,8 @@ const char* elsaa_status_str(elsaa_status s);
 
 /* Which kernel family the sparse branch and the hash take for `p`:
  * 1 = tcgen05 tensor-core kernels, 0 = CUDA-core kernels (fp32 data, head
- * dims other than 64/128, or chunk shapes the tensor kernels do not tile). */
+ * dims other than 64/128, N not a multiple of 128, or chunks that are not
+ * a multiple of 16). */
 int32_t elsaa_uses_tensor_cores(const elsaa_params* p);
 
 /* ---- Pieces of the operator for a sequence split across devices ---------
@@ -305,8 +312,9 @@ elsaa_status elsaa_race_value_grad(const elsaa_params* p, const void* k, const v
  * read-out from shared-memory table slabs (gate logits from the hash GEMM);
  * ELSAA_PATH_SLAB_BWD the RACE value gradient from shared-memory slabs;
  * ELSAA_PATH_TC_WIN the sparse forward on the tcgen05 kernel that streams
- * the window in 128-key blocks (d = 128, chunks above 128, lookback other
- * than 1; the backward of those shapes runs on CUDA cores). */
+ * the window in 128-key blocks (d = 128, chunks above or not dividing 128,
+ * lookback other than 1, causal, several hash rounds; their backward takes
+ * the key-major tcgen05 kernel). */
 #define ELSAA_PATH_TC_HASH 1
 #define ELSAA_PATH_TC_ATTN 2
 #define ELSAA_PATH_SLAB_FWD 4

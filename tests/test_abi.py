@@ -159,6 +159,16 @@ def test_tensor_core_path_selection(name):
     w = WORKLOADS[name]
     expect = w.dtype == "bf16"   # every bf16 workload tiles onto the tcgen05 kernels
     assert B.uses_tensor_cores(B.Params.from_workload(w)) == expect
+    if expect:
+        # and so do its extensions: other lookbacks, the causal mask, several rounds
+        # (where the library accepts them: causal needle-256k's 64 x 1024-bucket
+        # tables fit neither causal RACE kernel and are rejected)
+        for x in (w.replace(lookback=2), w.replace(causal=True), w.replace(hash_rounds=2)):
+            p = B.Params.from_workload(x)
+            if B.validate(p) == 0:
+                assert B.uses_tensor_cores(p) == 1, x
+            else:
+                assert x.causal and x.race_tables > 32 and B.uses_tensor_cores(p) == 0
 
 
 def test_kernel_launch_counts():
