@@ -48,7 +48,7 @@ ELSAA_DEV int code_at(const uint4* c, int p) {
 // for Ctot and the count tables); MODE 1: backward (x = g_r dy / Ctot by
 // query code; out = the RACE value gradient).  L = 2^LOGL tables; lane =
 // (sub, l), sub picking one of the warp's 32 / L columns.  Codes come
-// table-major ([BH][L][N]); tokens go in groups of 32, loaded one group
+// table-major ([BH][L][N]); tokens go in groups of 32, loaded two groups
 // ahead: a lane's 32 codes of its table in 16-byte words, and one x value
 // per lane that the shuffles hand to the lanes that need it.  After a
 // group's shared-memory steps each lane holds 32 partial sums (its table's
@@ -97,11 +97,14 @@ race_causal_walk_kernel(const CodeT* __restrict__ rtq, const CodeT* __restrict__
     for (int k = 0; k < PER; ++k)
       in.xv[k] = count_walk ? 0.f : to_f32(x[(u + base + l + L * k) * d + col]);
   };
-  In cur, nxt;
+  // two groups in flight ahead of the one being walked
+  In cur, nxt, nxt2;
   fetch(0, nxt);
+  if (ngroups > 1) fetch(1, nxt2);
   for (int g = 0; g < ngroups; ++g) {
     cur = nxt;
-    if (g + 1 < ngroups) fetch(g + 1, nxt);
+    nxt = nxt2;
+    if (g + 2 < ngroups) fetch(g + 2, nxt2);
     const int base = base_of(g);
     if (count_walk) {
       int c[G];
