@@ -70,6 +70,7 @@ class HostStepPipeline:
         self.s_in = torch.cuda.Stream(self.dev)
         self.s_comp = torch.cuda.Stream(self.dev)
         self.s_out = torch.cuda.Stream(self.dev)
+        self.n = 0   # groups enqueued so far (the slot use count runs across steps)
 
     def h2d_bytes(self, host: Dict[str, torch.Tensor]) -> int:
         return sum(host[k].numel() * host[k].element_size() for k in ("q", "k", "v", "dy"))
@@ -78,29 +79,47 @@ class HostStepPipeline:
                 stream: Optional[torch.cuda.Stream] = None) -> None:
         """Enqueue one step: host["q"|"k"|"v"|"dy"] in, out["y"|"dq"|"dk"|"dv"]
         written, all pinned [B, H, N, d]; the groups' parameter-gradient partial
-        sums land in self.pg_host.  `stream` (default: current) waits for the
-        whole step; call gradients() after synchronising it."""
+        sums land in self.pg_host.  The step starts after the work already on
+        `stream` (default: current), and `stream` waits for the whole step; call
+        gradients() after synchronising it."""
+        self.start_after(stream)
+        self.enqueue_chained(host, out)
+        self.join(stream)
+
+    def start_after(self, stream: Optional[torch.cuda.Stream] = None) -> None:
+        """What is enqueued next starts after the work already on `stream`
+        (default: current)."""
         main = stream if stream is not None else torch.cuda.current_stream(self.dev)
-        BH, N, d = self.groups * self.per, self.p.N, self.p.d
-        hin = {k: host[k].view(BH, N, d) for k in ("q", "k", "v", "dy")}
-        hout = {k: out[k].view(BH, N, d) for k in ("y", "dq", "dk", "dv")}
         start = torch.cuda.Event()
         start.record(main)
         for s in (self.s_in, self.s_comp, self.s_out):
             s.wait_event(start)
+
+    def enqueue_chained(self, host: Dict[str, torch.Tensor], out: Dict[str, torch.Tensor]) -> None:
+        """Enqueue one step behind the steps enqueued before it on the
+        pipeline's own streams, without waiting for any other stream: the
+        first groups' copy-in overlaps the previous step's last compute and
+        copy-out.  For back-to-back steps over host data; join() makes a
+        stream wait for everything enqueued so far.  (out and pg_host are
+        rewritten by every step.)"""
+        BH, N, d = self.groups * self.per, self.p.N, self.p.d
+        hin = {k: host[k].view(BH, N, d) for k in ("q", "k", "v", "dy")}
+        hout = {k: out[k].view(BH, N, d) for k in ("y", "dq", "dk", "dv")}
         sm = self.small
         for g in range(self.groups):
-            sl = self.slots[g % 2]
+            n = self.n
+            self.n += 1
+            sl = self.slots[n % 2]
             u0, u1 = g * self.per, (g + 1) * self.per
             with torch.cuda.stream(self.s_in):
-                if g >= 2:
+                if n >= 2:
                     self.s_in.wait_event(sl["ev_comp"])   # the slot's inputs are free again
                 for k in hin:
                     sl["in"][k][0].copy_(hin[k][u0:u1], non_blocking=True)
                 sl["ev_in"].record(self.s_in)
             with torch.cuda.stream(self.s_comp):
                 self.s_comp.wait_event(sl["ev_in"])
-                if g >= 2:
+                if n >= 2:
                     self.s_comp.wait_event(sl["ev_out"])   # the slot's outputs are out
                 i, o = sl["in"], sl["out"]
                 B.forward(self.pg, i["q"], i["k"], i["v"], sm["r_sort"], sm["r_race"],
@@ -119,6 +138,10 @@ class HostStepPipeline:
                 row[2 * d:2 * d + 2].copy_(sl["pg"][1], non_blocking=True)
                 row[2 * d + 2:].copy_(sl["pg"][2], non_blocking=True)
                 sl["ev_out"].record(self.s_out)
+
+    def join(self, stream: Optional[torch.cuda.Stream] = None) -> None:
+        """`stream` (default: current) waits for every step enqueued so far."""
+        main = stream if stream is not None else torch.cuda.current_stream(self.dev)
         for s in (self.s_in, self.s_comp, self.s_out):
             main.wait_stream(s)
 
