@@ -35,7 +35,9 @@
 // of 128: thread t reads the 32 projections of row t per tcgen05.ld and keeps
 // the sign mask.  The tile's codes leave as one contiguous row-major block and,
 // through a 4 x 4 (or 2 x 2) byte transpose across lanes, as 4-byte runs of
-// each table's table-major codes.
+// each table's table-major codes.  Shapes this word-aligned layout does not
+// fit take the bit-stream variant (hash_tc_stream.cu).
+#include "hash_tile.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
 
@@ -43,12 +45,13 @@ namespace elsaa {
 namespace {
 
 using namespace tc;
+using hash::kTile;
+using hash::kPass;
+using hash::kSmemLimit;
+using hash::load_tile;
 
-constexpr int kTile = 128;
 constexpr int kThreads = 128;
-constexpr int kPass = 128;            // TMEM columns per pass
 constexpr uint32_t kTmemCols = 128;
-constexpr int kSmemLimit = 227 * 1024;
 
 struct HashShape {
   int P16;       // columns: 32 Wr RACE columns, 16 sort columns (+ 16 with gate columns)
@@ -81,44 +84,6 @@ HashShape hash_shape(const Geometry& g, bool gates, int rounds) {
   h.nbuf = (dyn2 <= (uint32_t)kSmemLimit && per_sm(dyn2) >= per_sm(dyn1)) ? 2 : 1;
   h.dyn = h.nbuf == 2 ? dyn2 : dyn1;
   return h;
-}
-
-// Shapes the word-aligned layout does not fit (its padded hyperplanes above
-// shared memory, codes not filling whole words, tiles straddling units) take
-// the bit-stream variant below: P = sort_bits + L race_bits packed columns,
-// each complete code cut out of a running bit stream.
-struct StreamShape {
-  int P, P16, nbuf;
-  uint32_t r_bytes, a_bytes, code_bytes, dyn;
-};
-
-StreamShape stream_shape(const Geometry& g) {
-  StreamShape h;
-  h.P = g.sort_bits + g.L * g.kr;
-  h.P16 = (h.P + 15) / 16 * 16;
-  h.r_bytes = (uint32_t)h.P16 * g.d * 2;
-  h.a_bytes = (uint32_t)kTile * g.d * 2;
-  // per-tile staging of the codes: 128 sort codes (u16) then 128 rows of L RACE codes
-  h.code_bytes = (uint32_t)((kTile * 2 + kTile * g.L * g.rcode_bytes + 15) / 16 * 16);
-  h.nbuf = (h.r_bytes + 2 * h.a_bytes + h.code_bytes + 64 <= (uint32_t)kSmemLimit) ? 2 : 1;
-  h.dyn = h.r_bytes + h.nbuf * h.a_bytes + h.code_bytes + 64;
-  return h;
-}
-
-template <int D>
-ELSAA_DEV void load_tile(uint32_t dst, const __nv_bfloat16* q, const __nv_bfloat16* k,
-                         int64_t rows_per_tensor, int64_t tile) {
-  constexpr int kChunks = D / 8;
-  const int64_t total = 2 * rows_per_tensor;
-  for (int i = threadIdx.x; i < kTile * kChunks; i += kThreads) {
-    const int row = i / kChunks, ch = i % kChunks;
-    const int64_t grow = tile * kTile + row;
-    const bool valid = grow < total;
-    const int64_t g = valid ? grow : 0;
-    const __nv_bfloat16* src =
-        (g < rows_per_tensor ? q + g * D : k + (g - rows_per_tensor) * D) + ch * 8;
-    cp_async16(dst + (ch >> 3) * (kTile * 128) + sw128_off(row, ch & 7), src, valid ? 16 : 0);
-  }
 }
 
 template <int D, typename CodeT>
@@ -196,7 +161,7 @@ hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       *reinterpret_cast<uint4*>(smem + (ch >> 3) * (P16 * 128) + sw128_off(j, ch & 7)) = val;
     }
   }
-  load_tile<D>(s_a, q, k, rows_per_tensor, blockIdx.x);
+  load_tile<D, kThreads>(s_a, q, k, rows_per_tensor, blockIdx.x);
   cp_async_commit();
   fence_before();
   __syncthreads();
@@ -211,7 +176,7 @@ hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     const uint32_t buf = nbuf == 2 ? (uint32_t)(it & 1) : 0u;
     const int64_t next = tile + gridDim.x;
     if (nbuf == 2 && next < tiles) {
-      load_tile<D>(s_a + (buf ^ 1u) * a_bytes, q, k, rows_per_tensor, next);
+      load_tile<D, kThreads>(s_a + (buf ^ 1u) * a_bytes, q, k, rows_per_tensor, next);
       cp_async_commit();
       asm volatile("cp.async.wait_group 1;" ::: "memory");
     } else {
@@ -304,7 +269,7 @@ hash_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
     }
     if (nbuf == 1 && next < tiles) {
-      load_tile<D>(s_a, q, k, rows_per_tensor, next);
+      load_tile<D, kThreads>(s_a, q, k, rows_per_tensor, next);
       cp_async_commit();
     }
   }
@@ -349,203 +314,6 @@ cudaError_t run(const Geometry& g, const void* q, const void* k, const void* r_s
   return cudaGetLastError();
 }
 
-template <int D, typename CodeT>
-__global__ void __launch_bounds__(kThreads)
-hash_tc_stream_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-               const __nv_bfloat16* __restrict__ r_sort, const __nv_bfloat16* __restrict__ r_race,
-               int64_t rows_per_tensor, int N, int sort_bits, int L, int kr, int P, int P16,
-               int nbuf, uint16_t* __restrict__ code, CodeT* __restrict__ rcode,
-               CodeT* __restrict__ rcode_t, uint32_t* __restrict__ err) {
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const uint32_t sbase = smem_u32(smem);
-  const uint32_t r_bytes = (uint32_t)P16 * D * 2;
-  const uint32_t a_bytes = kTile * D * 2;
-  const uint32_t s_r = sbase, s_a = sbase + r_bytes;
-  // code staging: the tile's sort codes, then its rows of RACE codes, written
-  // to global memory as one contiguous block per tile
-  uint16_t* st_code = reinterpret_cast<uint16_t*>(smem + r_bytes + nbuf * a_bytes);
-  CodeT* st_rcode = reinterpret_cast<CodeT*>(st_code + kTile);
-  const uint32_t code_bytes =
-      (uint32_t)((kTile * 2 + kTile * L * (int)sizeof(CodeT) + 15) / 16 * 16);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + r_bytes + nbuf * a_bytes + code_bytes);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
-  const int tid = threadIdx.x, warp = tid >> 5;
-  if ((sbase & 1023u) != 0) {   // the swizzled tiles need a 1024-byte aligned base
-    if (tid == 0) raise_error(err, ERR_CHECK);
-    return;
-  }
-  const int64_t tiles = (2 * rows_per_tensor + kTile - 1) / kTile;
-  if ((int64_t)blockIdx.x >= tiles) return;
-
-  if (tid == 0) {
-    mbar_init(bar, 1);
-    fence_mbar_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
-  }
-  // resident hyperplanes: rows [0, sort_bits) from r_sort, then L*kr from r_race, zero padding
-  {
-    constexpr int kChunks = D / 8;
-    for (int i = tid; i < P16 * kChunks; i += kThreads) {
-      const int j = i / kChunks, ch = i % kChunks;
-      uint4 val = make_uint4(0, 0, 0, 0);
-      if (j < sort_bits)
-        val = *reinterpret_cast<const uint4*>(r_sort + (size_t)j * D + ch * 8);
-      else if (j < P)
-        val = *reinterpret_cast<const uint4*>(r_race + (size_t)(j - sort_bits) * D + ch * 8);
-      *reinterpret_cast<uint4*>(smem + (ch >> 3) * (P16 * 128) + sw128_off(j, ch & 7)) = val;
-    }
-  }
-  load_tile<D>(s_a, q, k, rows_per_tensor, blockIdx.x);
-  cp_async_commit();
-  fence_before();
-  __syncthreads();
-  fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  const int npass = (P16 + kPass - 1) / kPass;
-  const int nslots = 1 + L;
-  uint32_t phase = 0;
-  bool ok = true;
-  int it = 0;
-  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
-    const uint32_t buf = nbuf == 2 ? (uint32_t)(it & 1) : 0u;
-    const int64_t next = tile + gridDim.x;
-    if (nbuf == 2 && next < tiles) {
-      load_tile<D>(s_a + (buf ^ 1u) * a_bytes, q, k, rows_per_tensor, next);
-      cp_async_commit();
-      asm volatile("cp.async.wait_group 1;" ::: "memory");
-    } else {
-      cp_async_wait_all();
-    }
-    fence_async_smem();
-    __syncthreads();
-    uint64_t acc = 0;
-    int nacc = 0, slot = 0;
-    for (int p = 0; p < npass; ++p) {
-      const int ncol = min(kPass, P16 - p * kPass);
-      if (tid == 0) {
-        fence_after();
-        const uint32_t idesc = idesc_bf16(128, ncol, false, false);
-#pragma unroll
-        for (int s = 0; s < D / 16; ++s) {
-          const uint32_t koff = (s >> 2) * (kTile * 128) + (s & 3) * 32;
-          const uint32_t roff = (s >> 2) * (P16 * 128) + p * kPass * 128 + (s & 3) * 32;
-          mma_bf16_ss(tmem, sw128_desc(s_a + buf * a_bytes + koff, 16, 1024),
-                      sw128_desc(s_r + roff, 16, 1024), idesc, s > 0);
-        }
-        mma_commit(bar);
-      }
-      ok = mbar_wait(bar, phase & 1, err);
-      ++phase;
-      if (__syncthreads_or(!ok)) {  // every thread leaves with ok false
-        ok = false;
-        break;
-      }
-      fence_after();
-      for (int c0 = 0; c0 < ncol; c0 += 32) {
-        const int valid = min(32, P - (p * kPass + c0));
-        float v[32];
-        tmem_ld32(tmem + lane_off + c0, v);
-        tmem_ld_wait();
-        if (valid <= 0) continue;
-        uint32_t m = 0;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) m |= (v[i] > 0.f ? 1u : 0u) << i;
-        if (valid < 32) m &= (1u << valid) - 1u;
-        acc |= (uint64_t)m << nacc;
-        nacc += valid;
-        while (slot < nslots) {
-          const int bits = slot == 0 ? sort_bits : kr;
-          if (nacc < bits) break;
-          const uint32_t val = (uint32_t)(acc & ((1ull << bits) - 1ull));
-          acc >>= bits;
-          nacc -= bits;
-          if (slot == 0) st_code[tid] = (uint16_t)val;
-          else st_rcode[tid * L + slot - 1] = (CodeT)val;
-          ++slot;
-        }
-      }
-      fence_before();
-      __syncthreads();
-    }
-    if (!ok) break;
-    // zero-bit codes at the end of the stream
-    while (slot < nslots) {
-      if (slot == 0) st_code[tid] = 0;
-      else st_rcode[tid * L + slot - 1] = 0;
-      ++slot;
-    }
-    __syncthreads();
-    {
-      // the tile's rows are consecutive: copy its codes as contiguous blocks
-      const int64_t row0 = tile * kTile;
-      const int nrows = (int)min((int64_t)kTile, 2 * rows_per_tensor - row0);
-      const int rbytes = nrows * L * (int)sizeof(CodeT);
-      uint8_t* gdst = reinterpret_cast<uint8_t*>(rcode + row0 * L);
-      const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(st_rcode);
-      const int nvec = rbytes / 16;
-      for (int i = tid; i < nvec; i += kThreads)
-        reinterpret_cast<uint4*>(gdst)[i] = reinterpret_cast<const uint4*>(ssrc)[i];
-      for (int i = nvec * 16 + tid; i < rbytes; i += kThreads) gdst[i] = ssrc[i];
-      for (int i = tid; i < nrows; i += kThreads) code[row0 + i] = st_code[i];
-      // table-major copy: thread r writes its row's code of every table;
-      // consecutive rows of a unit are consecutive along N
-      if (tid < nrows) {
-        const int64_t gr = row0 + tid;
-        const int64_t u = gr / N;
-        CodeT* dst = rcode_t + (size_t)u * L * N + (gr - u * N);
-        for (int t = 0; t < L; ++t) dst[(size_t)t * N] = st_rcode[tid * L + t];
-      }
-    }
-    if (nbuf == 1 && next < tiles) {
-      load_tile<D>(s_a, q, k, rows_per_tensor, next);
-      cp_async_commit();
-    }
-  }
-  cp_async_wait_all();
-  fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    fence_after();
-    tmem_dealloc(tmem, kTmemCols);
-  }
-}
-
-template <int D, typename CodeT>
-cudaError_t run_stream(const Geometry& g, const void* q, const void* k, const void* r_sort,
-                const void* r_race, uint16_t* code, void* rcode, void* rcode_t, uint32_t* err,
-                cudaStream_t s) {
-  const StreamShape h = stream_shape(g);
-  cudaError_t e = cudaFuncSetAttribute(hash_tc_stream_kernel<D, CodeT>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)h.dyn);
-  if (e != cudaSuccess) return e;
-  // let shared memory take the whole carveout so several CTAs fit per SM
-  e = cudaFuncSetAttribute(hash_tc_stream_kernel<D, CodeT>,
-                           cudaFuncAttributePreferredSharedMemoryCarveout,
-                           cudaSharedmemCarveoutMaxShared);
-  if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // CTAs per SM: shared memory (228 KB per SM, 1 KB reserved per CTA) and
-  // TMEM (4 x 128 columns)
-  int per_sm = (int)((228u * 1024u) / (h.dyn + 1024u));
-  per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
-  const int64_t rows = (int64_t)g.BH * g.N;
-  const int64_t tiles = (2 * rows + kTile - 1) / kTile;
-  const int64_t want = (int64_t)sms * per_sm;
-  const int grid = (int)(tiles < want ? tiles : want);
-  hash_tc_stream_kernel<D, CodeT><<<grid, kThreads, h.dyn, s>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-      static_cast<const __nv_bfloat16*>(r_sort), static_cast<const __nv_bfloat16*>(r_race), rows,
-      g.N, g.sort_bits, g.L, g.kr, h.P, h.P16, h.nbuf, code, static_cast<CodeT*>(rcode),
-      static_cast<CodeT*>(rcode_t), err);
-  return cudaGetLastError();
-}
-
 bool aligned_layout_fits(const Geometry& g, bool gates, int rounds = 1) {
   // codes fill whole 32-bit words per row; 128-row tiles never straddle units
   if ((g.L * g.rcode_bytes) % 4 != 0 || g.N % kTile != 0 || g.sort_bits > 16) return false;
@@ -560,9 +328,7 @@ bool hash_tc_gate_logits_supported(const Geometry& g) {
 
 bool hash_tc_supported(const Geometry& g) {
   if (!g.bf16 || (g.d != 64 && g.d != 128)) return false;
-  if (aligned_layout_fits(g, false)) return true;
-  const StreamShape h = stream_shape(g);
-  return h.P > 0 && h.dyn <= (uint32_t)kSmemLimit;
+  return aligned_layout_fits(g, false) || hash_tc_stream_fits(g);
 }
 
 bool hash_tc_rounds_supported(const Geometry& g, bool gates) {
@@ -578,7 +344,7 @@ cudaError_t launch_hash_tc(const Geometry& g, const void* q, const void* k, cons
   const bool al = aligned_layout_fits(g, gl != nullptr, rounds);
 #define ELSAA_HASH(DD, CT)                                                                    \
   (al ? run<DD, CT>(g, q, k, r_sort, r_race, code, rcode, rcode_t, gate_w, gl, rounds, err, s) \
-      : run_stream<DD, CT>(g, q, k, r_sort, r_race, code, rcode, rcode_t, err, s))
+      : launch_hash_tc_stream(g, q, k, r_sort, r_race, code, rcode, rcode_t, err, s))
   if (g.d == 64) return g.rcode_bytes == 1 ? ELSAA_HASH(64, uint8_t) : ELSAA_HASH(64, uint16_t);
   return g.rcode_bytes == 1 ? ELSAA_HASH(128, uint8_t) : ELSAA_HASH(128, uint16_t);
 #undef ELSAA_HASH

@@ -95,6 +95,13 @@ cudaError_t launch_hash_tc(const Geometry& g, const void* q, const void* k, cons
 // The GEMM also gives the sort codes of hash rounds 1 .. R - 1 (rounds = R in
 // launch_hash_tc; code then holds [R][2][BH][N]).
 bool hash_tc_rounds_supported(const Geometry& g, bool gates);
+// The bit-stream variant of the tcgen05 hash (hash_tc_stream.cu) for shapes
+// whose codes do not fill whole words or whose word-aligned hyperplanes do not
+// fit shared memory; launch_hash_tc chooses it.
+bool hash_tc_stream_fits(const Geometry& g);
+cudaError_t launch_hash_tc_stream(const Geometry& g, const void* q, const void* k,
+                                  const void* r_sort, const void* r_race, uint16_t* code,
+                                  void* rcode, void* rcode_t, uint32_t* err, cudaStream_t s);
 bool hash_tc_supported(const Geometry& g);
 bool hash_tc_gate_logits_supported(const Geometry& g);
 
