@@ -127,7 +127,7 @@ def stage_roofline(flops, nbytes, sec, peaks):
 TRAFFIC_WORKLOAD, TRAFFIC_UNITS = "text-32k", 12
 RECORDED_TRAFFIC = {
     # stage: (kernel source, its sha1 at capture, bytes per 12-unit launch, path flag needed)
-    "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "0f6d6d0fa080567b642065af04df9b3345737c4f", 1.2331e+08, "tc_hash"),
+    "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "edcbdc68deae50db48e82ecf8d702c46c0678843", 1.2346e+08, "tc_hash"),
     "race_build": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "15a1fb45c20eb380372ec944794c10506c62861f", 6.874e+07, None),
     "sparse_fwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_pipe.cu", "b33f474224da484dfb1f6128dd2527644c56625a", 1.8644e+08, "tc_attn"),
     "race_fuse": ("sparse_rank_hybrid_simhash_b200/csrc/race_slab.cu", "5135a962ed6cf3d305d45cb27ffcdf41815cc38e", 1.4487e+08, "slab_fwd"),
