@@ -48,6 +48,24 @@ def test_needle_small_forward(cuda_device):
     _run(w, backward=False)
 
 
+@pytest.mark.parametrize("d,N,L,kr,sort_bits,chunk", [
+    (64, 960, 12, 5, 6, 64),      # N not a multiple of 128: tiles straddle units
+    (128, 640, 5, 9, 11, 128),    # 16-bit codes, 10 bytes of codes per row
+    (64, 1024, 3, 13, 1, 64),     # 16-bit codes, 6 bytes per row, 8192 buckets
+    (128, 1088, 20, 7, 8, 64),    # two passes (148 columns), ragged N
+    (64, 512, 3, 0, 5, 64),       # no RACE bits (one bucket): sort codes only
+    (64, 576, 6, 4, 0, 64),       # no sort bits: every code from the RACE columns
+])
+def test_bit_stream_hash_shapes(cuda_device, d, N, L, kr, sort_bits, chunk):
+    # shapes the word-aligned hash layout does not take (row codes not whole
+    # 32-bit words, or N not a multiple of 128): the bit-stream tcgen05 hash,
+    # with codes cut across word boundaries; every code compared
+    w = small(WORKLOADS["iid-4k"], B=2, H=2, N=N).replace(
+        d=d, race_tables=L, race_bits=kr, sort_bits=sort_bits, chunk=chunk, backward=False)
+    assert B.path_flags(B.Params.from_workload(w))["tc_hash"]
+    _run(w, backward=False)
+
+
 @pytest.mark.parametrize("lam,gates", [(0.0, (1.0, 0.0)), (2.0, (0.0, 1.0)), (0.0, (0.3, 0.9))])
 def test_ablation_and_single_branch_modes(cuda_device, lam, gates):
     w = small(WORKLOADS["iid-4k"], B=1, H=2, N=512).replace(
