@@ -873,7 +873,7 @@ constexpr int kSegWarps = kSegThreads / 32;
 constexpr int kSegKeys = 32768;
 
 struct SegSmem {
-  size_t list, codes, whist, bend, misc, total;
+  size_t list, codes, whist, bend, misc, stg, total;
 };
 __host__ __device__ inline SegSmem seg_smem(int seg, int NB, int code_bytes) {
   SegSmem m;
@@ -882,7 +882,8 @@ __host__ __device__ inline SegSmem seg_smem(int seg, int NB, int code_bytes) {
   m.whist = align16(m.codes + (size_t)seg * code_bytes);
   m.bend = align16(m.whist + (size_t)kSegWarps * NB * 4);
   m.misc = align16(m.bend + (size_t)NB * 4);
-  m.total = m.misc + 256;   // [0] C_max, [1] bad code, [16..32) warp sums of the scan
+  m.stg = m.misc + 256;     // misc: [0] C_max, [1] bad code, [16..32) warp sums of the scan
+  m.total = m.stg + (size_t)kSegThreads * 8 * 4;   // a run total per lane group (d ints)
   return m;
 }
 
@@ -1012,7 +1013,12 @@ race_build_seg_kernel(const CodeT* __restrict__ codes_t, const TV* __restrict__ 
   const int p0 = (int)((int64_t)n * gi / groups), p1 = (int)((int64_t)n * (gi + 1) / groups);
   const TV* vb = vals + ((size_t)bh * N + j0) * d + ql * EL;
   // the fp32 table's bytes hold the int32 sums until the finishing pass
-  uint32_t* tb = reinterpret_cast<uint32_t*>(sums + ((size_t)bh * L + t) * NB * d) + ql * EL;
+  uint32_t* tb = reinterpret_cast<uint32_t*>(sums + ((size_t)bh * L + t) * NB * d);
+  // a run total goes through the group's staging row, so that lane ql adds
+  // columns ql, ql + QL, ...: each add instruction of the group covers QL
+  // consecutive columns (two 32-byte sectors at QL = 16, not QL sectors)
+  int32_t* stg = reinterpret_cast<int32_t*>(sm + lay.stg) + gi * d;
+  const unsigned gmask = QL == 32 ? 0xffffffffu : ((1u << QL) - 1u) << (lane & ~(QL - 1));
   float acc[EL];
 #pragma unroll
   for (int e = 0; e < EL; ++e) acc[e] = 0.f;
@@ -1030,12 +1036,16 @@ race_build_seg_kernel(const CodeT* __restrict__ codes_t, const TV* __restrict__ 
   bool any = false;
   auto flush = [&]() {
     if (any) {
-      uint32_t* dst = tb + (size_t)b * d;
 #pragma unroll
       for (int e = 0; e < EL; ++e) {
-        atomicAdd(dst + e, (uint32_t)__float2int_rn(acc[e] * scale));
+        stg[ql * EL + e] = __float2int_rn(acc[e] * scale);
         acc[e] = 0.f;
       }
+      __syncwarp(gmask);
+      uint32_t* dst = tb + (size_t)b * d + ql;
+#pragma unroll
+      for (int e = 0; e < EL; ++e) atomicAdd(dst + e * QL, (uint32_t)stg[e * QL + ql]);
+      __syncwarp(gmask);   // the row is read before the group's next flush writes it
     }
     any = false;
   };
