@@ -934,8 +934,10 @@ race_build_seg_kernel(const CodeT* __restrict__ codes_t, const TV* __restrict__ 
   int32_t* misc = reinterpret_cast<int32_t*>(sm + lay.misc);        // [0] C_max, [1] bad code
   int32_t* wsum = misc + 16;                                        // [kSegWarps] scan sums
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int t = blockIdx.y, bh = blockIdx.z;
-  const int j0 = blockIdx.x * seg, n = min(N, j0 + seg) - j0;   // keys [j0, j0 + n)
+  // grid (table, segment, unit): the CTAs that run together share a few
+  // segments of the unit's value rows, which stay in L2 for all tables
+  const int t = blockIdx.x, bh = blockIdx.z;
+  const int j0 = blockIdx.y * seg, n = min(N, j0 + seg) - j0;   // keys [j0, j0 + n)
   const CodeT* ct = codes_t + ((size_t)bh * L + t) * N + j0;
   // warp w owns segment keys [k0, k1)
   const int k0 = (int)((int64_t)n * warp / kSegWarps);
@@ -1411,7 +1413,8 @@ cudaError_t build(const Geometry& g, const void* codes, const void* codes_t, con
       auto kernel = race_build_seg_kernel<TV, CodeT>;
       e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)m.total);
       if (e != cudaSuccess) return e;
-      kernel<<<grid, kSegThreads, m.total, s>>>(static_cast<const CodeT*>(codes_t),
+      const dim3 bgrid(g.L, (g.N + seg - 1) / seg, g.BH);
+      kernel<<<bgrid, kSegThreads, m.total, s>>>(static_cast<const CodeT*>(codes_t),
                                                 static_cast<const TV*>(vals), g.N, g.L, g.NB, g.d,
                                                 seg, absmax, cnt, sums, err);
       race_seg_finish_kernel<<<dim3(g.L, g.BH), 256, 0, s>>>(sums, gtab, cnt, absmax, g.L, g.NB,
