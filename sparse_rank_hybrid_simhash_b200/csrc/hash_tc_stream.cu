@@ -24,8 +24,20 @@ using hash::load_tile;
 // the bit-stream variant below: P = sort_bits + L race_bits packed columns.
 // Every row's P sign bits are staged as a bit array of SW words, and each code
 // is cut out of it where it is written.
-constexpr int kStreamThreads = 512;    // 16 warps: 4 lane quarters x 4 column words
+constexpr int kStreamThreads = 512;    // 8 reader warps, then 8 writer warps
+constexpr int kReaders = 256;
+constexpr int kReaderWarps = kReaders / 32;
 constexpr uint32_t kStreamTmemCols = 256;   // two 128-column pass buffers
+// named barriers (0 is __syncthreads): the readers' own, then per bit array
+// "full" (readers arrive, writers wait) and "empty" (writers arrive, readers wait)
+constexpr int kBarRead = 1, kBarFull = 2, kBarEmpty = 4;
+
+ELSAA_DEV void nbar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+ELSAA_DEV void nbar_arrive(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 
 struct StreamShape {
   int P, P16, SW, nbuf;
@@ -41,20 +53,22 @@ StreamShape stream_shape(const Geometry& g) {
   h.SW = ((h.P16 + 31) / 32 + 1) | 1;
   h.r_bytes = (uint32_t)h.P16 * g.d * 2;
   h.a_bytes = (uint32_t)kTile * g.d * 2;
-  h.code_bytes = (uint32_t)((kTile * h.SW * 4 + 15) / 16 * 16);
+  h.code_bytes = (uint32_t)((2 * kTile * h.SW * 4 + 15) / 16 * 16);   // two tiles' bit arrays
   h.nbuf = (h.r_bytes + 2 * h.a_bytes + h.code_bytes + 64 <= (uint32_t)kSmemLimit) ? 2 : 1;
   h.dyn = h.r_bytes + h.nbuf * h.a_bytes + h.code_bytes + 64;
   return h;
 }
 
-// Per tile: the passes' MMAs alternate between two TMEM buffers, so pass
-// p + 1 computes while pass p is read; warp w reads 32 columns (word w / 4 of
-// the pass) of lane quarter w % 4 and stores the sign mask of each of its 32
-// rows into the bit array; once the last pass's MMA has completed, the next
-// tile's load starts (one A buffer) under the read-out and the code writes.
-// Codes are then cut from the bit array twice: warps over rows for the
-// row-major codes, warps over tables for the table-major ones, so both global
-// writes are coalesced.
+// Roles: warps 0..7 read, warps 8..15 write.  Per tile the readers run the
+// passes, whose MMAs alternate between two TMEM buffers (pass p + 1 computes
+// while pass p is read); reader warp w reads lane quarter w % 4, 32-column
+// words w / 4 and w / 4 + 2 of every pass, and stores each row's sign masks
+// into one of two bit arrays; once the tile's last MMA has completed, the
+// next tile's load starts (one A buffer).  Meanwhile the writers cut the
+// previous tile's codes from the other bit array, twice: warps over rows for
+// the row-major codes, warps over tables for the table-major ones, so both
+// global writes are coalesced.  Named barriers hand each bit array from the
+// readers to the writers ("full") and back ("empty").
 template <int D, typename CodeT>
 __global__ void __launch_bounds__(kStreamThreads, 1)
 hash_tc_stream_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
@@ -67,9 +81,9 @@ hash_tc_stream_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
   const uint32_t r_bytes = (uint32_t)P16 * D * 2;
   const uint32_t a_bytes = kTile * D * 2;
   const uint32_t s_r = sbase, s_a = sbase + r_bytes;
-  // the tile's sign bits: [128 rows][SW words]
+  // two tiles' sign bits: [2][128 rows][SW words]
   uint32_t* st_w = reinterpret_cast<uint32_t*>(smem + r_bytes + nbuf * a_bytes);
-  const uint32_t code_bytes = (uint32_t)((kTile * SW * 4 + 15) / 16 * 16);
+  const uint32_t code_bytes = (uint32_t)((2 * kTile * SW * 4 + 15) / 16 * 16);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + r_bytes + nbuf * a_bytes + code_bytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 2);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -104,98 +118,141 @@ hash_tc_stream_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
     }
   }
   // words no pass writes stay zero (the window of the last code reads one)
-  for (int i = tid; i < kTile * SW; i += kStreamThreads) st_w[i] = 0u;
-  load_tile<D, kStreamThreads>(s_a, q, k, rows_per_tensor, blockIdx.x);
-  cp_async_commit();
+  for (int i = tid; i < 2 * kTile * SW; i += kStreamThreads) st_w[i] = 0u;
+  // s_abort: a reader's wait gave up (read by the readers after their own
+  // barrier); s_done[b]: the readers' verdict on the tile of bit array b,
+  // written before they arrive on its "full" barrier, so every writer reads
+  // the same value
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* s_done = s_abort + 1;
+  if (tid == 0) *s_abort = 0;
+  if (tid < kReaders) {
+    load_tile<D, kReaders>(s_a, q, k, rows_per_tensor, blockIdx.x);
+    cp_async_commit();
+  }
   fence_before();
   __syncthreads();
   fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int quarter = warp & 3, word = warp >> 2;
-  const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
   const int npass = (P16 + kPass - 1) / kPass;
-  const int srow = quarter * 32 + lane;   // the row this thread reads out
-  uint32_t ph = 0u;   // bit b: the phase parity of barrier b
-  bool ok = true;
-  int it = 0;
-  // bits [o, o + n) of row r's bit array, n <= 16
-  auto cut = [&](int r, int o, int n) -> uint32_t {
-    const uint32_t* row = st_w + r * SW + (o >> 5);
-    return __funnelshift_r(row[0], row[1], o & 31) & ((1u << n) - 1u);
-  };
-  auto issue = [&](int p, uint32_t abuf) {   // one thread: pass p into TMEM buffer p & 1
-    fence_after();
-    const int ncol = min(kPass, P16 - p * kPass);
-    const uint32_t idesc = idesc_bf16(128, ncol, false, false);
+  // this CTA's tiles: blockIdx.x, blockIdx.x + gridDim.x, ...
+  const int n_my = (int)((tiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
+  if (warp < kReaderWarps) {
+    // ------------------------------------------------------------ readers
+    // warp w reads lane quarter w % 4, words w / 4 and w / 4 + 2 of every pass
+    const int quarter = warp & 3, wsel = warp >> 2;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const int srow = quarter * 32 + lane;   // the row this thread reads out
+    uint32_t ph = 0u;   // bit b: the phase parity of mbarrier b
+    auto issue = [&](int p, uint32_t abuf) {   // one thread: pass p into TMEM buffer p & 1
+      fence_after();
+      const int ncol = min(kPass, P16 - p * kPass);
+      const uint32_t idesc = idesc_bf16(128, ncol, false, false);
 #pragma unroll
-    for (int s = 0; s < D / 16; ++s) {
-      const uint32_t koff = (s >> 2) * (kTile * 128) + (s & 3) * 32;
-      const uint32_t roff = (s >> 2) * (P16 * 128) + p * kPass * 128 + (s & 3) * 32;
-      mma_bf16_ss(tmem + (uint32_t)(p & 1) * kPass, sw128_desc(s_a + abuf + koff, 16, 1024),
-                  sw128_desc(s_r + roff, 16, 1024), idesc, s > 0);
-    }
-    mma_commit(bar + (p & 1));
-  };
-  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
-    const uint32_t abuf = nbuf == 2 ? (uint32_t)(it & 1) * a_bytes : 0u;
-    const int64_t next = tile + gridDim.x;
-    if (nbuf == 2 && next < tiles) {
-      load_tile<D, kStreamThreads>(s_a + (a_bytes - abuf), q, k, rows_per_tensor, next);
-      cp_async_commit();
-      asm volatile("cp.async.wait_group 1;" ::: "memory");
-    } else {
-      cp_async_wait_all();
-    }
-    fence_async_smem();
-    __syncthreads();
-    if (tid == 0) issue(0, abuf);
-    for (int p = 0; p < npass; ++p) {
-      // pass p + 1 goes into the other buffer, whose last read-out ended
-      // before the barrier that closed the previous pass
-      if (tid == 0 && p + 1 < npass) issue(p + 1, abuf);
-      const int b = p & 1;
-      ok = mbar_wait(bar + b, (ph >> b) & 1u, err);
-      ph ^= 1u << b;
-      if (__syncthreads_or(!ok)) {  // every thread leaves with ok false
-        ok = false;
+      for (int s = 0; s < D / 16; ++s) {
+        const uint32_t koff = (s >> 2) * (kTile * 128) + (s & 3) * 32;
+        const uint32_t roff = (s >> 2) * (P16 * 128) + p * kPass * 128 + (s & 3) * 32;
+        mma_bf16_ss(tmem + (uint32_t)(p & 1) * kPass, sw128_desc(s_a + abuf + koff, 16, 1024),
+                    sw128_desc(s_r + roff, 16, 1024), idesc, s > 0);
+      }
+      mma_commit(bar + (p & 1));
+    };
+    int it = 0;
+    for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
+      const int sb = it & 1;
+      uint32_t* bits = st_w + sb * kTile * SW;
+      const uint32_t abuf = nbuf == 2 ? (uint32_t)sb * a_bytes : 0u;
+      const int64_t next = tile + gridDim.x;
+      // the writers are done with this bit array (tile it - 2)
+      if (it >= 2) nbar_sync(kBarEmpty + sb, kStreamThreads);
+      if (nbuf == 2 && next < tiles) {
+        load_tile<D, kReaders>(s_a + (a_bytes - abuf), q, k, rows_per_tensor, next);
+        cp_async_commit();
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+      } else {
+        cp_async_wait_all();
+      }
+      fence_async_smem();
+      nbar_sync(kBarRead, kReaders);
+      if (tid == 0) issue(0, abuf);
+      bool ok = true;
+      for (int p = 0; p < npass; ++p) {
+        // pass p + 1 goes into the other TMEM buffer, whose last read-out
+        // ended before the barrier that closed the previous pass
+        if (tid == 0 && p + 1 < npass) issue(p + 1, abuf);
+        const int b = p & 1;
+        if (warp == 0 && !mbar_wait(bar + b, (ph >> b) & 1u, err)) *s_abort = 1;
+        ph ^= 1u << b;
+        nbar_sync(kBarRead, kReaders);
+        if (*s_abort) {   // every reader sees the same flag after the barrier
+          ok = false;
+          break;
+        }
+        fence_after();
+        if (p + 1 == npass && nbuf == 1 && next < tiles) {
+          // every MMA of the tile has completed: its A buffer takes the next tile
+          load_tile<D, kReaders>(s_a, q, k, rows_per_tensor, next);
+          cp_async_commit();
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int wd = wsel + 2 * h;
+          const int c0 = p * kPass + wd * 32;
+          if (c0 < P16) {   // uniform over the warp
+            float v[32];
+            tmem_ld32(tmem + lane_off + (uint32_t)b * kPass + wd * 32, v);
+            tmem_ld_wait();
+            const int valid = min(32, P - c0);
+            uint32_t m4[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int i = 0; i < 32; ++i) m4[i & 3] |= (v[i] > 0.f ? 1u : 0u) << i;
+            uint32_t m = (m4[0] | m4[1]) | (m4[2] | m4[3]);
+            if (valid <= 0) m = 0u;
+            else if (valid < 32) m &= (1u << valid) - 1u;
+            bits[srow * SW + (c0 >> 5)] = m;
+          }
+        }
+        fence_before();
+        nbar_sync(kBarRead, kReaders);
+      }
+      // this tile's bits (or the abort) go to the writers
+      if (tid == 0) s_done[sb] = ok ? 1 : 0;
+      nbar_arrive(kBarFull + sb, kStreamThreads);
+      if (!ok) {
+        // take the writers' release of the other bit array (tile it - 1), so
+        // that no barrier is left half-arrived
+        if (it >= 1 && it + 1 < n_my) nbar_sync(kBarEmpty + (sb ^ 1), kStreamThreads);
         break;
       }
-      fence_after();
-      if (p + 1 == npass && nbuf == 1 && next < tiles) {
-        // every MMA of the tile has completed: its A buffer takes the next tile
-        load_tile<D, kStreamThreads>(s_a, q, k, rows_per_tensor, next);
-        cp_async_commit();
-      }
-      const int c0 = p * kPass + word * 32;
-      if (c0 < P16) {   // uniform over the warp
-        float v[32];
-        tmem_ld32(tmem + lane_off + (uint32_t)b * kPass + word * 32, v);
-        tmem_ld_wait();
-        const int valid = min(32, P - c0);
-        uint32_t m4[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-        for (int i = 0; i < 32; ++i) m4[i & 3] |= (v[i] > 0.f ? 1u : 0u) << i;
-        uint32_t m = (m4[0] | m4[1]) | (m4[2] | m4[3]);
-        if (valid <= 0) m = 0u;
-        else if (valid < 32) m &= (1u << valid) - 1u;
-        st_w[srow * SW + (c0 >> 5)] = m;
-      }
-      fence_before();
-      __syncthreads();
     }
-    if (!ok) break;
-    {
+  } else {
+    // ------------------------------------------------------------ writers
+    // codes cut from the bit array of the previous tile while the readers
+    // run the next one: warps over rows for the row-major codes, warps over
+    // tables for the table-major ones, so both global writes are coalesced
+    const int ww = warp - kReaderWarps, wt = tid - kReaders;
+    constexpr int kWriterWarps = (kStreamThreads - kReaders) / 32;
+    int it = 0;
+    for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
+      const int sb = it & 1;
+      const uint32_t* bits = st_w + sb * kTile * SW;
+      nbar_sync(kBarFull + sb, kStreamThreads);
+      if (s_done[sb] == 0) break;   // the readers gave up on this tile
+      // bits [o, o + n) of row r, n <= 16
+      auto cut = [&](int r, int o, int n) -> uint32_t {
+        const uint32_t* row = bits + r * SW + (o >> 5);
+        return __funnelshift_r(row[0], row[1], o & 31) & ((1u << n) - 1u);
+      };
       const int64_t row0 = tile * kTile;
       const int nrows = (int)min((int64_t)kTile, total - row0);
-      for (int r = tid; r < nrows; r += kStreamThreads)
+      for (int r = wt; r < nrows; r += kStreamThreads - kReaders)
         code[row0 + r] = (uint16_t)cut(r, 0, sort_bits);
-      // row-major codes: a warp per row, lanes over tables
-      for (int r = warp; r < nrows; r += kStreamThreads / 32) {
+      for (int r = ww; r < nrows; r += kWriterWarps) {
         CodeT* dst = rcode + (row0 + r) * L;
         for (int t = lane; t < L; t += 32) dst[t] = (CodeT)cut(r, sort_bits + t * kr, kr);
       }
-      // table-major codes: a warp per table, lanes over rows (consecutive
-      // rows of a unit are consecutive along N)
+      // unit and position of each of the lane's rows (the tile's rows are
+      // consecutive; consecutive rows of a unit are consecutive along N)
       int64_t off[kTile / 32];
 #pragma unroll
       for (int j = 0; j < kTile / 32; ++j) {
@@ -203,15 +260,17 @@ hash_tc_stream_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
         const int64_t u = gr / N;
         off[j] = u * L * N + (gr - u * N);
       }
-      for (int t = warp; t < L; t += kStreamThreads / 32) {
+      for (int t = ww; t < L; t += kWriterWarps) {
 #pragma unroll
         for (int j = 0; j < kTile / 32; ++j) {
           const int r = lane + 32 * j;
           if (r < nrows) rcode_t[off[j] + (int64_t)t * N] = (CodeT)cut(r, sort_bits + t * kr, kr);
         }
       }
+      // the readers may overwrite this bit array for tile it + 2 (no arrival
+      // when there is no such tile, so no barrier is left half-arrived)
+      if (it + 2 < n_my) nbar_arrive(kBarEmpty + sb, kStreamThreads);
     }
-    __syncthreads();   // the bit array is read before the next tile's passes write it
   }
   cp_async_wait_all();
   fence_before();
