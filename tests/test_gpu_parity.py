@@ -66,6 +66,18 @@ def test_bit_stream_hash_shapes(cuda_device, d, N, L, kr, sort_bits, chunk):
     _run(w, backward=False)
 
 
+def test_bit_stream_hash_many_tiles_per_cta(cuda_device):
+    # 2056 tiles of 128 rows: every CTA of the bit-stream hash takes several,
+    # so both bit arrays and both handovers between its readers and writers
+    # are used; N is not a multiple of 128, so tiles straddle units
+    w = small(WORKLOADS["iid-4k"], B=2, H=4, N=16448).replace(
+        race_tables=12, race_bits=5, sort_bits=6, chunk=64, backward=False)
+    inp = make_inputs(w, with_dy=False)
+    gpu = run_gpu(w, inp, backward=False)
+    for b, h in [(0, 0), (1, 3)]:
+        check_unit(w, inp, gpu, b, h, False, {})
+
+
 @pytest.mark.parametrize("lam,gates", [(0.0, (1.0, 0.0)), (2.0, (0.0, 1.0)), (0.0, (0.3, 0.9))])
 def test_ablation_and_single_branch_modes(cuda_device, lam, gates):
     w = small(WORKLOADS["iid-4k"], B=1, H=2, N=512).replace(
