@@ -868,22 +868,28 @@ race_build_sorted_kernel(const CodeT* __restrict__ codes_t, const TV* __restrict
 // are exact and order-independent, so the table is the same on every run.  A
 // last pass turns each table into fp32 (and the bf16 copy) in place.
 
-constexpr int kSegThreads = 512;
+constexpr int kSegThreads = 1024;
 constexpr int kSegWarps = kSegThreads / 32;
 constexpr int kSegKeys = 32768;
 
+// whist: [warps][NB] 16-bit counts, then cursors, two to a 32-bit word (a
+// warp counts at most seg / warps keys of a bucket and a cursor is at most
+// seg <= 32768, so neither half ever carries into the other); after the
+// scatter the same bytes hold the lane groups' run totals (stg: d ints per
+// group).  The codes are read from global memory where they are counted and
+// scattered.
 struct SegSmem {
-  size_t list, codes, whist, bend, misc, stg, total;
+  size_t list, whist, stg, bend, misc, total;
 };
-__host__ __device__ inline SegSmem seg_smem(int seg, int NB, int code_bytes) {
+__host__ __device__ inline SegSmem seg_smem(int seg, int NB, int /*code_bytes*/) {
   SegSmem m;
   m.list = 0;
-  m.codes = align16((size_t)seg * 2);
-  m.whist = align16(m.codes + (size_t)seg * code_bytes);
-  m.bend = align16(m.whist + (size_t)kSegWarps * NB * 4);
+  m.whist = align16((size_t)seg * 2);
+  m.stg = m.whist;
+  const size_t hist = (size_t)kSegWarps * NB * 2, runs = (size_t)kSegThreads * 8 * 4;
+  m.bend = align16(m.whist + (hist > runs ? hist : runs));
   m.misc = align16(m.bend + (size_t)NB * 4);
-  m.stg = m.misc + 256;     // misc: [0] C_max, [1] bad code, [16..32) warp sums of the scan
-  m.total = m.stg + (size_t)kSegThreads * 8 * 4;   // a run total per lane group (d ints)
+  m.total = m.misc + 256;   // misc: [0] C_max, [1] bad code, [16..48) warp sums of the scan
   return m;
 }
 
@@ -928,8 +934,8 @@ race_build_seg_kernel(const CodeT* __restrict__ codes_t, const TV* __restrict__ 
   extern __shared__ __align__(16) uint8_t sm[];
   const SegSmem lay = seg_smem(seg, NB, (int)sizeof(CodeT));
   uint16_t* list = reinterpret_cast<uint16_t*>(sm + lay.list);      // segment keys, by bucket
-  CodeT* csm = reinterpret_cast<CodeT*>(sm + lay.codes);            // the segment's codes
-  uint32_t* whist = reinterpret_cast<uint32_t*>(sm + lay.whist);    // [warps][NB]
+  uint16_t* wh16 = reinterpret_cast<uint16_t*>(sm + lay.whist);     // [warps][NB] counts, cursors
+  uint32_t* wh32 = reinterpret_cast<uint32_t*>(sm + lay.whist);     // the same, two to a word
   int32_t* bend = reinterpret_cast<int32_t*>(sm + lay.bend);        // [NB] end of each bucket
   int32_t* misc = reinterpret_cast<int32_t*>(sm + lay.misc);        // [0] C_max, [1] bad code
   int32_t* wsum = misc + 16;                                        // [kSegWarps] scan sums
@@ -942,9 +948,8 @@ race_build_seg_kernel(const CodeT* __restrict__ codes_t, const TV* __restrict__ 
   // warp w owns segment keys [k0, k1)
   const int k0 = (int)((int64_t)n * warp / kSegWarps);
   const int k1 = (int)((int64_t)n * (warp + 1) / kSegWarps);
-  uint32_t* wh = whist + (size_t)warp * NB;
-  for (int i = tid; i < n; i += kSegThreads) csm[i] = ct[i];
-  for (int i = tid; i < kSegWarps * NB; i += kSegThreads) whist[i] = 0;
+  const int fw = warp * NB;   // this warp's counters: flat 16-bit index fw + bucket
+  for (int i = tid; i < (kSegWarps * NB + 1) / 2; i += kSegThreads) wh32[i] = 0;
   if (tid < 2) misc[tid] = 0;
   __syncthreads();
   // the table's largest bucket count (all segments), for the grid 2^-S
@@ -957,9 +962,13 @@ race_build_seg_kernel(const CodeT* __restrict__ codes_t, const TV* __restrict__ 
     if (lane == 0) atomicMax(misc, cm);
   }
   for (int j = k0 + lane; j < k1; j += 32) {
-    const int c = (int)csm[j];
-    if (c < NB) atomicAdd(wh + c, 1u);
-    else misc[1] = 1;
+    const int c = (int)ct[j];
+    if (c < NB) {
+      const int f = fw + c;
+      atomicAdd(wh32 + (f >> 1), 1u << (16 * (f & 1)));
+    } else {
+      misc[1] = 1;
+    }
   }
   __syncthreads();
   if (misc[1] != 0) {
@@ -973,7 +982,7 @@ race_build_seg_kernel(const CodeT* __restrict__ codes_t, const TV* __restrict__ 
     const int b = b0 + tid;
     int c = 0;
     if (b < NB)
-      for (int w = 0; w < kSegWarps; ++w) c += (int)whist[w * NB + b];
+      for (int w = 0; w < kSegWarps; ++w) c += (int)wh16[w * NB + b];
     int x = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -990,8 +999,8 @@ race_build_seg_kernel(const CodeT* __restrict__ codes_t, const TV* __restrict__ 
       uint32_t run = (uint32_t)(before + x - c);
       bend[b] = before + x;
       for (int w = 0; w < kSegWarps; ++w) {
-        const uint32_t h = whist[w * NB + b];
-        whist[w * NB + b] = run;
+        const uint32_t h = wh16[w * NB + b];
+        wh16[w * NB + b] = (uint16_t)run;
         run += h;
       }
     }
@@ -999,7 +1008,11 @@ race_build_seg_kernel(const CodeT* __restrict__ codes_t, const TV* __restrict__ 
     __syncthreads();
   }
   // scatter through the warp-private cursors
-  for (int j = k0 + lane; j < k1; j += 32) list[atomicAdd(wh + (int)csm[j], 1u)] = (uint16_t)j;
+  for (int j = k0 + lane; j < k1; j += 32) {
+    const int f = fw + (int)ct[j];
+    const uint32_t sh = 16u * (uint32_t)(f & 1);
+    list[(atomicAdd(wh32 + (f >> 1), 1u << sh) >> sh) & 0xFFFFu] = (uint16_t)j;
+  }
   const float vmax = absmax[bh];
   if (!(vmax < 3.0e38f)) {
     if (tid == 0) raise_error(err, ERR_CHECK);
