@@ -128,11 +128,11 @@ TRAFFIC_WORKLOAD, TRAFFIC_UNITS = "text-32k", 12
 RECORDED_TRAFFIC = {
     # stage: (kernel source, its sha1 at capture, bytes per 12-unit launch, path flag needed)
     "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "edcbdc68deae50db48e82ecf8d702c46c0678843", 1.2346e+08, "tc_hash"),
-    "race_build": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "cc5a64014700549217ed7c347f70d313512d6e7e", 6.9105e+07, None),
+    "race_build": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "ae4cba186ff862dc49a580bdd3aa2d9afe804f41", 6.8706e+07, None),
     "sparse_fwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_pipe.cu", "b33f474224da484dfb1f6128dd2527644c56625a", 1.8644e+08, "tc_attn"),
     "race_fuse": ("sparse_rank_hybrid_simhash_b200/csrc/race_slab.cu", "5135a962ed6cf3d305d45cb27ffcdf41815cc38e", 1.4487e+08, "slab_fwd"),
     "fuse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/fuse_bwd.cu", "d225c68863731ac35a2126d849af1623d8c512c7", 2.8098e+08, None),
-    "race_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "cc5a64014700549217ed7c347f70d313512d6e7e", 6.6224e+07, None),
+    "race_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "ae4cba186ff862dc49a580bdd3aa2d9afe804f41", 6.6587e+07, None),
     "sparse_bwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_bwd3.cu", "ffbd2e8b9a9bb8a1a16dfa244ec836a1dc90ccdc", 3.3276e+08, "tc_attn"),
     "finish": ("sparse_rank_hybrid_simhash_b200/csrc/race_slab.cu", "5135a962ed6cf3d305d45cb27ffcdf41815cc38e", 7.874e+07, "slab_bwd"),
 }
