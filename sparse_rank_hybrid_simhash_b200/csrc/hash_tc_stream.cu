@@ -120,7 +120,7 @@ hash_tc_stream_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
   // words no pass writes stay zero (the window of the last code reads one)
   for (int i = tid; i < 2 * kTile * SW; i += kStreamThreads) st_w[i] = 0u;
   // s_abort: a reader's wait gave up (read by the readers after their own
-  // barrier); s_done[b]: the readers' verdict on the tile of bit array b,
+  // barrier); s_done[b]: the readers' outcome for the tile of bit array b,
   // written before they arrive on its "full" barrier, so every writer reads
   // the same value
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
