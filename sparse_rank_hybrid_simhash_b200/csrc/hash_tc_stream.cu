@@ -40,14 +40,18 @@ ELSAA_DEV void nbar_arrive(int id, int n) {
 }
 
 struct StreamShape {
-  int P, P16, SW, nbuf;
+  int P, gcol, P16, SW, nbuf;
   uint32_t r_bytes, a_bytes, code_bytes, dyn;
 };
 
-StreamShape stream_shape(const Geometry& g) {
+// With learned gates, four more columns (w_s and w_r, each as a bf16 high
+// part and the bf16 remainder: their fp32 sums are w . q to about 16
+// significant bits) start at the first 32-column word after the codes, gcol.
+StreamShape stream_shape(const Geometry& g, bool gates) {
   StreamShape h;
   h.P = g.sort_bits + g.L * g.kr;
-  h.P16 = (h.P + 15) / 16 * 16;
+  h.gcol = gates ? (h.P + 31) / 32 * 32 : -1;
+  h.P16 = ((gates ? h.gcol + 4 : h.P) + 15) / 16 * 16;
   // words of 32 sign bits per row (whole 32-column reads) plus one zero word,
   // so every code's two-word window exists; odd, so rows fall on distinct banks
   h.SW = ((h.P16 + 31) / 32 + 1) | 1;
@@ -73,9 +77,10 @@ template <int D, typename CodeT>
 __global__ void __launch_bounds__(kStreamThreads, 1)
 hash_tc_stream_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                const __nv_bfloat16* __restrict__ r_sort, const __nv_bfloat16* __restrict__ r_race,
-               int64_t rows_per_tensor, int N, int sort_bits, int L, int kr, int P, int P16,
-               int SW, int nbuf, uint16_t* __restrict__ code, CodeT* __restrict__ rcode,
-               CodeT* __restrict__ rcode_t, uint32_t* __restrict__ err) {
+               int64_t rows_per_tensor, int N, int sort_bits, int L, int kr, int P, int gcol,
+               int P16, int SW, int nbuf, uint16_t* __restrict__ code, CodeT* __restrict__ rcode,
+               CodeT* __restrict__ rcode_t, const float* __restrict__ gate_w,
+               float2* __restrict__ gl, uint32_t* __restrict__ err) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   const uint32_t r_bytes = (uint32_t)P16 * D * 2;
@@ -110,10 +115,28 @@ hash_tc_stream_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
     for (int i = tid; i < P16 * kChunks; i += kStreamThreads) {
       const int j = i / kChunks, ch = i % kChunks;
       uint4 val = make_uint4(0, 0, 0, 0);
-      if (j < sort_bits)
+      if (j < sort_bits) {
         val = *reinterpret_cast<const uint4*>(r_sort + (size_t)j * D + ch * 8);
-      else if (j < P)
+      } else if (j < P) {
         val = *reinterpret_cast<const uint4*>(r_race + (size_t)(j - sort_bits) * D + ch * 8);
+      } else if (gcol >= 0 && j >= gcol && j < gcol + 4) {
+        // gate columns: w_s hi, w_s lo, w_r hi, w_r lo
+        const int gc = j - gcol;
+        const float* wrow = gate_w + (size_t)(gc >> 1) * D + ch * 8;
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          float x[2] = {wrow[e], wrow[e + 1]};
+#pragma unroll
+          for (int m = 0; m < 2; ++m) {
+            const float hi = __bfloat162float(__float2bfloat16_rn(x[m]));
+            x[m] = (gc & 1) ? x[m] - hi : hi;
+          }
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(x[0], x[1]);
+          pk[e >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        val = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
       *reinterpret_cast<uint4*>(smem + (ch >> 3) * (P16 * 128) + sw128_off(j, ch & 7)) = val;
     }
   }
@@ -210,6 +233,10 @@ hash_tc_stream_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
             if (valid <= 0) m = 0u;
             else if (valid < 32) m &= (1u << valid) - 1u;
             bits[srow * SW + (c0 >> 5)] = m;
+            if (c0 == gcol) {   // a query row's gate logits
+              const int64_t grow = tile * kTile + srow;
+              if (grow < rows_per_tensor) gl[grow] = make_float2(v[0] + v[1], v[2] + v[3]);
+            }
           }
         }
         fence_before();
@@ -284,8 +311,8 @@ hash_tc_stream_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
 template <int D, typename CodeT>
 cudaError_t run_stream(const Geometry& g, const void* q, const void* k, const void* r_sort,
                        const void* r_race, uint16_t* code, void* rcode, void* rcode_t,
-                       uint32_t* err, cudaStream_t s) {
-  const StreamShape h = stream_shape(g);
+                       const float* gate_w, float2* gl, uint32_t* err, cudaStream_t s) {
+  const StreamShape h = stream_shape(g, gl != nullptr);
   cudaError_t e = cudaFuncSetAttribute(hash_tc_stream_kernel<D, CodeT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)h.dyn);
   if (e != cudaSuccess) return e;
@@ -307,25 +334,26 @@ cudaError_t run_stream(const Geometry& g, const void* q, const void* k, const vo
   hash_tc_stream_kernel<D, CodeT><<<grid, kStreamThreads, h.dyn, s>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
       static_cast<const __nv_bfloat16*>(r_sort), static_cast<const __nv_bfloat16*>(r_race), rows,
-      g.N, g.sort_bits, g.L, g.kr, h.P, h.P16, h.SW, h.nbuf, code, static_cast<CodeT*>(rcode),
-      static_cast<CodeT*>(rcode_t), err);
+      g.N, g.sort_bits, g.L, g.kr, h.P, h.gcol, h.P16, h.SW, h.nbuf, code,
+      static_cast<CodeT*>(rcode), static_cast<CodeT*>(rcode_t), gate_w, gl, err);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-bool hash_tc_stream_fits(const Geometry& g) {
+bool hash_tc_stream_fits(const Geometry& g, bool gates) {
   if (!g.bf16 || (g.d != 64 && g.d != 128) || g.sort_bits > 16 || g.kr > 16) return false;
-  const StreamShape h = stream_shape(g);
+  const StreamShape h = stream_shape(g, gates);
   return h.P > 0 && h.dyn <= (uint32_t)kSmemLimit;
 }
 
 cudaError_t launch_hash_tc_stream(const Geometry& g, const void* q, const void* k,
                                   const void* r_sort, const void* r_race, uint16_t* code,
-                                  void* rcode, void* rcode_t, uint32_t* err, cudaStream_t s) {
-  if (!hash_tc_stream_fits(g)) return cudaErrorInvalidValue;
+                                  void* rcode, void* rcode_t, const float* gate_w, float2* gl,
+                                  uint32_t* err, cudaStream_t s) {
+  if (!hash_tc_stream_fits(g, gl != nullptr)) return cudaErrorInvalidValue;
 #define ELSAA_HASH_STREAM(DD, CT) \
-  run_stream<DD, CT>(g, q, k, r_sort, r_race, code, rcode, rcode_t, err, s)
+  run_stream<DD, CT>(g, q, k, r_sort, r_race, code, rcode, rcode_t, gate_w, gl, err, s)
   if (g.d == 64)
     return g.rcode_bytes == 1 ? ELSAA_HASH_STREAM(64, uint8_t) : ELSAA_HASH_STREAM(64, uint16_t);
   return g.rcode_bytes == 1 ? ELSAA_HASH_STREAM(128, uint8_t) : ELSAA_HASH_STREAM(128, uint16_t);

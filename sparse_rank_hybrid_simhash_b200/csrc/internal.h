@@ -98,10 +98,11 @@ bool hash_tc_rounds_supported(const Geometry& g, bool gates);
 // The bit-stream variant of the tcgen05 hash (hash_tc_stream.cu) for shapes
 // whose codes do not fill whole words or whose word-aligned hyperplanes do not
 // fit shared memory; launch_hash_tc chooses it.
-bool hash_tc_stream_fits(const Geometry& g);
+bool hash_tc_stream_fits(const Geometry& g, bool gates);
 cudaError_t launch_hash_tc_stream(const Geometry& g, const void* q, const void* k,
                                   const void* r_sort, const void* r_race, uint16_t* code,
-                                  void* rcode, void* rcode_t, uint32_t* err, cudaStream_t s);
+                                  void* rcode, void* rcode_t, const float* gate_w, float2* gl,
+                                  uint32_t* err, cudaStream_t s);
 bool hash_tc_supported(const Geometry& g);
 bool hash_tc_gate_logits_supported(const Geometry& g);
 
