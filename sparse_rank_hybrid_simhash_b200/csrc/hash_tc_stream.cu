@@ -204,21 +204,20 @@ hash_tc_stream_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
         // ended before the barrier that closed the previous pass
         if (tid == 0 && p + 1 < npass) issue(p + 1, abuf);
         const int b = p & 1;
-        if (warp == 0 && !mbar_wait(bar + b, (ph >> b) & 1u, err)) *s_abort = 1;
+        // every reader waits for the pass itself (no block barrier before the
+        // read-out; the outcome is uniform over the warp, as tcgen05.ld needs);
+        // a give-up is shared at the barrier after it
+        const bool wok = __all_sync(0xffffffffu, mbar_wait(bar + b, (ph >> b) & 1u, err));
         ph ^= 1u << b;
-        nbar_sync(kBarRead, kReaders);
-        if (*s_abort) {   // every reader sees the same flag after the barrier
-          ok = false;
-          break;
-        }
+        if (!wok) *s_abort = 1;
         fence_after();
-        if (p + 1 == npass && nbuf == 1 && next < tiles) {
+        if (wok && p + 1 == npass && nbuf == 1 && next < tiles) {
           // every MMA of the tile has completed: its A buffer takes the next tile
           load_tile<D, kReaders>(s_a, q, k, rows_per_tensor, next);
           cp_async_commit();
         }
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < 2 && wok; ++h) {
           const int wd = wsel + 2 * h;
           const int c0 = p * kPass + wd * 32;
           if (c0 < P16) {   // uniform over the warp
@@ -240,7 +239,11 @@ hash_tc_stream_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
           }
         }
         fence_before();
-        nbar_sync(kBarRead, kReaders);
+        nbar_sync(kBarRead, kReaders);   // the buffer's read-out is done: pass p + 2 may reuse it
+        if (*s_abort) {   // every reader sees the same flag after the barrier
+          ok = false;
+          break;
+        }
       }
       // this tile's bits (or the abort) go to the writers
       if (tid == 0) s_done[sb] = ok ? 1 : 0;
