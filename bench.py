@@ -127,7 +127,7 @@ def stage_roofline(flops, nbytes, sec, peaks):
 TRAFFIC_WORKLOAD, TRAFFIC_UNITS = "text-32k", 12
 RECORDED_TRAFFIC = {
     # stage: (kernel source, its sha1 at capture, bytes per 12-unit launch, path flag needed)
-    "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "edcbdc68deae50db48e82ecf8d702c46c0678843", 1.2346e+08, "tc_hash"),
+    "hash": ("sparse_rank_hybrid_simhash_b200/csrc/hash_tc.cu", "8587ef1efd310bd3546658819a84be087a7965da", 1.2358e+08, "tc_hash"),
     "race_build": ("sparse_rank_hybrid_simhash_b200/csrc/race.cu", "ae4cba186ff862dc49a580bdd3aa2d9afe804f41", 6.8706e+07, None),
     "sparse_fwd": ("sparse_rank_hybrid_simhash_b200/csrc/attn_tc_pipe.cu", "b33f474224da484dfb1f6128dd2527644c56625a", 1.8644e+08, "tc_attn"),
     "race_fuse": ("sparse_rank_hybrid_simhash_b200/csrc/race_slab.cu", "5135a962ed6cf3d305d45cb27ffcdf41815cc38e", 1.4487e+08, "slab_fwd"),
